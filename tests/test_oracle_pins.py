@@ -1,0 +1,455 @@
+"""Pins for the float64 oracle: each test ties it to something other than itself
+(exact rational arithmetic, brute-force enumeration, closed forms, library
+routines, the workload statements), so that a dropped term, a wrong sign or
+index, or a transposed operand in the oracle fails one of them.  CPU only.
+"""
+import itertools
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+import oracle as O
+
+GOLDEN = __import__("os").path.join(__import__("os").path.dirname(__file__), "golden")
+
+
+# ----------------------------------------------------------------------------
+# helpers (independent of the oracle's own arithmetic)
+# ----------------------------------------------------------------------------
+def rand_bf16(rng, shape, scale=1.0):
+    x = (rng.standard_normal(shape) * scale).astype(np.float32)
+    return (torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+
+
+def bf16_fraction(bits):
+    """Exact value of one bf16 pattern from its fields (sign, exponent, fraction)."""
+    bits = int(bits)
+    s = -1 if bits >> 15 else 1
+    e = (bits >> 7) & 0xFF
+    f = bits & 0x7F
+    if e == 0:
+        return s * Fraction(f, 1) * Fraction(2) ** (-133)
+    return s * Fraction(128 + f, 1) * Fraction(2) ** (e - 134)
+
+
+def nearest_bf16_bruteforce(x: Fraction, cands):
+    best = min(abs(v - x) for _, v in cands)
+    ties = [b for b, v in cands if abs(v - x) == best]
+    if len(ties) == 1:
+        return ties[0]
+    even = [b for b in ties if (b & 1) == 0]
+    assert len(even) >= 1
+    # +0 / -0 both even for x == 0: take the sign of x
+    return even[0] if len(even) == 1 else (even[1] if x < 0 else even[0])
+
+
+def exact_dot_fraction(a_bits, b_bits):
+    return sum((bf16_fraction(x) * bf16_fraction(y) for x, y in zip(a_bits, b_bits)), Fraction(0))
+
+
+# ----------------------------------------------------------------------------
+# bf16 conversions
+# ----------------------------------------------------------------------------
+def test_bf16_decode_against_field_definition():
+    rng = np.random.default_rng(1)
+    bits = np.concatenate([np.array([0x3F80, 0xC000, 0x0001, 0x7F7F, 0x8000, 0x0080, 0x007F],
+                                    dtype=np.uint16),
+                           rng.integers(0, 0x7F80, 500).astype(np.uint16)])
+    vals = O.bf16_to_f64(bits)
+    for b, v in zip(bits, vals):
+        assert Fraction(float(v)) == bf16_fraction(b)
+    assert vals[0] == 1.0 and vals[1] == -2.0 and vals[2] == 2.0 ** -133
+    assert vals[3] == (2 - 2 ** -7) * 2.0 ** 127
+
+
+def test_bf16_rne_against_bruteforce():
+    rng = np.random.default_rng(2)
+    xs = [1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -30, -(1 + 2 ** -8), 1.5 * 2.0 ** -133,
+          2.5 * 2.0 ** -133, 2.0 ** -126 * (1 - 2 ** -9), 0.0, 255.5, 256.5 * 2 ** -7]
+    xs += list(rng.standard_normal(20) * 10.0 ** rng.integers(-30, 30, 20))
+    got = O.f64_to_bf16_rne(np.array(xs))
+    for x, g in zip(xs, got):
+        fx = Fraction(x)
+        # candidates: the two bf16 neighbours of x found from float32 truncation
+        t = int(np.array([x], dtype=np.float32).view(np.uint32)[0] >> 16)
+        cands = [(c, bf16_fraction(c)) for c in {t - 1, t, t + 1, t + 2} if 0 <= (c & 0x7FFF) < 0x7F80]
+        assert int(g) == nearest_bf16_bruteforce(fx, cands), (x, hex(g))
+    assert O.f64_to_bf16_rne(np.array([1 + 2 ** -8]))[0] == 0x3F80        # tie -> even
+    assert O.f64_to_bf16_rne(np.array([1 + 3 * 2 ** -8]))[0] == 0x3F82    # tie -> even (up)
+    assert O.f64_to_bf16_rne(np.array([1.5 * 2.0 ** -133]))[0] == 0x0002  # subnormal tie
+
+
+# ----------------------------------------------------------------------------
+# page budget (the workload statements, tests/golden/page_budget.txt)
+# ----------------------------------------------------------------------------
+def test_page_budget_matches_workload_statements():
+    rows = []
+    for line in open(f"{GOLDEN}/page_budget.txt"):
+        line = line.split("#")[0].strip()
+        if line:
+            rows.append([int(x) for x in line.split()])
+    assert len(rows) == 3
+    for sink, local, budget, P, n_sink, n_local, pages, k_top in rows:
+        assert O.page_budget(sink, local, budget, P) == (n_sink, n_local, pages, k_top)
+
+
+# ----------------------------------------------------------------------------
+# exact dot products
+# ----------------------------------------------------------------------------
+def test_exact_dots_correctly_rounded():
+    rng = np.random.default_rng(3)
+    A = rand_bf16(rng, (5, 64))
+    Bm = rand_bf16(rng, (7, 64), scale=0.3)
+    # adversarial rows: huge cancelling terms around a small one
+    A[0, :3] = np.array([0x7180, 0x3F80, 0x7180], dtype=np.uint16)   # 2^100, 1, 2^100
+    Bm[0, :3] = np.array([0x3F80, 0x3F80, 0xBF80], dtype=np.uint16)  # 1, 1, -1
+    Bm[0, 3:] = 0
+    A[1, :] = 0x0001                                                 # subnormal q
+    got = O.exact_dots(O.bf16_to_f64(A), O.bf16_to_f64(Bm))
+    for i in range(A.shape[0]):
+        for j in range(Bm.shape[0]):
+            assert got[i, j] == float(exact_dot_fraction(A[i], Bm[j])), (i, j)
+    assert got[0, 0] == 1.0
+    assert (2.0 ** 100 + 1.0) - 2.0 ** 100 == 0.0     # left-to-right float64 loses it
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+def _tiny_select_case(rng, B, T, Hq, Hkv, D, P, lens, pool_perm=True, sig_scale=1.0):
+    q = rand_bf16(rng, (B, T, Hq, D))
+    npages = [-(-L // P) for L in lens]
+    pool = sum(npages)
+    perm = rng.permutation(pool) if pool_perm else np.arange(pool)
+    pt = np.full((B, max(npages)), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npages):
+        pt[b, :n] = perm[off:off + n]
+        off += n
+    sig = rand_bf16(rng, (pool, Hkv, D), scale=sig_scale)
+    return q, sig, pt, np.array(lens, dtype=np.int32)
+
+
+def _bruteforce_selection(q, sig, pt, lens, P, sink, local, budget, b, kvh, G):
+    n_sink, n_local = -(-sink // P), -(-local // P)
+    bp = budget // P
+    nb = -(-int(lens[b]) // P)
+    if nb <= bp:
+        return list(range(nb))
+    cand = list(range(n_sink, nb - n_local))
+    k = bp - n_sink - n_local
+    T = q.shape[1]
+    score = {}
+    for p in cand:
+        vals = [float(exact_dot_fraction(q[b, t, h], sig[pt[b, p], kvh]))
+                for t in range(T) for h in range(kvh * G, (kvh + 1) * G)]
+        score[p] = max(vals)
+    key = lambda p: (-score[p], p)  # noqa: E731
+    winners = []
+    for subset in itertools.combinations(cand, k):
+        rest = [p for p in cand if p not in subset]
+        if all(key(s) < key(r) for s in subset for r in rest):
+            winners.append(subset)
+    assert len(winners) == 1          # exactly one dominant subset
+    return sorted(list(range(n_sink)) + list(winners[0]) + list(range(nb - n_local, nb)))
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2, 3])
+def test_select_matches_bruteforce(seed):
+    rng = np.random.default_rng(10 + seed)
+    P, Hq, Hkv, D, T = 4, 4, 2, 16, (1 if seed % 2 == 0 else 2)
+    lens = [45, 37]   # 12 and 10 pages, ragged last page
+    sink, local, budget = 4, 8, 24   # 1 sink page, 2 local pages, 6-page budget -> k_top = 3
+    q, sig, pt, sl = _tiny_select_case(rng, 2, T, Hq, Hkv, D, P, lens)
+    pages, counts = O.select_pages(q, sig, pt, sl, P, sink, local, budget)
+    for b in range(2):
+        for kvh in range(Hkv):
+            want = _bruteforce_selection(q, sig, pt, sl, P, sink, local, budget, b, kvh, Hq // Hkv)
+            assert counts[b, kvh] == len(want)
+            assert list(pages[b, kvh, :counts[b, kvh]]) == want
+            assert all(pages[b, kvh, counts[b, kvh]:] == -1)
+
+
+def test_select_ties_go_to_lowest_index():
+    rng = np.random.default_rng(20)
+    P, Hq, Hkv, D = 4, 2, 1, 8
+    q, sig, pt, sl = _tiny_select_case(rng, 1, 1, Hq, Hkv, D, P, [48])
+    q[:] = 0                                      # every score is exactly 0
+    pages, counts = O.select_pages(q, sig, pt, sl, P, 4, 4, 20)   # 1 sink, 1 local, k_top 3
+    assert list(pages[0, 0, :counts[0, 0]]) == [0, 1, 2, 3, 11]
+    # duplicate summaries: the lower logical page wins the last slot
+    q, sig, pt, sl = _tiny_select_case(rng, 1, 1, Hq, Hkv, D, P, [48], pool_perm=True)
+    sig[pt[0, 7]] = sig[pt[0, 9]]
+    sc = O.page_scores(O.bf16_to_f64(q[0, 0]), O.bf16_to_f64(sig[pt[0, 1:11], 0]))
+    order = sorted(range(1, 11), key=lambda p: (-sc[p - 1], p))
+    pos7, pos9 = order.index(7), order.index(9)
+    assert pos7 + 1 == pos9                       # adjacent, 7 first
+    k = pos9                                      # budget cutting between them
+    pages, counts = O.select_pages(q, sig, pt, sl, P, 4, 4, 4 * (k + 2))
+    sel = set(pages[0, 0, :counts[0, 0]])
+    assert 7 in sel and 9 not in sel
+
+
+def test_streaming_and_dense_special_cases():
+    rng = np.random.default_rng(21)
+    q, sig, pt, sl = _tiny_select_case(rng, 2, 1, 4, 2, 8, 4, [40, 9])
+    # k_top = 0: StreamingLLM (sink + local only), [TS] "Configuration" streaming mode
+    pages, counts = O.select_pages(q, sig, pt, sl, 4, 8, 8, 16)
+    assert list(pages[0, 0, :counts[0, 0]]) == [0, 1, 8, 9]
+    # N_b <= budget pages: everything
+    assert list(pages[1, 1, :counts[1, 1]]) == [0, 1, 2]
+
+
+def test_selection_invariant_to_physical_page_ids():
+    rng = np.random.default_rng(22)
+    q, sig, pt, sl = _tiny_select_case(rng, 2, 2, 8, 2, 16, 4, [80, 61])
+    a, ca = O.select_pages(q, sig, pt, sl, 4, 4, 8, 36)
+    perm = rng.permutation(sig.shape[0])
+    sig2 = np.empty_like(sig)
+    sig2[perm] = sig                         # physical page i moves to perm[i]
+    pt2 = np.where(pt >= 0, perm[np.maximum(pt, 0)], -1).astype(np.int32)
+    b2, cb = O.select_pages(q, sig2, pt2, sl, 4, 4, 8, 36)
+    assert np.array_equal(a, b2) and np.array_equal(ca, cb)
+
+
+def test_selection_refines_cancelling_scores():
+    # page 1 scores exactly 1 but float64 BLAS gives 0; page 2 scores exactly 0.5
+    P, D = 1, 3
+    q = np.array([[[[0x3F80, 0x3F80, 0x3F80]]]], dtype=np.uint16)
+    sig = np.zeros((4, 1, D), dtype=np.uint16)
+    sig[1, 0] = [0x7180, 0x3F80, 0xF180]      # 2^100, 1, -2^100
+    sig[2, 0] = [0x3F00, 0, 0]                # 0.5
+    sig[3, 0] = [0x3E80, 0, 0]                # 0.25
+    pt = np.array([[0, 1, 2, 3]], dtype=np.int32)
+    pages, counts = O.select_pages(q, sig, pt, np.array([4], dtype=np.int32), P, 1, 1, 3)
+    assert list(pages[0, 0, :counts[0, 0]]) == [0, 1, 3]
+
+
+def test_mla_tiers():
+    rng = np.random.default_rng(23)
+    B, T, Hq, Dk, P = 2, 2, 8, 24, 4
+    q = rand_bf16(rng, (B, T, Hq, Dk))
+    pool = 2 * 10
+    sig = rand_bf16(rng, (pool, 1, Dk))
+    pt = rng.permutation(pool).astype(np.int32).reshape(2, 10)
+    sl = np.array([40, 37], dtype=np.int32)
+    crit, cc, amb, ac = O.select_pages_mla(q, sig, pt, sl, P, 3, 4)
+    for b in range(B):
+        nb = -(-int(sl[b]) // P)
+        exact = {p: max(float(exact_dot_fraction(q[b, t, h], sig[pt[b, p], 0]))
+                        for t in range(T) for h in range(Hq)) for p in range(nb)}
+        order = sorted(range(nb), key=lambda p: (-exact[p], p))
+        assert list(crit[b, :cc[b]]) == sorted(order[:3])
+        assert list(amb[b, :ac[b]]) == sorted(order[3:7])
+    # with every head ambient, crit u amb equals the untiered top-(alpha+beta)
+    pages, counts = O.select_pages(q, sig, pt, sl, P, 0, 0, 7 * P)
+    for b in range(B):
+        assert sorted(list(crit[b, :cc[b]]) + list(amb[b, :ac[b]])) == list(pages[b, 0, :counts[b, 0]])
+
+
+# ----------------------------------------------------------------------------
+# attention
+# ----------------------------------------------------------------------------
+def _attn_case(rng, B=2, T=1, Hq=4, Hkv=2, D=16, Dv=16, P=4, lens=(23, 14)):
+    q = rand_bf16(rng, (B, T, Hq, D))
+    npages = [-(-L // P) for L in lens]
+    pool = sum(npages)
+    perm = rng.permutation(pool)
+    pt = np.full((B, max(npages)), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npages):
+        pt[b, :n] = perm[off:off + n]
+        off += n
+    k = rand_bf16(rng, (pool, Hkv, P, D))
+    v = rand_bf16(rng, (pool, Hkv, P, Dv))
+    return q, k, v, pt, np.array(lens, dtype=np.int32), npages
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_dense_budget_equals_sdpa(T):
+    rng = np.random.default_rng(30 + T)
+    q, k, v, pt, sl, npages = _attn_case(rng, T=T)
+    B, _, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    P = 4
+    lists = np.full((B, Hkv, max(npages)), -1, dtype=np.int32)
+    counts = np.zeros((B, Hkv), dtype=np.int32)
+    for b in range(B):
+        lists[b, :, :npages[b]] = np.arange(npages[b])
+        counts[b] = npages[b]
+    h2l = np.arange(Hq) // G
+    scale = 1 / math.sqrt(D)
+    o, lse = O.sparse_attention(q, k, v, pt, sl, lists, counts, h2l, scale, P)
+    for b in range(B):
+        L = int(sl[b])
+        phys = pt[b, :npages[b]]
+        K = torch.from_numpy(O.bf16_to_f64(k[phys]).transpose(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :L])
+        V = torch.from_numpy(O.bf16_to_f64(v[phys]).transpose(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :L])
+        Q = torch.from_numpy(O.bf16_to_f64(q[b]).transpose(1, 0, 2))       # [Hq, T, D]
+        Kx = K.repeat_interleave(G, 0)
+        Vx = V.repeat_interleave(G, 0)
+        mask = torch.arange(L)[None, :] <= (L - T + torch.arange(T))[:, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(Q, Kx, Vx, attn_mask=mask, scale=scale)
+        np.testing.assert_allclose(o[b].transpose(1, 0, 2), ref.numpy(), rtol=0, atol=1e-12)
+        s = (scale * (Q @ Kx.transpose(1, 2))).numpy()
+        s = np.where(mask.numpy()[None], s, -np.inf)
+        np.testing.assert_allclose(lse[b].T, scipy.special.logsumexp(s, axis=-1), rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_sparse_equals_masked_dense(T):
+    rng = np.random.default_rng(40 + T)
+    q, k, v, pt, sl, npages = _attn_case(rng, T=T, lens=(37, 29))
+    B, _, Hq, D = q.shape
+    Hkv = k.shape[1]
+    n_lists = 3      # per-head lists, not tied to the kv head (QK 2D sparsity)
+    lists = np.full((B, n_lists, 6), -1, dtype=np.int32)
+    counts = np.zeros((B, n_lists), dtype=np.int32)
+    for b in range(B):
+        for li in range(n_lists):
+            c = int(rng.integers(0, min(6, npages[b]) + 1))
+            lists[b, li, :c] = np.sort(rng.choice(npages[b], c, replace=False))
+            counts[b, li] = c
+    h2l = rng.integers(0, n_lists, (B, Hq))
+    a = O.sparse_attention(q, k, v, pt, sl, lists, counts, h2l, 0.3, 4)
+    m = O.masked_dense_attention(q, k, v, pt, sl, lists, counts, h2l, 0.3, 4)
+    np.testing.assert_allclose(a[0], m[0], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(np.isinf(a[1]), np.isinf(m[1]))
+    fin = np.isfinite(a[1])
+    np.testing.assert_allclose(a[1][fin], m[1][fin], rtol=0, atol=1e-12)
+    assert np.all(a[0][~fin] == 0)
+
+
+def test_closed_forms():
+    rng = np.random.default_rng(50)
+    D, P = 8, 4
+    q = rand_bf16(rng, (1, 1, 1, D))
+    k = rand_bf16(rng, (1, 1, P, D))
+    v = rand_bf16(rng, (1, 1, P, D))
+    pt = np.array([[0]], dtype=np.int32)
+    lists = np.array([[[0]]], dtype=np.int32)
+    cnt = np.array([[1]], dtype=np.int32)
+    # one key: O = v, lse = scale q.k
+    o, lse = O.sparse_attention(q, k, v, pt, np.array([1]), lists, cnt, [0], 0.5, P)
+    np.testing.assert_array_equal(o[0, 0, 0], O.bf16_to_f64(v[0, 0, 0]))
+    qk = float(exact_dot_fraction(q[0, 0, 0], k[0, 0, 0]))
+    assert abs(lse[0, 0, 0] - 0.5 * qk) < 1e-14
+    # equal keys: O = mean(v), lse = s + log n
+    k2 = np.repeat(k[:, :, :1], P, axis=2)
+    o, lse = O.sparse_attention(q, k2, v, pt, np.array([P]), lists, cnt, [0], 0.5, P)
+    np.testing.assert_allclose(o[0, 0, 0], O.bf16_to_f64(v[0, 0]).mean(0), atol=1e-14)
+    assert abs(lse[0, 0, 0] - (0.5 * qk + math.log(P))) < 1e-13
+    # two keys: weights are sigmoid(s0 - s1), 1 - that
+    o, lse = O.sparse_attention(q, k, v, pt, np.array([2]), lists, cnt, [0], 0.5, P)
+    s0 = 0.5 * float(exact_dot_fraction(q[0, 0, 0], k[0, 0, 0]))
+    s1 = 0.5 * float(exact_dot_fraction(q[0, 0, 0], k[0, 0, 1]))
+    w0 = 1 / (1 + math.exp(s1 - s0))
+    want = w0 * O.bf16_to_f64(v[0, 0, 0]) + (1 - w0) * O.bf16_to_f64(v[0, 0, 1])
+    np.testing.assert_allclose(o[0, 0, 0], want, atol=1e-14)
+    assert abs(lse[0, 0, 0] - (max(s0, s1) + math.log1p(math.exp(-abs(s0 - s1))))) < 1e-14
+    # empty list: O = 0, lse = -inf
+    o, lse = O.sparse_attention(q, k, v, pt, np.array([P]), lists, np.array([[0]]), [0], 0.5, P)
+    assert np.all(o == 0) and lse[0, 0, 0] == -np.inf
+
+
+# ----------------------------------------------------------------------------
+# combine
+# ----------------------------------------------------------------------------
+def test_combine_partition_invariance():
+    rng = np.random.default_rng(60)
+    q, k, v, pt, sl, npages = _attn_case(rng, T=2, lens=(44, 41))
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[1]
+    h2l = np.arange(Hq) // (Hq // Hkv)
+    lists = np.tile(np.arange(11, dtype=np.int32), (B, Hkv, 1))
+    counts = np.full((B, Hkv), 11, dtype=np.int32)
+    full = O.sparse_attention(q, k, v, pt, sl, lists, counts, h2l, 0.25, 4)
+    for bounds in ([0, 11], [0, 3, 11], [0, 5, 6, 11], [0, 0, 4, 4, 11]):
+        parts = []
+        for s0, s1 in zip(bounds[:-1], bounds[1:]):
+            li = np.full_like(lists, -1)
+            li[:, :, :s1 - s0] = lists[:, :, s0:s1]
+            parts.append(O.sparse_attention(q, k, v, pt, sl, li, np.full_like(counts, s1 - s0),
+                                            h2l, 0.25, 4))
+        o_p = np.stack([p[0] for p in parts])
+        l_p = np.stack([p[1] for p in parts])
+        for perm in (None, np.arange(len(parts))[::-1]):
+            op, lp = (o_p, l_p) if perm is None else (o_p[perm], l_p[perm])
+            o, lse = O.combine(op, lp)
+            np.testing.assert_allclose(o, full[0], atol=1e-12)
+            np.testing.assert_allclose(lse, full[1], atol=1e-12)
+
+
+def test_combine_special_cases():
+    rng = np.random.default_rng(61)
+    o = rng.standard_normal((1, 5, 4))
+    lse = rng.standard_normal((1, 5))
+    a, la = O.combine(o, lse)
+    np.testing.assert_array_equal(a, o[0])
+    np.testing.assert_array_equal(la, lse[0])
+    o2 = np.concatenate([o, rng.standard_normal((1, 5, 4))])
+    l2 = np.concatenate([lse, np.full((1, 5), -np.inf)])
+    a, la = O.combine(o2, l2)
+    np.testing.assert_allclose(a, o[0], atol=1e-15)
+    np.testing.assert_allclose(la, lse[0], atol=1e-15)
+    a, la = O.combine(o2, np.full((2, 5), -np.inf))
+    assert np.all(a == 0) and np.all(la == -np.inf)
+    # two splits: closed form with scipy
+    l3 = rng.standard_normal((2, 5))
+    a, la = O.combine(o2, l3)
+    np.testing.assert_allclose(la, scipy.special.logsumexp(l3, axis=0), atol=1e-14)
+    w = scipy.special.softmax(l3, axis=0)
+    np.testing.assert_allclose(a, (w[..., None] * o2).sum(0), atol=1e-14)
+
+
+# ----------------------------------------------------------------------------
+# block union
+# ----------------------------------------------------------------------------
+def test_block_union_bruteforce():
+    rng = np.random.default_rng(70)
+    Hq, Hkv, NQB, off, top_k = 4, 2, 3, 6, 2
+    NKB = off + NQB
+    s = rng.standard_normal((Hq, NQB, NKB)).astype(np.float32)
+    s[0, 1, 2] = s[0, 1, 3]        # an exact tie: the lower block wins
+    tables, counts = O.block_union(s, Hkv, off, top_k)
+    for g in range(Hkv):
+        want = set()
+        for h in range(g * 2, g * 2 + 2):
+            for j in range(NQB):
+                d = off + j
+                cand = sorted(range(1, d), key=lambda c: (-float(s[h, j, c]), c))
+                mask = {0, d} | set(cand[:top_k])
+                assert mask <= set(tables[g, :counts[g]])
+                want |= mask
+        assert list(tables[g, :counts[g]]) == sorted(want)
+        assert all(tables[g, counts[g]:] == -1)
+    if s[0, 1, 2] >= np.sort(s[0, 1, 1:7])[-2]:
+        assert 2 in set(tables[0, :counts[0]])
+
+
+# ----------------------------------------------------------------------------
+# page summaries
+# ----------------------------------------------------------------------------
+def test_page_summaries_exact_mean():
+    rng = np.random.default_rng(80)
+    P, Hkv, D = 4, 2, 6
+    k = rand_bf16(rng, (3, Hkv, P, D))
+    k[2, 0, :, 0] = [0x7180, 0x3F80, 0xF180, 0x0001]      # cancellation + subnormal
+    pt = np.array([[2, 0, 1]], dtype=np.int32)
+    sl = np.array([10], dtype=np.int32)                  # last page has 2 valid keys
+    sig = O.page_summaries(k, pt, sl, P)
+    for p, nval in ((0, 4), (1, 4), (2, 2)):
+        phys = pt[0, p]
+        for h in range(Hkv):
+            for d in range(D):
+                mean = sum(bf16_fraction(k[phys, h, j, d]) for j in range(nval)) / nval
+                s64 = float(sum(bf16_fraction(k[phys, h, j, d]) for j in range(nval)))
+                want = O.f64_to_bf16_rne(np.array([s64 / nval]))[0]
+                assert sig[phys, h, d] == want
+                # the bf16 result is within one bf16 spacing of the exact mean
+                assert abs(bf16_fraction(sig[phys, h, d]) - mean) <= abs(mean) / 128 + Fraction(1, 2 ** 133)
