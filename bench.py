@@ -1,0 +1,404 @@
+"""Benchmark: sparse-attention decode steps on the Llama-3-8B-shaped workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: page selection
+(sa_select_pages), the gather split-KV decode (sa_sparse_decode) and the
+split merge (sa_combine).  Workload: B=16 sequences of 32768 tokens, Hq=32,
+Hkv=8, D=128, 16-token pages in a shuffled 2 GiB pool, budget 1024 tokens
+(2 sink + 32 local + 30 top-k pages per kv head), 5% of pages per kv head
+lifted 3 sigma along the group query; bf16 N(0,1) data, seed 0; summaries
+built once by sa_build_page_summaries (not part of a step).
+
+The metric is selected-KV GB/s: K+V bytes of the selected pages' valid
+tokens per step divided by the step time (inputs resident in HBM, L2 flushed
+before every timed step by writing a 256 MiB buffer outside the timed
+events).  The line also carries calls/s, the decode kernel's roofline
+fraction against the measured HBM copy bandwidth, an end-to-end number
+through the same API with the per-step inputs (q, page table, seq_lens)
+copied from pinned host memory and the outputs (O, LSE) copied back inside
+the timed region, and the float64 oracle timed on a bounded sample on the
+host cores.
+
+With --gpus N (torchrun), every rank runs its own batch of the same shape
+(replicas: the path has no exchange step); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "selected-KV GB/s (fraction of HBM peak) and sparse-attn calls/sec at 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = heuristic)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle samples while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def selected_kv_bytes(counts, pages, seq_lens, P, D):
+    """K+V bytes of the valid tokens of every selected page (per step)."""
+    import torch
+    B, Hkv, cap = pages.shape
+    L = seq_lens.to(torch.int64).view(B, 1, 1)
+    idx = torch.arange(cap, device=pages.device).view(1, 1, cap)
+    valid = idx < counts.view(B, Hkv, 1)
+    p = pages.to(torch.int64).clamp_min(0)
+    toks = (L - p * P).clamp(0, P)
+    toks = torch.where(valid, toks, torch.zeros_like(toks))
+    return int(toks.sum().item()) * D * 2 * 2
+
+
+def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0):
+    """Oracle (float64, host cores) on a bounded sample: n_units (b, kv head)
+    pairs, select + attention.  Returns GB/s of selected KV and the sample."""
+    import numpy as np
+
+    import oracle as O
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    pt = inp["page_table"].cpu().numpy()
+    sl = inp["seq_lens"].cpu().numpy()
+    qb = W.bf16_bits(inp["q"])
+    units = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)][:n_units]
+    G = cfg.G
+    t0 = time.perf_counter()
+    done, kv_bytes = 0, 0
+    for (b, h) in units:
+        pages_np, counts_np = O.select_pages(qb, sig_bits, pt, sl, cfg.page_size, cfg.sink_tokens,
+                                             cfg.local_tokens, cfg.budget_tokens, units=[(b, h)])
+        lst = pages_np[b, h, :counts_np[b, h]]
+        phys = pt[b, lst]
+        # gather only this unit's pages from the device pool
+        import torch
+        kb = W.bf16_bits(inp["k"][torch.as_tensor(phys, device=inp["k"].device)])
+        vb = W.bf16_bits(inp["v"][torch.as_tensor(phys, device=inp["v"].device)])
+        loc_pt = np.full_like(pt, -1)
+        loc_pt[b, lst] = np.arange(len(lst))
+        lists = np.full((cfg.B, cfg.Hkv, pages_np.shape[2]), -1, dtype=np.int32)
+        counts = np.zeros((cfg.B, cfg.Hkv), dtype=np.int32)
+        lists[b, h, :len(lst)] = lst
+        counts[b, h] = len(lst)
+        rows = [(b, 0, hh) for hh in range(h * G, (h + 1) * G)]
+        O.sparse_attention(qb, kb, vb, loc_pt, sl, lists, counts, np.arange(cfg.Hq) // G,
+                           1.0 / math.sqrt(cfg.D), cfg.page_size, rows=rows)
+        L = int(sl[b])
+        kv_bytes += sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst) * cfg.D * 4
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return kv_bytes / dt / 1e9, done, dt
+
+
+def main():
+    args = parse()
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference" and rank != 0:
+        return                      # the oracle arm runs on rank 0 only
+    if world > 1 and args.impl == "ours":
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    cfg = W.LLAMA8B_DECODE
+    cores = len(os.sched_getaffinity(0))
+
+    if args.impl == "reference":
+        # the reference arm is the float64 oracle on the host cores
+        import paged_sparse_kv_sa_b200 as sa
+        sa.load()
+        inp = W.gqa_decode_inputs(cfg, seed=args.seed, device=dev)
+        sig = sa.sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
+        torch.cuda.synchronize()
+        sig_bits = W.bf16_bits(sig)
+        for _ in range(args.warmup):
+            cpu_baseline(cfg, inp, sig_bits, 1, budget_s=5)
+        tot_b, tot_t, units = 0.0, 0.0, 0
+        for _ in range(args.steps):
+            gbs, n, dt = cpu_baseline(cfg, inp, sig_bits, 2, budget_s=10)
+            tot_b += gbs * dt
+            tot_t += dt
+            units += n
+        val = tot_b / tot_t
+        line = {"metric": METRIC, "value": round(val, 6), "unit": "GB/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1000 * tot_t / args.steps, 3), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "impl": "reference",
+                "config": {"workload": cfg.name, "B": cfg.B, "seq_len": cfg.seq_len_lo,
+                           "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
+                           "budget_tokens": cfg.budget_tokens},
+                "cpu_baseline": {"value": round(val, 6), "unit": "GB/s", "cores": cores,
+                                 "kind": "oracle",
+                                 "sample": f"{units} (sequence, kv head) units of select + "
+                                           f"attention per {args.steps} steps"},
+                "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import paged_sparse_kv_sa_b200 as sa
+    sa.load()
+    inp = W.gqa_decode_inputs(cfg, seed=args.seed + rank, device=dev)
+    q, k, v, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
+    sig = sa.sa_build_page_summaries(k, pt, sl)
+    step = sa.SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, pt.shape[1],
+                               cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens,
+                               n_splits=args.splits or None, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def run_step():
+        step.select(q, sig, pt, sl)
+        step.decode(q, k, v, pt, sl)
+        step.combine()
+
+    for _ in range(max(args.warmup, 3)):
+        run_step()
+    torch.cuda.synchronize()
+    kv_bytes = selected_kv_bytes(step.counts, step.pages, sl, cfg.page_size, cfg.D)
+    q_bytes = q.numel() * 2
+    part_bytes = step.o_part.numel() * 4 + step.lse_part.numel() * 4
+    list_bytes = step.pages.numel() * 4 + step.counts.numel() * 4
+    decode_alg_bytes = kv_bytes + q_bytes + part_bytes + list_bytes + \
+        int(step.counts.sum().item()) * 4
+
+    # Whole steps and the decode kernel alone are replayed from CUDA graphs, so
+    # that the events bracket device work only (no host enqueue gaps).
+    g_step = torch.cuda.CUDAGraph()
+    g_dec = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        run_step()
+    with torch.cuda.graph(g_dec):
+        step.decode(q, k, v, pt, sl)
+    for _ in range(3):
+        g_step.replay()
+        g_dec.replay()
+    torch.cuda.synchronize()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush.fill_(i & 0xFF)
+            ev[i][0].record(stream)
+            g_step.replay()
+            ev[i][1].record(stream)
+            flush.fill_((i + 1) & 0xFF)
+            ev[i][2].record(stream)
+            g_dec.replay()
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3           # seconds, K steps
+    t_dec = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3            # decode kernel alone
+    # per-stage split of one eager step (informational)
+    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    flush.fill_(0)
+    st_ev[0].record(stream)
+    step.select(q, sig, pt, sl)
+    st_ev[1].record(stream)
+    step.decode(q, k, v, pt, sl)
+    st_ev[2].record(stream)
+    step.combine()
+    st_ev[3].record(stream)
+    torch.cuda.synchronize()
+    t_sel = st_ev[0].elapsed_time(st_ev[1]) / 1e3 * K
+    t_cmb = st_ev[2].elapsed_time(st_ev[3]) / 1e3 * K
+    if world > 1:
+        t = torch.tensor([t_step], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_step_max = float(t.item())
+    else:
+        t_step_max = t_step
+    value = world * kv_bytes * K / t_step_max / 1e9
+    calls_per_sec = world * K / t_step_max
+
+    # ---- end to end through the same API: host inputs in, host outputs out
+    q_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
+    pt_h = torch.empty(pt.shape, dtype=pt.dtype, pin_memory=True).copy_(pt.cpu())
+    sl_h = torch.empty(sl.shape, dtype=sl.dtype, pin_memory=True).copy_(sl.cpu())
+    o_h = torch.empty(step.o.shape, dtype=torch.float32, pin_memory=True)
+    lse_h = torch.empty(step.lse.shape, dtype=torch.float32, pin_memory=True)
+    q_d, pt_d, sl_d = torch.empty_like(q), torch.empty_like(pt), torch.empty_like(sl)
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        pt_d.copy_(pt_h, non_blocking=True)
+        sl_d.copy_(sl_h, non_blocking=True)
+        step.select(q_d, sig, pt_d, sl_d)
+        step.decode(q_d, k, v, pt_d, sl_d)
+        step.combine()
+        o_h.copy_(step.o, non_blocking=True)
+        lse_h.copy_(step.lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    for i in range(K):
+        flush.fill_(i & 0xFF)
+        e2e_ev[i][0].record(stream)
+        e2e_step()
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
+    if world > 1:
+        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        t_e2e = float(t.item())
+    e2e_value = world * kv_bytes * K / t_e2e / 1e9
+    h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
+    d2h = o_h.numel() * 4 + lse_h.numel() * 4
+
+    # correctness guard on what was timed: the outputs are finite and selections full
+    assert torch.isfinite(step.o).all().item(), "non-finite output"
+    assert int(step.dev_error.item()) == 0, "device error flag set"
+
+    hbm_peak, peak_kind = peaks()
+    dec_avg = t_dec / K
+    achieved = decode_alg_bytes / dec_avg / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            td = json.load(f)
+        if td.get("workload") == cfg.name and td.get("splits") == step.n_splits:
+            traffic = td.get("bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(1e3 * t_step_max / K, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "B": cfg.B, "seq_len": cfg.seq_len_lo, "Hq": cfg.Hq,
+                   "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
+                   "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
+                   "local_tokens": cfg.local_tokens, "n_splits": step.n_splits,
+                   "l2": "flushed (256 MiB write) before every timed step",
+                   "parallelism": f"replicas x{world}"},
+        "calls_per_sec": round(calls_per_sec, 2),
+        "stage_ms": {"select_eager": round(1e3 * t_sel / K, 4),
+                     "decode_graph": round(1e3 * t_dec / K, 4),
+                     "combine_eager": round(1e3 * t_cmb / K, 4)},
+        "selected_kv_bytes_per_step": kv_bytes,
+        "roofline": {"kernel": "decode_gqa_kernel", "bound": "hbm", "achieved": round(achieved, 2),
+                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
+                     "peak_kind": peak_kind, "traffic": traffic,
+                     "alg_bytes_per_launch": decode_alg_bytes},
+        "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(1e3 * t_e2e / K, 4)},
+        "gpu_launches": 4 * K,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=8, budget_s=20.0)
+        line["cpu_baseline"] = {"value": round(gbs, 6), "unit": "GB/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{n} of {cfg.B * cfg.Hkv} (sequence, kv head) units: "
+                                          f"select + attention, {dt:.1f} s"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,195 @@
+/*
+ * sa.h — C ABI of the paged sparse-KV attention library (libsa.so, sm_100a).
+ *
+ * What the calls compute (sources are page titles and sections):
+ *  - sa_select_pages: page scoring against per-page key summaries and top-k
+ *    selection with forced sink and local pages ("Universal Attention Engine —
+ *    Declarative Sparse Attention for Production", "The Product" for the
+ *    sink/local/budget pattern and "Content-Dependent Dynamic Routing" for
+ *    top_k_blocks(q @ mean(k_blocks))).
+ *  - sa_select_pages_tiered: the Critical/Ambient tier selection of "TileSparse:
+ *    Arithmetic-Intensity-Aware Sparse Attention for Compute-Bound LLM
+ *    Decoding", "Motivation" (alpha pages for all heads, beta pages for h heads).
+ *  - sa_sparse_decode: attention over per-head page lists read in place from a
+ *    paged cache (UAE "Architecture": gather-based sparse KV decode over a
+ *    PagedAttention-compatible layout; TileSparse "Two implementations": a
+ *    per-head page-list Flash-decode kernel), split over the list.
+ *  - sa_combine: the log-sum-exp merge of split partials (the merge step of a
+ *    split-KV Flash-decode, TileSparse "Configuration", mode "full").
+ *  - sa_block_union: CompactAttention's Block-Union KV Selection (abstract on
+ *    the page titled "Causal Attention on CPU: ..."): Q-block union plus
+ *    intra-group union into per-group KV block tables, used in place.
+ *  - sa_build_page_summaries: the per-page key means the router scores
+ *    (UAE "Content-Dependent Dynamic Routing", mean(k_blocks)).
+ *
+ * Conventions for every call:
+ *  - Pointers marked (dev) are caller-owned device memory on the current
+ *    device; (host) pointers are read before the call returns.  The library
+ *    allocates nothing and keeps no state between calls except a cache of
+ *    TMA descriptors keyed by their inputs.
+ *  - bf16 tensors are passed as uint16_t bit patterns.  Strides are in
+ *    elements; the innermost (feature) stride must be 1, other strides of
+ *    bf16 tensors multiples of 8 elements, base pointers 16-byte aligned.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream).  Argument errors are found on the host
+ *    before any launch and return SA_ERR_INVALID_ARG or SA_ERR_UNSUPPORTED
+ *    with nothing launched.  Launch failures return SA_ERR_CUDA.
+ *  - dev_error (dev, optional, may be NULL): an int32 word the kernels OR
+ *    error bits into when data they read is out of range (a page id outside
+ *    the sequence or the pool, a list count above its capacity).  The
+ *    offending page is skipped; kernels never trap.  The caller zeroes it and
+ *    reads it back when it wants to know.
+ *
+ * Page-count reading of a token budget (the pages give tokens, not pages):
+ *   n_sink = ceil(sink/P), n_local = ceil(local/P), budget_pages = floor(budget/P),
+ *   k_top = budget_pages - n_sink - n_local (must be >= 0).
+ */
+#ifndef SA_H_
+#define SA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SA_API __attribute__((visibility("default")))
+#else
+#define SA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* a null pointer, a bad size, stride or alignment */
+  SA_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels implement   */
+  SA_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required      */
+  SA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed            */
+} sa_status;
+
+/* Bits kernels OR into *dev_error. */
+#define SA_DEVERR_PAGE_RANGE 1   /* logical page >= ceil(seq_len/P) or < 0      */
+#define SA_DEVERR_POOL_RANGE 2   /* physical page id outside [0, P_pool)        */
+#define SA_DEVERR_COUNT 4        /* list count < 0 or above its capacity        */
+#define SA_DEVERR_TIMEOUT 8      /* a bounded wait on a copy gave up             */
+
+/* Human-readable name of a status code (static storage). */
+SA_API const char* sa_status_string(int status);
+
+/* ABI version: 100 * major + minor. */
+SA_API int sa_abi_version(void);
+
+/*
+ * sa_select_pages — page scoring and top-k selection, GQA.
+ *
+ * For each (b, kv head g): every logical page p < N_b = ceil(seq_lens[b]/P)
+ * of the sequence has the summary sigma = summaries[page_table[b,p], g, :].
+ * Sink pages [0, n_sink) and local pages [N_b - n_local, N_b) are always
+ * selected; of the remaining candidates the k_top with the largest score win,
+ * ties to the lower logical page.  score_p = max over the group's query rows
+ * (t < T, heads h with h / (Hq/Hkv) == g) of the dot product q[b,t,h,:].sigma,
+ * unscaled and correctly rounded to float64 (so the selection equals the one
+ * exact arithmetic gives).  If N_b <= budget_pages every page is selected.
+ *
+ *  q          (dev) [B,T,Hq,Dk] bf16, strides q_strides (elements)
+ *  summaries  (dev) [P_pool,Hkv,Dk] bf16, contiguous
+ *  page_table (dev) [B,max_pages] int32 physical page ids, contiguous
+ *  seq_lens   (dev) [B] int32, 0 <= seq_lens[b] <= max_pages*P
+ *  out_pages  (dev) [B,Hkv,budget_pages] int32: selected logical ids ascending,
+ *                   then -1 padding
+ *  out_counts (dev) [B,Hkv] int32
+ * Supported: Dk in {64,128,256}, T*Hq/Hkv <= 16, max_pages <= 16384.
+ */
+SA_API int sa_select_pages(const uint16_t* q, const int64_t q_strides[4],
+                    const uint16_t* summaries, const int32_t* page_table,
+                    const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
+                    int page_size, int max_pages, int P_pool, int sink_tokens,
+                    int local_tokens, int budget_tokens, int32_t* out_pages,
+                    int32_t* out_counts, int32_t* dev_error, void* stream);
+
+/*
+ * sa_sparse_decode — split-KV attention over per-head page lists.
+ *
+ * Query row (b, t, h) attends the keys of list l = head_to_list[h] of
+ * sequence b, read from kv head h / (Hq/Hkv): the tokens j of every logical
+ * page p in lists[b,l,0:list_counts[b,l]] whose position p*P + j is below
+ * seq_lens[b] and at most seq_lens[b] - T + t (query token t sits at that
+ * position: causal MTP / chunked prefill).  s_j = scale * q.k_j; natural-log
+ * LSE.  The list is cut into n_splits contiguous pieces of
+ * ceil(count/n_splits) entries; split s writes its own normalised output
+ * and LSE (an empty split writes O = 0, LSE = -inf).  With n_splits == 1
+ * the partials are the final result; otherwise pass them to sa_combine.
+ *
+ *  q            (dev) [B,T,Hq,Dk] bf16, strides q_strides
+ *  k_cache      (dev) [P_pool,Hkv,P,Dk] bf16, strides k_strides (vLLM's
+ *                     [P_pool,P,Hkv,Dk] is the same tensor with other strides)
+ *  v_cache      (dev) [P_pool,Hkv,P,Dv] bf16, strides v_strides; may alias
+ *                     k_cache (MLA: V = first Dv columns of the latent K)
+ *  page_table   (dev) [B,max_pages] int32;  seq_lens (dev) [B] int32
+ *  lists        (dev) [B,n_lists,max_list] int32 logical page ids
+ *  list_counts  (dev) [B,n_lists] int32
+ *  head_to_list (host) [Hq] int32 in [0, n_lists)
+ *  o_partial    (dev) [n_splits,B,T,Hq,Dv] float32
+ *  lse_partial  (dev) [n_splits,B,T,Hq] float32
+ * Supported: Dk == Dv in {64,128,256}, P in {16,32,64,128}, and at most 16
+ * query rows (T x heads) sharing one (list, kv head) pair.
+ */
+SA_API int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                     const int64_t k_strides[4], const uint16_t* v_cache,
+                     const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                     const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
+                     int n_lists, int max_list, const int32_t* head_to_list, int B, int T,
+                     int Hq, int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                     int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
+                     void* stream);
+
+/*
+ * sa_combine — merge split partials: lse = log sum_s exp(lse_s),
+ * O = sum_s exp(lse_s - lse) O_s; splits with lse_s = -inf weigh nothing;
+ * rows whose splits are all empty give O = 0, lse = -inf.
+ *
+ *  o_partial  (dev) [n_splits,rows,Dv] float32;  lse_partial (dev) [n_splits,rows]
+ *  o_out      (dev, optional) [rows,Dv] float32
+ *  o_out_bf16 (dev, optional) [rows,Dv] bf16 (round to nearest even)
+ *  lse_out    (dev, optional) [rows] float32
+ * At least one output must be given.  Dv % 4 == 0.
+ */
+SA_API int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,
+               int Dv, float* o_out, uint16_t* o_out_bf16, float* lse_out, void* stream);
+
+/*
+ * sa_build_page_summaries — sigma[page_table[b,p], g, :] for every logical
+ * page p < ceil(seq_lens[b]/P): the mean of the page's valid keys
+ * (positions < seq_lens[b]), computed as RNE_bf16(RN64(RN64(exact sum)/n)).
+ * Rows of pages no sequence references are left untouched.
+ *
+ *  k_cache    (dev) [P_pool,Hkv,P,Dk] bf16, strides k_strides
+ *  summaries  (dev) [P_pool,Hkv,Dk] bf16, contiguous (written)
+ */
+SA_API int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
+                            const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                            int B, int Hkv, int Dk, int page_size, int P_pool,
+                            uint16_t* summaries, int32_t* dev_error, void* stream);
+
+/*
+ * sa_block_union — per-group KV block tables for chunked prefill.
+ * For head h and Q-block j the block mask is the sink blocks [0, n_sink),
+ * the diagonal block d = q_block_offset + j, and the top_k blocks of
+ * [n_sink, d) by (score desc, index asc).  Table g = the ascending union of
+ * the masks of every head of group g (h / (Hq/Hkv) == g) over all Q-blocks.
+ *
+ *  scores (dev) [Hq,NQB,NKB] float32 (finite)
+ *  tables (dev) [Hkv,NKB] int32: ascending block ids, then -1 padding
+ *  counts (dev) [Hkv] int32
+ * Requires q_block_offset + NQB <= NKB.
+ */
+SA_API int sa_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_block_offset,
+                   int top_k, int n_sink_blocks, int32_t* tables, int32_t* counts,
+                   void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_H_ */

@@ -1,0 +1,9 @@
+"""Paged sparse-KV attention for B200 (sm_100a).
+
+The computation lives in ``libsa.so`` (C ABI, ``include/sa.h``); this package
+is its thin Python binding plus the seeded workload generators the tests and
+benchmark share.  Build the library with ``python -m paged_sparse_kv_sa_b200.build``.
+"""
+from ._lib import (EXPORTED, LIB_PATH, SAError, load, page_budget, sa_block_union,  # noqa: F401
+                   sa_build_page_summaries, sa_combine, sa_select_pages, sa_sparse_decode)
+from .pipeline import SparseDecodeStep, default_splits  # noqa: F401

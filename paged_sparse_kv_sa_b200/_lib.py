@@ -1,0 +1,218 @@
+"""ctypes binding of ``libsa.so``: argument marshalling only.
+
+Each function has the name and argument order of the C entry point it wraps
+(include/sa.h); it takes torch tensors, checks dtypes and devices, passes
+their data pointers, strides and the current CUDA stream, and raises
+``SAError`` on a non-zero status.  Every step of the computation runs in the
+library's kernels: there is no fallback when the library or the GPU is
+missing; calls raise instead.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsa.so")
+
+_c_i64_4 = ctypes.c_int64 * 4
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_F = ctypes.c_float
+
+_SIGNATURES = {
+    "sa_status_string": (ctypes.c_char_p, [_I]),
+    "sa_abi_version": (_I, []),
+    "sa_select_pages": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                             _I, _P, _P, _P, _P]),
+    "sa_sparse_decode": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P, _I,
+                              _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P]),
+    "sa_combine": (_I, [_P, _P, _I, _I64, _I, _P, _P, _P, _P]),
+    "sa_build_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_block_union": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+}
+
+EXPORTED = tuple(_SIGNATURES)
+
+
+class SAError(RuntimeError):
+    pass
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the shared library (once) and declare its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m paged_sparse_kv_sa_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = load().sa_status_string(status).decode()
+        raise SAError(f"{what} failed: {msg} ({status})")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _strides4(t) -> "ctypes.Array":
+    s = list(t.stride())
+    if len(s) != 4:
+        raise ValueError("expected a 4-D tensor")
+    return _c_i64_4(*s)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("tensors must be on the GPU")
+
+
+def _bf16(t):
+    if t.dtype != torch.bfloat16:
+        raise TypeError("expected bfloat16")
+    return t
+
+
+def _i32(t):
+    if t.dtype != torch.int32 or not t.is_contiguous():
+        raise TypeError("expected a contiguous int32 tensor")
+    return t
+
+
+def page_budget(sink_tokens: int, local_tokens: int, budget_tokens: int, page_size: int):
+    """(n_sink, n_local, budget_pages, k_top): the header's token -> page reading."""
+    n_sink = -(-sink_tokens // page_size)
+    n_local = -(-local_tokens // page_size)
+    budget_pages = budget_tokens // page_size
+    return n_sink, n_local, budget_pages, budget_pages - n_sink - n_local
+
+
+def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tokens: int,
+                    local_tokens: int, budget_tokens: int, out_pages=None, out_counts=None,
+                    dev_error=None, P_pool: int = None, stream=None):
+    """q [B,T,Hq,Dk] bf16; summaries [P_pool,Hkv,Dk] bf16; page_table [B,max_pages];
+    seq_lens [B].  Returns (pages [B,Hkv,budget_pages], counts [B,Hkv])."""
+    lib = load()
+    _need_cuda(q, summaries, page_table, seq_lens)
+    _bf16(q), _bf16(summaries), _i32(page_table), _i32(seq_lens)
+    B, T, Hq, Dk = q.shape
+    P_pool_, Hkv, _ = summaries.shape
+    P_pool = P_pool_ if P_pool is None else P_pool
+    bp = budget_tokens // page_size
+    if out_pages is None:
+        out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
+    if out_counts is None:
+        out_counts = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    st = lib.sa_select_pages(_ptr(q), _strides4(q), _ptr(summaries.contiguous()), _ptr(page_table),
+                             _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size, page_table.shape[1],
+                             P_pool, sink_tokens, local_tokens, budget_tokens, _ptr(out_pages),
+                             _ptr(out_counts), _ptr(dev_error), _stream(stream))
+    _check(st, "sa_select_pages")
+    return out_pages, out_counts
+
+
+def sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, lists, list_counts, head_to_list,
+                     scale: float, n_splits: int = 1, o_partial=None, lse_partial=None,
+                     dev_error=None, stream=None):
+    """q [B,T,Hq,Dk]; k_cache [P_pool,Hkv,P,Dk]; v_cache [P_pool,Hkv,P,Dv] (any strides with a
+    unit feature stride); lists [B,n_lists,max_list]; list_counts [B,n_lists];
+    head_to_list: a host sequence of Hq list ids.  Returns (o_partial, lse_partial)."""
+    lib = load()
+    _need_cuda(q, k_cache, v_cache, page_table, seq_lens, lists, list_counts)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(page_table), _i32(seq_lens), _i32(lists)
+    _i32(list_counts)
+    B, T, Hq, Dk = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    Dv = v_cache.shape[-1]
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    if o_partial is None:
+        o_partial = torch.empty((n_splits, B, T, Hq, Dv), dtype=torch.float32, device=q.device)
+    if lse_partial is None:
+        lse_partial = torch.empty((n_splits, B, T, Hq), dtype=torch.float32, device=q.device)
+    st = lib.sa_sparse_decode(_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
+                              _ptr(v_cache), _strides4(v_cache), _ptr(page_table),
+                              page_table.shape[1], _ptr(seq_lens), _ptr(lists), _ptr(list_counts),
+                              n_lists, max_list, ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv,
+                              Dk, Dv, P, P_pool, float(scale), n_splits, _ptr(o_partial),
+                              _ptr(lse_partial), _ptr(dev_error), _stream(stream))
+    _check(st, "sa_sparse_decode")
+    return o_partial, lse_partial
+
+
+def sa_combine(o_partial, lse_partial, o_out=None, o_out_bf16=None, lse_out=None,
+               want_f32: bool = True, stream=None):
+    """o_partial [S,...,Dv] f32, lse_partial [S,...] f32 -> (O [...,Dv] f32, O bf16 or None,
+    lse [...])."""
+    lib = load()
+    _need_cuda(o_partial, lse_partial)
+    S = o_partial.shape[0]
+    Dv = o_partial.shape[-1]
+    lead = tuple(o_partial.shape[1:-1])
+    rows = lse_partial[0].numel()
+    if o_out is None and want_f32:
+        o_out = torch.empty(lead + (Dv,), dtype=torch.float32, device=o_partial.device)
+    if lse_out is None:
+        lse_out = torch.empty(lead, dtype=torch.float32, device=o_partial.device)
+    st = lib.sa_combine(_ptr(o_partial), _ptr(lse_partial), S, rows, Dv, _ptr(o_out),
+                        _ptr(o_out_bf16), _ptr(lse_out), _stream(stream))
+    _check(st, "sa_combine")
+    return o_out, o_out_bf16, lse_out
+
+
+def sa_build_page_summaries(k_cache, page_table, seq_lens, summaries=None, dev_error=None,
+                            stream=None):
+    """k_cache [P_pool,Hkv,P,Dk] bf16 -> summaries [P_pool,Hkv,Dk] bf16 (rows of referenced
+    pages written)."""
+    lib = load()
+    _need_cuda(k_cache, page_table, seq_lens)
+    _bf16(k_cache), _i32(page_table), _i32(seq_lens)
+    P_pool, Hkv, P, Dk = k_cache.shape
+    if summaries is None:
+        summaries = torch.zeros((P_pool, Hkv, Dk), dtype=torch.bfloat16, device=k_cache.device)
+    st = lib.sa_build_page_summaries(_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
+                                     page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], Hkv,
+                                     Dk, P, P_pool, _ptr(summaries), _ptr(dev_error),
+                                     _stream(stream))
+    _check(st, "sa_build_page_summaries")
+    return summaries
+
+
+def sa_block_union(scores, Hkv: int, q_block_offset: int, top_k: int, n_sink_blocks: int = 1,
+                   tables=None, counts=None, stream=None):
+    """scores [Hq,NQB,NKB] f32 -> (tables [Hkv,NKB] int32, counts [Hkv])."""
+    lib = load()
+    _need_cuda(scores)
+    if scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise TypeError("scores must be contiguous float32")
+    Hq, NQB, NKB = scores.shape
+    if tables is None:
+        tables = torch.empty((Hkv, NKB), dtype=torch.int32, device=scores.device)
+    if counts is None:
+        counts = torch.empty((Hkv,), dtype=torch.int32, device=scores.device)
+    st = lib.sa_block_union(_ptr(scores), Hq, Hkv, NQB, NKB, q_block_offset, top_k,
+                            n_sink_blocks, _ptr(tables), _ptr(counts), _stream(stream))
+    _check(st, "sa_block_union")
+    return tables, counts

@@ -1,0 +1,253 @@
+// C ABI: argument checks on the host, then kernel launches.  Nothing here
+// allocates device memory or synchronises.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace sa {
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Checks shared by the bf16 [*, Hkv, P, D] caches: feature stride 1, the
+// other strides multiples of 8 elements (16 bytes), 16-byte aligned base.
+int check_cache(const uint16_t* p, const int64_t s[4]) {
+  if (!p || !s) return SA_ERR_INVALID_ARG;
+  if (!aligned16(p) || s[3] != 1) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (s[i] <= 0 || (s[i] % 8) != 0) return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+int check_q(const uint16_t* q, const int64_t s[4]) {
+  if (!q || !s) return SA_ERR_INVALID_ARG;
+  if (!aligned16(q) || s[3] != 1) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (s[i] < 0 || (s[i] % 8) != 0) return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
+
+}  // namespace
+
+bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
+                   const int64_t strides[4]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)Hkv, (cuuint64_t)P_pool};
+  cuuint64_t gstr[3] = {(cuuint64_t)strides[2] * 2, (cuuint64_t)strides[1] * 2,
+                        (cuuint64_t)strides[0] * 2};
+  cuuint32_t box[4] = {64, 16, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, gstr,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+const char* sa_status_string(int status) {
+  switch (status) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA";
+    default: return "SA_ERR_UNKNOWN";
+  }
+}
+
+int sa_abi_version(void) { return 100; }
+
+int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                    const int32_t* page_table, const int32_t* seq_lens, int B, int T, int Hq,
+                    int Hkv, int Dk, int page_size, int max_pages, int P_pool, int sink_tokens,
+                    int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
+                    int32_t* dev_error, void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Dk <= 0 || page_size <= 0 ||
+      max_pages < 0 || P_pool < 0 || sink_tokens < 0 || local_tokens < 0 || budget_tokens < 0)
+    return SA_ERR_INVALID_ARG;
+  const int n_sink = (sink_tokens + page_size - 1) / page_size;
+  const int n_local = (local_tokens + page_size - 1) / page_size;
+  const int budget_pages = budget_tokens / page_size;
+  const int k_top = budget_pages - n_sink - n_local;
+  if (k_top < 0 || budget_pages <= 0) return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  if (int r = check_q(q, q_strides)) return r;
+  if (!summaries || !page_table || !seq_lens || !out_pages || !out_counts)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(summaries)) return SA_ERR_INVALID_ARG;
+  if (Dk != 64 && Dk != 128 && Dk != 256) return SA_ERR_UNSUPPORTED;
+  if (T * (Hq / Hkv) > 16 || max_pages > 16384) return SA_ERR_UNSUPPORTED;
+  SelectArgs a;
+  a.q = q;
+  a.qs0 = q_strides[0];
+  a.qs1 = q_strides[1];
+  a.qs2 = q_strides[2];
+  a.sig = summaries;
+  a.page_table = page_table;
+  a.seq_lens = seq_lens;
+  a.B = B;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Dk = Dk;
+  a.P = page_size;
+  a.max_pages = max_pages;
+  a.P_pool = P_pool;
+  a.n_sink = n_sink;
+  a.n_local = n_local;
+  a.budget_pages = budget_pages;
+  a.k_top = k_top;
+  a.out_pages = out_pages;
+  a.out_counts = out_counts;
+  a.err = dev_error;
+  return cuda_status(launch_select_gqa(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                     const int64_t k_strides[4], const uint16_t* v_cache,
+                     const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                     const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
+                     int n_lists, int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                     int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                     int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
+                     void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Dk <= 0 || Dv <= 0 ||
+      page_size <= 0 || max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 ||
+      n_splits <= 0 || !std::isfinite(scale) || !head_to_list)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  if (int r = check_q(q, q_strides)) return r;
+  if (int r = check_cache(k_cache, k_strides)) return r;
+  if (int r = check_cache(v_cache, v_strides)) return r;
+  if (!page_table || !seq_lens || !lists || !list_counts || !o_partial || !lse_partial)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(o_partial)) return SA_ERR_INVALID_ARG;
+  for (int h = 0; h < Hq; ++h)
+    if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
+  if (Dk != Dv || (Dk != 64 && Dk != 128 && Dk != 256)) return SA_ERR_UNSUPPORTED;
+  if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
+  if ((max_list + n_splits - 1) / n_splits > kMaxSplitEntries) return SA_ERR_UNSUPPORTED;
+
+  // (list, kv head) pairs and the heads that read them
+  PairTable pairs;
+  pairs.n_pairs = 0;
+  const int G = Hq / Hkv;
+  for (int kvh = 0; kvh < Hkv; ++kvh) {
+    for (int h = kvh * G; h < (kvh + 1) * G; ++h) {
+      const int l = head_to_list[h];
+      int pi = -1;
+      for (int i = 0; i < pairs.n_pairs; ++i)
+        if (pairs.list_of[i] == l && pairs.kvh_of[i] == kvh) pi = i;
+      if (pi < 0) {
+        if (pairs.n_pairs == kMaxPairs) return SA_ERR_UNSUPPORTED;
+        pi = pairs.n_pairs++;
+        pairs.list_of[pi] = l;
+        pairs.kvh_of[pi] = kvh;
+        pairs.n_heads[pi] = 0;
+      }
+      if ((pairs.n_heads[pi] + 1) * T > kMaxRowsPerPair) return SA_ERR_UNSUPPORTED;
+      pairs.heads[pi][pairs.n_heads[pi]++] = static_cast<int16_t>(h);
+    }
+  }
+  CUtensorMap kmap, vmap;
+  if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides) ||
+      !encode_kv_map(&vmap, v_cache, Dv, page_size, Hkv, P_pool, v_strides))
+    return SA_ERR_CUDA;
+  DecodeArgs a;
+  a.q = q;
+  a.qs0 = q_strides[0];
+  a.qs1 = q_strides[1];
+  a.qs2 = q_strides[2];
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.lists = lists;
+  a.counts = list_counts;
+  a.n_lists = n_lists;
+  a.max_list = max_list;
+  a.B = B;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Dk = Dk;
+  a.Dv = Dv;
+  a.P = page_size;
+  a.P_pool = P_pool;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_splits = n_splits;
+  a.o_part = o_partial;
+  a.lse_part = lse_partial;
+  a.err = dev_error;
+  return cuda_status(launch_decode_gqa(a, pairs, kmap, vmap, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,
+               int Dv, float* o_out, uint16_t* o_out_bf16, float* lse_out, void* stream) {
+  if (n_splits <= 0 || rows < 0 || Dv <= 0 || (Dv % 4) != 0) return SA_ERR_INVALID_ARG;
+  if (!o_partial || !lse_partial || (!o_out && !o_out_bf16 && !lse_out)) return SA_ERR_INVALID_ARG;
+  if (!aligned16(o_partial) || (o_out && !aligned16(o_out)) ||
+      (o_out_bf16 && (reinterpret_cast<uintptr_t>(o_out_bf16) & 7u)))
+    return SA_ERR_INVALID_ARG;
+  if (n_splits > 64) return SA_ERR_UNSUPPORTED;
+  if (rows == 0) return SA_OK;
+  return cuda_status(launch_combine(o_partial, lse_partial, n_splits, rows, Dv, o_out, o_out_bf16,
+                                    lse_out, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
+                            const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                            int B, int Hkv, int Dk, int page_size, int P_pool,
+                            uint16_t* summaries, int32_t* dev_error, void* stream) {
+  if (B < 0 || Hkv <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0 || max_pages == 0) return SA_OK;
+  if (!k_cache || !k_strides || k_strides[3] != 1 || !page_table || !seq_lens || !summaries)
+    return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k_strides[i] <= 0) return SA_ERR_INVALID_ARG;
+  if (max_pages > 65535 || B > 65535) return SA_ERR_UNSUPPORTED;
+  return cuda_status(launch_summaries(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv,
+                                      Dk, page_size, P_pool, summaries, dev_error,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int sa_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_block_offset,
+                   int top_k, int n_sink_blocks, int32_t* tables, int32_t* counts,
+                   void* stream) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv || NQB < 0 || NKB <= 0 || q_block_offset < 0 ||
+      top_k < 0 || n_sink_blocks < 0 || q_block_offset + NQB > NKB)
+    return SA_ERR_INVALID_ARG;
+  if (!tables || !counts || (NQB > 0 && !scores)) return SA_ERR_INVALID_ARG;
+  if (NKB > 16384 || NQB > 65535 || Hq > 65535) return SA_ERR_UNSUPPORTED;
+  return cuda_status(launch_block_union(scores, Hq, Hkv, NQB, NKB, q_block_offset, top_k,
+                                        n_sink_blocks, tables, counts,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

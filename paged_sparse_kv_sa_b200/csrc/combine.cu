@@ -1,0 +1,72 @@
+// Log-sum-exp merge of split-KV partials: lse = log sum_s exp(lse_s),
+// O = sum_s exp(lse_s - lse) O_s.  One thread per (row, 4 output columns),
+// 16-byte loads and stores; memory-bound.
+//
+// Source: the merge step of a split Flash-decode ("TileSparse", section
+// "Configuration": mode full = fused Flash-decode).
+#include "common.cuh"
+#include "internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kMaxSplitsCombine = 64;
+
+__global__ void __launch_bounds__(256)
+    combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                   int n_splits, int64_t rows, int Dv, float* __restrict__ o_out,
+                   uint16_t* __restrict__ o_bf16, float* __restrict__ lse_out) {
+  const int q4 = Dv / 4;
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= rows * q4) return;
+  const int64_t row = idx / q4;
+  const int c = (int)(idx % q4) * 4;
+  float m = -INFINITY;
+  for (int s = 0; s < n_splits; ++s) m = fmaxf(m, lse_part[s * rows + row]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lse = -INFINITY;
+  if (m != -INFINITY) {
+    float tot = 0.f;
+    float w[kMaxSplitsCombine];
+    for (int s = 0; s < n_splits; ++s) {
+      w[s] = __expf(lse_part[s * rows + row] - m);
+      tot += w[s];
+    }
+    const float inv = 1.f / tot;
+    for (int s = 0; s < n_splits; ++s) {
+      const float f = w[s] * inv;
+      if (f == 0.f) continue;
+      const float4 v = *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c);
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+      acc.z += f * v.z;
+      acc.w += f * v.w;
+    }
+    lse = m + logf(tot);
+  }
+  if (o_out) *reinterpret_cast<float4*>(o_out + row * Dv + c) = acc;
+  if (o_bf16) {
+    uint2 p;
+    p.x = pack_bf16(acc.x, acc.y);
+    p.y = pack_bf16(acc.z, acc.w);
+    *reinterpret_cast<uint2*>(o_bf16 + row * Dv + c) = p;
+  }
+  if (lse_out && c == 0) lse_out[row] = lse;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_splits, int64_t rows,
+                           int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,
+                           cudaStream_t stream) {
+  if (n_splits > kMaxSplitsCombine) return cudaErrorInvalidValue;
+  const int64_t n = rows * (Dv / 4);
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (n + threads - 1) / threads;
+  combine_kernel<<<(unsigned)blocks, threads, 0, stream>>>(o_part, lse_part, n_splits, rows, Dv,
+                                                           o_out, o_bf16, lse_out);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

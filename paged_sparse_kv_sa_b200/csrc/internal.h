@@ -1,0 +1,77 @@
+// Host-side declarations shared by the C-ABI layer and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/sa.h"
+
+namespace sa {
+
+constexpr int kMaxPairs = 128;       // (list, kv head) pairs one decode call may touch
+constexpr int kMaxRowsPerPair = 16;  // query rows (T x heads) one mma tile holds
+constexpr int kMaxSplitEntries = 1024;
+
+// Which heads of a call read which (list, kv head) pair; built on the host
+// from head_to_list so every CTA knows its query rows without a lookup.
+struct PairTable {
+  int n_pairs;
+  int list_of[kMaxPairs];
+  int kvh_of[kMaxPairs];
+  int n_heads[kMaxPairs];
+  int16_t heads[kMaxPairs][kMaxRowsPerPair];
+};
+
+struct DecodeArgs {
+  const uint16_t* q;
+  int64_t qs0, qs1, qs2;
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* seq_lens;
+  const int32_t* lists;
+  const int32_t* counts;
+  int n_lists, max_list;
+  int B, T, Hq, Hkv, Dk, Dv, P, P_pool;
+  float scale_log2;
+  int n_splits;
+  float* o_part;
+  float* lse_part;
+  int32_t* err;
+};
+
+// Encode a 4-D bf16 tensor map over a [P_pool, Hkv, P, D] cache with
+// 64-column x 16-row boxes and 128-byte swizzle.  false on failure.
+bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
+                   const int64_t strides[4]);
+
+cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
+                              const CUtensorMap& vmap, cudaStream_t stream);
+
+struct SelectArgs {
+  const uint16_t* q;
+  int64_t qs0, qs1, qs2;
+  const uint16_t* sig;
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  int B, T, Hq, Hkv, Dk, P, max_pages, P_pool;
+  int n_sink, n_local, budget_pages, k_top;
+  int32_t* out_pages;
+  int32_t* out_counts;
+  int32_t* err;
+};
+cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream);
+
+cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_splits, int64_t rows,
+                           int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,
+                           cudaStream_t stream);
+
+cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
+                             int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
+                             int P, int P_pool, uint16_t* sig, int32_t* err, cudaStream_t stream);
+
+cudaError_t launch_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_off,
+                               int top_k, int n_sink, int32_t* tables, int32_t* counts,
+                               cudaStream_t stream);
+
+}  // namespace sa

@@ -1,0 +1,77 @@
+// Per-page key summaries: sigma = RNE_bf16(RN64(RN64(sum of valid keys) / n)).
+//
+// One CTA per (logical page, sequence); threads walk the (kv head, feature)
+// columns.  The float64 sum of at most P bf16 values is exact whenever the
+// values span at most 53 - ceil(log2 P) - 1 bits (every bf16 is an integer
+// multiple of its lsb weight); columns that fail that test are re-summed in
+// the exact fixed-point accumulator.
+//
+// Source: "Universal Attention Engine — Declarative Sparse Attention for
+// Production", "Content-Dependent Dynamic Routing" (the router scores
+// mean(k_blocks), the block-mean key).
+#include "common.cuh"
+#include "exact.cuh"
+#include "internal.h"
+
+namespace sa {
+namespace {
+
+__global__ void __launch_bounds__(256)
+    summaries_kernel(const uint16_t* __restrict__ k, int64_t ks0, int64_t ks1, int64_t ks2,
+                     const int32_t* __restrict__ pt, int max_pages,
+                     const int32_t* __restrict__ seq_lens, int Hkv, int Dk, int P, int P_pool,
+                     uint16_t* __restrict__ sig, int32_t* err) {
+  const int p = blockIdx.x, b = blockIdx.y;
+  const int L = min(seq_lens[b], max_pages * P);
+  const int n = min(P, L - p * P);
+  if (n <= 0) return;
+  const int ph = pt[(int64_t)b * max_pages + p];
+  if (ph < 0 || ph >= P_pool) {
+    if (threadIdx.x == 0) set_dev_error(err, SA_DEVERR_POOL_RANGE);
+    return;
+  }
+  const int lg = 32 - __clz(n);   // >= ceil(log2 n) + 1 for n >= 1
+  for (int c = threadIdx.x; c < Hkv * Dk; c += blockDim.x) {
+    const int h = c / Dk, d = c % Dk;
+    const uint16_t* col = k + ph * ks0 + h * ks1 + d;
+    double s = 0.0;
+    int emax = -100000, umin = 100000;
+    for (int j = 0; j < n; ++j) {
+      const uint32_t bits = col[j * ks2];
+      if ((bits & 0x7fffu) == 0) continue;
+      const int E = (bits >> 7) & 0xff;
+      const int eb = E ? E : 1;
+      emax = max(emax, eb - 126);   // |x| < 2^(eb - 126)
+      umin = min(umin, eb - 134);   // x is a multiple of 2^(eb - 134)
+      s += static_cast<double>(bf16_bits_to_float(bits));
+    }
+    if (emax > -100000 && emax + lg - umin > 53) {
+      ExactAcc acc;
+      acc.clear();
+      for (int j = 0; j < n; ++j) {
+        uint32_t m;
+        int e;
+        bool neg;
+        bf16_fields(col[j * ks2], m, e, neg);
+        acc.add(m, e, neg);
+      }
+      s = acc.round_to_double();
+    }
+    const double mean = s / static_cast<double>(n);
+    sig[((int64_t)ph * Hkv + h) * Dk + d] = f64_to_bf16_rne(mean);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
+                             int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
+                             int P, int P_pool, uint16_t* sig, int32_t* err, cudaStream_t stream) {
+  if (B == 0 || max_pages == 0) return cudaSuccess;
+  dim3 grid(max_pages, B);
+  summaries_kernel<<<grid, 256, 0, stream>>>(k, ks[0], ks[1], ks[2], pt, max_pages, seq_lens, Hkv,
+                                             Dk, P, P_pool, sig, err);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

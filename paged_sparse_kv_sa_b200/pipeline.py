@@ -1,0 +1,77 @@
+"""One sparse-attention decode step (select -> decode -> combine) over
+preallocated buffers, so that a timed or graph-captured step allocates nothing.
+
+Every stage is a call through the C ABI; this module only sizes buffers and
+chooses the split count.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _lib
+
+
+def default_splits(n_units: int, max_list: int, sm_count: int = 148, ctas_per_sm: int = 4,
+                   min_pages: int = 4) -> int:
+    """Split count for ``n_units`` (sequence, list) pairs of up to ``max_list`` pages:
+    enough CTAs to cover ``ctas_per_sm`` per SM, but at least ``min_pages`` per split."""
+    if n_units <= 0 or max_list <= 0:
+        return 1
+    want = max(1, round(ctas_per_sm * sm_count / n_units))
+    cap = max(1, max_list // min_pages)
+    return max(1, min(want, cap, 64))
+
+
+class SparseDecodeStep:
+    """GQA sparse decode: per (sequence, kv head) page selection, then attention of
+    every head over its group's list, then the split merge.
+
+    Inputs live on the GPU (q, caches, page table, seq_lens, summaries); outputs are
+    ``self.o`` [B,T,Hq,D] float32 and ``self.lse`` [B,T,Hq].
+    """
+
+    def __init__(self, B: int, T: int, Hq: int, Hkv: int, D: int, page_size: int, max_pages: int,
+                 sink_tokens: int, local_tokens: int, budget_tokens: int, scale: float = None,
+                 n_splits: int = None, device="cuda", out_bf16: bool = False):
+        self.B, self.T, self.Hq, self.Hkv, self.D = B, T, Hq, Hkv, D
+        self.P = page_size
+        self.sink, self.local, self.budget = sink_tokens, local_tokens, budget_tokens
+        _, _, self.budget_pages, _ = _lib.page_budget(sink_tokens, local_tokens, budget_tokens,
+                                                      page_size)
+        self.scale = 1.0 / math.sqrt(D) if scale is None else scale
+        self.n_splits = (default_splits(B * Hkv, self.budget_pages) if n_splits is None
+                         else n_splits)
+        self.head_to_list = [h // (Hq // Hkv) for h in range(Hq)]
+        dev = torch.device(device)
+        self.pages = torch.empty((B, Hkv, self.budget_pages), dtype=torch.int32, device=dev)
+        self.counts = torch.empty((B, Hkv), dtype=torch.int32, device=dev)
+        self.o_part = torch.empty((self.n_splits, B, T, Hq, D), dtype=torch.float32, device=dev)
+        self.lse_part = torch.empty((self.n_splits, B, T, Hq), dtype=torch.float32, device=dev)
+        self.o = torch.empty((B, T, Hq, D), dtype=torch.float32, device=dev)
+        self.o_bf16 = (torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
+                       if out_bf16 else None)
+        self.lse = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
+        self.dev_error = torch.zeros((1,), dtype=torch.int32, device=dev)
+
+    def select(self, q, summaries, page_table, seq_lens, stream=None):
+        _lib.sa_select_pages(q, summaries, page_table, seq_lens, self.P, self.sink, self.local,
+                             self.budget, out_pages=self.pages, out_counts=self.counts,
+                             dev_error=self.dev_error, stream=stream)
+
+    def decode(self, q, k_cache, v_cache, page_table, seq_lens, stream=None):
+        _lib.sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, self.pages, self.counts,
+                              self.head_to_list, self.scale, self.n_splits,
+                              o_partial=self.o_part, lse_partial=self.lse_part,
+                              dev_error=self.dev_error, stream=stream)
+
+    def combine(self, stream=None):
+        _lib.sa_combine(self.o_part, self.lse_part, o_out=self.o, o_out_bf16=self.o_bf16,
+                        lse_out=self.lse, stream=stream)
+
+    def __call__(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
+        self.select(q, summaries, page_table, seq_lens, stream)
+        self.decode(q, k_cache, v_cache, page_table, seq_lens, stream)
+        self.combine(stream)
+        return self.o, self.lse

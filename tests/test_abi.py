@@ -1,0 +1,95 @@
+"""The C-ABI library loads, exports every entry point include/sa.h declares, and
+rejects bad arguments on the host before any launch.  CPU only: no call here
+reaches a kernel."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_sparse_kv_sa_b200 as sa
+from paged_sparse_kv_sa_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"SA_API\s+[\w\s\*]+?\b(sa_\w+)\s*\(", txt)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = sa.load()
+    names = declared_symbols()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) <= set(_lib.EXPORTED)
+
+
+def test_status_strings_and_version():
+    lib = sa.load()
+    assert lib.sa_abi_version() == 100
+    assert lib.sa_status_string(0) == b"SA_OK"
+    assert lib.sa_status_string(1) == b"SA_ERR_INVALID_ARG"
+    assert lib.sa_status_string(99) == b"SA_ERR_UNKNOWN"
+
+
+def _i64x4(*v):
+    return (ctypes.c_int64 * 4)(*v)
+
+
+def test_host_validation_rejects_bad_arguments():
+    lib = sa.load()
+    fake = ctypes.c_void_p(0x1000)      # never dereferenced: validation fails first
+    s = _i64x4(1024, 1024, 128, 1)
+    # Hq not a multiple of Hkv
+    assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 6, 4, 128, 16, 8, 8, 32, 64, 256,
+                               fake, fake, None, None) == 1
+    # sink + local above the budget
+    assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 8, 2, 128, 16, 8, 8, 512, 512,
+                               256, fake, fake, None, None) == 1
+    # null outputs
+    assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 8, 2, 128, 16, 8, 8, 32, 64, 256,
+                               None, fake, None, None) == 1
+    # unsupported head dim
+    assert lib.sa_select_pages(fake, _i64x4(96, 96, 96, 1), fake, fake, fake, 1, 1, 8, 2, 96, 16,
+                               8, 8, 32, 64, 256, fake, fake, None, None) == 2
+    # misaligned q / non-unit feature stride
+    assert lib.sa_select_pages(ctypes.c_void_p(0x1002), s, fake, fake, fake, 1, 1, 8, 2, 128, 16,
+                               8, 8, 32, 64, 256, fake, fake, None, None) == 1
+    assert lib.sa_select_pages(fake, _i64x4(1024, 1024, 128, 2), fake, fake, fake, 1, 1, 8, 2, 128,
+                               16, 8, 8, 32, 64, 256, fake, fake, None, None) == 1
+    h2l = (ctypes.c_int32 * 8)(0, 0, 0, 0, 1, 1, 1, 5)   # list id out of range
+    ks = _i64x4(4096, 2048, 128, 1)
+    args = [fake, s, fake, ks, fake, ks, fake, 8, fake, fake, fake, 2, 16,
+            ctypes.cast(h2l, ctypes.c_void_p), 1, 1, 8, 2, 128, 128, 16, 64, 0.1, 1, fake, fake,
+            None, None]
+    assert lib.sa_sparse_decode(*args) == 1
+    h2l[7] = 1
+    args[22] = float("nan")
+    assert lib.sa_sparse_decode(*args) == 1                  # non-finite scale
+    args[22] = 0.1
+    args[20] = 24                                              # page size not a multiple of 16
+    assert lib.sa_sparse_decode(*args) == 2
+    args[20] = 16
+    args[19] = 64                                              # Dk != Dv
+    assert lib.sa_sparse_decode(*args) == 2
+    # combine: Dv not a multiple of 4, no outputs
+    assert lib.sa_combine(fake, fake, 2, 10, 6, fake, None, None, None) == 1
+    assert lib.sa_combine(fake, fake, 2, 10, 8, None, None, None, None) == 1
+    # block union: offset past the end
+    assert lib.sa_block_union(fake, 8, 2, 4, 10, 8, 2, 1, fake, fake, None) == 1
+
+
+def test_calls_fail_loudly_without_gpu_tensors():
+    import torch
+    q = torch.zeros((1, 1, 8, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        sa.sa_select_pages(q, torch.zeros((4, 2, 64), dtype=torch.bfloat16),
+                           torch.zeros((1, 4), dtype=torch.int32),
+                           torch.zeros((1,), dtype=torch.int32), 16, 16, 16, 64)

@@ -1,0 +1,327 @@
+"""CUDA path vs the float64 oracle, through the C ABI (marked gpu).
+
+Tolerances: page selections and block tables bit-exact; summaries bit-exact;
+float32 outputs max-abs 2e-3 and LSE max-abs 1e-3 against the float64 oracle
+(bf16 inputs, float32 accumulation); the optional bf16 output within one bf16
+ulp of RNE_bf16(oracle) plus the float32 tolerance.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import paged_sparse_kv_sa_b200 as sa
+from paged_sparse_kv_sa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+O_TOL = 2e-3
+LSE_TOL = 1e-3
+DEV = "cuda"
+
+
+def bits(t):
+    return W.bf16_bits(t)
+
+
+def np_i32(t):
+    return t.detach().cpu().numpy().astype(np.int32)
+
+
+def assert_attn_close(o_gpu, lse_gpu, o_ref, lse_ref):
+    o_gpu = o_gpu.detach().cpu().double().numpy()
+    lse_gpu = lse_gpu.detach().cpu().double().numpy()
+    fin = np.isfinite(lse_ref)
+    assert np.array_equal(np.isfinite(lse_gpu), fin), "empty-row pattern differs"
+    err_o = np.abs(o_gpu - o_ref).max() if o_ref.size else 0.0
+    err_l = np.abs(lse_gpu[fin] - lse_ref[fin]).max() if fin.any() else 0.0
+    assert err_o <= O_TOL, f"max |O - O_ref| = {err_o}"
+    assert err_l <= LSE_TOL, f"max |lse - lse_ref| = {err_l}"
+    assert np.all(o_gpu[~fin] == 0)
+
+
+def gqa_case(cfg, seed=0, seq_lens=None):
+    inp = W.gqa_decode_inputs(cfg, seed=seed, device="cpu", seq_lens=seq_lens)
+    return inp, {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+
+
+def oracle_summaries(inp, cfg):
+    return O.page_summaries(bits(inp["k"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size)
+
+
+def to_bf16_dev(bits_np):
+    return torch.from_numpy(bits_np.view(np.int16)).view(torch.bfloat16).to(DEV)
+
+
+# ----------------------------------------------------------------------------
+# summaries
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("lens", [None, [2048 - 5]])
+def test_summaries_bitexact_tiny(lens):
+    cfg = W.TINY_GQA
+    inp, g = gqa_case(cfg, seed=1, seq_lens=lens)
+    ref = oracle_summaries(inp, cfg)
+    sig = sa.sa_build_page_summaries(g["k"], g["page_table"], g["seq_lens"])
+    torch.cuda.synchronize()
+    got = bits(sig)
+    used = np.unique(np_i32(inp["page_table"])[np_i32(inp["page_table"]) >= 0])
+    np.testing.assert_array_equal(got[used], ref[used])
+
+
+def test_summaries_exact_fallback_values():
+    # columns whose values span more than float64 can add exactly
+    P, Hkv, D = 16, 1, 64
+    k = torch.randn((3, Hkv, P, D)).to(torch.bfloat16)
+    kb = bits(k).copy()
+    kb[0, 0, :4, 0] = [0x7180, 0x3F80, 0xF180, 0x0001]   # 2^100, 1, -2^100, 2^-133
+    kb[1, 0, :, 1] = 0x0001                              # subnormals only
+    kb[2, 0, 0, 2] = 0x7F7F                              # near the top of the range
+    kb[2, 0, 1:, 2] = 0x0003
+    pt = np.array([[0, 1, 2]], dtype=np.int32)
+    sl = np.array([3 * P - 3], dtype=np.int32)
+    ref = O.page_summaries(kb, pt, sl, P)
+    sig = sa.sa_build_page_summaries(to_bf16_dev(kb), torch.from_numpy(pt).to(DEV),
+                                     torch.from_numpy(sl).to(DEV))
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(bits(sig), ref)
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+def run_select(g, sig_bits, cfg):
+    sig = to_bf16_dev(sig_bits)
+    pages, counts = sa.sa_select_pages(g["q"], sig, g["page_table"], g["seq_lens"], cfg.page_size,
+                                       cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    torch.cuda.synchronize()
+    return np_i32(pages), np_i32(counts)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_select_bitexact_tiny(seed):
+    cfg = W.TINY_GQA
+    inp, g = gqa_case(cfg, seed=seed)
+    sig = oracle_summaries(inp, cfg)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+
+
+def test_select_ragged_mtp_and_short_sequences():
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=5, T=2, Hq=16, Hkv=2, seq_len_lo=0, seq_len_hi=0,
+                   lift_frac=0.05, lift_sigma=3.0)
+    lens = [4000, 1023, 1025, 17, 0]
+    inp, g = gqa_case(cfg, seed=3, seq_lens=lens)
+    sig = oracle_summaries(inp, cfg)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+
+
+def test_select_ties_and_cancellation():
+    cfg = W.scaled(W.TINY_GQA, B=3)
+    inp, g = gqa_case(cfg, seed=4)
+    sig = oracle_summaries(inp, cfg).copy()
+    pt = np_i32(inp["page_table"])
+    qb = bits(inp["q"]).copy()
+    qb[0] = 0                                        # sequence 0: every score is 0
+    sig[pt[1, 40]] = sig[pt[1, 41]]                  # sequence 1: duplicated summaries
+    sig[pt[1, 42]] = sig[pt[1, 41]]
+    # sequence 2: a page whose exact score needs cancellation-free summation
+    sig[pt[2, 50], :, :] = 0
+    sig[pt[2, 50], :, 0] = 0x7180
+    sig[pt[2, 50], :, 1] = 0x7180
+    qb[2, 0, :, 0] = 0x3F80
+    qb[2, 0, :, 1] = 0xBF80
+    qb[2, 0, :, 2] = 0x4000
+    sig[pt[2, 50], :, 2] = 0x4480                    # 2 * 1024 = 2048 exactly
+    g["q"] = to_bf16_dev(qb)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(qb, sig, pt, np_i32(inp["seq_lens"]), cfg.page_size, cfg.sink_tokens,
+                            cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+    assert list(rp[0, 0, :12]) == list(range(12))   # ties -> lowest pages after the 2 sinks
+
+
+def test_select_streaming_k0():
+    cfg = W.scaled(W.TINY_GQA, budget_tokens=96)    # 2 sink + 4 local, no top-k
+    inp, g = gqa_case(cfg, seed=5)
+    sig = oracle_summaries(inp, cfg)
+    pages, counts = run_select(g, sig, cfg)
+    assert list(pages[0, 0, :counts[0, 0]]) == [0, 1, 124, 125, 126, 127]
+
+
+# ----------------------------------------------------------------------------
+# decode + combine
+# ----------------------------------------------------------------------------
+def oracle_lists(inp, cfg, sig):
+    return O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                          cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+
+
+def run_decode(g, lists, counts, cfg, n_splits, k=None, v=None, h2l=None):
+    Hq, Hkv = cfg.Hq, cfg.Hkv
+    h2l = [h // (Hq // Hkv) for h in range(Hq)] if h2l is None else h2l
+    o_p, l_p = sa.sa_sparse_decode(g["q"], g["k"] if k is None else k, g["v"] if v is None else v,
+                                   g["page_table"], g["seq_lens"],
+                                   torch.from_numpy(lists).to(DEV), torch.from_numpy(counts).to(DEV),
+                                   h2l, 1.0 / math.sqrt(cfg.D), n_splits)
+    o, ob, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+@pytest.mark.parametrize("n_splits", [1, 3])
+def test_decode_tiny_vs_oracle(n_splits):
+    cfg = W.TINY_GQA
+    inp, g = gqa_case(cfg, seed=0)
+    sig = oracle_summaries(inp, cfg)
+    lists, counts = oracle_lists(inp, cfg, sig)
+    o, lse = run_decode(g, lists, counts, cfg, n_splits)
+    h2l = np.arange(cfg.Hq) // cfg.G
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists, counts,
+                                h2l, 1.0 / math.sqrt(cfg.D), cfg.page_size)
+    assert_attn_close(o, lse, ro, rl)
+
+
+@pytest.mark.parametrize("D,P,T", [(128, 16, 1), (128, 16, 2), (64, 32, 2), (256, 16, 1),
+                                   (128, 64, 1)])
+def test_decode_shapes_ragged_vs_oracle(D, P, T):
+    cfg = W.GQADecode("case", B=3, Hq=8, Hkv=2, D=D, page_size=P, seq_len_lo=0, seq_len_hi=0,
+                      sink_tokens=P, local_tokens=2 * P, budget_tokens=12 * P, T=T)
+    lens = [50 * P + 7, 9 * P, 3 * P + 1]
+    inp, g = gqa_case(cfg, seed=6, seq_lens=lens)
+    sig = oracle_summaries(inp, cfg)
+    lists, counts = oracle_lists(inp, cfg, sig)
+    o, lse = run_decode(g, lists, counts, cfg, 2)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists, counts,
+                                np.arange(cfg.Hq) // cfg.G, 1.0 / math.sqrt(D), P)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_decode_per_head_lists_and_empty():
+    # QK 2D sparsity: heads of one kv group read different lists; one list empty
+    cfg = W.GQADecode("case", B=2, Hq=8, Hkv=2, D=128, page_size=16, seq_len_lo=0, seq_len_hi=0,
+                      sink_tokens=16, local_tokens=16, budget_tokens=160)
+    inp, g = gqa_case(cfg, seed=7, seq_lens=[700, 333])
+    rng = np.random.default_rng(7)
+    n_lists, cap = 3, 9
+    lists = np.full((2, n_lists, cap), -1, dtype=np.int32)
+    counts = np.zeros((2, n_lists), dtype=np.int32)
+    for b, L in enumerate([700, 333]):
+        nb = -(-L // 16)
+        for li in range(n_lists - 1):
+            c = int(rng.integers(1, cap + 1))
+            lists[b, li, :c] = np.sort(rng.choice(nb, c, replace=False))
+            counts[b, li] = c
+    h2l = [0, 1, 2, 0, 1, 1, 2, 0]
+    o, lse = run_decode(g, lists, counts, cfg, 2, h2l=h2l)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists, counts,
+                                np.array(h2l), 1.0 / math.sqrt(128), 16)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_decode_strided_cache_layout():
+    # the pool stored as [P_pool, P, Hkv, D] (vLLM order) and viewed through strides
+    cfg = W.scaled(W.TINY_GQA, B=2, seq_len_lo=1500, seq_len_hi=1500)
+    inp, g = gqa_case(cfg, seed=8)
+    sig = oracle_summaries(inp, cfg)
+    lists, counts = oracle_lists(inp, cfg, sig)
+    k_alt = g["k"].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    v_alt = g["v"].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    assert k_alt.stride() != g["k"].stride()
+    o, lse = run_decode(g, lists, counts, cfg, 2, k=k_alt, v=v_alt)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists, counts,
+                                np.arange(cfg.Hq) // cfg.G, 1.0 / math.sqrt(cfg.D), cfg.page_size)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_decode_bad_pages_flagged_not_trapped():
+    cfg = W.scaled(W.TINY_GQA, B=1)
+    inp, g = gqa_case(cfg, seed=9)
+    lists = np.array([[[0, 1, 5000, -3], [2, 3, 4, 5]]], dtype=np.int32)
+    counts = np.array([[4, 4]], dtype=np.int32)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    o_p, l_p = sa.sa_sparse_decode(g["q"], g["k"], g["v"], g["page_table"], g["seq_lens"],
+                                   torch.from_numpy(lists).to(DEV), torch.from_numpy(counts).to(DEV),
+                                   [0, 0, 0, 0, 1, 1, 1, 1], 0.125, 1, dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & 1          # SA_DEVERR_PAGE_RANGE
+    ok = np.array([[[0, 1, -1, -1], [2, 3, 4, 5]]], dtype=np.int32)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), ok,
+                                np.array([[2, 4]]), [0, 0, 0, 0, 1, 1, 1, 1], 0.125, 16)
+    assert_attn_close(o_p[0], l_p[0], ro, rl)
+
+
+def test_combine_vs_oracle():
+    rng = np.random.default_rng(11)
+    S, rows, Dv = 5, 37, 128
+    o = rng.standard_normal((S, rows, Dv)).astype(np.float32)
+    lse = (rng.standard_normal((S, rows)) * 3).astype(np.float32)
+    lse[1, :10] = -np.inf
+    lse[:, 20] = -np.inf                       # a row with every split empty
+    o[:, 20] = 0
+    ob = torch.empty((rows, Dv), dtype=torch.bfloat16, device=DEV)
+    go, _, gl = sa.sa_combine(torch.from_numpy(o).to(DEV), torch.from_numpy(lse).to(DEV),
+                              o_out_bf16=ob)
+    torch.cuda.synchronize()
+    ro, rl = O.combine(o.astype(np.float64), lse.astype(np.float64))
+    assert_attn_close(go, gl, ro, rl)
+    rb = O.bf16_to_f64(O.f64_to_bf16_rne(ro))
+    err = np.abs(ob.float().cpu().numpy() - rb)
+    assert np.all(err <= np.abs(rb) * 2.0 ** -7 + O_TOL)
+
+
+# ----------------------------------------------------------------------------
+# block union
+# ----------------------------------------------------------------------------
+def test_block_union_small_bitexact():
+    Hq, Hkv, NQB, off, top_k = 8, 2, 6, 40, 5
+    s = torch.randn((Hq, NQB, off + NQB), generator=torch.Generator().manual_seed(3))
+    s[0, 2, 10] = s[0, 2, 11]
+    tables, counts = sa.sa_block_union(s.to(DEV), Hkv, off, top_k)
+    torch.cuda.synchronize()
+    rt, rc = O.block_union(s.numpy(), Hkv, off, top_k)
+    np.testing.assert_array_equal(np_i32(counts), rc)
+    np.testing.assert_array_equal(np_i32(tables), rt)
+
+
+@pytest.mark.slow
+def test_block_union_full_size_sampled():
+    cfg = W.UNION_PREFILL
+    s = W.block_union_scores(cfg, seed=0, device="cpu")
+    off = cfg.q_offset // cfg.block
+    tables, counts = sa.sa_block_union(s.to(DEV), cfg.Hkv, off, cfg.top_k)
+    torch.cuda.synchronize()
+    t, c = np_i32(tables), np_i32(counts)
+    G = cfg.Hq // cfg.Hkv
+    rng = np.random.default_rng(0)
+    for g in range(cfg.Hkv):
+        row = t[g, :c[g]]
+        assert np.all(np.diff(row) > 0) and np.all(t[g, c[g]:] == -1)
+    # every sampled (head, Q-block) mask lies inside its group's table
+    sn = s.numpy()
+    for _ in range(24):
+        h, j = int(rng.integers(cfg.Hq)), int(rng.integers(cfg.n_q_blocks))
+        d = off + j
+        cand = np.arange(1, d)
+        win = O.rank_select(sn[h, j, cand].astype(np.float64), cand, cfg.top_k)
+        mask = {0, d} | set(cand[win].tolist())
+        assert mask <= set(t[h // G, :c[h // G]].tolist())
+    # exact equality on two full groups, recomputed by the oracle
+    rt, rc = O.block_union(sn[:2 * G], 2, off, cfg.top_k)
+    np.testing.assert_array_equal(c[:2], rc)
+    np.testing.assert_array_equal(t[:2], rt)
