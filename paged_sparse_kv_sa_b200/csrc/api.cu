@@ -152,7 +152,7 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
     if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
   if (Dk != Dv || (Dk != 64 && Dk != 128 && Dk != 256)) return SA_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
-  if ((max_list + n_splits - 1) / n_splits > kMaxSplitEntries) return SA_ERR_UNSUPPORTED;
+  if ((max_list + n_splits - 1) / n_splits > decode_max_split_entries()) return SA_ERR_UNSUPPORTED;
 
   // (list, kv head) pairs and the heads that read them
   PairTable pairs;

@@ -1,14 +1,17 @@
 // Gather-based split-KV Flash-decode over per-head page lists (GQA / MTP).
 //
-// One CTA per (split, (list, kv head) pair, sequence).  Each warp owns a ring
-// of shared-memory stages; its lane 0 gathers 16-token sub-pages of K and V
-// straight from the paged pool with TMA tile loads (page ids resolved through
-// the list and the page table), and the warp runs QK^T, an online softmax and
-// PV on them with m16n8k16 bf16 tensor-core MMAs: the 16 rows of the MMA are
-// the query rows (T x heads of the pair), the columns the 16 tokens.  The
-// probabilities enter PV as a bf16 hi + lo pair so that their rounding stays
-// far below the output tolerance.  Warps merge their (max, sum, O) states in
-// shared memory at the end and the CTA writes one normalised partial + LSE.
+// Every warp owns one split of one (list, kv head) pair of one sequence and
+// runs on its own: its lanes resolve the split's logical pages through the
+// list and the page table, lane 0 gathers 16-token sub-pages of K and V from
+// the paged pool with TMA tile loads (64-column x 16-row boxes, 128-byte
+// swizzle) into a private ring of shared-memory stages, and the warp runs
+// QK^T, an online softmax and PV with m16n8k16 bf16 tensor-core MMAs.  The 16
+// MMA rows are the query rows of the pair (T x heads), the columns the 16
+// tokens of a sub-page.  Probabilities enter PV as a bf16 hi + lo pair so
+// their rounding stays ~2^-17 relative; the running max is only moved when a
+// row's new maximum exceeds it by more than 2^8 (so P <= 256 and the O
+// rescale is rare).  The warp writes its normalised partial + LSE straight
+// from registers: no block-wide barrier, no merge through shared memory.
 //
 // Sources: "Universal Attention Engine — Declarative Sparse Attention for
 // Production" ("Architecture": gather-based sparse KV decode; "Key Design
@@ -20,8 +23,10 @@
 namespace sa {
 namespace {
 
-constexpr int kNW = 4;       // warps per CTA
-constexpr int kSub = 16;     // tokens per TMA sub-page (one MMA k-step of PV)
+constexpr int kNW = 4;              // warps (= splits) per CTA
+constexpr int kSub = 16;            // tokens per TMA sub-page (one MMA k-step of PV)
+constexpr int kWarpEntries = 128;   // list entries one split may hold
+constexpr float kLazy = 8.f;        // log2 headroom before the running max moves
 
 template <int D>
 struct DecodeCfg {
@@ -29,10 +34,8 @@ struct DecodeCfg {
   static constexpr int kBoxBytes = kSub * 128;              // 16 rows x 128 bytes
   static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one K (or V) sub-page
   static constexpr int kStageBytes = 2 * kTileBytes;        // K + V
-  static constexpr int kStages = D >= 256 ? 2 : 3;
-  static constexpr int kRingBytes = kNW * kStages * kStageBytes;
-  static constexpr int kMergeBytes = kNW * 16 * (D + 2) * 4;
-  static constexpr int kDynBytes = (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 1024;
+  static constexpr int kStages = D >= 128 ? 2 : 4;
+  static constexpr int kDynBytes = kNW * kStages * kStageBytes + 1024;
 };
 
 struct __align__(64) DecodeParams {
@@ -47,15 +50,15 @@ __global__ void __launch_bounds__(kNW * 32)
                       const __grid_constant__ CUtensorMap vmap) {
   using C = DecodeCfg<D>;
   const DecodeArgs& a = prm.a;
-  const int split = blockIdx.x, pair = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x * kNW + warp, pair = blockIdx.y, b = blockIdx.z;
+  if (split >= a.n_splits) return;
   const int gid = lane >> 2, tig = lane & 3;
 
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
   __shared__ uint64_t bars[kNW][C::kStages];
-  __shared__ int phys_s[kMaxSplitEntries];
-  __shared__ int page_s[kMaxSplitEntries];
+  __shared__ int2 ent_s[kNW][kWarpEntries];    // (physical page, first token) per entry
 
   const int list = prm.pairs.list_of[pair];
   const int kvh = prm.pairs.kvh_of[pair];
@@ -63,62 +66,55 @@ __global__ void __launch_bounds__(kNW * 32)
   const int R = a.T * nh;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) {  // a length the page table cannot hold
-    if (tid == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
+    if (lane == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
     L = L < 0 ? 0 : a.max_pages * a.P;
   }
   const int n_log = (L + a.P - 1) / a.P;
 
   int count = a.counts[b * a.n_lists + list];
   if (count < 0 || count > a.max_list) {
-    if (tid == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
+    if (lane == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
     count = count < 0 ? 0 : a.max_list;
   }
   const int chunk = (count + a.n_splits - 1) / a.n_splits;
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
 
-  // Resolve logical -> physical page ids for this split once.
-  const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list;
-  for (int i = tid; i < n_ent; i += blockDim.x) {
-    int p = lrow[e0 + i];
+  if (lane == 0) {
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+  }
+  // Resolve logical -> physical pages of this split (32 entries per round).
+  const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
+  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+  for (int i = lane; i < n_ent; i += 32) {
+    const int p = lrow[i];
     int ph = -1;
     if (p < 0 || p >= n_log) {
       set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
     } else {
-      ph = a.page_table[(int64_t)b * a.max_pages + p];
+      ph = ptrow[p];
       if (ph < 0 || ph >= a.P_pool) {
         set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
         ph = -1;
       }
     }
-    phys_s[i] = ph;
-    page_s[i] = p;
+    ent_s[warp][i] = make_int2(ph, p * a.P);
   }
-  if (lane == 0)
-    for (int s = 0; s < C::kStages; ++s) mbar_init(&bars[warp][s], 1);
-  if (tid == 0) {
-    prefetch_tmap(&kmap);
-    prefetch_tmap(&vmap);
-  }
-  fence_mbar_init();
-  __syncthreads();
+  __syncwarp();
 
   const int subs = a.P / kSub;
   const int n_units = n_ent * subs;
-  const int my_units = n_units > warp ? (n_units - warp + kNW - 1) / kNW : 0;
   uint8_t* ring = smem + warp * C::kStages * C::kStageBytes;
 
-  // A unit is (entry, 16-token sub-page); it carries data iff its page is
-  // valid and some of its tokens lie before the sequence end.
   auto unit_live = [&](int u, int& ph, int& tok0) {
-    const int e = u / subs, st = u % subs;
-    ph = phys_s[e];
-    tok0 = page_s[e] * a.P + st * kSub;
+    const int2 e = ent_s[warp][u / subs];
+    ph = e.x;
+    tok0 = e.y + (u % subs) * kSub;
     return ph >= 0 && tok0 < L;
   };
-  auto issue = [&](int k) {  // lane 0 only: unit number k of this warp
-    const int u = warp + k * kNW;
-    const int slot = k % C::kStages;
+  auto issue = [&](int u) {  // lane 0 only
+    const int slot = u % C::kStages;
     uint64_t* bar = &bars[warp][slot];
     int ph, tok0;
     if (unit_live(u, ph, tok0)) {
@@ -135,8 +131,11 @@ __global__ void __launch_bounds__(kNW * 32)
       mbar_arrive_expect_tx(bar, 0);
     }
   };
-  if (lane == 0)
-    for (int k = 0; k < my_units && k < C::kStages; ++k) issue(k);
+  if (lane == 0) {
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+    for (int u = 0; u < n_units && u < C::kStages; ++u) issue(u);
+  }
 
   // Query fragments (A operand of QK^T), rows r = t * nh + i.
   uint32_t qa[D / 16][4];
@@ -169,25 +168,25 @@ __global__ void __launch_bounds__(kNW * 32)
   float o[D / 8][4];
 #pragma unroll
   for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  float m_run[2] = {-INFINITY, -INFINITY};
+  float m_ref[2] = {-INFINITY, -INFINITY};   // base-2 reference max per row
   float l_run[2] = {0.f, 0.f};
-  int k_fail = -1;
+  int u_fail = -1;
+  const int mi = lane >> 3, ri = lane & 7;
 
-  for (int k = 0; k < my_units; ++k) {
-    const int u = warp + k * kNW;
-    const int slot = k % C::kStages;
-    if (!mbar_wait_bounded(&bars[warp][slot], (k / C::kStages) & 1)) {
-      k_fail = k;
+  for (int u = 0; u < n_units; ++u) {
+    const int slot = u % C::kStages;
+    if (!mbar_wait_bounded(&bars[warp][slot], (u / C::kStages) & 1)) {
+      u_fail = u;
       break;
     }
     int ph, tok0;
     if (unit_live(u, ph, tok0)) {
       const uint8_t* kt = ring + slot * C::kStageBytes;
-      const uint8_t* vt = kt + C::kTileBytes;
-      const uint32_t kbase = smem_u32(kt), vbase = smem_u32(vt);
-      // ---- S = Q K^T (16 rows x 16 tokens)
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      const int mi = lane >> 3, ri = lane & 7;
+      const uint32_t kbase = smem_u32(kt), vbase = smem_u32(kt + C::kTileBytes);
+      // ---- S = Q K^T (16 rows x 16 tokens): 4 independent accumulation chains
+      float s4[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) s4[i][0] = s4[i][1] = s4[i][2] = s4[i][3] = 0.f;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const int colb = (kk & 3) * 16;
@@ -195,10 +194,16 @@ __global__ void __launch_bounds__(kNW * 32)
                               swz128(8 * (mi >> 1) + ri, colb + 8 * (mi & 1));
         uint32_t r[4];
         ldmatrix_x4(r, addr);
-        mma_bf16_16816(s[0], qa[kk], r[0], r[1]);
-        mma_bf16_16816(s[1], qa[kk], r[2], r[3]);
+        mma_bf16_16816(s4[kk & 1], qa[kk], r[0], r[1]);
+        mma_bf16_16816(s4[2 + (kk & 1)], qa[kk], r[2], r[3]);
       }
-      // ---- mask, online softmax (base 2)
+      float s[2][4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        s[0][c] = s4[0][c] + s4[1][c];
+        s[1][c] = s4[2][c] + s4[3][c];
+      }
+      // ---- mask, lazily re-based online softmax (base 2)
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
@@ -210,33 +215,38 @@ __global__ void __launch_bounds__(kNW * 32)
           s[nt][c] = ok ? s[nt][c] * a.scale_log2 : -INFINITY;
           mx[h] = fmaxf(mx[h], s[nt][c]);
         }
-      float alpha[2], base[2];
+      bool move[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 1));
         mx[h] = fmaxf(mx[h], __shfl_xor_sync(0xffffffffu, mx[h], 2));
-        const float m_new = fmaxf(m_run[h], mx[h]);
-        base[h] = m_new == -INFINITY ? 0.f : m_new;
-        alpha[h] = exp2f(m_run[h] - base[h]);
-        m_run[h] = m_new;
+        move[h] = mx[h] > m_ref[h] + kLazy;
       }
-      float rs[2] = {0.f, 0.f};
+      if (__any_sync(0xffffffffu, move[0] || move[1])) {
+        float alpha[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          alpha[h] = move[h] ? exp2f(m_ref[h] - mx[h]) : 1.f;
+          if (move[h]) m_ref[h] = mx[h];
+          l_run[h] *= alpha[h];
+        }
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+          o[i][0] *= alpha[0];
+          o[i][1] *= alpha[0];
+          o[i][2] *= alpha[1];
+          o[i][3] *= alpha[1];
+        }
+      }
+      const float base[2] = {m_ref[0] == -INFINITY ? 0.f : m_ref[0],
+                             m_ref[1] == -INFINITY ? 0.f : m_ref[1]};
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           s[nt][c] = exp2f(s[nt][c] - base[c >> 1]);
-          rs[c >> 1] += s[nt][c];
+          l_run[c >> 1] += s[nt][c];
         }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) l_run[h] = l_run[h] * alpha[h] + rs[h];
-#pragma unroll
-      for (int i = 0; i < D / 8; ++i) {
-        o[i][0] *= alpha[0];
-        o[i][1] *= alpha[0];
-        o[i][2] *= alpha[1];
-        o[i][3] *= alpha[1];
-      }
       // ---- O += P V with P = hi + lo (both bf16)
       uint32_t ph_[4], pl_[4];
       {
@@ -258,77 +268,43 @@ __global__ void __launch_bounds__(kNW * 32)
         uint32_t r[4];
         ldmatrix_x4_trans(r, addr);
         mma_bf16_16816(o[2 * n2], ph_, r[0], r[1]);
-        mma_bf16_16816(o[2 * n2], pl_, r[0], r[1]);
         mma_bf16_16816(o[2 * n2 + 1], ph_, r[2], r[3]);
+        mma_bf16_16816(o[2 * n2], pl_, r[0], r[1]);
         mma_bf16_16816(o[2 * n2 + 1], pl_, r[2], r[3]);
       }
     }
     __syncwarp();
-    if (lane == 0 && k + C::kStages < my_units) issue(k + C::kStages);
+    if (lane == 0 && u + C::kStages < n_units) issue(u + C::kStages);
   }
-  if (k_fail >= 0) {
+  if (u_fail >= 0) {
     if (lane == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
-    // Units k_fail .. k_fail + kStages - 1 were issued; wait for them (again
-    // bounded) before the shared memory they target is reused.
-    for (int kk = k_fail + 1; kk < my_units && kk < k_fail + C::kStages; ++kk)
-      mbar_wait_bounded(&bars[warp][kk % C::kStages], (kk / C::kStages) & 1);
+    // units u_fail .. u_fail + kStages - 1 were issued: wait for them (bounded)
+    // before this warp's shared memory can be released
+    for (int u = u_fail + 1; u < n_units && u < u_fail + C::kStages; ++u)
+      mbar_wait_bounded(&bars[warp][u % C::kStages], (u / C::kStages) & 1);
   }
 
-  // ---- merge the warps' states
+  // ---- normalise and write this split's partial from registers
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
     l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
   }
-  __syncthreads();  // every warp is done with its ring
-  float* mrg = reinterpret_cast<float*>(smem);
-  float* mrg_m = mrg;                         // [kNW][16]
-  float* mrg_l = mrg + kNW * 16;              // [kNW][16]
-  float* mrg_o = mrg + 2 * kNW * 16;          // [kNW][16][D]
-  if (tig == 0) {
-    mrg_m[warp * 16 + gid] = m_run[0];
-    mrg_m[warp * 16 + gid + 8] = m_run[1];
-    mrg_l[warp * 16 + gid] = l_run[0];
-    mrg_l[warp * 16 + gid + 8] = l_run[1];
-  }
 #pragma unroll
-  for (int i = 0; i < D / 8; ++i) {
-    const int d = i * 8 + 2 * tig;
-    float* r0 = mrg_o + (warp * 16 + gid) * D + d;
-    float* r1 = mrg_o + (warp * 16 + gid + 8) * D + d;
-    *reinterpret_cast<float2*>(r0) = make_float2(o[i][0], o[i][1]);
-    *reinterpret_cast<float2*>(r1) = make_float2(o[i][2], o[i][3]);
-  }
-  __syncthreads();
-  const int64_t row_stride_t = (int64_t)a.Hq;
-  for (int idx = tid; idx < R * (D / 4); idx += blockDim.x) {
-    const int r = idx / (D / 4), d = (idx % (D / 4)) * 4;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kNW; ++w) M = fmaxf(M, mrg_m[w * 16 + r]);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float Lsum = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float f = exp2f(mrg_m[w * 16 + r] - M);
-        Lsum += mrg_l[w * 16 + r] * f;
-        const float4 v = *reinterpret_cast<const float4*>(mrg_o + (w * 16 + r) * D + d);
-        acc.x += v.x * f;
-        acc.y += v.y * f;
-        acc.z += v.z * f;
-        acc.w += v.w * f;
-      }
-      const float inv = 1.f / Lsum;
-      acc.x *= inv;
-      acc.y *= inv;
-      acc.z *= inv;
-      acc.w *= inv;
-    }
+  for (int h = 0; h < 2; ++h) {
+    const int r = gid + 8 * h;
+    if (r >= R) continue;
     const int t = r / nh, head = prm.pairs.heads[pair][r % nh];
-    const int64_t row = (((int64_t)split * a.B + b) * a.T + t) * row_stride_t + head;
-    *reinterpret_cast<float4*>(a.o_part + row * D + d) = acc;
-    if (d == 0) a.lse_part[row] = M == -INFINITY ? -INFINITY : (M + log2f(Lsum)) * kLn2;
+    const int64_t row = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
+    const bool empty = l_run[h] == 0.f;
+    const float inv = empty ? 0.f : 1.f / l_run[h];
+    float* dst = a.o_part + row * D;
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i)
+      *reinterpret_cast<float2*>(dst + i * 8 + 2 * tig) =
+          make_float2(o[i][2 * h] * inv, o[i][2 * h + 1] * inv);
+    if (tig == 0)
+      a.lse_part[row] = empty ? -INFINITY : (m_ref[h] + log2f(l_run[h])) * kLn2;
   }
 }
 
@@ -342,12 +318,14 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDynBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.n_splits, pairs.n_pairs, a.B);
+  dim3 grid((a.n_splits + kNW - 1) / kNW, pairs.n_pairs, a.B);
   decode_gqa_kernel<D><<<grid, kNW * 32, C::kDynBytes, stream>>>(prm, kmap, vmap);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+int decode_max_split_entries() { return kWarpEntries; }
 
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream) {

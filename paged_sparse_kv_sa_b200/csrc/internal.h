@@ -45,6 +45,7 @@ struct DecodeArgs {
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
                    const int64_t strides[4]);
 
+int decode_max_split_entries();
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream);
 

@@ -13,15 +13,21 @@ import torch
 from . import _lib
 
 
-def default_splits(n_units: int, max_list: int, sm_count: int = 148, ctas_per_sm: int = 4,
-                   min_pages: int = 4) -> int:
-    """Split count for ``n_units`` (sequence, list) pairs of up to ``max_list`` pages:
-    enough CTAs to cover ``ctas_per_sm`` per SM, but at least ``min_pages`` per split."""
+def default_splits(n_units: int, max_list: int, sm_count: int = 148, ctas_per_sm: int = 3,
+                   warps_per_cta: int = 4, max_entries: int = 128) -> int:
+    """Split count for ``n_units`` (sequence, list) pairs of up to ``max_list`` pages.
+
+    The decode kernel runs one split per warp, four warps per CTA, three CTAs per
+    SM; take as many whole CTAs per pair as fit in one wave, and at least enough
+    splits that none holds more than ``max_entries`` pages."""
     if n_units <= 0 or max_list <= 0:
         return 1
-    want = max(1, round(ctas_per_sm * sm_count / n_units))
-    cap = max(1, max_list // min_pages)
-    return max(1, min(want, cap, 64))
+    ctas = max(1, (ctas_per_sm * sm_count) // n_units)
+    n = warps_per_cta * ctas
+    n = min(n, max(1, max_list))
+    while -(-max_list // n) > max_entries:
+        n += 1
+    return max(1, min(n, 64))
 
 
 class SparseDecodeStep:
