@@ -7,9 +7,9 @@
  *    Declarative Sparse Attention for Production", "The Product" for the
  *    sink/local/budget pattern and "Content-Dependent Dynamic Routing" for
  *    top_k_blocks(q @ mean(k_blocks))).
- *  - sa_select_pages_tiered: the Critical/Ambient tier selection of "TileSparse:
+ *  - sa_select_pages_tiered: TileSparse's Critical/Ambient tiers ("TileSparse:
  *    Arithmetic-Intensity-Aware Sparse Attention for Compute-Bound LLM
- *    Decoding", "Motivation" (alpha pages for all heads, beta pages for h heads).
+ *    Decoding", "Motivation").
  *  - sa_sparse_decode: attention over per-head page lists read in place from a
  *    paged cache (UAE "Architecture": gather-based sparse KV decode over a
  *    PagedAttention-compatible layout; TileSparse "Two implementations": a
@@ -25,8 +25,8 @@
  * Conventions for every call:
  *  - Pointers marked (dev) are caller-owned device memory on the current
  *    device; (host) pointers are read before the call returns.  The library
- *    allocates nothing and keeps no state between calls except a cache of
- *    TMA descriptors keyed by their inputs.
+ *    allocates nothing and keeps no state between calls; scratch space
+ *    (workspace) is caller-owned device memory of the size a *_size call gives.
  *  - bf16 tensors are passed as uint16_t bit patterns.  Strides are in
  *    elements; the innermost (feature) stride must be 1, other strides of
  *    bf16 tensors multiples of 8 elements, base pointers 16-byte aligned.
@@ -99,14 +99,58 @@ SA_API int sa_abi_version(void);
  *  out_pages  (dev) [B,Hkv,budget_pages] int32: selected logical ids ascending,
  *                   then -1 padding
  *  out_counts (dev) [B,Hkv] int32
+ *  workspace  (dev) sa_select_workspace_size(B, Hkv, max_pages) bytes (may be
+ *                   NULL when k_top == 0); SA_ERR_WORKSPACE if missing or short
  * Supported: Dk in {64,128,256}, T*Hq/Hkv <= 16, max_pages <= 16384.
+ * Two launches: a scoring pass over all candidate pages (every SM streams
+ * summaries) and one selection block per (b, g).
  */
 SA_API int sa_select_pages(const uint16_t* q, const int64_t q_strides[4],
-                    const uint16_t* summaries, const int32_t* page_table,
-                    const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
-                    int page_size, int max_pages, int P_pool, int sink_tokens,
-                    int local_tokens, int budget_tokens, int32_t* out_pages,
-                    int32_t* out_counts, int32_t* dev_error, void* stream);
+                           const uint16_t* summaries, const int32_t* page_table,
+                           const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
+                           int page_size, int max_pages, int P_pool, int sink_tokens,
+                           int local_tokens, int budget_tokens, int32_t* out_pages,
+                           int32_t* out_counts, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_error, void* stream);
+
+/* Bytes of device workspace sa_select_pages needs (16-byte aligned, no
+ * initial contents; the call overwrites it): the float32 lower/upper score
+ * bounds of every page, [B, Hkv, max_pages] x 8 bytes.  0 for bad sizes. */
+SA_API size_t sa_select_workspace_size(int B, int Hkv, int max_pages);
+
+/*
+ * sa_select_pages_tiered — Critical / Ambient tier selection for one shared
+ * latent KV head (MLA; "TileSparse: Arithmetic-Intensity-Aware Sparse
+ * Attention for Compute-Bound LLM Decoding", "Motivation": a Critical Tier of
+ * alpha pages computed with all query heads, an Ambient Tier of beta pages
+ * computed with h heads).
+ *
+ * Every logical page p < N_b of sequence b is a candidate, scored by the max
+ * over all T x Hq query rows of q[b,t,h,:] . summaries[page_table[b,p],0,:]
+ * (unscaled, correctly rounded to float64).  Ranked by (score desc, logical
+ * page asc), the first alpha pages form the critical tier and the next beta
+ * the ambient tier.  Output as two decode lists per sequence:
+ *   lists[b,0,:] = critical pages ascending, lists[b,1,:] = critical + ambient
+ *   pages ascending, each -1 padded to alpha+beta; list_counts[b,0..1].
+ * Give sa_sparse_decode head_to_list[h] = 1 for the ambient heads, 0 for the
+ * rest.
+ *
+ *  q          (dev) [B,T,Hq,Dk] bf16, strides q_strides
+ *  summaries  (dev) [P_pool,1,Dk] bf16, contiguous
+ *  page_table (dev) [B,max_pages] int32;  seq_lens (dev) [B] int32
+ *  lists      (dev) [B,2,alpha+beta] int32;  list_counts (dev) [B,2] int32
+ *  workspace  (dev) sa_select_tiered_workspace_size(B,T,Hq,max_pages) bytes
+ * Supported: Dk % 8 == 0, Dk <= 1024, max_pages <= 16384.
+ */
+SA_API int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
+                                  const uint16_t* summaries, const int32_t* page_table,
+                                  const int32_t* seq_lens, int B, int T, int Hq, int Dk,
+                                  int page_size, int max_pages, int P_pool, int alpha, int beta,
+                                  int32_t* lists, int32_t* list_counts, void* workspace,
+                                  size_t workspace_bytes, int32_t* dev_error, void* stream);
+
+/* Bytes of workspace sa_select_pages_tiered needs (16-byte aligned). */
+SA_API size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_pages);
 
 /*
  * sa_sparse_decode — split-KV attention over per-head page lists.

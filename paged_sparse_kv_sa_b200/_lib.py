@@ -15,7 +15,7 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libsa.so")
+LIB_PATH = os.environ.get("PAGED_SPARSE_KV_SA_LIB") or os.path.join(_HERE, "libsa.so")
 
 _c_i64_4 = ctypes.c_int64 * 4
 _P = ctypes.c_void_p
@@ -27,7 +27,11 @@ _SIGNATURES = {
     "sa_status_string": (ctypes.c_char_p, [_I]),
     "sa_abi_version": (_I, []),
     "sa_select_pages": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
-                             _I, _P, _P, _P, _P]),
+                             _I, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "sa_select_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "sa_select_pages_tiered": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                    _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "sa_select_tiered_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "sa_sparse_decode": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P, _I,
                               _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P]),
     "sa_combine": (_I, [_P, _P, _I, _I64, _I, _P, _P, _P, _P]),
@@ -109,11 +113,16 @@ def page_budget(sink_tokens: int, local_tokens: int, budget_tokens: int, page_si
     return n_sink, n_local, budget_pages, budget_pages - n_sink - n_local
 
 
+def sa_select_workspace_size(B: int, Hkv: int, max_pages: int) -> int:
+    return int(load().sa_select_workspace_size(B, Hkv, max_pages))
+
+
 def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tokens: int,
                     local_tokens: int, budget_tokens: int, out_pages=None, out_counts=None,
-                    dev_error=None, P_pool: int = None, stream=None):
+                    workspace=None, dev_error=None, P_pool: int = None, stream=None):
     """q [B,T,Hq,Dk] bf16; summaries [P_pool,Hkv,Dk] bf16; page_table [B,max_pages];
-    seq_lens [B].  Returns (pages [B,Hkv,budget_pages], counts [B,Hkv])."""
+    seq_lens [B]; workspace: a uint8 device tensor of sa_select_workspace_size bytes
+    (allocated here when None).  Returns (pages [B,Hkv,budget_pages], counts [B,Hkv])."""
     lib = load()
     _need_cuda(q, summaries, page_table, seq_lens)
     _bf16(q), _bf16(summaries), _i32(page_table), _i32(seq_lens)
@@ -125,12 +134,44 @@ def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tok
         out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
     if out_counts is None:
         out_counts = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    max_pages = page_table.shape[1]
+    if workspace is None:
+        workspace = torch.empty(max(sa_select_workspace_size(B, Hkv, max_pages), 16),
+                                dtype=torch.uint8, device=q.device)
     st = lib.sa_select_pages(_ptr(q), _strides4(q), _ptr(summaries.contiguous()), _ptr(page_table),
-                             _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size, page_table.shape[1],
+                             _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size, max_pages,
                              P_pool, sink_tokens, local_tokens, budget_tokens, _ptr(out_pages),
-                             _ptr(out_counts), _ptr(dev_error), _stream(stream))
+                             _ptr(out_counts), _ptr(workspace), workspace.numel(),
+                             _ptr(dev_error), _stream(stream))
     _check(st, "sa_select_pages")
     return out_pages, out_counts
+
+
+def sa_select_pages_tiered(q, summaries, page_table, seq_lens, page_size: int, alpha: int,
+                           beta: int, lists=None, list_counts=None, workspace=None,
+                           dev_error=None, stream=None):
+    """q [B,T,Hq,Dk]; summaries [P_pool,1,Dk].  Returns (lists [B,2,alpha+beta],
+    counts [B,2]): list 0 = critical pages, list 1 = critical + ambient pages."""
+    lib = load()
+    _need_cuda(q, summaries, page_table, seq_lens)
+    _bf16(q), _bf16(summaries), _i32(page_table), _i32(seq_lens)
+    B, T, Hq, Dk = q.shape
+    P_pool = summaries.shape[0]
+    max_pages = page_table.shape[1]
+    if lists is None:
+        lists = torch.empty((B, 2, alpha + beta), dtype=torch.int32, device=q.device)
+    if list_counts is None:
+        list_counts = torch.empty((B, 2), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        n = int(lib.sa_select_tiered_workspace_size(B, T, Hq, max_pages))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    st = lib.sa_select_pages_tiered(_ptr(q), _strides4(q), _ptr(summaries.contiguous()),
+                                    _ptr(page_table), _ptr(seq_lens), B, T, Hq, Dk, page_size,
+                                    max_pages, P_pool, alpha, beta, _ptr(lists),
+                                    _ptr(list_counts), _ptr(workspace), workspace.numel(),
+                                    _ptr(dev_error), _stream(stream))
+    _check(st, "sa_select_pages_tiered")
+    return lists, list_counts
 
 
 def sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, lists, list_counts, head_to_list,

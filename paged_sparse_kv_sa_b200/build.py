@@ -19,8 +19,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
-SOURCES = ["api.cu", "decode.cu", "select.cu", "combine.cu", "summaries.cu", "union.cu"]
-HEADERS = ["common.cuh", "exact.cuh", "internal.h", os.path.join("..", "..", "include", "sa.h")]
+SOURCES = ["api.cu", "decode.cu", "prefill.cu", "select.cu", "select_mla.cu", "combine.cu", "summaries.cu",
+           "union.cu"]
+HEADERS = ["common.cuh", "exact.cuh", "tc05.cuh", "topk.cuh", "internal.h", os.path.join("..", "..", "include", "sa.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]
 
@@ -36,31 +37,35 @@ def _newest(paths):
     return max(os.path.getmtime(p) for p in paths if os.path.exists(p))
 
 
-def _compile(src: str, force: bool) -> str:
-    out = os.path.join(OBJ, os.path.splitext(src)[0] + ".o")
+def _compile(src: str, force: bool, obj_dir: str = OBJ, defines=()) -> str:
+    out = os.path.join(obj_dir, os.path.splitext(src)[0] + ".o")
     deps = [os.path.join(CSRC, src)] + [os.path.join(CSRC, h) for h in HEADERS]
     if not force and os.path.exists(out) and os.path.getmtime(out) >= _newest(deps):
         return out
-    cmd = [nvcc(), *ARCH, *FLAGS, "-c", os.path.join(CSRC, src), "-o", out]
+    cmd = [nvcc(), *ARCH, *FLAGS, *[f"-D{d}" for d in defines], "-c", os.path.join(CSRC, src),
+           "-o", out]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")
     return out
 
 
-def build(jobs: int = 0, force: bool = False, verbose: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(jobs: int = 0, force: bool = False, verbose: bool = False, defines=(), out: str = LIB,
+          obj_dir: str = OBJ) -> str:
+    """Compile every source and link ``out``; ``defines`` are extra -D macros
+    (build-time kernel shapes, e.g. SA_DECODE_WARPS=4)."""
+    os.makedirs(obj_dir, exist_ok=True)
     jobs = jobs or min(len(SOURCES), os.cpu_count() or 1)
     with cf.ThreadPoolExecutor(jobs) as ex:
-        objs = list(ex.map(lambda s: _compile(s, force), SOURCES))
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < _newest(objs):
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcudart"]
+        objs = list(ex.map(lambda s: _compile(s, force, obj_dir, defines), SOURCES))
+    if force or not os.path.exists(out) or os.path.getmtime(out) < _newest(objs):
+        cmd = [nvcc(), *ARCH, "-shared", "-o", out, *objs, "-lcudart"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
     if verbose:
-        print(LIB)
-    return LIB
+        print(out)
+    return out
 
 
 if __name__ == "__main__":

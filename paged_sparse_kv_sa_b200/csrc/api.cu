@@ -83,11 +83,20 @@ const char* sa_status_string(int status) {
 
 int sa_abi_version(void) { return 100; }
 
-int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
-                    const int32_t* page_table, const int32_t* seq_lens, int B, int T, int Hq,
-                    int Hkv, int Dk, int page_size, int max_pages, int P_pool, int sink_tokens,
-                    int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
-                    int32_t* dev_error, void* stream) {
+size_t sa_select_workspace_size(int B, int Hkv, int max_pages) {
+  if (B <= 0 || Hkv <= 0 || max_pages <= 0) return 0;
+  return select_workspace_bytes(B, Hkv, max_pages);
+}
+
+}  // extern "C"
+
+namespace {
+// Argument checks and argument block shared by the selection entry points.
+int select_args(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                const int32_t* page_table, const int32_t* seq_lens, int B, int T, int Hq, int Hkv,
+                int Dk, int page_size, int max_pages, int P_pool, int sink_tokens,
+                int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
+                int32_t* dev_error, SelectArgs* a) {
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Dk <= 0 || page_size <= 0 ||
       max_pages < 0 || P_pool < 0 || sink_tokens < 0 || local_tokens < 0 || budget_tokens < 0)
     return SA_ERR_INVALID_ARG;
@@ -103,7 +112,92 @@ int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_
   if (!aligned16(summaries)) return SA_ERR_INVALID_ARG;
   if (Dk != 64 && Dk != 128 && Dk != 256) return SA_ERR_UNSUPPORTED;
   if (T * (Hq / Hkv) > 16 || max_pages > 16384) return SA_ERR_UNSUPPORTED;
+  a->q = q;
+  a->qs0 = q_strides[0];
+  a->qs1 = q_strides[1];
+  a->qs2 = q_strides[2];
+  a->sig = summaries;
+  a->page_table = page_table;
+  a->seq_lens = seq_lens;
+  a->B = B;
+  a->T = T;
+  a->Hq = Hq;
+  a->Hkv = Hkv;
+  a->Dk = Dk;
+  a->P = page_size;
+  a->max_pages = max_pages;
+  a->P_pool = P_pool;
+  a->n_sink = n_sink;
+  a->n_local = n_local;
+  a->budget_pages = budget_pages;
+  a->k_top = k_top;
+  a->out_pages = out_pages;
+  a->out_counts = out_counts;
+  a->lohi = nullptr;
+  a->err = dev_error;
+  return SA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                    const int32_t* page_table, const int32_t* seq_lens, int B, int T, int Hq,
+                    int Hkv, int Dk, int page_size, int max_pages, int P_pool, int sink_tokens,
+                    int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
+                    void* workspace, size_t workspace_bytes, int32_t* dev_error, void* stream) {
   SelectArgs a;
+  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
+                          page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
+                          out_pages, out_counts, dev_error, &a))
+    return r;
+  if (B == 0) return SA_OK;
+  if (a.k_top > 0 && (!workspace || !aligned16(workspace) ||
+                      workspace_bytes < select_workspace_bytes(B, Hkv, max_pages)))
+    return SA_ERR_WORKSPACE;
+  a.lohi = static_cast<float2*>(workspace);
+  return cuda_status(launch_select_gqa(a, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4],
+                             const uint16_t* summaries, const int32_t* page_table,
+                             const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
+                             int page_size, int max_pages, int P_pool, int sink_tokens,
+                             int local_tokens, int budget_tokens, int32_t* out_pages,
+                             int32_t* out_counts, int32_t* dev_error, void* stream) {
+  SelectArgs a;
+  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
+                          page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
+                          out_pages, out_counts, dev_error, &a))
+    return r;
+  if (B == 0) return SA_OK;
+  if ((size_t)B * Hkv * max_pages > select_static_capacity()) return SA_ERR_UNSUPPORTED;
+  return cuda_status(launch_select_gqa_static(a, static_cast<cudaStream_t>(stream)));
+}
+
+size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_pages) {
+  if (B <= 0 || T <= 0 || Hq <= 0 || max_pages <= 0) return 0;
+  return tiered_workspace_bytes(B, T, Hq, max_pages);
+}
+
+int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
+                           const uint16_t* summaries, const int32_t* page_table,
+                           const int32_t* seq_lens, int B, int T, int Hq, int Dk, int page_size,
+                           int max_pages, int P_pool, int alpha, int beta, int32_t* lists,
+                           int32_t* list_counts, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_error, void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0 ||
+      alpha < 0 || beta < 0 || alpha + beta <= 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0 || max_pages == 0) return SA_OK;
+  if (int r = check_q(q, q_strides)) return r;
+  if (!summaries || !aligned16(summaries) || !page_table || !seq_lens || !lists || !list_counts)
+    return SA_ERR_INVALID_ARG;
+  if (Dk % 8 != 0 || Dk > 1024 || max_pages > 16384 || B > 65535) return SA_ERR_UNSUPPORTED;
+  if (!workspace || !aligned16(workspace) ||
+      workspace_bytes < tiered_workspace_bytes(B, T, Hq, max_pages))
+    return SA_ERR_WORKSPACE;
+  TieredArgs a;
   a.q = q;
   a.qs0 = q_strides[0];
   a.qs1 = q_strides[1];
@@ -114,19 +208,18 @@ int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_
   a.B = B;
   a.T = T;
   a.Hq = Hq;
-  a.Hkv = Hkv;
   a.Dk = Dk;
   a.P = page_size;
   a.max_pages = max_pages;
   a.P_pool = P_pool;
-  a.n_sink = n_sink;
-  a.n_local = n_local;
-  a.budget_pages = budget_pages;
-  a.k_top = k_top;
-  a.out_pages = out_pages;
-  a.out_counts = out_counts;
+  a.alpha = alpha;
+  a.beta = beta;
+  a.n_rg = 0;
+  a.lohi = static_cast<float2*>(workspace);
+  a.lists = lists;
+  a.counts = list_counts;
   a.err = dev_error;
-  return cuda_status(launch_select_gqa(a, static_cast<cudaStream_t>(stream)));
+  return cuda_status(launch_select_tiered(a, static_cast<cudaStream_t>(stream)));
 }
 
 int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
@@ -152,12 +245,12 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
     if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
   if (Dk != Dv || (Dk != 64 && Dk != 128 && Dk != 256)) return SA_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
-  if ((max_list + n_splits - 1) / n_splits > decode_max_split_entries()) return SA_ERR_UNSUPPORTED;
 
   // (list, kv head) pairs and the heads that read them
   PairTable pairs;
   pairs.n_pairs = 0;
   const int G = Hq / Hkv;
+  int max_rows = 0;
   for (int kvh = 0; kvh < Hkv; ++kvh) {
     for (int h = kvh * G; h < (kvh + 1) * G; ++h) {
       const int l = head_to_list[h];
@@ -171,10 +264,16 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
         pairs.kvh_of[pi] = kvh;
         pairs.n_heads[pi] = 0;
       }
-      if ((pairs.n_heads[pi] + 1) * T > kMaxRowsPerPair) return SA_ERR_UNSUPPORTED;
+      if (pairs.n_heads[pi] == kMaxHeadsPerPair) return SA_ERR_UNSUPPORTED;
       pairs.heads[pi][pairs.n_heads[pi]++] = static_cast<int16_t>(h);
+      max_rows = max_rows > pairs.n_heads[pi] * T ? max_rows : pairs.n_heads[pi] * T;
     }
   }
+  // Up to 16 query rows per pair: warp-MMA decode; more: the tcgen05 kernel.
+  const bool wide = max_rows > kMaxRowsPerPair;
+  const int cap = wide ? prefill_max_split_entries() : decode_max_split_entries();
+  if (wide && Dk > 128) return SA_ERR_UNSUPPORTED;
+  if ((max_list + n_splits - 1) / n_splits > cap) return SA_ERR_UNSUPPORTED;
   CUtensorMap kmap, vmap;
   if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides) ||
       !encode_kv_map(&vmap, v_cache, Dv, page_size, Hkv, P_pool, v_strides))
@@ -204,7 +303,9 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   a.o_part = o_partial;
   a.lse_part = lse_partial;
   a.err = dev_error;
-  return cuda_status(launch_decode_gqa(a, pairs, kmap, vmap, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return cuda_status(wide ? launch_prefill(a, pairs, kmap, vmap, st)
+                          : launch_decode_gqa(a, pairs, kmap, vmap, st));
 }
 
 int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,

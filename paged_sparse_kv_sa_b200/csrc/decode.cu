@@ -23,7 +23,14 @@
 namespace sa {
 namespace {
 
-constexpr int kNW = 4;              // warps (= splits) per CTA
+// Build-time shape of a CTA: warps (= splits) per CTA and ring stages per warp.
+#ifndef SA_DECODE_WARPS
+#define SA_DECODE_WARPS 4
+#endif
+#ifndef SA_DECODE_STAGES
+#define SA_DECODE_STAGES 2
+#endif
+constexpr int kNW = SA_DECODE_WARPS;
 constexpr int kSub = 16;            // tokens per TMA sub-page (one MMA k-step of PV)
 constexpr int kWarpEntries = 128;   // list entries one split may hold
 constexpr float kLazy = 8.f;        // log2 headroom before the running max moves
@@ -34,7 +41,7 @@ struct DecodeCfg {
   static constexpr int kBoxBytes = kSub * 128;              // 16 rows x 128 bytes
   static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one K (or V) sub-page
   static constexpr int kStageBytes = 2 * kTileBytes;        // K + V
-  static constexpr int kStages = D >= 128 ? 2 : 4;
+  static constexpr int kStages = D >= 128 ? SA_DECODE_STAGES : 2 * SA_DECODE_STAGES;
   static constexpr int kDynBytes = kNW * kStages * kStageBytes + 1024;
 };
 
@@ -326,6 +333,7 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
 }  // namespace
 
 int decode_max_split_entries() { return kWarpEntries; }
+int decode_warps_per_cta() { return kNW; }
 
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream) {

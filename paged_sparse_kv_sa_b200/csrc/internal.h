@@ -9,8 +9,9 @@
 
 namespace sa {
 
-constexpr int kMaxPairs = 128;       // (list, kv head) pairs one decode call may touch
-constexpr int kMaxRowsPerPair = 16;  // query rows (T x heads) one mma tile holds
+constexpr int kMaxPairs = 64;        // (list, kv head) pairs one decode call may touch
+constexpr int kMaxHeadsPerPair = 128;
+constexpr int kMaxRowsPerPair = 16;  // query rows (T x heads) one warp-MMA tile holds
 constexpr int kMaxSplitEntries = 1024;
 
 // Which heads of a call read which (list, kv head) pair; built on the host
@@ -20,7 +21,7 @@ struct PairTable {
   int list_of[kMaxPairs];
   int kvh_of[kMaxPairs];
   int n_heads[kMaxPairs];
-  int16_t heads[kMaxPairs][kMaxRowsPerPair];
+  int16_t heads[kMaxPairs][kMaxHeadsPerPair];
 };
 
 struct DecodeArgs {
@@ -46,6 +47,10 @@ bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, in
                    const int64_t strides[4]);
 
 int decode_max_split_entries();
+int prefill_max_split_entries();
+cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
+                           const CUtensorMap& vmap, cudaStream_t stream);
+int decode_warps_per_cta();
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream);
 
@@ -59,9 +64,29 @@ struct SelectArgs {
   int n_sink, n_local, budget_pages, k_top;
   int32_t* out_pages;
   int32_t* out_counts;
+  float2* lohi;      // workspace: [B, Hkv, max_pages] score bounds
   int32_t* err;
 };
+size_t select_workspace_bytes(int B, int Hkv, int max_pages);
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream);
+size_t select_static_capacity();
+cudaError_t launch_select_gqa_static(SelectArgs a, cudaStream_t stream);
+
+struct TieredArgs {
+  const uint16_t* q;
+  int64_t qs0, qs1, qs2;
+  const uint16_t* sig;       // [P_pool, 1, Dk]
+  const int32_t* page_table;
+  const int32_t* seq_lens;
+  int B, T, Hq, Dk, P, max_pages, P_pool, alpha, beta;
+  int n_rg;                  // query-row groups of the scoring pass (set by the launcher)
+  float2* lohi;              // workspace [B, n_rg, max_pages]
+  int32_t* lists;            // [B, 2, alpha + beta]
+  int32_t* counts;           // [B, 2]
+  int32_t* err;
+};
+size_t tiered_workspace_bytes(int B, int T, int Hq, int max_pages);
+cudaError_t launch_select_tiered(TieredArgs a, cudaStream_t stream);
 
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_splits, int64_t rows,
                            int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,

@@ -1,0 +1,422 @@
+// Sparse attention over per-head page lists for many query rows per (list,
+// kv head) pair — chunked prefill over block-union tables, long MTP — on the
+// 5th-generation tensor cores.
+//
+// One CTA computes 128 query rows (the pair's (token, head) rows, token-major)
+// against the keys of its split of the list, 64 keys per tile:
+//   warp 4      gathers K and V tiles from the paged pool with TMA (four
+//               16-key x 64-column boxes per 64-column chunk; an absent or
+//               invalid 16-key group is loaded from an out-of-range page
+//               coordinate, which TMA fills with zeros) into a 3-stage ring;
+//   warp 5      issues tcgen05.mma: S = Q K^T (M=128, N=64, K=D) into one of
+//               two TMEM S buffers, and O += P V (M=128, N=D, K=64) into TMEM,
+//               with tcgen05.commit arrivals on mbarriers;
+//   warps 0-3   own one query row per thread: load Q into shared memory,
+//               read S rows from TMEM, mask (page validity, sequence end,
+//               causal position), run a base-2 online softmax whose running
+//               max only moves when a row's max exceeds it by more than 2^8
+//               (the O rescale through TMEM is then rare), write P (bf16) to
+//               shared memory for the PV MMA, and finally normalise O.
+// The QK^T of tile j+1 overlaps the softmax of tile j (two S buffers).
+//
+// Sources: CompactAttention (abstract on the page titled "Causal Attention on
+// CPU: A Cache-Aware and Load-Balanced Scheduling Kernel for Prefill"):
+// per-group KV block tables used in place; "Universal Attention Engine —
+// Declarative Sparse Attention for Production", "Key Design Decisions" 3:
+// prefill is compute-bound, so the FLOPs go to the tensor cores.
+#include "common.cuh"
+#include "internal.h"
+#include "tc05.cuh"
+
+namespace sa {
+namespace {
+
+constexpr int kPThreads = 192;
+constexpr int kPStages = 3;
+constexpr int kKeys = 64;         // keys per tile
+constexpr int kM = 128;           // query rows per CTA
+constexpr int kMaxEnt = 1024;     // list entries per split
+constexpr float kLazyP = 8.f;
+
+template <int D>
+struct PCfg {
+  static constexpr int kChunks = D / 64;               // 64-column (128-byte) chunks
+  static constexpr int kQBytes = kM * D * 2;
+  static constexpr int kTileBytes = kKeys * D * 2;     // one K (or V) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kPBytes = kM * kKeys * 2;
+  static constexpr int kDyn = kQBytes + 2 * kPBytes + kPStages * kStageBytes + 1024;
+  static constexpr uint32_t kTmemCols = 256;           // S0 [0,64) S1 [64,128) O [128,128+D)
+  static constexpr uint32_t kIdQK = tc::idesc_bf16_f32(kM, kKeys, false, false);
+  static constexpr uint32_t kIdPV = tc::idesc_bf16_f32(kM, D, false, true);
+};
+
+struct __align__(64) PrefillParams {
+  DecodeArgs a;
+  PairTable pairs;
+};
+
+SA_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that also gives up as soon as another role has aborted.
+SA_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 1023u) == 1023u && *abort_flag) return false;
+  }
+  *abort_flag = 1;
+  return false;
+}
+
+// (physical page or -1, first token) of 16-key group g of tile j.
+SA_DEV int2 group_of(const int2* ent, int n_ent, int P, int j, int g) {
+  int e, row0;
+  if (P <= kKeys) {
+    const int per = kKeys / P;                 // entries per tile
+    e = j * per + (g * 16) / P;
+    row0 = (g * 16) % P;
+  } else {
+    const int per = P / kKeys;                 // tiles per entry
+    e = j / per;
+    row0 = (j % per) * kKeys + g * 16;
+  }
+  if (e >= n_ent) return make_int2(-1, 0);
+  const int2 en = ent[e];
+  return make_int2(en.x, en.y + row0);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPThreads, 1)
+    prefill_kernel(const __grid_constant__ PrefillParams prm,
+                   const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap) {
+  using C = PCfg<D>;
+  const DecodeArgs& a = prm.a;
+  const int pair = blockIdx.y, b = blockIdx.z;
+  const int qt = blockIdx.x / a.n_splits, split = blockIdx.x % a.n_splits;
+  const int nh = prm.pairs.n_heads[pair];
+  const int rows_total = a.T * nh;
+  if (qt * kM >= rows_total) return;                 // whole CTA: nothing to do
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int list = prm.pairs.list_of[pair], kvh = prm.pairs.kvh_of[pair];
+
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
+  uint8_t* q_s = smem;
+  uint8_t* p_s = smem + C::kQBytes;                          // 2 buffers
+  uint8_t* kv_s = p_s + 2 * C::kPBytes;                      // kPStages x (K | V)
+  __shared__ uint64_t kv_full[kPStages], kv_empty[kPStages];
+  __shared__ uint64_t s_full[2], p_full[2], o_done, q_full;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_s, n_act_s;
+  __shared__ int2 ent_s[kMaxEnt];
+  __shared__ int act_s[kMaxEnt];
+
+  int L = a.seq_lens[b];
+  if (L < 0 || L > a.max_pages * a.P) {
+    if (tid == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
+    L = L < 0 ? 0 : a.max_pages * a.P;
+  }
+  const int n_log = (L + a.P - 1) / a.P;
+  int count = a.counts[b * a.n_lists + list];
+  if (count < 0 || count > a.max_list) {
+    if (tid == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
+    count = count < 0 ? 0 : a.max_list;
+  }
+  const int chunk = (count + a.n_splits - 1) / a.n_splits;
+  const int e0 = min(split * chunk, count);
+  const int n_ent = min(chunk, count - e0);
+  const int r0 = qt * kM;
+  const int t_last = (min(rows_total, r0 + kM) - 1) / nh;
+  const int max_q = L - a.T + t_last;
+
+  // ---- resolve pages, set up barriers and TMEM
+  const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
+  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+  for (int i = tid; i < n_ent; i += kPThreads) {
+    const int p = lrow[i];
+    int ph = -1;
+    if (p < 0 || p >= n_log) {
+      set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
+    } else {
+      ph = ptrow[p];
+      if (ph < 0 || ph >= a.P_pool) {
+        set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
+        ph = -1;
+      }
+    }
+    ent_s[i] = make_int2(ph, p * a.P);
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kPStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], 128);
+    }
+    mbar_init(&o_done, 1);
+    mbar_init(&q_full, 128);
+    abort_s = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) tc::tmem_alloc(&tmem_base_s, C::kTmemCols);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base_s;
+
+  // ---- tiles with at least one causally visible key, in list order
+  const int n_tiles = a.P <= kKeys ? (n_ent * a.P + kKeys - 1) / kKeys : n_ent * (a.P / kKeys);
+  if (warp == 0) {
+    int n_act = 0;
+    for (int j0 = 0; j0 < n_tiles; j0 += 32) {
+      const int j = j0 + lane;
+      bool live = false;
+      if (j < n_tiles)
+        for (int g = 0; g < 4; ++g) {
+          const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
+          live |= gr.x >= 0 && gr.y < L && gr.y <= max_q;
+        }
+      const uint32_t m = __ballot_sync(0xffffffffu, live);
+      if (live) act_s[n_act + __popc(m & ((1u << lane) - 1u))] = j;
+      n_act += __popc(m);
+    }
+    if (lane == 0) n_act_s = n_act;
+  }
+  __syncthreads();
+  const int n_act = n_act_s;
+  volatile int* abort_flag = &abort_s;
+
+  if (warp == 4) {
+    // ================= producer: TMA gathers of K and V tiles
+    if (lane == 0) {
+      prefetch_tmap(&kmap);
+      prefetch_tmap(&vmap);
+      for (int jj = 0; jj < n_act; ++jj) {
+        const int st = jj % kPStages;
+        if (jj >= kPStages &&
+            !wait_or_abort(&kv_empty[st], ((jj / kPStages) - 1) & 1, abort_flag))
+          break;
+        const int j = act_s[jj];
+        uint8_t* kt = kv_s + st * C::kStageBytes;
+        uint8_t* vt = kt + C::kTileBytes;
+        mbar_arrive_expect_tx(&kv_full[st], C::kStageBytes);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
+          const bool ok = gr.x >= 0 && gr.y < L;
+          // an out-of-range page coordinate makes TMA write zeros for the box
+          const int page = ok ? gr.x : a.P_pool;
+          const int row0 = ok ? gr.y % a.P : 0;
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c) {
+            tma_load_4d(kt + c * (kKeys * 128) + g * 2048, &kmap, &kv_full[st], c * 64, row0, kvh,
+                        page);
+            tma_load_4d(vt + c * (kKeys * 128) + g * 2048, &vmap, &kv_full[st], c * 64, row0, kvh,
+                        page);
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ================= MMA issuer (one thread)
+    if (lane == 0 && n_act > 0) {
+      const uint32_t q_addr = smem_u32(q_s), p_addr = smem_u32(p_s), kv_addr = smem_u32(kv_s);
+      auto pv = [&](int jp) -> bool {
+        const int sb = jp & 1, st = jp % kPStages;
+        if (!wait_or_abort(&p_full[sb], (jp >> 1) & 1, abort_flag)) return false;
+        tc::fence_after_sync();
+        const uint32_t vbase = kv_addr + st * C::kStageBytes + C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint64_t ad = tc::sdesc_sw128(p_addr + sb * C::kPBytes + kk * 32, 16, 1024);
+          const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
+          tc::mma_bf16(tmem + 128, ad, bd, C::kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc::commit(&o_done);
+        tc::commit(&kv_empty[st]);
+        return true;
+      };
+      bool ok = wait_or_abort(&q_full, 0, abort_flag);
+      tc::fence_after_sync();
+      for (int jj = 0; ok && jj < n_act; ++jj) {
+        const int st = jj % kPStages, sb = jj & 1;
+        if (!wait_or_abort(&kv_full[st], (jj / kPStages) & 1, abort_flag)) break;
+        tc::fence_after_sync();
+        const uint32_t kbase = kv_addr + st * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad =
+              tc::sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              tc::sdesc_sw128(kbase + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + sb * kKeys, ad, bd, C::kIdQK, kk > 0 ? 1u : 0u);
+        }
+        tc::commit(&s_full[sb]);
+        if (jj >= 1 && !pv(jj - 1)) ok = false;
+      }
+      if (ok) pv(n_act - 1);
+    }
+  } else {
+    // ================= softmax / epilogue: one query row per thread
+    const int r = warp * 32 + lane;
+    const int rg = r0 + r;
+    const bool row_ok = rg < rows_total;
+    const int t = row_ok ? rg / nh : 0;
+    const int head = prm.pairs.heads[pair][row_ok ? rg % nh : 0];
+    const int qpos = row_ok ? L - a.T + t : -1;
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + head * a.qs2);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c)
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const uint4 v = row_ok ? src[c * 8 + ch] : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(q_s + c * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+        }
+    }
+    tc::fence_proxy_async();
+    mbar_arrive(&q_full);
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int jj = 0; jj < n_act; ++jj) {
+      const int sb = jj & 1, j = act_s[jj];
+      if (!wait_or_abort(&s_full[sb], (jj >> 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      float x[64];
+      tc::ld32(tmem + lane_base + sb * kKeys, *reinterpret_cast<float(*)[32]>(&x[0]));
+      tc::ld32(tmem + lane_base + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+      tc::wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
+        const bool gok = gr.x >= 0;
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int kp = gr.y + c;
+          const bool vis = gok && kp < L && kp <= qpos;
+          const float v = vis ? x[g * 16 + c] * a.scale_log2 : -INFINITY;
+          x[g * 16 + c] = v;
+          mx = fmaxf(mx, v);
+        }
+      }
+      // PV(jj-1) must be done before O is rescaled or P buffer sb is rewritten
+      if (jj >= 1 && !wait_or_abort(&o_done, (jj - 1) & 1, abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc::fence_after_sync();
+      const bool move = mx > m_ref + kLazyP;
+      if (__any_sync(0xffffffffu, move)) {
+        const float alpha = move ? exp2f(m_ref - mx) : 1.f;
+        if (move) m_ref = mx;
+        l *= alpha;
+        if (jj >= 1) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tc::ld32(tmem + lane_base + 128 + c * 32, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tc::st32(tmem + lane_base + 128 + c * 32, o);
+          }
+          tc::wait_st();
+        }
+      }
+      const float base = m_ref == -INFINITY ? 0.f : m_ref;
+      uint8_t* prow = p_s + sb * C::kPBytes + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          p[i] = exp2f(x[ch * 8 + i] - base);
+          l += p[i];
+        }
+        uint4 w;
+        w.x = pack_bf16(p[0], p[1]);
+        w.y = pack_bf16(p[2], p[3]);
+        w.z = pack_bf16(p[4], p[5]);
+        w.w = pack_bf16(p[6], p[7]);
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = w;
+      }
+      tc::fence_proxy_async();
+      tc::fence_before_sync();
+      mbar_arrive(&p_full[sb]);
+    }
+    if (ok && n_act > 0) ok = wait_or_abort(&o_done, (n_act - 1) & 1, abort_flag);
+    tc::fence_after_sync();
+    // ---- epilogue: O / l and LSE for this row
+    const bool empty = !ok || n_act == 0 || l == 0.f;
+    const float inv = empty ? 0.f : 1.f / l;
+    float* dst = a.o_part + ((((int64_t)split * a.B + b) * a.T + t) * a.Hq + head) * D;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      float o[32];
+      if (n_act > 0) {
+        tc::ld32(tmem + lane_base + 128 + c * 32, o);
+        tc::wait_ld();
+      }
+      if (row_ok) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(dst + c * 32 + i) =
+              empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                    : make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+      }
+    }
+    if (row_ok)
+      a.lse_part[(((int64_t)split * a.B + b) * a.T + t) * a.Hq + head] =
+          empty ? -INFINITY : (m_ref + log2f(l)) * kLn2;
+    if (!ok && lane == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 5) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_p(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
+                     const CUtensorMap& vmap, cudaStream_t stream) {
+  using C = PCfg<D>;
+  PrefillParams prm;
+  prm.a = a;
+  prm.pairs = pairs;
+  int max_rows = 0;
+  for (int i = 0; i < pairs.n_pairs; ++i) max_rows = max(max_rows, a.T * pairs.n_heads[i]);
+  const int qtiles = (max_rows + kM - 1) / kM;
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDyn);
+  if (e != cudaSuccess) return e;
+  dim3 grid(qtiles * a.n_splits, pairs.n_pairs, a.B);
+  prefill_kernel<D><<<grid, kPThreads, C::kDyn, stream>>>(prm, kmap, vmap);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+int prefill_max_split_entries() { return kMaxEnt; }
+
+cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
+                           const CUtensorMap& vmap, cudaStream_t stream) {
+  switch (a.Dk) {
+    case 64: return launch_p<64>(a, pairs, kmap, vmap, stream);
+    case 128: return launch_p<128>(a, pairs, kmap, vmap, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sa

@@ -1,4 +1,7 @@
-// Page scoring and top-k selection (GQA): one CTA per (kv head, sequence).
+// Page scoring and top-k selection (GQA), in two launches.
+//
+// score_kernel (one CTA per 256 pages of one (kv head, sequence), so every SM
+// streams summaries) and choose_kernel (one CTA per (kv head, sequence)):
 //
 // 1. Every candidate page (neither sink nor local) is scored in float32 with a
 //    fixed-order FMA chain per query row, and given a rigorous error bound
@@ -16,39 +19,20 @@
 // Source: "Universal Attention Engine — Declarative Sparse Attention for
 // Production", "Content-Dependent Dynamic Routing" (top_k_blocks over
 // q @ mean(k_blocks), at block granularity) and "The Product" (sink + local).
+#include <mutex>
+
 #include "common.cuh"
 #include "exact.cuh"
 #include "internal.h"
+#include "topk.cuh"
 
 namespace sa {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 512;       // choose_kernel
+constexpr int kScoreThreads = 256;  // score_kernel: one page per thread
 constexpr int kMaxRows = 16;
 constexpr int kMaxDk = 256;
-
-SA_DEV uint32_t f2key(float x) {
-  const uint32_t b = __float_as_uint(x);
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-SA_DEV float key2f(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-// RN64(q . sigma) for a query row held as float32 copies of bf16 values.
-__device__ double exact_dot_f32q(const float* q, const uint16_t* sig, int n) {
-  ExactAcc acc;
-  acc.clear();
-  for (int d = 0; d < n; ++d) {
-    uint32_t ma, mb;
-    int ea, eb;
-    bool na, nb;
-    bf16_fields(__float_as_uint(q[d]) >> 16, ma, ea, na);
-    bf16_fields(sig[d], mb, eb, nb);
-    acc.add(ma * mb, ea + eb, na != nb);
-  }
-  return acc.round_to_double();
-}
 
 // Shared-memory layout (dynamic): lo[Nmax] f32, hi[Nmax] f32, u_list[Nmax] u16,
 // flag[Nmax] u8; q rows [R][Dk] f32 in static memory.
@@ -59,77 +43,125 @@ struct SelSmem {
   uint16_t* u_list;
 };
 
-// Radix-select the (k_lo)-th largest key of `lo` and the (k_hi)-th largest of
-// `hi` over n entries (1-based ranks; entries with key 0 never match).
-SA_DEV void radix_select2(const float* lo, const float* hi, int n, int k_lo, int k_hi,
-                          uint32_t* hist /*[2][256]*/, uint32_t* shared_out /*[4]*/,
-                          float& out_lo, float& out_hi) {
-  uint32_t pre[2] = {0u, 0u}, msk[2] = {0u, 0u};
-  int kk[2] = {k_lo, k_hi};
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 512; i += blockDim.x) hist[i] = 0u;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const float a = lo[i], c = hi[i];
-      const uint32_t ka = f2key(a), kc = f2key(c);
-      if (!isnan(a) && (ka & msk[0]) == pre[0]) atomicAdd(&hist[(ka >> shift) & 255u], 1u);
-      if (!isnan(c) && (kc & msk[1]) == pre[1]) atomicAdd(&hist[256 + ((kc >> shift) & 255u)], 1u);
+// Sequence length clamped to what its page-table row can hold.
+SA_DEV int clamped_len(const SelectArgs& a, int b, bool report) {
+  int L = a.seq_lens[b];
+  if (L < 0 || L > a.max_pages * a.P) {
+    if (report) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
+    L = L < 0 ? 0 : a.max_pages * a.P;
+  }
+  return L;
+}
+
+// The group's query rows (t, h) as exact float32 copies in q_s[R][Dk]; returns
+// an upper bound on max_r ||q_r||_2.  Called by every thread of the block.
+SA_DEV float load_q_rows(const SelectArgs& a, int b, int kvh, float* q_s, float* red) {
+  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
+  for (int i = threadIdx.x; i < R * Dk; i += blockDim.x) {
+    const int r = i / Dk, d = i % Dk;
+    const int t = r / G, h = kvh * G + r % G;
+    q_s[i] = bf16_bits_to_float(a.q[b * a.qs0 + t * a.qs1 + h * a.qs2 + d]);
+  }
+  __syncthreads();
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  float qn = 0.f;
+  for (int r = w; r < R; r += nw) {
+    float ss = 0.f;
+    for (int d = lane; d < Dk; d += 32) ss = fmaf(q_s[r * Dk + d], q_s[r * Dk + d], ss);
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    qn = fmaxf(qn, ss);
+  }
+  if (lane == 0) red[w] = qn;
+  __syncthreads();
+  qn = 0.f;
+  for (int i = 0; i < nw; ++i) qn = fmaxf(qn, red[i]);
+  // the float32 sum of squares is within (1 + gamma_Dk) of the truth
+  return sqrtf(qn * (1.f + 2.f * Dk * 5.96046448e-8f)) * (1.f + 1.2e-7f);
+}
+
+// lo/hi bounds of every candidate page's score; NaN for forced pages.
+__global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a) {
+  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int L = clamped_len(a, b, false);
+  const int N = (L + a.P - 1) / a.P;
+  if (N <= a.budget_pages || a.k_top == 0) return;   // no ranking needed
+  const int p0 = chunk * kScoreThreads;
+  if (p0 >= N) return;
+  __shared__ __align__(16) float q_s[kMaxRows * kMaxDk];
+  __shared__ float red[kScoreThreads / 32];
+  const float qn = load_q_rows(a, b, kvh, q_s, red);
+  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
+  const float nu = Dk * 5.96046448e-8f;
+  const float gfac = nu / (1.f - nu) * 1.0001f * qn * 1.0001f;
+  const float sq_pad = 1.f + 2.f * nu;
+  const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
+
+  const int p = p0 + threadIdx.x;
+  if (p >= N) return;
+  float2* out = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages + p;
+  if (p < n_sink || p >= local0) {
+    *out = make_float2(NAN, NAN);
+    return;
+  }
+  const int ph = a.page_table[(int64_t)b * a.max_pages + p];
+  if (ph < 0 || ph >= a.P_pool) {
+    set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
+    *out = make_float2(-INFINITY, -INFINITY);   // an unreadable page never wins a slot
+    return;
+  }
+  const uint4* row = reinterpret_cast<const uint4*>(a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk);
+  float acc[kMaxRows];
+#pragma unroll
+  for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
+  float ss = 0.f;
+  // 64 features per batch: 8 x 16-byte loads, unpacked once, then every query
+  // row streams its 64 float32 coefficients from shared memory (broadcast).
+  for (int d0 = 0; d0 < Dk; d0 += 64) {
+    uint4 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = __ldcs(row + d0 / 8 + j);
+    float x[64];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        x[8 * j + 2 * e] = __uint_as_float(w4[e] << 16);
+        x[8 * j + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+      }
     }
-    __syncthreads();
-    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (w < 2) {
-      // lane holds bins [255 - 8*lane - 7, 255 - 8*lane], scanned from the top
-      uint32_t c8[8], tot = 0;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        c8[j] = hist[w * 256 + 255 - (8 * lane + j)];
-        tot += c8[j];
-      }
-      uint32_t incl = tot;
+    for (int i = 0; i < 64; ++i) ss = fmaf(x[i], x[i], ss);
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += v;
-      }
-      uint32_t before = incl - tot;   // count in higher bins than this lane's
-      const uint32_t want = static_cast<uint32_t>(kk[w]);
-      if (before < want && incl >= want) {
-        uint32_t run = before;
-        for (int j = 0; j < 8; ++j) {
-          if (run + c8[j] >= want) {
-            shared_out[2 * w] = 255u - (8u * lane + j);
-            shared_out[2 * w + 1] = run;
-            break;
-          }
-          run += c8[j];
+    for (int r = 0; r < kMaxRows; ++r) {
+      if (r < R) {
+        const float4* qr = reinterpret_cast<const float4*>(&q_s[r * Dk + d0]);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 qq = qr[i];
+          acc[r] = fmaf(qq.x, x[4 * i], acc[r]);
+          acc[r] = fmaf(qq.y, x[4 * i + 1], acc[r]);
+          acc[r] = fmaf(qq.z, x[4 * i + 2], acc[r]);
+          acc[r] = fmaf(qq.w, x[4 * i + 3], acc[r]);
         }
       }
     }
-    __syncthreads();
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      pre[s] |= shared_out[2 * s] << shift;
-      msk[s] |= 255u << shift;
-      kk[s] -= static_cast<int>(shared_out[2 * s + 1]);
-    }
-    __syncthreads();
   }
-  out_lo = key2f(pre[0]);
-  out_hi = key2f(pre[1]);
+  float s = -INFINITY;
+#pragma unroll
+  for (int r = 0; r < kMaxRows; ++r)
+    if (r < R) s = fmaxf(s, acc[r]);
+  const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(ss, sq_pad)));
+  // + 0 turns -0 into +0 (the radix keys order -0 below +0)
+  *out = make_float2(__fsub_rd(s, E) + 0.f, __fadd_ru(s, E) + 0.f);
 }
 
-__global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a) {
+// Radix selection of the bounds, exact rescoring of the undecided pages, and
+// the ascending output of forced + selected pages.
+__global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
-  const int G = a.Hq / a.Hkv;
-  const int R = a.T * G;
-  const int Dk = a.Dk;
-  int L = a.seq_lens[b];
-  if (L < 0 || L > a.max_pages * a.P) {  // a length the page table cannot hold
-    if (tid == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
-    L = L < 0 ? 0 : a.max_pages * a.P;
-  }
+  const int L = clamped_len(a, b, tid == 0);
   const int N = (L + a.P - 1) / a.P;
   int32_t* outp = a.out_pages + ((int64_t)b * a.Hkv + kvh) * a.budget_pages;
   int32_t* outc = a.out_counts + (int64_t)b * a.Hkv + kvh;
@@ -141,7 +173,7 @@ __global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a
   }
 
   extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ float q_s[kMaxRows * kMaxDk];
+  __shared__ __align__(16) float q_s[kMaxRows * kMaxDk];
   __shared__ uint32_t hist[512];
   __shared__ uint32_t sel_out[4];
   __shared__ float red_f[kThreads / 32];
@@ -155,113 +187,28 @@ __global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a
   S.u_list = reinterpret_cast<uint16_t*>(S.hi + a.max_pages);
   S.flag = reinterpret_cast<uint8_t*>(S.u_list + a.max_pages);
 
-  // ---- query rows (t, h in group) as float32 (exact), and max_r ||q_r||
-  for (int i = tid; i < R * Dk; i += blockDim.x) {
-    const int r = i / Dk, d = i % Dk;
-    const int t = r / G, h = kvh * G + r % G;
-    q_s[i] = bf16_bits_to_float(a.q[b * a.qs0 + t * a.qs1 + h * a.qs2 + d]);
-  }
+  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
+  const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
+  const int k = a.k_top;
+  const float2* lohi = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
   if (tid == 0) {
     n_unc = 0;
     n_certain = 0;
   }
-  __syncthreads();
-  float qn = 0.f;
-  {
-    const int w = tid >> 5, lane = tid & 31;
-    for (int r = w; r < R; r += blockDim.x / 32) {
-      float ss = 0.f;
-      for (int d = lane; d < Dk; d += 32) ss = fmaf(q_s[r * Dk + d], q_s[r * Dk + d], ss);
-      for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      qn = fmaxf(qn, ss);
-    }
-    if (lane == 0) red_f[w] = qn;
-    __syncthreads();
-    qn = 0.f;
-    for (int i = 0; i < (int)(blockDim.x / 32); ++i) qn = fmaxf(qn, red_f[i]);
-    // sum of squares within (1 + gamma_Dk) of the truth: inflate before sqrt
-    qn = sqrtf(qn * (1.f + 2.f * Dk * 5.96046448e-8f)) * (1.f + 1.2e-7f);
-  }
-  // gamma_n = n u / (1 - n u), u = 2^-24, padded for the products below
-  const float nu = Dk * 5.96046448e-8f;
-  const float gamma = nu / (1.f - nu) * 1.0001f;
-  const float gfac = gamma * qn * 1.0001f;
-  const float sq_pad = 1.f + 2.f * nu;
-
-  const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
-  const int k = a.k_top;
-
-  // ---- 1. score candidates
-  const uint16_t* sig_base = a.sig + (int64_t)kvh * Dk;
-  const int64_t sig_page = (int64_t)a.Hkv * Dk;
-  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
   for (int p = tid; p < N; p += blockDim.x) {
     const bool cand = p >= n_sink && p < local0;
     S.flag[p] = cand ? 0 : 1;
-    float lo = NAN, hi = NAN;
-    if (cand) {
-      const int ph = ptrow[p];
-      if (ph < 0 || ph >= a.P_pool) {
-        set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
-        lo = hi = -INFINITY;     // an unreadable page never wins a slot
-      } else {
-        const uint4* row = reinterpret_cast<const uint4*>(sig_base + ph * sig_page);
-        float acc[kMaxRows];
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-        float ss = 0.f;
-        // 64 features per batch: 8 x 16-byte loads, unpacked once, then every
-        // query row streams its 64 float32 coefficients from shared memory.
-        for (int d0 = 0; d0 < Dk; d0 += 64) {
-          uint4 v[8];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[j] = row[d0 / 8 + j];
-          float x[64];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              x[8 * j + 2 * e] = __uint_as_float(w4[e] << 16);
-              x[8 * j + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
-            }
-          }
-#pragma unroll
-          for (int i = 0; i < 64; ++i) ss = fmaf(x[i], x[i], ss);
-#pragma unroll
-          for (int r = 0; r < kMaxRows; ++r) {
-            if (r < R) {
-              const float4* qr = reinterpret_cast<const float4*>(&q_s[r * Dk + d0]);
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const float4 qq = qr[i];
-                acc[r] = fmaf(qq.x, x[4 * i], acc[r]);
-                acc[r] = fmaf(qq.y, x[4 * i + 1], acc[r]);
-                acc[r] = fmaf(qq.z, x[4 * i + 2], acc[r]);
-                acc[r] = fmaf(qq.w, x[4 * i + 3], acc[r]);
-              }
-            }
-          }
-        }
-        float s = -INFINITY;
-#pragma unroll
-        for (int r = 0; r < kMaxRows; ++r)
-          if (r < R) s = fmaxf(s, acc[r]);
-        const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(ss, sq_pad)));
-        lo = __fsub_rd(s, E) + 0.f;     // + 0 turns -0 into +0 (keys order -0 < +0)
-        hi = __fadd_ru(s, E) + 0.f;
-      }
-    }
-    S.lo[p] = lo;
-    S.hi[p] = hi;
+    const float2 v = cand && k > 0 ? lohi[p] : make_float2(NAN, NAN);
+    S.lo[p] = v.x;
+    S.hi[p] = v.y;
   }
   __syncthreads();
 
-  // ---- 2. order statistics of the bounds (k == 0: streaming, no winners)
+  // ---- order statistics of the bounds (k == 0: streaming, no winners)
   float Lk = INFINITY, H = INFINITY;
   if (k > 0) radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
 
-  // ---- classify
+  // ---- classify: certainly in (lo > H), undecided (hi >= Lk), else out
   for (int p = tid; p < N; p += blockDim.x) {
     if (S.flag[p] != 0) continue;
     if (S.lo[p] > H) {
@@ -276,29 +223,30 @@ __global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a
   const int nu_ = n_unc;
   const int slots = k - n_certain;
 
-  // ---- 3. exact scores of the uncertain pages (lo/hi reused as double storage)
+  // ---- exact scores of the undecided pages (lo/hi storage reused as doubles)
   double* ex = reinterpret_cast<double*>(S.lo);
+  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
   if (nu_ > 0 && slots > 0) {
-    const int per = max(1, kThreads / R);            // uncertain pages per batch
+    load_q_rows(a, b, kvh, q_s, red_f);
+    const int per = max(1, kThreads / R);            // undecided pages per batch
     for (int u0 = 0; u0 < nu_; u0 += per) {
-      const int i = tid;
-      const int u = u0 + i / R, r = i % R;
-      if (i < per * R && u < nu_) {
-        const int p = S.u_list[u];
-        const int ph = ptrow[p];
-        ex_tmp[i] = (ph < 0 || ph >= a.P_pool)
-                        ? -INFINITY
-                        : exact_dot_f32q(&q_s[r * Dk], sig_base + ph * sig_page, Dk);
+      const int u = u0 + tid / R, r = tid % R;
+      if (tid < per * R && u < nu_) {
+        const int ph = ptrow[S.u_list[u]];
+        ex_tmp[tid] = (ph < 0 || ph >= a.P_pool)
+                          ? -INFINITY
+                          : exact_dot_f32q(&q_s[r * Dk],
+                                           a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk, Dk);
       }
       __syncthreads();
-      if (i < per && u0 + i < nu_) {
+      if (tid < per && u0 + tid < nu_) {
         double m = -INFINITY;
-        for (int rr = 0; rr < R; ++rr) m = fmax(m, ex_tmp[i * R + rr]);
-        ex[u0 + i] = m;
+        for (int rr = 0; rr < R; ++rr) m = fmax(m, ex_tmp[tid * R + rr]);
+        ex[u0 + tid] = m;
       }
       __syncthreads();
     }
-    // rank among the uncertain pages: (exact desc, logical asc)
+    // rank among the undecided pages: (exact desc, logical asc)
     for (int u = tid; u < nu_; u += blockDim.x) {
       const double su = ex[u];
       const int pu = S.u_list[u];
@@ -314,12 +262,11 @@ __global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a
   }
   __syncthreads();
 
-  // ---- 4. ascending compaction of the selected pages
+  // ---- ascending compaction of the selected pages
   const int per_t = (N + blockDim.x - 1) / blockDim.x;
   const int p0 = tid * per_t, p1 = min(N, p0 + per_t);
   int cnt = 0;
   for (int p = p0; p < p1; ++p) cnt += S.flag[p] == 1;
-  // block exclusive scan of cnt
   const int w = tid >> 5, lane = tid & 31;
   int incl = cnt;
   for (int o = 1; o < 32; o <<= 1) {
@@ -342,14 +289,71 @@ __global__ void __launch_bounds__(kThreads) select_gqa_kernel(const SelectArgs a
 
 }  // namespace
 
+size_t select_workspace_bytes(int B, int Hkv, int max_pages) {
+  return (size_t)B * Hkv * max_pages * sizeof(float2);
+}
+
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
+  if (a.k_top > 0) {
+    dim3 g1((a.max_pages + kScoreThreads - 1) / kScoreThreads, a.Hkv, a.B);
+    score_kernel<<<g1, kScoreThreads, 0, stream>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   const size_t dyn = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
-  cudaError_t e = cudaFuncSetAttribute(select_gqa_kernel,
+  cudaError_t e = cudaFuncSetAttribute(choose_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
   if (e != cudaSuccess) return e;
-  dim3 grid(a.Hkv, a.B);
-  select_gqa_kernel<<<grid, kThreads, dyn, stream>>>(a);
+  choose_kernel<<<dim3(a.Hkv, a.B), kThreads, dyn, stream>>>(a);
   return cudaGetLastError();
+}
+
+
+// ---------------------------------------------------------------------------
+// Selection without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they select
+// pages: code running inside a CUDA-graph capture region, a serving loop
+// whose memory pool is sealed after warm-up, or a host framework that owns
+// every allocation and hands this library raw pointers only.  For them the
+// score bounds live in a fixed-size array in the library's own device memory,
+// reserved when the library is loaded (on every GPU that loads it, until the
+// process exits).
+constexpr size_t kStaticScoreEntries = size_t(1) << 21;   // 2,097,152 pages x 8 bytes = 16 MiB
+static __device__ __align__(256) float2 g_static_score_bounds[kStaticScoreEntries];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+float2* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the static array on the current device; looked up once per
+// device (the host-side symbol is only a stand-in and must not reach a kernel).
+cudaError_t static_scores_ptr(float2** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_score_bounds);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = static_cast<float2*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t select_static_capacity() { return kStaticScoreEntries; }
+
+cudaError_t launch_select_gqa_static(SelectArgs a, cudaStream_t stream) {
+  float2* p = nullptr;
+  cudaError_t e = static_scores_ptr(&p);
+  if (e != cudaSuccess) return e;
+  a.lohi = p;
+  return launch_select_gqa(a, stream);
 }
 
 }  // namespace sa

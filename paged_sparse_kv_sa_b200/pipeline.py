@@ -60,11 +60,13 @@ class SparseDecodeStep:
                        if out_bf16 else None)
         self.lse = torch.empty((B, T, Hq), dtype=torch.float32, device=dev)
         self.dev_error = torch.zeros((1,), dtype=torch.int32, device=dev)
+        self.sel_ws = torch.empty(max(_lib.sa_select_workspace_size(B, Hkv, max_pages), 16),
+                                  dtype=torch.uint8, device=dev)
 
     def select(self, q, summaries, page_table, seq_lens, stream=None):
         _lib.sa_select_pages(q, summaries, page_table, seq_lens, self.P, self.sink, self.local,
                              self.budget, out_pages=self.pages, out_counts=self.counts,
-                             dev_error=self.dev_error, stream=stream)
+                             workspace=self.sel_ws, dev_error=self.dev_error, stream=stream)
 
     def decode(self, q, k_cache, v_cache, page_table, seq_lens, stream=None):
         _lib.sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, self.pages, self.counts,

@@ -49,21 +49,25 @@ def test_host_validation_rejects_bad_arguments():
     s = _i64x4(1024, 1024, 128, 1)
     # Hq not a multiple of Hkv
     assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 6, 4, 128, 16, 8, 8, 32, 64, 256,
-                               fake, fake, None, None) == 1
+                               fake, fake, fake, 1 << 30, None, None) == 1
     # sink + local above the budget
     assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 8, 2, 128, 16, 8, 8, 512, 512,
-                               256, fake, fake, None, None) == 1
+                               256, fake, fake, fake, 1 << 30, None, None) == 1
     # null outputs
     assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 8, 2, 128, 16, 8, 8, 32, 64, 256,
-                               None, fake, None, None) == 1
+                               None, fake, fake, 1 << 30, None, None) == 1
+    # workspace too small
+    assert lib.sa_select_pages(fake, s, fake, fake, fake, 1, 1, 8, 2, 128, 16, 8, 8, 32, 64, 256,
+                               fake, fake, fake, 16, None, None) == 3
+    assert lib.sa_select_workspace_size(2, 8, 100) == 2 * 8 * 100 * 8
     # unsupported head dim
     assert lib.sa_select_pages(fake, _i64x4(96, 96, 96, 1), fake, fake, fake, 1, 1, 8, 2, 96, 16,
-                               8, 8, 32, 64, 256, fake, fake, None, None) == 2
+                               8, 8, 32, 64, 256, fake, fake, fake, 1 << 30, None, None) == 2
     # misaligned q / non-unit feature stride
     assert lib.sa_select_pages(ctypes.c_void_p(0x1002), s, fake, fake, fake, 1, 1, 8, 2, 128, 16,
-                               8, 8, 32, 64, 256, fake, fake, None, None) == 1
+                               8, 8, 32, 64, 256, fake, fake, fake, 1 << 30, None, None) == 1
     assert lib.sa_select_pages(fake, _i64x4(1024, 1024, 128, 2), fake, fake, fake, 1, 1, 8, 2, 128,
-                               16, 8, 8, 32, 64, 256, fake, fake, None, None) == 1
+                               16, 8, 8, 32, 64, 256, fake, fake, fake, 1 << 30, None, None) == 1
     h2l = (ctypes.c_int32 * 8)(0, 0, 0, 0, 1, 1, 1, 5)   # list id out of range
     ks = _i64x4(4096, 2048, 128, 1)
     args = [fake, s, fake, ks, fake, ks, fake, 8, fake, fake, fake, 2, 16,

@@ -325,3 +325,140 @@ def test_block_union_full_size_sampled():
     rt, rc = O.block_union(sn[:2 * G], 2, off, cfg.top_k)
     np.testing.assert_array_equal(c[:2], rc)
     np.testing.assert_array_equal(t[:2], rt)
+
+
+# ----------------------------------------------------------------------------
+# many query rows per pair: the tcgen05 path (chunked prefill, long MTP)
+# ----------------------------------------------------------------------------
+def prefill_case(seed, T, q_off, P, Hq=8, Hkv=2, D=128, top_k=3, n_sink=1, ragged=0):
+    """Chunk of T queries at q_off over a KV of q_off + T - ragged tokens, block-union
+    tables (64-token blocks) from random block scores, expressed as lists of P-token
+    pages (a block of 64 tokens = 64 / P pages)."""
+    g = torch.Generator().manual_seed(seed)
+    L = q_off + T - ragged
+    nkb = -(-L // 64)
+    nqb = -(-T // 64)
+    qb_off = q_off // 64
+    scores = torch.randn((Hq, nqb, nkb), generator=g)
+    tables, counts = O.block_union(scores.numpy(), Hkv, qb_off, top_k, n_sink)
+    per = 64 // P if P <= 64 else 1
+    npg = -(-L // P)
+    lists = np.full((1, Hkv, nkb * per), -1, dtype=np.int32)
+    cnt = np.zeros((1, Hkv), dtype=np.int32)
+    for h in range(Hkv):
+        pages = []
+        for blk in tables[h, :counts[h]]:
+            if P <= 64:
+                pages += [p for p in range(blk * per, blk * per + per) if p < npg]
+            else:
+                if blk * 64 // P not in pages:
+                    pages.append(blk * 64 // P)
+        lists[0, h, :len(pages)] = pages
+        cnt[0, h] = len(pages)
+    q = torch.randn((1, T, Hq, D), generator=g).to(torch.bfloat16)
+    perm = torch.randperm(npg, generator=g)
+    k = torch.randn((npg, Hkv, P, D), generator=g).to(torch.bfloat16)
+    v = torch.randn((npg, Hkv, P, D), generator=g).to(torch.bfloat16)
+    pt = perm.to(torch.int32).reshape(1, npg)
+    sl = torch.tensor([L], dtype=torch.int32)
+    return q, k, v, pt, sl, lists, cnt
+
+
+@pytest.mark.parametrize("T,q_off,P,n_splits,ragged", [(64, 640, 64, 1, 0), (96, 448, 64, 2, 0),
+                                                       (8, 700, 16, 1, 5), (40, 1000, 32, 3, 17)])
+def test_prefill_tcgen05_vs_oracle(T, q_off, P, n_splits, ragged):
+    q, k, v, pt, sl, lists, cnt = prefill_case(1, T, q_off, P, ragged=ragged)
+    Hq, Hkv, D = q.shape[2], k.shape[1], q.shape[3]
+    h2l = [h // (Hq // Hkv) for h in range(Hq)]
+    o_p, l_p = sa.sa_sparse_decode(q.to(DEV), k.to(DEV), v.to(DEV), pt.to(DEV), sl.to(DEV),
+                                   torch.from_numpy(lists).to(DEV), torch.from_numpy(cnt).to(DEV),
+                                   h2l, 1.0 / math.sqrt(D), n_splits)
+    o, _, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    ro, rl = O.sparse_attention(bits(q), bits(k), bits(v), np_i32(pt), np_i32(sl), lists, cnt,
+                                np.array(h2l), 1.0 / math.sqrt(D), P)
+    assert_attn_close(o, lse, ro, rl)
+
+
+@pytest.mark.slow
+def test_prefill_full_size_sampled_rows():
+    cfg = W.UNION_PREFILL
+    s = W.block_union_scores(cfg, seed=0, device=DEV)
+    inp = W.prefill_inputs(cfg, seed=0, device=DEV)
+    off = cfg.q_offset // cfg.block
+    tables, counts = sa.sa_block_union(s, cfg.Hkv, off, cfg.top_k)
+    h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)]
+    o_p, l_p = sa.sa_sparse_decode(inp["q"], inp["k"], inp["v"], inp["page_table"],
+                                   inp["seq_lens"], tables.view(1, cfg.Hkv, -1).contiguous(),
+                                   counts.view(1, cfg.Hkv).contiguous(), h2l,
+                                   1.0 / math.sqrt(cfg.D), 2)
+    o, _, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    ts = sorted(set(rng.integers(0, cfg.chunk, 12).tolist()) | {0, cfg.chunk - 1})
+    rows = [(0, t, int(h)) for t in ts for h in rng.integers(0, cfg.Hq, 3)]
+    tb = np_i32(tables).reshape(1, cfg.Hkv, -1)
+    cb = np_i32(counts).reshape(1, cfg.Hkv)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), tb, cb,
+                                np.array(h2l), 1.0 / math.sqrt(cfg.D), cfg.block, rows=rows)
+    og = o.cpu().double().numpy()
+    lg = lse.cpu().double().numpy()
+    for (b, t, h) in rows:
+        assert np.abs(og[b, t, h] - ro[b, t, h]).max() <= O_TOL, (t, h)
+        assert abs(lg[b, t, h] - rl[b, t, h]) <= LSE_TOL, (t, h)
+
+
+# ----------------------------------------------------------------------------
+# tiered (critical / ambient) selection for one latent head
+# ----------------------------------------------------------------------------
+def tiered_case(seed, B, T, Hq, Dk, P, L, alpha, beta):
+    cfg = W.MLADecode("case", B=B, T=T, Hq=Hq, Dk=Dk, Dv=Dk - 64, page_size=P, seq_len=L,
+                      alpha=alpha, beta=beta, h_ambient=max(1, Hq // 4))
+    inp = W.mla_decode_inputs(cfg, seed=seed, device="cpu")
+    sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), P)
+    return cfg, inp, sig
+
+
+def check_tiered(cfg, inp, sig, units=None):
+    g = {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+    lists, counts = sa.sa_select_pages_tiered(g["q"], to_bf16_dev(sig), g["page_table"],
+                                              g["seq_lens"], cfg.page_size, cfg.alpha, cfg.beta)
+    torch.cuda.synchronize()
+    lists, counts = np_i32(lists), np_i32(counts)
+    crit, cc, amb, ac = O.select_pages_mla(bits(inp["q"]), sig, np_i32(inp["page_table"]),
+                                           np_i32(inp["seq_lens"]), cfg.page_size, cfg.alpha,
+                                           cfg.beta, units=units)
+    for b in (range(cfg.B) if units is None else units):
+        want0 = list(crit[b, :cc[b]])
+        want1 = sorted(want0 + list(amb[b, :ac[b]]))
+        assert counts[b, 0] == len(want0) and counts[b, 1] == len(want1)
+        assert list(lists[b, 0, :counts[b, 0]]) == want0
+        assert list(lists[b, 1, :counts[b, 1]]) == want1
+        assert np.all(lists[b, 0, counts[b, 0]:] == -1) and np.all(lists[b, 1, counts[b, 1]:] == -1)
+
+
+@pytest.mark.parametrize("seed,L", [(0, 40 * 16 - 3), (1, 9 * 16), (2, 5 * 16)])
+def test_select_tiered_small(seed, L):
+    cfg, inp, sig = tiered_case(seed, B=2, T=2, Hq=16, Dk=576, P=16, L=L, alpha=3, beta=5)
+    check_tiered(cfg, inp, sig)
+
+
+def test_select_tiered_ties():
+    cfg, inp, sig = tiered_case(3, B=2, T=1, Hq=8, Dk=128, P=16, L=30 * 16, alpha=2, beta=4)
+    inp["q"][0] = 0                                     # all scores tie: lowest pages
+    sig = sig.copy()
+    pt = np_i32(inp["page_table"])
+    sig[pt[1, 7]] = sig[pt[1, 9]]                       # duplicated summaries
+    check_tiered(cfg, inp, sig)
+
+
+@pytest.mark.slow
+def test_select_tiered_mla_workload_sampled():
+    cfg = W.MLA_MTP
+    inp = W.mla_decode_inputs(cfg, seed=0, device="cpu")
+    n = cfg.seq_len // cfg.page_size
+    units = [(b, p) for b in (0, 5) for p in range(n)]
+    sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                           cfg.page_size, units=units)
+    check_tiered(cfg, inp, sig, units=[0, 5])
