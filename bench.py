@@ -49,6 +49,11 @@ def parse():
     ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = heuristic)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--workload", choices=["llama8b", "llama70b", "mla", "prefill"],
+                    default="llama8b",
+                    help="llama8b (default, the headline workload); the others print the same "
+                         "line for the Llama-70B long decode, MLA+MTP tiered decode and "
+                         "block-union prefill workloads")
     return ap.parse_args()
 
 
@@ -170,6 +175,220 @@ def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0):
     return kv_bytes / dt / 1e9, done, dt
 
 
+def _timed_graphs(g_step, g_kernel, K, flush_l2, stream, local):
+    """Replay a whole-step graph and a single-kernel graph K times each, L2 flushed
+    before every replay outside the events; device seconds for each, and clocks."""
+    import torch
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(K):
+            flush_l2(i)
+            ev[i][0].record(stream)
+            g_step.replay()
+            ev[i][1].record(stream)
+            flush_l2(i + 1)
+            ev[i][2].record(stream)
+            g_kernel.replay()
+            ev[i][3].record(stream)
+        torch.cuda.synchronize()
+    t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_kern = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
+    return t_step, t_kern, clk.summary()
+
+
+def _peak_tflops():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    return 1590.0, "fallback"
+
+
+def run_extra(args, dev, world, rank, local, cores):
+    """MLA+MTP tiered decode or block-union chunked prefill: same timing protocol."""
+    import numpy as np
+    import torch
+
+    import paged_sparse_kv_sa_b200 as sa
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    if args.impl == "reference":
+        print(json.dumps({"impl": "reference", "unavailable":
+                          "the oracle arm is timed on the default (Llama-8B decode) workload"}))
+        return
+    sa.load()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    flush_rd = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def flush_l2(i):
+        flush.fill_(i & 0xFF)
+        torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
+
+    K = args.steps
+    if args.workload == "mla":
+        cfg = W.MLA_MTP
+        inp = W.mla_decode_inputs(cfg, seed=args.seed + rank, device=dev)
+        q, kv, pt, sl = inp["q"], inp["kv"], inp["page_table"], inp["seq_lens"]
+        sig = sa.sa_build_page_summaries(kv, pt, sl)
+        amb = set(int(h) for h in inp["ambient_heads"].tolist())
+        h2l = [1 if h in amb else 0 for h in range(cfg.Hq)]
+        cap = cfg.alpha + cfg.beta
+        lists = torch.empty((cfg.B, 2, cap), dtype=torch.int32, device=dev)
+        counts = torch.empty((cfg.B, 2), dtype=torch.int32, device=dev)
+        ws = torch.empty(max(int(sa.load().sa_select_tiered_workspace_size(
+            cfg.B, cfg.T, cfg.Hq, pt.shape[1])), 16), dtype=torch.uint8, device=dev)
+        n_splits = args.splits or 4
+        o_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
+        l_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
+        o = torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
+        lse = torch.empty((cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(cfg.Dk)
+
+        def select(qq, ptt, sll):
+            sa.sa_select_pages_tiered(qq, sig, ptt, sll, cfg.page_size, cfg.alpha, cfg.beta,
+                                      lists=lists, list_counts=counts, workspace=ws)
+
+        def decode(qq, ptt, sll):
+            sa.sa_sparse_decode(qq, kv, kv[..., :cfg.Dv], ptt, sll, lists, counts, h2l, scale,
+                                n_splits, o_partial=o_p, lse_partial=l_p)
+
+        step_inputs = (q, pt, sl)
+        kern = "mla_kernel"
+    else:
+        cfg = W.UNION_PREFILL
+        inp = W.prefill_inputs(cfg, seed=args.seed + rank, device=dev)
+        q, kk, vv, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
+        scores = W.block_union_scores(cfg, seed=args.seed + rank, device=dev)
+        off = cfg.q_offset // cfg.block
+        tables = torch.empty((cfg.Hkv, cfg.n_kv_blocks), dtype=torch.int32, device=dev)
+        tcounts = torch.empty((cfg.Hkv,), dtype=torch.int32, device=dev)
+        h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)]
+        n_splits = args.splits or 2
+        o_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
+        l_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
+        o = torch.empty((1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
+        lse = torch.empty((1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
+        scale = 1.0 / math.sqrt(cfg.D)
+
+        def select(sc, ptt, sll):
+            sa.sa_block_union(sc, cfg.Hkv, off, cfg.top_k, cfg.n_sink_blocks, tables=tables,
+                              counts=tcounts)
+
+        def decode(qq, ptt, sll):
+            sa.sa_sparse_decode(qq, kk, vv, ptt, sll, tables.view(1, cfg.Hkv, -1),
+                                tcounts.view(1, cfg.Hkv), h2l, scale, n_splits,
+                                o_partial=o_p, lse_partial=l_p)
+
+        step_inputs = (scores, pt, sl)
+        kern = "prefill_kernel"
+
+    def run_step(a0, ptt, sll, qq):
+        select(a0, ptt, sll)
+        decode(qq, ptt, sll)
+        sa.sa_combine(o_p, l_p, o_out=o, lse_out=lse)
+
+    first = step_inputs[0]
+    for _ in range(max(args.warmup, 3)):
+        run_step(first, pt, sl, q)
+    torch.cuda.synchronize()
+
+    # algorithmic work of one step (from the lists the step produced)
+    if args.workload == "mla":
+        L = sl.cpu().numpy()
+        ls, cs = lists.cpu().numpy(), counts.cpu().numpy()
+        flops, kv_bytes = 0, 0
+        for b in range(cfg.B):
+            for t in range(cfg.T):
+                qpos = int(L[b]) - cfg.T + t
+                for li, nh in ((0, cfg.Hq - len(amb)), (1, len(amb))):
+                    pg = ls[b, li, :cs[b, li]].astype(np.int64)
+                    keys = np.clip(np.minimum(qpos + 1, int(L[b])) - pg * cfg.page_size, 0,
+                                   cfg.page_size).sum()
+                    flops += 2 * nh * int(keys) * (cfg.Dk + cfg.Dv)
+            pg = ls[b, 1, :cs[b, 1]].astype(np.int64)
+            kv_bytes += int(np.clip(int(L[b]) - pg * cfg.page_size, 0, cfg.page_size).sum()) \
+                * cfg.Dk * 2
+    else:
+        tb, tc_ = tables.cpu().numpy(), tcounts.cpu().numpy()
+        G = cfg.Hq // cfg.Hkv
+        qpos = cfg.q_offset + np.arange(cfg.chunk)
+        flops, kv_bytes = 0, 0
+        for g in range(cfg.Hkv):
+            blk = tb[g, :tc_[g]].astype(np.int64)
+            vis = np.clip(np.minimum(qpos[:, None] + 1, cfg.kv_len) - blk[None, :] * cfg.block, 0,
+                          cfg.block).sum()
+            flops += 2 * G * int(vis) * (2 * cfg.D)
+            kv_bytes += int(np.clip(cfg.kv_len - blk * cfg.block, 0, cfg.block).sum()) \
+                * cfg.D * 2 * 2
+
+    g_step, g_kern = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step):
+        run_step(first, pt, sl, q)
+    with torch.cuda.graph(g_kern):
+        decode(q, pt, sl)
+    for _ in range(3):
+        g_step.replay()
+        g_kern.replay()
+    t_step, t_kern, clocks = _timed_graphs(g_step, g_kern, K, flush_l2, stream, local)
+
+    # end to end through the same API: the step's inputs from pinned host memory
+    srcs = (first, pt, sl) if first is q else (first, pt, sl, q)
+    hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in srcs]
+    devs = [torch.empty_like(x) for x in srcs]
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+    def e2e():
+        for d_, h_ in zip(devs, hosts):
+            d_.copy_(h_, non_blocking=True)
+        run_step(devs[0], devs[1], devs[2], devs[-1] if len(devs) == 4 else devs[0])
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e()
+    torch.cuda.synchronize()
+    e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    for i in range(K):
+        flush_l2(i)
+        e_ev[i][0].record(stream)
+        e2e()
+        e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_e2e = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
+    h2d = sum(h.numel() * h.element_size() for h in hosts)
+    d2h = o_h.numel() * 4 + lse_h.numel() * 4
+    assert torch.isfinite(o).all().item(), "non-finite output"
+
+    peak, kind = _peak_tflops()
+    achieved = flops / (t_kern / K) / 1e12
+    line = {
+        "metric": METRIC, "value": round(kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_step / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "n_splits": n_splits,
+                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
+        "calls_per_sec": round(K / t_step, 2),
+        "step_tflops": round(flops * K / t_step / 1e12, 2),
+        "selected_kv_bytes_per_step": kv_bytes, "flops_per_step": flops,
+        "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_kind": kind, "traffic": None,
+                     "kernel_ms": round(1e3 * t_kern / K, 4)},
+        "e2e": {"value": round(kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(1e3 * t_e2e / K, 4)},
+        "gpu_launches": (5 if args.workload == "prefill" else 4) * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line))
+
+
 def main():
     args = parse()
     import numpy as np
@@ -190,8 +409,10 @@ def main():
 
     from paged_sparse_kv_sa_b200 import workloads as W
 
-    cfg = W.LLAMA8B_DECODE
     cores = len(os.sched_getaffinity(0))
+    if args.workload in ("mla", "prefill"):
+        return run_extra(args, dev, world, rank, local, cores)
+    cfg = {"llama8b": W.LLAMA8B_DECODE, "llama70b": W.LLAMA70B_LONG}[args.workload]
 
     if args.impl == "reference":
         # the reference arm is the float64 oracle on the host cores

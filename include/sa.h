@@ -176,8 +176,15 @@ SA_API size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_page
  *  head_to_list (host) [Hq] int32 in [0, n_lists)
  *  o_partial    (dev) [n_splits,B,T,Hq,Dv] float32
  *  lse_partial  (dev) [n_splits,B,T,Hq] float32
- * Supported: Dk == Dv in {64,128,256}, P in {16,32,64,128}, and at most 16
- * query rows (T x heads) sharing one (list, kv head) pair.
+ * Kernels, chosen from the shapes (P in {16,32,64,128} throughout):
+ *  - at most 16 query rows (T x heads) per (list, kv head) pair, Dk == Dv in
+ *    {64,128,256}: one warp per split, warp-level tensor-core MMAs;
+ *  - more rows per pair (chunked prefill, long MTP), Dk == Dv in {64,128}:
+ *    128-row tiles on tcgen05 with TMEM accumulators;
+ *  - MLA, Dk == 576 with Dv == 512 and v_cache == k_cache (same strides: the
+ *    values are the first 512 key columns): 64-row tiles on tcgen05.
+ * Pool rows past a sequence's end are read with the page but masked; they
+ * must hold finite values (a NaN there could reach the output through 0*NaN).
  */
 SA_API int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
                      const int64_t k_strides[4], const uint16_t* v_cache,

@@ -159,22 +159,6 @@ int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_
   return cuda_status(launch_select_gqa(a, static_cast<cudaStream_t>(stream)));
 }
 
-int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4],
-                             const uint16_t* summaries, const int32_t* page_table,
-                             const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
-                             int page_size, int max_pages, int P_pool, int sink_tokens,
-                             int local_tokens, int budget_tokens, int32_t* out_pages,
-                             int32_t* out_counts, int32_t* dev_error, void* stream) {
-  SelectArgs a;
-  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
-                          page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
-                          out_pages, out_counts, dev_error, &a))
-    return r;
-  if (B == 0) return SA_OK;
-  if ((size_t)B * Hkv * max_pages > select_static_capacity()) return SA_ERR_UNSUPPORTED;
-  return cuda_status(launch_select_gqa_static(a, static_cast<cudaStream_t>(stream)));
-}
-
 size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_pages) {
   if (B <= 0 || T <= 0 || Hq <= 0 || max_pages <= 0) return 0;
   return tiered_workspace_bytes(B, T, Hq, max_pages);
@@ -243,7 +227,10 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   if (!aligned16(o_partial)) return SA_ERR_INVALID_ARG;
   for (int h = 0; h < Hq; ++h)
     if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
-  if (Dk != Dv || (Dk != 64 && Dk != 128 && Dk != 256)) return SA_ERR_UNSUPPORTED;
+  // MLA: keys of 576 columns whose first 512 are the values (V aliases K)
+  const bool mla = Dk == 576 && Dv == 512 && k_cache == v_cache &&
+                   std::memcmp(k_strides, v_strides, 4 * sizeof(int64_t)) == 0;
+  if (!mla && (Dk != Dv || (Dk != 64 && Dk != 128 && Dk != 256))) return SA_ERR_UNSUPPORTED;
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
 
   // (list, kv head) pairs and the heads that read them
@@ -271,8 +258,9 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   }
   // Up to 16 query rows per pair: warp-MMA decode; more: the tcgen05 kernel.
   const bool wide = max_rows > kMaxRowsPerPair;
-  const int cap = wide ? prefill_max_split_entries() : decode_max_split_entries();
-  if (wide && Dk > 128) return SA_ERR_UNSUPPORTED;
+  const int cap = mla ? mla_max_split_entries(page_size)
+                      : (wide ? prefill_max_split_entries() : decode_max_split_entries());
+  if (!mla && wide && Dk > 128) return SA_ERR_UNSUPPORTED;
   if ((max_list + n_splits - 1) / n_splits > cap) return SA_ERR_UNSUPPORTED;
   CUtensorMap kmap, vmap;
   if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides) ||
@@ -304,6 +292,7 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   a.lse_part = lse_partial;
   a.err = dev_error;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (mla) return cuda_status(launch_mla(a, pairs, kmap, st));
   return cuda_status(wide ? launch_prefill(a, pairs, kmap, vmap, st)
                           : launch_decode_gqa(a, pairs, kmap, vmap, st));
 }

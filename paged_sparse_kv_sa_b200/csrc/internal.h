@@ -48,6 +48,9 @@ bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, in
 
 int decode_max_split_entries();
 int prefill_max_split_entries();
+int mla_max_split_entries(int P);
+cudaError_t launch_mla(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
+                       cudaStream_t stream);
 cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, cudaStream_t stream);
 int decode_warps_per_cta();
@@ -69,8 +72,6 @@ struct SelectArgs {
 };
 size_t select_workspace_bytes(int B, int Hkv, int max_pages);
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream);
-size_t select_static_capacity();
-cudaError_t launch_select_gqa_static(SelectArgs a, cudaStream_t stream);
 
 struct TieredArgs {
   const uint16_t* q;

@@ -462,3 +462,74 @@ def test_select_tiered_mla_workload_sampled():
     sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
                            cfg.page_size, units=units)
     check_tiered(cfg, inp, sig, units=[0, 5])
+
+
+# ----------------------------------------------------------------------------
+# MLA + MTP tiered decode (tcgen05, V = first 512 key columns)
+# ----------------------------------------------------------------------------
+def mla_lists_from_oracle(inp, sig, cfg, units=None):
+    crit, cc, amb, ac = O.select_pages_mla(bits(inp["q"]), sig, np_i32(inp["page_table"]),
+                                           np_i32(inp["seq_lens"]), cfg.page_size, cfg.alpha,
+                                           cfg.beta, units=units)
+    cap = cfg.alpha + cfg.beta
+    lists = np.full((cfg.B, 2, cap), -1, dtype=np.int32)
+    counts = np.zeros((cfg.B, 2), dtype=np.int32)
+    for b in range(cfg.B):
+        c0 = list(crit[b, :cc[b]])
+        c1 = sorted(c0 + list(amb[b, :ac[b]]))
+        lists[b, 0, :len(c0)] = c0
+        lists[b, 1, :len(c1)] = c1
+        counts[b] = (len(c0), len(c1))
+    return lists, counts
+
+
+def run_mla(inp, cfg, lists, counts, n_splits):
+    g = {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+    amb = set(int(h) for h in inp["ambient_heads"].tolist())
+    h2l = [1 if h in amb else 0 for h in range(cfg.Hq)]
+    kv = g["kv"]
+    o_p, l_p = sa.sa_sparse_decode(g["q"], kv, kv[..., :cfg.Dv], g["page_table"], g["seq_lens"],
+                                   torch.from_numpy(lists).to(DEV),
+                                   torch.from_numpy(counts).to(DEV), h2l,
+                                   1.0 / math.sqrt(cfg.Dk), n_splits)
+    o, _, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    return o, lse, h2l
+
+
+@pytest.mark.parametrize("seed,L,n_splits", [(0, 2500, 1), (1, 2500, 3), (2, 700, 2)])
+def test_mla_decode_vs_oracle(seed, L, n_splits):
+    cfg = W.MLADecode("case", B=2, T=2, Hq=16, Dk=576, Dv=512, page_size=64, seq_len=L,
+                      alpha=3, beta=6, h_ambient=4)
+    inp = W.mla_decode_inputs(cfg, seed=seed, device="cpu")
+    sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), 64)
+    lists, counts = mla_lists_from_oracle(inp, sig, cfg)
+    o, lse, h2l = run_mla(inp, cfg, lists, counts, n_splits)
+    kvb = bits(inp["kv"])
+    ro, rl = O.sparse_attention(bits(inp["q"]), kvb, kvb[..., :cfg.Dv], np_i32(inp["page_table"]),
+                                np_i32(inp["seq_lens"]), lists, counts, np.array(h2l),
+                                1.0 / math.sqrt(cfg.Dk), 64)
+    assert_attn_close(o, lse, ro, rl)
+
+
+@pytest.mark.slow
+def test_mla_decode_full_size_sampled():
+    cfg = W.MLA_MTP
+    inp = W.mla_decode_inputs(cfg, seed=0, device="cpu")
+    n = cfg.seq_len // cfg.page_size
+    units = [(b, p) for b in (0, 3) for p in range(n)]
+    sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                           cfg.page_size, units=units)
+    lists, counts = mla_lists_from_oracle(inp, sig, cfg, units=[0, 3])
+    o, lse, h2l = run_mla(inp, cfg, lists, counts, 4)
+    rng = np.random.default_rng(1)
+    rows = [(b, t, int(h)) for b in (0, 3) for t in range(cfg.T) for h in rng.integers(0, cfg.Hq, 6)]
+    rows += [(0, 1, int(h)) for h in inp["ambient_heads"][:3].tolist()]
+    kvb = bits(inp["kv"])
+    ro, rl = O.sparse_attention(bits(inp["q"]), kvb, kvb[..., :cfg.Dv], np_i32(inp["page_table"]),
+                                np_i32(inp["seq_lens"]), lists, counts, np.array(h2l),
+                                1.0 / math.sqrt(cfg.Dk), cfg.page_size, rows=rows)
+    og, lg = o.cpu().double().numpy(), lse.cpu().double().numpy()
+    for (b, t, h) in rows:
+        assert np.abs(og[b, t, h] - ro[b, t, h]).max() <= O_TOL, (b, t, h)
+        assert abs(lg[b, t, h] - rl[b, t, h]) <= LSE_TOL, (b, t, h)
