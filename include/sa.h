@@ -119,6 +119,33 @@ SA_API int sa_select_pages(const uint16_t* q, const int64_t q_strides[4],
 SA_API size_t sa_select_workspace_size(int B, int Hkv, int max_pages);
 
 /*
+ * sa_select_pages_no_alloc — sa_select_pages for callers that cannot
+ * allocate device memory at the call site: code running inside a CUDA-graph
+ * capture, a serving loop whose memory pool is sealed after warm-up, or a host
+ * framework that owns every allocation and passes only raw pointers.  (The
+ * pages this library implements have no counterpart of this entry point; it
+ * is a deployment convenience.)
+ *
+ * Same arguments, outputs and results as sa_select_pages, minus the
+ * workspace: the score bounds go to a 16 MiB array of the library's own device
+ * memory (2,097,152 pages x 8 bytes), which every GPU that loads the library
+ * holds until the process exits.  Limit: B * Hkv * max_pages <= 2,097,152;
+ * larger calls return SA_ERR_UNSUPPORTED and launch nothing.  The first call
+ * on a device looks up the array's device address (cudaGetSymbolAddress); make
+ * that first call before any stream capture.  All calls share the one array
+ * (it needs no clearing: each call writes every entry it reads), so calls
+ * whose kernels overlap on the GPU — on different streams, or from different
+ * threads — race and must be serialised by the caller.
+ */
+SA_API int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4],
+                                    const uint16_t* summaries, const int32_t* page_table,
+                                    const int32_t* seq_lens, int B, int T, int Hq, int Hkv,
+                                    int Dk, int page_size, int max_pages, int P_pool,
+                                    int sink_tokens, int local_tokens, int budget_tokens,
+                                    int32_t* out_pages, int32_t* out_counts, int32_t* dev_error,
+                                    void* stream);
+
+/*
  * sa_select_pages_tiered — Critical / Ambient tier selection for one shared
  * latent KV head (MLA; "TileSparse: Arithmetic-Intensity-Aware Sparse
  * Attention for Compute-Bound LLM Decoding", "Motivation": a Critical Tier of

@@ -29,6 +29,8 @@ _SIGNATURES = {
     "sa_select_pages": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                              _I, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "sa_select_workspace_size": (ctypes.c_size_t, [_I, _I, _I]),
+    "sa_select_pages_no_alloc": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                      _I, _I, _I, _P, _P, _P, _P]),
     "sa_select_pages_tiered": (_I, [_P, _c_i64_4, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                     _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "sa_select_tiered_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
@@ -144,6 +146,27 @@ def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tok
                              _ptr(out_counts), _ptr(workspace), workspace.numel(),
                              _ptr(dev_error), _stream(stream))
     _check(st, "sa_select_pages")
+    return out_pages, out_counts
+
+
+def sa_select_pages_no_alloc(q, summaries, page_table, seq_lens, page_size: int,
+                             sink_tokens: int, local_tokens: int, budget_tokens: int, out_pages,
+                             out_counts, dev_error=None, P_pool: int = None, stream=None):
+    """sa_select_pages without a workspace: the score bounds go to the library's
+    static device array (shared by all calls; calls must not overlap on the GPU).
+    The outputs must be preallocated; nothing is allocated here."""
+    lib = load()
+    _need_cuda(q, summaries, page_table, seq_lens, out_pages, out_counts)
+    _bf16(q), _bf16(summaries), _i32(page_table), _i32(seq_lens)
+    B, T, Hq, Dk = q.shape
+    P_pool_, Hkv, _ = summaries.shape
+    P_pool = P_pool_ if P_pool is None else P_pool
+    st = lib.sa_select_pages_no_alloc(_ptr(q), _strides4(q), _ptr(summaries), _ptr(page_table),
+                                      _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size,
+                                      page_table.shape[1], P_pool, sink_tokens, local_tokens,
+                                      budget_tokens, _ptr(out_pages), _ptr(out_counts),
+                                      _ptr(dev_error), _stream(stream))
+    _check(st, "sa_select_pages_no_alloc")
     return out_pages, out_counts
 
 

@@ -159,6 +159,22 @@ int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_
   return cuda_status(launch_select_gqa(a, static_cast<cudaStream_t>(stream)));
 }
 
+int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4],
+                             const uint16_t* summaries, const int32_t* page_table,
+                             const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int Dk,
+                             int page_size, int max_pages, int P_pool, int sink_tokens,
+                             int local_tokens, int budget_tokens, int32_t* out_pages,
+                             int32_t* out_counts, int32_t* dev_error, void* stream) {
+  SelectArgs a;
+  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
+                          page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
+                          out_pages, out_counts, dev_error, &a))
+    return r;
+  if (B == 0) return SA_OK;
+  if ((size_t)B * Hkv * max_pages > select_static_capacity()) return SA_ERR_UNSUPPORTED;
+  return cuda_status(launch_select_gqa_static(a, static_cast<cudaStream_t>(stream)));
+}
+
 size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_pages) {
   if (B <= 0 || T <= 0 || Hq <= 0 || max_pages <= 0) return 0;
   return tiered_workspace_bytes(B, T, Hq, max_pages);

@@ -72,6 +72,8 @@ struct SelectArgs {
 };
 size_t select_workspace_bytes(int B, int Hkv, int max_pages);
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream);
+size_t select_static_capacity();
+cudaError_t launch_select_gqa_static(SelectArgs a, cudaStream_t stream);
 
 struct TieredArgs {
   const uint16_t* q;

@@ -19,6 +19,8 @@
 // Source: "Universal Attention Engine — Declarative Sparse Attention for
 // Production", "Content-Dependent Dynamic Routing" (top_k_blocks over
 // q @ mean(k_blocks), at block granularity) and "The Product" (sink + local).
+#include <mutex>
+
 #include "common.cuh"
 #include "exact.cuh"
 #include "internal.h"
@@ -306,5 +308,52 @@ cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+
+// ---------------------------------------------------------------------------
+// Selection without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they select
+// pages: code running inside a CUDA-graph capture region, a serving loop
+// whose memory pool is sealed after warm-up, or a host framework that owns
+// every allocation and hands this library raw pointers only.  For them the
+// score bounds live in a fixed-size array in the library's own device memory,
+// reserved when the library is loaded (on every GPU that loads it, until the
+// process exits).
+constexpr size_t kStaticScoreEntries = size_t(1) << 21;   // 2,097,152 pages x 8 bytes = 16 MiB
+static __device__ __align__(256) float2 g_static_score_bounds[kStaticScoreEntries];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+float2* g_static_ptr[kMaxDevices] = {};
+
+// Device address of the static array on the current device; looked up once per
+// device (the host-side symbol is only a stand-in and must not reach a kernel).
+cudaError_t static_scores_ptr(float2** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_score_bounds);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = static_cast<float2*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
+size_t select_static_capacity() { return kStaticScoreEntries; }
+
+cudaError_t launch_select_gqa_static(SelectArgs a, cudaStream_t stream) {
+  float2* p = nullptr;
+  cudaError_t e = static_scores_ptr(&p);
+  if (e != cudaSuccess) return e;
+  a.lohi = p;
+  return launch_select_gqa(a, stream);
+}
 
 }  // namespace sa
