@@ -17,6 +17,8 @@
 // Production" ("Architecture": gather-based sparse KV decode; "Key Design
 // Decisions" 3: decode is memory-bound, optimise bytes loaded) and "TileSparse"
 // ("Two implementations": a per-head page-list Flash-decode kernel).
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -51,15 +53,13 @@ struct __align__(64) DecodeParams {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kNW * 32)
+__global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     decode_gqa_kernel(const __grid_constant__ DecodeParams prm,
                       const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap) {
   using C = DecodeCfg<D>;
   const DecodeArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int split = blockIdx.x * kNW + warp, pair = blockIdx.y, b = blockIdx.z;
-  if (split >= a.n_splits) return;
   const int gid = lane >> 2, tig = lane & 3;
 
   extern __shared__ uint8_t dyn_smem[];
@@ -67,6 +67,25 @@ __global__ void __launch_bounds__(kNW * 32)
   __shared__ uint64_t bars[kNW][C::kStages];
   __shared__ int2 ent_s[kNW][kWarpEntries];    // (physical page, first token) per entry
 
+  if (lane == 0) {
+    for (int s = 0; s < C::kStages; ++s) mbar_init(&bars[warp][s], 1);
+    fence_mbar_init();
+    prefetch_tmap(&kmap);
+    prefetch_tmap(&vmap);
+  }
+  __syncwarp();
+  // Work items are (split, pair, sequence) triples, flattened; each warp takes
+  // items warp_id, warp_id + total_warps, ... so that every SM gets the same
+  // share whatever the grid's shape.  The ring's unit counter `base` runs on
+  // across items, which keeps the mbarrier phases in step.
+  const int n_items = a.n_splits * prm.pairs.n_pairs * a.B;
+  const int total_warps = gridDim.x * kNW;
+  uint8_t* ring = smem + warp * C::kStages * C::kStageBytes;
+  int base = 0;
+  for (int item = blockIdx.x * kNW + warp; item < n_items; item += total_warps) {
+  const int split = item % a.n_splits;
+  const int pair = (item / a.n_splits) % prm.pairs.n_pairs;
+  const int b = item / (a.n_splits * prm.pairs.n_pairs);
   const int list = prm.pairs.list_of[pair];
   const int kvh = prm.pairs.kvh_of[pair];
   const int nh = prm.pairs.n_heads[pair];
@@ -87,10 +106,6 @@ __global__ void __launch_bounds__(kNW * 32)
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
 
-  if (lane == 0) {
-    for (int s = 0; s < C::kStages; ++s) mbar_init(&bars[warp][s], 1);
-    fence_mbar_init();
-  }
   // Resolve logical -> physical pages of this split (32 entries per round).
   const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
   const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
@@ -112,7 +127,6 @@ __global__ void __launch_bounds__(kNW * 32)
 
   const int subs = a.P / kSub;
   const int n_units = n_ent * subs;
-  uint8_t* ring = smem + warp * C::kStages * C::kStageBytes;
 
   auto unit_live = [&](int u, int& ph, int& tok0) {
     const int2 e = ent_s[warp][u / subs];
@@ -121,7 +135,7 @@ __global__ void __launch_bounds__(kNW * 32)
     return ph >= 0 && tok0 < L;
   };
   auto issue = [&](int u) {  // lane 0 only
-    const int slot = u % C::kStages;
+    const int slot = (base + u) % C::kStages;
     uint64_t* bar = &bars[warp][slot];
     int ph, tok0;
     if (unit_live(u, ph, tok0)) {
@@ -138,11 +152,8 @@ __global__ void __launch_bounds__(kNW * 32)
       mbar_arrive_expect_tx(bar, 0);
     }
   };
-  if (lane == 0) {
-    prefetch_tmap(&kmap);
-    prefetch_tmap(&vmap);
+  if (lane == 0)
     for (int u = 0; u < n_units && u < C::kStages; ++u) issue(u);
-  }
 
   // Query fragments (A operand of QK^T), rows r = t * nh + i.
   uint32_t qa[D / 16][4];
@@ -181,8 +192,8 @@ __global__ void __launch_bounds__(kNW * 32)
   const int mi = lane >> 3, ri = lane & 7;
 
   for (int u = 0; u < n_units; ++u) {
-    const int slot = u % C::kStages;
-    if (!mbar_wait_bounded(&bars[warp][slot], (u / C::kStages) & 1)) {
+    const int slot = (base + u) % C::kStages;
+    if (!mbar_wait_bounded(&bars[warp][slot], ((base + u) / C::kStages) & 1)) {
       u_fail = u;
       break;
     }
@@ -288,7 +299,8 @@ __global__ void __launch_bounds__(kNW * 32)
     // units u_fail .. u_fail + kStages - 1 were issued: wait for them (bounded)
     // before this warp's shared memory can be released
     for (int u = u_fail + 1; u < n_units && u < u_fail + C::kStages; ++u)
-      mbar_wait_bounded(&bars[warp][u % C::kStages], (u / C::kStages) & 1);
+      mbar_wait_bounded(&bars[warp][(base + u) % C::kStages], ((base + u) / C::kStages) & 1);
+    return;
   }
 
   // ---- normalise and write this split's partial from registers
@@ -313,6 +325,8 @@ __global__ void __launch_bounds__(kNW * 32)
     if (tig == 0)
       a.lse_part[row] = empty ? -INFINITY : (m_ref[h] + log2f(l_run[h])) * kLn2;
   }
+  base += n_units;
+  }  // items
 }
 
 template <int D>
@@ -325,7 +339,17 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDynBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.n_splits + kNW - 1) / kNW, pairs.n_pairs, a.B);
+  // one wave of resident CTAs (or fewer when there is less work)
+  int dev = 0, sms = 0, per_sm = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess)
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D>, kNW * 32,
+                                                      C::kDynBytes);
+  if (e != cudaSuccess) return e;
+  const long long items = (long long)a.n_splits * pairs.n_pairs * a.B;
+  const long long want = (items + kNW - 1) / kNW;
+  const int grid = (int)std::min<long long>(want, (long long)std::max(1, per_sm) * sms);
   decode_gqa_kernel<D><<<grid, kNW * 32, C::kDynBytes, stream>>>(prm, kmap, vmap);
   return cudaGetLastError();
 }

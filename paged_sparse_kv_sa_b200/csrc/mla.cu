@@ -115,6 +115,17 @@ __global__ void __launch_bounds__(kMThreads, 1)
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
   const int r0 = qt * kMRows;
+  if (n_ent == 0) {   // an empty split: its partial is O = 0, LSE = -inf
+    const int nr = min(kMRows, rows_total - r0);
+    for (int i = tid; i < nr * (kDv / 4); i += blockDim.x) {
+      const int rr = r0 + i / (kDv / 4), c = (i % (kDv / 4)) * 4;
+      const int t = rr / nh, head = prm.pairs.heads[pair][rr % nh];
+      const int64_t orow = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
+      *reinterpret_cast<float4*>(a.o_part + orow * kDv + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c == 0) a.lse_part[orow] = -INFINITY;
+    }
+    return;
+  }
   const int t_last = (min(rows_total, r0 + kMRows) - 1) / nh;
   const int max_q = L - a.T + t_last;
 

@@ -2,22 +2,25 @@
 // kv head) pair — chunked prefill over block-union tables, long MTP — on the
 // 5th-generation tensor cores.
 //
-// One CTA computes 128 query rows (the pair's (token, head) rows, token-major)
-// against the keys of its split of the list, 64 keys per tile:
-//   warp 4      gathers K and V tiles from the paged pool with TMA (four
+// One CTA computes 256 query rows of a pair (token-major) as two 128-row tiles
+// A and B against the keys of its split of the list, 64 keys per tile; each
+// K/V tile is loaded once and used by both:
+//   warp 8      gathers K and V tiles from the paged pool with TMA (four
 //               16-key x 64-column boxes per 64-column chunk; an absent or
 //               invalid 16-key group is loaded from an out-of-range page
 //               coordinate, which TMA fills with zeros) into a 3-stage ring;
-//   warp 5      issues tcgen05.mma: S = Q K^T (M=128, N=64, K=D) into one of
-//               two TMEM S buffers, and O += P V (M=128, N=D, K=64) into TMEM,
-//               with tcgen05.commit arrivals on mbarriers;
-//   warps 0-3   own one query row per thread: load Q into shared memory,
-//               read S rows from TMEM, mask (page validity, sequence end,
-//               causal position), run a base-2 online softmax whose running
-//               max only moves when a row's max exceeds it by more than 2^8
-//               (the O rescale through TMEM is then rare), write P (bf16) to
-//               shared memory for the PV MMA, and finally normalise O.
-// The QK^T of tile j+1 overlaps the softmax of tile j (two S buffers).
+//   warp 9      issues tcgen05.mma, alternating between the tiles: S_A = Q_A K^T
+//               and S_B = Q_B K^T (M=128, N=64, K=D) into double-buffered TMEM
+//               S buffers, then O_A += P_A V and O_B += P_B V (M=128, N=D) into
+//               TMEM, with tcgen05.commit arrivals on mbarriers;
+//   warps 0-3 / 4-7   (one warpgroup per tile) own one query row per thread:
+//               Q into shared memory, S rows from TMEM, masking (page validity,
+//               sequence end, causal position; skipped for tiles every row sees
+//               whole), a base-2 online softmax whose running max only moves when
+//               a row's max exceeds it by more than 2^8 (the O rescale through
+//               TMEM is then rare), P (bf16) to shared memory, and the epilogue.
+// While one warpgroup runs its softmax the tensor core works on the other's
+// tile, and QK^T of tile j+1 overlaps the softmax of tile j.
 //
 // Sources: CompactAttention (abstract on the page titled "Causal Attention on
 // CPU: A Cache-Aware and Load-Balanced Scheduling Kernel for Prefill"):
@@ -31,10 +34,11 @@
 namespace sa {
 namespace {
 
-constexpr int kPThreads = 192;
+constexpr int kPThreads = 320;    // 2 softmax warpgroups, producer warp, MMA warp
 constexpr int kPStages = 3;
 constexpr int kKeys = 64;         // keys per tile
-constexpr int kM = 128;           // query rows per CTA
+constexpr int kM = 128;           // query rows per warpgroup tile
+constexpr int kRows = 2 * kM;     // query rows per CTA
 constexpr int kMaxEnt = 1024;     // list entries per split
 constexpr float kLazyP = 8.f;
 
@@ -45,8 +49,9 @@ struct PCfg {
   static constexpr int kTileBytes = kKeys * D * 2;     // one K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kPBytes = kM * kKeys * 2;
-  static constexpr int kDyn = kQBytes + 2 * kPBytes + kPStages * kStageBytes + 1024;
-  static constexpr uint32_t kTmemCols = 256;           // S0 [0,64) S1 [64,128) O [128,128+D)
+  static constexpr int kDyn = 2 * kQBytes + 2 * kPBytes + kPStages * kStageBytes + 1024;
+  // per tile w: S buffers at 128w + {0, 64}, O at 256 + 128w
+  static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdQK = tc::idesc_bf16_f32(kM, kKeys, false, false);
   static constexpr uint32_t kIdPV = tc::idesc_bf16_f32(kM, D, false, true);
 };
@@ -98,21 +103,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int qt = blockIdx.x / a.n_splits, split = blockIdx.x % a.n_splits;
   const int nh = prm.pairs.n_heads[pair];
   const int rows_total = a.T * nh;
-  if (qt * kM >= rows_total) return;                 // whole CTA: nothing to do
+  if (qt * kRows >= rows_total) return;               // whole CTA: nothing to do
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int list = prm.pairs.list_of[pair], kvh = prm.pairs.kvh_of[pair];
 
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
-  uint8_t* q_s = smem;
-  uint8_t* p_s = smem + C::kQBytes;                          // 2 buffers
+  uint8_t* q_s = smem;                                       // 2 tiles
+  uint8_t* p_s = smem + 2 * C::kQBytes;                      // 2 tiles
   uint8_t* kv_s = p_s + 2 * C::kPBytes;                      // kPStages x (K | V)
   __shared__ uint64_t kv_full[kPStages], kv_empty[kPStages];
-  __shared__ uint64_t s_full[2], p_full[2], o_done, q_full;
+  __shared__ uint64_t s_full[2][2], p_full[2], o_done[2], q_full;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, n_act_s;
   __shared__ int2 ent_s[kMaxEnt];
-  __shared__ int act_s[kMaxEnt];
+  __shared__ int act_s[kMaxEnt];     // (tile << 1) | needs_mask
 
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) {
@@ -128,9 +133,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int chunk = (count + a.n_splits - 1) / a.n_splits;
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
-  const int r0 = qt * kM;
-  const int t_last = (min(rows_total, r0 + kM) - 1) / nh;
-  const int max_q = L - a.T + t_last;
+  const int r0 = qt * kRows;
+  if (n_ent == 0) {   // an empty split: its partial is O = 0, LSE = -inf
+    const int nr = min(kRows, rows_total - r0);
+    for (int i = tid; i < nr * (D / 4); i += blockDim.x) {
+      const int rr = r0 + i / (D / 4), c = (i % (D / 4)) * 4;
+      const int t = rr / nh, head = prm.pairs.heads[pair][rr % nh];
+      const int64_t orow = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
+      *reinterpret_cast<float4*>(a.o_part + orow * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (c == 0) a.lse_part[orow] = -INFINITY;
+    }
+    return;
+  }
+  const int t_first = r0 / nh;
+  const int t_last = (min(rows_total, r0 + kRows) - 1) / nh;
+  const int min_q = L - a.T + t_first, max_q = L - a.T + t_last;
 
   // ---- resolve pages, set up barriers and TMEM
   const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
@@ -154,35 +171,39 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&p_full[s], 128);
+    for (int w = 0; w < 2; ++w) {
+      mbar_init(&s_full[w][0], 1);
+      mbar_init(&s_full[w][1], 1);
+      mbar_init(&p_full[w], 128);
+      mbar_init(&o_done[w], 1);
     }
-    mbar_init(&o_done, 1);
-    mbar_init(&q_full, 128);
+    mbar_init(&q_full, 256);
     abort_s = 0;
     fence_mbar_init();
   }
-  if (warp == 5) tc::tmem_alloc(&tmem_base_s, C::kTmemCols);
+  if (warp == 9) tc::tmem_alloc(&tmem_base_s, C::kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_base_s;
 
-  // ---- tiles with at least one causally visible key, in list order
+  // ---- tiles with at least one causally visible key, in list order; a tile
+  // every row of the CTA sees whole (all groups valid and below min_q) skips
+  // the per-element mask
   const int n_tiles = a.P <= kKeys ? (n_ent * a.P + kKeys - 1) / kKeys : n_ent * (a.P / kKeys);
   if (warp == 0) {
     int n_act = 0;
     for (int j0 = 0; j0 < n_tiles; j0 += 32) {
       const int j = j0 + lane;
-      bool live = false;
+      bool live = false, whole = true;
       if (j < n_tiles)
         for (int g = 0; g < 4; ++g) {
           const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
           live |= gr.x >= 0 && gr.y < L && gr.y <= max_q;
+          whole &= gr.x >= 0 && gr.y + 15 < L && gr.y + 15 <= min_q;
         }
       const uint32_t m = __ballot_sync(0xffffffffu, live);
-      if (live) act_s[n_act + __popc(m & ((1u << lane) - 1u))] = j;
+      if (live) act_s[n_act + __popc(m & ((1u << lane) - 1u))] = (j << 1) | (whole ? 0 : 1);
       n_act += __popc(m);
     }
     if (lane == 0) n_act_s = n_act;
@@ -191,7 +212,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int n_act = n_act_s;
   volatile int* abort_flag = &abort_s;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ================= producer: TMA gathers of K and V tiles
     if (lane == 0) {
       prefetch_tmap(&kmap);
@@ -201,7 +222,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (jj >= kPStages &&
             !wait_or_abort(&kv_empty[st], ((jj / kPStages) - 1) & 1, abort_flag))
           break;
-        const int j = act_s[jj];
+        const int j = act_s[jj] >> 1;
         uint8_t* kt = kv_s + st * C::kStageBytes;
         uint8_t* vt = kt + C::kTileBytes;
         mbar_arrive_expect_tx(&kv_full[st], C::kStageBytes);
@@ -222,22 +243,24 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
       }
     }
-  } else if (warp == 5) {
-    // ================= MMA issuer (one thread)
+  } else if (warp == 9) {
+    // ================= MMA issuer (one thread), alternating tiles A and B
     if (lane == 0 && n_act > 0) {
       const uint32_t q_addr = smem_u32(q_s), p_addr = smem_u32(p_s), kv_addr = smem_u32(kv_s);
       auto pv = [&](int jp) -> bool {
-        const int sb = jp & 1, st = jp % kPStages;
-        if (!wait_or_abort(&p_full[sb], (jp >> 1) & 1, abort_flag)) return false;
-        tc::fence_after_sync();
+        const int st = jp % kPStages;
         const uint32_t vbase = kv_addr + st * C::kStageBytes + C::kTileBytes;
+        for (int w = 0; w < 2; ++w) {
+          if (!wait_or_abort(&p_full[w], jp & 1, abort_flag)) return false;
+          tc::fence_after_sync();
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint64_t ad = tc::sdesc_sw128(p_addr + sb * C::kPBytes + kk * 32, 16, 1024);
-          const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
-          tc::mma_bf16(tmem + 128, ad, bd, C::kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kKeys / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(p_addr + w * C::kPBytes + kk * 32, 16, 1024);
+            const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
+            tc::mma_bf16(tmem + 256 + 128 * w, ad, bd, C::kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc::commit(&o_done[w]);
         }
-        tc::commit(&o_done);
         tc::commit(&kv_empty[st]);
         return true;
       };
@@ -248,27 +271,31 @@ __global__ void __launch_bounds__(kPThreads, 1)
         if (!wait_or_abort(&kv_full[st], (jj / kPStages) & 1, abort_flag)) break;
         tc::fence_after_sync();
         const uint32_t kbase = kv_addr + st * C::kStageBytes;
+        for (int w = 0; w < 2; ++w) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad =
-              tc::sdesc_sw128(q_addr + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd =
-              tc::sdesc_sw128(kbase + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
-          tc::mma_bf16(tmem + sb * kKeys, ad, bd, C::kIdQK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = tc::sdesc_sw128(
+                q_addr + w * C::kQBytes + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd =
+                tc::sdesc_sw128(kbase + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
+            tc::mma_bf16(tmem + 128 * w + sb * kKeys, ad, bd, C::kIdQK, kk > 0 ? 1u : 0u);
+          }
+          tc::commit(&s_full[w][sb]);
         }
-        tc::commit(&s_full[sb]);
         if (jj >= 1 && !pv(jj - 1)) ok = false;
       }
       if (ok) pv(n_act - 1);
     }
   } else {
     // ================= softmax / epilogue: one query row per thread
-    const int r = warp * 32 + lane;
-    const int rg = r0 + r;
+    const int wg = warp >> 2;                       // tile A (0) or B (1)
+    const int r = (warp & 3) * 32 + lane;           // row within the tile = TMEM lane
+    const int rg = r0 + wg * kM + r;
     const bool row_ok = rg < rows_total;
     const int t = row_ok ? rg / nh : 0;
     const int head = prm.pairs.heads[pair][row_ok ? rg % nh : 0];
     const int qpos = row_ok ? L - a.T + t : -1;
+    uint8_t* qt_s = q_s + wg * C::kQBytes;
     {
       const uint4* src = reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + head * a.qs2);
 #pragma unroll
@@ -276,41 +303,51 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const uint4 v = row_ok ? src[c * 8 + ch] : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(q_s + c * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+          *reinterpret_cast<uint4*>(qt_s + c * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
         }
     }
     tc::fence_proxy_async();
     mbar_arrive(&q_full);
-    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t s_col = 128 * wg, o_col = 256 + 128 * wg;
+    uint8_t* prow = p_s + wg * C::kPBytes + r * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int jj = 0; jj < n_act; ++jj) {
-      const int sb = jj & 1, j = act_s[jj];
-      if (!wait_or_abort(&s_full[sb], (jj >> 1) & 1, abort_flag)) {
+      const int sb = jj & 1, code = act_s[jj], j = code >> 1;
+      if (!wait_or_abort(&s_full[wg][sb], (jj >> 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
       float x[64];
-      tc::ld32(tmem + lane_base + sb * kKeys, *reinterpret_cast<float(*)[32]>(&x[0]));
-      tc::ld32(tmem + lane_base + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+      tc::ld32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(&x[0]));
+      tc::ld32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
       tc::wait_ld();
       float mx = -INFINITY;
+      if (code & 1) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
-        const bool gok = gr.x >= 0;
+        for (int g = 0; g < 4; ++g) {
+          const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
+          const bool gok = gr.x >= 0;
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int kp = gr.y + c;
-          const bool vis = gok && kp < L && kp <= qpos;
-          const float v = vis ? x[g * 16 + c] * a.scale_log2 : -INFINITY;
-          x[g * 16 + c] = v;
-          mx = fmaxf(mx, v);
+          for (int c = 0; c < 16; ++c) {
+            const int kp = gr.y + c;
+            const bool vis = gok && kp < L && kp <= qpos;
+            const float v = vis ? x[g * 16 + c] * a.scale_log2 : -INFINITY;
+            x[g * 16 + c] = v;
+            mx = fmaxf(mx, v);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          x[c] *= a.scale_log2;
+          mx = fmaxf(mx, x[c]);
         }
       }
-      // PV(jj-1) must be done before O is rescaled or P buffer sb is rewritten
-      if (jj >= 1 && !wait_or_abort(&o_done, (jj - 1) & 1, abort_flag)) {
+      // PV(jj-1) must be done before O is rescaled or P is rewritten
+      if (jj >= 1 && !wait_or_abort(&o_done[wg], (jj - 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
@@ -324,17 +361,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             float o[32];
-            tc::ld32(tmem + lane_base + 128 + c * 32, o);
+            tc::ld32(tmem + lane_base + o_col + c * 32, o);
             tc::wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tc::st32(tmem + lane_base + 128 + c * 32, o);
+            tc::st32(tmem + lane_base + o_col + c * 32, o);
           }
           tc::wait_st();
         }
       }
       const float base = m_ref == -INFINITY ? 0.f : m_ref;
-      uint8_t* prow = p_s + sb * C::kPBytes + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         float p[8];
@@ -352,9 +388,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[wg]);
     }
-    if (ok && n_act > 0) ok = wait_or_abort(&o_done, (n_act - 1) & 1, abort_flag);
+    if (ok && n_act > 0) ok = wait_or_abort(&o_done[wg], (n_act - 1) & 1, abort_flag);
     tc::fence_after_sync();
     // ---- epilogue: O / l and LSE for this row
     const bool empty = !ok || n_act == 0 || l == 0.f;
@@ -364,7 +400,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     for (int c = 0; c < D / 32; ++c) {
       float o[32];
       if (n_act > 0) {
-        tc::ld32(tmem + lane_base + 128 + c * 32, o);
+        tc::ld32(tmem + lane_base + o_col + c * 32, o);
         tc::wait_ld();
       }
       if (row_ok) {
@@ -382,7 +418,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, C::kTmemCols);
   }
@@ -397,7 +433,7 @@ cudaError_t launch_p(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   prm.pairs = pairs;
   int max_rows = 0;
   for (int i = 0; i < pairs.n_pairs; ++i) max_rows = max(max_rows, a.T * pairs.n_heads[i]);
-  const int qtiles = (max_rows + kM - 1) / kM;
+  const int qtiles = (max_rows + kRows - 1) / kRows;
   cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDyn);
   if (e != cudaSuccess) return e;

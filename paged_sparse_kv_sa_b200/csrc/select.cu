@@ -20,6 +20,7 @@
 // Production", "Content-Dependent Dynamic Routing" (top_k_blocks over
 // q @ mean(k_blocks), at block granularity) and "The Product" (sink + local).
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "exact.cuh"
@@ -30,7 +31,8 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 512;       // choose_kernel
-constexpr int kScoreThreads = 256;  // score_kernel: one page per thread
+constexpr int kScoreThreads = 128;  // score_kernel: 4 warps x 32 pages
+constexpr int kScorePages = 128;
 constexpr int kMaxRows = 16;
 constexpr int kMaxDk = 256;
 
@@ -79,81 +81,156 @@ SA_DEV float load_q_rows(const SelectArgs& a, int b, int kvh, float* q_s, float*
   return sqrtf(qn * (1.f + 2.f * Dk * 5.96046448e-8f)) * (1.f + 1.2e-7f);
 }
 
+SA_DEV void cp_async16(void* smem_dst, const void* gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
+               : "memory");
+}
+
+// Packed float32 FMA (two lanes of a 64-bit register pair, each rounded as
+// an ordinary fma.rn.f32).
+SA_DEV void ffma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
+  asm volatile("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+SA_DEV float hsum2(unsigned long long v) {
+  return __uint_as_float(static_cast<uint32_t>(v)) + __uint_as_float(static_cast<uint32_t>(v >> 32));
+}
+// bf16x2 word -> the two features as a float32 pair (low half first)
+SA_DEV unsigned long long unpack2(uint32_t w) {
+  return (static_cast<unsigned long long>(w & 0xffff0000u) << 32) |
+         static_cast<unsigned long long>(w << 16);
+}
+
 // lo/hi bounds of every candidate page's score; NaN for forced pages.
+// LPP = Dk / FPL lanes share a page, each holding FPL features of every query
+// row in registers; a warp scores 32 / LPP pages per step, reading each page
+// row as one coalesced run.  Per page a lane does FPL/2 packed FMAs per row
+// (two float32 lanes: even / odd features), then the row sums are reduced over
+// the LPP lanes with xor shuffles.  Any summation order obeys the bound
+// |fl(q.s) - q.s| <= gamma_Dk ||q|| ||s||, so the bracket stays rigorous.
+template <int RP, int DK>   // rows rounded up to a power of two; feature count
 __global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a) {
-  const int chunk = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  constexpr int FPL = RP <= 8 ? 16 : 8;            // features per lane
+  constexpr int LPP = DK / FPL;                    // lanes per page
+  constexpr int NSTEPS = LPP;                      // 32 pages / (32 / LPP) per step
+  constexpr int HOIST = NSTEPS < 8 ? NSTEPS : 8;   // pages steps loaded at once
+  // kv heads vary fastest across the grid: the CTAs reading the Hkv adjacent
+  // rows of the same pages run together and share DRAM pages / L2 lines
+  const int kvh = blockIdx.x, chunk = blockIdx.y, b = blockIdx.z;
   const int L = clamped_len(a, b, false);
   const int N = (L + a.P - 1) / a.P;
   if (N <= a.budget_pages || a.k_top == 0) return;   // no ranking needed
-  const int p0 = chunk * kScoreThreads;
+  const int p0 = chunk * kScorePages;
   if (p0 >= N) return;
-  __shared__ __align__(16) float q_s[kMaxRows * kMaxDk];
-  __shared__ float red[kScoreThreads / 32];
-  const float qn = load_q_rows(a, b, kvh, q_s, red);
-  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
+  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = DK;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int fb = lane % LPP, slot = lane / LPP, pages_per_step = 32 / LPP;
+  const int f0 = fb * FPL;
+  // query rows: FPL features each, as float32 pairs; row norms for the bound
+  unsigned long long qv[RP][FPL / 2];
+  float qn2 = 0.f;
+#pragma unroll
+  for (int r = 0; r < RP; ++r) {
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < FPL / 8; ++i) {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (r < R) {
+        const int t = r / G, h = kvh * G + r % G;
+        w = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 + f0 + 8 * i);
+      }
+      const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qv[r][4 * i + e] = unpack2(w4[e]);
+        const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
+        part = fmaf(x0, x0, fmaf(x1, x1, part));
+      }
+    }
+#pragma unroll
+    for (int o = LPP / 2; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    qn2 = fmaxf(qn2, part);
+  }
   const float nu = Dk * 5.96046448e-8f;
+  // the float32 sums of squares are within (1 + gamma_Dk) of the truth
+  const float qn = sqrtf(qn2 * (1.f + 2.f * nu)) * (1.f + 1.2e-7f);
   const float gfac = nu / (1.f - nu) * 1.0001f * qn * 1.0001f;
   const float sq_pad = 1.f + 2.f * nu;
   const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
-
-  const int p = p0 + threadIdx.x;
-  if (p >= N) return;
-  float2* out = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages + p;
-  if (p < n_sink || p >= local0) {
-    *out = make_float2(NAN, NAN);
-    return;
-  }
-  const int ph = a.page_table[(int64_t)b * a.max_pages + p];
-  if (ph < 0 || ph >= a.P_pool) {
-    set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
-    *out = make_float2(-INFINITY, -INFINITY);   // an unreadable page never wins a slot
-    return;
-  }
-  const uint4* row = reinterpret_cast<const uint4*>(a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk);
-  float acc[kMaxRows];
+  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+  float2* outrow = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
+  // this warp's 32 pages, pages_per_step at a time, HOIST steps per batch: first
+  // every page-table lookup, then every row load, so that they are in flight
+  // together, then the arithmetic
+  const int wp0 = p0 + warp * 32;
+#pragma unroll 1
+  for (int sb = 0; sb < NSTEPS; sb += HOIST) {
+    int phs[HOIST];
+    uint4 v[HOIST][FPL / 8];
 #pragma unroll
-  for (int r = 0; r < kMaxRows; ++r) acc[r] = 0.f;
-  float ss = 0.f;
-  // 64 features per batch: 8 x 16-byte loads, unpacked once, then every query
-  // row streams its 64 float32 coefficients from shared memory (broadcast).
-  for (int d0 = 0; d0 < Dk; d0 += 64) {
-    uint4 v[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = __ldcs(row + d0 / 8 + j);
-    float x[64];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t w4[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[8 * j + 2 * e] = __uint_as_float(w4[e] << 16);
-        x[8 * j + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+    for (int k = 0; k < HOIST; ++k) {
+      phs[k] = -1;
+      const int p = wp0 + (sb + k) * pages_per_step + slot;
+      if (p < N && p >= n_sink && p < local0) {
+        const int ph = ptrow[p];
+        phs[k] = (ph < 0 || ph >= a.P_pool) ? -2 : ph;
       }
     }
 #pragma unroll
-    for (int i = 0; i < 64; ++i) ss = fmaf(x[i], x[i], ss);
+    for (int k = 0; k < HOIST; ++k) {
 #pragma unroll
-    for (int r = 0; r < kMaxRows; ++r) {
-      if (r < R) {
-        const float4* qr = reinterpret_cast<const float4*>(&q_s[r * Dk + d0]);
+      for (int i = 0; i < FPL / 8; ++i) v[k][i] = make_uint4(0, 0, 0, 0);
+      if (phs[k] >= 0) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(a.sig + ((int64_t)phs[k] * a.Hkv + kvh) * Dk + f0);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float4 qq = qr[i];
-          acc[r] = fmaf(qq.x, x[4 * i], acc[r]);
-          acc[r] = fmaf(qq.y, x[4 * i + 1], acc[r]);
-          acc[r] = fmaf(qq.z, x[4 * i + 2], acc[r]);
-          acc[r] = fmaf(qq.w, x[4 * i + 3], acc[r]);
+        for (int i = 0; i < FPL / 8; ++i) v[k][i] = __ldcs(src + i);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < HOIST; ++k) {
+      const int p = wp0 + (sb + k) * pages_per_step + slot;
+      const bool cand = p < N && p >= n_sink && p < local0;
+      const int ph = phs[k];
+      if (ph == -2 && fb == 0) set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
+      unsigned long long acc[RP], ss = 0ull;
+#pragma unroll
+      for (int r = 0; r < RP; ++r) acc[r] = 0ull;
+#pragma unroll
+      for (int i = 0; i < FPL / 8; ++i) {
+        const uint32_t w4[4] = {v[k][i].x, v[k][i].y, v[k][i].z, v[k][i].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const unsigned long long x = unpack2(w4[e]);
+          ffma2(ss, x, x);
+#pragma unroll
+          for (int r = 0; r < RP; ++r) ffma2(acc[r], qv[r][4 * i + e], x);
         }
       }
+      float sc = -INFINITY, sq = hsum2(ss);
+#pragma unroll
+      for (int r = 0; r < RP; ++r) {
+        float t = hsum2(acc[r]);
+#pragma unroll
+        for (int o = LPP / 2; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+        if (r < R) sc = fmaxf(sc, t);
+      }
+#pragma unroll
+      for (int o = LPP / 2; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      if (fb == 0 && p < N) {
+        float2 out;
+        if (!cand) {
+          out = make_float2(NAN, NAN);
+        } else if (ph < 0) {
+          out = make_float2(-INFINITY, -INFINITY);   // an unreadable page never wins a slot
+        } else {
+          const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(sq, sq_pad)));
+          // + 0 turns -0 into +0 (the radix keys order -0 below +0)
+          out = make_float2(__fsub_rd(sc, E) + 0.f, __fadd_ru(sc, E) + 0.f);
+        }
+        outrow[p] = out;
+      }
     }
   }
-  float s = -INFINITY;
-#pragma unroll
-  for (int r = 0; r < kMaxRows; ++r)
-    if (r < R) s = fmaxf(s, acc[r]);
-  const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(ss, sq_pad)));
-  // + 0 turns -0 into +0 (the radix keys order -0 below +0)
-  *out = make_float2(__fsub_rd(s, E) + 0.f, __fadd_ru(s, E) + 0.f);
 }
 
 // Radix selection of the bounds, exact rescoring of the undecided pages, and
@@ -174,8 +251,8 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
 
   extern __shared__ __align__(16) uint8_t dsm[];
   __shared__ __align__(16) float q_s[kMaxRows * kMaxDk];
-  __shared__ uint32_t hist[512];
-  __shared__ uint32_t sel_out[4];
+  __shared__ uint32_t hist[1024];
+  __shared__ uint32_t sel_out[8];
   __shared__ float red_f[kThreads / 32];
   __shared__ int red_i[kThreads / 32];
   __shared__ int n_unc, n_certain;
@@ -295,8 +372,22 @@ size_t select_workspace_bytes(int B, int Hkv, int max_pages) {
 
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
   if (a.k_top > 0) {
-    dim3 g1((a.max_pages + kScoreThreads - 1) / kScoreThreads, a.Hkv, a.B);
-    score_kernel<<<g1, kScoreThreads, 0, stream>>>(a);
+    dim3 g1(a.Hkv, (a.max_pages + kScorePages - 1) / kScorePages, a.B);
+    const int R = a.T * (a.Hq / a.Hkv);
+    const int rp = R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : R <= 8 ? 8 : 16;
+    auto pick = [&](auto dk) {
+      constexpr int DK = decltype(dk)::value;
+      switch (rp) {
+        case 1: score_kernel<1, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
+        case 2: score_kernel<2, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
+        case 4: score_kernel<4, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
+        case 8: score_kernel<8, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
+        default: score_kernel<16, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
+      }
+    };
+    if (a.Dk == 64) pick(std::integral_constant<int, 64>{});
+    else if (a.Dk == 128) pick(std::integral_constant<int, 128>{});
+    else pick(std::integral_constant<int, 256>{});
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

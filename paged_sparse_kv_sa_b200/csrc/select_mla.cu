@@ -221,8 +221,8 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   float* hi = lo + a.max_pages;
   uint16_t* u_list = reinterpret_cast<uint16_t*>(hi + a.max_pages);
   uint8_t* flag = reinterpret_cast<uint8_t*>(u_list + a.max_pages);
-  __shared__ uint32_t hist[512];
-  __shared__ uint32_t sel_out[4];
+  __shared__ uint32_t hist[1024];
+  __shared__ uint32_t sel_out[8];
   __shared__ int red_i[kChooseThreads / 32];
   __shared__ int n_unc, n_cert[2];
   __shared__ double ex_tmp[kChooseThreads];

@@ -32,21 +32,37 @@ __device__ __forceinline__ double exact_dot_f32q(const float* q, const uint16_t*
 }
 
 // Radix-select the (k_lo)-th largest key of `lo` and the (k_hi)-th largest of
-// `hi` over n entries (1-based ranks; entries with key 0 never match).
+// `hi` over n entries (1-based ranks; NaN entries never match).  Four 8-bit
+// digit passes; the histograms and digit results are double-buffered so each
+// pass needs two block barriers.  hist: [2][512] words, shared_out: [2][4].
 SA_DEV void radix_select2(const float* lo, const float* hi, int n, int k_lo, int k_hi,
-                          uint32_t* hist /*[2][256]*/, uint32_t* shared_out /*[4]*/,
-                          float& out_lo, float& out_hi) {
+                          uint32_t* hist, uint32_t* shared_out, float& out_lo, float& out_hi) {
   uint32_t pre[2] = {0u, 0u}, msk[2] = {0u, 0u};
   int kk[2] = {k_lo, k_hi};
+  for (int i = threadIdx.x; i < 512; i += blockDim.x) hist[i] = 0u;
+  __syncthreads();
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 512; i += blockDim.x) hist[i] = 0u;
-    __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const float a = lo[i], c = hi[i];
-      const uint32_t ka = f2key(a), kc = f2key(c);
-      if (!isnan(a) && (ka & msk[0]) == pre[0]) atomicAdd(&hist[(ka >> shift) & 255u], 1u);
-      if (!isnan(c) && (kc & msk[1]) == pre[1]) atomicAdd(&hist[256 + ((kc >> shift) & 255u)], 1u);
+    uint32_t* h = hist + (pass & 1) * 512;
+    uint32_t* nxt = hist + ((pass + 1) & 1) * 512;
+    uint32_t* so = shared_out + (pass & 1) * 4;
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) nxt[i] = 0u;   // next pass's bins
+    // warp-aggregated increments: the keys crowd into a few top-digit bins,
+    // so lanes with equal bins add their count with one atomic
+    const int ln = threadIdx.x & 31;
+    for (int i0 = 0; i0 < n; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      uint32_t ba = 0xffffffffu, bc = 0xffffffffu;
+      if (i < n) {
+        const float a = lo[i], c = hi[i];
+        const uint32_t ka = f2key(a), kc = f2key(c);
+        if (!isnan(a) && (ka & msk[0]) == pre[0]) ba = (ka >> shift) & 255u;
+        if (!isnan(c) && (kc & msk[1]) == pre[1]) bc = 256u + ((kc >> shift) & 255u);
+      }
+      const uint32_t pa = __match_any_sync(0xffffffffu, ba);
+      const uint32_t pc = __match_any_sync(0xffffffffu, bc);
+      if (ba != 0xffffffffu && ln == __ffs(pa) - 1) atomicAdd(&h[ba], __popc(pa));
+      if (bc != 0xffffffffu && ln == __ffs(pc) - 1) atomicAdd(&h[bc], __popc(pc));
     }
     __syncthreads();
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -55,7 +71,7 @@ SA_DEV void radix_select2(const float* lo, const float* hi, int n, int k_lo, int
       uint32_t c8[8], tot = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        c8[j] = hist[w * 256 + 255 - (8 * lane + j)];
+        c8[j] = h[w * 256 + 255 - (8 * lane + j)];
         tot += c8[j];
       }
       uint32_t incl = tot;
@@ -64,14 +80,14 @@ SA_DEV void radix_select2(const float* lo, const float* hi, int n, int k_lo, int
         const uint32_t v = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += v;
       }
-      uint32_t before = incl - tot;   // count in higher bins than this lane's
+      const uint32_t before = incl - tot;   // count in higher bins than this lane's
       const uint32_t want = static_cast<uint32_t>(kk[w]);
       if (before < want && incl >= want) {
         uint32_t run = before;
         for (int j = 0; j < 8; ++j) {
           if (run + c8[j] >= want) {
-            shared_out[2 * w] = 255u - (8u * lane + j);
-            shared_out[2 * w + 1] = run;
+            so[2 * w] = 255u - (8u * lane + j);
+            so[2 * w + 1] = run;
             break;
           }
           run += c8[j];
@@ -80,17 +96,15 @@ SA_DEV void radix_select2(const float* lo, const float* hi, int n, int k_lo, int
     }
     __syncthreads();
 #pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      pre[s] |= shared_out[2 * s] << shift;
-      msk[s] |= 255u << shift;
-      kk[s] -= static_cast<int>(shared_out[2 * s + 1]);
+    for (int t = 0; t < 2; ++t) {
+      pre[t] |= so[2 * t] << shift;
+      msk[t] |= 255u << shift;
+      kk[t] -= static_cast<int>(so[2 * t + 1]);
     }
-    __syncthreads();
   }
+  __syncthreads();   // the buffers may be reused by the caller
   out_lo = key2f(pre[0]);
   out_hi = key2f(pre[1]);
 }
-
-
 
 }  // namespace sa

@@ -13,17 +13,20 @@ import torch
 from . import _lib
 
 
-def default_splits(n_units: int, max_list: int, sm_count: int = 148, ctas_per_sm: int = 3,
-                   warps_per_cta: int = 4, max_entries: int = 128) -> int:
+def default_splits(n_units: int, max_list: int, sm_count: int = None, warps_per_sm: int = 12,
+                   max_entries: int = 128) -> int:
     """Split count for ``n_units`` (sequence, list) pairs of up to ``max_list`` pages.
 
-    The decode kernel runs one split per warp, four warps per CTA, three CTAs per
-    SM; take as many whole CTAs per pair as fit in one wave, and at least enough
-    splits that none holds more than ``max_entries`` pages."""
+    The decode kernel runs one split per warp and keeps one wave of warps
+    resident (twelve per SM: three CTAs of four), striding over the flattened
+    (split, pair, sequence) items; take as many splits as fill that wave, and at
+    least enough that no split holds more than ``max_entries`` pages."""
     if n_units <= 0 or max_list <= 0:
         return 1
-    ctas = max(1, (ctas_per_sm * sm_count) // n_units)
-    n = warps_per_cta * ctas
+    if sm_count is None:
+        sm_count = (torch.cuda.get_device_properties(torch.cuda.current_device()).multi_processor_count
+                    if torch.cuda.is_available() else 148)
+    n = max(1, (warps_per_sm * sm_count) // n_units)
     n = min(n, max(1, max_list))
     while -(-max_list // n) > max_entries:
         n += 1
