@@ -10,8 +10,6 @@
 namespace sa {
 namespace {
 
-constexpr int kMaxSplitsCombine = 64;
-
 __global__ void __launch_bounds__(256)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    int n_splits, int64_t rows, int Dv, float* __restrict__ o_out,
@@ -27,21 +25,21 @@ __global__ void __launch_bounds__(256)
   float lse = -INFINITY;
   if (m != -INFINITY) {
     float tot = 0.f;
-    float w[kMaxSplitsCombine];
     for (int s = 0; s < n_splits; ++s) {
-      w[s] = __expf(lse_part[s * rows + row] - m);
-      tot += w[s];
+      const float w = __expf(lse_part[s * rows + row] - m);
+      tot += w;
+      if (w == 0.f) continue;
+      const float4 v = *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
     }
     const float inv = 1.f / tot;
-    for (int s = 0; s < n_splits; ++s) {
-      const float f = w[s] * inv;
-      if (f == 0.f) continue;
-      const float4 v = *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c);
-      acc.x += f * v.x;
-      acc.y += f * v.y;
-      acc.z += f * v.z;
-      acc.w += f * v.w;
-    }
+    acc.x *= inv;
+    acc.y *= inv;
+    acc.z *= inv;
+    acc.w *= inv;
     lse = m + logf(tot);
   }
   if (o_out) *reinterpret_cast<float4*>(o_out + row * Dv + c) = acc;
@@ -59,7 +57,6 @@ __global__ void __launch_bounds__(256)
 cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_splits, int64_t rows,
                            int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,
                            cudaStream_t stream) {
-  if (n_splits > kMaxSplitsCombine) return cudaErrorInvalidValue;
   const int64_t n = rows * (Dv / 4);
   if (n == 0) return cudaSuccess;
   const int threads = 256;

@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a
   const int G = a.Hq / a.Hkv, R = a.T * G, Dk = DK;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int fb = lane % LPP, slot = lane / LPP, pages_per_step = 32 / LPP;
-  const int f0 = fb * FPL;
+  // lane fb holds features [i*8*LPP + 8*fb, +8) for i < FPL/8: consecutive lanes
+  // read consecutive 16-byte pieces of a page row
   // query rows: FPL features each, as float32 pairs; row norms for the bound
   unsigned long long qv[RP][FPL / 2];
   float qn2 = 0.f;
@@ -136,7 +137,8 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a
       uint4 w = make_uint4(0, 0, 0, 0);
       if (r < R) {
         const int t = r / G, h = kvh * G + r % G;
-        w = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 + f0 + 8 * i);
+        w = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 +
+                                            i * 8 * LPP + 8 * fb);
       }
       const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -162,18 +164,18 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a
   // every page-table lookup, then every row load, so that they are in flight
   // together, then the arithmetic
   const int wp0 = p0 + warp * 32;
+  // the warp's 32 page-table entries in one coalesced load
+  const int pt_lane = wp0 + lane < N ? ptrow[wp0 + lane] : -1;
 #pragma unroll 1
   for (int sb = 0; sb < NSTEPS; sb += HOIST) {
     int phs[HOIST];
     uint4 v[HOIST][FPL / 8];
 #pragma unroll
     for (int k = 0; k < HOIST; ++k) {
-      phs[k] = -1;
       const int p = wp0 + (sb + k) * pages_per_step + slot;
-      if (p < N && p >= n_sink && p < local0) {
-        const int ph = ptrow[p];
-        phs[k] = (ph < 0 || ph >= a.P_pool) ? -2 : ph;
-      }
+      const int ph = __shfl_sync(0xffffffffu, pt_lane, (sb + k) * pages_per_step + slot);
+      phs[k] = -1;
+      if (p < N && p >= n_sink && p < local0) phs[k] = (ph < 0 || ph >= a.P_pool) ? -2 : ph;
     }
 #pragma unroll
     for (int k = 0; k < HOIST; ++k) {
@@ -181,9 +183,9 @@ __global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a
       for (int i = 0; i < FPL / 8; ++i) v[k][i] = make_uint4(0, 0, 0, 0);
       if (phs[k] >= 0) {
         const uint4* src =
-            reinterpret_cast<const uint4*>(a.sig + ((int64_t)phs[k] * a.Hkv + kvh) * Dk + f0);
+            reinterpret_cast<const uint4*>(a.sig + ((int64_t)phs[k] * a.Hkv + kvh) * Dk + 8 * fb);
 #pragma unroll
-        for (int i = 0; i < FPL / 8; ++i) v[k][i] = __ldcs(src + i);
+        for (int i = 0; i < FPL / 8; ++i) v[k][i] = __ldcs(src + i * LPP);
       }
     }
 #pragma unroll
