@@ -9,6 +9,7 @@
 // once to the nearest float64, ties to even.
 #pragma once
 
+#include <math.h>
 #include <stdint.h>
 
 namespace sa {
@@ -88,7 +89,7 @@ struct ExactAcc {
 };
 
 // Fields of one bf16 pattern: significand integer and the weight of its lsb.
-__device__ __forceinline__ void bf16_fields(uint32_t bits, uint32_t& m, int& e, bool& neg) {
+__host__ __device__ __forceinline__ void bf16_fields(uint32_t bits, uint32_t& m, int& e, bool& neg) {
   const uint32_t E = (bits >> 7) & 0xffu, F = bits & 0x7fu;
   neg = (bits >> 15) & 1u;
   m = E ? (128u + F) : F;
@@ -110,6 +111,156 @@ __device__ __forceinline__ double exact_dot_bf16(const uint16_t* a, int sa, cons
   }
   return acc.round_to_double();
 }
+
+// ---------------------------------------------------------------------------
+// Warp-cooperative exact dot product.
+//
+// In one dot product the product exponents usually span a few dozen bits, so
+// every product is an integer multiple of 2^emin (emin = the smallest product
+// exponent) below 2^(16 + span).  With span <= 100 and n <= 1024 terms, the
+// sum of those integers fits a signed 128-bit word: each lane accumulates its
+// products there, the lanes' words are added with xor shuffles, and the total
+// is rounded once to float64.  A wider span falls back to the superaccumulator
+// (one lane).
+
+// Two's complement 128-bit value hi:lo.
+struct I128 {
+  uint64_t lo, hi;
+};
+__host__ __device__ __forceinline__ void i128_add(I128& a, uint64_t blo, uint64_t bhi) {
+  const uint64_t lo = a.lo + blo;
+  a.hi = a.hi + bhi + (lo < a.lo ? 1ull : 0ull);
+  a.lo = lo;
+}
+__host__ __device__ __forceinline__ void i128_sub(I128& a, uint64_t blo, uint64_t bhi) {
+  const uint64_t lo = a.lo - blo;
+  a.hi = a.hi - bhi - (a.lo < blo ? 1ull : 0ull);
+  a.lo = lo;
+}
+// m << sh as a 128-bit word (sh in [0, 127], m < 2^16).
+__host__ __device__ __forceinline__ void shl128(uint64_t m, int sh, uint64_t& lo, uint64_t& hi) {
+  if (sh >= 64) {
+    lo = 0;
+    hi = m << (sh - 64);
+  } else {
+    lo = m << sh;
+    hi = sh ? m >> (64 - sh) : 0ull;
+  }
+}
+__host__ __device__ __forceinline__ int clz64(uint64_t x) {
+#ifdef __CUDA_ARCH__
+  return __clzll(static_cast<long long>(x));
+#else
+  return __builtin_clzll(x);
+#endif
+}
+// Nearest float64 (ties to even) to the integer hi:lo times 2^e0; the result
+// must be a normal float64.
+__host__ __device__ __forceinline__ double i128_to_double_rn(I128 v, int e0) {
+  const bool neg = static_cast<int64_t>(v.hi) < 0;
+  if (neg) {   // magnitude
+    v.lo = ~v.lo + 1ull;
+    v.hi = ~v.hi + (v.lo == 0 ? 1ull : 0ull);
+  }
+  if (v.hi == 0 && v.lo == 0) return 0.0;
+  const int msb = v.hi ? 127 - clz64(v.hi) : 63 - clz64(v.lo);
+  uint64_t mant;
+  int sh = 0;
+  if (msb <= 52) {
+    mant = v.lo;
+  } else {
+    sh = msb - 52;                       // bits dropped: 1 .. 75
+    // mant = v >> sh (53 bits)
+    if (sh >= 64) mant = v.hi >> (sh - 64);
+    else mant = (v.lo >> sh) | (v.hi << (64 - sh));
+    // round bit = bit sh - 1; sticky = any bit below it
+    const int rb = sh - 1;
+    const bool round = rb >= 64 ? ((v.hi >> (rb - 64)) & 1ull) : ((v.lo >> rb) & 1ull);
+    bool sticky;
+    if (rb == 0) sticky = false;
+    else if (rb < 64) sticky = (v.lo & ((1ull << rb) - 1ull)) != 0;
+    else if (rb == 64) sticky = v.lo != 0;
+    else sticky = v.lo != 0 || (v.hi & ((1ull << (rb - 64)) - 1ull)) != 0;
+    if (round && (sticky || (mant & 1ull))) {
+      ++mant;
+      if (mant == (1ull << 53)) {
+        mant >>= 1;
+        ++sh;
+      }
+    }
+  }
+  const double r = scalbn(static_cast<double>(mant), e0 + sh);
+  return neg ? -r : r;
+}
+
+#ifdef __CUDACC__
+// RN64(sum_d a[d] * b[d]) for two bf16 rows of n elements (n % 8 == 0, both
+// 16-byte aligned, n <= 1024), computed by all 32 lanes of a warp; every lane
+// returns the result.
+__device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const uint16_t* b, int n) {
+  const int lane = threadIdx.x & 31;
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  const uint4* b4 = reinterpret_cast<const uint4*>(b);
+  const int nc = n >> 3;
+  // pass 1: exponent range of the nonzero products
+  int emin = 1 << 20, emax = -(1 << 20);
+  for (int c = lane; c < nc; c += 32) {
+    const uint4 x = a4[c], y = b4[c];
+    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t ma, mb;
+      int ea, eb;
+      bool na, nb;
+      bf16_fields((xa[i >> 1] >> (16 * (i & 1))) & 0xffffu, ma, ea, na);
+      bf16_fields((ya[i >> 1] >> (16 * (i & 1))) & 0xffffu, mb, eb, nb);
+      if (ma && mb) {
+        emin = min(emin, ea + eb);
+        emax = max(emax, ea + eb);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+    emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+  }
+  if (emax < emin) return 0.0;          // every product is zero
+  if (emax - emin > 100) {              // wide span: superaccumulator, lane 0
+    double r = 0.0;
+    if (lane == 0) r = exact_dot_bf16(a, 1, b, n);
+    return __shfl_sync(0xffffffffu, r, 0);
+  }
+  // pass 2: fixed-point sums anchored at 2^emin
+  I128 acc{0ull, 0ull};
+  for (int c = lane; c < nc; c += 32) {
+    const uint4 x = a4[c], y = b4[c];
+    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t ma, mb;
+      int ea, eb;
+      bool na, nb;
+      bf16_fields((xa[i >> 1] >> (16 * (i & 1))) & 0xffffu, ma, ea, na);
+      bf16_fields((ya[i >> 1] >> (16 * (i & 1))) & 0xffffu, mb, eb, nb);
+      const uint32_t m = ma * mb;
+      if (m) {
+        uint64_t lo, hi;
+        shl128(m, ea + eb - emin, lo, hi);
+        if (na != nb) i128_sub(acc, lo, hi);
+        else i128_add(acc, lo, hi);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const uint64_t lo = __shfl_xor_sync(0xffffffffu, acc.lo, o);
+    const uint64_t hi = __shfl_xor_sync(0xffffffffu, acc.hi, o);
+    i128_add(acc, lo, hi);
+  }
+  return i128_to_double_rn(acc, emin);
+}
+#endif
 
 // Nearest bf16 to a float64 (ties to even), for |x| below the bf16 overflow
 // threshold.  Works on the binary64 fields: keep the top 8 significant bits

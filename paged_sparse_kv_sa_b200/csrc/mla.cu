@@ -57,9 +57,6 @@ struct __align__(64) MlaParams {
   PairTable pairs;
 };
 
-SA_DEV void mbar_arrive_m(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
 SA_DEV bool wait_or_abort_m(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -279,7 +276,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
       }
     }
     tc::fence_proxy_async();
-    mbar_arrive_m(&q_full);
+    mbar_arrive(&q_full);
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
@@ -353,7 +350,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();
-      mbar_arrive_m(&p_full[sb]);
+      mbar_arrive(&p_full[sb]);
     }
     if (ok && n_act > 0) ok = wait_or_abort_m(&o_done, (n_act - 1) & 1, abort_flag);
     tc::fence_after_sync();

@@ -61,10 +61,6 @@ struct __align__(64) PrefillParams {
   PairTable pairs;
 };
 
-SA_DEV void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Bounded wait that also gives up as soon as another role has aborted.
 SA_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   for (uint32_t i = 0; i < kSpinLimit; ++i) {

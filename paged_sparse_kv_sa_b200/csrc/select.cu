@@ -1,7 +1,8 @@
 // Page scoring and top-k selection (GQA), in two launches.
 //
-// score_kernel (one CTA per 256 pages of one (kv head, sequence), so every SM
-// streams summaries) and choose_kernel (one CTA per (kv head, sequence)):
+// score_kernel (one CTA per 128 pages of one sequence and a block of kv heads,
+// so every SM streams summaries) and choose_kernel (one CTA per (kv head,
+// sequence)):
 //
 // 1. Every candidate page (neither sink nor local) is scored in float32 with a
 //    fixed-order FMA chain per query row, and given a rigorous error bound
@@ -31,10 +32,9 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 512;       // choose_kernel
-constexpr int kScoreThreads = 128;  // score_kernel: 4 warps x 32 pages
-constexpr int kScorePages = 128;
-constexpr int kMaxRows = 16;
-constexpr int kMaxDk = 256;
+constexpr int kScoreChunk = 128;    // score_kernel: logical pages per CTA
+constexpr int kScoreStages = 2;     // ring slots of 16 pages
+constexpr int kScoreMaxHB = 8;      // kv heads per CTA (one consumer warp each)
 
 // Shared-memory layout (dynamic): lo[Nmax] f32, hi[Nmax] f32, u_list[Nmax] u16,
 // flag[Nmax] u8; q rows [R][Dk] f32 in static memory.
@@ -55,182 +55,233 @@ SA_DEV int clamped_len(const SelectArgs& a, int b, bool report) {
   return L;
 }
 
-// The group's query rows (t, h) as exact float32 copies in q_s[R][Dk]; returns
-// an upper bound on max_r ||q_r||_2.  Called by every thread of the block.
-SA_DEV float load_q_rows(const SelectArgs& a, int b, int kvh, float* q_s, float* red) {
-  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
-  for (int i = threadIdx.x; i < R * Dk; i += blockDim.x) {
-    const int r = i / Dk, d = i % Dk;
-    const int t = r / G, h = kvh * G + r % G;
-    q_s[i] = bf16_bits_to_float(a.q[b * a.qs0 + t * a.qs1 + h * a.qs2 + d]);
-  }
-  __syncthreads();
-  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  float qn = 0.f;
-  for (int r = w; r < R; r += nw) {
-    float ss = 0.f;
-    for (int d = lane; d < Dk; d += 32) ss = fmaf(q_s[r * Dk + d], q_s[r * Dk + d], ss);
-    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    qn = fmaxf(qn, ss);
-  }
-  if (lane == 0) red[w] = qn;
-  __syncthreads();
-  qn = 0.f;
-  for (int i = 0; i < nw; ++i) qn = fmaxf(qn, red[i]);
-  // the float32 sum of squares is within (1 + gamma_Dk) of the truth
-  return sqrtf(qn * (1.f + 2.f * Dk * 5.96046448e-8f)) * (1.f + 1.2e-7f);
-}
-
-SA_DEV void cp_async16(void* smem_dst, const void* gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc)
-               : "memory");
-}
-
-// Packed float32 FMA (two lanes of a 64-bit register pair, each rounded as
-// an ordinary fma.rn.f32).
-SA_DEV void ffma2(unsigned long long& acc, unsigned long long a, unsigned long long b) {
-  asm volatile("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-SA_DEV float hsum2(unsigned long long v) {
-  return __uint_as_float(static_cast<uint32_t>(v)) + __uint_as_float(static_cast<uint32_t>(v >> 32));
-}
-// bf16x2 word -> the two features as a float32 pair (low half first)
-SA_DEV unsigned long long unpack2(uint32_t w) {
-  return (static_cast<unsigned long long>(w & 0xffff0000u) << 32) |
-         static_cast<unsigned long long>(w << 16);
-}
-
 // lo/hi bounds of every candidate page's score; NaN for forced pages.
-// LPP = Dk / FPL lanes share a page, each holding FPL features of every query
-// row in registers; a warp scores 32 / LPP pages per step, reading each page
-// row as one coalesced run.  Per page a lane does FPL/2 packed FMAs per row
-// (two float32 lanes: even / odd features), then the row sums are reduced over
-// the LPP lanes with xor shuffles.  Any summation order obeys the bound
-// |fl(q.s) - q.s| <= gamma_Dk ||q|| ||s||, so the bracket stays rigorous.
-template <int RP, int DK>   // rows rounded up to a power of two; feature count
-__global__ void __launch_bounds__(kScoreThreads) score_kernel(const SelectArgs a) {
-  constexpr int FPL = RP <= 8 ? 16 : 8;            // features per lane
-  constexpr int LPP = DK / FPL;                    // lanes per page
-  constexpr int NSTEPS = LPP;                      // 32 pages / (32 / LPP) per step
-  constexpr int HOIST = NSTEPS < 8 ? NSTEPS : 8;   // pages steps loaded at once
-  // kv heads vary fastest across the grid: the CTAs reading the Hkv adjacent
-  // rows of the same pages run together and share DRAM pages / L2 lines
-  const int kvh = blockIdx.x, chunk = blockIdx.y, b = blockIdx.z;
+//
+// Data movement.  Summaries are stored [P_pool, Hkv, Dk], so the rows of
+// adjacent kv heads of one page form one contiguous run.  A CTA scores a chunk
+// of kScoreChunk logical pages of one sequence for a block of hb adjacent kv
+// heads (hb <= 8, hb * Dk * 2 <= 2 KB): warp hb (the producer) looks the pages
+// up in the page table and gathers each page's hb-head run with one bulk copy
+// into a ring of kScoreStages slots of 16 pages; warps 0 .. hb-1 (one per kv
+// head) score the slots.  Gathering whole runs instead of single 256-byte rows
+// matters: scattered 256-byte reads reach a fraction of HBM bandwidth.
+//
+// Arithmetic.  A slot's scores for one head are a (16 pages x Dk) by (Dk x R
+// rows) product, done with m16n8k16 bf16 warp MMAs (float32 accumulation),
+// which keeps the instruction count per page far below a float32 FMA loop.
+// Three products per tile:
+//   S = sigma q^T             the scores,
+//   T = |sigma| |q|^T          an upper bound of sum_d |q_d sigma_d| per row,
+//   U = |sigma| f^T            f_d = 2^-126 where q_d is subnormal, else 0
+//                              (only when the head's rows hold a subnormal).
+// Every bf16 x bf16 product is exact in float32.  The score bracket of row r is
+//   s_r -/+ E_r,  E_r = c_acc T_r + (1 + 2^-10) U_r + 2^-126 ||q_r||_1 + Dk 2^-124
+// with directed rounding.  c_acc T_r covers the rounding of the float32
+// accumulation (c_acc = Dk 2^-19: the accumulation of each 16-term step loses
+// less than 2^-17.8 of the running magnitude sum, which leaves a margin of
+// 7x); U_r covers subnormal q_d flushed to zero inside the MMA, 2^-126
+// ||q_r||_1 the same for sigma_d, and Dk 2^-124 any product that underflows
+// float32.  A page's bracket is [max_r (s_r - E_r), max_r (s_r + E_r)].
+template <int NT, int DK>   // 8-row tiles of query rows (R <= 8 NT); feature count
+__global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const SelectArgs a, int hb) {
+  constexpr int KS = DK / 16;                      // k-steps
+  constexpr int ROWB = DK * 2;                     // bytes per summary row
+  constexpr int QS = ROWB + 16;                    // padded query-row stride
+  constexpr int QROWS = 8 * NT;
+  const int rec = hb * ROWB;                       // bytes per page run
+  const int RSB = rec + 16;                        // padded slot-row stride
+  extern __shared__ __align__(128) uint8_t score_smem[];
+  uint8_t* q_s = score_smem;                                 // [hb][QROWS][QS]
+  uint8_t* ring = score_smem + hb * QROWS * QS;              // [stages][16][RSB]
+  __shared__ uint64_t full[kScoreStages], empty[kScoreStages];
+  __shared__ int8_t stat_s[kScoreStages][16];   // per slot page: 1 scored, 0 forced, -1 bad
+  __shared__ float qn1_s[kScoreMaxHB][QROWS];
+  __shared__ int sub_s[kScoreMaxHB];
+  const int chunk = blockIdx.x, hblk = blockIdx.y, b = blockIdx.z;
   const int L = clamped_len(a, b, false);
   const int N = (L + a.P - 1) / a.P;
   if (N <= a.budget_pages || a.k_top == 0) return;   // no ranking needed
-  const int p0 = chunk * kScorePages;
+  const int p0 = chunk * kScoreChunk;
   if (p0 >= N) return;
-  const int G = a.Hq / a.Hkv, R = a.T * G, Dk = DK;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int fb = lane % LPP, slot = lane / LPP, pages_per_step = 32 / LPP;
-  // lane fb holds features [i*8*LPP + 8*fb, +8) for i < FPL/8: consecutive lanes
-  // read consecutive 16-byte pieces of a page row
-  // query rows: FPL features each, as float32 pairs; row norms for the bound
-  unsigned long long qv[RP][FPL / 2];
-  float qn2 = 0.f;
-#pragma unroll
-  for (int r = 0; r < RP; ++r) {
-    float part = 0.f;
-#pragma unroll
-    for (int i = 0; i < FPL / 8; ++i) {
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (r < R) {
-        const int t = r / G, h = kvh * G + r % G;
-        w = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 +
-                                            i * 8 * LPP + 8 * fb);
-      }
-      const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qv[r][4 * i + e] = unpack2(w4[e]);
-        const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
-        part = fmaf(x0, x0, fmaf(x1, x1, part));
-      }
-    }
-#pragma unroll
-    for (int o = LPP / 2; o; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-    qn2 = fmaxf(qn2, part);
-  }
-  const float nu = Dk * 5.96046448e-8f;
-  // the float32 sums of squares are within (1 + gamma_Dk) of the truth
-  const float qn = sqrtf(qn2 * (1.f + 2.f * nu)) * (1.f + 1.2e-7f);
-  const float gfac = nu / (1.f - nu) * 1.0001f * qn * 1.0001f;
-  const float sq_pad = 1.f + 2.f * nu;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = a.Hq / a.Hkv, R = a.T * G, h0 = hblk * hb;
+  const int n_groups = (min(kScoreChunk, N - p0) + 15) / 16;
   const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
-  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
-  float2* outrow = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
-  // this warp's 32 pages, pages_per_step at a time, HOIST steps per batch: first
-  // every page-table lookup, then every row load, so that they are in flight
-  // together, then the arithmetic
-  const int wp0 = p0 + warp * 32;
-  // the warp's 32 page-table entries in one coalesced load
-  const int pt_lane = wp0 + lane < N ? ptrow[wp0 + lane] : -1;
-#pragma unroll 1
-  for (int sb = 0; sb < NSTEPS; sb += HOIST) {
-    int phs[HOIST];
-    uint4 v[HOIST][FPL / 8];
-#pragma unroll
-    for (int k = 0; k < HOIST; ++k) {
-      const int p = wp0 + (sb + k) * pages_per_step + slot;
-      const int ph = __shfl_sync(0xffffffffu, pt_lane, (sb + k) * pages_per_step + slot);
-      phs[k] = -1;
-      if (p < N && p >= n_sink && p < local0) phs[k] = (ph < 0 || ph >= a.P_pool) ? -2 : ph;
+  if (tid == 0) {
+    for (int s = 0; s < kScoreStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], hb);
     }
+    fence_mbar_init();
+  }
+  // query rows of the block's heads, zero past R; 16-byte pieces
+  for (int i = tid; i < hb * QROWS * (ROWB / 16); i += blockDim.x) {
+    const int piece = i % (ROWB / 16), r = (i / (ROWB / 16)) % QROWS, w = i / (QROWS * (ROWB / 16));
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < R) {
+      const int t = r / G, h = (h0 + w) * G + r % G;
+      v = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 + piece * 8);
+    }
+    *reinterpret_cast<uint4*>(q_s + (w * QROWS + r) * QS + piece * 16) = v;
+  }
+  // per head: ||q_r||_1 (rounded up) and whether any row element is subnormal
+  for (int w = warp; w < hb; w += blockDim.x / 32) {
+    int sub = 0;
+    for (int r = 0; r < QROWS; ++r) {
+      float s1 = 0.f;
+      if (r < R) {
+        const int t = r / G, h = (h0 + w) * G + r % G;
+        const uint16_t* qr = a.q + b * a.qs0 + t * a.qs1 + h * a.qs2;
+        for (int d = lane; d < DK; d += 32) {
+          const uint32_t x = qr[d];
+          s1 += fabsf(bf16_bits_to_float(x));
+          sub |= ((x & 0x7f80u) == 0 && (x & 0x7fu) != 0);
+        }
 #pragma unroll
-    for (int k = 0; k < HOIST; ++k) {
-#pragma unroll
-      for (int i = 0; i < FPL / 8; ++i) v[k][i] = make_uint4(0, 0, 0, 0);
-      if (phs[k] >= 0) {
-        const uint4* src =
-            reinterpret_cast<const uint4*>(a.sig + ((int64_t)phs[k] * a.Hkv + kvh) * Dk + 8 * fb);
-#pragma unroll
-        for (int i = 0; i < FPL / 8; ++i) v[k][i] = __ldcs(src + i * LPP);
+        for (int o = 16; o; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
       }
+      if (lane == 0) qn1_s[w][r] = s1 * (1.f + DK * 1.2e-7f);
     }
+    sub = __any_sync(0xffffffffu, sub);
+    if (lane == 0) sub_s[w] = sub;
+  }
+  __syncthreads();
+
+  if (warp == hb) {
+    // ================= producer: page-table lookups and bulk gathers
+    const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+    int ph_r[kScoreChunk / 32];
 #pragma unroll
-    for (int k = 0; k < HOIST; ++k) {
-      const int p = wp0 + (sb + k) * pages_per_step + slot;
+    for (int i = 0; i < kScoreChunk / 32; ++i) {
+      const int p = p0 + 32 * i + lane;
+      ph_r[i] = (p < N && p >= n_sink && p < local0) ? ptrow[p] : -1;
+    }
+    for (int g = 0; g < n_groups; ++g) {
+      const int st = g % kScoreStages;
+      if (g >= kScoreStages &&
+          !mbar_wait_bounded(&empty[st], ((g / kScoreStages) - 1) & 1)) {
+        if (lane == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+        break;
+      }
+      int phx = -1;
+#pragma unroll
+      for (int i = 0; i < kScoreChunk / 32; ++i)
+        if (i == (g >> 1)) phx = ph_r[i];
+      const int j = lane & 15;                       // page of the slot
+      const int p = p0 + 16 * g + j;
+      const int ph = __shfl_sync(0xffffffffu, phx, 16 * (g & 1) + j);
       const bool cand = p < N && p >= n_sink && p < local0;
-      const int ph = phs[k];
-      if (ph == -2 && fb == 0) set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
-      unsigned long long acc[RP], ss = 0ull;
+      const bool ok = cand && ph >= 0 && ph < a.P_pool;
+      const int st8 = ok ? 1 : (cand ? -1 : 0);
+      const uint32_t m = __ballot_sync(0xffffffffu, ok && lane < 16);
+      if (lane < 16) stat_s[st][j] = static_cast<int8_t>(st8);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[st], __popc(m) * rec);
+      __syncwarp();
+      if (lane < 16 && ok)
+        bulk_load(ring + (st * 16 + j) * RSB, a.sig + ((int64_t)ph * a.Hkv + h0) * DK, rec,
+                  &full[st]);
+    }
+  } else if (warp < hb) {
+    // ================= consumers: one kv head each
+    const int kvh = h0 + warp;
+    const bool sub = sub_s[warp] != 0;
+    constexpr float c_acc = DK * 1.9073486328125e-06f;   // Dk * 2^-19
+    constexpr float e_abs = DK * 4.70197740328915e-38f;  // Dk * 2^-124
+    float2* outrow = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
+    const int gq = lane >> 2, cq = lane & 3;           // fragment row / column pair
+    float fl[NT][2];                                   // per fragment column: 2^-126 ||q_r||_1
 #pragma unroll
-      for (int r = 0; r < RP; ++r) acc[r] = 0ull;
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-      for (int i = 0; i < FPL / 8; ++i) {
-        const uint32_t w4[4] = {v[k][i].x, v[k][i].y, v[k][i].z, v[k][i].w};
+      for (int i = 0; i < 2; ++i) fl[nt][i] = qn1_s[warp][nt * 8 + 2 * cq + i] * 1.1754943508222875e-38f;
+    // ldmatrix addresses: A rows = slot pages (lane & 15), k + 8 (lane >> 4);
+    // B rows = query rows (lane & 7), k + 8 ((lane >> 3) & 1)
+    const uint32_t a_off = (lane & 15) * RSB + warp * ROWB + 16 * (lane >> 4);
+    const uint32_t b_base = smem_u32(q_s + (warp * QROWS + (lane & 7)) * QS + 16 * ((lane >> 3) & 1));
+    const uint32_t ring_u = smem_u32(ring);
+    for (int g = 0; g < n_groups; ++g) {
+      const int st = g % kScoreStages;
+      if (!mbar_wait_bounded(&full[st], (g / kScoreStages) & 1)) {
+        if (lane == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+        break;
+      }
+      float acc[3][NT][4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const unsigned long long x = unpack2(w4[e]);
-          ffma2(ss, x, x);
+      for (int x = 0; x < 3; ++x)
 #pragma unroll
-          for (int r = 0; r < RP; ++r) ffma2(acc[r], qv[r][4 * i + e], x);
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[x][nt][i] = 0.f;
+      const uint32_t a_addr = ring_u + st * 16 * RSB + a_off;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t af[4], aa[4];
+        ldmatrix_x4(af, a_addr + ks * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) aa[i] = af[i] & 0x7fff7fffu;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t bq[2];
+          ldmatrix_x2(bq, b_base + nt * 8 * QS + ks * 32);
+          mma_bf16_16816(acc[0][nt], af, bq[0], bq[1]);
+          mma_bf16_16816(acc[1][nt], aa, bq[0] & 0x7fff7fffu, bq[1] & 0x7fff7fffu);
+          if (sub) {
+            uint32_t bf[2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint32_t x = bq[i];
+              const bool s0 = (x & 0x7f80u) == 0 && (x & 0x7fu) != 0;
+              const bool s1 = (x & 0x7f800000u) == 0 && (x & 0x7f0000u) != 0;
+              bf[i] = (s0 ? 0x0080u : 0u) | (s1 ? 0x00800000u : 0u);
+            }
+            mma_bf16_16816(acc[2][nt], aa, bf[0], bf[1]);
+          }
         }
       }
-      float sc = -INFINITY, sq = hsum2(ss);
+      // epilogue: this lane holds pages gq (i = 0, 1) and gq + 8 (i = 2, 3),
+      // query rows 8 nt + 2 cq + (i & 1)
+      float lo[2] = {-INFINITY, -INFINITY}, hi[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int r = 0; r < RP; ++r) {
-        float t = hsum2(acc[r]);
+      for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int o = LPP / 2; o; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-        if (r < R) sc = fmaxf(sc, t);
-      }
-#pragma unroll
-      for (int o = LPP / 2; o; o >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      if (fb == 0 && p < N) {
-        float2 out;
-        if (!cand) {
-          out = make_float2(NAN, NAN);
-        } else if (ph < 0) {
-          out = make_float2(-INFINITY, -INFINITY);   // an unreadable page never wins a slot
-        } else {
-          const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(sq, sq_pad)));
-          // + 0 turns -0 into +0 (the radix keys order -0 below +0)
-          out = make_float2(__fsub_rd(sc, E) + 0.f, __fadd_ru(sc, E) + 0.f);
+        for (int i = 0; i < 4; ++i) {
+          const int r = nt * 8 + 2 * cq + (i & 1);
+          if (r < R) {
+            const float E = __fadd_ru(__fadd_ru(__fmul_ru(c_acc, acc[1][nt][i]),
+                                                __fmul_ru(1.0009765625f, acc[2][nt][i])),
+                                      __fadd_ru(fl[nt][i & 1], e_abs));
+            const float sv = acc[0][nt][i];
+            lo[i >> 1] = fmaxf(lo[i >> 1], __fsub_rd(sv, E));
+            hi[i >> 1] = fmaxf(hi[i >> 1], __fadd_ru(sv, E));
+          }
         }
-        outrow[p] = out;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int o = 1; o <= 2; o <<= 1) {
+          lo[h] = fmaxf(lo[h], __shfl_xor_sync(0xffffffffu, lo[h], o));
+          hi[h] = fmaxf(hi[h], __shfl_xor_sync(0xffffffffu, hi[h], o));
+        }
+        const int j = gq + 8 * h;
+        const int p = p0 + 16 * g + j;
+        if (cq == 0 && p < N) {
+          const int stv = stat_s[st][j];
+          float2 out;
+          if (stv == 0) {
+            out = make_float2(NAN, NAN);
+          } else if (stv < 0) {
+            set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
+            out = make_float2(-INFINITY, -INFINITY);   // an unreadable page never wins a slot
+          } else {
+            // + 0 turns -0 into +0 (the radix keys order -0 below +0)
+            out = make_float2(lo[h] + 0.f, hi[h] + 0.f);
+          }
+          outrow[p] = out;
+        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
     }
   }
 }
@@ -252,10 +303,9 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   }
 
   extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ __align__(16) float q_s[kMaxRows * kMaxDk];
   __shared__ uint32_t hist[1024];
   __shared__ uint32_t sel_out[8];
-  __shared__ float red_f[kThreads / 32];
+  __shared__ SelScratch scratch;
   __shared__ int red_i[kThreads / 32];
   __shared__ int n_unc, n_certain;
   __shared__ double ex_tmp[kThreads];
@@ -285,7 +335,8 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
 
   // ---- order statistics of the bounds (k == 0: streaming, no winners)
   float Lk = INFINITY, H = INFINITY;
-  if (k > 0) radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
+  if (k > 0 && !filtered_select2(S.lo, S.hi, N, k, k + 1, &scratch, Lk, H))
+    radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
 
   // ---- classify: certainly in (lo > H), undecided (hi >= Lk), else out
   for (int p = tid; p < N; p += blockDim.x) {
@@ -306,19 +357,24 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   double* ex = reinterpret_cast<double*>(S.lo);
   const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
   if (nu_ > 0 && slots > 0) {
-    load_q_rows(a, b, kvh, q_s, red_f);
-    const int per = max(1, kThreads / R);            // undecided pages per batch
+    // one warp per (page, query row): exact dot, then the max over the rows
+    const int nw = kThreads / 32, warp = tid >> 5, lane = tid & 31;
+    const int per = max(1, kThreads / R);            // undecided pages per round
     for (int u0 = 0; u0 < nu_; u0 += per) {
-      const int u = u0 + tid / R, r = tid % R;
-      if (tid < per * R && u < nu_) {
-        const int ph = ptrow[S.u_list[u]];
-        ex_tmp[tid] = (ph < 0 || ph >= a.P_pool)
-                          ? -INFINITY
-                          : exact_dot_f32q(&q_s[r * Dk],
-                                           a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk, Dk);
+      const int np = min(per, nu_ - u0);
+      for (int pr = warp; pr < np * R; pr += nw) {
+        const int r = pr % R;
+        const int ph = ptrow[S.u_list[u0 + pr / R]];
+        double e = -INFINITY;
+        if (ph >= 0 && ph < a.P_pool) {
+          const int t = r / G, h = kvh * G + r % G;
+          e = warp_exact_dot_bf16(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2,
+                                  a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk, Dk);
+        }
+        if (lane == 0) ex_tmp[pr] = e;
       }
       __syncthreads();
-      if (tid < per && u0 + tid < nu_) {
+      if (tid < np) {
         double m = -INFINITY;
         for (int rr = 0; rr < R; ++rr) m = fmax(m, ex_tmp[tid * R + rr]);
         ex[u0 + tid] = m;
@@ -374,18 +430,22 @@ size_t select_workspace_bytes(int B, int Hkv, int max_pages) {
 
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
   if (a.k_top > 0) {
-    dim3 g1(a.Hkv, (a.max_pages + kScorePages - 1) / kScorePages, a.B);
+    // kv-head block: the largest divisor of Hkv with hb <= 8 and an hb-head
+    // run of at most 2 KB
+    int hb = 1;
+    for (int d = 1; d <= kScoreMaxHB && d <= a.Hkv; ++d)
+      if (a.Hkv % d == 0 && d * a.Dk * 2 <= 2048) hb = d;
+    dim3 g1((a.max_pages + kScoreChunk - 1) / kScoreChunk, a.Hkv / hb, a.B);
     const int R = a.T * (a.Hq / a.Hkv);
-    const int rp = R <= 1 ? 1 : R <= 2 ? 2 : R <= 4 ? 4 : R <= 8 ? 8 : 16;
     auto pick = [&](auto dk) {
       constexpr int DK = decltype(dk)::value;
-      switch (rp) {
-        case 1: score_kernel<1, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
-        case 2: score_kernel<2, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
-        case 4: score_kernel<4, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
-        case 8: score_kernel<8, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
-        default: score_kernel<16, DK><<<g1, kScoreThreads, 0, stream>>>(a); break;
-      }
+      auto launch = [&](auto kern, int nt) {
+        const int dyn = hb * 8 * nt * (DK * 2 + 16) + kScoreStages * 16 * (hb * DK * 2 + 16);
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        kern<<<g1, (hb + 1) * 32, dyn, stream>>>(a, hb);
+      };
+      if (R <= 8) launch(score_kernel<1, DK>, 1);
+      else launch(score_kernel<2, DK>, 2);
     };
     if (a.Dk == 64) pick(std::integral_constant<int, 64>{});
     else if (a.Dk == 128) pick(std::integral_constant<int, 128>{});

@@ -223,9 +223,11 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   uint8_t* flag = reinterpret_cast<uint8_t*>(u_list + a.max_pages);
   __shared__ uint32_t hist[1024];
   __shared__ uint32_t sel_out[8];
+  __shared__ SelScratch scratch;
   __shared__ int red_i[kChooseThreads / 32];
   __shared__ int n_unc, n_cert[2];
-  __shared__ double ex_tmp[kChooseThreads];
+  __shared__ uint32_t mlo_s[kChooseThreads];
+  __shared__ unsigned long long best_s[kChooseThreads];
   const int R = a.T * a.Hq;
   const int kb[2] = {min(a.alpha, N), min(a.alpha + a.beta, N)};
   // flag bits: 1 / 2 = in tier boundary 0 / 1, 4 / 8 = undecided for it
@@ -253,7 +255,8 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     }
     if (kb[i] == 0) continue;
     float Lk, H;
-    radix_select2(lo, hi, N, kb[i], kb[i] + 1, hist, sel_out, Lk, H);
+    if (!filtered_select2(lo, hi, N, kb[i], kb[i] + 1, &scratch, Lk, H))
+      radix_select2(lo, hi, N, kb[i], kb[i] + 1, hist, sel_out, Lk, H);
     for (int p = tid; p < N; p += blockDim.x) {
       if (lo[p] > H) {
         flag[p] |= in_bit;
@@ -268,31 +271,42 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   const int nu_ = n_unc;
   double* ex = reinterpret_cast<double*>(lo);   // lo/hi storage reused as doubles
   if (nu_ > 0) {
-    // exact row-max scores of the undecided pages: `per` pages per round, the
-    // block's threads split evenly over them, each thread over a stride of rows
-    const int per = max(1, min(nu_, kChooseThreads / 32));
-    const int tpp = kChooseThreads / per;               // threads per page
+    // exact row-max scores of the undecided pages, up to 512 pages per round.
+    // Pass 1: a float32 bracket of every (page, row) score, one warp each; per
+    // page the largest lower end m.  Pass 2: only rows whose upper end reaches
+    // m can hold the page's maximum (the row that attains the exact maximum
+    // has exact score >= m); those rows are rescored exactly.
     const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
-    for (int u0 = 0; u0 < nu_; u0 += per) {
-      const int slot = tid / tpp, rt = tid % tpp;
-      const int u = u0 + slot;
-      double m = -INFINITY;
-      if (slot < per && u < nu_) {
-        const int ph = ptrow[u_list[u]];
-        if (ph >= 0 && ph < a.P_pool) {
-          for (int r = rt; r < R; r += tpp) {
-            const int t = r / a.Hq, h = r % a.Hq;
-            m = fmax(m, exact_dot_bf16(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2, 1,
-                                       a.sig + (int64_t)ph * a.Dk, a.Dk));
+    const int nw = kChooseThreads / 32, warp = tid >> 5, lane = tid & 31;
+    for (int u0 = 0; u0 < nu_; u0 += kChooseThreads) {
+      const int np = min(kChooseThreads, nu_ - u0);
+      for (int i = tid; i < np; i += blockDim.x) {
+        mlo_s[i] = 0u;
+        best_s[i] = 0ull;
+      }
+      __syncthreads();
+      const int64_t n_pairs = (int64_t)np * R;
+      for (int pass = 0; pass < 2; ++pass) {
+        for (int64_t pr = warp; pr < n_pairs; pr += nw) {
+          const int uu = static_cast<int>(pr / R), r = static_cast<int>(pr % R);
+          const int ph = ptrow[u_list[u0 + uu]];
+          if (ph < 0 || ph >= a.P_pool) continue;
+          const int t = r / a.Hq, h = r % a.Hq;
+          const uint16_t* qr = a.q + b * a.qs0 + t * a.qs1 + h * a.qs2;
+          const uint16_t* sg = a.sig + (int64_t)ph * a.Dk;
+          const float2 br = warp_score_bracket(qr, sg, a.Dk);
+          if (pass == 0) {
+            if (lane == 0) atomicMax(&mlo_s[uu], f2key(br.x));
+          } else if (br.y >= key2f(mlo_s[uu])) {
+            const double e = warp_exact_dot_bf16(qr, sg, a.Dk);
+            if (lane == 0) atomicMax(&best_s[uu], d2key(e));
           }
         }
+        __syncthreads();
       }
-      ex_tmp[tid] = m;
-      __syncthreads();
-      if (tid < per && u0 + tid < nu_) {
-        double mm = -INFINITY;
-        for (int i = 0; i < tpp; ++i) mm = fmax(mm, ex_tmp[tid * tpp + i]);
-        ex[u0 + tid] = mm;
+      for (int i = tid; i < np; i += blockDim.x) {
+        const int ph = ptrow[u_list[u0 + i]];
+        ex[u0 + i] = (ph < 0 || ph >= a.P_pool) ? -INFINITY : key2d(best_s[i]);
       }
       __syncthreads();
     }

@@ -1,6 +1,6 @@
-// Shared pieces of the page selectors: order-preserving float keys, a
-// two-sequence radix select over shared memory, and exact float64 scores of a
-// query row held as float32 copies of bf16 values.
+// Shared pieces of the page selectors: order-preserving float / double keys,
+// a warp-wide rigorous float32 score bracket, and a two-sequence radix select
+// over shared memory.
 #pragma once
 
 #include "common.cuh"
@@ -16,19 +16,148 @@ SA_DEV float key2f(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-// RN64(q . sigma) for a query row held as float32 copies of bf16 values.
-__device__ __forceinline__ double exact_dot_f32q(const float* q, const uint16_t* sig, int n) {
-  ExactAcc acc;
-  acc.clear();
-  for (int d = 0; d < n; ++d) {
-    uint32_t ma, mb;
-    int ea, eb;
-    bool na, nb;
-    bf16_fields(__float_as_uint(q[d]) >> 16, ma, ea, na);
-    bf16_fields(sig[d], mb, eb, nb);
-    acc.add(ma * mb, ea + eb, na != nb);
+// Order-preserving 64-bit key of a float64 (larger key = larger value; -0 < +0).
+SA_DEV unsigned long long d2key(double x) {
+  const unsigned long long b = static_cast<unsigned long long>(__double_as_longlong(x));
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+SA_DEV double key2d(unsigned long long k) {
+  return __longlong_as_double(
+      static_cast<long long>((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+// A rigorous float32 bracket [lo, hi] of the exact q . sigma for two bf16 rows
+// of n elements (n % 8 == 0, both 16-byte aligned), computed by a whole warp;
+// every lane returns it.  Each product of two bf16 values is exact in float32
+// and every term passes through at most n roundings on its way to the total,
+// so |fl(q.s) - q.s| <= gamma_n sum |q_d s_d| <= gamma_n ||q|| ||s||.
+SA_DEV float2 warp_score_bracket(const uint16_t* q, const uint16_t* sg, int n) {
+  const int lane = threadIdx.x & 31;
+  const uint4* q4 = reinterpret_cast<const uint4*>(q);
+  const uint4* s4 = reinterpret_cast<const uint4*>(sg);
+  float s = 0.f, qq = 0.f, ss = 0.f;
+  for (int c = lane; c < (n >> 3); c += 32) {
+    const uint4 x = q4[c], y = s4[c];
+    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float x0 = __uint_as_float(xa[e] << 16), x1 = __uint_as_float(xa[e] & 0xffff0000u);
+      const float y0 = __uint_as_float(ya[e] << 16), y1 = __uint_as_float(ya[e] & 0xffff0000u);
+      s = fmaf(x0, y0, s);
+      s = fmaf(x1, y1, s);
+      qq = fmaf(x0, x0, fmaf(x1, x1, qq));
+      ss = fmaf(y0, y0, fmaf(y1, y1, ss));
+    }
   }
-  return acc.round_to_double();
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    s += __shfl_xor_sync(0xffffffffu, s, o);
+    qq += __shfl_xor_sync(0xffffffffu, qq, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  }
+  const float nu = n * 5.96046448e-8f;
+  // the float32 sums of squares are within (1 + gamma_n) of the truth
+  const float qn = sqrtf(qq * (1.f + 2.f * nu)) * (1.f + 1.2e-7f);
+  const float gfac = nu / (1.f - nu) * 1.0001f * qn * 1.0001f;
+  const float E = __fmul_ru(gfac, __fsqrt_ru(__fmul_ru(ss, 1.f + 2.f * nu)));
+  return make_float2(__fsub_rd(s, E) + 0.f, __fadd_ru(s, E) + 0.f);
+}
+
+// Workspace of filtered_select2 (shared memory).
+constexpr int kSelGroupsMax = 512;   // n <= 32 * kSelGroupsMax
+constexpr int kSelCap = 1024;        // candidates kept per sequence
+struct SelScratch {
+  float glo[kSelGroupsMax], ghi[kSelGroupsMax];   // per 32-entry group: max lo / hi
+  float clo[kSelCap], chi[kSelCap];               // entries at or above the thresholds
+  int cnt[2];
+  float tau[2], res[2];
+};
+
+// The (k_lo)-th largest of lo[0, n) and the (k_hi)-th largest of hi[0, n)
+// (1-based ranks; NaN entries never count), by thresholding: the k-th largest
+// of the 32-entry group maxima is a lower bound of the k-th largest entry (k
+// distinct entries reach it), so every entry at or above the k-th largest
+// entry is kept by the filter entry >= that bound; the answer is then ranked
+// among the kept entries only.  Returns false (results unset) when n exceeds
+// 32 * kSelGroupsMax or more than kSelCap entries pass a filter.  Called by
+// every thread of the block.
+SA_DEV bool filtered_select2(const float* lo, const float* hi, int n, int k_lo, int k_hi,
+                             SelScratch* sc, float& out_lo, float& out_hi) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int ng = (n + 31) >> 5;
+  if (ng > kSelGroupsMax) return false;
+  for (int gi = warp; gi < ng; gi += nw) {
+    const int i = gi * 32 + lane;
+    float a = i < n ? lo[i] : -INFINITY, c = i < n ? hi[i] : -INFINITY;
+    a = isnan(a) ? -INFINITY : a;
+    c = isnan(c) ? -INFINITY : c;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
+    }
+    if (lane == 0) {
+      sc->glo[gi] = a;
+      sc->ghi[gi] = c;
+    }
+  }
+  if (tid == 0) {
+    sc->cnt[0] = sc->cnt[1] = 0;
+    sc->tau[0] = sc->tau[1] = -INFINITY;   // fewer groups than k: keep everything
+    sc->res[0] = sc->res[1] = -INFINITY;
+  }
+  __syncthreads();
+  // thresholds: the k-th largest group maximum (g values above, e equal:
+  // g < k <= g + e)
+  for (int x = tid; x < 2 * ng; x += blockDim.x) {
+    const int w = x >= ng;
+    const float* arr = w ? sc->ghi : sc->glo;
+    const int kk = w ? k_hi : k_lo;
+    if (ng < kk) continue;
+    const float v = arr[x - w * ng];
+    int g = 0, e = 0;
+    for (int y = 0; y < ng; ++y) {
+      g += arr[y] > v;
+      e += arr[y] == v;
+    }
+    if (g < kk && g + e >= kk) sc->tau[w] = v;
+  }
+  __syncthreads();
+  const float t_lo = sc->tau[0], t_hi = sc->tau[1];
+  for (int i = tid; i < n; i += blockDim.x) {
+    const float a = lo[i], c = hi[i];
+    if (a >= t_lo) {
+      const int sl = atomicAdd(&sc->cnt[0], 1);
+      if (sl < kSelCap) sc->clo[sl] = a;
+    }
+    if (c >= t_hi) {
+      const int sl = atomicAdd(&sc->cnt[1], 1);
+      if (sl < kSelCap) sc->chi[sl] = c;
+    }
+  }
+  __syncthreads();
+  const int c0 = sc->cnt[0], c1 = sc->cnt[1];
+  if (c0 > kSelCap || c1 > kSelCap) {
+    __syncthreads();
+    return false;
+  }
+  for (int x = tid; x < c0 + c1; x += blockDim.x) {
+    const int w = x >= c0;
+    const float* arr = w ? sc->chi : sc->clo;
+    const int cn = w ? c1 : c0, kk = w ? k_hi : k_lo;
+    const float v = arr[x - w * c0];
+    int g = 0, e = 0;
+    for (int y = 0; y < cn; ++y) {
+      g += arr[y] > v;
+      e += arr[y] == v;
+    }
+    if (g < kk && g + e >= kk) sc->res[w] = v;
+  }
+  __syncthreads();
+  out_lo = sc->res[0];
+  out_hi = sc->res[1];
+  __syncthreads();   // the scratch may be reused by the caller
+  return true;
 }
 
 // Radix-select the (k_lo)-th largest key of `lo` and the (k_hi)-th largest of

@@ -151,6 +151,81 @@ def test_select_ties_and_cancellation():
     assert list(rp[0, 0, :12]) == list(range(12))   # ties -> lowest pages after the 2 sinks
 
 
+def test_select_long_all_ties():
+    # one long sequence whose scores all tie (q = 0): more equal candidates than
+    # the selector's threshold filter keeps, so its radix path decides; the
+    # winners are the lowest candidate pages
+    cfg = W.scaled(W.TINY_GQA, B=2, seq_len_lo=40000, seq_len_hi=40000)
+    inp, g = gqa_case(cfg, seed=6)
+    sig = oracle_summaries(inp, cfg)
+    qb = bits(inp["q"]).copy()
+    qb[1] = 0
+    g["q"] = to_bf16_dev(qb)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(qb, sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+    n_sink, _, _, k = O.page_budget(cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens,
+                                    cfg.page_size)
+    assert list(rp[1, 0, :n_sink + k]) == list(range(n_sink + k))
+
+
+def _random_bf16_bits(rng, shape, e_lo, e_hi, p_sub=0.03, p_zero=0.03):
+    """bf16 bit patterns: random sign and fraction, exponent field uniform in
+    [e_lo, e_hi]; a share of subnormals and zeros."""
+    sign = rng.integers(0, 2, shape, dtype=np.uint16) << 15
+    frac = rng.integers(0, 128, shape, dtype=np.uint16)
+    expo = rng.integers(e_lo, e_hi + 1, shape, dtype=np.uint16)
+    out = sign | (expo << 7) | frac
+    u = rng.random(shape)
+    out = np.where(u < p_sub, sign | np.maximum(frac, 1).astype(np.uint16), out)
+    out = np.where((u >= p_sub) & (u < p_sub + p_zero), sign, out)
+    return out.astype(np.uint16)
+
+
+@pytest.mark.parametrize("T,Hq,Hkv", [(1, 8, 2), (2, 16, 2)])
+def test_select_score_brackets_hold(T, Hq, Hkv):
+    # The selector's per-page score brackets (its workspace) must contain the
+    # exact row-max score for every candidate page, on inputs with a wide
+    # exponent range, subnormals and zeros; the selection must equal the oracle's.
+    cfg = W.scaled(W.TINY_GQA, B=2, T=T, Hq=Hq, Hkv=Hkv, D=128)
+    inp, g = gqa_case(cfg, seed=11)
+    rng = np.random.default_rng(11)
+    pt = np_i32(inp["page_table"])
+    sl = np_i32(inp["seq_lens"])
+    qb = _random_bf16_bits(rng, tuple(inp["q"].shape), 112, 136)
+    sig = _random_bf16_bits(rng, (int(pt.max()) + 1, Hkv, cfg.D), 100, 146)
+    g["q"] = to_bf16_dev(qb)
+    max_pages = pt.shape[1]
+    ws = torch.zeros(sa.sa_select_workspace_size(cfg.B, Hkv, max_pages), dtype=torch.uint8,
+                     device=DEV)
+    pages, counts = sa.sa_select_pages(g["q"], to_bf16_dev(sig), g["page_table"], g["seq_lens"],
+                                       cfg.page_size, cfg.sink_tokens, cfg.local_tokens,
+                                       cfg.budget_tokens, workspace=ws)
+    torch.cuda.synchronize()
+    lohi = ws.view(torch.float32).cpu().numpy().reshape(cfg.B, Hkv, max_pages, 2).astype(np.float64)
+    n_sink, n_local, budget_pages, _ = O.page_budget(cfg.sink_tokens, cfg.local_tokens,
+                                                     cfg.budget_tokens, cfg.page_size)
+    q = O.bf16_to_f64(qb)
+    G = Hq // Hkv
+    checked = 0
+    for b in range(cfg.B):
+        nb = -(-int(sl[b]) // cfg.page_size)
+        cand = np.arange(n_sink, nb - n_local)
+        for kvh in range(Hkv):
+            rows = q[b, :, kvh * G:(kvh + 1) * G, :].reshape(T * G, cfg.D)
+            ex = O.page_scores(rows, O.bf16_to_f64(sig[pt[b, cand], kvh, :]))
+            lo, hi = lohi[b, kvh, cand, 0], lohi[b, kvh, cand, 1]
+            assert np.all(lo <= ex) and np.all(ex <= hi), "score bracket misses the exact score"
+            checked += len(cand)
+    assert checked > 0
+    rp, rc = O.select_pages(qb, sig, pt, sl, cfg.page_size, cfg.sink_tokens, cfg.local_tokens,
+                            cfg.budget_tokens)
+    np.testing.assert_array_equal(np_i32(counts), rc)
+    np.testing.assert_array_equal(np_i32(pages), rp)
+
+
 def test_select_streaming_k0():
     cfg = W.scaled(W.TINY_GQA, budget_tokens=96)    # 2 sink + 4 local, no top-k
     inp, g = gqa_case(cfg, seed=5)
