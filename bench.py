@@ -240,7 +240,7 @@ def run_extra(args, dev, world, rank, local, cores):
         counts = torch.empty((cfg.B, 2), dtype=torch.int32, device=dev)
         ws = torch.empty(max(int(sa.load().sa_select_tiered_workspace_size(
             cfg.B, cfg.T, cfg.Hq, pt.shape[1])), 16), dtype=torch.uint8, device=dev)
-        n_splits = args.splits or 4
+        n_splits = args.splits or 8
         o_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
         l_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
         o = torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)

@@ -187,9 +187,11 @@ SA_API size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_page
  * page p in lists[b,l,0:list_counts[b,l]] whose position p*P + j is below
  * seq_lens[b] and at most seq_lens[b] - T + t (query token t sits at that
  * position: causal MTP / chunked prefill).  s_j = scale * q.k_j; natural-log
- * LSE.  The list is cut into n_splits contiguous pieces of
- * ceil(count/n_splits) entries; split s writes its own normalised output
- * and LSE (an empty split writes O = 0, LSE = -inf).  With n_splits == 1
+ * LSE.  Split s takes the entries [s*c, (s+1)*c) of the list with
+ * c = ceil(max_list/n_splits) (so a short list leaves its last splits empty)
+ * and writes its own normalised output and LSE.  A split without a visible
+ * key writes LSE = -inf; its O rows are 0 when n_splits == 1 and otherwise
+ * unspecified (sa_combine gives such a split no weight).  With n_splits == 1
  * the partials are the final result; otherwise pass them to sa_combine.
  *
  *  q            (dev) [B,T,Hq,Dk] bf16, strides q_strides
@@ -210,6 +212,8 @@ SA_API size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_page
  *    128-row tiles on tcgen05 with TMEM accumulators;
  *  - MLA, Dk == 576 with Dv == 512 and v_cache == k_cache (same strides: the
  *    values are the first 512 key columns): 64-row tiles on tcgen05.
+ * Limits: Hq <= 256, at most 64 (list, kv head) pairs read by some head, at
+ * most 128 heads per pair (SA_ERR_UNSUPPORTED beyond).
  * Pool rows past a sequence's end are read with the page but masked; they
  * must hold finite values (a NaN there could reach the output through 0*NaN).
  */
@@ -224,7 +228,8 @@ SA_API int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const
 
 /*
  * sa_combine — merge split partials: lse = log sum_s exp(lse_s),
- * O = sum_s exp(lse_s - lse) O_s; splits with lse_s = -inf weigh nothing;
+ * O = sum_s exp(lse_s - lse) O_s; splits with lse_s = -inf weigh nothing
+ * (their O rows are not used, whatever they hold);
  * rows whose splits are all empty give O = 0, lse = -inf.
  *
  *  o_partial  (dev) [n_splits,rows,Dv] float32;  lse_partial (dev) [n_splits,rows]

@@ -250,10 +250,11 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
 
   // (list, kv head) pairs and the heads that read them
+  if (Hq > kMaxHeads) return SA_ERR_UNSUPPORTED;
   PairTable pairs;
   pairs.n_pairs = 0;
   const int G = Hq / Hkv;
-  int max_rows = 0;
+  int pair_of[kMaxHeads];
   for (int kvh = 0; kvh < Hkv; ++kvh) {
     for (int h = kvh * G; h < (kvh + 1) * G; ++h) {
       const int l = head_to_list[h];
@@ -268,9 +269,20 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
         pairs.n_heads[pi] = 0;
       }
       if (pairs.n_heads[pi] == kMaxHeadsPerPair) return SA_ERR_UNSUPPORTED;
-      pairs.heads[pi][pairs.n_heads[pi]++] = static_cast<int16_t>(h);
-      max_rows = max_rows > pairs.n_heads[pi] * T ? max_rows : pairs.n_heads[pi] * T;
+      ++pairs.n_heads[pi];
+      pair_of[h] = pi;
     }
+  }
+  int max_rows = 0;
+  for (int i = 0, off = 0; i < pairs.n_pairs; ++i) {
+    pairs.head_off[i] = off;
+    off += pairs.n_heads[i];
+    max_rows = max_rows > pairs.n_heads[i] * T ? max_rows : pairs.n_heads[i] * T;
+    pairs.n_heads[i] = 0;   // refilled below, in head order
+  }
+  for (int h = 0; h < Hq; ++h) {
+    const int pi = pair_of[h];
+    pairs.heads[pairs.head_off[pi] + pairs.n_heads[pi]++] = static_cast<int16_t>(h);
   }
   // Up to 16 query rows per pair: warp-MMA decode; more: the tcgen05 kernel.
   const bool wide = max_rows > kMaxRowsPerPair;

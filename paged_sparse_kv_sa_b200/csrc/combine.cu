@@ -17,6 +17,7 @@ __global__ void __launch_bounds__(128)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    int n_splits, int64_t rows, int Dv, float* __restrict__ o_out,
                    uint16_t* __restrict__ o_bf16, float* __restrict__ lse_out) {
+  pdl_wait_and_release();
   const int q4 = Dv / 4;
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= rows * q4) return;
@@ -88,9 +89,8 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
   if (n == 0) return cudaSuccess;
   const int threads = 128;
   const int64_t blocks = (n + threads - 1) / threads;
-  combine_kernel<<<(unsigned)blocks, threads, 0, stream>>>(o_part, lse_part, n_splits, rows, Dv,
-                                                           o_out, o_bf16, lse_out);
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, o_part,
+                    lse_part, n_splits, rows, Dv, o_out, o_bf16, lse_out);
 }
 
 }  // namespace sa

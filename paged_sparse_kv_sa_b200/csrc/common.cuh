@@ -76,6 +76,17 @@ SA_DEV void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+// Plain bulk copy shared -> global (both 16-byte aligned, bytes % 16 == 0),
+// tracked by this thread's bulk async-groups.
+SA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                   reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+SA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every bulk store this thread committed has completed.
+SA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 SA_DEV void prefetch_tmap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -117,6 +128,15 @@ SA_DEV float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16
 // XOR-ed with (row mod 8).  `col` < 64.
 SA_DEV uint32_t swz128(int row, int col) {
   return static_cast<uint32_t>(row * 128 + ((((col >> 3) ^ row) & 7) << 4) + ((col & 7) << 1));
+}
+
+// Programmatic dependent launch: wait until the preceding kernel of the stream
+// has completed and its writes are visible (a no-op when this kernel was not
+// launched as a dependent), then allow the next kernel to begin launching so
+// that its launch overlaps this kernel's tail.  Called first by every kernel.
+SA_DEV void pdl_wait_and_release() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 SA_DEV void set_dev_error(int32_t* err, int bits) {

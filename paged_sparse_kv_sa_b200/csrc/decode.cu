@@ -57,6 +57,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     decode_gqa_kernel(const __grid_constant__ DecodeParams prm,
                       const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap) {
+  pdl_wait_and_release();
   using C = DecodeCfg<D>;
   const DecodeArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -102,7 +103,8 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     if (lane == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
     count = count < 0 ? 0 : a.max_list;
   }
-  const int chunk = (count + a.n_splits - 1) / a.n_splits;
+  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(max_list / n_splits)
+  const int chunk = (a.max_list + a.n_splits - 1) / a.n_splits;
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
 
@@ -165,7 +167,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     for (int h = 0; h < 2; ++h) {
       const int r = rows[h];
       if (r < R) {
-        const int t = r / nh, head = prm.pairs.heads[pair][r % nh];
+        const int t = r / nh, head = prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)];
         qp[h] = a.q + b * a.qs0 + t * a.qs1 + head * a.qs2;
         lim[h] = L - a.T + t;
       } else {
@@ -313,7 +315,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   for (int h = 0; h < 2; ++h) {
     const int r = gid + 8 * h;
     if (r >= R) continue;
-    const int t = r / nh, head = prm.pairs.heads[pair][r % nh];
+    const int t = r / nh, head = prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)];
     const int64_t row = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
     const bool empty = l_run[h] == 0.f;
     const float inv = empty ? 0.f : 1.f / l_run[h];
@@ -350,8 +352,8 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   const long long items = (long long)a.n_splits * pairs.n_pairs * a.B;
   const long long want = (items + kNW - 1) / kNW;
   const int grid = (int)std::min<long long>(want, (long long)std::max(1, per_sm) * sms);
-  decode_gqa_kernel<D><<<grid, kNW * 32, C::kDynBytes, stream>>>(prm, kmap, vmap);
-  return cudaGetLastError();
+  return launch_pdl(decode_gqa_kernel<D>, grid, dim3(kNW * 32), C::kDynBytes, stream, prm, kmap,
+                    vmap);
 }
 
 }  // namespace

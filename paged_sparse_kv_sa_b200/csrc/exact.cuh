@@ -195,18 +195,27 @@ __host__ __device__ __forceinline__ double i128_to_double_rn(I128 v, int e0) {
 
 #ifdef __CUDACC__
 // RN64(sum_d a[d] * b[d]) for two bf16 rows of n elements (n % 8 == 0, both
-// 16-byte aligned, n <= 1024), computed by all 32 lanes of a warp; every lane
-// returns the result.
+// 16-byte aligned, n <= 256 kMaxC), computed by all 32 lanes of a warp (each
+// loads its 16-byte chunks once); every lane returns the result.
+template <int kMaxC>   // 16-byte chunks per lane: n <= 256 kMaxC
 __device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const uint16_t* b, int n) {
   const int lane = threadIdx.x & 31;
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
   const uint4* b4 = reinterpret_cast<const uint4*>(b);
   const int nc = n >> 3;
+  uint4 xs[kMaxC], ys[kMaxC];
+#pragma unroll
+  for (int j = 0; j < kMaxC; ++j) {
+    const int c = lane + 32 * j;
+    xs[j] = c < nc ? a4[c] : make_uint4(0, 0, 0, 0);
+    ys[j] = c < nc ? b4[c] : make_uint4(0, 0, 0, 0);
+  }
   // pass 1: exponent range of the nonzero products
   int emin = 1 << 20, emax = -(1 << 20);
-  for (int c = lane; c < nc; c += 32) {
-    const uint4 x = a4[c], y = b4[c];
-    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int j = 0; j < kMaxC; ++j) {
+    const uint32_t xa[4] = {xs[j].x, xs[j].y, xs[j].z, xs[j].w};
+    const uint32_t ya[4] = {ys[j].x, ys[j].y, ys[j].z, ys[j].w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       uint32_t ma, mb;
@@ -233,9 +242,10 @@ __device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const u
   }
   // pass 2: fixed-point sums anchored at 2^emin
   I128 acc{0ull, 0ull};
-  for (int c = lane; c < nc; c += 32) {
-    const uint4 x = a4[c], y = b4[c];
-    const uint32_t xa[4] = {x.x, x.y, x.z, x.w}, ya[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int j = 0; j < kMaxC; ++j) {
+    const uint32_t xa[4] = {xs[j].x, xs[j].y, xs[j].z, xs[j].w};
+    const uint32_t ya[4] = {ys[j].x, ys[j].y, ys[j].z, ys[j].w};
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       uint32_t ma, mb;

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillParams prm,
                    const __grid_constant__ CUtensorMap kmap,
                    const __grid_constant__ CUtensorMap vmap) {
+  pdl_wait_and_release();
   using C = PCfg<D>;
   const DecodeArgs& a = prm.a;
   const int pair = blockIdx.y, b = blockIdx.z;
@@ -126,7 +127,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (tid == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
     count = count < 0 ? 0 : a.max_list;
   }
-  const int chunk = (count + a.n_splits - 1) / a.n_splits;
+  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(max_list / n_splits)
+  const int chunk = (a.max_list + a.n_splits - 1) / a.n_splits;
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
   const int r0 = qt * kRows;
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int nr = min(kRows, rows_total - r0);
     for (int i = tid; i < nr * (D / 4); i += blockDim.x) {
       const int rr = r0 + i / (D / 4), c = (i % (D / 4)) * 4;
-      const int t = rr / nh, head = prm.pairs.heads[pair][rr % nh];
+      const int t = rr / nh, head = prm.pairs.heads[prm.pairs.head_off[pair] + (rr % nh)];
       const int64_t orow = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
       *reinterpret_cast<float4*>(a.o_part + orow * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
       if (c == 0) a.lse_part[orow] = -INFINITY;
@@ -289,7 +291,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const int rg = r0 + wg * kM + r;
     const bool row_ok = rg < rows_total;
     const int t = row_ok ? rg / nh : 0;
-    const int head = prm.pairs.heads[pair][row_ok ? rg % nh : 0];
+    const int head = prm.pairs.heads[prm.pairs.head_off[pair] + (row_ok ? rg % nh : 0)];
     const int qpos = row_ok ? L - a.T + t : -1;
     uint8_t* qt_s = q_s + wg * C::kQBytes;
     {
@@ -434,8 +436,7 @@ cudaError_t launch_p(const DecodeArgs& a, const PairTable& pairs, const CUtensor
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDyn);
   if (e != cudaSuccess) return e;
   dim3 grid(qtiles * a.n_splits, pairs.n_pairs, a.B);
-  prefill_kernel<D><<<grid, kPThreads, C::kDyn, stream>>>(prm, kmap, vmap);
-  return cudaGetLastError();
+  return launch_pdl(prefill_kernel<D>, grid, dim3(kPThreads), C::kDyn, stream, prm, kmap, vmap);
 }
 
 }  // namespace

@@ -84,6 +84,7 @@ SA_DEV int clamped_len(const SelectArgs& a, int b, bool report) {
 // float32.  A page's bracket is [max_r (s_r - E_r), max_r (s_r + E_r)].
 template <int NT, int DK>   // 8-row tiles of query rows (R <= 8 NT); feature count
 __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const SelectArgs a, int hb) {
+  pdl_wait_and_release();
   constexpr int KS = DK / 16;                      // k-steps
   constexpr int ROWB = DK * 2;                     // bytes per summary row
   constexpr int QS = ROWB + 16;                    // padded query-row stride
@@ -289,6 +290,7 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
 // Radix selection of the bounds, exact rescoring of the undecided pages, and
 // the ascending output of forced + selected pages.
 __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
+  pdl_wait_and_release();
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x;
   const int L = clamped_len(a, b, tid == 0);
@@ -350,12 +352,13 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
     }
   }
   __syncthreads();
+  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+
   const int nu_ = n_unc;
   const int slots = k - n_certain;
 
   // ---- exact scores of the undecided pages (lo/hi storage reused as doubles)
   double* ex = reinterpret_cast<double*>(S.lo);
-  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
   if (nu_ > 0 && slots > 0) {
     // one warp per (page, query row): exact dot, then the max over the rows
     const int nw = kThreads / 32, warp = tid >> 5, lane = tid & 31;
@@ -368,7 +371,7 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
         double e = -INFINITY;
         if (ph >= 0 && ph < a.P_pool) {
           const int t = r / G, h = kvh * G + r % G;
-          e = warp_exact_dot_bf16(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2,
+          e = warp_exact_dot_bf16<1>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2,
                                   a.sig + ((int64_t)ph * a.Hkv + kvh) * Dk, Dk);
         }
         if (lane == 0) ex_tmp[pr] = e;
@@ -441,24 +444,22 @@ cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
       constexpr int DK = decltype(dk)::value;
       auto launch = [&](auto kern, int nt) {
         const int dyn = hb * 8 * nt * (DK * 2 + 16) + kScoreStages * 16 * (hb * DK * 2 + 16);
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
-        kern<<<g1, (hb + 1) * 32, dyn, stream>>>(a, hb);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, g1, dim3((hb + 1) * 32), dyn, stream, a, hb);
       };
-      if (R <= 8) launch(score_kernel<1, DK>, 1);
-      else launch(score_kernel<2, DK>, 2);
+      return R <= 8 ? launch(score_kernel<1, DK>, 1) : launch(score_kernel<2, DK>, 2);
     };
-    if (a.Dk == 64) pick(std::integral_constant<int, 64>{});
-    else if (a.Dk == 128) pick(std::integral_constant<int, 128>{});
-    else pick(std::integral_constant<int, 256>{});
-    cudaError_t e = cudaGetLastError();
+    const cudaError_t e = a.Dk == 64    ? pick(std::integral_constant<int, 64>{})
+                          : a.Dk == 128 ? pick(std::integral_constant<int, 128>{})
+                                        : pick(std::integral_constant<int, 256>{});
     if (e != cudaSuccess) return e;
   }
   const size_t dyn = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
   cudaError_t e = cudaFuncSetAttribute(choose_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
   if (e != cudaSuccess) return e;
-  choose_kernel<<<dim3(a.Hkv, a.B), kThreads, dyn, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(choose_kernel, dim3(a.Hkv, a.B), dim3(kThreads), dyn, stream, a);
 }
 
 

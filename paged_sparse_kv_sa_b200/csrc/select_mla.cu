@@ -35,6 +35,7 @@ constexpr int kPad = 4;            // float padding per staged row (bank spread)
 constexpr int kChooseThreads = 512;
 
 __global__ void __launch_bounds__(256) tiered_score_kernel(const TieredArgs a) {
+  pdl_wait_and_release();
   const int pc = blockIdx.x, rg = blockIdx.y, b = blockIdx.z;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) L = L < 0 ? 0 : a.max_pages * a.P;
@@ -205,7 +206,14 @@ SA_DEV int compact_pages(const uint8_t* flag, int N, uint8_t bit, int32_t* out, 
   return min(total, cap);
 }
 
+// Out of line: the exact dot needs many registers, and inlined it would raise
+// the register count (and spills) of the whole choose kernel.
+__device__ __noinline__ double exact_row_dot(const uint16_t* q, const uint16_t* sg, int n) {
+  return warp_exact_dot_bf16<4>(q, sg, n);
+}
+
 __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const TieredArgs a) {
+  pdl_wait_and_release();
   const int b = blockIdx.x, tid = threadIdx.x;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) {
@@ -298,7 +306,7 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
           if (pass == 0) {
             if (lane == 0) atomicMax(&mlo_s[uu], f2key(br.x));
           } else if (br.y >= key2f(mlo_s[uu])) {
-            const double e = warp_exact_dot_bf16(qr, sg, a.Dk);
+            const double e = exact_row_dot(qr, sg, a.Dk);
             if (lane == 0) atomicMax(&best_s[uu], d2key(e));
           }
         }
@@ -352,15 +360,13 @@ cudaError_t launch_select_tiered(TieredArgs a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, dyn1);
   if (e != cudaSuccess) return e;
   dim3 g1((a.max_pages + kTP - 1) / kTP, a.n_rg, a.B);
-  tiered_score_kernel<<<g1, 256, dyn1, stream>>>(a);
-  e = cudaGetLastError();
+  e = launch_pdl(tiered_score_kernel, g1, dim3(256), dyn1, stream, a);
   if (e != cudaSuccess) return e;
   const size_t dyn2 = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
   e = cudaFuncSetAttribute(tiered_choose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn2);
   if (e != cudaSuccess) return e;
-  tiered_choose_kernel<<<a.B, kChooseThreads, dyn2, stream>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(tiered_choose_kernel, dim3(a.B), dim3(kChooseThreads), dyn2, stream, a);
 }
 
 }  // namespace sa

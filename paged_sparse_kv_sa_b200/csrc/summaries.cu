@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(256)
                      const int32_t* __restrict__ pt, int max_pages,
                      const int32_t* __restrict__ seq_lens, int Hkv, int Dk, int P, int P_pool,
                      uint16_t* __restrict__ sig, int32_t* err) {
+  pdl_wait_and_release();
   const int p = blockIdx.x, b = blockIdx.y;
   const int L = min(seq_lens[b], max_pages * P);
   const int n = min(P, L - p * P);
@@ -69,9 +70,8 @@ cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32
                              int P, int P_pool, uint16_t* sig, int32_t* err, cudaStream_t stream) {
   if (B == 0 || max_pages == 0) return cudaSuccess;
   dim3 grid(max_pages, B);
-  summaries_kernel<<<grid, 256, 0, stream>>>(k, ks[0], ks[1], ks[2], pt, max_pages, seq_lens, Hkv,
-                                             Dk, P, P_pool, sig, err);
-  return cudaGetLastError();
+  return launch_pdl(summaries_kernel, grid, dim3(256), 0, stream, k, ks[0], ks[1], ks[2], pt,
+                    max_pages, seq_lens, Hkv, Dk, P, P_pool, sig, err);
 }
 
 }  // namespace sa

@@ -26,6 +26,7 @@ SA_DEV uint32_t f2key_u(float x) {
 }
 
 __global__ void union_clear_kernel(int32_t* tables, int64_t n) {
+  pdl_wait_and_release();
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
     tables[i] = 0;
@@ -34,6 +35,7 @@ __global__ void union_clear_kernel(int32_t* tables, int64_t n) {
 __global__ void __launch_bounds__(kUThreads)
     union_mark_kernel(const float* __restrict__ scores, int Hq, int Hkv, int NQB, int NKB,
                       int q_off, int top_k, int n_sink, int32_t* tables) {
+  pdl_wait_and_release();
   const int j = blockIdx.x, h = blockIdx.y;
   const int g = h / (Hq / Hkv);
   const int d = q_off + j;
@@ -75,6 +77,7 @@ __global__ void __launch_bounds__(kUThreads)
 
 __global__ void __launch_bounds__(kUThreads)
     union_compact_kernel(int32_t* tables, int32_t* counts, int NKB) {
+  pdl_wait_and_release();
   const int g = blockIdx.x;
   int32_t* row = tables + (int64_t)g * NKB;
   extern __shared__ uint8_t fl[];   // [NKB]
@@ -112,21 +115,20 @@ cudaError_t launch_block_union(const float* scores, int Hq, int Hkv, int NQB, in
                                cudaStream_t stream) {
   if (NKB > kMaxBlocks) return cudaErrorInvalidValue;
   const int64_t n = (int64_t)Hkv * NKB;
-  union_clear_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(tables, n);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e =
+      launch_pdl(union_clear_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream, tables, n);
   if (e != cudaSuccess) return e;
   const size_t kbytes = sizeof(unsigned long long) * (size_t)NKB;
   e = cudaFuncSetAttribute(union_mark_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kbytes);
   if (e != cudaSuccess) return e;
   if (NQB > 0) {
-    union_mark_kernel<<<dim3(NQB, Hq), kUThreads, kbytes, stream>>>(scores, Hq, Hkv, NQB, NKB,
-                                                                    q_off, top_k, n_sink, tables);
-    e = cudaGetLastError();
+    e = launch_pdl(union_mark_kernel, dim3(NQB, Hq), dim3(kUThreads), kbytes, stream, scores, Hq,
+                   Hkv, NQB, NKB, q_off, top_k, n_sink, tables);
     if (e != cudaSuccess) return e;
   }
-  union_compact_kernel<<<Hkv, kUThreads, NKB, stream>>>(tables, counts, NKB);
-  return cudaGetLastError();
+  return launch_pdl(union_compact_kernel, dim3(Hkv), dim3(kUThreads), NKB, stream, tables, counts,
+                    NKB);
 }
 
 }  // namespace sa
