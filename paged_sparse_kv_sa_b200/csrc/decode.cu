@@ -91,28 +91,42 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   const int kvh = prm.pairs.kvh_of[pair];
   const int nh = prm.pairs.n_heads[pair];
   const int R = a.T * nh;
+  // The loads that depend on nothing but the item go out together: the
+  // sequence length, the list count and the split's list entries (read up to
+  // the split's capacity; only those below the count are used).  The
+  // page-table lookups follow in a second round, the query fragments after
+  // the first key/value gathers are issued.
+  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(max_list / n_splits)
+  const int chunk = (a.max_list + a.n_splits - 1) / a.n_splits;
+  const int s0 = split * chunk;
+  const int32_t* lbase = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list;
+  int pre[kWarpEntries / 32];
+#pragma unroll
+  for (int j = 0; j < kWarpEntries / 32; ++j) {
+    const int i = lane + 32 * j;
+    pre[j] = (i < chunk && s0 + i < a.max_list) ? lbase[s0 + i] : -1;
+  }
   int L = a.seq_lens[b];
+  int count = a.counts[b * a.n_lists + list];
   if (L < 0 || L > a.max_pages * a.P) {  // a length the page table cannot hold
     if (lane == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
     L = L < 0 ? 0 : a.max_pages * a.P;
   }
   const int n_log = (L + a.P - 1) / a.P;
-
-  int count = a.counts[b * a.n_lists + list];
   if (count < 0 || count > a.max_list) {
     if (lane == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
     count = count < 0 ? 0 : a.max_list;
   }
-  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(max_list / n_splits)
-  const int chunk = (a.max_list + a.n_splits - 1) / a.n_splits;
-  const int e0 = min(split * chunk, count);
+  const int e0 = min(s0, count);
   const int n_ent = min(chunk, count - e0);
 
-  // Resolve logical -> physical pages of this split (32 entries per round).
-  const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
+  // Resolve logical -> physical pages of this split.
   const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
-  for (int i = lane; i < n_ent; i += 32) {
-    const int p = lrow[i];
+#pragma unroll
+  for (int j = 0; j < kWarpEntries / 32; ++j) {
+    const int i = lane + 32 * j;
+    if (i >= n_ent) continue;
+    const int p = pre[j];
     int ph = -1;
     if (p < 0 || p >= n_log) {
       set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
@@ -159,21 +173,17 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
 
   // Query fragments (A operand of QK^T), rows r = t * nh + i.
   uint32_t qa[D / 16][4];
-  int lim[2];
+  int qt_[2];
   {
     const int rows[2] = {gid, gid + 8};
     const uint16_t* qp[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int r = rows[h];
-      if (r < R) {
-        const int t = r / nh, head = prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)];
-        qp[h] = a.q + b * a.qs0 + t * a.qs1 + head * a.qs2;
-        lim[h] = L - a.T + t;
-      } else {
-        qp[h] = nullptr;
-        lim[h] = -1;
-      }
+      qt_[h] = r < R ? r / nh : -1;
+      qp[h] = r < R ? a.q + b * a.qs0 + qt_[h] * a.qs1 +
+                          prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)] * a.qs2
+                    : nullptr;
     }
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -184,6 +194,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
       qa[kk][3] = qp[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + c + 8) : 0u;
     }
   }
+  const int lim[2] = {qt_[0] >= 0 ? L - a.T + qt_[0] : -1, qt_[1] >= 0 ? L - a.T + qt_[1] : -1};
 
   float o[D / 8][4];
 #pragma unroll

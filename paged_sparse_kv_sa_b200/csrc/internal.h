@@ -111,7 +111,10 @@ struct TieredArgs {
   const int32_t* seq_lens;
   int B, T, Hq, Dk, P, max_pages, P_pool, alpha, beta;
   int n_rg;                  // query-row groups of the scoring pass (set by the launcher)
-  float2* lohi;              // workspace [B, n_rg, max_pages]
+  float2* lohi;              // workspace [B, n_rg, max_pages] score brackets
+  unsigned long long* rmask; // workspace [B, n_rg, max_pages] candidate rows (set by the launcher)
+  unsigned long long* exkey; // workspace [B, max_pages] exact scores (order keys)
+  unsigned int* counter;     // workspace [B] CTAs done with the exact rescoring
   int32_t* lists;            // [B, 2, alpha + beta]
   int32_t* counts;           // [B, 2]
   int32_t* err;

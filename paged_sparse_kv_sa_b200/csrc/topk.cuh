@@ -75,30 +75,36 @@ struct SelScratch {
 
 // The (k_lo)-th largest of lo[0, n) and the (k_hi)-th largest of hi[0, n)
 // (1-based ranks; NaN entries never count), by thresholding: the k-th largest
-// of the 32-entry group maxima is a lower bound of the k-th largest entry (k
-// distinct entries reach it), so every entry at or above the k-th largest
-// entry is kept by the filter entry >= that bound; the answer is then ranked
-// among the kept entries only.  Returns false (results unset) when n exceeds
-// 32 * kSelGroupsMax or more than kSelCap entries pass a filter.  Called by
-// every thread of the block.
+// of the group maxima (groups of gs consecutive entries) is a lower bound of
+// the k-th largest entry (k distinct entries reach it), so every entry at or
+// above the k-th largest entry is kept by the filter entry >= that bound; the
+// answer is then ranked among the kept entries only.  gs (a power of two up
+// to 32) is chosen so that there are about 4k groups or more: the bound is
+// then close to the answer and few entries pass.  Returns false (results
+// unset) when more than kSelGroupsMax groups would be needed or more than
+// kSelCap entries pass a filter.  Called by every thread of the block.
 SA_DEV bool filtered_select2(const float* lo, const float* hi, int n, int k_lo, int k_hi,
                              SelScratch* sc, float& out_lo, float& out_hi) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  const int ng = (n + 31) >> 5;
+  const int kmax = max(k_lo, k_hi);
+  int gs = 32;
+  while (gs > 1 && (n + gs - 1) / gs < 4 * kmax && (n + gs / 2 - 1) / (gs / 2) <= kSelGroupsMax)
+    gs >>= 1;
+  const int ng = (n + gs - 1) / gs;
   if (ng > kSelGroupsMax) return false;
-  for (int gi = warp; gi < ng; gi += nw) {
-    const int i = gi * 32 + lane;
+  // lane l of a warp step covers entry 32 i + l, in group (32 i + l) / gs
+  for (int i0 = warp * 32; i0 < ng * gs; i0 += nw * 32) {
+    const int i = i0 + lane;
     float a = i < n ? lo[i] : -INFINITY, c = i < n ? hi[i] : -INFINITY;
     a = isnan(a) ? -INFINITY : a;
     c = isnan(c) ? -INFINITY : c;
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
+    for (int o = 1; o < gs; o <<= 1) {
       a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
       c = fmaxf(c, __shfl_xor_sync(0xffffffffu, c, o));
     }
-    if (lane == 0) {
-      sc->glo[gi] = a;
-      sc->ghi[gi] = c;
+    if ((lane & (gs - 1)) == 0 && i < ng * gs) {
+      sc->glo[i / gs] = a;
+      sc->ghi[i / gs] = c;
     }
   }
   if (tid == 0) {

@@ -528,6 +528,55 @@ def test_select_tiered_ties():
     check_tiered(cfg, inp, sig)
 
 
+@pytest.mark.parametrize("Dk", [576, 136])
+def test_select_tiered_brackets_and_row_masks(Dk):
+    # The tiered scorer's workspace: per (sequence, 32-row group, page) a float32
+    # bracket that must contain the exact row-group maximum, and a row mask that
+    # must flag every row attaining it; wide exponents, subnormals and zeros.
+    # Dk = 136 exercises the zero-padded last 16-feature step.
+    cfg, inp, _ = tiered_case(7, B=2, T=2, Hq=64, Dk=Dk, P=16, L=70 * 16 - 5, alpha=3, beta=6)
+    rng = np.random.default_rng(7)
+    pt = np_i32(inp["page_table"])
+    sl = np_i32(inp["seq_lens"])
+    qb = _random_bf16_bits(rng, tuple(inp["q"].shape), 114, 136)
+    sig = _random_bf16_bits(rng, (int(pt.max()) + 1, 1, Dk), 104, 144)
+    max_pages = pt.shape[1]
+    nbytes = sa.load().sa_select_tiered_workspace_size(cfg.B, cfg.T, cfg.Hq, max_pages)
+    ws = torch.zeros(int(nbytes), dtype=torch.uint8, device=DEV)
+    lists, counts = sa.sa_select_pages_tiered(to_bf16_dev(qb), to_bf16_dev(sig),
+                                              inp["page_table"].to(DEV), inp["seq_lens"].to(DEV),
+                                              cfg.page_size, cfg.alpha, cfg.beta, workspace=ws)
+    torch.cuda.synchronize()
+    R = cfg.T * cfg.Hq
+    RG = 32                                   # query rows per scoring group
+    n_rg = -(-R // RG)
+    raw = ws.cpu().numpy()
+    nl = cfg.B * n_rg * max_pages
+    lohi = raw[:nl * 8].view(np.float32).reshape(cfg.B, n_rg, max_pages, 2).astype(np.float64)
+    masks = raw[nl * 8:nl * 16].view(np.uint64).reshape(cfg.B, n_rg, max_pages)
+    q = O.bf16_to_f64(qb)
+    for b in range(cfg.B):
+        nb = -(-int(sl[b]) // cfg.page_size)
+        rows = q[b].reshape(R, Dk)
+        ex = O.exact_dots(rows, O.bf16_to_f64(sig[pt[b, :nb], 0, :]))   # [R, nb]
+        for g in range(n_rg):
+            eg = ex[g * RG:(g + 1) * RG]
+            gmax = eg.max(axis=0)
+            lo, hi = lohi[b, g, :nb, 0], lohi[b, g, :nb, 1]
+            assert np.all(lo <= gmax) and np.all(gmax <= hi), "bracket misses the group maximum"
+            for p in range(nb):
+                arg = np.flatnonzero(eg[:, p] == gmax[p])
+                m = int(masks[b, g, p])
+                assert all((m >> int(r)) & 1 for r in arg), "a maximising row is not flagged"
+    # and the selection itself
+    crit, cc, amb, ac = O.select_pages_mla(qb, sig, pt, sl, cfg.page_size, cfg.alpha, cfg.beta)
+    lists, counts = np_i32(lists), np_i32(counts)
+    for b in range(cfg.B):
+        want0 = list(crit[b, :cc[b]])
+        assert list(lists[b, 0, :counts[b, 0]]) == want0
+        assert list(lists[b, 1, :counts[b, 1]]) == sorted(want0 + list(amb[b, :ac[b]]))
+
+
 @pytest.mark.slow
 def test_select_tiered_mla_workload_sampled():
     cfg = W.MLA_MTP
