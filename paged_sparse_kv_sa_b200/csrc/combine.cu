@@ -1,7 +1,7 @@
 // Log-sum-exp merge of split-KV partials: lse = log sum_s exp(lse_s),
 // O = sum_s exp(lse_s - lse) O_s.  One thread per (row, 4 output columns),
-// 16-byte loads and stores, the loads of 8 splits in flight together;
-// memory-bound.
+// 16-byte loads and stores, the loads of 8 splits in flight together, no load
+// of a split without keys; memory-bound.
 //
 // Source: the merge step of a split Flash-decode ("TileSparse", section
 // "Configuration": mode full = fused Flash-decode).
@@ -11,7 +11,8 @@
 namespace sa {
 namespace {
 
-constexpr int kCombineBatch = 8;   // splits whose loads are in flight together
+constexpr int kCombineBatch = 8;   // splits whose loads are in flight together (many splits)
+constexpr int kRegSplits = 16;     // up to this many splits: every load of a phase at once
 
 __global__ void __launch_bounds__(128)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
@@ -23,43 +24,64 @@ __global__ void __launch_bounds__(128)
   if (idx >= rows * q4) return;
   const int64_t row = idx / q4;
   const int c = (int)(idx % q4) * 4;
-  // running merge over batches of splits: every load of a batch is issued
-  // before any of them is used
+  // The split LSEs first, then the O rows of the splits that have keys (a
+  // split without keys is not read at all); with up to kRegSplits splits every
+  // load of a phase is issued before any is used.
   float m = -INFINITY, tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s0 = 0; s0 < n_splits; s0 += kCombineBatch) {
-    float ls[kCombineBatch];
-    float4 v[kCombineBatch];
+  if (n_splits <= kRegSplits) {
+    float w[kRegSplits];
 #pragma unroll
-    for (int i = 0; i < kCombineBatch; ++i) {
-      const int s = s0 + i;
-      ls[i] = s < n_splits ? lse_part[s * rows + row] : -INFINITY;
-      v[i] = s < n_splits ? *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c)
+    for (int s = 0; s < kRegSplits; ++s)
+      w[s] = s < n_splits ? __ldg(lse_part + s * rows + row) : -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kRegSplits; ++s) m = fmaxf(m, w[s]);
+    if (m != -INFINITY) {
+      float4 v[kRegSplits];
+#pragma unroll
+      for (int s = 0; s < kRegSplits; ++s) {
+        w[s] = __expf(w[s] - m);
+        v[s] = w[s] > 0.f ? *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c)
                           : make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-    float mb = m;
+      }
 #pragma unroll
-    for (int i = 0; i < kCombineBatch; ++i) mb = fmaxf(mb, ls[i]);
-    if (mb == -INFINITY) continue;
-    const float sc = __expf(m - mb);   // 0 while nothing has been merged
-    tot *= sc;
-    acc.x *= sc;
-    acc.y *= sc;
-    acc.z *= sc;
-    acc.w *= sc;
-#pragma unroll
-    for (int i = 0; i < kCombineBatch; ++i) {
-      const float w = __expf(ls[i] - mb);
-      tot += w;
-      // a split without keys (weight 0) adds nothing, whatever its O holds
-      if (w > 0.f) {
-        acc.x += w * v[i].x;
-        acc.y += w * v[i].y;
-        acc.z += w * v[i].z;
-        acc.w += w * v[i].w;
+      for (int s = 0; s < kRegSplits; ++s) {
+        tot += w[s];
+        acc.x += w[s] * v[s].x;
+        acc.y += w[s] * v[s].y;
+        acc.z += w[s] * v[s].z;
+        acc.w += w[s] * v[s].w;
       }
     }
-    m = mb;
+  } else {
+    for (int s0 = 0; s0 < n_splits; s0 += kCombineBatch) {
+      float ls[kCombineBatch];
+#pragma unroll
+      for (int i = 0; i < kCombineBatch; ++i)
+        ls[i] = s0 + i < n_splits ? __ldg(lse_part + (s0 + i) * rows + row) : -INFINITY;
+#pragma unroll
+      for (int i = 0; i < kCombineBatch; ++i) m = fmaxf(m, ls[i]);
+    }
+    if (m != -INFINITY)
+      for (int s0 = 0; s0 < n_splits; s0 += kCombineBatch) {
+        float w[kCombineBatch];
+        float4 v[kCombineBatch];
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i)
+          w[i] = s0 + i < n_splits ? __expf(__ldg(lse_part + (s0 + i) * rows + row) - m) : 0.f;
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i)
+          v[i] = w[i] > 0.f ? *reinterpret_cast<const float4*>(o_part + ((s0 + i) * rows + row) * Dv + c)
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int i = 0; i < kCombineBatch; ++i) {
+          tot += w[i];
+          acc.x += w[i] * v[i].x;
+          acc.y += w[i] * v[i].y;
+          acc.z += w[i] * v[i].z;
+          acc.w += w[i] * v[i].w;
+        }
+      }
   }
   float lse = -INFINITY;
   if (m != -INFINITY) {

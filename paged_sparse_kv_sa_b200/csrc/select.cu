@@ -77,9 +77,10 @@ SA_DEV int clamped_len(const SelectArgs& a, int b, bool report) {
 // Every bf16 x bf16 product is exact in float32.  The score bracket of row r is
 //   s_r -/+ E_r,  E_r = c_acc T_r + (1 + 2^-10) U_r + 2^-126 ||q_r||_1 + Dk 2^-124
 // with directed rounding.  c_acc T_r covers the rounding of the float32
-// accumulation (c_acc = Dk 2^-19: the accumulation of each 16-term step loses
-// less than 2^-17.8 of the running magnitude sum, which leaves a margin of
-// 7x); U_r covers subnormal q_d flushed to zero inside the MMA, 2^-126
+// accumulation (c_acc = Dk 2^-20: the accumulation of each 16-term step loses
+// less than 2^-17.9 of the running magnitude sum even if every addend were
+// truncated at the largest exponent, a margin of about 3.5x); U_r covers
+// subnormal q_d flushed to zero inside the MMA, 2^-126
 // ||q_r||_1 the same for sigma_d, and Dk 2^-124 any product that underflows
 // float32.  A page's bracket is [max_r (s_r - E_r), max_r (s_r + E_r)].
 template <int NT, int DK>   // 8-row tiles of query rows (R <= 8 NT); feature count
@@ -115,38 +116,57 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
     }
     fence_mbar_init();
   }
-  // query rows of the block's heads, zero past R; 16-byte pieces
-  for (int i = tid; i < hb * QROWS * (ROWB / 16); i += blockDim.x) {
-    const int piece = i % (ROWB / 16), r = (i / (ROWB / 16)) % QROWS, w = i / (QROWS * (ROWB / 16));
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < R) {
-      const int t = r / G, h = (h0 + w) * G + r % G;
-      v = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 + piece * 8);
-    }
-    *reinterpret_cast<uint4*>(q_s + (w * QROWS + r) * QS + piece * 16) = v;
-  }
-  // per head: ||q_r||_1 (rounded up) and whether any row element is subnormal
-  for (int w = warp; w < hb; w += blockDim.x / 32) {
-    int sub = 0;
-    for (int r = 0; r < QROWS; ++r) {
-      float s1 = 0.f;
+  __syncthreads();   // barriers initialised: the producer starts at once
+
+  if (warp < hb) {
+    // consumers: the query rows of the block's heads (zero past R) into shared
+    // memory, then per head ||q_r||_1 (rounded up) and whether an element is
+    // subnormal, while the producer's first gathers are in flight
+    // (every thread's loads are issued before any is stored: one round trip)
+    constexpr int kPer = QROWS * (ROWB / 16) / 32;   // pieces per consumer thread
+    uint4 v[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * hb * 32;
+      const int r = (i / (ROWB / 16)) % QROWS, w = i / (QROWS * (ROWB / 16));
+      v[j] = make_uint4(0, 0, 0, 0);
       if (r < R) {
         const int t = r / G, h = (h0 + w) * G + r % G;
-        const uint16_t* qr = a.q + b * a.qs0 + t * a.qs1 + h * a.qs2;
-        for (int d = lane; d < DK; d += 32) {
-          const uint32_t x = qr[d];
-          s1 += fabsf(bf16_bits_to_float(x));
-          sub |= ((x & 0x7f80u) == 0 && (x & 0x7fu) != 0);
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        v[j] = *reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2 +
+                                               (i % (ROWB / 16)) * 8);
       }
-      if (lane == 0) qn1_s[w][r] = s1 * (1.f + DK * 1.2e-7f);
     }
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+      const int i = tid + j * hb * 32;
+      const int r = (i / (ROWB / 16)) % QROWS, w = i / (QROWS * (ROWB / 16));
+      *reinterpret_cast<uint4*>(q_s + (w * QROWS + r) * QS + (i % (ROWB / 16)) * 16) = v[j];
+    }
+    asm volatile("bar.sync 1, %0;" ::"r"(hb * 32) : "memory");
+    // LPR lanes per query row, each over DK / LPR features in 16-byte pieces
+    constexpr int LPR = 32 / QROWS;
+    const int r = lane / LPR, part = lane % LPR;
+    float s1 = 0.f;
+    int sub = 0;
+#pragma unroll
+    for (int c = 0; c < DK / 8 / LPR; ++c) {
+      const uint4 x4 = *reinterpret_cast<const uint4*>(q_s + (warp * QROWS + r) * QS +
+                                                      (c * LPR + part) * 16);
+      const uint32_t w4[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        s1 += fabsf(__uint_as_float(w4[e] << 16)) + fabsf(__uint_as_float(w4[e] & 0xffff0000u));
+        sub |= ((w4[e] & 0x7f80u) == 0 && (w4[e] & 0x7fu) != 0) |
+               ((w4[e] & 0x7f800000u) == 0 && (w4[e] & 0x7f0000u) != 0);
+      }
+    }
+#pragma unroll
+    for (int o = LPR / 2; o; o >>= 1) s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    if (part == 0) qn1_s[warp][r] = s1 * (1.f + DK * 1.2e-7f);
     sub = __any_sync(0xffffffffu, sub);
-    if (lane == 0) sub_s[w] = sub;
+    if (lane == 0) sub_s[warp] = sub;
+    __syncwarp();
   }
-  __syncthreads();
 
   if (warp == hb) {
     // ================= producer: page-table lookups and bulk gathers
@@ -187,7 +207,7 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
     // ================= consumers: one kv head each
     const int kvh = h0 + warp;
     const bool sub = sub_s[warp] != 0;
-    constexpr float c_acc = DK * 1.9073486328125e-06f;   // Dk * 2^-19
+    constexpr float c_acc = DK * 9.5367431640625e-07f;   // Dk * 2^-20
     constexpr float e_abs = DK * 4.70197740328915e-38f;  // Dk * 2^-124
     float2* outrow = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
     const int gq = lane >> 2, cq = lane & 3;           // fragment row / column pair
@@ -326,12 +346,24 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
     n_unc = 0;
     n_certain = 0;
   }
-  for (int p = tid; p < N; p += blockDim.x) {
-    const bool cand = p >= n_sink && p < local0;
-    S.flag[p] = cand ? 0 : 1;
-    const float2 v = cand && k > 0 ? lohi[p] : make_float2(NAN, NAN);
-    S.lo[p] = v.x;
-    S.hi[p] = v.y;
+  // (loads in batches of 8 per thread, all in flight together)
+  for (int p0 = 0; p0 < N; p0 += 8 * kThreads) {
+    float2 v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int p = p0 + tid + j * kThreads;
+      const bool cand = p < N && p >= n_sink && p < local0;
+      v[j] = cand && k > 0 ? lohi[p] : make_float2(NAN, NAN);
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int p = p0 + tid + j * kThreads;
+      if (p < N) {
+        S.flag[p] = (p >= n_sink && p < local0) ? 0 : 1;
+        S.lo[p] = v[j].x;
+        S.hi[p] = v[j].y;
+      }
+    }
   }
   __syncthreads();
 

@@ -119,24 +119,30 @@ __global__ void __launch_bounds__(kTScoreThreads) tiered_score_kernel(const Tier
   }
   // norms: per query row ||q_r||_2 and ||q_r||_1, per page ||sigma_p||_2 (float32
   // sums, within (1 + gamma_Dk) of the truth: padded up); one warp per row
+  // 4 lanes per row, 8 rows per warp step, the rows in parallel
   const float pad = 1.f + 2.f * Dk * 5.96046448e-8f;
-  for (int rr = warp; rr < kTR + kTP; rr += kTScoreThreads / 32) {
+  for (int rr0 = warp * 8; rr0 < kTR + kTP; rr0 += kTScoreThreads / 4) {
+    const int rr = rr0 + (lane >> 2), part = lane & 3;
     const uint8_t* row = rr < kTR ? q_s + rr * RS : sg_s + (rr - kTR) * RS;
-    const bool live = rr < kTR ? rr < n_rows : phys_s[rr - kTR] >= 0;
+    const bool live = rr < kTR + kTP && (rr < kTR ? rr < n_rows : phys_s[rr - kTR] >= 0);
     float s1 = 0.f, s2 = 0.f;
     if (live)
-      for (int d = 2 * lane; d < Dk; d += 64) {
-        const uint32_t w = *reinterpret_cast<const uint32_t*>(row + d * 2);
-        const float x0 = __uint_as_float(w << 16), x1 = __uint_as_float(w & 0xffff0000u);
-        s1 += fabsf(x0) + fabsf(x1);
-        s2 = fmaf(x0, x0, fmaf(x1, x1, s2));
+      for (int c = part; c < Dk / 8; c += 4) {
+        const uint4 x4 = *reinterpret_cast<const uint4*>(row + c * 16);
+        const uint32_t w4[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
+          s1 += fabsf(x0) + fabsf(x1);
+          s2 = fmaf(x0, x0, fmaf(x1, x1, s2));
+        }
       }
 #pragma unroll
-    for (int o = 16; o; o >>= 1) {
+    for (int o = 2; o; o >>= 1) {
       s1 += __shfl_xor_sync(0xffffffffu, s1, o);
       s2 += __shfl_xor_sync(0xffffffffu, s2, o);
     }
-    if (lane == 0) {
+    if (part == 0 && rr < kTR + kTP) {
       const float n2 = __fmul_ru(__fsqrt_ru(__fmul_ru(s2, pad)), 1.0000002f);
       if (rr < kTR) {
         qn_s[rr] = n2;
@@ -335,12 +341,20 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   __shared__ int last_s;
   const int kb[2] = {min(a.alpha, N), min(a.alpha + a.beta, N)};
   // flag bits: 1 / 2 = in tier boundary 0 / 1, 4 / 8 = undecided for it
+  // (the row groups' brackets of a thread's pages, 8 loads in flight at a time)
   for (int p = tid; p < N; p += blockDim.x) {
     float l = -INFINITY, h = -INFINITY;
-    for (int rg = 0; rg < a.n_rg; ++rg) {
-      const float2 v = a.lohi[((int64_t)b * a.n_rg + rg) * a.max_pages + p];
-      l = fmaxf(l, v.x);
-      h = fmaxf(h, v.y);
+    for (int rg0 = 0; rg0 < a.n_rg; rg0 += 8) {
+      float2 v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j)
+        v[j] = rg0 + j < a.n_rg ? a.lohi[((int64_t)b * a.n_rg + rg0 + j) * a.max_pages + p]
+                                : make_float2(-INFINITY, -INFINITY);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        l = fmaxf(l, v[j].x);
+        h = fmaxf(h, v[j].y);
+      }
     }
     lo[p] = l;
     hi[p] = h;
