@@ -19,7 +19,9 @@
  *  - sa_block_union: CompactAttention's Block-Union KV Selection (abstract on
  *    the page titled "Causal Attention on CPU: ..."): Q-block union plus
  *    intra-group union into per-group KV block tables, used in place.
- *  - sa_build_page_summaries: the per-page key means the router scores
+ *  - sa_build_page_summaries / sa_update_page_summaries: the per-page key
+ *    means the router scores (all referenced pages / the pages an append
+ *    changed)
  *    (UAE "Content-Dependent Dynamic Routing", mean(k_blocks)).
  *
  * Conventions for every call:
@@ -254,6 +256,21 @@ SA_API int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_stri
                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                             int B, int Hkv, int Dk, int page_size, int P_pool,
                             uint16_t* summaries, int32_t* dev_error, void* stream);
+
+/*
+ * sa_update_page_summaries — the same summaries, rewritten only for the pages
+ * that hold the last n_new tokens of each sequence (positions
+ * [seq_lens[b] - n_new, seq_lens[b]) clamped at 0): the pages an append of
+ * n_new tokens per sequence changed (normally the one last page, two when the
+ * append crosses a page boundary).  Call it after the new keys are in the
+ * cache and seq_lens counts them; every other summary row stays as it was.
+ * Arguments as for sa_build_page_summaries; n_new >= 1 (SA_ERR_INVALID_ARG
+ * otherwise).
+ */
+SA_API int sa_update_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int B, int Hkv, int Dk, int page_size, int P_pool, int n_new,
+                             uint16_t* summaries, int32_t* dev_error, void* stream);
 
 /*
  * sa_block_union — per-group KV block tables for chunked prefill.

@@ -7,6 +7,6 @@ benchmark share.  Build the library with ``python -m paged_sparse_kv_sa_b200.bui
 from ._lib import (EXPORTED, LIB_PATH, SAError, load, page_budget, sa_block_union,  # noqa: F401
                    sa_build_page_summaries, sa_combine, sa_select_pages,
                    sa_select_pages_no_alloc, sa_select_pages_tiered,
-                   sa_select_workspace_size,
+                   sa_select_workspace_size, sa_update_page_summaries,
                    sa_sparse_decode)
 from .pipeline import SparseDecodeStep, default_splits  # noqa: F401

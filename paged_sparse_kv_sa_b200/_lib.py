@@ -38,6 +38,8 @@ _SIGNATURES = {
                               _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P]),
     "sa_combine": (_I, [_P, _P, _I, _I64, _I, _P, _P, _P, _P]),
     "sa_build_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_update_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P,
+                                      _P]),
     "sa_block_union": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 
@@ -261,6 +263,22 @@ def sa_build_page_summaries(k_cache, page_table, seq_lens, summaries=None, dev_e
                                      Dk, P, P_pool, _ptr(summaries), _ptr(dev_error),
                                      _stream(stream))
     _check(st, "sa_build_page_summaries")
+    return summaries
+
+
+def sa_update_page_summaries(k_cache, page_table, seq_lens, summaries, n_new: int,
+                             dev_error=None, stream=None):
+    """Rewrite, in place, the summaries of the pages holding each sequence's last
+    n_new tokens (after an append); returns summaries."""
+    lib = load()
+    _need_cuda(k_cache, page_table, seq_lens, summaries)
+    _bf16(k_cache), _i32(page_table), _i32(seq_lens), _bf16(summaries)
+    P_pool, Hkv, P, Dk = k_cache.shape
+    st = lib.sa_update_page_summaries(_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
+                                      page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0],
+                                      Hkv, Dk, P, P_pool, int(n_new), _ptr(summaries),
+                                      _ptr(dev_error), _stream(stream))
+    _check(st, "sa_update_page_summaries")
     return summaries
 
 

@@ -338,11 +338,12 @@ int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, i
                                     lse_out, static_cast<cudaStream_t>(stream)));
 }
 
-int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
-                            const int32_t* page_table, int max_pages, const int32_t* seq_lens,
-                            int B, int Hkv, int Dk, int page_size, int P_pool,
-                            uint16_t* summaries, int32_t* dev_error, void* stream) {
-  if (B < 0 || Hkv <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0)
+namespace {
+int summaries_call(const uint16_t* k_cache, const int64_t k_strides[4],
+                   const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B,
+                   int Hkv, int Dk, int page_size, int P_pool, int n_new, uint16_t* summaries,
+                   int32_t* dev_error, void* stream) {
+  if (B < 0 || Hkv <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0 || n_new < 0)
     return SA_ERR_INVALID_ARG;
   if (B == 0 || max_pages == 0) return SA_OK;
   if (!k_cache || !k_strides || k_strides[3] != 1 || !page_table || !seq_lens || !summaries)
@@ -351,8 +352,26 @@ int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
     if (k_strides[i] <= 0) return SA_ERR_INVALID_ARG;
   if (max_pages > 65535 || B > 65535) return SA_ERR_UNSUPPORTED;
   return cuda_status(launch_summaries(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv,
-                                      Dk, page_size, P_pool, summaries, dev_error,
+                                      Dk, page_size, P_pool, n_new, summaries, dev_error,
                                       static_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+
+int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
+                            const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                            int B, int Hkv, int Dk, int page_size, int P_pool,
+                            uint16_t* summaries, int32_t* dev_error, void* stream) {
+  return summaries_call(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv, Dk,
+                        page_size, P_pool, 0, summaries, dev_error, stream);
+}
+
+int sa_update_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
+                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                             int B, int Hkv, int Dk, int page_size, int P_pool, int n_new,
+                             uint16_t* summaries, int32_t* dev_error, void* stream) {
+  if (n_new <= 0) return SA_ERR_INVALID_ARG;
+  return summaries_call(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv, Dk,
+                        page_size, P_pool, n_new, summaries, dev_error, stream);
 }
 
 int sa_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_block_offset,

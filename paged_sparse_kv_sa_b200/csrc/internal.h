@@ -128,7 +128,8 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
 
 cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
-                             int P, int P_pool, uint16_t* sig, int32_t* err, cudaStream_t stream);
+                             int P, int P_pool, int n_new, uint16_t* sig, int32_t* err,
+                             cudaStream_t stream);
 
 cudaError_t launch_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_off,
                                int top_k, int n_sink, int32_t* tables, int32_t* counts,

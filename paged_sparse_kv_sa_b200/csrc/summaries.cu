@@ -1,7 +1,8 @@
 // Per-page key summaries: sigma = RNE_bf16(RN64(RN64(sum of valid keys) / n)).
 //
 // One CTA per (logical page, sequence); threads walk the (kv head, feature)
-// columns.  The float64 sum of at most P bf16 values is exact whenever the
+// columns.  With n_new > 0 only the pages holding the last n_new tokens of
+// each sequence are rewritten (the pages an append of n_new tokens changed).  The float64 sum of at most P bf16 values is exact whenever the
 // values span at most 53 - ceil(log2 P) - 1 bits (every bf16 is an integer
 // multiple of its lsb weight); columns that fail that test are re-summed in
 // the exact fixed-point accumulator.
@@ -20,10 +21,11 @@ __global__ void __launch_bounds__(256)
     summaries_kernel(const uint16_t* __restrict__ k, int64_t ks0, int64_t ks1, int64_t ks2,
                      const int32_t* __restrict__ pt, int max_pages,
                      const int32_t* __restrict__ seq_lens, int Hkv, int Dk, int P, int P_pool,
-                     uint16_t* __restrict__ sig, int32_t* err) {
+                     int n_new, uint16_t* __restrict__ sig, int32_t* err) {
   pdl_wait_and_release();
-  const int p = blockIdx.x, b = blockIdx.y;
+  const int b = blockIdx.y;
   const int L = min(seq_lens[b], max_pages * P);
+  const int p = (n_new > 0 ? max(L - n_new, 0) / P : 0) + blockIdx.x;
   const int n = min(P, L - p * P);
   if (n <= 0) return;
   const int ph = pt[(int64_t)b * max_pages + p];
@@ -67,11 +69,14 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
-                             int P, int P_pool, uint16_t* sig, int32_t* err, cudaStream_t stream) {
+                             int P, int P_pool, int n_new, uint16_t* sig, int32_t* err,
+                             cudaStream_t stream) {
   if (B == 0 || max_pages == 0) return cudaSuccess;
-  dim3 grid(max_pages, B);
+  // n_new tokens end in at most ceil((n_new - 1) / P) + 1 pages
+  const int pages = n_new > 0 ? min(max_pages, (n_new - 1 + P - 1) / P + 1) : max_pages;
+  dim3 grid(pages, B);
   return launch_pdl(summaries_kernel, grid, dim3(256), 0, stream, k, ks[0], ks[1], ks[2], pt,
-                    max_pages, seq_lens, Hkv, Dk, P, P_pool, sig, err);
+                    max_pages, seq_lens, Hkv, Dk, P, P_pool, n_new, sig, err);
 }
 
 }  // namespace sa

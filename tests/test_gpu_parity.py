@@ -89,6 +89,26 @@ def test_summaries_exact_fallback_values():
     np.testing.assert_array_equal(bits(sig), ref)
 
 
+@pytest.mark.parametrize("n_new", [1, 3, 40])
+def test_summaries_update_after_append(n_new):
+    # summaries built for the shorter sequences, then updated for the pages an
+    # append of n_new tokens touched: every referenced row must equal the oracle
+    # for the new lengths (rows before the append are unchanged by it)
+    cfg = W.scaled(W.TINY_GQA, B=3)
+    lens_new = [2048 - 5, 1000, 17 + n_new]
+    inp, g = gqa_case(cfg, seed=12, seq_lens=lens_new)
+    sl_old = torch.tensor([max(x - n_new, 0) for x in lens_new], dtype=torch.int32, device=DEV)
+    sig = sa.sa_build_page_summaries(g["k"], g["page_table"], sl_old)
+    sa.sa_update_page_summaries(g["k"], g["page_table"], g["seq_lens"], sig, n_new)
+    torch.cuda.synchronize()
+    ref = oracle_summaries(inp, cfg)
+    got = bits(sig)
+    pt = np_i32(inp["page_table"])
+    for b, L in enumerate(lens_new):
+        used = pt[b, :-(-L // cfg.page_size)]
+        np.testing.assert_array_equal(got[used], ref[used])
+
+
 # ----------------------------------------------------------------------------
 # selection
 # ----------------------------------------------------------------------------
