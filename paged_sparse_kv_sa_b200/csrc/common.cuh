@@ -85,6 +85,19 @@ SA_DEV void bulk_store(void* dst, const void* src, uint32_t bytes) {
                : "memory");
 }
 SA_DEV void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// 16-byte asynchronous copy global -> shared by one thread; src_bytes < 16
+// fills the rest with zeros (0: writes 16 zero bytes, reads nothing).
+SA_DEV void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+               "r"(src_bytes)
+               : "memory");
+}
+SA_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's most recent cp.async groups are pending.
+template <int N>
+SA_DEV void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 // Wait until every bulk store this thread committed has completed.
 SA_DEV void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 SA_DEV void prefetch_tmap(const CUtensorMap* map) {

@@ -7,14 +7,14 @@
 // page asc).  The result is written as two decode lists per sequence: list 0
 // = critical pages, list 1 = critical + ambient pages, both ascending.
 //
-// tiered_score_kernel: one CTA per (64 pages, 64 query rows, sequence) scores
-// with warp MMAs and emits, per page and row group, a rigorous bracket of the
-// row-max score and the mask of rows that can attain it.
-// tiered_choose_kernel: one CTA per sequence merges the row groups' brackets,
-// selects the order statistics for both boundaries (alpha, alpha+beta),
-// rescores the undecided pages exactly on their flagged rows only (fixed-point
-// accumulation of the bf16 products, one rounding to float64) and writes both
-// lists.
+// tiered_score_kernel: one CTA per (128 pages, 128 query rows, sequence) scores
+// on the tensor cores (tcgen05) and emits, per page and row group, a rigorous
+// bracket of the row-max score and the mask of rows that can attain it.
+// tiered_choose_kernel: up to kChooseCtas CTAs per sequence each merge the row
+// groups' brackets and select the order statistics for both boundaries
+// (alpha, alpha+beta) in one pass; together they rescore the undecided pages
+// exactly on their flagged rows only (fixed-point accumulation of the bf16
+// products, one rounding to float64), and the last to finish writes both lists.
 //
 // Source: "TileSparse: Arithmetic-Intensity-Aware Sparse Attention for
 // Compute-Bound LLM Decoding", "Motivation" (Critical Tier: alpha pages
@@ -22,235 +22,226 @@
 #include "common.cuh"
 #include "exact.cuh"
 #include "internal.h"
+#include "tc05.cuh"
 #include "topk.cuh"
+
+#include <algorithm>
 
 namespace sa {
 namespace {
 
-constexpr int kTP = 64;            // pages per scoring CTA
-constexpr int kTR = 32;            // query rows per scoring CTA (one 32-bit row mask)
-constexpr int kTNT = kTR / 16;     // 8-row MMA tiles per warp
-constexpr int kTScoreThreads = 256;
+constexpr int kTR = 32;            // query rows per row group (one 32-bit row mask)
 constexpr int kChooseThreads = 512;
-constexpr int kChooseCtas = 8;     // CTAs per sequence sharing the exact rescoring
+constexpr int kChooseCtas = 16;    // at most this many CTAs per sequence share the exact rescoring
 
-// Scores of 64 pages x 32 query rows of one sequence, S = sigma q^T as warp
-// MMAs over the Dk features (m16n8k16, bf16 in, float32 accumulation).  Per
-// (page, row) the exact score lies in s -/+ E with (directed rounding)
-//   E = c_acc ||q_r|| ||sigma|| + 2^-126 (||q_r||_1 + sqrt(Dk) ||sigma||) + Dk 2^-124,
+// Scores of 128 pages x 128 query rows of one sequence, S = sigma q^T, on the
+// tensor cores: tcgen05.mma (M = 128 pages, N = 128 rows, K = 16 per
+// instruction, bf16 in, float32 accumulation in tensor memory) over the Dk
+// features in chunks of 64 (one 128-byte swizzle row).  Warps 0-3 gather the
+// chunk's summary rows (through the page table) and query rows with 16-byte
+// cp.async copies straight into the 128-byte-swizzled K-major layout of a
+// kSStages-deep ring, and sum each row's squares from their own copies; warp 4
+// allocates the tensor memory and issues the MMAs; warps 0-3 then read one
+// page (TMEM lane) each.  Per (page, row) the exact score lies in s -/+ E with
+// (directed rounding)
+//   E = c_acc ||q_r|| ||sigma|| + 2^-126 sqrt(Dk) (||q_r|| + ||sigma||) + Dk 2^-124,
 // c_acc = Dk 2^-20: the accumulation of each 16-product step loses less than
 // 2^-17.9 of the running magnitude sum sum_d |q_d sigma_d| <= ||q|| ||sigma||
 // even if every addend were truncated at the largest exponent (a margin of
 // about 3.5x); the 2^-126 terms cover subnormal inputs flushed to zero inside
-// the MMA, Dk 2^-124 products that underflow float32.  The norms are float32
-// sums of squares, rounded up.  Emitted per page: [max_r (s_r - E_r),
-// max_r (s_r + E_r)] over the CTA's rows, and a mask of the rows whose upper
-// end reaches that largest lower end (only those rows can hold the page's
-// maximum within this row group).  Summary and query rows arrive with one bulk
-// copy each (rows padded by 16 bytes so that ldmatrix row addresses hit
-// distinct banks).  Two CTAs fit an SM, so one's loads overlap the other's MMAs.
-__global__ void __launch_bounds__(kTScoreThreads) tiered_score_kernel(const TieredArgs a) {
+// the MMA (sum_d |x_d| <= sqrt(Dk) ||x||), Dk 2^-124 products that underflow
+// float32.  The norms are float32 sums of squares, padded by (1 + gamma_Dk) and
+// rounded up.  Emitted per page and row group of kTR rows: [max_r (s_r - E_r),
+// max_r (s_r + E_r)] and the mask of the rows whose upper end reaches that
+// largest lower end (only those rows can hold the page's maximum in the group).
+constexpr int kSP = 128;                     // pages per CTA (MMA M, TMEM lanes)
+constexpr int kSR = 128;                     // query rows per CTA (MMA N, TMEM columns)
+constexpr int kSStages = 4;                  // K-chunk ring depth
+constexpr int kSLag = kSStages - 1;          // chunks a loader keeps in flight
+constexpr int kSChunk = 64;                  // features per K chunk
+constexpr int kSTile = kSP * 128;            // bytes of one operand's chunk (16 KB)
+constexpr int kSStageBytes = 2 * kSTile;     // summaries, then query rows
+constexpr int kSThreads = 160;
+constexpr uint32_t kSIdesc = tc::idesc_bf16_f32(kSP, kSR, false, false);
+static_assert(kSR % kTR == 0, "row groups tile the CTA's rows");
+
+__global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const TieredArgs a) {
   pdl_wait_and_release();
-  const int pc = blockIdx.x, rg = blockIdx.y, b = blockIdx.z;
+  const int pc = blockIdx.x, rt = blockIdx.y, b = blockIdx.z;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) L = L < 0 ? 0 : a.max_pages * a.P;
   const int N = (L + a.P - 1) / a.P;
   const int R = a.T * a.Hq;
-  const int p0 = pc * kTP, r0 = rg * kTR;
+  const int p0 = pc * kSP, r0 = rt * kSR;
   if (p0 >= N || r0 >= R) return;
-  const int Dk = a.Dk, KP = (Dk + 15) & ~15, RS = KP * 2 + 16;
-  // the choose kernel's exact-score slots and completion counter start at 0
-  if (rg == 0 && threadIdx.x < kTP && p0 + threadIdx.x < N)
-    a.exkey[(int64_t)b * a.max_pages + p0 + threadIdx.x] = 0ull;
-  if (pc == 0 && rg == 0 && threadIdx.x == 0) a.counter[b] = 0u;
-  extern __shared__ __align__(128) uint8_t tsm[];
-  uint8_t* sg_s = tsm;                  // [kTP][RS] summaries
-  uint8_t* q_s = tsm + kTP * RS;        // [kTR][RS] query rows
-  __shared__ uint64_t ld_bar;
-  __shared__ int phys_s[kTP];
-  __shared__ float qn_s[kTR];           // ||q_r||_2, rounded up
-  __shared__ float fl_s[kTR];           // 2^-126 ||q_r||_1, rounded up
-  __shared__ float sn_s[kTP];           // ||sigma_p||_2, rounded up
-  __shared__ float2 half_s[4][16];      // rows of the second warp half: per page (lo, hi)
-  __shared__ float mlo_s[kTP];          // per page: largest lower end over the rows
-  __shared__ unsigned long long mhalf_s[4][16];
+  const int Dk = a.Dk, KC = (Dk + kSChunk - 1) / kSChunk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid < kTP) {
-    const int p = p0 + tid;
-    int ph = -1;
-    if (p < N) {
-      ph = a.page_table[(int64_t)b * a.max_pages + p];
-      if (ph < 0 || ph >= a.P_pool) {
-        set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
-        ph = -1;
-      }
-    }
-    phys_s[tid] = ph;
-  }
+  // the choose kernel's exact-score slots and completion counter start at 0
+  if (rt == 0 && tid < kSP && p0 + tid < N) a.exkey[(int64_t)b * a.max_pages + p0 + tid] = 0ull;
+  if (pc == 0 && rt == 0 && tid == 0) a.counter[b] = 0u;
+  extern __shared__ uint8_t tsm_raw[];
+  uint8_t* ring = tsm_raw + ((1024 - (smem_u32(tsm_raw) & 1023)) & 1023);
+  __shared__ uint64_t full[kSStages], empty[kSStages], mma_done;
+  __shared__ uint32_t tmem_s;
+  __shared__ float sn_s[kSP];          // ||sigma_p||, rounded up
+  __shared__ float cq_s[kSR];          // c_acc ||q_r||, rounded up
+  __shared__ float fq_s[kSR];          // 2^-126 sqrt(Dk) ||q_r||, rounded up
+  __shared__ int8_t pok_s[kSP];        // page readable
   if (tid == 0) {
-    mbar_init(&ld_bar, 1);
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&full[s], 4 * 32);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&mma_done, 1);
     fence_mbar_init();
   }
+  if (warp == 4) tc::tmem_alloc(&tmem_s, kSR);
+  tc::fence_before_sync();
   __syncthreads();
-  const int n_rows = min(kTR, R - r0);
-  const uint32_t rowb = Dk * 2;
-  if (warp == 0) {
-    const uint32_t m0 = __ballot_sync(0xffffffffu, phys_s[lane] >= 0);
-    const uint32_t m1 = __ballot_sync(0xffffffffu, phys_s[32 + lane] >= 0);
-    if (lane == 0) mbar_arrive_expect_tx(&ld_bar, (__popc(m0) + __popc(m1) + n_rows) * rowb);
-    __syncwarp();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_s;
+  const uint32_t ring_u = smem_u32(ring);
+
+  if (warp < 4) {
+    // this thread: 16-byte unit j of every chunk, rows rb + 16 i (i < 8) of
+    // both operands; in the swizzled layout row rr's unit j sits at
+    // (rr / 8) * 1024 + (rr % 8) * 128 + ((j ^ (rr % 8)) * 16), and rr % 8 = rb % 8
+    const int j = tid & 7, rb = tid >> 3;
+    const uint32_t soff = (rb >> 3) * 1024 + (rb & 7) * 128 + ((j ^ (rb & 7)) << 4);
+    const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
+    const uint16_t* arow[8];
+    const uint16_t* brow[8];
 #pragma unroll
-    for (int i = lane; i < kTP; i += 32)
-      if (phys_s[i] >= 0) bulk_load(sg_s + i * RS, a.sig + (int64_t)phys_s[i] * Dk, rowb, &ld_bar);
-  } else if (warp == 1) {
-#pragma unroll
-    for (int i = lane; i < kTR; i += 32)
-      if (i < n_rows) {
-        const int r = r0 + i, t = r / a.Hq, h = r % a.Hq;
-        bulk_load(q_s + i * RS, a.q + b * a.qs0 + t * a.qs1 + h * a.qs2, rowb, &ld_bar);
-      }
-  }
-  if (KP != Dk)   // the last 8 features of a 16-feature step: zeros
-    for (int i = tid; i < kTP + kTR; i += blockDim.x)
-      *reinterpret_cast<uint4*>(tsm + i * RS + rowb) = make_uint4(0, 0, 0, 0);
-  if (__syncthreads_or(!mbar_wait_bounded(&ld_bar, 0))) {
-    if (tid == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
-    return;
-  }
-  // norms: per query row ||q_r||_2 and ||q_r||_1, per page ||sigma_p||_2 (float32
-  // sums, within (1 + gamma_Dk) of the truth: padded up); one warp per row
-  // 4 lanes per row, 8 rows per warp step, the rows in parallel
-  const float pad = 1.f + 2.f * Dk * 5.96046448e-8f;
-  for (int rr0 = warp * 8; rr0 < kTR + kTP; rr0 += kTScoreThreads / 4) {
-    const int rr = rr0 + (lane >> 2), part = lane & 3;
-    const uint8_t* row = rr < kTR ? q_s + rr * RS : sg_s + (rr - kTR) * RS;
-    const bool live = rr < kTR + kTP && (rr < kTR ? rr < n_rows : phys_s[rr - kTR] >= 0);
-    float s1 = 0.f, s2 = 0.f;
-    if (live)
-      for (int c = part; c < Dk / 8; c += 4) {
-        const uint4 x4 = *reinterpret_cast<const uint4*>(row + c * 16);
-        const uint32_t w4[4] = {x4.x, x4.y, x4.z, x4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float x0 = __uint_as_float(w4[e] << 16), x1 = __uint_as_float(w4[e] & 0xffff0000u);
-          s1 += fabsf(x0) + fabsf(x1);
-          s2 = fmaf(x0, x0, fmaf(x1, x1, s2));
+    for (int i = 0; i < 8; ++i) {
+      const int p = p0 + rb + 16 * i, r = r0 + rb + 16 * i;
+      int ph = -1;
+      if (p < N) {
+        ph = ptrow[p];
+        if (ph < 0 || ph >= a.P_pool) {
+          if (j == 0) set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
+          ph = -1;
         }
       }
-#pragma unroll
-    for (int o = 2; o; o >>= 1) {
-      s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-      s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+      if (j == 0) pok_s[rb + 16 * i] = ph >= 0;
+      arow[i] = ph >= 0 ? a.sig + (int64_t)ph * Dk : nullptr;
+      brow[i] = r < R ? a.q + b * a.qs0 + (r / a.Hq) * a.qs1 + (r % a.Hq) * a.qs2 : nullptr;
     }
-    if (part == 0 && rr < kTR + kTP) {
-      const float n2 = __fmul_ru(__fsqrt_ru(__fmul_ru(s2, pad)), 1.0000002f);
-      if (rr < kTR) {
-        qn_s[rr] = n2;
-        fl_s[rr] = __fmul_ru(__fmul_ru(s1, pad), 1.1754943508222875e-38f);
-      } else {
-        sn_s[rr - kTR] = n2;
+    float sa2[8], sb2[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) sa2[i] = sb2[i] = 0.f;
+    for (int kc = 0; kc < KC + kSLag; ++kc) {
+      if (kc < KC) {
+        const int s = kc % kSStages;
+        if (kc >= kSStages && !mbar_wait_bounded(&empty[s], ((kc / kSStages) - 1) & 1))
+          set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+        const int f0 = kc * kSChunk + 8 * j;      // Dk % 8 == 0: a unit is all in or all out
+        const uint32_t da = ring_u + s * kSStageBytes + soff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const bool va = arow[i] != nullptr && f0 < Dk, vb = brow[i] != nullptr && f0 < Dk;
+          cp_async16(da + 2048 * i, va ? arow[i] + f0 : a.sig, va ? 16u : 0u);
+          cp_async16(da + kSTile + 2048 * i, vb ? brow[i] + f0 : a.q, vb ? 16u : 0u);
+        }
+      }
+      cp_async_commit();          // (empty groups past the end keep the count uniform)
+      if (kc >= kSLag) {
+        cp_async_wait<kSLag>();   // this thread's part of chunk kc - kSLag has landed
+        const int s = (kc - kSLag) % kSStages;
+        const uint8_t* src = ring + s * kSStageBytes + soff;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(src + 2048 * i);
+          const uint4 y = *reinterpret_cast<const uint4*>(src + kSTile + 2048 * i);
+          const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
+            const float y0 = __uint_as_float(yw[e] << 16), y1 = __uint_as_float(yw[e] & 0xffff0000u);
+            sa2[i] = fmaf(x0, x0, fmaf(x1, x1, sa2[i]));
+            sb2[i] = fmaf(y0, y0, fmaf(y1, y1, sb2[i]));
+          }
+        }
+        tc::fence_proxy_async();   // the copies are read by the tensor core
+        mbar_arrive(&full[s]);
       }
     }
-  }
-  __syncthreads();
-
-  // warp w: pages 16 (w & 3) .. + 15, query rows 8 kTNT (w >> 2) .. + 8 kTNT - 1
-  const int mt = warp & 3, nh = warp >> 2;
-  const int gq = lane >> 2, cq = lane & 3;
-  const uint32_t a_addr = smem_u32(sg_s) + (16 * mt + (lane & 15)) * RS + 16 * (lane >> 4);
-  const uint32_t b_addr =
-      smem_u32(q_s) + (8 * kTNT * nh + (lane & 7)) * RS + 16 * ((lane >> 3) & 1);
-  float acc[kTNT][4];
+    // row norms: the 8 lanes of a row group hold its 8 feature slices
 #pragma unroll
-  for (int nt = 0; nt < kTNT; ++nt)
+    for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
-#pragma unroll 4
-  for (int ks = 0; ks < KP / 16; ++ks) {
-    uint32_t af[4];
-    ldmatrix_x4(af, a_addr + ks * 32);
-#pragma unroll
-    for (int nt = 0; nt < kTNT; ++nt) {
-      uint32_t bq[2];
-      ldmatrix_x2(bq, b_addr + nt * 8 * RS + ks * 32);
-      mma_bf16_16816(acc[nt], af, bq[0], bq[1]);
-    }
-  }
-  // this lane: pages 16 mt + gq (i = 0, 1) and + 8 (i = 2, 3); rows
-  // 8 kTNT nh + 8 nt + 2 cq + (i & 1) of the CTA
-  const float c_acc = Dk * 9.5367431640625e-07f;       // Dk * 2^-20
-  const float e_abs = Dk * 4.70197740328915e-38f;      // Dk * 2^-124
-  const float rt = __fsqrt_ru(static_cast<float>(Dk)) * 1.1754943508222875e-38f;
-  float sn[2], en[2];
-#pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    sn[h] = sn_s[16 * mt + gq + 8 * h];
-    en[h] = __fadd_ru(__fmul_ru(rt, sn[h]), e_abs);
-  }
-  float hr[kTNT][4];                    // per element: s + E (for the row mask)
-  float lo[2] = {-INFINITY, -INFINITY}, hi[2] = {-INFINITY, -INFINITY};
-#pragma unroll
-  for (int nt = 0; nt < kTNT; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rr = 8 * kTNT * nh + 8 * nt + 2 * cq + (i & 1);
-      const int h = i >> 1;
-      hr[nt][i] = -INFINITY;
-      if (rr < n_rows) {
-        const float E = __fadd_ru(__fmul_ru(__fmul_ru(c_acc, qn_s[rr]), sn[h]),
-                                  __fadd_ru(fl_s[rr], en[h]));
-        const float sv = acc[nt][i];
-        hr[nt][i] = __fadd_ru(sv, E);
-        lo[h] = fmaxf(lo[h], __fsub_rd(sv, E));
-        hi[h] = fmaxf(hi[h], hr[nt][i]);
+      for (int o = 1; o < 8; o <<= 1) {
+        sa2[i] += __shfl_xor_sync(0xffffffffu, sa2[i], o);
+        sb2[i] += __shfl_xor_sync(0xffffffffu, sb2[i], o);
       }
-    }
+    const float pad = 1.f + 2.f * Dk * 5.96046448e-8f;
+    const float c_acc = Dk * 9.5367431640625e-07f;                                 // Dk 2^-20
+    const float rt_d = __fmul_ru(__fsqrt_ru(static_cast<float>(Dk)), 1.1754943508222875e-38f);
+    if (j == 0)
 #pragma unroll
-  for (int h = 0; h < 2; ++h)
+      for (int i = 0; i < 8; ++i) {
+        const int rr = rb + 16 * i;
+        sn_s[rr] = __fmul_ru(__fsqrt_ru(__fmul_ru(sa2[i], pad)), 1.0000002f);
+        const float qn = __fmul_ru(__fsqrt_ru(__fmul_ru(sb2[i], pad)), 1.0000002f);
+        cq_s[rr] = __fmul_ru(c_acc, qn);
+        fq_s[rr] = __fmul_ru(rt_d, qn);
+      }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // epilogue: thread = page p0 + tid = TMEM lane tid
+    if (!mbar_wait_bounded(&mma_done, 0)) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+    tc::fence_after_sync();
+    const int p = p0 + tid;
+    const bool pok = pok_s[tid] != 0;
+    const float sn = sn_s[tid];
+    const float es = __fadd_ru(__fmul_ru(rt_d, sn), Dk * 4.70197740328915e-38f);   // + Dk 2^-124
+    for (int g = 0; g < kSR / kTR && r0 + g * kTR < R; ++g) {
+      float sv[32];
+      tc::ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + g * kTR, sv);
+      tc::wait_ld();
+      float lo = -INFINITY, hi = -INFINITY;
 #pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      lo[h] = fmaxf(lo[h], __shfl_xor_sync(0xffffffffu, lo[h], o));
-      hi[h] = fmaxf(hi[h], __shfl_xor_sync(0xffffffffu, hi[h], o));
-    }
-  if (nh == 1 && cq == 0)
-    for (int h = 0; h < 2; ++h) half_s[mt][gq + 8 * h] = make_float2(lo[h], hi[h]);
-  __syncthreads();
-  if (nh == 0 && cq == 0)
-    for (int h = 0; h < 2; ++h) {
-      const int pl = 16 * mt + gq + 8 * h, p = p0 + pl;
-      const float2 o2 = half_s[mt][gq + 8 * h];
-      const float l2 = fmaxf(lo[h], o2.x), h2 = fmaxf(hi[h], o2.y);
-      mlo_s[pl] = l2;
+      for (int c = 0; c < 32; ++c) {
+        const int rr = g * kTR + c;
+        if (r0 + rr < R) {
+          const float E = __fadd_ru(__fmul_ru(cq_s[rr], sn), __fadd_ru(fq_s[rr], es));
+          lo = fmaxf(lo, __fsub_rd(sv[c], E));
+          sv[c] = __fadd_ru(sv[c], E);
+          hi = fmaxf(hi, sv[c]);
+        } else {
+          sv[c] = -INFINITY;
+        }
+      }
+      uint32_t m = 0;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) m |= static_cast<uint32_t>(sv[c] >= lo) << c;
       if (p < N) {
+        const int64_t at = ((int64_t)b * a.n_rg + r0 / kTR + g) * a.max_pages + p;
         // + 0 turns -0 into +0 (the radix keys order -0 below +0)
-        a.lohi[((int64_t)b * a.n_rg + rg) * a.max_pages + p] =
-            phys_s[pl] < 0 ? make_float2(-INFINITY, -INFINITY) : make_float2(l2 + 0.f, h2 + 0.f);
+        a.lohi[at] = pok ? make_float2(lo + 0.f, hi + 0.f) : make_float2(-INFINITY, -INFINITY);
+        a.rmask[at] = pok ? m : 0ull;
       }
     }
-  __syncthreads();
-  // rows whose upper end reaches the page's largest lower end
-  unsigned long long bits[2] = {0ull, 0ull};
+  } else if (lane == 0) {
+    // ================= MMA issuer.  Descriptors advance by (byte offset >> 4).
+    const uint64_t da0 = tc::sdesc_sw128(ring_u, 16, 1024);
+    const uint64_t db0 = tc::sdesc_sw128(ring_u + kSTile, 16, 1024);
+    for (int kc = 0; kc < KC; ++kc) {
+      const int s = kc % kSStages;
+      if (!mbar_wait_bounded(&full[s], (kc / kSStages) & 1)) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
+      tc::fence_after_sync();
+      const uint64_t off = static_cast<uint64_t>((s * kSStageBytes) >> 4);
 #pragma unroll
-  for (int nt = 0; nt < kTNT; ++nt)
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int rr = 8 * kTNT * nh + 8 * nt + 2 * cq + (i & 1);
-      if (hr[nt][i] >= mlo_s[16 * mt + gq + 8 * (i >> 1)]) bits[i >> 1] |= 1ull << rr;
+      for (int kk = 0; kk < kSChunk / 16; ++kk)
+        tc::mma_bf16(tmem, da0 + off + kk * 2, db0 + off + kk * 2, kSIdesc, (kc | kk) ? 1u : 0u);
+      tc::commit(&empty[s]);
     }
-#pragma unroll
-  for (int h = 0; h < 2; ++h)
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) bits[h] |= __shfl_xor_sync(0xffffffffu, bits[h], o);
-  if (nh == 1 && cq == 0)
-    for (int h = 0; h < 2; ++h) mhalf_s[mt][gq + 8 * h] = bits[h];
+    tc::commit(&mma_done);
+  }
+  tc::fence_before_sync();
   __syncthreads();
-  if (nh == 0 && cq == 0)
-    for (int h = 0; h < 2; ++h) {
-      const int pl = 16 * mt + gq + 8 * h, p = p0 + pl;
-      if (p < N)
-        a.rmask[((int64_t)b * a.n_rg + rg) * a.max_pages + p] =
-            phys_s[pl] < 0 ? 0ull : (bits[h] | mhalf_s[mt][gq + 8 * h]);
-    }
+  if (warp == 4) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kSR);
+  }
 }
 
 // Block-wide ascending compaction of the pages whose flag has `bit` set.
@@ -316,9 +307,14 @@ __device__ __noinline__ double exact_row_dot(const uint16_t* q, const uint16_t* 
   return warp_exact_dot_bf16<4>(q, sg, n);
 }
 
+// kChoosePairs bounds the (undecided page, row group) pairs whose rescoring
+// tasks are flattened to (page, row) and spread evenly over every warp of the
+// sequence's CTAs; beyond it each warp takes whole (page, row group) pairs.
+constexpr int kChoosePairs = 2048;
+
 __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const TieredArgs a) {
   pdl_wait_and_release();
-  const int b = blockIdx.x, cta = blockIdx.y, tid = threadIdx.x;
+  const int b = blockIdx.x, cta = blockIdx.y, n_cta = gridDim.y, tid = threadIdx.x;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) {
     if (tid == 0 && cta == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
@@ -331,11 +327,14 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   extern __shared__ __align__(16) uint8_t dsm[];
   float* lo = reinterpret_cast<float*>(dsm);
   float* hi = lo + a.max_pages;
-  uint16_t* u_list = reinterpret_cast<uint16_t*>(hi + a.max_pages);
+  int* ph_s = reinterpret_cast<int*>(hi + a.max_pages);        // physical page of u_list[i]
+  uint16_t* u_list = reinterpret_cast<uint16_t*>(ph_s + a.max_pages);
   uint8_t* flag = reinterpret_cast<uint8_t*>(u_list + a.max_pages);
   __shared__ uint32_t hist[1024];
   __shared__ uint32_t sel_out[8];
-  __shared__ SelScratch scratch;
+  __shared__ BucketScratch bscr;
+  __shared__ int pfx[kChoosePairs];          // exclusive prefix of the flagged rows per pair
+  __shared__ uint32_t msk[kChoosePairs];     // flagged rows of (undecided page, row group)
   __shared__ int red_i[kChooseThreads / 32];
   __shared__ int n_cert[2];
   __shared__ int last_s;
@@ -358,32 +357,48 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     }
     lo[p] = l;
     hi[p] = h;
-    flag[p] = 0;
   }
-  if (tid == 0) {
-    n_cert[0] = n_cert[1] = 0;
-  }
+  if (tid == 0) n_cert[0] = n_cert[1] = 0;
   __syncthreads();
-  for (int i = 0; i < 2; ++i) {
-    const uint8_t in_bit = 1u << i, unc_bit = 4u << i;
-    if (kb[i] >= N) {   // every page is inside this boundary
-      for (int p = tid; p < N; p += blockDim.x) flag[p] |= in_bit;
-      continue;
-    }
-    if (kb[i] == 0) continue;
-    float Lk, H;
-    if (!filtered_select2(lo, hi, N, kb[i], kb[i] + 1, &scratch, Lk, H))
-      radix_select2(lo, hi, N, kb[i], kb[i] + 1, hist, sel_out, Lk, H);
-    for (int p = tid; p < N; p += blockDim.x) {
-      if (lo[p] > H) {
-        flag[p] |= in_bit;
-        atomicAdd(&n_cert[i], 1);
-      } else if (hi[p] >= Lk) {
-        flag[p] |= unc_bit;
+  // both boundaries' order statistics in one selection pass
+  float Lk[2] = {INFINITY, INFINITY}, H[2] = {INFINITY, INFINITY};
+  {
+    int act[2], kl[2], kh[2], na = 0;
+    for (int i = 0; i < 2; ++i)
+      if (kb[i] > 0 && kb[i] < N) {
+        act[na] = i;
+        kl[na] = kb[i];
+        kh[na] = kb[i] + 1;
+        ++na;
+      }
+    if (na > 0) {
+      float ol[2], oh[2];
+      if (!bucket_select(lo, hi, N, na, kl, kh, &bscr, ol, oh))
+        for (int j = 0; j < na; ++j) radix_select2(lo, hi, N, kl[j], kh[j], hist, sel_out, ol[j], oh[j]);
+      for (int j = 0; j < na; ++j) {
+        Lk[act[j]] = ol[j];
+        H[act[j]] = oh[j];
       }
     }
-    __syncthreads();
   }
+  for (int p = tid; p < N; p += blockDim.x) {
+    uint8_t f = 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      if (kb[i] >= N) {            // every page is inside this boundary
+        f |= 1u << i;
+      } else if (kb[i] > 0) {
+        if (lo[p] > H[i]) {
+          f |= 1u << i;
+          atomicAdd(&n_cert[i], 1);
+        } else if (hi[p] >= Lk[i]) {
+          f |= 4u << i;
+        }
+      }
+    }
+    flag[p] = f;
+  }
+  __syncthreads();
   // the undecided pages, ascending (the same list in every CTA of the sequence)
   const int nu_ = compact_flag_list(flag, N, 12u, u_list, red_i);
   double* ex = reinterpret_cast<double*>(lo);   // lo/hi storage reused as doubles
@@ -392,58 +407,113 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     // exact row-max scores of the undecided pages: only the query rows the
     // scoring pass flagged for a page (per row group, the rows whose upper end
     // reaches the group's largest lower end) can hold its maximum.  One warp
-    // rescores each such (page, row) exactly; the (page, row group) tasks are
-    // dealt round-robin over the sequence's CTAs and their warps, the results
-    // merged with atomic max in global memory; the last CTA to finish ranks.
+    // rescores each such (page, row) exactly; the results are merged with an
+    // atomic max in global memory and the last CTA to finish ranks.
     const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
     const int nw = kChooseThreads / 32, warp = tid >> 5, lane = tid & 31;
+    const int gw = cta + n_cta * warp, n_gw = n_cta * nw;   // this warp among the sequence's
     unsigned long long* exk = a.exkey + (int64_t)b * a.max_pages;
-    for (int x = cta + kChooseCtas * warp; x < nu_ * a.n_rg; x += kChooseCtas * nw) {
-      const int uu = x / a.n_rg, g = x % a.n_rg;
-      const int pu = u_list[uu];
-      const int ph = ptrow[pu];
-      if (ph < 0 || ph >= a.P_pool) continue;
-      unsigned long long bits = a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + pu];
-      const uint16_t* sg = a.sig + (int64_t)ph * a.Dk;
-      while (bits) {
-        const int r = g * kTR + __ffsll(static_cast<long long>(bits)) - 1;
-        bits &= bits - 1;
-        const int t = r / a.Hq, h = r % a.Hq;
-        const double e = exact_row_dot(a.q + b * a.qs0 + t * a.qs1 + h * a.qs2, sg, a.Dk);
+    const int npair = nu_ * a.n_rg;
+    for (int i = tid; i < nu_; i += blockDim.x) {
+      const int ph = ptrow[u_list[i]];
+      ph_s[i] = (ph < 0 || ph >= a.P_pool) ? -1 : ph;
+    }
+    if (npair <= kChoosePairs) {
+      // (page, row) tasks numbered through a block scan of the pairs' row counts
+      const int per_t = (npair + blockDim.x - 1) / blockDim.x;
+      const int x0 = tid * per_t, x1 = min(npair, x0 + per_t);
+      int cnt = 0;
+      for (int x = x0; x < x1; ++x) {
+        const int uu = x / a.n_rg, g = x % a.n_rg;
+        const uint32_t m =
+            static_cast<uint32_t>(a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + u_list[uu]]);
+        msk[x] = m;
+        cnt += __popc(m);
+      }
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      if (lane == 31) red_i[warp] = incl;
+      __syncthreads();
+      int run = incl - cnt, total = 0;
+      for (int i = 0; i < nw; ++i) {
+        if (i < warp) run += red_i[i];
+        total += red_i[i];
+      }
+      for (int x = x0; x < x1; ++x) {
+        pfx[x] = run;
+        run += __popc(msk[x]);
+      }
+      __syncthreads();
+      for (int t = gw; t < total; t += n_gw) {
+        int l0 = 0, l1 = npair - 1;   // the last pair whose first task is <= t
+        while (l0 < l1) {
+          const int mid = (l0 + l1 + 1) >> 1;
+          if (pfx[mid] <= t) l0 = mid;
+          else l1 = mid - 1;
+        }
+        uint32_t bits = msk[l0];
+        for (int j = t - pfx[l0]; j > 0; --j) bits &= bits - 1;
+        const int uu = l0 / a.n_rg, r = (l0 % a.n_rg) * kTR + __ffs(bits) - 1;
+        const int ph = ph_s[uu];
+        if (ph < 0) continue;
+        const int tt = r / a.Hq, h = r % a.Hq;
+        const double e = exact_row_dot(a.q + b * a.qs0 + tt * a.qs1 + h * a.qs2,
+                                       a.sig + (int64_t)ph * a.Dk, a.Dk);
         if (lane == 0) atomicMax(&exk[uu], d2key(e));
+      }
+    } else {
+      __syncthreads();
+      for (int x = gw; x < npair; x += n_gw) {
+        const int uu = x / a.n_rg, g = x % a.n_rg;
+        const int ph = ph_s[uu];
+        if (ph < 0) continue;
+        unsigned long long bits = a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + u_list[uu]];
+        const uint16_t* sg = a.sig + (int64_t)ph * a.Dk;
+        while (bits) {
+          const int r = g * kTR + __ffsll(static_cast<long long>(bits)) - 1;
+          bits &= bits - 1;
+          const int tt = r / a.Hq, h = r % a.Hq;
+          const double e = exact_row_dot(a.q + b * a.qs0 + tt * a.qs1 + h * a.qs2, sg, a.Dk);
+          if (lane == 0) atomicMax(&exk[uu], d2key(e));
+        }
       }
     }
     __threadfence();
     __syncthreads();
-    if (tid == 0) last_s = atomicAdd(&a.counter[b], 1u) == kChooseCtas - 1;
+    if (tid == 0) last_s = atomicAdd(&a.counter[b], 1u) == static_cast<unsigned>(n_cta - 1);
     __syncthreads();
     if (!last_s) return;
     __threadfence();
     for (int i = tid; i < nu_; i += blockDim.x) {
       const unsigned long long k = __ldcg(&exk[i]);
-      const int ph = ptrow[u_list[i]];
-      ex[i] = (ph < 0 || ph >= a.P_pool || k == 0ull) ? -INFINITY : key2d(k);
+      ex[i] = (ph_s[i] < 0 || k == 0ull) ? -INFINITY : key2d(k);
     }
     __syncthreads();
     // per boundary: the undecided pages fill the slots the certain ones left
-    for (int i = 0; i < 2; ++i) {
-      const uint8_t in_bit = 1u << i, unc_bit = 4u << i;
-      const int slots = kb[i] - n_cert[i];
-      for (int u = tid; u < nu_; u += blockDim.x) {
-        const int pu = u_list[u];
-        if (!(flag[pu] & unc_bit)) continue;
-        const double su = ex[u];
-        int rank = 0;
-        for (int v = 0; v < nu_; ++v) {
-          const int pv = u_list[v];
-          if (!(flag[pv] & unc_bit)) continue;
-          const double sv = ex[v];
-          rank += (sv > su) || (sv == su && pv < pu);
-        }
-        if (rank < slots) flag[pu] |= in_bit;
+    for (int u = tid; u < nu_; u += blockDim.x) {
+      const int pu = u_list[u];
+      const uint8_t fu = flag[pu];
+      const double su = ex[u];
+      int rank[2] = {0, 0};
+      for (int v = 0; v < nu_; ++v) {
+        const int pv = u_list[v];
+        const uint8_t fv = flag[pv];
+        const double sv = ex[v];
+        const int ahead = (sv > su) || (sv == su && pv < pu);
+        rank[0] += ahead & (fv >> 2);
+        rank[1] += ahead & (fv >> 3);
       }
-      __syncthreads();
+      uint8_t add = 0;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        if (((fu >> (2 + i)) & 1u) && rank[i] < kb[i] - n_cert[i]) add |= 1u << i;
+      if (add) flag[pu] = fu | add;
     }
+    __syncthreads();
   }
   const int c0 = compact_pages(flag, N, 1u, out0, cap, red_i);
   const int c1 = compact_pages(flag, N, 2u, out1, cap, red_i);
@@ -470,20 +540,24 @@ cudaError_t launch_select_tiered(TieredArgs a, cudaStream_t stream) {
   a.rmask = reinterpret_cast<unsigned long long*>(a.lohi + nl);
   a.exkey = a.rmask + nl;
   a.counter = reinterpret_cast<unsigned int*>(a.exkey + (size_t)a.B * a.max_pages);
-  const int RS = ((a.Dk + 15) & ~15) * 2 + 16;
-  const int dyn1 = (kTP + kTR) * RS;
+  const int dyn1 = kSStages * kSStageBytes + 1024;   // + alignment slack
   cudaError_t e = cudaFuncSetAttribute(tiered_score_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, dyn1);
   if (e != cudaSuccess) return e;
-  dim3 g1((a.max_pages + kTP - 1) / kTP, a.n_rg, a.B);
-  e = launch_pdl(tiered_score_kernel, g1, dim3(kTScoreThreads), dyn1, stream, a);
+  dim3 g1((a.max_pages + kSP - 1) / kSP, (a.T * a.Hq + kSR - 1) / kSR, a.B);
+  e = launch_pdl(tiered_score_kernel, g1, dim3(kSThreads), dyn1, stream, a);
   if (e != cudaSuccess) return e;
-  const size_t dyn2 = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
+  const size_t dyn2 = (size_t)a.max_pages * (4 + 4 + 4 + 2 + 1) + 16;
   e = cudaFuncSetAttribute(tiered_choose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn2);
   if (e != cudaSuccess) return e;
-  return launch_pdl(tiered_choose_kernel, dim3(a.B, kChooseCtas), dim3(kChooseThreads), dyn2,
-                    stream, a);
+  // enough CTAs per sequence to spread the exact rescoring over the SMs
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const int n_cta = std::max(1, std::min(kChooseCtas, sms / std::max(1, a.B)));
+  return launch_pdl(tiered_choose_kernel, dim3(a.B, n_cta), dim3(kChooseThreads), dyn2, stream, a);
 }
 
 }  // namespace sa

@@ -191,6 +191,30 @@ def test_select_long_all_ties():
     assert list(rp[1, 0, :n_sink + k]) == list(range(n_sink + k))
 
 
+def test_select_workspace_contents_do_not_matter():
+    # The selection workspace has no initial contents to rely on: a workspace
+    # full of random bytes, reused over several calls, gives the oracle's
+    # selection every time.
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=3, seq_len_lo=8192, seq_len_hi=8192)
+    inp, g = gqa_case(cfg, seed=21)
+    sig = oracle_summaries(inp, cfg)
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    max_pages = g["page_table"].shape[1]
+    n = sa.sa_select_workspace_size(cfg.B, cfg.Hkv, max_pages)
+    gen = torch.Generator(device=DEV)
+    gen.manual_seed(5)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, device=DEV, generator=gen)
+    sigd = to_bf16_dev(sig)
+    for _ in range(3):
+        pages, counts = sa.sa_select_pages(g["q"], sigd, g["page_table"], g["seq_lens"],
+                                           cfg.page_size, cfg.sink_tokens, cfg.local_tokens,
+                                           cfg.budget_tokens, workspace=ws)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(np_i32(counts), rc)
+        np.testing.assert_array_equal(np_i32(pages), rp)
+
+
 def _random_bf16_bits(rng, shape, e_lo, e_hi, p_sub=0.03, p_zero=0.03):
     """bf16 bit patterns: random sign and fraction, exponent field uniform in
     [e_lo, e_hi]; a share of subnormals and zeros."""
@@ -224,7 +248,9 @@ def test_select_score_brackets_hold(T, Hq, Hkv):
                                        cfg.page_size, cfg.sink_tokens, cfg.local_tokens,
                                        cfg.budget_tokens, workspace=ws)
     torch.cuda.synchronize()
-    lohi = ws.view(torch.float32).cpu().numpy().reshape(cfg.B, Hkv, max_pages, 2).astype(np.float64)
+    n_bounds = cfg.B * Hkv * max_pages * 2
+    lohi = (ws.view(torch.float32)[:n_bounds].cpu().numpy()
+            .reshape(cfg.B, Hkv, max_pages, 2).astype(np.float64))
     n_sink, n_local, budget_pages, _ = O.page_budget(cfg.sink_tokens, cfg.local_tokens,
                                                      cfg.budget_tokens, cfg.page_size)
     q = O.bf16_to_f64(qb)
