@@ -195,22 +195,32 @@ __host__ __device__ __forceinline__ double i128_to_double_rn(I128 v, int e0) {
 
 #ifdef __CUDACC__
 // RN64(sum_d a[d] * b[d]) for two bf16 rows of n elements (n % 8 == 0, both
-// 16-byte aligned, n <= 256 kMaxC), computed by all 32 lanes of a warp (each
-// loads its 16-byte chunks once); every lane returns the result.
+// 16-byte aligned, n <= 256 kMaxC <= 1024), computed by all 32 lanes of a warp
+// (each loads its 16-byte chunks once); every lane returns the result.  The
+// exponent span of the nonzero products picks the method: up to 26 bits a
+// float64 sum that never rounds, up to 100 bits a signed 128-bit fixed-point
+// sum anchored at the smallest exponent, beyond that the superaccumulator.
 template <int kMaxC>   // 16-byte chunks per lane: n <= 256 kMaxC
 __device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const uint16_t* b, int n) {
+  static_assert(kMaxC >= 1 && kMaxC <= 4, "n <= 1024 keeps the float64 path exact");
   const int lane = threadIdx.x & 31;
   const uint4* a4 = reinterpret_cast<const uint4*>(a);
   const uint4* b4 = reinterpret_cast<const uint4*>(b);
   const int nc = n >> 3;
+  if (nc == 0) return 0.0;
   uint4 xs[kMaxC], ys[kMaxC];
+  // every load is issued unconditionally (index clamped, zeroed afterwards), so
+  // all of them are in flight together instead of one round trip each
 #pragma unroll
   for (int j = 0; j < kMaxC; ++j) {
-    const int c = lane + 32 * j;
-    xs[j] = c < nc ? a4[c] : make_uint4(0, 0, 0, 0);
-    ys[j] = c < nc ? b4[c] : make_uint4(0, 0, 0, 0);
+    const int c = min(lane + 32 * j, nc - 1);
+    xs[j] = a4[c];
+    ys[j] = b4[c];
   }
-  // pass 1: exponent range of the nonzero products
+#pragma unroll
+  for (int j = 0; j < kMaxC; ++j)
+    if (lane + 32 * j >= nc) xs[j] = ys[j] = make_uint4(0, 0, 0, 0);
+  // pass 1: exponent range of the nonzero products (selects, no branches)
   int emin = 1 << 20, emax = -(1 << 20);
 #pragma unroll
   for (int j = 0; j < kMaxC; ++j) {
@@ -223,10 +233,9 @@ __device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const u
       bool na, nb;
       bf16_fields((xa[i >> 1] >> (16 * (i & 1))) & 0xffffu, ma, ea, na);
       bf16_fields((ya[i >> 1] >> (16 * (i & 1))) & 0xffffu, mb, eb, nb);
-      if (ma && mb) {
-        emin = min(emin, ea + eb);
-        emax = max(emax, ea + eb);
-      }
+      const bool nz = (ma != 0u) & (mb != 0u);
+      emin = min(emin, nz ? ea + eb : (1 << 20));
+      emax = max(emax, nz ? ea + eb : -(1 << 20));
     }
   }
 #pragma unroll
@@ -235,6 +244,29 @@ __device__ __forceinline__ double warp_exact_dot_bf16(const uint16_t* a, const u
     emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
   }
   if (emax < emin) return 0.0;          // every product is zero
+  if (emax - emin <= 26) {
+    // Narrow span: every product is an integer multiple of 2^emin below
+    // 2^(emax + 16), so every partial sum of at most 1024 of them is a
+    // multiple of 2^emin smaller than 2^(emin + 52): float64 represents all
+    // of them, and fma(x, y, acc) (x*y exact: 16 significant bits) never
+    // rounds.  The float64 sum is the exact sum.
+    double acc = 0.0;
+#pragma unroll
+    for (int j = 0; j < kMaxC; ++j) {
+      const uint32_t xa[4] = {xs[j].x, xs[j].y, xs[j].z, xs[j].w};
+      const uint32_t ya[4] = {ys[j].x, ys[j].y, ys[j].z, ys[j].w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc = fma(static_cast<double>(__uint_as_float(xa[i] << 16)),
+                  static_cast<double>(__uint_as_float(ya[i] << 16)), acc);
+        acc = fma(static_cast<double>(__uint_as_float(xa[i] & 0xffff0000u)),
+                  static_cast<double>(__uint_as_float(ya[i] & 0xffff0000u)), acc);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    return acc;
+  }
   if (emax - emin > 100) {              // wide span: superaccumulator, lane 0
     double r = 0.0;
     if (lane == 0) r = exact_dot_bf16(a, 1, b, n);

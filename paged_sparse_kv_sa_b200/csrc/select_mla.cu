@@ -37,12 +37,13 @@ constexpr int kChooseCtas = 16;    // at most this many CTAs per sequence share 
 // Scores of 128 pages x 128 query rows of one sequence, S = sigma q^T, on the
 // tensor cores: tcgen05.mma (M = 128 pages, N = 128 rows, K = 16 per
 // instruction, bf16 in, float32 accumulation in tensor memory) over the Dk
-// features in chunks of 64 (one 128-byte swizzle row).  Warps 0-3 gather the
+// features in chunks of 64 (one 128-byte swizzle row).  Warps 0-7 gather the
 // chunk's summary rows (through the page table) and query rows with 16-byte
 // cp.async copies straight into the 128-byte-swizzled K-major layout of a
-// kSStages-deep ring, and sum each row's squares from their own copies; warp 4
-// allocates the tensor memory and issues the MMAs; warps 0-3 then read one
-// page (TMEM lane) each.  Per (page, row) the exact score lies in s -/+ E with
+// kSStages-deep ring, and sum each row's squares from their own copies (packed
+// float32 pairs); warp 8 allocates the tensor memory and issues the MMAs;
+// warps 0-7 then read the accumulator, one page (TMEM lane) and half of the
+// rows per thread.  Per (page, row) the exact score lies in s -/+ E with
 // (directed rounding)
 //   E = c_acc ||q_r|| ||sigma|| + 2^-126 sqrt(Dk) (||q_r|| + ||sigma||) + Dk 2^-124,
 // c_acc = Dk 2^-20: the accumulation of each 16-product step loses less than
@@ -61,9 +62,18 @@ constexpr int kSLag = kSStages - 1;          // chunks a loader keeps in flight
 constexpr int kSChunk = 64;                  // features per K chunk
 constexpr int kSTile = kSP * 128;            // bytes of one operand's chunk (16 KB)
 constexpr int kSStageBytes = 2 * kSTile;     // summaries, then query rows
-constexpr int kSThreads = 160;
+constexpr int kSLoaders = 8 * 32;            // warps 0-7: loads, norms, epilogue
+constexpr int kSThreads = kSLoaders + 32;     // warp 8: MMA issue
 constexpr uint32_t kSIdesc = tc::idesc_bf16_f32(kSP, kSR, false, false);
-static_assert(kSR % kTR == 0, "row groups tile the CTA's rows");
+static_assert(kSR == 4 * kTR && kSP == 128, "epilogue: 4 TMEM lane quarters x 2 halves of 2 row groups");
+
+// acc + (x0^2, x1^2) for the two bf16 of w, as packed float32 (x0 = low half).
+SA_DEV unsigned long long fma2_sq(uint32_t w, unsigned long long acc) {
+  const unsigned long long x =
+      (static_cast<unsigned long long>(w & 0xffff0000u) << 32) | static_cast<unsigned long long>(w << 16);
+  asm("fma.rn.f32x2 %0, %1, %1, %0;" : "+l"(acc) : "l"(x));
+  return acc;
+}
 
 __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const TieredArgs a) {
   pdl_wait_and_release();
@@ -83,37 +93,37 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
   uint8_t* ring = tsm_raw + ((1024 - (smem_u32(tsm_raw) & 1023)) & 1023);
   __shared__ uint64_t full[kSStages], empty[kSStages], mma_done;
   __shared__ uint32_t tmem_s;
-  __shared__ float sn_s[kSP];          // ||sigma_p||, rounded up
-  __shared__ float cq_s[kSR];          // c_acc ||q_r||, rounded up
-  __shared__ float fq_s[kSR];          // 2^-126 sqrt(Dk) ||q_r||, rounded up
+  __shared__ float sn_s[kSP];                    // ||sigma_p||, rounded up
+  __shared__ __align__(16) float cq_s[kSR];      // c_acc ||q_r||, rounded up
+  __shared__ __align__(16) float fq_s[kSR];      // 2^-126 sqrt(Dk) ||q_r||, rounded up
   __shared__ int8_t pok_s[kSP];        // page readable
   if (tid == 0) {
     for (int s = 0; s < kSStages; ++s) {
-      mbar_init(&full[s], 4 * 32);
+      mbar_init(&full[s], kSLoaders);
       mbar_init(&empty[s], 1);
     }
     mbar_init(&mma_done, 1);
     fence_mbar_init();
   }
-  if (warp == 4) tc::tmem_alloc(&tmem_s, kSR);
+  if (warp == 8) tc::tmem_alloc(&tmem_s, kSR);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = tmem_s;
   const uint32_t ring_u = smem_u32(ring);
 
-  if (warp < 4) {
-    // this thread: 16-byte unit j of every chunk, rows rb + 16 i (i < 8) of
+  if (warp < 8) {
+    // this thread: 16-byte unit j of every chunk, rows rb + 32 i (i < 4) of
     // both operands; in the swizzled layout row rr's unit j sits at
     // (rr / 8) * 1024 + (rr % 8) * 128 + ((j ^ (rr % 8)) * 16), and rr % 8 = rb % 8
     const int j = tid & 7, rb = tid >> 3;
     const uint32_t soff = (rb >> 3) * 1024 + (rb & 7) * 128 + ((j ^ (rb & 7)) << 4);
     const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
-    const uint16_t* arow[8];
-    const uint16_t* brow[8];
+    const uint16_t* arow[4];
+    const uint16_t* brow[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int p = p0 + rb + 16 * i, r = r0 + rb + 16 * i;
+    for (int i = 0; i < 4; ++i) {
+      const int p = p0 + rb + 32 * i, r = r0 + rb + 32 * i;
       int ph = -1;
       if (p < N) {
         ph = ptrow[p];
@@ -122,13 +132,14 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
           ph = -1;
         }
       }
-      if (j == 0) pok_s[rb + 16 * i] = ph >= 0;
+      if (j == 0) pok_s[rb + 32 * i] = ph >= 0;
       arow[i] = ph >= 0 ? a.sig + (int64_t)ph * Dk : nullptr;
       brow[i] = r < R ? a.q + b * a.qs0 + (r / a.Hq) * a.qs1 + (r % a.Hq) * a.qs2 : nullptr;
     }
-    float sa2[8], sb2[8];
+    // sums of squares as packed float32 pairs (even, odd features)
+    unsigned long long sa2[4], sb2[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) sa2[i] = sb2[i] = 0.f;
+    for (int i = 0; i < 4; ++i) sa2[i] = sb2[i] = 0ull;
     for (int kc = 0; kc < KC + kSLag; ++kc) {
       if (kc < KC) {
         const int s = kc % kSStages;
@@ -137,10 +148,10 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
         const int f0 = kc * kSChunk + 8 * j;      // Dk % 8 == 0: a unit is all in or all out
         const uint32_t da = ring_u + s * kSStageBytes + soff;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
           const bool va = arow[i] != nullptr && f0 < Dk, vb = brow[i] != nullptr && f0 < Dk;
-          cp_async16(da + 2048 * i, va ? arow[i] + f0 : a.sig, va ? 16u : 0u);
-          cp_async16(da + kSTile + 2048 * i, vb ? brow[i] + f0 : a.q, vb ? 16u : 0u);
+          cp_async16(da + 4096 * i, va ? arow[i] + f0 : a.sig, va ? 16u : 0u);
+          cp_async16(da + kSTile + 4096 * i, vb ? brow[i] + f0 : a.q, vb ? 16u : 0u);
         }
       }
       cp_async_commit();          // (empty groups past the end keep the count uniform)
@@ -149,16 +160,14 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
         const int s = (kc - kSLag) % kSStages;
         const uint8_t* src = ring + s * kSStageBytes + soff;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 x = *reinterpret_cast<const uint4*>(src + 2048 * i);
-          const uint4 y = *reinterpret_cast<const uint4*>(src + kSTile + 2048 * i);
+        for (int i = 0; i < 4; ++i) {
+          const uint4 x = *reinterpret_cast<const uint4*>(src + 4096 * i);
+          const uint4 y = *reinterpret_cast<const uint4*>(src + kSTile + 4096 * i);
           const uint32_t xw[4] = {x.x, x.y, x.z, x.w}, yw[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float x0 = __uint_as_float(xw[e] << 16), x1 = __uint_as_float(xw[e] & 0xffff0000u);
-            const float y0 = __uint_as_float(yw[e] << 16), y1 = __uint_as_float(yw[e] & 0xffff0000u);
-            sa2[i] = fmaf(x0, x0, fmaf(x1, x1, sa2[i]));
-            sb2[i] = fmaf(y0, y0, fmaf(y1, y1, sb2[i]));
+            sa2[i] = fma2_sq(xw[e], sa2[i]);
+            sb2[i] = fma2_sq(yw[e], sb2[i]);
           }
         }
         tc::fence_proxy_async();   // the copies are read by the tensor core
@@ -166,48 +175,61 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
       }
     }
     // row norms: the 8 lanes of a row group hold its 8 feature slices
+    float na[4], nb[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i) {
+      na[i] = __uint_as_float(static_cast<uint32_t>(sa2[i])) +
+              __uint_as_float(static_cast<uint32_t>(sa2[i] >> 32));
+      nb[i] = __uint_as_float(static_cast<uint32_t>(sb2[i])) +
+              __uint_as_float(static_cast<uint32_t>(sb2[i] >> 32));
 #pragma unroll
       for (int o = 1; o < 8; o <<= 1) {
-        sa2[i] += __shfl_xor_sync(0xffffffffu, sa2[i], o);
-        sb2[i] += __shfl_xor_sync(0xffffffffu, sb2[i], o);
+        na[i] += __shfl_xor_sync(0xffffffffu, na[i], o);
+        nb[i] += __shfl_xor_sync(0xffffffffu, nb[i], o);
       }
+    }
     const float pad = 1.f + 2.f * Dk * 5.96046448e-8f;
     const float c_acc = Dk * 9.5367431640625e-07f;                                 // Dk 2^-20
     const float rt_d = __fmul_ru(__fsqrt_ru(static_cast<float>(Dk)), 1.1754943508222875e-38f);
     if (j == 0)
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int rr = rb + 16 * i;
-        sn_s[rr] = __fmul_ru(__fsqrt_ru(__fmul_ru(sa2[i], pad)), 1.0000002f);
-        const float qn = __fmul_ru(__fsqrt_ru(__fmul_ru(sb2[i], pad)), 1.0000002f);
+      for (int i = 0; i < 4; ++i) {
+        const int rr = rb + 32 * i;
+        sn_s[rr] = __fmul_ru(__fsqrt_ru(__fmul_ru(na[i], pad)), 1.0000002f);
+        const float qn = __fmul_ru(__fsqrt_ru(__fmul_ru(nb[i], pad)), 1.0000002f);
         cq_s[rr] = __fmul_ru(c_acc, qn);
         fq_s[rr] = __fmul_ru(rt_d, qn);
       }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    // epilogue: thread = page p0 + tid = TMEM lane tid
+    asm volatile("bar.sync 1, %0;" ::"n"(kSLoaders) : "memory");
+    // epilogue: thread = page p0 + 32 (warp % 4) + lane = TMEM lane, row
+    // groups 2 (warp / 4) and 2 (warp / 4) + 1
     if (!mbar_wait_bounded(&mma_done, 0)) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
     tc::fence_after_sync();
-    const int p = p0 + tid;
-    const bool pok = pok_s[tid] != 0;
-    const float sn = sn_s[tid];
+    const int pl = 32 * (warp & 3) + lane, p = p0 + pl;
+    const bool pok = pok_s[pl] != 0;
+    const float sn = sn_s[pl];
     const float es = __fadd_ru(__fmul_ru(rt_d, sn), Dk * 4.70197740328915e-38f);   // + Dk 2^-124
-    for (int g = 0; g < kSR / kTR && r0 + g * kTR < R; ++g) {
+    for (int g = 2 * (warp >> 2); g < 2 * (warp >> 2) + 2 && r0 + g * kTR < R; ++g) {
       float sv[32];
-      tc::ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + g * kTR, sv);
+      tc::ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + g * kTR, sv);
       tc::wait_ld();
+      // (no branch per row: a conditional shared load per element would
+      // serialise the loop; rows past R are masked by selects)
+      const int nv = R - (r0 + g * kTR);   // valid rows of the group (>= 1)
       float lo = -INFINITY, hi = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const int rr = g * kTR + c;
-        if (r0 + rr < R) {
-          const float E = __fadd_ru(__fmul_ru(cq_s[rr], sn), __fadd_ru(fq_s[rr], es));
-          lo = fmaxf(lo, __fsub_rd(sv[c], E));
-          sv[c] = __fadd_ru(sv[c], E);
+      for (int c4 = 0; c4 < 32; c4 += 4) {
+        const float4 cq = *reinterpret_cast<const float4*>(cq_s + g * kTR + c4);
+        const float4 fq = *reinterpret_cast<const float4*>(fq_s + g * kTR + c4);
+        const float cqa[4] = {cq.x, cq.y, cq.z, cq.w}, fqa[4] = {fq.x, fq.y, fq.z, fq.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c4 + e;
+          const float E = __fadd_ru(__fmul_ru(cqa[e], sn), __fadd_ru(fqa[e], es));
+          const float l = __fsub_rd(sv[c], E), h = __fadd_ru(sv[c], E);
+          lo = fmaxf(lo, c < nv ? l : -INFINITY);
+          sv[c] = c < nv ? h : -INFINITY;
           hi = fmaxf(hi, sv[c]);
-        } else {
-          sv[c] = -INFINITY;
         }
       }
       uint32_t m = 0;
@@ -238,20 +260,21 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kSR);
   }
 }
 
-// Block-wide ascending compaction of the pages whose flag has `bit` set.
-SA_DEV int compact_pages(const uint8_t* flag, int N, uint8_t bit, int32_t* out, int cap,
-                         int* red_i) {
-  const int tid = threadIdx.x;
+// Block-wide ascending compaction of the pages whose flag has bit 1 (into
+// out0) and bit 2 (into out1), each padded with -1 to cap; one pass, one scan.
+SA_DEV void compact_pages2(const uint8_t* flag, int N, int32_t* out0, int32_t* out1, int cap,
+                           int* red_i, int& c0, int& c1) {
+  const int tid = threadIdx.x, nw = blockDim.x / 32;
   const int per_t = (N + blockDim.x - 1) / blockDim.x;
   const int p0 = tid * per_t, p1 = min(N, p0 + per_t);
-  int cnt = 0;
-  for (int p = p0; p < p1; ++p) cnt += (flag[p] & bit) != 0;
+  int cnt = 0;   // low 16 bits: bit 1 pages, high 16 bits: bit 2 pages
+  for (int p = p0; p < p1; ++p) cnt += (flag[p] & 1u) + ((flag[p] & 2u) << 15);
   const int w = tid >> 5, lane = tid & 31;
   int incl = cnt;
   for (int o = 1; o < 32; o <<= 1) {
@@ -261,16 +284,20 @@ SA_DEV int compact_pages(const uint8_t* flag, int N, uint8_t bit, int32_t* out, 
   if (lane == 31) red_i[w] = incl;
   __syncthreads();
   int wbase = 0, total = 0;
-  for (int i = 0; i < (int)(blockDim.x / 32); ++i) {
+  for (int i = 0; i < nw; ++i) {
     if (i < w) wbase += red_i[i];
     total += red_i[i];
   }
-  int pos = wbase + incl - cnt;
-  for (int p = p0; p < p1; ++p)
-    if ((flag[p] & bit) && pos < cap) out[pos++] = p;
-  for (int i = total + tid; i < cap; i += blockDim.x) out[i] = -1;
-  __syncthreads();   // red_i is reused by the next call
-  return min(total, cap);
+  int pos0 = (wbase + incl - cnt) & 0xffff, pos1 = (wbase + incl - cnt) >> 16;
+  for (int p = p0; p < p1; ++p) {
+    if ((flag[p] & 1u) && pos0 < cap) out0[pos0++] = p;
+    if ((flag[p] & 2u) && pos1 < cap) out1[pos1++] = p;
+  }
+  c0 = min(total & 0xffff, cap);
+  c1 = min(total >> 16, cap);
+  for (int i = c0 + tid; i < cap; i += blockDim.x) out0[i] = -1;
+  for (int i = c1 + tid; i < cap; i += blockDim.x) out1[i] = -1;
+  __syncthreads();   // red_i is reused by the caller
 }
 
 // Block-wide ascending list (in shared memory) of the pages whose flag has any
@@ -344,11 +371,10 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   for (int p = tid; p < N; p += blockDim.x) {
     float l = -INFINITY, h = -INFINITY;
     for (int rg0 = 0; rg0 < a.n_rg; rg0 += 8) {
-      float2 v[8];
+      float2 v[8];   // (index clamped: the loads are unconditional; a repeat does not change a max)
 #pragma unroll
       for (int j = 0; j < 8; ++j)
-        v[j] = rg0 + j < a.n_rg ? a.lohi[((int64_t)b * a.n_rg + rg0 + j) * a.max_pages + p]
-                                : make_float2(-INFINITY, -INFINITY);
+        v[j] = a.lohi[((int64_t)b * a.n_rg + min(rg0 + j, a.n_rg - 1)) * a.max_pages + p];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         l = fmaxf(l, v[j].x);
@@ -515,8 +541,8 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     }
     __syncthreads();
   }
-  const int c0 = compact_pages(flag, N, 1u, out0, cap, red_i);
-  const int c1 = compact_pages(flag, N, 2u, out1, cap, red_i);
+  int c0, c1;
+  compact_pages2(flag, N, out0, out1, cap, red_i, c0, c1);
   if (tid == 0) {
     a.counts[2 * b] = c0;
     a.counts[2 * b + 1] = c1;
