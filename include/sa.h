@@ -238,7 +238,8 @@ SA_API int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const
  *  o_out      (dev, optional) [rows,Dv] float32
  *  o_out_bf16 (dev, optional) [rows,Dv] bf16 (round to nearest even)
  *  lse_out    (dev, optional) [rows] float32
- * At least one output must be given.  Dv % 4 == 0.
+ * At least one output must be given.  Dv % 4 == 0.  Limits: n_splits <= 64
+ * and rows * Dv / 4 < 2^32 (SA_ERR_UNSUPPORTED otherwise).
  */
 SA_API int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,
                int Dv, float* o_out, uint16_t* o_out_bf16, float* lse_out, void* stream);

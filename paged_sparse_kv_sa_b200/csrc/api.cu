@@ -332,7 +332,7 @@ int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, i
   if (!aligned16(o_partial) || (o_out && !aligned16(o_out)) ||
       (o_out_bf16 && (reinterpret_cast<uintptr_t>(o_out_bf16) & 7u)))
     return SA_ERR_INVALID_ARG;
-  if (n_splits > 64) return SA_ERR_UNSUPPORTED;
+  if (n_splits > 64 || rows * (Dv / 4) >= (int64_t(1) << 32)) return SA_ERR_UNSUPPORTED;
   if (rows == 0) return SA_OK;
   return cuda_status(launch_combine(o_partial, lse_partial, n_splits, rows, Dv, o_out, o_out_bf16,
                                     lse_out, static_cast<cudaStream_t>(stream)));

@@ -14,16 +14,30 @@ namespace {
 constexpr int kCombineBatch = 8;   // splits whose loads are in flight together (many splits)
 constexpr int kRegSplits = 16;     // up to this many splits: every load of a phase at once
 
+// 16-byte load that happens only when `pred` holds (a predicated instruction,
+// not a branch: a run of them is issued back to back); zeros otherwise.
+SA_DEV float4 ld4_if(const float* p, bool pred) {
+  float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+  asm volatile(
+      "{\n .reg .pred q;\n setp.ne.b32 q, %5, 0;\n"
+      " @q ld.global.nc.v4.f32 {%0, %1, %2, %3}, [%4];\n}\n"
+      : "+f"(v.x), "+f"(v.y), "+f"(v.z), "+f"(v.w)
+      : "l"(p), "r"(static_cast<int>(pred)));
+  return v;
+}
+
 __global__ void __launch_bounds__(128)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    int n_splits, int64_t rows, int Dv, float* __restrict__ o_out,
                    uint16_t* __restrict__ o_bf16, float* __restrict__ lse_out) {
   pdl_wait_and_release();
-  const int q4 = Dv / 4;
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= rows * q4) return;
-  const int64_t row = idx / q4;
-  const int c = (int)(idx % q4) * 4;
+  // (32-bit index arithmetic: the launcher guarantees rows * Dv / 4 < 2^32)
+  const uint32_t q4 = static_cast<uint32_t>(Dv) / 4u;
+  const uint32_t idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= static_cast<uint32_t>(rows) * q4) return;
+  const uint32_t row_ = idx / q4;
+  const int64_t row = row_;
+  const int c = static_cast<int>(idx - row_ * q4) * 4;
   // The split LSEs first, then the O rows of the splits that have keys (a
   // split without keys is not read at all); with up to kRegSplits splits every
   // load of a phase is issued before any is used.
@@ -32,17 +46,19 @@ __global__ void __launch_bounds__(128)
   if (n_splits <= kRegSplits) {
     float w[kRegSplits];
 #pragma unroll
-    for (int s = 0; s < kRegSplits; ++s)
-      w[s] = s < n_splits ? __ldg(lse_part + s * rows + row) : -INFINITY;
+    for (int s = 0; s < kRegSplits; ++s)   // (index clamped: unconditional loads)
+      w[s] = __ldg(lse_part + min(s, n_splits - 1) * rows + row);
 #pragma unroll
-    for (int s = 0; s < kRegSplits; ++s) m = fmaxf(m, w[s]);
+    for (int s = 0; s < kRegSplits; ++s) {
+      if (s >= n_splits) w[s] = -INFINITY;
+      m = fmaxf(m, w[s]);
+    }
     if (m != -INFINITY) {
       float4 v[kRegSplits];
 #pragma unroll
       for (int s = 0; s < kRegSplits; ++s) {
         w[s] = __expf(w[s] - m);
-        v[s] = w[s] > 0.f ? *reinterpret_cast<const float4*>(o_part + (s * rows + row) * Dv + c)
-                          : make_float4(0.f, 0.f, 0.f, 0.f);
+        v[s] = ld4_if(o_part + (s * rows + row) * Dv + c, w[s] > 0.f);
       }
 #pragma unroll
       for (int s = 0; s < kRegSplits; ++s) {
@@ -71,8 +87,7 @@ __global__ void __launch_bounds__(128)
           w[i] = s0 + i < n_splits ? __expf(__ldg(lse_part + (s0 + i) * rows + row) - m) : 0.f;
 #pragma unroll
         for (int i = 0; i < kCombineBatch; ++i)
-          v[i] = w[i] > 0.f ? *reinterpret_cast<const float4*>(o_part + ((s0 + i) * rows + row) * Dv + c)
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+          v[i] = ld4_if(o_part + ((s0 + i) * rows + row) * Dv + c, w[i] > 0.f);
 #pragma unroll
         for (int i = 0; i < kCombineBatch; ++i) {
           tot += w[i];
@@ -109,6 +124,7 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
                            cudaStream_t stream) {
   const int64_t n = rows * (Dv / 4);
   if (n == 0) return cudaSuccess;
+  if (n >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   const int threads = 128;
   const int64_t blocks = (n + threads - 1) / threads;
   return launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, o_part,
