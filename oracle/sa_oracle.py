@@ -39,6 +39,11 @@ Readings where the pages are silent (each also listed in the design notes):
      tokens, no forced pages; critical = rank < alpha, ambient = next beta.
   R8 block union: sink block(s) + the Q-block's diagonal block + the top_k of
      the blocks strictly between them, by (score desc, index asc).
+  R15 quantized KV pages ([UAE] "Key Design Decisions" 2: cache format
+     (paged, block-sparse, quantized); "Roadmap": quantized KV cache support):
+     K and V pages stored as FP8 E4M3 codes with one float32 scale per
+     (physical page, kv head); a key is e4m3(code) * scale, likewise a value.
+     Attention and summaries are those of the dequantized pages.
 """
 from __future__ import annotations
 
@@ -47,9 +52,10 @@ import math
 import numpy as np
 
 __all__ = [
-    "bf16_to_f64", "f64_to_bf16_rne", "page_budget", "exact_dots", "page_summaries",
-    "page_scores", "rank_select", "select_pages", "select_pages_mla", "sparse_attention",
-    "masked_dense_attention", "combine", "block_union", "NEG_INF",
+    "bf16_to_f64", "f64_to_bf16_rne", "e4m3_to_f64", "page_budget", "exact_dots",
+    "page_summaries", "page_summaries_fp8", "page_scores", "rank_select", "select_pages",
+    "select_pages_mla", "sparse_attention", "sparse_attention_fp8", "masked_dense_attention",
+    "combine", "block_union", "NEG_INF",
 ]
 
 NEG_INF = float("-inf")
@@ -79,6 +85,29 @@ def f64_to_bf16_rne(x) -> np.ndarray:
     if np.any(np.abs(r) > 3.3895313892515355e38):
         raise OverflowError("value outside the bf16 range")
     return (r.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 -> float64 (R15): 1 sign, 4 exponent (bias 7), 3 fraction bits;
+# exponent field 0 holds the subnormals 2^-6 * f/8; S.1111.111 is NaN; no
+# infinities (largest finite value 1.75 * 2^8 = 448)
+# --------------------------------------------------------------------------
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Exact value of FP8 E4M3 codes (NaN for the two NaN codes)."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    f = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, np.ldexp(f / 8.0, -6), np.ldexp(1.0 + f / 8.0, e - 7))
+    mag = np.where((c & 0x7F) == 0x7F, np.nan, mag)
+    return sign * mag
+
+
+def _dequant(codes, scale, phys, kvh):
+    """float64 values of pages `phys` of kv head `kvh`: e4m3(code) * scale (R15).
+    Each product is exact in float64 (4 x 24 significant bits)."""
+    return e4m3_to_f64(codes[phys, kvh]) * np.asarray(scale, dtype=np.float32)[phys, kvh].astype(
+        np.float64)[..., None, None]
 
 
 # --------------------------------------------------------------------------
@@ -160,9 +189,30 @@ def page_summaries(k_bits, page_table, seq_lens, page_size: int, units=None) -> 
     ``units``: optional iterable of (b, logical page) to restrict the work.
     """
     k_bits = np.asarray(k_bits, dtype=np.uint16)
+    return _summaries(lambda phys, n: bf16_to_f64(k_bits[phys, :, :n, :]), k_bits.shape,
+                      page_table, seq_lens, page_size, units)
+
+
+def page_summaries_fp8(k_codes, k_scale, page_table, seq_lens, page_size: int,
+                       units=None) -> np.ndarray:
+    """page_summaries of FP8 pages (R15): the mean of the dequantized valid keys.
+
+    All keys of a (page, kv head) share its scale, so the exact sum of the
+    dequantized keys is scale * (exact sum of the E4M3 values); that product is
+    exact in float64 (24 x 25 significant bits: at most 128 E4M3 values, each a
+    multiple of 2^-9 below 2^9)."""
+    k_codes = np.asarray(k_codes, dtype=np.uint8)
+    assert k_codes.shape[2] <= 128
+    sc = np.asarray(k_scale, dtype=np.float32).astype(np.float64)
+    return _summaries(lambda phys, n: e4m3_to_f64(k_codes[phys, :, :n, :]), k_codes.shape,
+                      page_table, seq_lens, page_size, units, post_scale=lambda phys: sc[phys])
+
+
+def _summaries(keys_of, shape, page_table, seq_lens, page_size: int, units,
+               post_scale=None) -> np.ndarray:
     pt = np.asarray(page_table, dtype=np.int64)
     sl = np.asarray(seq_lens, dtype=np.int64)
-    P_pool, Hkv, P, D = k_bits.shape
+    P_pool, Hkv, P, D = shape
     assert P == page_size
     out = np.zeros((P_pool, Hkv, D), dtype=np.uint16)
     if units is None:
@@ -172,10 +222,12 @@ def page_summaries(k_bits, page_table, seq_lens, page_size: int, units=None) -> 
         if n_valid <= 0:
             continue
         phys = int(pt[b, p])
-        keys = bf16_to_f64(k_bits[phys, :, :n_valid, :])          # [Hkv, n_valid, D]
+        keys = keys_of(phys, n_valid)                            # [Hkv, n_valid, D]
         terms = np.moveaxis(keys, 1, -1)                         # [Hkv, D, n_valid]
         e, u = _exp_and_ulp(terms)
         s = _exact_row_sums(terms.copy(), e, u)                  # [Hkv, D]
+        if post_scale is not None:
+            s = s * post_scale(phys)[:, None]
         out[phys] = f64_to_bf16_rne(s / float(n_valid))
     return out
 
@@ -312,17 +364,36 @@ def sparse_attention(q_bits, k_bits, v_bits, page_table, seq_lens, lists, counts
     head_to_list [Hq] (or [B,Hq]).  ``rows``: optional iterable of (b, t, h)
     to compute; the others stay 0 / -inf.
     """
-    q = bf16_to_f64(q_bits)
     k_bits = np.asarray(k_bits, dtype=np.uint16)
     v_bits = np.asarray(v_bits, dtype=np.uint16)
+    return _sparse_attention(q_bits, lambda phys, kvh: bf16_to_f64(k_bits[phys, kvh]),
+                             lambda phys, kvh: bf16_to_f64(v_bits[phys, kvh]), k_bits.shape[1],
+                             v_bits.shape[-1], page_table, seq_lens, lists, counts,
+                             head_to_list, scale, page_size, rows)
+
+
+def sparse_attention_fp8(q_bits, k_codes, k_scale, v_codes, v_scale, page_table, seq_lens, lists,
+                         counts, head_to_list, scale: float, page_size: int, rows=None):
+    """sparse_attention over FP8 pages (R15): keys e4m3(k_codes) * k_scale[page,
+    kv head], values e4m3(v_codes) * v_scale[page, kv head]; k_codes/v_codes
+    [P_pool,Hkv,P,D] uint8, scales [P_pool,Hkv] float32."""
+    k_codes = np.asarray(k_codes, dtype=np.uint8)
+    v_codes = np.asarray(v_codes, dtype=np.uint8)
+    return _sparse_attention(q_bits, lambda phys, kvh: _dequant(k_codes, k_scale, phys, kvh),
+                             lambda phys, kvh: _dequant(v_codes, v_scale, phys, kvh),
+                             k_codes.shape[1], v_codes.shape[-1], page_table, seq_lens, lists,
+                             counts, head_to_list, scale, page_size, rows)
+
+
+def _sparse_attention(q_bits, k_of, v_of, Hkv, Dv, page_table, seq_lens, lists, counts,
+                      head_to_list, scale, page_size, rows):
+    q = bf16_to_f64(q_bits)
     pt = np.asarray(page_table, dtype=np.int64)
     sl = np.asarray(seq_lens, dtype=np.int64)
     lists = np.asarray(lists, dtype=np.int64)
     counts = np.asarray(counts, dtype=np.int64)
     h2l = np.asarray(head_to_list, dtype=np.int64)
     B, T, Hq, Dk = q.shape
-    Hkv = k_bits.shape[1]
-    Dv = v_bits.shape[-1]
     G = Hq // Hkv
     P = page_size
     O = np.zeros((B, T, Hq, Dv), dtype=np.float64)
@@ -338,8 +409,8 @@ def sparse_attention(q_bits, k_bits, v_bits, page_table, seq_lens, lists, counts
             pages = lists[b, li, :int(counts[b, li])]
             phys = pt[b, pages]
             pos = (pages[:, None] * P + np.arange(P)[None, :]).reshape(-1)
-            K = bf16_to_f64(k_bits[phys, kvh]).reshape(-1, Dk)
-            V = bf16_to_f64(v_bits[phys, kvh]).reshape(-1, Dv)
+            K = k_of(phys, kvh).reshape(-1, Dk)
+            V = v_of(phys, kvh).reshape(-1, Dv)
             valid = pos < Lb
             pos, K, V = pos[valid], K[valid], V[valid]
             for t in range(T):

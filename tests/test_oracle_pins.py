@@ -453,3 +453,122 @@ def test_page_summaries_exact_mean():
                 assert sig[phys, h, d] == want
                 # the bf16 result is within one bf16 spacing of the exact mean
                 assert abs(bf16_fraction(sig[phys, h, d]) - mean) <= abs(mean) / 128 + Fraction(1, 2 ** 133)
+
+
+# ----------------------------------------------------------------------------
+# FP8 E4M3 pages with per-(page, kv head) scales (reading R15)
+# ----------------------------------------------------------------------------
+def e4m3_fraction(code):
+    """Exact value of one E4M3 code from its fields (None for NaN codes)."""
+    code = int(code)
+    s = -1 if code >> 7 else 1
+    e = (code >> 3) & 0xF
+    f = code & 0x7
+    if e == 0xF and f == 0x7:
+        return None
+    if e == 0:
+        return s * Fraction(f, 8) * Fraction(1, 64)
+    return s * (1 + Fraction(f, 8)) * Fraction(2) ** (e - 7)
+
+
+def rand_e4m3(rng, shape):
+    """Random non-NaN E4M3 codes."""
+    c = rng.integers(0, 256, size=shape).astype(np.uint8)
+    return np.where((c & 0x7F) == 0x7F, c ^ 0x01, c).astype(np.uint8)
+
+
+def test_e4m3_decode_against_fields_and_library():
+    codes = np.arange(256, dtype=np.uint8)
+    mine = O.e4m3_to_f64(codes)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    for c in range(256):
+        want = e4m3_fraction(c)
+        if want is None:
+            assert np.isnan(mine[c]) and np.isnan(lib[c])
+        else:
+            assert mine[c] == float(want) == lib[c]
+    # the format's landmarks: largest finite, smallest subnormal, smallest normal, one
+    assert mine[0x7E] == 448.0 and mine[0x01] == 2.0 ** -9 and mine[0x08] == 2.0 ** -6
+    assert mine[0x38] == 1.0 and mine[0xB8] == -1.0 and np.signbit(mine[0x80])
+
+
+def _fp8_case(rng, pow2_scales):
+    P_pool, Hkv, P, D = 5, 2, 8, 16
+    kc = rand_e4m3(rng, (P_pool, Hkv, P, D))
+    vc = rand_e4m3(rng, (P_pool, Hkv, P, D))
+    if pow2_scales:
+        ks = np.ldexp(1.0, rng.integers(-12, 4, size=(P_pool, Hkv))).astype(np.float32)
+        vs = np.ldexp(1.0, rng.integers(-12, 4, size=(P_pool, Hkv))).astype(np.float32)
+    else:
+        ks = (rng.random((P_pool, Hkv)) * 0.02 + 1e-3).astype(np.float32)
+        vs = (rng.random((P_pool, Hkv)) * 0.02 + 1e-3).astype(np.float32)
+    return kc, vc, ks, vs
+
+
+def _to_bf16_bits(x):
+    """bf16 patterns of float64 values that are exactly bf16 (checked)."""
+    f = x.astype(np.float32)
+    assert np.array_equal(f.astype(np.float64), x)
+    b = f.view(np.uint32)
+    assert np.all((b & 0xFFFF) == 0)
+    return (b >> 16).astype(np.uint16)
+
+
+def test_fp8_attention_reduces_to_bf16_with_power_of_two_scales():
+    # With power-of-two scales every dequantized key and value is a bf16 value,
+    # so the FP8 oracle must give exactly the bf16 oracle's result on them.
+    rng = np.random.default_rng(90)
+    kc, vc, ks, vs = _fp8_case(rng, True)
+    P = kc.shape[2]
+    kb = _to_bf16_bits(O.e4m3_to_f64(kc) * ks.astype(np.float64)[..., None, None])
+    vb = _to_bf16_bits(O.e4m3_to_f64(vc) * vs.astype(np.float64)[..., None, None])
+    B, T, Hq = 2, 2, 4
+    q = rand_bf16(rng, (B, T, Hq, kc.shape[3]))
+    pt = np.array([[3, 1, 4], [0, 2, 1]], dtype=np.int32)
+    sl = np.array([21, 13], dtype=np.int32)
+    lists = np.array([[[0, 2, 1]], [[1, 0, 0]]], dtype=np.int32)
+    cnt = np.array([[3], [2]], dtype=np.int32)
+    h2l = [0] * Hq
+    o8, l8 = O.sparse_attention_fp8(q, kc, ks, vc, vs, pt, sl, lists, cnt, h2l, 0.25, P)
+    ob, lb = O.sparse_attention(q, kb, vb, pt, sl, lists, cnt, h2l, 0.25, P)
+    np.testing.assert_array_equal(o8, ob)
+    np.testing.assert_array_equal(l8, lb)
+    s8 = O.page_summaries_fp8(kc, ks, pt, sl, P)
+    sb = O.page_summaries(kb, pt, sl, P)
+    np.testing.assert_array_equal(s8, sb)
+
+
+def test_fp8_summaries_exact_mean_general_scale():
+    # Non-power-of-two scales: the summary is RNE_bf16(RN64(RN64(exact sum of
+    # the dequantized keys) / n)), checked with exact rationals per element.
+    rng = np.random.default_rng(91)
+    kc, _, ks, _ = _fp8_case(rng, False)
+    P = kc.shape[2]
+    pt = np.array([[2, 0, 3]], dtype=np.int32)
+    sl = np.array([19], dtype=np.int32)                  # last page: 3 valid keys
+    sig = O.page_summaries_fp8(kc, ks, pt, sl, P)
+    for p, nval in ((0, 8), (1, 8), (2, 3)):
+        phys = pt[0, p]
+        for h in range(kc.shape[1]):
+            sc = Fraction(float(ks[phys, h]))
+            for d in range(kc.shape[3]):
+                tot = sum(e4m3_fraction(kc[phys, h, j, d]) * sc for j in range(nval))
+                want = O.f64_to_bf16_rne(np.array([float(tot) / nval]))[0]
+                assert sig[phys, h, d] == want
+
+
+def test_fp8_attention_closed_forms():
+    rng = np.random.default_rng(92)
+    kc, vc, ks, vs = _fp8_case(rng, False)
+    P, D = kc.shape[2], kc.shape[3]
+    q = rand_bf16(rng, (1, 1, 2, D))                     # head 0 reads kv head 0
+    pt = np.array([[3]], dtype=np.int32)
+    lists = np.array([[[0]]], dtype=np.int32)
+    cnt = np.array([[1]], dtype=np.int32)
+    # one key: O = its dequantized value, lse = scale q . k
+    o, lse = O.sparse_attention_fp8(q, kc, ks, vc, vs, pt, np.array([1]), lists, cnt, [0, 0], 0.5,
+                                    P)
+    v0 = [e4m3_fraction(c) * Fraction(float(vs[3, 0])) for c in vc[3, 0, 0]]
+    np.testing.assert_array_equal(o[0, 0, 0], np.array([float(x) for x in v0]))
+    qk = sum(bf16_fraction(a) * e4m3_fraction(c) for a, c in zip(q[0, 0, 0], kc[3, 0, 0]))
+    assert abs(lse[0, 0, 0] - 0.5 * float(qk * Fraction(float(ks[3, 0])))) < 1e-12
