@@ -229,6 +229,37 @@ SA_API int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const
                      void* stream);
 
 /*
+ * sa_sparse_decode_fp8 — sa_sparse_decode over K and V pages stored as FP8
+ * E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 fraction bits; the two
+ * NaN codes must not occur) with one float32 scale per (physical page, kv
+ * head): key j of a page is e4m3(k_codes[...]) * k_scale[page, kv head], and
+ * likewise for values.  Source: "Universal Attention Engine — Declarative
+ * Sparse Attention for Production", "Key Design Decisions" 2 (cache format:
+ * paged, block-sparse, quantized) and "Roadmap" (quantized KV cache support);
+ * the E4M3 format and the per-(page, kv head) scale are this library's
+ * reading of "quantized".
+ *
+ *  k_codes, v_codes (dev) [P_pool,Hkv,P,D] uint8, strides k_strides/v_strides
+ *                   (elements = bytes; unit feature stride, the others
+ *                   multiples of 16; 16-byte aligned base)
+ *  k_scale, v_scale (dev) [P_pool,Hkv] float32, contiguous, finite
+ * Everything else (q, page table, lists, head_to_list, splits, partials,
+ * device errors) as sa_sparse_decode.  Supported: D == 128 (keys and values),
+ * page_size a multiple of 16 up to 128, at most 16 query rows (T x heads) per
+ * (list, kv head) pair; other shapes return SA_ERR_UNSUPPORTED.
+ */
+SA_API int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4],
+                                const uint8_t* k_codes, const int64_t k_strides[4],
+                                const uint8_t* v_codes, const int64_t v_strides[4],
+                                const float* k_scale, const float* v_scale,
+                                const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                                const int32_t* lists, const int32_t* list_counts, int n_lists,
+                                int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                                int Hkv, int D, int page_size, int P_pool, float scale,
+                                int n_splits, float* o_partial, float* lse_partial,
+                                int32_t* dev_error, void* stream);
+
+/*
  * sa_combine — merge split partials: lse = log sum_s exp(lse_s),
  * O = sum_s exp(lse_s - lse) O_s; splits with lse_s = -inf weigh nothing
  * (their O rows are not used, whatever they hold);
@@ -272,6 +303,22 @@ SA_API int sa_update_page_summaries(const uint16_t* k_cache, const int64_t k_str
                              const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                              int B, int Hkv, int Dk, int page_size, int P_pool, int n_new,
                              uint16_t* summaries, int32_t* dev_error, void* stream);
+
+/*
+ * sa_build_page_summaries_fp8 — sa_build_page_summaries for FP8 E4M3 key
+ * pages with per-(page, kv head) scales (as sa_sparse_decode_fp8): the mean of
+ * the dequantized valid keys, RNE_bf16(RN64(RN64(exact sum)/n)).
+ *
+ *  k_codes    (dev) [P_pool,Hkv,P,Dk] uint8, strides k_strides (elements)
+ *  k_scale    (dev) [P_pool,Hkv] float32, contiguous
+ *  summaries  (dev) [P_pool,Hkv,Dk] bf16, contiguous (written)
+ * page_size <= 128.  Other arguments as sa_build_page_summaries.
+ */
+SA_API int sa_build_page_summaries_fp8(const uint8_t* k_codes, const int64_t k_strides[4],
+                                       const float* k_scale, const int32_t* page_table,
+                                       int max_pages, const int32_t* seq_lens, int B, int Hkv,
+                                       int Dk, int page_size, int P_pool, uint16_t* summaries,
+                                       int32_t* dev_error, void* stream);
 
 /*
  * sa_block_union — per-group KV block tables for chunked prefill.

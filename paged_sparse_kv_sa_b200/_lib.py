@@ -36,10 +36,15 @@ _SIGNATURES = {
     "sa_select_tiered_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
     "sa_sparse_decode": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P, _I,
                               _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P]),
+    "sa_sparse_decode_fp8": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _P, _P, _I, _P,
+                                  _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P,
+                                  _P, _P]),
     "sa_combine": (_I, [_P, _P, _I, _I64, _I, _P, _P, _P, _P]),
     "sa_build_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sa_update_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                       _P]),
+    "sa_build_page_summaries_fp8": (_I, [_P, _c_i64_4, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P,
+                                         _P]),
     "sa_block_union": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 
@@ -100,6 +105,18 @@ def _need_cuda(*ts):
 def _bf16(t):
     if t.dtype != torch.bfloat16:
         raise TypeError("expected bfloat16")
+    return t
+
+
+def _u8(t):
+    if t.dtype != torch.uint8:
+        raise TypeError("expected uint8 (FP8 E4M3 codes)")
+    return t
+
+
+def _f32c(t):
+    if t.dtype != torch.float32 or not t.is_contiguous():
+        raise TypeError("expected a contiguous float32 tensor")
     return t
 
 
@@ -226,6 +243,52 @@ def sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, lists, list_coun
                               _ptr(lse_partial), _ptr(dev_error), _stream(stream))
     _check(st, "sa_sparse_decode")
     return o_partial, lse_partial
+
+
+def sa_sparse_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, lists,
+                         list_counts, head_to_list, scale: float, n_splits: int = 1,
+                         o_partial=None, lse_partial=None, dev_error=None, stream=None):
+    """sa_sparse_decode over FP8 E4M3 pages: k_codes, v_codes [P_pool,Hkv,P,D] uint8 (unit
+    feature stride), k_scale, v_scale [P_pool,Hkv] float32.  Returns (o_partial, lse_partial)."""
+    lib = load()
+    _need_cuda(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, lists, list_counts)
+    _bf16(q), _u8(k_codes), _u8(v_codes), _f32c(k_scale), _f32c(v_scale)
+    _i32(page_table), _i32(seq_lens), _i32(lists), _i32(list_counts)
+    B, T, Hq, D = q.shape
+    P_pool, Hkv, P, _ = k_codes.shape
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    if o_partial is None:
+        o_partial = torch.empty((n_splits, B, T, Hq, D), dtype=torch.float32, device=q.device)
+    if lse_partial is None:
+        lse_partial = torch.empty((n_splits, B, T, Hq), dtype=torch.float32, device=q.device)
+    st = lib.sa_sparse_decode_fp8(_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
+                                  _ptr(v_codes), _strides4(v_codes), _ptr(k_scale), _ptr(v_scale),
+                                  _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
+                                  _ptr(lists), _ptr(list_counts), n_lists, max_list,
+                                  ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, D, P, P_pool,
+                                  float(scale), n_splits, _ptr(o_partial), _ptr(lse_partial),
+                                  _ptr(dev_error), _stream(stream))
+    _check(st, "sa_sparse_decode_fp8")
+    return o_partial, lse_partial
+
+
+def sa_build_page_summaries_fp8(k_codes, k_scale, page_table, seq_lens, summaries=None,
+                                dev_error=None, stream=None):
+    """k_codes [P_pool,Hkv,P,Dk] uint8 E4M3, k_scale [P_pool,Hkv] float32 -> summaries
+    [P_pool,Hkv,Dk] bf16 (rows of referenced pages written)."""
+    lib = load()
+    _need_cuda(k_codes, k_scale, page_table, seq_lens)
+    _u8(k_codes), _f32c(k_scale), _i32(page_table), _i32(seq_lens)
+    P_pool, Hkv, P, Dk = k_codes.shape
+    if summaries is None:
+        summaries = torch.zeros((P_pool, Hkv, Dk), dtype=torch.bfloat16, device=k_codes.device)
+    st = lib.sa_build_page_summaries_fp8(_ptr(k_codes), _strides4(k_codes), _ptr(k_scale),
+                                         _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
+                                         seq_lens.shape[0], Hkv, Dk, P, P_pool, _ptr(summaries),
+                                         _ptr(dev_error), _stream(stream))
+    _check(st, "sa_build_page_summaries_fp8")
+    return summaries
 
 
 def sa_combine(o_partial, lse_partial, o_out=None, o_out_bf16=None, lse_out=None,

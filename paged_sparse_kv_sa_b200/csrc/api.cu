@@ -47,6 +47,59 @@ int check_q(const uint16_t* q, const int64_t s[4]) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? SA_OK : SA_ERR_CUDA; }
 
+// The (list, kv head) pairs a decode call reads, the heads of each (in head
+// order) and the most query rows (T x heads) one pair holds.
+int build_pairs(const int32_t* head_to_list, int Hq, int Hkv, int T, PairTable* out,
+                int* max_rows_out) {
+  if (Hq > kMaxHeads) return SA_ERR_UNSUPPORTED;
+  PairTable& pairs = *out;
+  pairs.n_pairs = 0;
+  const int G = Hq / Hkv;
+  int pair_of[kMaxHeads];
+  for (int kvh = 0; kvh < Hkv; ++kvh) {
+    for (int h = kvh * G; h < (kvh + 1) * G; ++h) {
+      const int l = head_to_list[h];
+      int pi = -1;
+      for (int i = 0; i < pairs.n_pairs; ++i)
+        if (pairs.list_of[i] == l && pairs.kvh_of[i] == kvh) pi = i;
+      if (pi < 0) {
+        if (pairs.n_pairs == kMaxPairs) return SA_ERR_UNSUPPORTED;
+        pi = pairs.n_pairs++;
+        pairs.list_of[pi] = l;
+        pairs.kvh_of[pi] = kvh;
+        pairs.n_heads[pi] = 0;
+      }
+      if (pairs.n_heads[pi] == kMaxHeadsPerPair) return SA_ERR_UNSUPPORTED;
+      ++pairs.n_heads[pi];
+      pair_of[h] = pi;
+    }
+  }
+  int max_rows = 0;
+  for (int i = 0, off = 0; i < pairs.n_pairs; ++i) {
+    pairs.head_off[i] = off;
+    off += pairs.n_heads[i];
+    max_rows = max_rows > pairs.n_heads[i] * T ? max_rows : pairs.n_heads[i] * T;
+    pairs.n_heads[i] = 0;   // refilled below, in head order
+  }
+  for (int h = 0; h < Hq; ++h) {
+    const int pi = pair_of[h];
+    pairs.heads[pairs.head_off[pi] + pairs.n_heads[pi]++] = static_cast<int16_t>(h);
+  }
+  *max_rows_out = max_rows;
+  return SA_OK;
+}
+
+// FP8 pages: 16-byte aligned base, unit feature stride, other strides
+// positive multiples of 16 bytes (= 16 elements).
+int check_cache_u8(const uint8_t* p, const int64_t s[4]) {
+  if (!p || !s) return SA_ERR_INVALID_ARG;
+  if (!aligned16(p) || s[3] != 1) return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (s[i] <= 0 || (s[i] % 16) != 0) return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+
 }  // namespace
 
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
@@ -60,6 +113,20 @@ bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, in
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, gstr,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool encode_kv_map_u8(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
+                      const int64_t strides[4]) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)Hkv, (cuuint64_t)P_pool};
+  cuuint64_t gstr[3] = {(cuuint64_t)strides[2], (cuuint64_t)strides[1], (cuuint64_t)strides[0]};
+  cuuint32_t box[4] = {128, 16, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, gstr, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -250,40 +317,9 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
 
   // (list, kv head) pairs and the heads that read them
-  if (Hq > kMaxHeads) return SA_ERR_UNSUPPORTED;
   PairTable pairs;
-  pairs.n_pairs = 0;
-  const int G = Hq / Hkv;
-  int pair_of[kMaxHeads];
-  for (int kvh = 0; kvh < Hkv; ++kvh) {
-    for (int h = kvh * G; h < (kvh + 1) * G; ++h) {
-      const int l = head_to_list[h];
-      int pi = -1;
-      for (int i = 0; i < pairs.n_pairs; ++i)
-        if (pairs.list_of[i] == l && pairs.kvh_of[i] == kvh) pi = i;
-      if (pi < 0) {
-        if (pairs.n_pairs == kMaxPairs) return SA_ERR_UNSUPPORTED;
-        pi = pairs.n_pairs++;
-        pairs.list_of[pi] = l;
-        pairs.kvh_of[pi] = kvh;
-        pairs.n_heads[pi] = 0;
-      }
-      if (pairs.n_heads[pi] == kMaxHeadsPerPair) return SA_ERR_UNSUPPORTED;
-      ++pairs.n_heads[pi];
-      pair_of[h] = pi;
-    }
-  }
   int max_rows = 0;
-  for (int i = 0, off = 0; i < pairs.n_pairs; ++i) {
-    pairs.head_off[i] = off;
-    off += pairs.n_heads[i];
-    max_rows = max_rows > pairs.n_heads[i] * T ? max_rows : pairs.n_heads[i] * T;
-    pairs.n_heads[i] = 0;   // refilled below, in head order
-  }
-  for (int h = 0; h < Hq; ++h) {
-    const int pi = pair_of[h];
-    pairs.heads[pairs.head_off[pi] + pairs.n_heads[pi]++] = static_cast<int16_t>(h);
-  }
+  if (int r = build_pairs(head_to_list, Hq, Hkv, T, &pairs, &max_rows)) return r;
   // Up to 16 query rows per pair: warp-MMA decode; more: the tcgen05 kernel.
   const bool wide = max_rows > kMaxRowsPerPair;
   const int cap = mla ? mla_max_split_entries(page_size)
@@ -319,10 +355,74 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   a.o_part = o_partial;
   a.lse_part = lse_partial;
   a.err = dev_error;
+  a.k_scale = a.v_scale = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (mla) return cuda_status(launch_mla(a, pairs, kmap, st));
   return cuda_status(wide ? launch_prefill(a, pairs, kmap, vmap, st)
                           : launch_decode_gqa(a, pairs, kmap, vmap, st));
+}
+
+int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const uint8_t* k_codes,
+                         const int64_t k_strides[4], const uint8_t* v_codes,
+                         const int64_t v_strides[4], const float* k_scale, const float* v_scale,
+                         const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                         const int32_t* lists, const int32_t* list_counts, int n_lists,
+                         int max_list, const int32_t* head_to_list, int B, int T, int Hq, int Hkv,
+                         int D, int page_size, int P_pool, float scale, int n_splits,
+                         float* o_partial, float* lse_partial, int32_t* dev_error, void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0 ||
+      max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 || n_splits <= 0 ||
+      !std::isfinite(scale) || !head_to_list)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  if (int r = check_q(q, q_strides)) return r;
+  if (int r = check_cache_u8(k_codes, k_strides)) return r;
+  if (int r = check_cache_u8(v_codes, v_strides)) return r;
+  if (!k_scale || !v_scale || !page_table || !seq_lens || !lists || !list_counts || !o_partial ||
+      !lse_partial)
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(o_partial)) return SA_ERR_INVALID_ARG;
+  for (int h = 0; h < Hq; ++h)
+    if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
+  if (D != 128 || page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
+  PairTable pairs;
+  int max_rows = 0;
+  if (int r = build_pairs(head_to_list, Hq, Hkv, T, &pairs, &max_rows)) return r;
+  if (max_rows > kMaxRowsPerPair) return SA_ERR_UNSUPPORTED;
+  if ((max_list + n_splits - 1) / n_splits > decode_max_split_entries()) return SA_ERR_UNSUPPORTED;
+  CUtensorMap kmap, vmap;
+  if (!encode_kv_map_u8(&kmap, k_codes, D, page_size, Hkv, P_pool, k_strides) ||
+      !encode_kv_map_u8(&vmap, v_codes, D, page_size, Hkv, P_pool, v_strides))
+    return SA_ERR_CUDA;
+  DecodeArgs a;
+  a.q = q;
+  a.qs0 = q_strides[0];
+  a.qs1 = q_strides[1];
+  a.qs2 = q_strides[2];
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.lists = lists;
+  a.counts = list_counts;
+  a.n_lists = n_lists;
+  a.max_list = max_list;
+  a.B = B;
+  a.T = T;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.Dk = D;
+  a.Dv = D;
+  a.P = page_size;
+  a.P_pool = P_pool;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.n_splits = n_splits;
+  a.o_part = o_partial;
+  a.lse_part = lse_partial;
+  a.err = dev_error;
+  a.k_scale = k_scale;
+  a.v_scale = v_scale;
+  return cuda_status(
+      launch_decode_gqa_fp8(a, pairs, kmap, vmap, static_cast<cudaStream_t>(stream)));
 }
 
 int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,
@@ -372,6 +472,25 @@ int sa_update_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4]
   if (n_new <= 0) return SA_ERR_INVALID_ARG;
   return summaries_call(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv, Dk,
                         page_size, P_pool, n_new, summaries, dev_error, stream);
+}
+
+int sa_build_page_summaries_fp8(const uint8_t* k_codes, const int64_t k_strides[4],
+                                const float* k_scale, const int32_t* page_table, int max_pages,
+                                const int32_t* seq_lens, int B, int Hkv, int Dk, int page_size,
+                                int P_pool, uint16_t* summaries, int32_t* dev_error,
+                                void* stream) {
+  if (B < 0 || Hkv <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0 || max_pages == 0) return SA_OK;
+  if (!k_codes || !k_strides || k_strides[3] != 1 || !k_scale || !page_table || !seq_lens ||
+      !summaries)
+    return SA_ERR_INVALID_ARG;
+  for (int i = 0; i < 3; ++i)
+    if (k_strides[i] <= 0) return SA_ERR_INVALID_ARG;
+  if (max_pages > 65535 || B > 65535 || page_size > 128) return SA_ERR_UNSUPPORTED;
+  return cuda_status(launch_summaries_fp8(k_codes, k_strides, k_scale, page_table, max_pages,
+                                          seq_lens, B, Hkv, Dk, page_size, P_pool, summaries,
+                                          dev_error, static_cast<cudaStream_t>(stream)));
 }
 
 int sa_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_block_offset,

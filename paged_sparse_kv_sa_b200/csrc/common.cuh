@@ -4,6 +4,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -135,6 +136,13 @@ SA_DEV uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 SA_DEV float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+// Value of one FP8 E4M3 code (not one of the two NaN codes), through the
+// hardware E4M3 -> f16 conversion (exact: every E4M3 value is an f16 value).
+SA_DEV float e4m3_to_float(uint32_t code) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(code & 0xffu)));
+  return __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xffffu)));
+}
 
 // Byte offset of 16-bit element (row, col) inside a TMA box written with
 // CU_TENSOR_MAP_SWIZZLE_128B: rows of 128 bytes, the 16-byte chunk index

@@ -37,28 +37,69 @@ constexpr int kSub = 16;            // tokens per TMA sub-page (one MMA k-step o
 constexpr int kWarpEntries = 128;   // list entries one split may hold
 constexpr float kLazy = 8.f;        // log2 headroom before the running max moves
 
-template <int D>
+// F8: pages hold FP8 E4M3 codes (one byte per element) with a float32 scale per
+// (page, kv head); a sub-page arrives as one 128-column box and the warp
+// widens it to bf16 in a staging tile of the bf16 layout before the MMAs.
+template <int D, bool F8 = false>
 struct DecodeCfg {
-  static constexpr int kBoxes = D / 64;                     // 64-column TMA boxes per row set
+  static_assert(!F8 || D == 128, "FP8 pages: D == 128");
+  static constexpr int kBoxes = D / 64;                     // 64-column bf16 boxes per row set
   static constexpr int kBoxBytes = kSub * 128;              // 16 rows x 128 bytes
-  static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one K (or V) sub-page
-  static constexpr int kStageBytes = 2 * kTileBytes;        // K + V
-  static constexpr int kStages = D >= 128 ? SA_DECODE_STAGES : 2 * SA_DECODE_STAGES;
-  static constexpr int kDynBytes = kNW * kStages * kStageBytes + 1024;
+  static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one bf16 K (or V) sub-page
+  static constexpr int kInTile = F8 ? kSub * D : kTileBytes;   // one sub-page as stored
+  static constexpr int kStageBytes = 2 * kInTile;           // K + V
+  static constexpr int kStages = F8 ? 2 : (D >= 128 ? SA_DECODE_STAGES : 2 * SA_DECODE_STAGES);
+  static constexpr int kWarpBytes = kStages * kStageBytes + (F8 ? 2 * kTileBytes : 0);
+  static constexpr int kDynBytes = kNW * kWarpBytes + 1024;
 };
+
+// Two E4M3 codes (low byte -> low half) to two bf16 (exact: every E4M3 value
+// is a bf16 value), through the hardware E4M3 -> f16 conversion.
+SA_DEV uint32_t e4m3x2_to_bf16x2(uint32_t two) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(two & 0xffffu)));
+  const float f0 = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xffffu)));
+  const float f1 = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
+  return pack_bf16(f0, f1);
+}
+
+// One FP8 sub-page (16 rows x 128 codes, 128-byte swizzle) -> the bf16 layout
+// of two 64-column swizzled boxes.  Lane l takes row l / 2 and columns
+// 64 (l % 2) .. + 63: four 16-byte code chunks in, eight 16-byte bf16 chunks out.
+SA_DEV void widen_fp8_tile(const uint8_t* src, uint8_t* dst, int lane) {
+  const int t = lane >> 1, hb = lane & 1;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = 4 * hb + i;
+    const uint4 c = *reinterpret_cast<const uint4*>(src + t * 128 + (((j ^ t) & 7) << 4));
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint4 o0, o1;
+    o0.x = e4m3x2_to_bf16x2(w[0]);
+    o0.y = e4m3x2_to_bf16x2(w[0] >> 16);
+    o0.z = e4m3x2_to_bf16x2(w[1]);
+    o0.w = e4m3x2_to_bf16x2(w[1] >> 16);
+    o1.x = e4m3x2_to_bf16x2(w[2]);
+    o1.y = e4m3x2_to_bf16x2(w[2] >> 16);
+    o1.z = e4m3x2_to_bf16x2(w[3]);
+    o1.w = e4m3x2_to_bf16x2(w[3] >> 16);
+    uint8_t* box = dst + hb * (kSub * 128) + t * 128;
+    *reinterpret_cast<uint4*>(box + ((((2 * i) ^ t) & 7) << 4)) = o0;
+    *reinterpret_cast<uint4*>(box + ((((2 * i + 1) ^ t) & 7) << 4)) = o1;
+  }
+}
 
 struct __align__(64) DecodeParams {
   DecodeArgs a;
   PairTable pairs;
 };
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     decode_gqa_kernel(const __grid_constant__ DecodeParams prm,
                       const __grid_constant__ CUtensorMap kmap,
                       const __grid_constant__ CUtensorMap vmap) {
   pdl_wait_and_release();
-  using C = DecodeCfg<D>;
+  using C = DecodeCfg<D, F8>;
   const DecodeArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -67,6 +108,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
   __shared__ uint64_t bars[kNW][C::kStages];
   __shared__ int2 ent_s[kNW][kWarpEntries];    // (physical page, first token) per entry
+  __shared__ float2 scl_s[F8 ? kNW : 1][F8 ? kWarpEntries : 1];   // FP8: (k, v) scale per entry
 
   if (lane == 0) {
     for (int s = 0; s < C::kStages; ++s) mbar_init(&bars[warp][s], 1);
@@ -81,7 +123,8 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   // across items, which keeps the mbarrier phases in step.
   const int n_items = a.n_splits * prm.pairs.n_pairs * a.B;
   const int total_warps = gridDim.x * kNW;
-  uint8_t* ring = smem + warp * C::kStages * C::kStageBytes;
+  uint8_t* ring = smem + warp * C::kWarpBytes;
+  uint8_t* wide = ring + C::kStages * C::kStageBytes;   // FP8: the widened bf16 K, V tiles
   int base = 0;
   for (int item = blockIdx.x * kNW + warp; item < n_items; item += total_warps) {
   const int split = item % a.n_splits;
@@ -138,6 +181,10 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
       }
     }
     ent_s[warp][i] = make_int2(ph, p * a.P);
+    if constexpr (F8)
+      scl_s[warp][i] = ph >= 0 ? make_float2(a.k_scale[(int64_t)ph * a.Hkv + kvh],
+                                             a.v_scale[(int64_t)ph * a.Hkv + kvh])
+                               : make_float2(0.f, 0.f);
   }
   __syncwarp();
 
@@ -156,13 +203,18 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     int ph, tok0;
     if (unit_live(u, ph, tok0)) {
       uint8_t* kt = ring + slot * C::kStageBytes;
-      uint8_t* vt = kt + C::kTileBytes;
+      uint8_t* vt = kt + C::kInTile;
       const int row0 = (u % subs) * kSub;
       mbar_arrive_expect_tx(bar, C::kStageBytes);
+      if constexpr (F8) {
+        tma_load_4d(kt, &kmap, bar, 0, row0, kvh, ph);
+        tma_load_4d(kt + C::kInTile, &vmap, bar, 0, row0, kvh, ph);
+      } else {
 #pragma unroll
-      for (int bx = 0; bx < C::kBoxes; ++bx) {
-        tma_load_4d(kt + bx * C::kBoxBytes, &kmap, bar, bx * 64, row0, kvh, ph);
-        tma_load_4d(vt + bx * C::kBoxBytes, &vmap, bar, bx * 64, row0, kvh, ph);
+        for (int bx = 0; bx < C::kBoxes; ++bx) {
+          tma_load_4d(kt + bx * C::kBoxBytes, &kmap, bar, bx * 64, row0, kvh, ph);
+          tma_load_4d(vt + bx * C::kBoxBytes, &vmap, bar, bx * 64, row0, kvh, ph);
+        }
       }
     } else {
       mbar_arrive_expect_tx(bar, 0);
@@ -213,7 +265,18 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     int ph, tok0;
     if (unit_live(u, ph, tok0)) {
       const uint8_t* kt = ring + slot * C::kStageBytes;
-      const uint32_t kbase = smem_u32(kt), vbase = smem_u32(kt + C::kTileBytes);
+      uint32_t kbase = smem_u32(kt), vbase = smem_u32(kt + C::kTileBytes);
+      float ksc = 1.f, vsc = 1.f;   // FP8 page scales
+      if constexpr (F8) {
+        widen_fp8_tile(kt, wide, lane);
+        widen_fp8_tile(kt + C::kInTile, wide + C::kTileBytes, lane);
+        __syncwarp();
+        kbase = smem_u32(wide);
+        vbase = smem_u32(wide + C::kTileBytes);
+        const float2 sc = scl_s[warp][u / subs];
+        ksc = sc.x;
+        vsc = sc.y;
+      }
       // ---- S = Q K^T (16 rows x 16 tokens): 4 independent accumulation chains
       float s4[4][4];
 #pragma unroll
@@ -243,7 +306,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
           const int h = c >> 1;
           const int pos = tok0 + nt * 8 + 2 * tig + (c & 1);
           const bool ok = pos < L && pos <= lim[h];
-          s[nt][c] = ok ? s[nt][c] * a.scale_log2 : -INFINITY;
+          s[nt][c] = ok ? s[nt][c] * (a.scale_log2 * ksc) : -INFINITY;
           mx[h] = fmaxf(mx[h], s[nt][c]);
         }
       bool move[2];
@@ -281,8 +344,9 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
       // ---- O += P V with P = hi + lo (both bf16)
       uint32_t ph_[4], pl_[4];
       {
-        const float pv[4][2] = {{s[0][0], s[0][1]}, {s[0][2], s[0][3]},
-                                {s[1][0], s[1][1]}, {s[1][2], s[1][3]}};
+        // (FP8: the value scale rides on P; the denominator l_run does not)
+        const float pv[4][2] = {{s[0][0] * vsc, s[0][1] * vsc}, {s[0][2] * vsc, s[0][3] * vsc},
+                                {s[1][0] * vsc, s[1][1] * vsc}, {s[1][2] * vsc, s[1][3] * vsc}};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           ph_[i] = pack_bf16(pv[i][0], pv[i][1]);
@@ -304,7 +368,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
         mma_bf16_16816(o[2 * n2 + 1], pl_, r[2], r[3]);
       }
     }
-    __syncwarp();
+    __syncwarp();   // (FP8: the staging tiles are free again)
     if (lane == 0 && u + C::kStages < n_units) issue(u + C::kStages);
   }
   if (u_fail >= 0) {
@@ -342,14 +406,14 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   }  // items
 }
 
-template <int D>
+template <int D, bool F8 = false>
 cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                      const CUtensorMap& vmap, cudaStream_t stream) {
-  using C = DecodeCfg<D>;
+  using C = DecodeCfg<D, F8>;
   DecodeParams prm;
   prm.a = a;
   prm.pairs = pairs;
-  cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, F8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDynBytes);
   if (e != cudaSuccess) return e;
   // one wave of resident CTAs (or fewer when there is less work)
@@ -357,13 +421,13 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D>, kNW * 32,
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D, F8>, kNW * 32,
                                                       C::kDynBytes);
   if (e != cudaSuccess) return e;
   const long long items = (long long)a.n_splits * pairs.n_pairs * a.B;
   const long long want = (items + kNW - 1) / kNW;
   const int grid = (int)std::min<long long>(want, (long long)std::max(1, per_sm) * sms);
-  return launch_pdl(decode_gqa_kernel<D>, grid, dim3(kNW * 32), C::kDynBytes, stream, prm, kmap,
+  return launch_pdl(decode_gqa_kernel<D, F8>, grid, dim3(kNW * 32), C::kDynBytes, stream, prm, kmap,
                     vmap);
 }
 
@@ -380,6 +444,13 @@ cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const
     case 256: return launch_d<256>(a, pairs, kmap, vmap, stream);
     default: return cudaErrorInvalidValue;
   }
+}
+
+cudaError_t launch_decode_gqa_fp8(const DecodeArgs& a, const PairTable& pairs,
+                                  const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                  cudaStream_t stream) {
+  if (a.Dk != 128 || !a.k_scale || !a.v_scale) return cudaErrorInvalidValue;
+  return launch_d<128, true>(a, pairs, kmap, vmap, stream);
 }
 
 }  // namespace sa

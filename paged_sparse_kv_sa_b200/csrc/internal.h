@@ -67,12 +67,18 @@ struct DecodeArgs {
   float* o_part;
   float* lse_part;
   int32_t* err;
+  const float* k_scale;   // FP8 pages: [P_pool, Hkv] float32 scales (null for bf16 pages)
+  const float* v_scale;
 };
 
 // Encode a 4-D bf16 tensor map over a [P_pool, Hkv, P, D] cache with
 // 64-column x 16-row boxes and 128-byte swizzle.  false on failure.
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
                    const int64_t strides[4]);
+// The same over FP8 (one byte per element) pages, D == 128: 128-column x 16-row
+// boxes (128-byte rows), 128-byte swizzle.
+bool encode_kv_map_u8(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
+                      const int64_t strides[4]);
 
 int decode_max_split_entries();
 int prefill_max_split_entries();
@@ -84,6 +90,9 @@ cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CU
 int decode_warps_per_cta();
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream);
+cudaError_t launch_decode_gqa_fp8(const DecodeArgs& a, const PairTable& pairs,
+                                  const CUtensorMap& kmap, const CUtensorMap& vmap,
+                                  cudaStream_t stream);
 
 struct SelectArgs {
   const uint16_t* q;
@@ -126,6 +135,10 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
                            int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,
                            cudaStream_t stream);
 
+cudaError_t launch_summaries_fp8(const uint8_t* k, const int64_t ks[4], const float* k_scale,
+                                 const int32_t* pt, int max_pages, const int32_t* seq_lens, int B,
+                                 int Hkv, int Dk, int P, int P_pool, uint16_t* sig, int32_t* err,
+                                 cudaStream_t stream);
 cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
                              int P, int P_pool, int n_new, uint16_t* sig, int32_t* err,

@@ -65,7 +65,46 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// FP8 pages: every E4M3 value is a multiple of 2^-9 below 2^9, so the float64
+// sum of at most 128 of them is exact; all keys of a (page, kv head) share its
+// scale, and scale * sum (24 x 25 significant bits) is exact too: the mean is
+// RN64(exact sum of the dequantized keys / n), as for bf16 pages.
+__global__ void __launch_bounds__(256)
+    summaries_fp8_kernel(const uint8_t* __restrict__ k, int64_t ks0, int64_t ks1, int64_t ks2,
+                         const float* __restrict__ k_scale, const int32_t* __restrict__ pt,
+                         int max_pages, const int32_t* __restrict__ seq_lens, int Hkv, int Dk,
+                         int P, int P_pool, uint16_t* __restrict__ sig, int32_t* err) {
+  pdl_wait_and_release();
+  const int b = blockIdx.y, p = blockIdx.x;
+  const int L = min(seq_lens[b], max_pages * P);
+  const int n = min(P, L - p * P);
+  if (n <= 0) return;
+  const int ph = pt[(int64_t)b * max_pages + p];
+  if (ph < 0 || ph >= P_pool) {
+    if (threadIdx.x == 0) set_dev_error(err, SA_DEVERR_POOL_RANGE);
+    return;
+  }
+  for (int c = threadIdx.x; c < Hkv * Dk; c += blockDim.x) {
+    const int h = c / Dk, d = c % Dk;
+    const uint8_t* col = k + ph * ks0 + h * ks1 + d;
+    double s = 0.0;
+    for (int j = 0; j < n; ++j) s += static_cast<double>(e4m3_to_float(col[j * ks2]));
+    s *= static_cast<double>(k_scale[(int64_t)ph * Hkv + h]);
+    sig[((int64_t)ph * Hkv + h) * Dk + d] = f64_to_bf16_rne(s / static_cast<double>(n));
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_summaries_fp8(const uint8_t* k, const int64_t ks[4], const float* k_scale,
+                                 const int32_t* pt, int max_pages, const int32_t* seq_lens, int B,
+                                 int Hkv, int Dk, int P, int P_pool, uint16_t* sig, int32_t* err,
+                                 cudaStream_t stream) {
+  if (B == 0 || max_pages == 0) return cudaSuccess;
+  dim3 grid(max_pages, B);
+  return launch_pdl(summaries_fp8_kernel, grid, dim3(256), 0, stream, k, ks[0], ks[1], ks[2],
+                    k_scale, pt, max_pages, seq_lens, Hkv, Dk, P, P_pool, sig, err);
+}
 
 cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,

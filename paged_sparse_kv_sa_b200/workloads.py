@@ -196,6 +196,19 @@ def gqa_decode_inputs(cfg: GQADecode, seed: int = 0, device="cpu", seq_lens: Opt
     return dict(q=q, k=k, v=v, page_table=pt, seq_lens=sl, pool=pool)
 
 
+def fp8_pages(x):
+    """FP8 E4M3 codes and per-(page, kv head) float32 scales of a bf16 pool x
+    [P_pool, Hkv, P, D] (input preparation for the FP8-page workloads): scale =
+    max |x| over the (page, kv head) / 448 (1 for an all-zero page), codes =
+    x / scale rounded to the nearest E4M3 value (ties to even; torch's float8 cast),
+    clamped to the format's +-448.  Returns (codes uint8, scales float32)."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=(2, 3))
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    y = (xf / scale[:, :, None, None]).clamp(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8), scale.contiguous()
+
+
 def mla_decode_inputs(cfg: MLADecode, seed: int = 0, device="cpu", seq_len: Optional[int] = None):
     """q [B,T,Hq,Dk], latent pool [P_pool,1,P,Dk] (V = first Dv columns), page table,
     seq_lens, and the ambient head set (``h_ambient`` sorted head ids, seeded)."""

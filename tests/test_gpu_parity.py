@@ -703,3 +703,111 @@ def test_mla_decode_full_size_sampled():
     for (b, t, h) in rows:
         assert np.abs(og[b, t, h] - ro[b, t, h]).max() <= O_TOL, (b, t, h)
         assert abs(lg[b, t, h] - rl[b, t, h]) <= LSE_TOL, (b, t, h)
+
+
+# ----------------------------------------------------------------------------
+# FP8 E4M3 pages with per-(page, kv head) scales
+# ----------------------------------------------------------------------------
+def fp8_case(cfg, seed, seq_lens=None):
+    inp, g = gqa_case(cfg, seed=seed, seq_lens=seq_lens)
+    kc, ks = W.fp8_pages(inp["k"])
+    vc, vs = W.fp8_pages(inp["v"])
+    f8 = dict(kc=kc, ks=ks, vc=vc, vs=vs)
+    return inp, g, f8, {k: v.to(DEV) for k, v in f8.items()}
+
+
+def run_decode_fp8(g, f8d, lists, counts, cfg, n_splits, h2l=None):
+    h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)] if h2l is None else h2l
+    o_p, l_p = sa.sa_sparse_decode_fp8(g["q"], f8d["kc"], f8d["vc"], f8d["ks"], f8d["vs"],
+                                       g["page_table"], g["seq_lens"],
+                                       torch.from_numpy(lists).to(DEV),
+                                       torch.from_numpy(counts).to(DEV), h2l,
+                                       1.0 / math.sqrt(cfg.D), n_splits)
+    o, ob, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    return o, lse
+
+
+def oracle_fp8(inp, f8, lists, counts, cfg, h2l=None, rows=None):
+    h2l = np.arange(cfg.Hq) // (cfg.Hq // cfg.Hkv) if h2l is None else np.asarray(h2l)
+    return O.sparse_attention_fp8(bits(inp["q"]), f8["kc"].numpy(), f8["ks"].numpy(),
+                                  f8["vc"].numpy(), f8["vs"].numpy(), np_i32(inp["page_table"]),
+                                  np_i32(inp["seq_lens"]), lists, counts, h2l,
+                                  1.0 / math.sqrt(cfg.D), cfg.page_size, rows=rows)
+
+
+def test_summaries_fp8_bitexact():
+    cfg = W.scaled(W.TINY_GQA, D=128, B=3)
+    inp, g, f8, f8d = fp8_case(cfg, seed=30, seq_lens=[2048, 1000 + 3, 17])
+    ref = O.page_summaries_fp8(f8["kc"].numpy(), f8["ks"].numpy(), np_i32(inp["page_table"]),
+                               np_i32(inp["seq_lens"]), cfg.page_size)
+    sig = sa.sa_build_page_summaries_fp8(f8d["kc"], f8d["ks"], g["page_table"], g["seq_lens"])
+    torch.cuda.synchronize()
+    pt = np_i32(inp["page_table"])
+    for b, L in enumerate([2048, 1003, 17]):
+        used = pt[b, :-(-L // cfg.page_size)]
+        np.testing.assert_array_equal(bits(sig)[used], ref[used])
+
+
+@pytest.mark.parametrize("n_splits", [1, 3])
+def test_decode_fp8_vs_oracle(n_splits):
+    # selection on the FP8 pages' summaries, then decode over the FP8 pages
+    cfg = W.scaled(W.TINY_GQA, D=128, B=3)
+    inp, g, f8, f8d = fp8_case(cfg, seed=31, seq_lens=[2048, 1000 + 3, 37])
+    sig = O.page_summaries_fp8(f8["kc"].numpy(), f8["ks"].numpy(), np_i32(inp["page_table"]),
+                               np_i32(inp["seq_lens"]), cfg.page_size)
+    lists, counts = oracle_lists(inp, cfg, sig)
+    o, lse = run_decode_fp8(g, f8d, lists, counts, cfg, n_splits)
+    ro, rl = oracle_fp8(inp, f8, lists, counts, cfg)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_decode_fp8_mtp_per_head_lists_and_empty():
+    # T = 2 and 8 heads per kv head (16 rows per pair); the heads of a group
+    # read different lists, one of them empty
+    cfg = W.GQADecode("case", B=2, Hq=16, Hkv=2, D=128, page_size=16, seq_len_lo=0,
+                      seq_len_hi=0, sink_tokens=16, local_tokens=16, budget_tokens=160, T=2)
+    lens = [700, 333]
+    inp, g, f8, f8d = fp8_case(cfg, seed=32, seq_lens=lens)
+    rng = np.random.default_rng(32)
+    n_lists, cap = 3, 9
+    lists = np.full((2, n_lists, cap), -1, dtype=np.int32)
+    counts = np.zeros((2, n_lists), dtype=np.int32)
+    for b, L in enumerate(lens):
+        nb = -(-L // 16)
+        for li in range(n_lists - 1):
+            pick = np.sort(rng.choice(nb, size=min(cap, nb), replace=False))
+            lists[b, li, :len(pick)] = pick
+            counts[b, li] = len(pick)
+    h2l = [h % n_lists for h in range(cfg.Hq)]
+    o, lse = run_decode_fp8(g, f8d, lists, counts, cfg, 2, h2l=h2l)
+    ro, rl = oracle_fp8(inp, f8, lists, counts, cfg, h2l=h2l)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_decode_fp8_llama8b_length_sampled():
+    # Llama-8B-shaped sequences at full length (32768 tokens, 2048 pages) with
+    # seeded page lists of the workload's budget, 13 splits; sampled rows
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=4)
+    inp, g, f8, f8d = fp8_case(cfg, seed=33)
+    rng = np.random.default_rng(33)
+    nb = cfg.seq_len_hi // cfg.page_size
+    lists = np.stack([np.stack([np.sort(rng.choice(nb, size=64, replace=False))
+                                for _ in range(cfg.Hkv)]) for _ in range(cfg.B)]).astype(np.int32)
+    counts = np.full((cfg.B, cfg.Hkv), 64, dtype=np.int32)
+    o, lse = run_decode_fp8(g, f8d, lists, counts, cfg, 13)
+    rows = [(b, 0, int(h)) for b in range(cfg.B) for h in rng.integers(0, cfg.Hq, 5)]
+    ro, rl = oracle_fp8(inp, f8, lists, counts, cfg, rows=rows)
+    og, lg = o.cpu().double().numpy(), lse.cpu().double().numpy()
+    for (b, t, h) in rows:
+        assert np.abs(og[b, t, h] - ro[b, t, h]).max() <= O_TOL, (b, t, h)
+        assert abs(lg[b, t, h] - rl[b, t, h]) <= LSE_TOL, (b, t, h)
+
+
+def test_decode_fp8_rejects_unsupported_shapes():
+    cfg = W.TINY_GQA                                      # D = 64
+    inp, g, f8, f8d = fp8_case(cfg, seed=34)
+    lists = np.zeros((cfg.B, cfg.Hkv, 4), dtype=np.int32)
+    counts = np.zeros((cfg.B, cfg.Hkv), dtype=np.int32)
+    with pytest.raises(sa.SAError, match="UNSUPPORTED"):
+        run_decode_fp8(g, f8d, lists, counts, cfg, 1)
