@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = heuristic)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--workload", choices=["llama8b", "llama70b", "mla", "prefill"],
+    ap.add_argument("--workload", choices=["llama8b", "llama70b", "mla", "prefill", "llama8b_fp8"],
                     default="llama8b",
                     help="llama8b (default, the headline workload); the others print the same "
                          "line for the Llama-70B long decode, MLA+MTP tiered decode and "
@@ -120,8 +120,9 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def selected_kv_bytes(counts, pages, seq_lens, P, D):
-    """K+V bytes of the valid tokens of every selected page (per step)."""
+def selected_kv_bytes(counts, pages, seq_lens, P, D, elem_bytes=2):
+    """K+V bytes of the valid tokens of every selected page (per step); FP8 pages
+    (elem_bytes 1) add their two float32 scales per selected (page, kv head)."""
     import torch
     B, Hkv, cap = pages.shape
     L = seq_lens.to(torch.int64).view(B, 1, 1)
@@ -130,12 +131,14 @@ def selected_kv_bytes(counts, pages, seq_lens, P, D):
     p = pages.to(torch.int64).clamp_min(0)
     toks = (L - p * P).clamp(0, P)
     toks = torch.where(valid, toks, torch.zeros_like(toks))
-    return int(toks.sum().item()) * D * 2 * 2
+    scales = int(valid.sum().item()) * 8 if elem_bytes == 1 else 0
+    return int(toks.sum().item()) * D * elem_bytes * 2 + scales
 
 
-def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0):
+def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=None):
     """Oracle (float64, host cores) on a bounded sample: n_units (b, kv head)
-    pairs, select + attention.  Returns GB/s of selected KV and the sample."""
+    pairs, select + attention (over FP8 pages when f8 holds their codes and
+    scales).  Returns GB/s of selected KV and the sample."""
     import numpy as np
 
     import oracle as O
@@ -155,8 +158,6 @@ def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0):
         phys = pt[b, lst]
         # gather only this unit's pages from the device pool
         import torch
-        kb = W.bf16_bits(inp["k"][torch.as_tensor(phys, device=inp["k"].device)])
-        vb = W.bf16_bits(inp["v"][torch.as_tensor(phys, device=inp["v"].device)])
         loc_pt = np.full_like(pt, -1)
         loc_pt[b, lst] = np.arange(len(lst))
         lists = np.full((cfg.B, cfg.Hkv, pages_np.shape[2]), -1, dtype=np.int32)
@@ -164,10 +165,20 @@ def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0):
         lists[b, h, :len(lst)] = lst
         counts[b, h] = len(lst)
         rows = [(b, 0, hh) for hh in range(h * G, (h + 1) * G)]
-        O.sparse_attention(qb, kb, vb, loc_pt, sl, lists, counts, np.arange(cfg.Hq) // G,
-                           1.0 / math.sqrt(cfg.D), cfg.page_size, rows=rows)
+        # gather only this unit's pages from the device pool
+        ix = torch.as_tensor(phys, device=inp["q"].device)
+        if f8 is None:
+            O.sparse_attention(qb, W.bf16_bits(inp["k"][ix]), W.bf16_bits(inp["v"][ix]), loc_pt,
+                               sl, lists, counts, np.arange(cfg.Hq) // G, 1.0 / math.sqrt(cfg.D),
+                               cfg.page_size, rows=rows)
+        else:
+            O.sparse_attention_fp8(qb, f8["kc"][ix].cpu().numpy(), f8["ks"][ix].cpu().numpy(),
+                                   f8["vc"][ix].cpu().numpy(), f8["vs"][ix].cpu().numpy(), loc_pt,
+                                   sl, lists, counts, np.arange(cfg.Hq) // G,
+                                   1.0 / math.sqrt(cfg.D), cfg.page_size, rows=rows)
         L = int(sl[b])
-        kv_bytes += sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst) * cfg.D * 4
+        eb = 2 if f8 is None else 1
+        kv_bytes += sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst) * cfg.D * 2 * eb
         done += 1
         if time.perf_counter() - t0 > budget_s:
             break
@@ -412,21 +423,30 @@ def main():
     cores = len(os.sched_getaffinity(0))
     if args.workload in ("mla", "prefill"):
         return run_extra(args, dev, world, rank, local, cores)
-    cfg = {"llama8b": W.LLAMA8B_DECODE, "llama70b": W.LLAMA70B_LONG}[args.workload]
+    cfg = {"llama8b": W.LLAMA8B_DECODE, "llama70b": W.LLAMA70B_LONG,
+           "llama8b_fp8": W.LLAMA8B_DECODE}[args.workload]
+    fp8 = args.workload == "llama8b_fp8"
 
     if args.impl == "reference":
         # the reference arm is the float64 oracle on the host cores
         import paged_sparse_kv_sa_b200 as sa
         sa.load()
         inp = W.gqa_decode_inputs(cfg, seed=args.seed, device=dev)
-        sig = sa.sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
+        f8 = None
+        if fp8:
+            kc, ks = W.fp8_pages(inp["k"])
+            vc, vs = W.fp8_pages(inp["v"])
+            f8 = dict(kc=kc, ks=ks, vc=vc, vs=vs)
+            sig = sa.sa_build_page_summaries_fp8(kc, ks, inp["page_table"], inp["seq_lens"])
+        else:
+            sig = sa.sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
         torch.cuda.synchronize()
         sig_bits = W.bf16_bits(sig)
         for _ in range(args.warmup):
-            cpu_baseline(cfg, inp, sig_bits, 1, budget_s=5)
+            cpu_baseline(cfg, inp, sig_bits, 1, budget_s=5, f8=f8)
         tot_b, tot_t, units = 0.0, 0.0, 0
         for _ in range(args.steps):
-            gbs, n, dt = cpu_baseline(cfg, inp, sig_bits, 2, budget_s=10)
+            gbs, n, dt = cpu_baseline(cfg, inp, sig_bits, 2, budget_s=10, f8=f8)
             tot_b += gbs * dt
             tot_t += dt
             units += n
@@ -436,7 +456,8 @@ def main():
                 "ms_per_step": round(1000 * tot_t / args.steps, 3), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "impl": "reference",
-                "config": {"workload": cfg.name, "B": cfg.B, "seq_len": cfg.seq_len_lo,
+                "config": {"workload": cfg.name + ("_fp8" if fp8 else ""), "B": cfg.B,
+                           "seq_len": cfg.seq_len_lo,
                            "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
                            "budget_tokens": cfg.budget_tokens},
                 "cpu_baseline": {"value": round(val, 6), "unit": "GB/s", "cores": cores,
@@ -452,7 +473,15 @@ def main():
     sa.load()
     inp = W.gqa_decode_inputs(cfg, seed=args.seed + rank, device=dev)
     q, k, v, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
-    sig = sa.sa_build_page_summaries(k, pt, sl)
+    f8 = None
+    if fp8:
+        # FP8 E4M3 pages with per-(page, kv head) scales, quantized from the bf16 pools
+        kc, ks = W.fp8_pages(k)
+        vc, vs = W.fp8_pages(v)
+        f8 = dict(kc=kc, ks=ks, vc=vc, vs=vs)
+        sig = sa.sa_build_page_summaries_fp8(kc, ks, pt, sl)
+    else:
+        sig = sa.sa_build_page_summaries(k, pt, sl)
     step = sa.SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, pt.shape[1],
                                cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens,
                                n_splits=args.splits or None, device=dev)
@@ -467,15 +496,22 @@ def main():
         flush.fill_(i & 0xFF)
         torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
 
+    def decode_call(qq, ptt, sll):
+        if fp8:
+            step.decode_fp8(qq, kc, vc, ks, vs, ptt, sll)
+        else:
+            step.decode(qq, k, v, ptt, sll)
+
     def run_step():
         step.select(q, sig, pt, sl)
-        step.decode(q, k, v, pt, sl)
+        decode_call(q, pt, sl)
         step.combine()
 
     for _ in range(max(args.warmup, 3)):
         run_step()
     torch.cuda.synchronize()
-    kv_bytes = selected_kv_bytes(step.counts, step.pages, sl, cfg.page_size, cfg.D)
+    kv_bytes = selected_kv_bytes(step.counts, step.pages, sl, cfg.page_size, cfg.D,
+                                 elem_bytes=1 if fp8 else 2)
     q_bytes = q.numel() * 2
     part_bytes = step.o_part.numel() * 4 + step.lse_part.numel() * 4
     list_bytes = step.pages.numel() * 4 + step.counts.numel() * 4
@@ -489,7 +525,7 @@ def main():
     with torch.cuda.graph(g_step):
         run_step()
     with torch.cuda.graph(g_dec):
-        step.decode(q, k, v, pt, sl)
+        decode_call(q, pt, sl)
     for _ in range(3):
         g_step.replay()
         g_dec.replay()
@@ -520,7 +556,7 @@ def main():
     st_ev[0].record(stream)
     step.select(q, sig, pt, sl)
     st_ev[1].record(stream)
-    step.decode(q, k, v, pt, sl)
+    decode_call(q, pt, sl)
     st_ev[2].record(stream)
     step.combine()
     st_ev[3].record(stream)
@@ -549,7 +585,7 @@ def main():
         pt_d.copy_(pt_h, non_blocking=True)
         sl_d.copy_(sl_h, non_blocking=True)
         step.select(q_d, sig, pt_d, sl_d)
-        step.decode(q_d, k, v, pt_d, sl_d)
+        decode_call(q_d, pt_d, sl_d)
         step.combine()
         o_h.copy_(step.o, non_blocking=True)
         lse_h.copy_(step.lse, non_blocking=True)
@@ -587,7 +623,7 @@ def main():
     if os.path.exists(tp):
         with open(tp) as f:
             td = json.load(f)
-        if td.get("workload") == cfg.name and td.get("splits") == step.n_splits:
+        if td.get("workload") == cfg.name and td.get("splits") == step.n_splits and not fp8:
             traffic = td.get("bytes_per_launch")
 
     line = {
@@ -595,8 +631,11 @@ def main():
         "steps": K, "warmup": args.warmup, "ms_per_step": round(1e3 * t_step_max / K, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": cfg.name, "B": cfg.B, "seq_len": cfg.seq_len_lo, "Hq": cfg.Hq,
+        "config": {"workload": cfg.name + ("_fp8" if fp8 else ""), "B": cfg.B,
+                   "seq_len": cfg.seq_len_lo, "Hq": cfg.Hq,
                    "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
+                   "kv_pages": ("fp8 e4m3 + float32 scale per (page, kv head)" if fp8
+                                else "bf16"),
                    "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
                    "local_tokens": cfg.local_tokens, "n_splits": step.n_splits,
                    "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)",
@@ -606,7 +645,7 @@ def main():
                      "decode_graph": round(1e3 * t_dec / K, 4),
                      "combine_eager": round(1e3 * t_cmb / K, 4)},
         "selected_kv_bytes_per_step": kv_bytes,
-        "roofline": {"kernel": "decode_gqa_kernel", "bound": "hbm", "achieved": round(achieved, 2),
+        "roofline": {"kernel": "decode_gqa_kernel" + ("<fp8>" if fp8 else ""), "bound": "hbm", "achieved": round(achieved, 2),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_kind": peak_kind, "traffic": traffic,
                      "alg_bytes_per_launch": decode_alg_bytes},
@@ -617,7 +656,7 @@ def main():
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=8, budget_s=20.0)
+        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=8, budget_s=20.0, f8=f8)
         line["cpu_baseline"] = {"value": round(gbs, 6), "unit": "GB/s", "cores": cores,
                                 "kind": "oracle",
                                 "sample": f"{n} of {cfg.B * cfg.Hkv} (sequence, kv head) units: "

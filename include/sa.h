@@ -75,6 +75,7 @@ typedef enum {
 #define SA_DEVERR_POOL_RANGE 2   /* physical page id outside [0, P_pool)        */
 #define SA_DEVERR_COUNT 4        /* list count < 0 or above its capacity        */
 #define SA_DEVERR_TIMEOUT 8      /* a bounded wait on a copy gave up             */
+#define SA_DEVERR_VALUE_RANGE 16 /* FP8 pages: a query value beyond +-65504      */
 
 /* Human-readable name of a status code (static storage). */
 SA_API const char* sa_status_string(int status);

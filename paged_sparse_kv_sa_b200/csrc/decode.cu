@@ -32,14 +32,18 @@ namespace {
 #ifndef SA_DECODE_STAGES
 #define SA_DECODE_STAGES 2
 #endif
+#ifndef SA_DECODE_STAGES_F8
+#define SA_DECODE_STAGES_F8 2
+#endif
 constexpr int kNW = SA_DECODE_WARPS;
 constexpr int kSub = 16;            // tokens per TMA sub-page (one MMA k-step of PV)
 constexpr int kWarpEntries = 128;   // list entries one split may hold
 constexpr float kLazy = 8.f;        // log2 headroom before the running max moves
 
 // F8: pages hold FP8 E4M3 codes (one byte per element) with a float32 scale per
-// (page, kv head); a sub-page arrives as one 128-column box and the warp
-// widens it to bf16 in a staging tile of the bf16 layout before the MMAs.
+// (page, kv head); a sub-page arrives as one 128-column box.  The MMAs run in
+// f16 (E4M3 -> f16 is one exact instruction per pair): K fragments straight
+// from the code tile, V through an f16 staging tile.
 template <int D, bool F8 = false>
 struct DecodeCfg {
   static_assert(!F8 || D == 128, "FP8 pages: D == 128");
@@ -48,24 +52,15 @@ struct DecodeCfg {
   static constexpr int kTileBytes = kBoxes * kBoxBytes;     // one bf16 K (or V) sub-page
   static constexpr int kInTile = F8 ? kSub * D : kTileBytes;   // one sub-page as stored
   static constexpr int kStageBytes = 2 * kInTile;           // K + V
-  static constexpr int kStages = F8 ? 2 : (D >= 128 ? SA_DECODE_STAGES : 2 * SA_DECODE_STAGES);
-  static constexpr int kWarpBytes = kStages * kStageBytes + (F8 ? 2 * kTileBytes : 0);
+  static constexpr int kStages = F8 ? SA_DECODE_STAGES_F8 : (D >= 128 ? SA_DECODE_STAGES : 2 * SA_DECODE_STAGES);
+  static constexpr int kWarpBytes = kStages * kStageBytes + (F8 ? kTileBytes : 0);
   static constexpr int kDynBytes = kNW * kWarpBytes + 1024;
 };
 
-// Two E4M3 codes (low byte -> low half) to two bf16 (exact: every E4M3 value
-// is a bf16 value), through the hardware E4M3 -> f16 conversion.
-SA_DEV uint32_t e4m3x2_to_bf16x2(uint32_t two) {
-  uint32_t h;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(two & 0xffffu)));
-  const float f0 = __half2float(__ushort_as_half(static_cast<unsigned short>(h & 0xffffu)));
-  const float f1 = __half2float(__ushort_as_half(static_cast<unsigned short>(h >> 16)));
-  return pack_bf16(f0, f1);
-}
-
-// One FP8 sub-page (16 rows x 128 codes, 128-byte swizzle) -> the bf16 layout
-// of two 64-column swizzled boxes.  Lane l takes row l / 2 and columns
-// 64 (l % 2) .. + 63: four 16-byte code chunks in, eight 16-byte bf16 chunks out.
+// One FP8 sub-page (16 rows x 128 codes, 128-byte swizzle) -> f16 in the
+// layout of two 64-column swizzled boxes (what the bf16 path's ldmatrix reads).
+// Lane l takes row l / 2 and columns 64 (l % 2) .. + 63: four 16-byte code
+// chunks in, eight 16-byte f16 chunks out.
 SA_DEV void widen_fp8_tile(const uint8_t* src, uint8_t* dst, int lane) {
   const int t = lane >> 1, hb = lane & 1;
 #pragma unroll
@@ -74,14 +69,14 @@ SA_DEV void widen_fp8_tile(const uint8_t* src, uint8_t* dst, int lane) {
     const uint4 c = *reinterpret_cast<const uint4*>(src + t * 128 + (((j ^ t) & 7) << 4));
     const uint32_t w[4] = {c.x, c.y, c.z, c.w};
     uint4 o0, o1;
-    o0.x = e4m3x2_to_bf16x2(w[0]);
-    o0.y = e4m3x2_to_bf16x2(w[0] >> 16);
-    o0.z = e4m3x2_to_bf16x2(w[1]);
-    o0.w = e4m3x2_to_bf16x2(w[1] >> 16);
-    o1.x = e4m3x2_to_bf16x2(w[2]);
-    o1.y = e4m3x2_to_bf16x2(w[2] >> 16);
-    o1.z = e4m3x2_to_bf16x2(w[3]);
-    o1.w = e4m3x2_to_bf16x2(w[3] >> 16);
+    o0.x = e4m3x2_to_f16x2(w[0]);
+    o0.y = e4m3x2_to_f16x2(w[0] >> 16);
+    o0.z = e4m3x2_to_f16x2(w[1]);
+    o0.w = e4m3x2_to_f16x2(w[1] >> 16);
+    o1.x = e4m3x2_to_f16x2(w[2]);
+    o1.y = e4m3x2_to_f16x2(w[2] >> 16);
+    o1.z = e4m3x2_to_f16x2(w[3]);
+    o1.w = e4m3x2_to_f16x2(w[3] >> 16);
     uint8_t* box = dst + hb * (kSub * 128) + t * 128;
     *reinterpret_cast<uint4*>(box + ((((2 * i) ^ t) & 7) << 4)) = o0;
     *reinterpret_cast<uint4*>(box + ((((2 * i + 1) ^ t) & 7) << 4)) = o1;
@@ -124,7 +119,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   const int n_items = a.n_splits * prm.pairs.n_pairs * a.B;
   const int total_warps = gridDim.x * kNW;
   uint8_t* ring = smem + warp * C::kWarpBytes;
-  uint8_t* wide = ring + C::kStages * C::kStageBytes;   // FP8: the widened bf16 K, V tiles
+  uint8_t* wide = ring + C::kStages * C::kStageBytes;   // FP8: the f16 V staging tile
   int base = 0;
   for (int item = blockIdx.x * kNW + warp; item < n_items; item += total_warps) {
   const int split = item % a.n_splits;
@@ -237,14 +232,47 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
                           prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)] * a.qs2
                     : nullptr;
     }
+    if constexpr (F8) {
+      // f16 fragments in a permuted feature order: k-slots (2 tig, 2 tig + 1)
+      // and (2 tig + 8, 2 tig + 9) of step kk hold features kk 16 + 4 tig + 0..3,
+      // so a key fragment is one 4-byte code load (the same permutation on both
+      // operands leaves the dot products unchanged)
+      bool big = false;
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const int c = kk * 16 + 2 * tig;
-      qa[kk][0] = qp[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + c) : 0u;
-      qa[kk][1] = qp[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + c) : 0u;
-      qa[kk][2] = qp[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + c + 8) : 0u;
-      qa[kk][3] = qp[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + c + 8) : 0u;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int c = kk * 16 + 4 * tig;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint2 x = qp[h] ? *reinterpret_cast<const uint2*>(qp[h] + c) : make_uint2(0u, 0u);
+          const float f0 = bf16_bits_to_float(x.x & 0xffffu), f1 = bf16_bits_to_float(x.x >> 16);
+          const float f2 = bf16_bits_to_float(x.y & 0xffffu), f3 = bf16_bits_to_float(x.y >> 16);
+          big |= fmaxf(fmaxf(fabsf(f0), fabsf(f1)), fmaxf(fabsf(f2), fabsf(f3))) > 65504.f;
+          qa[kk][h] = pack_f16(f0, f1);
+          qa[kk][2 + h] = pack_f16(f2, f3);
+        }
+      }
+      if (big) set_dev_error(a.err, SA_DEVERR_VALUE_RANGE);
+    } else {
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const int c = kk * 16 + 2 * tig;
+        qa[kk][0] = qp[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + c) : 0u;
+        qa[kk][1] = qp[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + c) : 0u;
+        qa[kk][2] = qp[0] ? *reinterpret_cast<const uint32_t*>(qp[0] + c + 8) : 0u;
+        qa[kk][3] = qp[1] ? *reinterpret_cast<const uint32_t*>(qp[1] + c + 8) : 0u;
+      }
     }
+  }
+  // FP8: values enter PV scaled by (page scale / v_ref), v_ref = the largest
+  // value scale of the split's pages (so P stays <= 256 in f16); the output is
+  // multiplied back by v_ref.
+  float v_ref = 1.f;
+  if constexpr (F8) {
+    float m = 0.f;
+    for (int i = lane; i < n_ent; i += 32) m = fmaxf(m, scl_s[warp][i].y);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    v_ref = m > 0.f ? m : 1.f;
   }
   const int lim[2] = {qt_[0] >= 0 ? L - a.T + qt_[0] : -1, qt_[1] >= 0 ? L - a.T + qt_[1] : -1};
 
@@ -266,30 +294,41 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     if (unit_live(u, ph, tok0)) {
       const uint8_t* kt = ring + slot * C::kStageBytes;
       uint32_t kbase = smem_u32(kt), vbase = smem_u32(kt + C::kTileBytes);
-      float ksc = 1.f, vsc = 1.f;   // FP8 page scales
+      float ksc = 1.f, vsc = 1.f;   // FP8: key scale, value scale / v_ref
       if constexpr (F8) {
-        widen_fp8_tile(kt, wide, lane);
-        widen_fp8_tile(kt + C::kInTile, wide + C::kTileBytes, lane);
+        widen_fp8_tile(kt + C::kInTile, wide, lane);
         __syncwarp();
-        kbase = smem_u32(wide);
-        vbase = smem_u32(wide + C::kTileBytes);
+        vbase = smem_u32(wide);
         const float2 sc = scl_s[warp][u / subs];
         ksc = sc.x;
-        vsc = sc.y;
+        vsc = sc.y / v_ref;
       }
       // ---- S = Q K^T (16 rows x 16 tokens): 4 independent accumulation chains
       float s4[4][4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) s4[i][0] = s4[i][1] = s4[i][2] = s4[i][3] = 0.f;
+      if constexpr (F8) {
+        // key fragments straight from the code tile: token rows gid and
+        // gid + 8 (both with swizzle row gid), 4 codes per lane per k-step
+        const uint8_t* k8 = kt + gid * 128 + 4 * tig;
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int colb = (kk & 3) * 16;
-        const uint32_t addr = kbase + (kk >> 2) * C::kBoxBytes +
-                              swz128(8 * (mi >> 1) + ri, colb + 8 * (mi & 1));
-        uint32_t r[4];
-        ldmatrix_x4(r, addr);
-        mma_bf16_16816(s4[kk & 1], qa[kk], r[0], r[1]);
-        mma_bf16_16816(s4[2 + (kk & 1)], qa[kk], r[2], r[3]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t w0 = *reinterpret_cast<const uint32_t*>(k8 + ((kk ^ gid) << 4));
+          const uint32_t w1 = *reinterpret_cast<const uint32_t*>(k8 + 8 * 128 + ((kk ^ gid) << 4));
+          mma_f16_16816(s4[kk & 1], qa[kk], e4m3x2_to_f16x2(w0), e4m3x2_to_f16x2(w0 >> 16));
+          mma_f16_16816(s4[2 + (kk & 1)], qa[kk], e4m3x2_to_f16x2(w1), e4m3x2_to_f16x2(w1 >> 16));
+        }
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int colb = (kk & 3) * 16;
+          const uint32_t addr = kbase + (kk >> 2) * C::kBoxBytes +
+                                swz128(8 * (mi >> 1) + ri, colb + 8 * (mi & 1));
+          uint32_t r[4];
+          ldmatrix_x4(r, addr);
+          mma_bf16_16816(s4[kk & 1], qa[kk], r[0], r[1]);
+          mma_bf16_16816(s4[2 + (kk & 1)], qa[kk], r[2], r[3]);
+        }
       }
       float s[2][4];
 #pragma unroll
@@ -349,10 +388,17 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
                                 {s[1][0] * vsc, s[1][1] * vsc}, {s[1][2] * vsc, s[1][3] * vsc}};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          ph_[i] = pack_bf16(pv[i][0], pv[i][1]);
-          const float h0 = bf16_bits_to_float(ph_[i] & 0xffffu);
-          const float h1 = bf16_bits_to_float(ph_[i] >> 16);
-          pl_[i] = pack_bf16(pv[i][0] - h0, pv[i][1] - h1);
+          if constexpr (F8) {
+            ph_[i] = pack_f16(pv[i][0], pv[i][1]);
+            const float h0 = f16_bits_to_float(ph_[i] & 0xffffu);
+            const float h1 = f16_bits_to_float(ph_[i] >> 16);
+            pl_[i] = pack_f16(pv[i][0] - h0, pv[i][1] - h1);
+          } else {
+            ph_[i] = pack_bf16(pv[i][0], pv[i][1]);
+            const float h0 = bf16_bits_to_float(ph_[i] & 0xffffu);
+            const float h1 = bf16_bits_to_float(ph_[i] >> 16);
+            pl_[i] = pack_bf16(pv[i][0] - h0, pv[i][1] - h1);
+          }
         }
       }
 #pragma unroll
@@ -362,10 +408,17 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
                               swz128(8 * (mi & 1) + ri, colb + 8 * (mi >> 1));
         uint32_t r[4];
         ldmatrix_x4_trans(r, addr);
-        mma_bf16_16816(o[2 * n2], ph_, r[0], r[1]);
-        mma_bf16_16816(o[2 * n2 + 1], ph_, r[2], r[3]);
-        mma_bf16_16816(o[2 * n2], pl_, r[0], r[1]);
-        mma_bf16_16816(o[2 * n2 + 1], pl_, r[2], r[3]);
+        if constexpr (F8) {
+          mma_f16_16816(o[2 * n2], ph_, r[0], r[1]);
+          mma_f16_16816(o[2 * n2 + 1], ph_, r[2], r[3]);
+          mma_f16_16816(o[2 * n2], pl_, r[0], r[1]);
+          mma_f16_16816(o[2 * n2 + 1], pl_, r[2], r[3]);
+        } else {
+          mma_bf16_16816(o[2 * n2], ph_, r[0], r[1]);
+          mma_bf16_16816(o[2 * n2 + 1], ph_, r[2], r[3]);
+          mma_bf16_16816(o[2 * n2], pl_, r[0], r[1]);
+          mma_bf16_16816(o[2 * n2 + 1], pl_, r[2], r[3]);
+        }
       }
     }
     __syncwarp();   // (FP8: the staging tiles are free again)
@@ -393,7 +446,7 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     const int t = r / nh, head = prm.pairs.heads[prm.pairs.head_off[pair] + (r % nh)];
     const int64_t row = (((int64_t)split * a.B + b) * a.T + t) * a.Hq + head;
     const bool empty = l_run[h] == 0.f;
-    const float inv = empty ? 0.f : 1.f / l_run[h];
+    const float inv = empty ? 0.f : v_ref / l_run[h];
     float* dst = a.o_part + row * D;
 #pragma unroll
     for (int i = 0; i < D / 8; ++i)

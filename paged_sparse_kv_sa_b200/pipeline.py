@@ -77,6 +77,14 @@ class SparseDecodeStep:
                               o_partial=self.o_part, lse_partial=self.lse_part,
                               dev_error=self.dev_error, stream=stream)
 
+    def decode_fp8(self, q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens,
+                   stream=None):
+        """decode over FP8 E4M3 pages with per-(page, kv head) scales (D == 128)."""
+        _lib.sa_sparse_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens,
+                                  self.pages, self.counts, self.head_to_list, self.scale,
+                                  self.n_splits, o_partial=self.o_part, lse_partial=self.lse_part,
+                                  dev_error=self.dev_error, stream=stream)
+
     def combine(self, stream=None):
         _lib.sa_combine(self.o_part, self.lse_part, o_out=self.o, o_out_bf16=self.o_bf16,
                         lse_out=self.lse, stream=stream)
