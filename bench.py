@@ -618,6 +618,28 @@ def main():
     hbm_peak, peak_kind = peaks()
     dec_avg = t_dec / K
     achieved = decode_alg_bytes / dec_avg / 1e9
+    # context for the roofline: one library device copy moving the same number
+    # of bytes (half read, half written) in one launch, from its own graph with
+    # L2 flushed first -- the kind of copy the peak is measured with, at this
+    # size (a single launch pays a fixed cost that a multi-GiB copy hides)
+    half = max(decode_alg_bytes // 2 // 16, 1)
+    rd_buf = torch.ones((half, 4), dtype=torch.int32, device=dev)
+    rd_out = torch.empty_like(rd_buf)
+    g_rd = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_rd):
+        rd_out.copy_(rd_buf)
+    for _ in range(3):
+        g_rd.replay()
+    rd_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(K, 50))]
+    for i in range(len(rd_ev)):
+        flush_l2(i)
+        rd_ev[i][0].record(stream)
+        g_rd.replay()
+        rd_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_rd = sum(a.elapsed_time(b) for a, b in rd_ev) / 1e3 / len(rd_ev)
+    read_gbs = 2 * rd_buf.numel() * 4 / t_rd / 1e9
+    del rd_buf, rd_out
     traffic = None
     tp = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if os.path.exists(tp):
@@ -648,7 +670,11 @@ def main():
         "roofline": {"kernel": "decode_gqa_kernel" + ("<fp8>" if fp8 else ""), "bound": "hbm", "achieved": round(achieved, 2),
                      "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
                      "peak_kind": peak_kind, "traffic": traffic,
-                     "alg_bytes_per_launch": decode_alg_bytes},
+                     "alg_bytes_per_launch": decode_alg_bytes,
+                     "same_bytes_copy": {"gbs": round(read_gbs, 1),
+                                         "what": "one device copy (torch copy_) moving the same "
+                                                 "bytes, read + write, L2 flushed"},
+                     "frac_of_same_bytes_copy": round(achieved / read_gbs, 4)},
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(1e3 * t_e2e / K, 4)},
