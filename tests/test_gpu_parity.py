@@ -215,6 +215,39 @@ def test_select_workspace_contents_do_not_matter():
         np.testing.assert_array_equal(np_i32(pages), rp)
 
 
+@pytest.mark.parametrize("D,T", [(128, 1), (64, 2)])
+def test_select_eight_kv_heads_ragged(D, T):
+    # Hkv = 8 (one scoring CTA covers all kv heads of a page): a long sequence
+    # (16 scoring chunks), one of a single chunk, one shorter than the budget
+    # (nothing to rank) and a ragged one, in the same call.
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=4, Hq=16 if T == 2 else 32, Hkv=8, D=D, T=T,
+                   seq_len_lo=0, seq_len_hi=0)
+    lens = [32768 - 7, 1100, 700, 9000 + 5]
+    inp, g = gqa_case(cfg, seed=40 + D, seq_lens=lens)
+    sig = oracle_summaries(inp, cfg)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+
+
+def test_select_eight_kv_heads_ties():
+    # Hkv = 8 and all scores of one sequence tie (q = 0): resolved by the
+    # lowest logical pages
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=2, seq_len_lo=8192, seq_len_hi=8192)
+    inp, g = gqa_case(cfg, seed=44)
+    sig = oracle_summaries(inp, cfg)
+    qb = bits(inp["q"]).copy()
+    qb[1] = 0
+    g["q"] = to_bf16_dev(qb)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(qb, sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+
+
 def _random_bf16_bits(rng, shape, e_lo, e_hi, p_sub=0.03, p_zero=0.03):
     """bf16 bit patterns: random sign and fraction, exponent field uniform in
     [e_lo, e_hi]; a share of subnormals and zeros."""
