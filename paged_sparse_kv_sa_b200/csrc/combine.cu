@@ -26,6 +26,8 @@ SA_DEV float4 ld4_if(const float* p, bool pred) {
   return v;
 }
 
+// KS: splits handled in registers (n_splits <= KS), 0 = any count in batches.
+template <int KS>
 __global__ void __launch_bounds__(128)
     combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part,
                    int n_splits, int64_t rows, int Dv, float* __restrict__ o_out,
@@ -34,7 +36,8 @@ __global__ void __launch_bounds__(128)
   // (32-bit index arithmetic: the launcher guarantees rows * Dv / 4 < 2^32)
   const uint32_t q4 = static_cast<uint32_t>(Dv) / 4u;
   const uint32_t idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= static_cast<uint32_t>(rows) * q4) return;
+  const bool live = idx < static_cast<uint32_t>(rows) * q4;
+  if (!live) return;
   const uint32_t row_ = idx / q4;
   const int64_t row = row_;
   const int c = static_cast<int>(idx - row_ * q4) * 4;
@@ -43,25 +46,25 @@ __global__ void __launch_bounds__(128)
   // load of a phase is issued before any is used.
   float m = -INFINITY, tot = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (n_splits <= kRegSplits) {
-    float w[kRegSplits];
+  if constexpr (KS > 0) {
+    float w[KS];
 #pragma unroll
-    for (int s = 0; s < kRegSplits; ++s)   // (index clamped: unconditional loads)
+    for (int s = 0; s < KS; ++s)   // (index clamped: unconditional loads)
       w[s] = __ldg(lse_part + min(s, n_splits - 1) * rows + row);
 #pragma unroll
-    for (int s = 0; s < kRegSplits; ++s) {
+    for (int s = 0; s < KS; ++s) {
       if (s >= n_splits) w[s] = -INFINITY;
       m = fmaxf(m, w[s]);
     }
     if (m != -INFINITY) {
-      float4 v[kRegSplits];
+      float4 v[KS];
 #pragma unroll
-      for (int s = 0; s < kRegSplits; ++s) {
+      for (int s = 0; s < KS; ++s) {
         w[s] = __expf(w[s] - m);
         v[s] = ld4_if(o_part + (s * rows + row) * Dv + c, w[s] > 0.f);
       }
 #pragma unroll
-      for (int s = 0; s < kRegSplits; ++s) {
+      for (int s = 0; s < KS; ++s) {
         tot += w[s];
         acc.x += w[s] * v[s].x;
         acc.y += w[s] * v[s].y;
@@ -127,8 +130,14 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
   if (n >= (int64_t(1) << 32)) return cudaErrorInvalidValue;
   const int threads = 128;
   const int64_t blocks = (n + threads - 1) / threads;
-  return launch_pdl(combine_kernel, dim3((unsigned)blocks), dim3(threads), 0, stream, o_part,
-                    lse_part, n_splits, rows, Dv, o_out, o_bf16, lse_out);
+  auto go = [&](auto kern) {
+    return launch_pdl(kern, dim3((unsigned)blocks), dim3(threads), 0, stream, o_part, lse_part,
+                      n_splits, rows, Dv, o_out, o_bf16, lse_out);
+  };
+  if (n_splits <= 4) return go(combine_kernel<4>);
+  if (n_splits <= 8) return go(combine_kernel<8>);
+  if (n_splits <= kRegSplits) return go(combine_kernel<kRegSplits>);
+  return go(combine_kernel<0>);
 }
 
 }  // namespace sa
