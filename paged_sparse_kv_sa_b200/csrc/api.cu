@@ -103,13 +103,13 @@ int check_cache_u8(const uint8_t* p, const int64_t s[4]) {
 }  // namespace
 
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
-                   const int64_t strides[4]) {
+                   const int64_t strides[4], int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)P, (cuuint64_t)Hkv, (cuuint64_t)P_pool};
   cuuint64_t gstr[3] = {(cuuint64_t)strides[2] * 2, (cuuint64_t)strides[1] * 2,
                         (cuuint64_t)strides[0] * 2};
-  cuuint32_t box[4] = {64, 16, 1, 1};
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, gstr,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -327,7 +327,9 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   if (!mla && wide && Dk > 128) return SA_ERR_UNSUPPORTED;
   if ((max_list + n_splits - 1) / n_splits > cap) return SA_ERR_UNSUPPORTED;
   CUtensorMap kmap, vmap;
-  if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides) ||
+  // MLA tiles of 64 keys: one 64-row box per column chunk when a tile lies in one page
+  const int k_box_rows = mla && page_size % 64 == 0 ? 64 : 16;
+  if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides, k_box_rows) ||
       !encode_kv_map(&vmap, v_cache, Dv, page_size, Hkv, P_pool, v_strides))
     return SA_ERR_CUDA;
   DecodeArgs a;

@@ -72,9 +72,10 @@ struct DecodeArgs {
 };
 
 // Encode a 4-D bf16 tensor map over a [P_pool, Hkv, P, D] cache with
-// 64-column x 16-row boxes and 128-byte swizzle.  false on failure.
+// 64-column x box_rows-row boxes (box_rows 16 or 64, at most P) and 128-byte
+// swizzle.  false on failure.
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
-                   const int64_t strides[4]);
+                   const int64_t strides[4], int box_rows = 16);
 // The same over FP8 (one byte per element) pages, D == 128: 128-column x 16-row
 // boxes (128-byte rows), 128-byte swizzle.
 bool encode_kv_map_u8(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,

@@ -4,29 +4,36 @@
 // query rows (T x heads) per list.
 //
 // One CTA computes 64 query rows of one (list, kv head) pair against its split
-// of the list, 32 keys per tile.  The MMAs are M = 64: TMEM then holds a
+// of the list, 64 keys per tile.  The MMAs are M = 64: TMEM then holds a
 // 64-row accumulator in the low 16 lanes of each 32-lane subpartition, and a
 // second one in the high 16 lanes of the same columns.  O (64 x 512 float32)
 // is kept as two such halves — value columns 0-255 in the low lanes, 256-511
-// in the high lanes — in TMEM columns [0, 256); the two S buffers (64 x 32)
-// sit in columns [256, 288) and [288, 320).  So the whole output fits in TMEM
+// in the high lanes — in TMEM columns [0, 256); the two S buffers (64 x 64)
+// sit in columns [256, 320) and [320, 384).  So the whole output fits in TMEM
 // next to S and no FLOP is spent twice.
 //
-// Per 32-key tile S = Q K^T takes 36 MMAs of 64 x 32 x 16 and O += P V two
-// halves of two 64 x 256 x 16 MMAs.  Shared memory: the query tile (72 KB,
-// resident), four key stages of 36 KB and one P buffer of 8 KB: the deep ring
-// is what hides the gather latency (a stage is free only once the PV of its
-// tile is done, since the values are read from it).
+// Per 64-key tile S = Q K^T takes 36 MMAs of 64 x 64 x 16 (an MMA of N <= 64
+// costs the same issue time as one of N = 32, so 64-key tiles halve the QK
+// issue cost per key) and O += P V two halves of four 64 x 256 x 16 MMAs.
+// Shared memory: the query tile (72 KB, resident), two key stages of 72 KB and
+// one P buffer of 8 KB.  A stage is free only once the PV of its tile is done
+// (the values are read from it), so the ring is kept moving by issuing MMAs
+// as their inputs arrive: every 64-column chunk of a stage has its own full
+// barrier (the QK MMAs of chunk 0 start while chunks 1-8 are in flight), and
+// PV of tile j goes out as soon as P of tile j is written, ahead of QK
+// chunks of tile j + 1 that have not landed, so the stage of tile j is
+// refilled while tile j + 1 is being scored.
 //   warp 4      resolves the split's pages, then TMA-gathers key tiles (9
-//               column chunks x two 16-key boxes; an absent or invalid group
+//               column chunks; one 64-row box per chunk when a tile lies in
+//               one page, else four 16-row boxes; an absent or invalid group
 //               is read at an out-of-range page, which TMA fills with zeros)
-//               into the 4-stage ring;
-//   warp 5      issues the MMAs (fully unrolled, descriptors advanced by
+//               into the 2-stage ring;
+//   warp 5      issues the MMAs in arrival order (descriptors advanced by
 //               constants);
 //   warps 0-3   stage the query tile (bulk row copies, then a swizzling
 //               rearrangement in shared memory), then own a row per
 //               lane pair (l, l + 16): mask, lazily re-based base-2 online
-//               softmax and P for 16 keys each; the low lane rescales / writes
+//               softmax and P for 32 keys each; the low lane rescales / writes
 //               value columns 0-255 of O, the high lane 256-511.
 //
 // Sources: "TileSparse: Arithmetic-Intensity-Aware Sparse Attention for
@@ -42,22 +49,25 @@ namespace sa {
 namespace {
 
 constexpr int kMThreads = 192;
-constexpr int kMStages = 4;
-constexpr int kMKeys = 32;          // keys per tile
+constexpr int kMStages = 2;
+constexpr int kMKeys = 64;          // keys per tile
+constexpr int kMGroups = kMKeys / 16;   // 16-key groups per tile
 constexpr int kMRows = 64;          // query rows per CTA
 constexpr int kMMaxEnt = 128;       // list entries per split
-constexpr int kMMaxTiles = 128;     // tiles per split
+constexpr int kMMaxTiles = 128;     // tiles per split (tile ids fit 7 bits)
 constexpr int kDk = 576, kDv = 512;
 constexpr int kKC = kDk / 64;       // 9 key column chunks
 constexpr int kQBytes = kKC * kMRows * 128;          // 73728
-constexpr int kChunkBytes = kMKeys * 128;            // 4096: one column chunk of a tile
-constexpr int kTileBytes = kKC * kChunkBytes;        // 36864
-constexpr int kPBytes = kMRows * 128;                // 8192: 64 rows of 128 bytes (32 keys used)
+constexpr int kChunkBytes = kMKeys * 128;            // 8192: one column chunk of a tile
+constexpr int kTileBytes = kKC * kChunkBytes;        // 73728
+constexpr int kPBytes = kMRows * 128;                // 8192: 64 rows of 64 bf16 keys
 constexpr int kMDyn = kQBytes + kMStages * kTileBytes + kPBytes + 1024;
 constexpr int kStageRow = kDv * 4 + 16;              // O staging row (padded: no bank conflicts)
 static_assert(kMRows * kStageRow <= kMStages * kTileBytes, "O staging must fit the key ring");
+static_assert(kQBytes <= kTileBytes, "the raw query rows are staged in the last key stage");
+static_assert(kMDyn + 2048 <= 232448, "shared memory per CTA");
 constexpr uint32_t kMTmemCols = 512;
-constexpr uint32_t kSCol = 256;                      // S buffers at 256 and 288
+constexpr uint32_t kSCol = 256;                      // S buffers at 256 and 320
 constexpr uint32_t kHiLanes = 16u << 16;             // second M=64 accumulator
 constexpr uint32_t kIdQK = tc::idesc_bf16_f32(kMRows, kMKeys, false, false);
 constexpr uint32_t kIdPV = tc::idesc_bf16_f32(kMRows, 256, false, true);
@@ -69,6 +79,7 @@ struct __align__(64) MlaParams {
   DecodeArgs a;
   PairTable pairs;
   int n_items;
+  int box_rows;                     // rows per TMA box: 64 (tiles within one page) or 16
   int16_t item_pair[kMMaxItems], item_qt[kMMaxItems];
 };
 
@@ -87,7 +98,7 @@ SA_DEV bool warp_wait_m(uint64_t* bar, uint32_t parity, volatile int* abort_flag
 }
 // (physical page or -1, first token) of 16-key group g of tile j.
 SA_DEV int2 mgroup(const int2* ent, int n_ent, int P, int j, int g) {
-  const int key0 = (2 * j + g) * 16;
+  const int key0 = (kMGroups * j + g) * 16;
   const int e = key0 / P;
   if (e >= n_ent) return make_int2(-1, 0);
   const int2 en = ent[e];
@@ -110,7 +121,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
   uint8_t* q_s = smem;
   uint8_t* k_s = smem + kQBytes;                              // kMStages tiles
   uint8_t* p_s = k_s + kMStages * kTileBytes;                 // one P buffer
-  __shared__ uint64_t kv_full[kMStages], kv_empty[kMStages];
+  __shared__ uint64_t kv_full[kMStages][kKC], kv_empty[kMStages];   // full: per column chunk
   __shared__ uint64_t s_full[2], p_full, o_done, q_full, q_stage, ent_ready;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, n_act_s;
@@ -151,52 +162,20 @@ __global__ void __launch_bounds__(kMThreads, 1)
   const int t_last = (min(rows_total, r0 + kMRows) - 1) / nh;
   const int max_q = L - a.T + t_last;
 
-  if (tid == 0) {
-    for (int s = 0; s < kMStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) mbar_init(&s_full[s], 1);
-    mbar_init(&p_full, 128);
-    mbar_init(&o_done, 1);
-    mbar_init(&q_full, 1);
-    mbar_init(&q_stage, 1);
-    mbar_init(&ent_ready, 1);
-    abort_s = 0;
-    fence_mbar_init();
-  }
-  if (warp == 5) tc::tmem_alloc(&tmem_base_s, kMTmemCols);
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = tmem_base_s;
-  volatile int* abort_flag = &abort_s;
   const int n_tiles = min((n_ent * a.P + kMKeys - 1) / kMKeys, kMMaxTiles);
-
   // query tile: 64 rows x 9 chunks of 128 bytes, 128-byte swizzle.  Each row
-  // (1152 contiguous bytes) arrives with one bulk copy in the last two key
-  // stages, then the softmax warps rearrange it into the swizzled layout; the
-  // producer fills those two stages only after that (q_full).
-  uint8_t* q_raw = k_s + (kMStages - 2) * kTileBytes;
+  // (1152 contiguous bytes) arrives with one bulk copy in the last key stage,
+  // then the softmax warps rearrange it into the swizzled layout; the producer
+  // fills that stage only after that (q_full).
+  uint8_t* q_raw = k_s + (kMStages - 1) * kTileBytes;
   const int n_qrows = min(kMRows, rows_total - r0);
-  if (warp < 4) {
-    if (tid == 0) mbar_arrive_expect_tx(&q_stage, n_qrows * kDk * 2);
-    __syncwarp();
-    if (lane < 16) {
-      const int qr = warp * 16 + lane;
-      if (qr < n_qrows) {
-        const int qrg = r0 + qr;
-        const int qh = prm.pairs.heads[prm.pairs.head_off[pair] + qrg % nh];
-        bulk_load(q_raw + qr * (kDk * 2), a.q + b * a.qs0 + (qrg / nh) * a.qs1 + qh * a.qs2,
-                  kDk * 2, &q_stage);
-      }
-    }
-  }
+
+  // warp 4: the split's entries (list -> page table) and the tiles with a
+  // causally visible key (flag 128: the tile also holds a key some row must
+  // not see, or an unreadable group).  Done before the CTA barrier, so that
+  // these two dependent global reads overlap the barrier and TMEM set-up.
+  int n_act = 0;
   if (warp == 4) {
-    // ================= producer: the split's entries (list -> page table),
-    // the tiles with a causally visible key (flag 128: the tile also holds a
-    // key some row must not see, or an unreadable group), then TMA gathers of
-    // key tiles (values alias them)
     const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
     const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
     for (int i = lane; i < n_ent; i += 32) {
@@ -215,12 +194,11 @@ __global__ void __launch_bounds__(kMThreads, 1)
     }
     __syncwarp();
     const int q_lo = L - a.T + r0 / nh;   // smallest query position among the rows
-    int n_act = 0;
     for (int j0 = 0; j0 < n_tiles; j0 += 32) {
       const int j = j0 + lane;
       bool live = false, full = true;
       if (j < n_tiles)
-        for (int g = 0; g < 2; ++g) {
+        for (int g = 0; g < kMGroups; ++g) {
           const int2 gr = mgroup(ent_s, n_ent, a.P, j, g);
           live |= gr.x >= 0 && gr.y < L && gr.y <= max_q;
           full &= gr.x >= 0 && gr.y + 15 < L && gr.y + 15 <= q_lo;
@@ -231,35 +209,91 @@ __global__ void __launch_bounds__(kMThreads, 1)
       n_act += __popc(m);
     }
     __syncwarp();
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kMStages; ++s) {
+      for (int c = 0; c < kKC; ++c) mbar_init(&kv_full[s][c], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) mbar_init(&s_full[s], 1);
+    mbar_init(&p_full, 128);
+    mbar_init(&o_done, 1);
+    mbar_init(&q_full, 1);
+    mbar_init(&q_stage, 1);
+    mbar_init(&ent_ready, 1);
+    abort_s = 0;
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&q_stage, n_qrows * kDk * 2);
+  }
+  if (warp == 0) {   // the query rows, two per lane, as soon as q_stage exists
+    __syncwarp();
+    for (int qr = lane; qr < n_qrows; qr += 32) {
+      const int qrg = r0 + qr;
+      const int qh = prm.pairs.heads[prm.pairs.head_off[pair] + qrg % nh];
+      bulk_load(q_raw + qr * (kDk * 2), a.q + b * a.qs0 + (qrg / nh) * a.qs1 + qh * a.qs2,
+                kDk * 2, &q_stage);
+    }
+  }
+  if (warp == 5) {
+    tc::tmem_alloc(&tmem_base_s, kMTmemCols);
+    if (lane == 0) prefetch_tmap(&kmap);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = tmem_base_s;
+  volatile int* abort_flag = &abort_s;
+
+  if (warp == 4) {
+    // ================= producer: TMA gathers of key tiles (values alias them)
     if (lane == 0) {
       n_act_s = n_act;
       mbar_arrive(&ent_ready);
-      prefetch_tmap(&kmap);
+      const bool box64 = prm.box_rows == 64;
+      // (page, first row) of the boxes of tile j: one 64-row box (the tile lies
+      // in one page) or four 16-row groups; an absent group reads an
+      // out-of-range page (zero-filled)
+      auto boxes = [&](int j, int (&page)[kMGroups], int (&row0)[kMGroups]) {
+#pragma unroll
+        for (int g = 0; g < kMGroups; ++g) {
+          const int2 gr = mgroup(ent_s, n_ent, a.P, j, g);
+          const bool ok = gr.x >= 0 && gr.y < L;
+          page[g] = ok ? gr.x : a.P_pool;
+          row0[g] = ok ? gr.y % a.P : 0;
+        }
+      };
       for (int jj = 0; jj < n_act; ++jj) {
         const int st = jj % kMStages;
         if (jj >= kMStages &&
             !wait_or_abort_m(&kv_empty[st], ((jj / kMStages) - 1) & 1, abort_flag))
           break;
-        if (jj == kMStages - 2 && !wait_or_abort_m(&q_full, 0, abort_flag)) break;
-        const int j = act_s[jj] & 127;
+        if (jj == kMStages - 1 && !wait_or_abort_m(&q_full, 0, abort_flag)) break;
+        int page[kMGroups], row0[kMGroups];
+        boxes(act_s[jj] & 127, page, row0);
         uint8_t* kt = k_s + st * kTileBytes;
-        mbar_arrive_expect_tx(&kv_full[st], kTileBytes);
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const int2 gr = mgroup(ent_s, n_ent, a.P, j, g);
-          const bool ok = gr.x >= 0 && gr.y < L;
-          const int page = ok ? gr.x : a.P_pool;     // out of range: zero-filled box
-          const int row0 = ok ? gr.y % a.P : 0;
+        for (int c = 0; c < kKC; ++c) {
+          mbar_arrive_expect_tx(&kv_full[st][c], kChunkBytes);
+          if (box64) {
+            tma_load_4d(kt + c * kChunkBytes, &kmap, &kv_full[st][c], c * 64, row0[0], kvh,
+                        page[0]);
+          } else {
 #pragma unroll
-          for (int c = 0; c < kKC; ++c)
-            tma_load_4d(kt + c * kChunkBytes + g * 2048, &kmap, &kv_full[st], c * 64, row0, kvh,
-                        page);
+            for (int g = 0; g < kMGroups; ++g)
+              tma_load_4d(kt + c * kChunkBytes + g * 2048, &kmap, &kv_full[st][c], c * 64,
+                          row0[g], kvh, page[g]);
+          }
         }
       }
     }
   } else if (warp == 5) {
     // ================= MMA issuer (one thread).  Descriptors are advanced by
-    // adding (byte offset >> 4) to their start-address field.
+    // adding (byte offset >> 4) to their start-address field.  The MMAs go out
+    // in the order their inputs arrive, not tile by tile: PV of tile jp as soon
+    // as its P is in shared memory (it frees the tile's stage for the producer),
+    // else the next landed column chunk of QK of tile jq.  The tensor pipe runs
+    // them in issue order; QK of tile jq writes the S buffer that tile jq - 2
+    // used, which is free once PV of tile jq - 2 was issued (jq <= jp + 1).
     const bool ready = warp_wait_m(&ent_ready, 0, abort_flag);
     const int n_act = ready ? n_act_s : 0;
     if (lane == 0 && n_act > 0) {
@@ -267,41 +301,53 @@ __global__ void __launch_bounds__(kMThreads, 1)
       const uint64_t dk0 = tc::sdesc_sw128(smem_u32(k_s), 16, 1024);
       const uint64_t dp0 = tc::sdesc_sw128(smem_u32(p_s), 16, 1024);
       const uint64_t dv0 = tc::sdesc_sw128(smem_u32(k_s), kChunkBytes, 1024);
-      auto pv = [&](int jp) -> bool {
-        const int st = jp % kMStages;
-        if (!wait_or_abort_m(&p_full, jp & 1, abort_flag)) return false;
-        tc::fence_after_sync();
-        const uint64_t dv = dv0 + static_cast<uint64_t>((st * kTileBytes) >> 4);
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-          for (int kk = 0; kk < kMKeys / 16; ++kk)
-            tc::mma_bf16(tmem + (h ? kHiLanes : 0u), dp0 + static_cast<uint64_t>(kk * 2),
-                         dv + static_cast<uint64_t>((4 * h * kChunkBytes + kk * 2048) >> 4),
-                         kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
-        tc::commit(&o_done);
-        tc::commit(&kv_empty[st]);
-        return true;
-      };
       bool ok = wait_or_abort_m(&q_full, 0, abort_flag);
       tc::fence_after_sync();
-      for (int jj = 0; ok && jj < n_act; ++jj) {
-        const int st = jj % kMStages, sb = jj & 1;
-        if (!wait_or_abort_m(&kv_full[st], (jj / kMStages) & 1, abort_flag)) break;
-        tc::fence_after_sync();
-        const uint64_t dk = dk0 + static_cast<uint64_t>((st * kTileBytes) >> 4);
+      int jq = 0, cq = 0, jp = 0;   // next QK tile, its next column chunk; next PV tile
+      uint32_t idle = 0;
+      while (ok && jp < n_act) {
+        if (jp < jq && mbar_test_wait(&p_full, jp & 1)) {
+          tc::fence_after_sync();
+          const int st = jp % kMStages;
+          const uint64_t dv = dv0 + static_cast<uint64_t>((st * kTileBytes) >> 4);
 #pragma unroll
-        for (int c = 0; c < kKC; ++c)
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int kk = 0; kk < kMKeys / 16; ++kk)
+              tc::mma_bf16(tmem + (h ? kHiLanes : 0u), dp0 + static_cast<uint64_t>(kk * 2),
+                           dv + static_cast<uint64_t>((4 * h * kChunkBytes + kk * 2048) >> 4),
+                           kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+          tc::commit(&o_done);
+          tc::commit(&kv_empty[st]);
+          ++jp;
+          idle = 0;
+          continue;
+        }
+        if (jq < n_act && jq <= jp + 1 &&
+            mbar_test_wait(&kv_full[jq % kMStages][cq], (jq / kMStages) & 1)) {
+          tc::fence_after_sync();
+          const uint64_t dk = dk0 + static_cast<uint64_t>(((jq % kMStages) * kTileBytes +
+                                                           cq * kChunkBytes) >> 4);
+          const uint64_t dq = dq0 + static_cast<uint64_t>((cq * kMRows * 128) >> 4);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc::mma_bf16(tmem + kSCol + sb * kMKeys,
-                         dq0 + static_cast<uint64_t>((c * kMRows * 128 + kk * 32) >> 4),
-                         dk + static_cast<uint64_t>((c * kChunkBytes + kk * 32) >> 4), kIdQK,
-                         (c | kk) ? 1u : 0u);
-        tc::commit(&s_full[sb]);
-        if (jj >= 1 && !pv(jj - 1)) ok = false;
+            tc::mma_bf16(tmem + kSCol + (jq & 1) * kMKeys, dq + static_cast<uint64_t>(kk * 2),
+                         dk + static_cast<uint64_t>(kk * 2), kIdQK, (cq | kk) ? 1u : 0u);
+          if (++cq == kKC) {
+            tc::commit(&s_full[jq & 1]);
+            cq = 0;
+            ++jq;
+          }
+          idle = 0;
+          continue;
+        }
+        ++idle;
+        if ((idle & 1023u) == 0u && *abort_flag) ok = false;
+        if (idle >= kSpinLimit) {
+          *abort_flag = 1;
+          ok = false;
+        }
       }
-      if (ok) pv(n_act - 1);
     }
   } else {
     // ================= softmax / epilogue.  Row 16w + (l & 15) is shared by
@@ -313,10 +359,11 @@ __global__ void __launch_bounds__(kMThreads, 1)
     {
       // raw query rows -> swizzled K-major chunks (rows past the CTA's: zeros)
       const bool qok = warp_wait_m(&q_stage, 0, abort_flag);
+#pragma unroll 4
       for (int i = tid; i < kMRows * kKC * 8; i += 128) {
         const int row = i / (kKC * 8), ch = i % (kKC * 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (qok && row < n_qrows) v = *reinterpret_cast<const uint4*>(q_raw + row * (kDk * 2) + ch * 16);
+        uint4 v = *reinterpret_cast<const uint4*>(q_raw + row * (kDk * 2) + ch * 16);
+        if (!(qok && row < n_qrows)) v = make_uint4(0, 0, 0, 0);
         *reinterpret_cast<uint4*>(q_s + (ch >> 3) * (kMRows * 128) + row * 128 +
                                   (((ch & 7) ^ (row & 7)) << 4)) = v;
       }
@@ -344,28 +391,36 @@ __global__ void __launch_bounds__(kMThreads, 1)
         break;
       }
       tc::fence_after_sync();
-      float x[32];
-      tc::ld32(tmem + lane_base + kSCol + sb * kMKeys, x);
-      tc::wait_ld();
-      float v[16];   // this lane's 16 keys: 0-15 (low lane) or 16-31 (high lane)
+      float v[32];   // this lane's 32 keys: 0-31 (low lane) or 32-63 (high lane)
+      {
+        float x[32];
+        tc::ld32(tmem + lane_base + kSCol + sb * kMKeys, v);
+        tc::ld32(tmem + lane_base + kSCol + sb * kMKeys + 32, x);
+        tc::wait_ld();
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float hv = __shfl_sync(0xffffffffu, x[16 + i], lane & 15);
-        v[i] = low ? x[i] : hv;
-      }
-      if (code & 128) {   // mask this lane's 16-key group
-        const int2 gr = mgroup(ent_s, n_ent, a.P, j, low ? 0 : 1);
-        const bool gok = gr.x >= 0;
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int kp = gr.y + c;
-          if (!(gok && kp < L && kp <= qpos)) v[c] = -INFINITY;
+        for (int i = 0; i < 32; ++i) {
+          const float hv = __shfl_sync(0xffffffffu, x[i], lane & 15);
+          v[i] = low ? v[i] : hv;
         }
       }
-      float m4[4];
+      if (code & 128) {   // mask this lane's two 16-key groups
 #pragma unroll
-      for (int i = 0; i < 4; ++i) m4[i] = fmaxf(fmaxf(v[i], v[i + 4]), fmaxf(v[i + 8], v[i + 12]));
-      float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        for (int gg = 0; gg < 2; ++gg) {
+          const int2 gr = mgroup(ent_s, n_ent, a.P, j, (low ? 0 : 2) + gg);
+          const bool gok = gr.x >= 0;
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int kp = gr.y + c;
+            if (!(gok && kp < L && kp <= qpos)) v[gg * 16 + c] = -INFINITY;
+          }
+        }
+      }
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        m8[i] = fmaxf(fmaxf(v[i], v[i + 8]), fmaxf(v[i + 16], v[i + 24]));
+      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * sl2;   // the row's max, scaled
       // PV of the previous tile done: O is stable and the P buffer free
       if (jj >= 1 && !warp_wait_m(&o_done, (jj - 1) & 1, abort_flag)) {
@@ -393,19 +448,17 @@ __global__ void __launch_bounds__(kMThreads, 1)
       const float nb = m_ref == -INFINITY ? 0.f : -m_ref;
       uint8_t* prow = p_s + r * 128;
 #pragma unroll
-      for (int ch = 0; ch < 2; ++ch) {
+      for (int ch = 0; ch < 4; ++ch) {
         float p[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          p[i] = exp2f(fmaf(v[ch * 8 + i], sl2, nb));
-          l += p[i];
-        }
+        for (int i = 0; i < 8; ++i) p[i] = exp2f(fmaf(v[ch * 8 + i], sl2, nb));
+        l += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         uint4 w;
         w.x = pack_bf16(p[0], p[1]);
         w.y = pack_bf16(p[2], p[3]);
         w.z = pack_bf16(p[4], p[5]);
         w.w = pack_bf16(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + ((((low ? 0 : 2) + ch) ^ (r & 7)) << 4)) = w;
+        *reinterpret_cast<uint4*>(prow + ((((low ? 0 : 4) + ch) ^ (r & 7)) << 4)) = w;
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();
@@ -459,6 +512,7 @@ cudaError_t launch_mla(const DecodeArgs& a, const PairTable& pairs, const CUtens
   MlaParams prm;
   prm.a = a;
   prm.pairs = pairs;
+  prm.box_rows = a.P % 64 == 0 ? 64 : 16;
   // one work item per (pair, 64-row tile): no CTA for row tiles a pair lacks
   prm.n_items = 0;
   for (int i = 0; i < pairs.n_pairs; ++i)

@@ -715,6 +715,26 @@ def test_mla_decode_vs_oracle(seed, L, n_splits):
     assert_attn_close(o, lse, ro, rl)
 
 
+@pytest.mark.parametrize("page_size,L,Hq,n_splits", [(32, 1000, 48, 2), (48, 1100, 40, 3),
+                                                     (128, 2300, 48, 2), (16, 777, 36, 1)])
+def test_mla_decode_page_sizes(page_size, L, Hq, n_splits):
+    """64-key tiles over pages of 16-48 tokens (a tile spans pages: 16-row groups), of 128
+    tokens (two tiles per page: boxes start at row 0 or 64) and ragged row tiles (T x Hq
+    rows not a multiple of 64)."""
+    cfg = W.MLADecode("case", B=2, T=2, Hq=Hq, Dk=576, Dv=512, page_size=page_size, seq_len=L,
+                      alpha=3, beta=6, h_ambient=8)
+    inp = W.mla_decode_inputs(cfg, seed=7, device="cpu")
+    sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                           page_size)
+    lists, counts = mla_lists_from_oracle(inp, sig, cfg)
+    o, lse, h2l = run_mla(inp, cfg, lists, counts, n_splits)
+    kvb = bits(inp["kv"])
+    ro, rl = O.sparse_attention(bits(inp["q"]), kvb, kvb[..., :cfg.Dv], np_i32(inp["page_table"]),
+                                np_i32(inp["seq_lens"]), lists, counts, np.array(h2l),
+                                1.0 / math.sqrt(cfg.Dk), page_size)
+    assert_attn_close(o, lse, ro, rl)
+
+
 @pytest.mark.slow
 def test_mla_decode_full_size_sampled():
     cfg = W.MLA_MTP
