@@ -170,7 +170,8 @@ SA_API int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4
  *  page_table (dev) [B,max_pages] int32;  seq_lens (dev) [B] int32
  *  lists      (dev) [B,2,alpha+beta] int32;  list_counts (dev) [B,2] int32
  *  workspace  (dev) sa_select_tiered_workspace_size(B,T,Hq,max_pages) bytes
- * Supported: Dk % 8 == 0, Dk <= 880, max_pages <= 16384.
+ * Supported: Dk % 8 == 0, Dk <= 880, max_pages <= 8192 (the choose pass keeps
+ * 21 bytes per page in shared memory).
  */
 SA_API int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
                                   const uint16_t* summaries, const int32_t* page_table,

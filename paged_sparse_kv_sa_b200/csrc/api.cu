@@ -260,7 +260,7 @@ int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
   if (int r = check_q(q, q_strides)) return r;
   if (!summaries || !aligned16(summaries) || !page_table || !seq_lens || !lists || !list_counts)
     return SA_ERR_INVALID_ARG;
-  if (Dk % 8 != 0 || Dk > 880 || max_pages > 16384 || B > 65535) return SA_ERR_UNSUPPORTED;
+  if (Dk % 8 != 0 || Dk > 880 || max_pages > 8192 || B > 65535) return SA_ERR_UNSUPPORTED;
   if (!workspace || !aligned16(workspace) ||
       workspace_bytes < tiered_workspace_bytes(B, T, Hq, max_pages))
     return SA_ERR_WORKSPACE;

@@ -337,11 +337,32 @@ __device__ __noinline__ double exact_row_dot(const uint16_t* q, const uint16_t* 
 // kChoosePairs bounds the (undecided page, row group) pairs whose rescoring
 // tasks are flattened to (page, row) and spread evenly over every warp of the
 // sequence's CTAs; beyond it each warp takes whole (page, row group) pairs.
-constexpr int kChoosePairs = 2048;
+constexpr int kChoosePairs = 1024;
+// Boundaries up to kChooseGroups pages deep prune the pages by a threshold
+// first (below); deeper ones classify every page.
+constexpr int kChooseGroups = 256;
+// Shared memory per page of the choose kernel: two brackets, two indices, a flag.
+constexpr int kChooseBytesPerPage = 8 + 8 + 2 + 2 + 1;
+static_assert(kChooseGroups <= kChooseThreads, "one thread clears each group maximum");
 
+// Classification of a page p for a boundary of k pages (k < N), from the
+// brackets [lo, hi] of every page's score (rigorous: the exact score lies in
+// them), ties to the lower logical page:
+//   certainly inside   iff  #{q : hi_q >= lo_p} <= k   (p included: even at
+//                            lo_p it cannot be passed by k others)
+//   undecided           iff  not inside and #{q : lo_q > hi_p} < k
+//   certainly outside   otherwise (k pages are above it whatever the scores).
+// Both counts only need the candidate pages, those with hi >= tau, where tau
+// is the kmax-th largest of the largest lower ends of G disjoint groups of
+// pages (kmax = the deepest boundary, kmax <= G): kmax pages have lo >= tau,
+// so a page with hi < tau is outside every boundary, adds nothing to
+// #{lo_q > hi_p} for a candidate p, and adds nothing to #{hi_q >= lo_p} when
+// lo_p >= tau; a page with lo_p < tau has at least kmax + 1 upper ends at or
+// above lo_p, so it is never inside.
 __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const TieredArgs a) {
   pdl_wait_and_release();
   const int b = blockIdx.x, cta = blockIdx.y, n_cta = gridDim.y, tid = threadIdx.x;
+  const int nw = kChooseThreads / 32, warp = tid >> 5, lane = tid & 31;
   int L = a.seq_lens[b];
   if (L < 0 || L > a.max_pages * a.P) {
     if (tid == 0 && cta == 0) set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
@@ -351,83 +372,174 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
   const int cap = a.alpha + a.beta;
   int32_t* out0 = a.lists + (int64_t)b * 2 * cap;
   int32_t* out1 = out0 + cap;
+  // per page: the merged brackets (later (page, flags) of each undecided
+  // page), the candidates' brackets (later the physical page of each undecided
+  // page, then its exact score), the page of each candidate, the candidate of
+  // each undecided page, the candidates' flags
   extern __shared__ __align__(16) uint8_t dsm[];
-  float* lo = reinterpret_cast<float*>(dsm);
-  float* hi = lo + a.max_pages;
-  int* ph_s = reinterpret_cast<int*>(hi + a.max_pages);        // physical page of u_list[i]
-  uint16_t* u_list = reinterpret_cast<uint16_t*>(ph_s + a.max_pages);
-  uint8_t* flag = reinterpret_cast<uint8_t*>(u_list + a.max_pages);
-  __shared__ uint32_t hist[1024];
-  __shared__ uint32_t sel_out[8];
-  __shared__ BucketScratch bscr;
+  float2* lohi = reinterpret_cast<float2*>(dsm);
+  int* uf = reinterpret_cast<int*>(dsm);
+  float2* c_lohi = reinterpret_cast<float2*>(dsm + 8 * (size_t)a.max_pages);
+  int* ph_s = reinterpret_cast<int*>(c_lohi);
+  double* ex = reinterpret_cast<double*>(c_lohi);
+  uint16_t* c_pg = reinterpret_cast<uint16_t*>(dsm + 16 * (size_t)a.max_pages);
+  uint16_t* u_list = c_pg + a.max_pages;
+  uint8_t* c_fl = reinterpret_cast<uint8_t*>(u_list + a.max_pages);
+  __shared__ __align__(16) uint32_t gmax[kChooseGroups];   // order keys of the groups' largest lower ends
+  __shared__ uint32_t cmask[kChoosePairs];   // flagged rows of (candidate, row group), when they fit
+  __shared__ uint32_t tau_key;
   __shared__ int pfx[kChoosePairs];          // exclusive prefix of the flagged rows per pair
   __shared__ uint32_t msk[kChoosePairs];     // flagged rows of (undecided page, row group)
-  __shared__ int red_i[kChooseThreads / 32];
+  __shared__ int red_i[nw];
   __shared__ int n_cert[2];
-  __shared__ int last_s;
+  __shared__ int nu_s, last_s;
   const int kb[2] = {min(a.alpha, N), min(a.alpha + a.beta, N)};
-  // flag bits: 1 / 2 = in tier boundary 0 / 1, 4 / 8 = undecided for it
-  // (the row groups' brackets of a thread's pages, 8 loads in flight at a time)
-  for (int p = tid; p < N; p += blockDim.x) {
-    float l = -INFINITY, h = -INFINITY;
-    for (int rg0 = 0; rg0 < a.n_rg; rg0 += 8) {
-      float2 v[8];   // (index clamped: the loads are unconditional; a repeat does not change a max)
+  int kmax = 0;
+  bool every = false;   // a boundary holds every page: no pruning
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        v[j] = a.lohi[((int64_t)b * a.n_rg + min(rg0 + j, a.n_rg - 1)) * a.max_pages + p];
+  for (int i = 0; i < 2; ++i) {
+    if (kb[i] > 0 && kb[i] >= N) every = true;
+    if (kb[i] > 0 && kb[i] < N) kmax = max(kmax, kb[i]);
+  }
+  const int G = min(kChooseGroups, N);   // groups p G / N: none empty
+  const bool prune = !every && kmax > 0 && kmax <= G;
+  if (tid < kChooseGroups) gmax[tid] = 0u;   // below every non-NaN key
+  if (tid == 0) {
+    n_cert[0] = n_cert[1] = 0;
+    tau_key = 0u;
+  }
+  __syncthreads();
+  // the row groups' brackets of a thread's pages p and p + blockDim.x, 16 loads
+  // in flight at a time (indices clamped: the loads are unconditional, and a
+  // repeated row group or page does not change a max)
+  for (int p = tid; p < N; p += 2 * blockDim.x) {
+    const int p2 = p + blockDim.x, pc = min(p2, N - 1);
+    float l[2] = {-INFINITY, -INFINITY}, h[2] = {-INFINITY, -INFINITY};
+    for (int rg0 = 0; rg0 < a.n_rg; rg0 += 8) {
+      float2 v[2][8];
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
-        l = fmaxf(l, v[j].x);
-        h = fmaxf(h, v[j].y);
+        const int64_t row = ((int64_t)b * a.n_rg + min(rg0 + j, a.n_rg - 1)) * a.max_pages;
+        v[0][j] = a.lohi[row + p];
+        v[1][j] = a.lohi[row + pc];
       }
-    }
-    lo[p] = l;
-    hi[p] = h;
-  }
-  if (tid == 0) n_cert[0] = n_cert[1] = 0;
-  __syncthreads();
-  // both boundaries' order statistics in one selection pass
-  float Lk[2] = {INFINITY, INFINITY}, H[2] = {INFINITY, INFINITY};
-  {
-    int act[2], kl[2], kh[2], na = 0;
-    for (int i = 0; i < 2; ++i)
-      if (kb[i] > 0 && kb[i] < N) {
-        act[na] = i;
-        kl[na] = kb[i];
-        kh[na] = kb[i] + 1;
-        ++na;
-      }
-    if (na > 0) {
-      float ol[2], oh[2];
-      if (!bucket_select(lo, hi, N, na, kl, kh, &bscr, ol, oh))
-        for (int j = 0; j < na; ++j) radix_select2(lo, hi, N, kl[j], kh[j], hist, sel_out, ol[j], oh[j]);
-      for (int j = 0; j < na; ++j) {
-        Lk[act[j]] = ol[j];
-        H[act[j]] = oh[j];
-      }
-    }
-  }
-  for (int p = tid; p < N; p += blockDim.x) {
-    uint8_t f = 0;
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      if (kb[i] >= N) {            // every page is inside this boundary
-        f |= 1u << i;
-      } else if (kb[i] > 0) {
-        if (lo[p] > H[i]) {
-          f |= 1u << i;
-          atomicAdd(&n_cert[i], 1);
-        } else if (hi[p] >= Lk[i]) {
-          f |= 4u << i;
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          l[i] = fmaxf(l[i], v[i][j].x);
+          h[i] = fmaxf(h[i], v[i][j].y);
+        }
+    }
+    lohi[p] = make_float2(l[0], h[0]);
+    if (prune) atomicMax(&gmax[p * G / N], f2key(l[0]));
+    if (p2 < N) {
+      lohi[p2] = make_float2(l[1], h[1]);
+      if (prune) atomicMax(&gmax[p2 * G / N], f2key(l[1]));
+    }
+  }
+  __syncthreads();
+  float tau = -INFINITY;
+  if (prune) {   // tau: the largest group maximum with at least kmax group maxima at or above it
+    if (tid < G) {   // (groups G.. hold 0, below every key: never counted)
+      const uint32_t mine = gmax[tid];
+      const uint4* g4 = reinterpret_cast<const uint4*>(gmax);
+      int c = 0;
+#pragma unroll 8
+      for (int j = 0; j < kChooseGroups / 4; ++j) {
+        const uint4 v = g4[j];
+        c += (v.x >= mine) + (v.y >= mine) + (v.z >= mine) + (v.w >= mine);
+      }
+      if (c >= kmax) atomicMax(&tau_key, mine);
+    }
+    __syncthreads();
+    tau = key2f(tau_key);
+  }
+  // the candidates (hi >= tau), ascending: thread t scans pages [t ppt, (t + 1) ppt)
+  int nc;
+  {
+    const int ppt = (N + blockDim.x - 1) / blockDim.x;
+    const int q0 = tid * ppt, q1 = min(N, q0 + ppt);
+    int cnt = 0;
+    for (int p = q0; p < q1; ++p) cnt += lohi[p].y >= tau;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) red_i[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    nc = 0;
+    for (int i = 0; i < nw; ++i) {
+      if (i < warp) pos += red_i[i];
+      nc += red_i[i];
+    }
+    for (int p = q0; p < q1; ++p) {
+      const float2 v = lohi[p];
+      if (v.y >= tau) {
+        c_pg[pos] = static_cast<uint16_t>(p);
+        c_lohi[pos++] = v;
+      }
+    }
+    __syncthreads();
+  }
+  // classify the candidates by counting over the candidates, one thread each
+  // (every lane reads the same bracket: a broadcast); meanwhile the candidate's
+  // row masks are fetched for the exact rescoring, when they fit
+  const bool cm = a.n_rg <= 8 && nc * a.n_rg <= kChoosePairs;
+  for (int i = tid; i < nc; i += blockDim.x) {
+    uint32_t rm[8];
+    if (cm) {
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        rm[g] = static_cast<uint32_t>(
+            a.rmask[((int64_t)b * a.n_rg + min(g, a.n_rg - 1)) * a.max_pages + c_pg[i]]);
+    }
+    const float2 me = c_lohi[i];
+    int n_hi = 0, n_lo = 0;   // #{hi_q >= lo_p}, #{lo_q > hi_p}
+#pragma unroll 4
+    for (int j = 0; j < nc; ++j) {
+      const float2 o = c_lohi[j];
+      n_hi += o.y >= me.x;
+      n_lo += o.x > me.y;
+    }
+    uint8_t f = 0;   // bits 1 / 2: inside boundary 0 / 1; 4 / 8: undecided for it
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      if (kb[k] >= N) {
+        if (kb[k] > 0) f |= 1u << k;
+      } else if (kb[k] > 0) {
+        if (me.x >= tau && n_hi <= kb[k]) {
+          f |= 1u << k;
+          atomicAdd(&n_cert[k], 1);
+        } else if (n_lo < kb[k]) {
+          f |= 4u << k;
         }
       }
     }
-    flag[p] = f;
+    c_fl[i] = f;
+    if (cm)
+#pragma unroll
+      for (int g = 0; g < 8; ++g)
+        if (g < a.n_rg) cmask[i * a.n_rg + g] = rm[g];
   }
   __syncthreads();
-  // the undecided pages, ascending (the same list in every CTA of the sequence)
-  const int nu_ = compact_flag_list(flag, N, 12u, u_list, red_i);
-  double* ex = reinterpret_cast<double*>(lo);   // lo/hi storage reused as doubles
+  // the undecided candidates, ascending (one warp, ballots)
+  if (warp == 0) {
+    int nu = 0;
+    for (int j0 = 0; j0 < nc; j0 += 32) {
+      const int j = j0 + lane;
+      const bool u = j < nc && (c_fl[j] & 12u);
+      const uint32_t m = __ballot_sync(0xffffffffu, u);
+      if (u) u_list[nu + __popc(m & ((1u << lane) - 1u))] = static_cast<uint16_t>(j);
+      nu += __popc(m);
+    }
+    if (lane == 0) nu_s = nu;
+  }
+  __syncthreads();
+  const int nu_ = nu_s;
   if (nu_ == 0 && cta != 0) return;             // nothing to share: CTA 0 writes
   if (nu_ > 0) {
     // exact row-max scores of the undecided pages: only the query rows the
@@ -436,12 +548,11 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     // rescores each such (page, row) exactly; the results are merged with an
     // atomic max in global memory and the last CTA to finish ranks.
     const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
-    const int nw = kChooseThreads / 32, warp = tid >> 5, lane = tid & 31;
     const int gw = cta + n_cta * warp, n_gw = n_cta * nw;   // this warp among the sequence's
     unsigned long long* exk = a.exkey + (int64_t)b * a.max_pages;
     const int npair = nu_ * a.n_rg;
-    for (int i = tid; i < nu_; i += blockDim.x) {
-      const int ph = ptrow[u_list[i]];
+    for (int i = tid; i < nu_; i += blockDim.x) {   // (the brackets are dead: ph_s aliases them)
+      const int ph = ptrow[c_pg[u_list[i]]];
       ph_s[i] = (ph < 0 || ph >= a.P_pool) ? -1 : ph;
     }
     if (npair <= kChoosePairs) {
@@ -452,7 +563,9 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
       for (int x = x0; x < x1; ++x) {
         const int uu = x / a.n_rg, g = x % a.n_rg;
         const uint32_t m =
-            static_cast<uint32_t>(a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + u_list[uu]]);
+            cm ? cmask[u_list[uu] * a.n_rg + g]
+               : static_cast<uint32_t>(
+                     a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + c_pg[u_list[uu]]]);
         msk[x] = m;
         cnt += __popc(m);
       }
@@ -497,7 +610,8 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
         const int uu = x / a.n_rg, g = x % a.n_rg;
         const int ph = ph_s[uu];
         if (ph < 0) continue;
-        unsigned long long bits = a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + u_list[uu]];
+        unsigned long long bits =
+            a.rmask[((int64_t)b * a.n_rg + g) * a.max_pages + c_pg[u_list[uu]]];
         const uint16_t* sg = a.sig + (int64_t)ph * a.Dk;
         while (bits) {
           const int r = g * kTR + __ffsll(static_cast<long long>(bits)) - 1;
@@ -514,20 +628,22 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
     __syncthreads();
     if (!last_s) return;
     __threadfence();
+    // (no exact result: an unreadable page, scored -inf; ex now aliases ph_s)
     for (int i = tid; i < nu_; i += blockDim.x) {
       const unsigned long long k = __ldcg(&exk[i]);
-      ex[i] = (ph_s[i] < 0 || k == 0ull) ? -INFINITY : key2d(k);
+      ex[i] = k == 0ull ? -INFINITY : key2d(k);
+      const int ci = u_list[i];
+      uf[i] = c_pg[ci] | (c_fl[ci] << 16);
     }
     __syncthreads();
     // per boundary: the undecided pages fill the slots the certain ones left
     for (int u = tid; u < nu_; u += blockDim.x) {
-      const int pu = u_list[u];
-      const uint8_t fu = flag[pu];
+      const int cu = u_list[u], pu = c_pg[cu];
+      const uint8_t fu = c_fl[cu];
       const double su = ex[u];
       int rank[2] = {0, 0};
       for (int v = 0; v < nu_; ++v) {
-        const int pv = u_list[v];
-        const uint8_t fv = flag[pv];
+        const int pf = uf[v], pv = pf & 0xffff, fv = pf >> 16;
         const double sv = ex[v];
         const int ahead = (sv > su) || (sv == su && pv < pu);
         rank[0] += ahead & (fv >> 2);
@@ -537,15 +653,32 @@ __global__ void __launch_bounds__(kChooseThreads) tiered_choose_kernel(const Tie
 #pragma unroll
       for (int i = 0; i < 2; ++i)
         if (((fu >> (2 + i)) & 1u) && rank[i] < kb[i] - n_cert[i]) add |= 1u << i;
-      if (add) flag[pu] = fu | add;
+      if (add) c_fl[cu] = fu | add;
     }
     __syncthreads();
   }
-  int c0, c1;
-  compact_pages2(flag, N, out0, out1, cap, red_i, c0, c1);
-  if (tid == 0) {
-    a.counts[2 * b] = c0;
-    a.counts[2 * b + 1] = c1;
+  // both lists: the candidates inside each boundary, ascending, -1 padded
+  if (warp == 0) {
+    int c[2] = {0, 0};
+    for (int j0 = 0; j0 < nc; j0 += 32) {
+      const int j = j0 + lane;
+      const uint8_t f = j < nc ? c_fl[j] : 0;
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const bool in = (f >> k) & 1u;
+        const uint32_t m = __ballot_sync(0xffffffffu, in);
+        const int pos = c[k] + __popc(m & ((1u << lane) - 1u));
+        if (in && pos < cap) (k ? out1 : out0)[pos] = c_pg[j];
+        c[k] += __popc(m);
+      }
+    }
+    const int c0 = min(c[0], cap), c1 = min(c[1], cap);
+    for (int i = c0 + lane; i < cap; i += 32) out0[i] = -1;
+    for (int i = c1 + lane; i < cap; i += 32) out1[i] = -1;
+    if (lane == 0) {
+      a.counts[2 * b] = c0;
+      a.counts[2 * b + 1] = c1;
+    }
   }
 }
 
@@ -573,7 +706,7 @@ cudaError_t launch_select_tiered(TieredArgs a, cudaStream_t stream) {
   dim3 g1((a.max_pages + kSP - 1) / kSP, (a.T * a.Hq + kSR - 1) / kSR, a.B);
   e = launch_pdl(tiered_score_kernel, g1, dim3(kSThreads), dyn1, stream, a);
   if (e != cudaSuccess) return e;
-  const size_t dyn2 = (size_t)a.max_pages * (4 + 4 + 4 + 2 + 1) + 16;
+  const size_t dyn2 = (size_t)a.max_pages * kChooseBytesPerPage + 16;
   e = cudaFuncSetAttribute(tiered_choose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)dyn2);
   if (e != cudaSuccess) return e;

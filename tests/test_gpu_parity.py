@@ -598,6 +598,29 @@ def test_select_tiered_small(seed, L):
     check_tiered(cfg, inp, sig)
 
 
+@pytest.mark.parametrize("alpha,beta,n_pages,Dk", [(0, 12, 200, 576), (100, 200, 400, 128),
+                                                   (5, 35, 3000, 128)])
+def test_select_tiered_depths(alpha, beta, n_pages, Dk):
+    """No critical tier; a boundary deeper than the threshold pruning covers (every page
+    classified by counting); several thousand pages (several pages per thread)."""
+    cfg, inp, sig = tiered_case(11, B=2, T=2, Hq=16, Dk=Dk, P=16, L=n_pages * 16 - 7,
+                                alpha=alpha, beta=beta)
+    check_tiered(cfg, inp, sig)
+
+
+def test_select_tiered_max_pages_limit():
+    """The widest page table the tiered selection takes (8192 pages: its choose pass keeps
+    21 bytes per page in shared memory) runs and matches; one page wider is refused."""
+    cfg, inp, sig = tiered_case(5, B=1, T=1, Hq=8, Dk=64, P=16, L=8192 * 16, alpha=4, beta=28)
+    assert inp["page_table"].shape[1] == 8192
+    check_tiered(cfg, inp, sig)
+    g = {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+    wide = torch.cat([g["page_table"], torch.full((1, 1), -1, dtype=torch.int32, device=DEV)], 1)
+    with pytest.raises(sa.SAError, match="UNSUPPORTED"):
+        sa.sa_select_pages_tiered(g["q"], to_bf16_dev(sig), wide, g["seq_lens"], cfg.page_size,
+                                  cfg.alpha, cfg.beta)
+
+
 def test_select_tiered_ties():
     cfg, inp, sig = tiered_case(3, B=2, T=1, Hq=8, Dk=128, P=16, L=30 * 16, alpha=2, beta=4)
     inp["q"][0] = 0                                     # all scores tie: lowest pages
