@@ -32,6 +32,10 @@ namespace sa {
 namespace {
 
 constexpr int kThreads = 512;       // choose_kernel
+constexpr int kSelGroups = 256;     // choose_kernel: group maxima behind the pruning threshold
+constexpr int kCandCap = 1024;      // choose_kernel: candidates classified by counting (more:
+                                    // order statistics of the bounds over every page)
+static_assert(kSelGroups <= kThreads, "one thread clears each group maximum");
 constexpr int kScoreChunk = 128;    // score_kernel: logical pages per CTA
 constexpr int kScoreStages = 2;     // ring slots of 16 pages
 constexpr int kScoreMaxHB = 8;      // kv heads per CTA (one consumer warp each)
@@ -307,12 +311,26 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
   }
 }
 
-// Radix selection of the bounds, exact rescoring of the undecided pages, and
-// the ascending output of forced + selected pages.
+// Classification of the candidate pages (neither sink nor local) for the k
+// slots, from the bracket [lo, hi] of each page's score (rigorous: the exact
+// score lies in it), ties to the lower logical page:
+//   certainly selected  iff  #{q : hi_q >= lo_p} <= k   (p included)
+//   undecided           iff  not certain and #{q : lo_q > hi_p} < k
+//   out                 otherwise.
+// The counts only need the pages with hi >= tau, where tau is the k-th largest
+// of the largest lower ends of G disjoint groups of pages (k <= G): k pages have
+// lo >= tau, so a page with hi < tau is out, adds nothing to #{lo_q > hi_p} for
+// a kept page p, and adds nothing to #{hi_q >= lo_p} when lo_p >= tau; a page
+// with lo_p < tau has at least k + 1 upper ends at or above lo_p and is never
+// certain.  With more than kCandCap kept pages the same classification is
+// made from the order statistics of the bounds (lo_p > the (k+1)-th largest hi;
+// hi_p >= the k-th largest lo) over every page.  The undecided pages are then
+// rescored exactly and ranked, and the output is the sink pages, the selected
+// pages and the local pages, ascending.
 __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   pdl_wait_and_release();
   const int kvh = blockIdx.x, b = blockIdx.y;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int L = clamped_len(a, b, tid == 0);
   const int N = (L + a.P - 1) / a.P;
   int32_t* outp = a.out_pages + ((int64_t)b * a.Hkv + kvh) * a.budget_pages;
@@ -331,6 +349,10 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   __shared__ int red_i[kThreads / 32];
   __shared__ int n_unc, n_certain;
   __shared__ double ex_tmp[kThreads];
+  __shared__ __align__(16) uint32_t gmax[kSelGroups];   // order keys of the groups' largest lo
+  __shared__ uint32_t tau_key;
+  __shared__ float2 c_lohi[kCandCap];                   // the kept pages' bounds, ascending
+  __shared__ uint16_t c_pg[kCandCap];
 
   SelSmem S;
   S.lo = reinterpret_cast<float*>(dsm);
@@ -341,11 +363,17 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   const int G = a.Hq / a.Hkv, R = a.T * G, Dk = a.Dk;
   const int n_sink = min(a.n_sink, N), local0 = max(N - a.n_local, 0);
   const int k = a.k_top;
+  const int M = local0 - n_sink;              // candidate pages (more than k here)
+  const int Gs = min(kSelGroups, M);          // groups (p - n_sink) Gs / M: none empty
+  const bool prune = k > 0 && k <= Gs;
   const float2* lohi = a.lohi + ((int64_t)b * a.Hkv + kvh) * a.max_pages;
   if (tid == 0) {
     n_unc = 0;
     n_certain = 0;
+    tau_key = 0u;
   }
+  if (tid < kSelGroups) gmax[tid] = 0u;        // below every non-NaN key
+  __syncthreads();
   // (loads in batches of 8 per thread, all in flight together)
   for (int p0 = 0; p0 < N; p0 += 8 * kThreads) {
     float2 v[8];
@@ -362,25 +390,92 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
         S.flag[p] = (p >= n_sink && p < local0) ? 0 : 1;
         S.lo[p] = v[j].x;
         S.hi[p] = v[j].y;
+        if (prune && p >= n_sink && p < local0 && !isnan(v[j].x))
+          atomicMax(&gmax[(p - n_sink) * Gs / M], f2key(v[j].x));
       }
     }
   }
   __syncthreads();
-
-  // ---- order statistics of the bounds (k == 0: streaming, no winners)
-  float Lk = INFINITY, H = INFINITY;
-  if (k > 0 && !filtered_select2(S.lo, S.hi, N, k, k + 1, &scratch, Lk, H))
-    radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
-
-  // ---- classify: certainly in (lo > H), undecided (hi >= Lk), else out
-  for (int p = tid; p < N; p += blockDim.x) {
-    if (S.flag[p] != 0) continue;
-    if (S.lo[p] > H) {
-      S.flag[p] = 1;
-      atomicAdd(&n_certain, 1);
-    } else if (S.hi[p] >= Lk) {
-      S.flag[p] = 2;
-      S.u_list[atomicAdd(&n_unc, 1)] = static_cast<uint16_t>(p);
+  float tau = -INFINITY;
+  if (prune) {   // the largest group maximum with at least k group maxima at or above it
+    if (tid < Gs) {   // (groups Gs.. hold 0, below every key: never counted)
+      const uint32_t mine = gmax[tid];
+      const uint4* g4 = reinterpret_cast<const uint4*>(gmax);
+      int c = 0;
+#pragma unroll 8
+      for (int j = 0; j < kSelGroups / 4; ++j) {
+        const uint4 w = g4[j];
+        c += (w.x >= mine) + (w.y >= mine) + (w.z >= mine) + (w.w >= mine);
+      }
+      if (c >= k) atomicMax(&tau_key, mine);
+    }
+    __syncthreads();
+    tau = key2f(tau_key);
+  }
+  // the kept candidate pages (hi >= tau), ascending: thread t scans [t ppt, (t + 1) ppt)
+  int nc = 0;
+  if (k > 0) {
+    const int ppt = (N + blockDim.x - 1) / blockDim.x;
+    const int q0 = tid * ppt, q1 = min(N, q0 + ppt);
+    int cnt = 0;
+    for (int p = q0; p < q1; ++p) cnt += S.flag[p] == 0 && S.hi[p] >= tau;
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int w = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += w;
+    }
+    if (lane == 31) red_i[warp] = incl;
+    __syncthreads();
+    int pos = incl - cnt;
+    for (int i = 0; i < kThreads / 32; ++i) {
+      if (i < warp) pos += red_i[i];
+      nc += red_i[i];
+    }
+    if (nc <= kCandCap)
+      for (int p = q0; p < q1; ++p)
+        if (S.flag[p] == 0 && S.hi[p] >= tau) {
+          c_pg[pos] = static_cast<uint16_t>(p);
+          c_lohi[pos++] = make_float2(S.lo[p], S.hi[p]);
+        }
+    __syncthreads();
+  }
+  const bool counted = k > 0 && nc <= kCandCap;
+  if (counted) {
+    // one thread per kept page; every lane reads the same bound (a broadcast)
+    for (int i = tid; i < nc; i += blockDim.x) {
+      const float2 me = c_lohi[i];
+      int n_hi = 0, n_lo = 0;   // #{hi_q >= lo_p}, #{lo_q > hi_p}
+#pragma unroll 4
+      for (int j = 0; j < nc; ++j) {
+        const float2 o = c_lohi[j];
+        n_hi += o.y >= me.x;
+        n_lo += o.x > me.y;
+      }
+      const int p = c_pg[i];
+      if (me.x >= tau && n_hi <= k) {
+        S.flag[p] = 1;
+        atomicAdd(&n_certain, 1);
+      } else if (n_lo < k) {
+        S.flag[p] = 2;
+        S.u_list[atomicAdd(&n_unc, 1)] = static_cast<uint16_t>(p);
+      }
+    }
+  } else if (k > 0) {
+    // ---- order statistics of the bounds, then: certainly in (lo > H),
+    // undecided (hi >= Lk), else out
+    float Lk = INFINITY, H = INFINITY;
+    if (!filtered_select2(S.lo, S.hi, N, k, k + 1, &scratch, Lk, H))
+      radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
+    for (int p = tid; p < N; p += blockDim.x) {
+      if (S.flag[p] != 0) continue;
+      if (S.lo[p] > H) {
+        S.flag[p] = 1;
+        atomicAdd(&n_certain, 1);
+      } else if (S.hi[p] >= Lk) {
+        S.flag[p] = 2;
+        S.u_list[atomicAdd(&n_unc, 1)] = static_cast<uint16_t>(p);
+      }
     }
   }
   __syncthreads();
@@ -393,7 +488,7 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   double* ex = reinterpret_cast<double*>(S.lo);
   if (nu_ > 0 && slots > 0) {
     // one warp per (page, query row): exact dot, then the max over the rows
-    const int nw = kThreads / 32, warp = tid >> 5, lane = tid & 31;
+    const int nw = kThreads / 32;
     const int per = max(1, kThreads / R);            // undecided pages per round
     for (int u0 = 0; u0 < nu_; u0 += per) {
       const int np = min(per, nu_ - u0);
@@ -432,22 +527,43 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   }
   __syncthreads();
 
+  if (counted) {
+    // ---- sink pages, the selected kept pages (ascending), local pages
+    if (warp == 0) {
+      for (int i = lane; i < n_sink; i += 32) outp[i] = i;
+      int pos = n_sink;
+      for (int j0 = 0; j0 < nc; j0 += 32) {
+        const int j = j0 + lane;
+        const bool sel = j < nc && S.flag[c_pg[j]] == 1;
+        const uint32_t m = __ballot_sync(0xffffffffu, sel);
+        const int q = pos + __popc(m & ((1u << lane) - 1u));
+        if (sel && q < a.budget_pages) outp[q] = c_pg[j];
+        pos += __popc(m);
+      }
+      const int n_loc = N - local0;
+      for (int i = lane; i < n_loc; i += 32)
+        if (pos + i < a.budget_pages) outp[pos + i] = local0 + i;
+      const int total = pos + n_loc;
+      for (int i = total + lane; i < a.budget_pages; i += 32) outp[i] = -1;
+      if (lane == 0) *outc = min(total, a.budget_pages);
+    }
+    return;
+  }
   // ---- ascending compaction of the selected pages
   const int per_t = (N + blockDim.x - 1) / blockDim.x;
   const int p0 = tid * per_t, p1 = min(N, p0 + per_t);
   int cnt = 0;
   for (int p = p0; p < p1; ++p) cnt += S.flag[p] == 1;
-  const int w = tid >> 5, lane = tid & 31;
   int incl = cnt;
   for (int o = 1; o < 32; o <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, o);
     if (lane >= o) incl += v;
   }
-  if (lane == 31) red_i[w] = incl;
+  if (lane == 31) red_i[warp] = incl;
   __syncthreads();
   int wbase = 0, total = 0;
   for (int i = 0; i < (int)(blockDim.x / 32); ++i) {
-    if (i < w) wbase += red_i[i];
+    if (i < warp) wbase += red_i[i];
     total += red_i[i];
   }
   int pos = wbase + incl - cnt;

@@ -191,6 +191,20 @@ def test_select_long_all_ties():
     assert list(rp[1, 0, :n_sink + k]) == list(range(n_sink + k))
 
 
+def test_select_deep_budget():
+    # 403 top-k slots over 966 candidate pages: deeper than the threshold pruning
+    # covers, so every candidate is classified by counting
+    cfg = W.scaled(W.LLAMA8B_DECODE, B=2, Hq=8, Hkv=2, seq_len_lo=16000, seq_len_hi=16000,
+                   budget_tokens=7000)
+    inp, g = gqa_case(cfg, seed=8)
+    sig = oracle_summaries(inp, cfg)
+    pages, counts = run_select(g, sig, cfg)
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]), np_i32(inp["seq_lens"]),
+                            cfg.page_size, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    np.testing.assert_array_equal(counts, rc)
+    np.testing.assert_array_equal(pages, rp)
+
+
 def test_select_workspace_contents_do_not_matter():
     # The selection workspace has no initial contents to rely on: a workspace
     # full of random bytes, reused over several calls, gives the oracle's
