@@ -12,9 +12,11 @@ built once by sa_build_page_summaries (not part of a step).
 
 The metric is selected-KV GB/s: K+V bytes of the selected pages' valid
 tokens per step divided by the step time (inputs resident in HBM, L2 flushed
-before every timed step by writing a 256 MiB buffer outside the timed
-events).  The line also carries calls/s, the decode kernel's roofline
-fraction against the measured HBM copy bandwidth, an end-to-end number
+before every timed step by writing a 256 MiB buffer and reading another
+outside the timed events).  The line also carries calls/s, the decode
+kernel's roofline fraction against the measured HBM copy bandwidth (with two
+references beside it: a library copy of the same bytes in one launch, and
+the event-timed cost of launching a one-element kernel), an end-to-end number
 through the same API with the per-step inputs (q, page table, seq_lens)
 copied from pinned host memory and the outputs (O, LSE) copied back inside
 the timed region, and the float64 oracle timed on a bounded sample on the
@@ -208,6 +210,31 @@ def _timed_graphs(g_step, g_kernel, K, flush_l2, stream, local):
     return t_step, t_kern, clk.summary()
 
 
+def _launch_floor(flush_l2, stream, n):
+    """Event-timed seconds of one graph-replayed launch of a one-element kernel, L2
+    flushed first: the fixed cost inside every kernel time measured here (launch,
+    first wave, drain, timestamp granularity)."""
+    import torch
+    x = torch.zeros(1, device=torch.device("cuda", torch.cuda.current_device()))
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        x.add_(1.0)
+    for _ in range(3):
+        g.replay()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    for i in range(n):
+        flush_l2(i)
+        ev[i][0].record(stream)
+        g.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / 1e3 / n
+
+
+LAUNCH_FLOOR_WHAT = ("event-timed graph replay of a one-element kernel, L2 flushed: the fixed "
+                     "cost inside every single-launch kernel time")
+
+
 def _peak_tflops():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -376,6 +403,7 @@ def run_extra(args, dev, world, rank, local, cores):
 
     peak, kind = _peak_tflops()
     achieved = flops / (t_kern / K) / 1e12
+    t_floor = _launch_floor(flush_l2, stream, min(K, 50))
     line = {
         "metric": METRIC, "value": round(kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -389,7 +417,9 @@ def run_extra(args, dev, world, rank, local, cores):
         "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "peak_kind": kind, "traffic": None,
-                     "kernel_ms": round(1e3 * t_kern / K, 4)},
+                     "kernel_ms": round(1e3 * t_kern / K, 4),
+                     "launch_floor_us": round(1e6 * t_floor, 2),
+                     "launch_floor_what": LAUNCH_FLOOR_WHAT},
         "e2e": {"value": round(kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(1e3 * t_e2e / K, 4)},
@@ -640,6 +670,7 @@ def main():
     t_rd = sum(a.elapsed_time(b) for a, b in rd_ev) / 1e3 / len(rd_ev)
     read_gbs = 2 * rd_buf.numel() * 4 / t_rd / 1e9
     del rd_buf, rd_out
+    t_floor = _launch_floor(flush_l2, stream, min(K, 50))
     traffic = None
     tp = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if os.path.exists(tp):
@@ -674,7 +705,10 @@ def main():
                      "same_bytes_copy": {"gbs": round(read_gbs, 1),
                                          "what": "one device copy (torch copy_) moving the same "
                                                  "bytes, read + write, L2 flushed"},
-                     "frac_of_same_bytes_copy": round(achieved / read_gbs, 4)},
+                     "frac_of_same_bytes_copy": round(achieved / read_gbs, 4),
+                     "kernel_us": round(1e6 * dec_avg, 2),
+                     "launch_floor_us": round(1e6 * t_floor, 2),
+                     "launch_floor_what": LAUNCH_FLOOR_WHAT},
         "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(1e3 * t_e2e / K, 4)},
