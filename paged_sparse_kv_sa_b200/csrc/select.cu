@@ -343,16 +343,28 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
   }
 
   extern __shared__ __align__(16) uint8_t dsm[];
-  __shared__ uint32_t hist[1024];
-  __shared__ uint32_t sel_out[8];
-  __shared__ SelScratch scratch;
+  // the kept pages' bounds and pages (counting path) or the order-statistics
+  // scratch (the other path): never both, so they share storage -- which lets
+  // two CTAs share an SM at 8192 pages
+  union ChooseScratch {
+    struct {
+      float2 lohi[kCandCap];
+      uint16_t pg[kCandCap];
+    } kept;
+    struct {
+      uint32_t hist[1024];
+      uint32_t sel_out[8];
+      SelScratch sel;
+    } stats;
+  };
+  __shared__ __align__(16) ChooseScratch cs;
   __shared__ int red_i[kThreads / 32];
   __shared__ int n_unc, n_certain;
   __shared__ double ex_tmp[kThreads];
   __shared__ __align__(16) uint32_t gmax[kSelGroups];   // order keys of the groups' largest lo
   __shared__ uint32_t tau_key;
-  __shared__ float2 c_lohi[kCandCap];                   // the kept pages' bounds, ascending
-  __shared__ uint16_t c_pg[kCandCap];
+  float2* c_lohi = cs.kept.lohi;                        // the kept pages' bounds, ascending
+  uint16_t* c_pg = cs.kept.pg;
 
   SelSmem S;
   S.lo = reinterpret_cast<float*>(dsm);
@@ -465,8 +477,8 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
     // ---- order statistics of the bounds, then: certainly in (lo > H),
     // undecided (hi >= Lk), else out
     float Lk = INFINITY, H = INFINITY;
-    if (!filtered_select2(S.lo, S.hi, N, k, k + 1, &scratch, Lk, H))
-      radix_select2(S.lo, S.hi, N, k, k + 1, hist, sel_out, Lk, H);
+    if (!filtered_select2(S.lo, S.hi, N, k, k + 1, &cs.stats.sel, Lk, H))
+      radix_select2(S.lo, S.hi, N, k, k + 1, cs.stats.hist, cs.stats.sel_out, Lk, H);
     for (int p = tid; p < N; p += blockDim.x) {
       if (S.flag[p] != 0) continue;
       if (S.lo[p] > H) {
@@ -606,6 +618,9 @@ cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
   const size_t dyn = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
   cudaError_t e = cudaFuncSetAttribute(choose_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  // the largest shared-memory carveout: two CTAs per SM up to 8192 pages
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(choose_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   return launch_pdl(choose_kernel, dim3(a.Hkv, a.B), dim3(kThreads), dyn, stream, a);
 }
