@@ -278,6 +278,58 @@ SA_API int sa_combine(const float* o_partial, const float* lse_partial, int n_sp
                int Dv, float* o_out, uint16_t* o_out_bf16, float* lse_out, void* stream);
 
 /*
+ * sa_sparse_attention — sa_sparse_decode followed by the sa_combine merge, in
+ * one call with final outputs: the decode launch writes the split partials
+ * into the workspace, then the combine launch merges them.  (A merge inside
+ * the decode kernel, by the last split of each pair to finish, was measured
+ * slower than the separate merge launch: one warp's dependent L2 round trips
+ * over the pair's partials cost more than the launch.)  Sources: as
+ * sa_sparse_decode and sa_combine (the merge step of a split Flash-decode,
+ * "TileSparse", "Configuration": mode full = fused Flash-decode).
+ *
+ *  q ... n_splits   as sa_sparse_decode
+ *  o_out      (dev, optional) [B,T,Hq,Dv] float32, 16-byte aligned
+ *  o_out_bf16 (dev, optional) [B,T,Hq,Dv] bf16, 8-byte aligned
+ *  lse_out    (dev, optional) [B,T,Hq] float32
+ *  workspace  (dev) sa_sparse_attention_workspace_size(B,T,Hq,Dv,n_splits)
+ *             bytes, 16-byte aligned, owned by the caller (the split partials;
+ *             no initial contents needed).  Calls sharing a workspace must not
+ *             overlap.
+ * At least one output must be given.  Errors: as sa_sparse_decode and
+ * sa_combine (n_splits <= 64); SA_ERR_WORKSPACE for a missing, misaligned or
+ * short workspace.
+ */
+SA_API size_t sa_sparse_attention_workspace_size(int B, int T, int Hq, int Dv, int n_splits);
+SA_API int sa_sparse_attention(const uint16_t* q, const int64_t q_strides[4],
+                               const uint16_t* k_cache, const int64_t k_strides[4],
+                               const uint16_t* v_cache, const int64_t v_strides[4],
+                               const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                               const int32_t* lists, const int32_t* list_counts, int n_lists,
+                               int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                               int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                               int n_splits, float* o_out, uint16_t* o_out_bf16, float* lse_out,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                               void* stream);
+
+/*
+ * sa_sparse_attention_fp8 — sa_sparse_decode_fp8 followed by the merge, in one
+ * call.  Arguments as sa_sparse_decode_fp8 for the inputs and as
+ * sa_sparse_attention for the outputs and the workspace (sized with Dv = D).
+ */
+SA_API int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],
+                                   const uint8_t* k_codes, const int64_t k_strides[4],
+                                   const uint8_t* v_codes, const int64_t v_strides[4],
+                                   const float* k_scale, const float* v_scale,
+                                   const int32_t* page_table, int max_pages,
+                                   const int32_t* seq_lens, const int32_t* lists,
+                                   const int32_t* list_counts, int n_lists, int max_list,
+                                   const int32_t* head_to_list, int B, int T, int Hq, int Hkv,
+                                   int D, int page_size, int P_pool, float scale, int n_splits,
+                                   float* o_out, uint16_t* o_out_bf16, float* lse_out,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                   void* stream);
+
+/*
  * sa_build_page_summaries — sigma[page_table[b,p], g, :] for every logical
  * page p < ceil(seq_lens[b]/P): the mean of the page's valid keys
  * (positions < seq_lens[b]), computed as RNE_bf16(RN64(RN64(exact sum)/n)).

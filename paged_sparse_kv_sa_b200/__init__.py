@@ -8,5 +8,6 @@ from ._lib import (EXPORTED, LIB_PATH, SAError, load, page_budget, sa_block_unio
                    sa_build_page_summaries, sa_combine, sa_select_pages,
                    sa_select_pages_no_alloc, sa_select_pages_tiered,
                    sa_select_workspace_size, sa_update_page_summaries,
-                   sa_sparse_decode, sa_sparse_decode_fp8, sa_build_page_summaries_fp8)
+                   sa_sparse_decode, sa_sparse_decode_fp8, sa_build_page_summaries_fp8,
+                   sa_sparse_attention, sa_sparse_attention_fp8, attention_workspace)
 from .pipeline import SparseDecodeStep, default_splits  # noqa: F401

@@ -40,6 +40,13 @@ _SIGNATURES = {
                                   _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P,
                                   _P, _P]),
     "sa_combine": (_I, [_P, _P, _I, _I64, _I, _P, _P, _P, _P]),
+    "sa_sparse_attention_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I]),
+    "sa_sparse_attention": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P,
+                                 _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P,
+                                 _P, ctypes.c_size_t, _P, _P]),
+    "sa_sparse_attention_fp8": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _P, _P, _I,
+                                     _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
+                                     _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
     "sa_build_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sa_update_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                       _P]),
@@ -271,6 +278,84 @@ def sa_sparse_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_
                                   _ptr(dev_error), _stream(stream))
     _check(st, "sa_sparse_decode_fp8")
     return o_partial, lse_partial
+
+
+def attention_workspace(B, T, Hq, Dv, n_splits, device):
+    """A workspace for sa_sparse_attention(_fp8): the split partials."""
+    n = int(load().sa_sparse_attention_workspace_size(B, T, Hq, Dv, n_splits))
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def _attn_outputs(B, T, Hq, Dv, device, o_out, o_out_bf16, lse_out, want_f32, want_bf16):
+    if o_out is None and want_f32:
+        o_out = torch.empty((B, T, Hq, Dv), dtype=torch.float32, device=device)
+    if o_out_bf16 is None and want_bf16:
+        o_out_bf16 = torch.empty((B, T, Hq, Dv), dtype=torch.bfloat16, device=device)
+    if lse_out is None:
+        lse_out = torch.empty((B, T, Hq), dtype=torch.float32, device=device)
+    return o_out, o_out_bf16, lse_out
+
+
+def sa_sparse_attention(q, k_cache, v_cache, page_table, seq_lens, lists, list_counts,
+                        head_to_list, scale: float, n_splits: int = 1, o_out=None,
+                        o_out_bf16=None, lse_out=None, want_f32: bool = True,
+                        want_bf16: bool = False, workspace=None, dev_error=None, stream=None):
+    """sa_sparse_decode + merge in one call.  Inputs as sa_sparse_decode; returns
+    (O [B,T,Hq,Dv] f32 or None, O bf16 or None, lse [B,T,Hq]).  `workspace`: from
+    attention_workspace (reusable); a fresh one is made when omitted."""
+    lib = load()
+    _need_cuda(q, k_cache, v_cache, page_table, seq_lens, lists, list_counts)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(page_table), _i32(seq_lens), _i32(lists)
+    _i32(list_counts)
+    B, T, Hq, Dk = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    Dv = v_cache.shape[-1]
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, Dv, q.device, o_out, o_out_bf16,
+                                               lse_out, want_f32, want_bf16)
+    if workspace is None:
+        workspace = attention_workspace(B, T, Hq, Dv, n_splits, q.device)
+    st = lib.sa_sparse_attention(_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
+                                 _ptr(v_cache), _strides4(v_cache), _ptr(page_table),
+                                 page_table.shape[1], _ptr(seq_lens), _ptr(lists),
+                                 _ptr(list_counts), n_lists, max_list,
+                                 ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, Dk, Dv, P,
+                                 P_pool, float(scale), n_splits, _ptr(o_out), _ptr(o_out_bf16),
+                                 _ptr(lse_out), _ptr(workspace), workspace.numel(),
+                                 _ptr(dev_error), _stream(stream))
+    _check(st, "sa_sparse_attention")
+    return o_out, o_out_bf16, lse_out
+
+
+def sa_sparse_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, lists,
+                            list_counts, head_to_list, scale: float, n_splits: int = 1,
+                            o_out=None, o_out_bf16=None, lse_out=None, want_f32: bool = True,
+                            want_bf16: bool = False, workspace=None, dev_error=None, stream=None):
+    """sa_sparse_decode_fp8 + merge in one call; inputs as sa_sparse_decode_fp8, outputs and
+    workspace as sa_sparse_attention."""
+    lib = load()
+    _need_cuda(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, lists, list_counts)
+    _bf16(q), _u8(k_codes), _u8(v_codes), _f32c(k_scale), _f32c(v_scale)
+    _i32(page_table), _i32(seq_lens), _i32(lists), _i32(list_counts)
+    B, T, Hq, D = q.shape
+    P_pool, Hkv, P, _ = k_codes.shape
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, D, q.device, o_out, o_out_bf16, lse_out,
+                                               want_f32, want_bf16)
+    if workspace is None:
+        workspace = attention_workspace(B, T, Hq, D, n_splits, q.device)
+    st = lib.sa_sparse_attention_fp8(_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
+                                     _ptr(v_codes), _strides4(v_codes), _ptr(k_scale),
+                                     _ptr(v_scale), _ptr(page_table), page_table.shape[1],
+                                     _ptr(seq_lens), _ptr(lists), _ptr(list_counts), n_lists,
+                                     max_list, ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, D,
+                                     P, P_pool, float(scale), n_splits, _ptr(o_out),
+                                     _ptr(o_out_bf16), _ptr(lse_out), _ptr(workspace),
+                                     workspace.numel(), _ptr(dev_error), _stream(stream))
+    _check(st, "sa_sparse_attention_fp8")
+    return o_out, o_out_bf16, lse_out
 
 
 def sa_build_page_summaries_fp8(k_codes, k_scale, page_table, seq_lens, summaries=None,

@@ -289,14 +289,33 @@ int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
   return cuda_status(launch_select_tiered(a, static_cast<cudaStream_t>(stream)));
 }
 
-int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
-                     const int64_t k_strides[4], const uint16_t* v_cache,
-                     const int64_t v_strides[4], const int32_t* page_table, int max_pages,
-                     const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
-                     int n_lists, int max_list, const int32_t* head_to_list, int B, int T, int Hq,
-                     int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
-                     int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
-                     void* stream) {
+}  // extern "C"
+
+namespace sa {
+namespace {
+// Where a merged call puts its final outputs (any of them null).
+struct MergeSpec {
+  float* o_out;
+  uint16_t* o_bf16;
+  float* lse_out;
+};
+
+int merge_outputs_ok(const MergeSpec& m) {
+  if (!m.o_out && !m.o_bf16 && !m.lse_out) return SA_ERR_INVALID_ARG;
+  if ((m.o_out && !aligned16(m.o_out)) ||
+      (m.o_bf16 && (reinterpret_cast<uintptr_t>(m.o_bf16) & 7u)))
+    return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                       const int64_t k_strides[4], const uint16_t* v_cache,
+                       const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                       const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
+                       int n_lists, int max_list, const int32_t* head_to_list, int B, int T,
+                       int Hq, int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                       int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
+                       void* stream, const MergeSpec* merge) {
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Dk <= 0 || Dv <= 0 ||
       page_size <= 0 || max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 ||
       n_splits <= 0 || !std::isfinite(scale) || !head_to_list)
@@ -332,7 +351,7 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   if (!encode_kv_map(&kmap, k_cache, Dk, page_size, Hkv, P_pool, k_strides, k_box_rows) ||
       !encode_kv_map(&vmap, v_cache, Dv, page_size, Hkv, P_pool, v_strides))
     return SA_ERR_CUDA;
-  DecodeArgs a;
+  DecodeArgs a{};
   a.q = q;
   a.qs0 = q_strides[0];
   a.qs1 = q_strides[1];
@@ -359,19 +378,27 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
   a.err = dev_error;
   a.k_scale = a.v_scale = nullptr;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (mla) return cuda_status(launch_mla(a, pairs, kmap, st));
-  return cuda_status(wide ? launch_prefill(a, pairs, kmap, vmap, st)
-                          : launch_decode_gqa(a, pairs, kmap, vmap, st));
+  if (merge && (n_splits > 64 || (int64_t)B * T * Hq * (Dv / 4) >= (int64_t(1) << 32)))
+    return SA_ERR_UNSUPPORTED;   // the combine kernel's limits
+  cudaError_t e = mla ? launch_mla(a, pairs, kmap, st)
+                      : (wide ? launch_prefill(a, pairs, kmap, vmap, st)
+                              : launch_decode_gqa(a, pairs, kmap, vmap, st));
+  if (e == cudaSuccess && merge)
+    e = launch_combine(o_partial, lse_partial, n_splits, (int64_t)B * T * Hq, Dv, merge->o_out,
+                       merge->o_bf16, merge->lse_out, st);
+  return cuda_status(e);
 }
 
-int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const uint8_t* k_codes,
-                         const int64_t k_strides[4], const uint8_t* v_codes,
-                         const int64_t v_strides[4], const float* k_scale, const float* v_scale,
-                         const int32_t* page_table, int max_pages, const int32_t* seq_lens,
-                         const int32_t* lists, const int32_t* list_counts, int n_lists,
-                         int max_list, const int32_t* head_to_list, int B, int T, int Hq, int Hkv,
-                         int D, int page_size, int P_pool, float scale, int n_splits,
-                         float* o_partial, float* lse_partial, int32_t* dev_error, void* stream) {
+int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
+                           const uint8_t* k_codes, const int64_t k_strides[4],
+                           const uint8_t* v_codes, const int64_t v_strides[4],
+                           const float* k_scale, const float* v_scale, const int32_t* page_table,
+                           int max_pages, const int32_t* seq_lens, const int32_t* lists,
+                           const int32_t* list_counts, int n_lists, int max_list,
+                           const int32_t* head_to_list, int B, int T, int Hq, int Hkv, int D,
+                           int page_size, int P_pool, float scale, int n_splits, float* o_partial,
+                           float* lse_partial, int32_t* dev_error, void* stream,
+                           const MergeSpec* merge) {
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0 ||
       max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 || n_splits <= 0 ||
       !std::isfinite(scale) || !head_to_list)
@@ -396,7 +423,7 @@ int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const ui
   if (!encode_kv_map_u8(&kmap, k_codes, D, page_size, Hkv, P_pool, k_strides) ||
       !encode_kv_map_u8(&vmap, v_codes, D, page_size, Hkv, P_pool, v_strides))
     return SA_ERR_CUDA;
-  DecodeArgs a;
+  DecodeArgs a{};
   a.q = q;
   a.qs0 = q_strides[0];
   a.qs1 = q_strides[1];
@@ -423,8 +450,117 @@ int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const ui
   a.err = dev_error;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
-  return cuda_status(
-      launch_decode_gqa_fp8(a, pairs, kmap, vmap, static_cast<cudaStream_t>(stream)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (merge && (n_splits > 64 || (int64_t)B * T * Hq * (D / 4) >= (int64_t(1) << 32)))
+    return SA_ERR_UNSUPPORTED;   // the combine kernel's limits
+  cudaError_t e = launch_decode_gqa_fp8(a, pairs, kmap, vmap, st);
+  if (e == cudaSuccess && merge)
+    e = launch_combine(o_partial, lse_partial, n_splits, (int64_t)B * T * Hq, D, merge->o_out,
+                       merge->o_bf16, merge->lse_out, st);
+  return cuda_status(e);
+}
+
+// Workspace of a merged call: the split partials.
+struct AttnWs {
+  size_t o_bytes, lse_bytes;
+};
+AttnWs attn_ws(int B, int T, int Hq, int Dv, int n_splits) {
+  auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  AttnWs w;
+  const size_t rows = (size_t)B * T * Hq;
+  w.o_bytes = r16(rows * Dv * n_splits * sizeof(float));
+  w.lse_bytes = r16(rows * n_splits * sizeof(float));
+  return w;
+}
+}  // namespace
+}  // namespace sa
+
+extern "C" {
+
+int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                     const int64_t k_strides[4], const uint16_t* v_cache,
+                     const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                     const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
+                     int n_lists, int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                     int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                     int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
+                     void* stream) {
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+                            max_pages, seq_lens, lists, list_counts, n_lists, max_list,
+                            head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
+                            n_splits, o_partial, lse_partial, dev_error, stream, nullptr);
+}
+
+int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const uint8_t* k_codes,
+                         const int64_t k_strides[4], const uint8_t* v_codes,
+                         const int64_t v_strides[4], const float* k_scale, const float* v_scale,
+                         const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                         const int32_t* lists, const int32_t* list_counts, int n_lists,
+                         int max_list, const int32_t* head_to_list, int B, int T, int Hq, int Hkv,
+                         int D, int page_size, int P_pool, float scale, int n_splits,
+                         float* o_partial, float* lse_partial, int32_t* dev_error, void* stream) {
+  return sparse_decode_fp8_impl(q, q_strides, k_codes, k_strides, v_codes, v_strides, k_scale,
+                                v_scale, page_table, max_pages, seq_lens, lists, list_counts,
+                                n_lists, max_list, head_to_list, B, T, Hq, Hkv, D, page_size,
+                                P_pool, scale, n_splits, o_partial, lse_partial, dev_error, stream,
+                                nullptr);
+}
+
+size_t sa_sparse_attention_workspace_size(int B, int T, int Hq, int Dv, int n_splits) {
+  if (B < 0 || T < 0 || Hq < 0 || Dv < 0 || n_splits < 0) return 0;
+  const AttnWs w = attn_ws(B, T, Hq, Dv, n_splits);
+  return w.o_bytes + w.lse_bytes;
+}
+
+int sa_sparse_attention(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                        const int64_t k_strides[4], const uint16_t* v_cache,
+                        const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                        const int32_t* seq_lens, const int32_t* lists, const int32_t* list_counts,
+                        int n_lists, int max_list, const int32_t* head_to_list, int B, int T,
+                        int Hq, int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                        int n_splits, float* o_out, uint16_t* o_out_bf16, float* lse_out,
+                        void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                        void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || n_lists <= 0 || Dv <= 0 || n_splits <= 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  const AttnWs w = attn_ws(B, T, Hq, Dv, n_splits);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.o_bytes + w.lse_bytes)
+    return SA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  MergeSpec m{o_out, o_out_bf16, lse_out};
+  if (int r = merge_outputs_ok(m)) return r;
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+                            max_pages, seq_lens, lists, list_counts, n_lists, max_list,
+                            head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
+                            n_splits, reinterpret_cast<float*>(ws),
+                            reinterpret_cast<float*>(ws + w.o_bytes), dev_error, stream, &m);
+}
+
+int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],
+                            const uint8_t* k_codes, const int64_t k_strides[4],
+                            const uint8_t* v_codes, const int64_t v_strides[4],
+                            const float* k_scale, const float* v_scale,
+                            const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                            const int32_t* lists, const int32_t* list_counts, int n_lists,
+                            int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                            int Hkv, int D, int page_size, int P_pool, float scale, int n_splits,
+                            float* o_out, uint16_t* o_out_bf16, float* lse_out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_error, void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || n_lists <= 0 || D <= 0 || n_splits <= 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  const AttnWs w = attn_ws(B, T, Hq, D, n_splits);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.o_bytes + w.lse_bytes)
+    return SA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  MergeSpec m{o_out, o_out_bf16, lse_out};
+  if (int r = merge_outputs_ok(m)) return r;
+  return sparse_decode_fp8_impl(q, q_strides, k_codes, k_strides, v_codes, v_strides, k_scale,
+                                v_scale, page_table, max_pages, seq_lens, lists, list_counts,
+                                n_lists, max_list, head_to_list, B, T, Hq, Hkv, D, page_size,
+                                P_pool, scale, n_splits, reinterpret_cast<float*>(ws),
+                                reinterpret_cast<float*>(ws + w.o_bytes), dev_error, stream, &m);
 }
 
 int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,

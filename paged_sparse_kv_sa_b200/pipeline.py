@@ -1,5 +1,6 @@
-"""One sparse-attention decode step (select -> decode -> combine) over
-preallocated buffers, so that a timed or graph-captured step allocates nothing.
+"""One sparse-attention decode step (select -> decode -> combine; or select ->
+attend, which is decode + combine in one call) over preallocated buffers, so
+that a timed or graph-captured step allocates nothing.
 
 Every stage is a call through the C ABI; this module only sizes buffers and
 chooses the split count.
@@ -65,6 +66,8 @@ class SparseDecodeStep:
         self.dev_error = torch.zeros((1,), dtype=torch.int32, device=dev)
         self.sel_ws = torch.empty(max(_lib.sa_select_workspace_size(B, Hkv, max_pages), 16),
                                   dtype=torch.uint8, device=dev)
+        # the split partials of sa_sparse_attention
+        self.attn_ws = _lib.attention_workspace(B, T, Hq, D, self.n_splits, dev)
 
     def select(self, q, summaries, page_table, seq_lens, stream=None):
         _lib.sa_select_pages(q, summaries, page_table, seq_lens, self.P, self.sink, self.local,
@@ -85,12 +88,27 @@ class SparseDecodeStep:
                                   self.n_splits, o_partial=self.o_part, lse_partial=self.lse_part,
                                   dev_error=self.dev_error, stream=stream)
 
+    def attend(self, q, k_cache, v_cache, page_table, seq_lens, stream=None):
+        """decode + combine in one call (sa_sparse_attention) into self.o / self.lse."""
+        _lib.sa_sparse_attention(q, k_cache, v_cache, page_table, seq_lens, self.pages,
+                                 self.counts, self.head_to_list, self.scale, self.n_splits,
+                                 o_out=self.o, o_out_bf16=self.o_bf16, lse_out=self.lse,
+                                 workspace=self.attn_ws, dev_error=self.dev_error, stream=stream)
+
+    def attend_fp8(self, q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens,
+                   stream=None):
+        """attend over FP8 E4M3 pages (sa_sparse_attention_fp8)."""
+        _lib.sa_sparse_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens,
+                                     self.pages, self.counts, self.head_to_list, self.scale,
+                                     self.n_splits, o_out=self.o, o_out_bf16=self.o_bf16,
+                                     lse_out=self.lse, workspace=self.attn_ws,
+                                     dev_error=self.dev_error, stream=stream)
+
     def combine(self, stream=None):
         _lib.sa_combine(self.o_part, self.lse_part, o_out=self.o, o_out_bf16=self.o_bf16,
                         lse_out=self.lse, stream=stream)
 
     def __call__(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
         self.select(q, summaries, page_table, seq_lens, stream)
-        self.decode(q, k_cache, v_cache, page_table, seq_lens, stream)
-        self.combine(stream)
+        self.attend(q, k_cache, v_cache, page_table, seq_lens, stream)
         return self.o, self.lse
