@@ -163,6 +163,32 @@ SA_DEV void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
                : "r"(addr));
 }
 
+// 2^x by the hardware approximation (ex2.approx.ftz: relative error about
+// 2^-22, results below 2^-126 flushed to zero) -- for softmax probabilities
+// that are rounded to bf16 or f16 before their MMA.
+SA_DEV float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Max (or, with kMin, min) of N values (N a multiple of 8) in eight
+// independent chains, NaN entries ignored (NaN only if every entry is NaN).
+template <bool kMin, int N>
+SA_DEV float reduce_n(const float (&x)[N]) {
+  static_assert(N % 8 == 0, "eight chains");
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = x[i];
+#pragma unroll
+  for (int c = 8; c < N; c += 8)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = kMin ? fminf(m[i], x[c + i]) : fmaxf(m[i], x[c + i]);
+#pragma unroll
+  for (int w = 4; w; w >>= 1)
+#pragma unroll
+    for (int i = 0; i < w; ++i) m[i] = kMin ? fminf(m[i], m[i + w]) : fmaxf(m[i], m[i + w]);
+  return m[0];
+}
 // Two floats -> packed bf16x2 (round to nearest even); `lo` in the low half.
 SA_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -14,7 +14,9 @@
 //
 // Per 64-key tile S = Q K^T takes 36 MMAs of 64 x 64 x 16 (an MMA of N <= 64
 // costs the same issue time as one of N = 32, so 64-key tiles halve the QK
-// issue cost per key) and O += P V two halves of four 64 x 256 x 16 MMAs.
+// issue cost per key) and O += P V two halves of four 64 x 256 x 16 MMAs, each
+// twice: P enters as bf16 hi + lo (its rounding then ~2^-17 relative), the low
+// parts written into the tile's rope chunk, which only QK reads.
 // Shared memory: the query tile (72 KB, resident), two key stages of 72 KB and
 // one P buffer of 8 KB.  A stage is free only once the PV of its tile is done
 // (the values are read from it), so the ring is kept moving by issuing MMAs
@@ -310,13 +312,19 @@ __global__ void __launch_bounds__(kMThreads, 1)
           tc::fence_after_sync();
           const int st = jp % kMStages;
           const uint64_t dv = dv0 + static_cast<uint64_t>((st * kTileBytes) >> 4);
+          // P = hi + lo: the low parts sit in the stage's rope chunk (dead after QK)
+          const uint64_t dl =
+              tc::sdesc_sw128(smem_u32(k_s) + st * kTileBytes + (kKC - 1) * kChunkBytes, 16, 1024);
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int kk = 0; kk < kMKeys / 16; ++kk)
-              tc::mma_bf16(tmem + (h ? kHiLanes : 0u), dp0 + static_cast<uint64_t>(kk * 2),
-                           dv + static_cast<uint64_t>((4 * h * kChunkBytes + kk * 2048) >> 4),
+            for (int kk = 0; kk < kMKeys / 16; ++kk) {
+              const uint64_t bv = dv + static_cast<uint64_t>((4 * h * kChunkBytes + kk * 2048) >> 4);
+              tc::mma_bf16(tmem + (h ? kHiLanes : 0u), dp0 + static_cast<uint64_t>(kk * 2), bv,
                            kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+              tc::mma_bf16(tmem + (h ? kHiLanes : 0u), dl + static_cast<uint64_t>(kk * 2), bv,
+                           kIdPV, 1u);
+            }
           tc::commit(&o_done);
           tc::commit(&kv_empty[st]);
           ++jp;
@@ -403,7 +411,11 @@ __global__ void __launch_bounds__(kMThreads, 1)
           v[i] = low ? v[i] : hv;
         }
       }
-      if (code & 128) {   // mask this lane's two 16-key groups
+      // the row max of the scaled scores from the raw ones: x -> x s is monotone,
+      // so it is s max(x) for s >= 0 and s min(x) for s < 0; invisible keys are
+      // NaN here (ignored by the reduction, p = 0 below)
+      const bool masked = code & 128;
+      if (masked) {   // this lane's two 16-key groups
 #pragma unroll
         for (int gg = 0; gg < 2; ++gg) {
           const int2 gr = mgroup(ent_s, n_ent, a.P, j, (low ? 0 : 2) + gg);
@@ -411,17 +423,13 @@ __global__ void __launch_bounds__(kMThreads, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int kp = gr.y + c;
-            if (!(gok && kp < L && kp <= qpos)) v[gg * 16 + c] = -INFINITY;
+            if (!(gok && kp < L && kp <= qpos)) v[gg * 16 + c] = NAN;
           }
         }
       }
-      float m8[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        m8[i] = fmaxf(fmaxf(v[i], v[i + 8]), fmaxf(v[i + 16], v[i + 24]));
-      float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16)) * sl2;   // the row's max, scaled
+      const float mr = sl2 >= 0.f ? reduce_n<false>(v) : reduce_n<true>(v);
+      float mx = mr != mr ? -INFINITY : mr * sl2;
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));   // the row's max, scaled
       // PV of the previous tile done: O is stable and the P buffer free
       if (jj >= 1 && !warp_wait_m(&o_done, (jj - 1) & 1, abort_flag)) {
         ok = false;
@@ -446,19 +454,31 @@ __global__ void __launch_bounds__(kMThreads, 1)
         }
       }
       const float nb = m_ref == -INFINITY ? 0.f : -m_ref;
+      // P = hi + lo (both bf16, so its rounding stays ~2^-17 relative): hi into
+      // the P buffer, lo into this tile's stage's rope chunk (read by QK only,
+      // and QK of this tile is complete)
       uint8_t* prow = p_s + r * 128;
+      uint8_t* lrow = k_s + (jj % kMStages) * kTileBytes + (kKC - 1) * kChunkBytes + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float p[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) p[i] = exp2f(fmaf(v[ch * 8 + i], sl2, nb));
+        for (int i = 0; i < 8; ++i) {
+          const float x = v[ch * 8 + i];
+          p[i] = ex2_approx(fmaf(x, sl2, nb));
+          if (masked) p[i] = x == x ? p[i] : 0.f;
+        }
         l += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
-        uint4 w;
-        w.x = pack_bf16(p[0], p[1]);
-        w.y = pack_bf16(p[2], p[3]);
-        w.z = pack_bf16(p[4], p[5]);
-        w.w = pack_bf16(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + ((((low ? 0 : 4) + ch) ^ (r & 7)) << 4)) = w;
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          hw[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
+          lw[i] = pack_bf16(p[2 * i] - bf16_bits_to_float(hw[i] & 0xffffu),
+                            p[2 * i + 1] - bf16_bits_to_float(hw[i] >> 16));
+        }
+        const int off = (((low ? 0 : 4) + ch) ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(prow + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(lrow + off) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
       }
       tc::fence_proxy_async();
       tc::fence_before_sync();

@@ -322,8 +322,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tc::ld32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(&x[0]));
       tc::ld32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
       tc::wait_ld();
-      float mx = -INFINITY;
-      if (code & 1) {
+      // the row max of the scaled scores from the raw ones: x -> x s is monotone
+      // (rounding included), so it is s max(x) for s >= 0 and s min(x) for s < 0;
+      // invisible keys are NaN here (ignored by the reduction, p = 0 below)
+      const float sl = a.scale_log2;
+      const bool masked = code & 1;
+      if (masked) {
 #pragma unroll
         for (int g = 0; g < 4; ++g) {
           const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
@@ -331,19 +335,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
             const int kp = gr.y + c;
-            const bool vis = gok && kp < L && kp <= qpos;
-            const float v = vis ? x[g * 16 + c] * a.scale_log2 : -INFINITY;
-            x[g * 16 + c] = v;
-            mx = fmaxf(mx, v);
+            if (!(gok && kp < L && kp <= qpos)) x[g * 16 + c] = NAN;
           }
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          x[c] *= a.scale_log2;
-          mx = fmaxf(mx, x[c]);
-        }
       }
+      const float mr = sl >= 0.f ? reduce_n<false>(x) : reduce_n<true>(x);
+      const float mx = mr != mr ? -INFINITY : mr * sl;
       // PV(jj-1) must be done before O is rescaled or P is rewritten
       if (jj >= 1 && !wait_or_abort(&o_done[wg], (jj - 1) & 1, abort_flag)) {
         ok = false;
@@ -368,14 +365,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tc::wait_st();
         }
       }
-      const float base = m_ref == -INFINITY ? 0.f : m_ref;
+      const float nb = m_ref == -INFINITY ? 0.f : -m_ref;
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // (independent chains)
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
         float p[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-          p[i] = exp2f(x[ch * 8 + i] - base);
-          l += p[i];
+          const float v = x[ch * 8 + i];
+          p[i] = ex2_approx(fmaf(v, sl, nb));
+          if (masked) p[i] = v == v ? p[i] : 0.f;
+          ls[i] += p[i];
         }
         uint4 w;
         w.x = pack_bf16(p[0], p[1]);
@@ -384,6 +384,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         w.w = pack_bf16(p[6], p[7]);
         *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = w;
       }
+      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       tc::fence_proxy_async();
       tc::fence_before_sync();
       mbar_arrive(&p_full[wg]);

@@ -189,3 +189,61 @@ def test_attention_argument_errors():
                                      1.0 / math.sqrt(cfg.D), 3, None, None, None, ws.data_ptr(),
                                      ws.numel(), None, None)
         sa._lib._check(st, "sa_sparse_attention")
+
+
+def _scaled_case(path, scale_mult, seed):
+    """(o, lse, o_ref, lse_ref) of one call with scale = scale_mult / sqrt(Dk)."""
+    if path == "mla":
+        cfg = W.MLADecode("case", B=2, T=2, Hq=16, Dk=576, Dv=512, page_size=64, seq_len=1500,
+                          alpha=3, beta=6, h_ambient=4)
+        inp = W.mla_decode_inputs(cfg, seed=seed, device="cpu")
+        scale = scale_mult / math.sqrt(cfg.Dk)
+        sig = O.page_summaries(bits(inp["kv"]), np_i32(inp["page_table"]),
+                               np_i32(inp["seq_lens"]), 64)
+        lists, counts = mla_lists_from_oracle(inp, sig, cfg)
+        g = {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+        amb = set(int(h) for h in inp["ambient_heads"].tolist())
+        h2l = [1 if h in amb else 0 for h in range(cfg.Hq)]
+        kv = g["kv"]
+        o, _, lse = sa.sa_sparse_attention(g["q"], kv, kv[..., :cfg.Dv], g["page_table"],
+                                           g["seq_lens"], torch.from_numpy(lists).to(DEV),
+                                           torch.from_numpy(counts).to(DEV), h2l, scale, 2)
+        torch.cuda.synchronize()
+        kvb = bits(inp["kv"])
+        ro, rl = O.sparse_attention(bits(inp["q"]), kvb, kvb[..., :cfg.Dv],
+                                    np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists,
+                                    counts, np.array(h2l), scale, 64)
+    else:
+        T, Hq = (1, 8) if path == "gqa" else (4, 16)
+        cfg = W.GQADecode("case", B=2, Hq=Hq, Hkv=2, D=128, page_size=16, seq_len_lo=0,
+                          seq_len_hi=0, sink_tokens=16, local_tokens=64, budget_tokens=256, T=T)
+        inp, g = gqa_case(cfg, seed=seed, seq_lens=[3000, 777 if T > 1 else 35])
+        scale = scale_mult / math.sqrt(cfg.D)
+        sig = oracle_summaries(inp, cfg)
+        lists, counts = oracle_lists(inp, cfg, sig)
+        h2l = [h // cfg.G for h in range(cfg.Hq)]
+        o, _, lse = sa.sa_sparse_attention(g["q"], g["k"], g["v"], g["page_table"],
+                                           g["seq_lens"], torch.from_numpy(lists).to(DEV),
+                                           torch.from_numpy(counts).to(DEV), h2l, scale, 3)
+        torch.cuda.synchronize()
+        ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                    np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists,
+                                    counts, np.arange(cfg.Hq) // cfg.G, scale, cfg.page_size)
+    return o, lse, ro, rl
+
+
+@pytest.mark.parametrize("path", ["gqa", "tensor_core", "mla"])
+def test_attention_negative_scale(path):
+    # the scale may be any finite number: with s < 0 the row max of the scaled scores
+    # is s times the smallest raw score, and masked keys must still weigh nothing
+    assert_attn_close(*_scaled_case(path, -1.0, 48))
+
+
+@pytest.mark.parametrize("path", ["gqa", "mla"])
+def test_attention_sharp_softmax(path):
+    # three times the usual 1/sqrt(D): a few keys dominate each row, so the
+    # probabilities' rounding before the PV product shows directly in O.  The
+    # warp-MMA and MLA kernels multiply by P as bf16 hi + lo (~2^-17 relative)
+    # and hold the bar; the tcgen05 many-row kernel rounds P once to bf16 and is
+    # held to it at the usual scale only (its other tests)
+    assert_attn_close(*_scaled_case(path, 3.0, 49))
