@@ -266,68 +266,6 @@ __global__ void __launch_bounds__(kSThreads, 1) tiered_score_kernel(const Tiered
   }
 }
 
-// Block-wide ascending compaction of the pages whose flag has bit 1 (into
-// out0) and bit 2 (into out1), each padded with -1 to cap; one pass, one scan.
-SA_DEV void compact_pages2(const uint8_t* flag, int N, int32_t* out0, int32_t* out1, int cap,
-                           int* red_i, int& c0, int& c1) {
-  const int tid = threadIdx.x, nw = blockDim.x / 32;
-  const int per_t = (N + blockDim.x - 1) / blockDim.x;
-  const int p0 = tid * per_t, p1 = min(N, p0 + per_t);
-  int cnt = 0;   // low 16 bits: bit 1 pages, high 16 bits: bit 2 pages
-  for (int p = p0; p < p1; ++p) cnt += (flag[p] & 1u) + ((flag[p] & 2u) << 15);
-  const int w = tid >> 5, lane = tid & 31;
-  int incl = cnt;
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) red_i[w] = incl;
-  __syncthreads();
-  int wbase = 0, total = 0;
-  for (int i = 0; i < nw; ++i) {
-    if (i < w) wbase += red_i[i];
-    total += red_i[i];
-  }
-  int pos0 = (wbase + incl - cnt) & 0xffff, pos1 = (wbase + incl - cnt) >> 16;
-  for (int p = p0; p < p1; ++p) {
-    if ((flag[p] & 1u) && pos0 < cap) out0[pos0++] = p;
-    if ((flag[p] & 2u) && pos1 < cap) out1[pos1++] = p;
-  }
-  c0 = min(total & 0xffff, cap);
-  c1 = min(total >> 16, cap);
-  for (int i = c0 + tid; i < cap; i += blockDim.x) out0[i] = -1;
-  for (int i = c1 + tid; i < cap; i += blockDim.x) out1[i] = -1;
-  __syncthreads();   // red_i is reused by the caller
-}
-
-// Block-wide ascending list (in shared memory) of the pages whose flag has any
-// of `bits` set; returns its length.
-SA_DEV int compact_flag_list(const uint8_t* flag, int N, uint8_t bits, uint16_t* list, int* red_i) {
-  const int tid = threadIdx.x;
-  const int per_t = (N + blockDim.x - 1) / blockDim.x;
-  const int p0 = tid * per_t, p1 = min(N, p0 + per_t);
-  int cnt = 0;
-  for (int p = p0; p < p1; ++p) cnt += (flag[p] & bits) != 0;
-  const int w = tid >> 5, lane = tid & 31;
-  int incl = cnt;
-  for (int o = 1; o < 32; o <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += v;
-  }
-  if (lane == 31) red_i[w] = incl;
-  __syncthreads();
-  int wbase = 0, total = 0;
-  for (int i = 0; i < (int)(blockDim.x / 32); ++i) {
-    if (i < w) wbase += red_i[i];
-    total += red_i[i];
-  }
-  int pos = wbase + incl - cnt;
-  for (int p = p0; p < p1; ++p)
-    if (flag[p] & bits) list[pos++] = static_cast<uint16_t>(p);
-  __syncthreads();   // red_i is reused; the list is complete
-  return total;
-}
-
 // Out of line: the exact dot needs many registers, and inlined it would raise
 // the register count (and spills) of the whole choose kernel.
 __device__ __noinline__ double exact_row_dot(const uint16_t* q, const uint16_t* sg, int n) {

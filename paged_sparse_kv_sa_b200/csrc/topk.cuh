@@ -63,197 +63,6 @@ SA_DEV float2 warp_score_bracket(const uint16_t* q, const uint16_t* sg, int n) {
   return make_float2(__fsub_rd(s, E) + 0.f, __fadd_ru(s, E) + 0.f);
 }
 
-// Workspace of bucket_select (shared memory).
-constexpr int kBkBins = 1024;   // buckets per array; bucket 0 holds -inf
-constexpr int kBkCap = 256;     // entries kept from one boundary bucket
-constexpr int kBkPairs = 2;     // (k_lo, k_hi) pairs answered by one call
-struct BucketScratch {
-  uint32_t hist[2][kBkBins];
-  float cand[2 * kBkPairs][kBkCap];
-  uint32_t mxk[2], mnk[2];      // order-preserving keys of the finite max / min
-  int wtot[2][32];              // per-warp totals of the bucket scan
-  int bucket[2 * kBkPairs], above[2 * kBkPairs], ccnt[2 * kBkPairs];
-  float res[2 * kBkPairs];
-};
-
-// Bucket of v: -inf -> 0, finite v -> 1 + floor((v - mn) * inv) (capped).  Each
-// step is monotone non-decreasing in v (a rounded subtraction of a fixed mn, a
-// rounded product with a fixed inv >= 0, truncation, min), so v <= w implies
-// bucket(v) <= bucket(w), and equal values share a bucket.
-SA_DEV int bk_bucket(float v, float mn, float inv) {
-  if (v == -INFINITY) return 0;
-  return 1 + min(static_cast<int>((v - mn) * inv), kBkBins - 2);
-}
-
-// For each pair j < npairs: out_lo[j] = the (k_lo[j])-th largest of lo[0, n)
-// and out_hi[j] = the (k_hi[j])-th largest of hi[0, n) (1-based ranks, NaN
-// entries never count, -inf when fewer than k entries count; k >= 1).  One
-// pass: the entries are histogrammed into kBkBins monotone buckets over the
-// finite range of each array, a block scan from the top finds the bucket that
-// holds the k-th entry and how many entries lie in higher buckets, and the
-// answer is ranked among that bucket's entries only (counting entries greater
-// than and equal to each).  Returns false (results unset) when the finite
-// range overflows or a boundary bucket holds more than kBkCap entries; the
-// caller then falls back to radix_select2.  Called by every thread of the block.
-SA_DEV bool bucket_select(const float* lo, const float* hi, int n, int npairs, const int* k_lo,
-                          const int* k_hi, BucketScratch* sc, float* out_lo, float* out_hi) {
-  const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
-  const int nq = 2 * npairs;   // request q: array q & 1 (0 = lo, 1 = hi), pair q >> 1
-  for (int i = tid; i < 2 * kBkBins; i += nt) (&sc->hist[0][0])[i] = 0u;
-  if (tid < 2) {
-    sc->mxk[tid] = 0u;            // below every non-NaN key
-    sc->mnk[tid] = 0xffffffffu;
-  }
-  if (tid < nq) {
-    sc->bucket[tid] = -1;
-    sc->above[tid] = 0;
-    sc->ccnt[tid] = 0;
-    sc->res[tid] = -INFINITY;
-  }
-  float mx[2] = {-INFINITY, -INFINITY}, mn[2] = {INFINITY, INFINITY};
-  for (int i = tid; i < n; i += nt) {
-    const float v[2] = {lo[i], hi[i]};
-#pragma unroll
-    for (int w = 0; w < 2; ++w)
-      if (isfinite(v[w])) {
-        mx[w] = fmaxf(mx[w], v[w]);
-        mn[w] = fminf(mn[w], v[w]);
-      }
-  }
-#pragma unroll
-  for (int w = 0; w < 2; ++w)
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      mx[w] = fmaxf(mx[w], __shfl_xor_sync(0xffffffffu, mx[w], o));
-      mn[w] = fminf(mn[w], __shfl_xor_sync(0xffffffffu, mn[w], o));
-    }
-  __syncthreads();   // scratch initialised
-  if (lane == 0)
-#pragma unroll
-    for (int w = 0; w < 2; ++w)
-      if (mx[w] >= mn[w]) {
-        atomicMax(&sc->mxk[w], f2key(mx[w]));
-        atomicMin(&sc->mnk[w], f2key(mn[w]));
-      }
-  __syncthreads();
-  float base[2], inv[2];
-  bool ok = true;
-#pragma unroll
-  for (int w = 0; w < 2; ++w) {
-    base[w] = 0.f;
-    inv[w] = 0.f;
-    if (sc->mxk[w] != 0u) {     // some finite entry
-      const float M = key2f(sc->mxk[w]), m = key2f(sc->mnk[w]);
-      const float range = M - m;
-      base[w] = m;
-      if (!(range < INFINITY)) ok = false;
-      else if (range > 0.f) inv[w] = static_cast<float>(kBkBins - 2) / range;
-      if (!(inv[w] < INFINITY)) ok = false;
-    }
-  }
-  if (!ok) {
-    __syncthreads();
-    return false;
-  }
-  for (int i = tid; i < n; i += nt) {
-    const float v[2] = {lo[i], hi[i]};
-#pragma unroll
-    for (int w = 0; w < 2; ++w)
-      if (!isnan(v[w])) atomicAdd(&sc->hist[w][bk_bucket(v[w], base[w], inv[w])], 1u);
-  }
-  __syncthreads();
-  // thread t holds buckets kBkBins-1 - (t*bpt + j), j < bpt: the scan runs from the top
-  const int bpt = (kBkBins + nt - 1) / nt;
-  int cnt[2] = {0, 0};
-  for (int j = 0; j < bpt; ++j) {
-    const int bin = kBkBins - 1 - (tid * bpt + j);
-    if (bin >= 0) {
-      cnt[0] += sc->hist[0][bin];
-      cnt[1] += sc->hist[1][bin];
-    }
-  }
-  int incl[2] = {cnt[0], cnt[1]};
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1)
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      const int v = __shfl_up_sync(0xffffffffu, incl[w], o);
-      if (lane >= o) incl[w] += v;
-    }
-  if (lane == 31) {
-    sc->wtot[0][warp] = incl[0];
-    sc->wtot[1][warp] = incl[1];
-  }
-  __syncthreads();
-  for (int q = 0; q < nq; ++q) {
-    const int w = q & 1, k = w ? k_hi[q >> 1] : k_lo[q >> 1];
-    int run = incl[w] - cnt[w];
-    for (int i = 0; i < warp; ++i) run += sc->wtot[w][i];
-    if (run < k && run + cnt[w] >= k)
-      for (int j = 0; j < bpt; ++j) {
-        const int bin = kBkBins - 1 - (tid * bpt + j);
-        const int c = sc->hist[w][bin];
-        if (run + c >= k) {
-          sc->bucket[q] = bin;
-          sc->above[q] = run;
-          break;
-        }
-        run += c;
-      }
-  }
-  __syncthreads();
-  int bq[2 * kBkPairs];
-#pragma unroll
-  for (int q = 0; q < 2 * kBkPairs; ++q) bq[q] = q < nq ? sc->bucket[q] : -1;
-  // bucket 0 holds only -inf: that answer needs no ranking (res stays -inf)
-  for (int i = tid; i < n; i += nt) {
-    const float v[2] = {lo[i], hi[i]};
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      if (isnan(v[w])) continue;
-      const int bb = bk_bucket(v[w], base[w], inv[w]);
-#pragma unroll
-      for (int q = w; q < 2 * kBkPairs; q += 2)
-        if (bb > 0 && bb == bq[q]) {
-          const int slot = atomicAdd(&sc->ccnt[q], 1);
-          if (slot < kBkCap) sc->cand[q][slot] = v[w];
-        }
-    }
-  }
-  __syncthreads();
-  int total = 0;
-  for (int q = 0; q < nq; ++q) {
-    const int c = sc->ccnt[q];
-    if (c > kBkCap) ok = false;
-    total += c;
-  }
-  if (!ok) {
-    __syncthreads();
-    return false;
-  }
-  for (int x = tid; x < total; x += nt) {
-    int q = 0, xi = x;
-    while (xi >= sc->ccnt[q]) xi -= sc->ccnt[q++];
-    const int w = q & 1, k = (w ? k_hi[q >> 1] : k_lo[q >> 1]) - sc->above[q];
-    const float* arr = sc->cand[q];
-    const int cn = sc->ccnt[q];
-    const float v = arr[xi];
-    int g = 0, e = 0;
-    for (int y = 0; y < cn; ++y) {
-      g += arr[y] > v;
-      e += arr[y] == v;
-    }
-    if (g < k && g + e >= k) sc->res[q] = v;
-  }
-  __syncthreads();
-  for (int j = 0; j < npairs; ++j) {
-    out_lo[j] = sc->res[2 * j];
-    out_hi[j] = sc->res[2 * j + 1];
-  }
-  __syncthreads();   // the scratch may be reused by the caller
-  return true;
-}
-
 // Workspace of filtered_select2 (shared memory).
 constexpr int kSelGroupsMax = 512;   // n <= 32 * kSelGroupsMax
 constexpr int kSelCap = 1024;        // candidates kept per sequence
