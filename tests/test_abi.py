@@ -97,3 +97,34 @@ def test_calls_fail_loudly_without_gpu_tensors():
         sa.sa_select_pages(q, torch.zeros((4, 2, 64), dtype=torch.bfloat16),
                            torch.zeros((1, 4), dtype=torch.int32),
                            torch.zeros((1,), dtype=torch.int32), 16, 16, 16, 64)
+
+
+def test_attention_workspace_size_and_host_checks():
+    lib = sa.load()
+    # the split partials: [n_splits, rows, Dv] float32 then [n_splits, rows] float32,
+    # each rounded up to 16 bytes
+    rows, dv, ns = 2 * 1 * 8, 128, 3
+    r16 = lambda x: (x + 15) // 16 * 16
+    assert lib.sa_sparse_attention_workspace_size(2, 1, 8, dv, ns) == \
+        r16(rows * dv * ns * 4) + r16(rows * ns * 4)
+    assert lib.sa_sparse_attention_workspace_size(3, 2, 5, 64, 1) == r16(30 * 64 * 4) + r16(30 * 4)
+    fake = ctypes.c_void_p(0x1000)
+    s = _i64x4(1024, 1024, 128, 1)
+    ks = _i64x4(4096, 2048, 128, 1)
+    h2l = (ctypes.c_int32 * 8)(0, 0, 0, 0, 1, 1, 1, 1)
+    need = lib.sa_sparse_attention_workspace_size(1, 1, 8, 128, 2)
+
+    def call(o_out, ws, ws_bytes):
+        return lib.sa_sparse_attention(fake, s, fake, ks, fake, ks, fake, 8, fake, fake, fake, 2,
+                                       16, ctypes.cast(h2l, ctypes.c_void_p), 1, 1, 8, 2, 128,
+                                       128, 16, 64, 0.1, 2, o_out, None, None, ws, ws_bytes, None,
+                                       None)
+    assert call(fake, None, need) == 3                        # no workspace
+    assert call(fake, fake, need - 16) == 3                   # too small
+    assert call(fake, ctypes.c_void_p(0x1008), need) == 3     # not 16-byte aligned
+    assert call(None, fake, need) == 1                        # no output at all
+    assert call(ctypes.c_void_p(0x1004), fake, need) == 1     # float32 output misaligned
+    assert lib.sa_sparse_attention_fp8(fake, s, fake, ks, fake, ks, fake, fake, fake, 8, fake,
+                                       fake, fake, 2, 16, ctypes.cast(h2l, ctypes.c_void_p), 1, 1,
+                                       8, 2, 128, 16, 64, 0.1, 2, fake, None, None, None, need,
+                                       None, None) == 3
