@@ -19,8 +19,8 @@ references beside it: a library copy of the same bytes in one launch, and
 the event-timed cost of launching a one-element kernel), an end-to-end number
 through the same API with the per-step inputs (q, page table, seq_lens)
 copied from pinned host memory and the outputs (O, LSE) copied back inside
-the timed region, and the float64 oracle timed on a bounded sample on the
-host cores.
+the timed region (each side packed into one buffer: one copy each way), and
+the float64 oracle timed on a bounded sample on the host cores.
 
 With --gpus N (torchrun), every rank runs its own batch of the same shape
 (replicas: the path has no exchange step); time is the max over ranks.
@@ -210,6 +210,23 @@ def _timed_graphs(g_step, g_kernel, K, flush_l2, stream, local):
     return t_step, t_kern, clk.summary()
 
 
+def _packed(like, device):
+    """One contiguous byte buffer holding tensors shaped like `like` back to back
+    (16-byte aligned offsets; pinned when on the host), and a view of each: a
+    step's inputs, or its outputs, then cross PCIe in one copy."""
+    import torch
+    offs, n = [], 0
+    for t in like:
+        n = (n + 15) // 16 * 16
+        offs.append(n)
+        n += t.numel() * t.element_size()
+    host = torch.device(device).type == "cpu"
+    buf = torch.empty(max(n, 16), dtype=torch.uint8, device=device, pin_memory=host)
+    views = [buf[o:o + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+             for o, t in zip(offs, like)]
+    return buf, views
+
+
 def _launch_floor(flush_l2, stream, n):
     """Event-timed seconds of one graph-replayed launch of a one-element kernel, L2
     flushed first: the fixed cost inside every kernel time measured here (launch,
@@ -373,18 +390,19 @@ def run_extra(args, dev, world, rank, local, cores):
     t_step, t_kern, clocks = _timed_graphs(g_step, g_kern, K, flush_l2, stream, local)
 
     # end to end through the same API: the step's inputs from pinned host memory
+    # (packed: one host-to-device copy) and its outputs back (packed: one copy)
     srcs = (first, pt, sl) if first is q else (first, pt, sl, q)
-    hosts = [torch.empty(x.shape, dtype=x.dtype, pin_memory=True).copy_(x.cpu()) for x in srcs]
-    devs = [torch.empty_like(x) for x in srcs]
-    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-    lse_h = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    h_in, hosts = _packed(srcs, "cpu")
+    for h_, x in zip(hosts, srcs):
+        h_.copy_(x.cpu())
+    d_in, devs = _packed(srcs, dev)
+    d_out, (o, lse) = _packed((o, lse), dev)      # the step now writes these views
+    h_out, (o_h, lse_h) = _packed((o, lse), "cpu")
 
     def e2e():
-        for d_, h_ in zip(devs, hosts):
-            d_.copy_(h_, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
         run_step(devs[0], devs[1], devs[2], devs[-1] if len(devs) == 4 else devs[0])
-        o_h.copy_(o, non_blocking=True)
-        lse_h.copy_(lse, non_blocking=True)
+        h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(3):
         e2e()
@@ -397,8 +415,8 @@ def run_extra(args, dev, world, rank, local, cores):
         e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     t_e2e = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
-    h2d = sum(h.numel() * h.element_size() for h in hosts)
-    d2h = o_h.numel() * 4 + lse_h.numel() * 4
+    h2d = h_in.numel()
+    d2h = h_out.numel()
     assert torch.isfinite(o).all().item(), "non-finite output"
 
     peak, kind = _peak_tflops()
@@ -603,22 +621,22 @@ def main():
     calls_per_sec = world * K / t_step_max
 
     # ---- end to end through the same API: host inputs in, host outputs out
-    q_h = torch.empty(q.shape, dtype=q.dtype, pin_memory=True).copy_(q.cpu())
-    pt_h = torch.empty(pt.shape, dtype=pt.dtype, pin_memory=True).copy_(pt.cpu())
-    sl_h = torch.empty(sl.shape, dtype=sl.dtype, pin_memory=True).copy_(sl.cpu())
-    o_h = torch.empty(step.o.shape, dtype=torch.float32, pin_memory=True)
-    lse_h = torch.empty(step.lse.shape, dtype=torch.float32, pin_memory=True)
-    q_d, pt_d, sl_d = torch.empty_like(q), torch.empty_like(pt), torch.empty_like(sl)
+    # inputs packed in one pinned buffer (one host-to-device copy), outputs in one
+    # device buffer the step writes (one device-to-host copy)
+    h_in, (q_h, pt_h, sl_h) = _packed((q, pt, sl), "cpu")
+    q_h.copy_(q.cpu())
+    pt_h.copy_(pt.cpu())
+    sl_h.copy_(sl.cpu())
+    d_in, (q_d, pt_d, sl_d) = _packed((q, pt, sl), dev)
+    d_out, (step.o, step.lse) = _packed((step.o, step.lse), dev)
+    h_out, (o_h, lse_h) = _packed((step.o, step.lse), "cpu")
 
     def e2e_step():
-        q_d.copy_(q_h, non_blocking=True)
-        pt_d.copy_(pt_h, non_blocking=True)
-        sl_d.copy_(sl_h, non_blocking=True)
+        d_in.copy_(h_in, non_blocking=True)
         step.select(q_d, sig, pt_d, sl_d)
         decode_call(q_d, pt_d, sl_d)
         step.combine()
-        o_h.copy_(step.o, non_blocking=True)
-        lse_h.copy_(step.lse, non_blocking=True)
+        h_out.copy_(d_out, non_blocking=True)
 
     for _ in range(3):
         e2e_step()
@@ -638,8 +656,8 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         t_e2e = float(t.item())
     e2e_value = world * kv_bytes * K / t_e2e / 1e9
-    h2d = q_h.numel() * 2 + pt_h.numel() * 4 + sl_h.numel() * 4
-    d2h = o_h.numel() * 4 + lse_h.numel() * 4
+    h2d = h_in.numel()
+    d2h = h_out.numel()
 
     # correctness guard on what was timed: the outputs are finite and selections full
     assert torch.isfinite(step.o).all().item(), "non-finite output"
