@@ -137,10 +137,12 @@ def selected_kv_bytes(counts, pages, seq_lens, P, D, elem_bytes=2):
     return int(toks.sum().item()) * D * elem_bytes * 2 + scales
 
 
-def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=None):
+def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=None,
+                 min_s: float = 0.0):
     """Oracle (float64, host cores) on a bounded sample: n_units (b, kv head)
     pairs, select + attention (over FP8 pages when f8 holds their codes and
-    scales).  Returns GB/s of selected KV and the sample."""
+    scales), in repeated passes until min_s seconds have elapsed (and never
+    past budget_s).  Returns GB/s of selected KV, units done, seconds."""
     import numpy as np
 
     import oracle as O
@@ -153,7 +155,8 @@ def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=No
     G = cfg.G
     t0 = time.perf_counter()
     done, kv_bytes = 0, 0
-    for (b, h) in units:
+    import itertools
+    for (b, h) in itertools.cycle(units):   # (ends by the checks at the bottom)
         pages_np, counts_np = O.select_pages(qb, sig_bits, pt, sl, cfg.page_size, cfg.sink_tokens,
                                              cfg.local_tokens, cfg.budget_tokens, units=[(b, h)])
         lst = pages_np[b, h, :counts_np[b, h]]
@@ -182,7 +185,8 @@ def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=No
         eb = 2 if f8 is None else 1
         kv_bytes += sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst) * cfg.D * 2 * eb
         done += 1
-        if time.perf_counter() - t0 > budget_s:
+        el = time.perf_counter() - t0
+        if el > budget_s or (done % len(units) == 0 and el >= min_s):
             break
     dt = time.perf_counter() - t0
     return kv_bytes / dt / 1e9, done, dt
@@ -734,11 +738,14 @@ def main():
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=8, budget_s=20.0, f8=f8)
+        n_all = cfg.B * cfg.Hkv
+        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=n_all, budget_s=20.0, f8=f8,
+                                  min_s=10.0)
         line["cpu_baseline"] = {"value": round(gbs, 6), "unit": "GB/s", "cores": cores,
                                 "kind": "oracle",
-                                "sample": f"{n} of {cfg.B * cfg.Hkv} (sequence, kv head) units: "
-                                          f"select + attention, {dt:.1f} s"}
+                                "sample": f"{n} (sequence, kv head) units = {n / n_all:.2f} passes "
+                                          f"over all {n_all} of the workload: select + "
+                                          f"attention, {dt:.1f} s"}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
