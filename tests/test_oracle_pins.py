@@ -269,8 +269,9 @@ def _attn_case(rng, B=2, T=1, Hq=4, Hkv=2, D=16, Dv=16, P=4, lens=(23, 14)):
     return q, k, v, pt, np.array(lens, dtype=np.int32), npages
 
 
-@pytest.mark.parametrize("T", [1, 3])
-def test_dense_budget_equals_sdpa(T):
+@pytest.mark.parametrize("T,scale_mult", [(1, 1.0), (3, 1.0), (2, -1.0), (2, 3.0)])
+def test_dense_budget_equals_sdpa(T, scale_mult):
+    # also at a negative scale and a 3x sharper one (the GPU parity cases use both)
     rng = np.random.default_rng(30 + T)
     q, k, v, pt, sl, npages = _attn_case(rng, T=T)
     B, _, Hq, D = q.shape
@@ -283,7 +284,7 @@ def test_dense_budget_equals_sdpa(T):
         lists[b, :, :npages[b]] = np.arange(npages[b])
         counts[b] = npages[b]
     h2l = np.arange(Hq) // G
-    scale = 1 / math.sqrt(D)
+    scale = scale_mult / math.sqrt(D)
     o, lse = O.sparse_attention(q, k, v, pt, sl, lists, counts, h2l, scale, P)
     for b in range(B):
         L = int(sl[b])
