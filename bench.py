@@ -214,6 +214,18 @@ def _timed_graphs(g_step, g_kernel, K, flush_l2, stream, local):
     return t_step, t_kern, clk.summary()
 
 
+def max_over_ranks(x: float, world: int, dev) -> float:
+    """The largest of every rank's x: a multi-GPU job takes as long as its slowest
+    rank (replicas: each rank runs its own batch; no data-path collective)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def _packed(like, device):
     """One contiguous byte buffer holding tensors shaped like `like` back to back
     (16-byte aligned offsets; pinned when on the host), and a view of each: a
@@ -391,7 +403,12 @@ def run_extra(args, dev, world, rank, local, cores):
     for _ in range(3):
         g_step.replay()
         g_kern.replay()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
     t_step, t_kern, clocks = _timed_graphs(g_step, g_kern, K, flush_l2, stream, local)
+    if world > 1:
+        dist.barrier()
 
     # end to end through the same API: the step's inputs from pinned host memory
     # (packed: one host-to-device copy) and its outputs back (packed: one copy)
@@ -423,18 +440,20 @@ def run_extra(args, dev, world, rank, local, cores):
     d2h = h_out.numel()
     assert torch.isfinite(o).all().item(), "non-finite output"
 
+    t_step = max_over_ranks(t_step, world, dev)
+    t_e2e = max_over_ranks(t_e2e, world, dev)
     peak, kind = _peak_tflops()
     achieved = flops / (t_kern / K) / 1e12
     t_floor = _launch_floor(flush_l2, stream, min(K, 50))
     line = {
-        "metric": METRIC, "value": round(kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s",
+        "metric": METRIC, "value": round(world * kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(1e3 * t_step / K, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": cfg.name, "n_splits": n_splits,
                    "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
-        "calls_per_sec": round(K / t_step, 2),
-        "step_tflops": round(flops * K / t_step / 1e12, 2),
+        "calls_per_sec": round(world * K / t_step, 2),
+        "step_tflops": round(world * flops * K / t_step / 1e12, 2),
         "selected_kv_bytes_per_step": kv_bytes, "flops_per_step": flops,
         "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -442,7 +461,7 @@ def run_extra(args, dev, world, rank, local, cores):
                      "kernel_ms": round(1e3 * t_kern / K, 4),
                      "launch_floor_us": round(1e6 * t_floor, 2),
                      "launch_floor_what": LAUNCH_FLOOR_WHAT},
-        "e2e": {"value": round(kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
+        "e2e": {"value": round(world * kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(1e3 * t_e2e / K, 4)},
         "gpu_launches": (5 if args.workload == "prefill" else 4) * K,
@@ -450,6 +469,10 @@ def run_extra(args, dev, world, rank, local, cores):
     }
     if rank == 0:
         print(json.dumps(line))
+    if world > 1:
+        del g_step, g_kern
+        dist.barrier()
+        dist.destroy_process_group()
 
 
 def main():
@@ -615,12 +638,7 @@ def main():
     torch.cuda.synchronize()
     t_sel = st_ev[0].elapsed_time(st_ev[1]) / 1e3 * K
     t_cmb = st_ev[2].elapsed_time(st_ev[3]) / 1e3 * K
-    if world > 1:
-        t = torch.tensor([t_step], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_step_max = float(t.item())
-    else:
-        t_step_max = t_step
+    t_step_max = max_over_ranks(t_step, world, dev)
     value = world * kv_bytes * K / t_step_max / 1e9
     calls_per_sec = world * K / t_step_max
 
@@ -655,10 +673,7 @@ def main():
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     t_e2e = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
-    if world > 1:
-        t = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        t_e2e = float(t.item())
+    t_e2e = max_over_ranks(t_e2e, world, dev)
     e2e_value = world * kv_bytes * K / t_e2e / 1e9
     h2d = h_in.numel()
     d2h = h_out.numel()
