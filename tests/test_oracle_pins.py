@@ -229,7 +229,10 @@ def test_selection_refines_cancelling_scores():
     assert list(pages[0, 0, :counts[0, 0]]) == [0, 1, 3]
 
 
-def test_mla_tiers():
+@pytest.mark.parametrize("alpha,beta", [(3, 4), (0, 7), (6, 6)])
+def test_mla_tiers(alpha, beta):
+    # (0, 7): no critical tier; (6, 6): the tiers ask for more pages than a
+    # sequence holds (every page in, the critical ones first by rank)
     rng = np.random.default_rng(23)
     B, T, Hq, Dk, P = 2, 2, 8, 24, 4
     q = rand_bf16(rng, (B, T, Hq, Dk))
@@ -237,16 +240,16 @@ def test_mla_tiers():
     sig = rand_bf16(rng, (pool, 1, Dk))
     pt = rng.permutation(pool).astype(np.int32).reshape(2, 10)
     sl = np.array([40, 37], dtype=np.int32)
-    crit, cc, amb, ac = O.select_pages_mla(q, sig, pt, sl, P, 3, 4)
+    crit, cc, amb, ac = O.select_pages_mla(q, sig, pt, sl, P, alpha, beta)
     for b in range(B):
         nb = -(-int(sl[b]) // P)
         exact = {p: max(float(exact_dot_fraction(q[b, t, h], sig[pt[b, p], 0]))
                         for t in range(T) for h in range(Hq)) for p in range(nb)}
         order = sorted(range(nb), key=lambda p: (-exact[p], p))
-        assert list(crit[b, :cc[b]]) == sorted(order[:3])
-        assert list(amb[b, :ac[b]]) == sorted(order[3:7])
+        assert list(crit[b, :cc[b]]) == sorted(order[:alpha])
+        assert list(amb[b, :ac[b]]) == sorted(order[alpha:alpha + beta])
     # with every head ambient, crit u amb equals the untiered top-(alpha+beta)
-    pages, counts = O.select_pages(q, sig, pt, sl, P, 0, 0, 7 * P)
+    pages, counts = O.select_pages(q, sig, pt, sl, P, 0, 0, (alpha + beta) * P)
     for b in range(B):
         assert sorted(list(crit[b, :cc[b]]) + list(amb[b, :ac[b]])) == list(pages[b, 0, :counts[b, 0]])
 
