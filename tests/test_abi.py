@@ -128,3 +128,16 @@ def test_attention_workspace_size_and_host_checks():
                                        fake, fake, 2, 16, ctypes.cast(h2l, ctypes.c_void_p), 1, 1,
                                        8, 2, 128, 16, 64, 0.1, 2, fake, None, None, None, need,
                                        None, None) == 3
+
+
+def test_default_split_policy():
+    from paged_sparse_kv_sa_b200.pipeline import default_splits
+    # one wave of decode warps (12 per SM on 148 SMs) over the (sequence, kv head) units
+    assert default_splits(16 * 8, 64, 148) == 13      # Llama-8B-shaped decode
+    assert default_splits(32 * 8, 128, 148) == 6      # Llama-70B-shaped decode
+    assert default_splits(2, 16, 148) == 16           # never more splits than list entries
+    assert default_splits(0, 5, 148) == 1
+    for units, max_list in [(4, 1000), (1, 5000), (300, 300), (7, 129)]:
+        n = default_splits(units, max_list, 148)
+        assert 1 <= n <= 64
+        assert -(-max_list // n) <= 128 or n == 64   # a split holds at most 128 entries
