@@ -141,3 +141,25 @@ def test_default_split_policy():
         n = default_splits(units, max_list, 148)
         assert 1 <= n <= 64
         assert -(-max_list // n) <= 128 or n == 64   # a split holds at most 128 entries
+
+
+def test_tiered_selection_host_checks():
+    lib = sa.load()
+    fake = ctypes.c_void_p(0x1000)
+    s = _i64x4(2 * 128 * 576, 128 * 576, 576, 1)
+
+    def call(max_pages, alpha=8, beta=24, Dk=576, ws_bytes=1 << 40):
+        return lib.sa_select_pages_tiered(fake, s, fake, fake, fake, 8, 2, 128, Dk, 64, max_pages,
+                                          8192, alpha, beta, fake, fake, fake, ws_bytes, None,
+                                          None)
+    assert call(8193) == 2                    # above the 8192 pages its choose pass holds
+    assert call(1024, Dk=572) == 2            # Dk not a multiple of 8
+    assert call(1024, alpha=0, beta=0) == 1   # no page asked for
+    assert call(1024, alpha=-1) == 1
+    assert call(1024, ws_bytes=16) == 3       # workspace too small
+    assert call(0) == 0                       # nothing to select: no launch
+    # workspace: brackets and row masks per (sequence, 32-row group, page), exact-score
+    # keys per (sequence, page), one counter per sequence (16-byte rounded)
+    n_rg = (2 * 128 + 31) // 32
+    want = 8 * 1024 * (n_rg * (8 + 8) + 8) + (8 * 4 + 15) // 16 * 16
+    assert lib.sa_select_tiered_workspace_size(8, 2, 128, 1024) == want
