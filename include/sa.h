@@ -134,7 +134,9 @@ SA_API size_t sa_select_workspace_size(int B, int Hkv, int max_pages);
  * memory (2,097,152 pages x 8 bytes), which every GPU that loads the library
  * holds until the process exits.  Limit: B * Hkv * max_pages <= 2,097,152;
  * larger calls return SA_ERR_UNSUPPORTED and launch nothing.  The first call
- * on a device looks up the array's device address (cudaGetSymbolAddress); make
+ * on a device looks up the array's device address (cudaGetSymbolAddress) and
+ * keeps it for that device's current context; the first call after the
+ * context is created again (cudaDeviceReset, say) looks it up afresh.  Make
  * that first call before any stream capture.  All calls share the one array
  * (it needs no clearing: each call writes every entry it reads), so calls
  * whose kernels overlap on the GPU — on different streams, or from different

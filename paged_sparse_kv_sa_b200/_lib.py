@@ -141,6 +141,26 @@ def page_budget(sink_tokens: int, local_tokens: int, budget_tokens: int, page_si
     return n_sink, n_local, budget_pages, budget_pages - n_sink - n_local
 
 
+def _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts, bp):
+    """The shapes the selection kernels assume (dense [P_pool,Hkv,Dk] summaries,
+    [B,max_pages] table, [B] lengths, [B,Hkv,budget_pages] / [B,Hkv] outputs):
+    a view with other strides would be read or written in the wrong layout."""
+    B = q.shape[0]
+    Hkv = summaries.shape[1]
+    if summaries.dim() != 3 or summaries.shape[2] != q.shape[3]:
+        raise ValueError("summaries must be [P_pool, Hkv, Dk] with the query's Dk")
+    if page_table.dim() != 2 or page_table.shape[0] != B:
+        raise ValueError("page_table must be [B, max_pages]")
+    if tuple(seq_lens.shape) != (B,):
+        raise ValueError("seq_lens must be [B]")
+    for t, shape, what in ((out_pages, (B, Hkv, max(bp, 1)), "out_pages"),
+                           (out_counts, (B, Hkv), "out_counts")):
+        if t is None:
+            continue
+        if t.dtype != torch.int32 or not t.is_contiguous() or tuple(t.shape) != shape:
+            raise TypeError(f"{what} must be a contiguous int32 tensor of shape {shape}")
+
+
 def sa_select_workspace_size(B: int, Hkv: int, max_pages: int) -> int:
     return int(load().sa_select_workspace_size(B, Hkv, max_pages))
 
@@ -158,6 +178,7 @@ def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tok
     P_pool_, Hkv, _ = summaries.shape
     P_pool = P_pool_ if P_pool is None else P_pool
     bp = budget_tokens // page_size
+    _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts, bp)
     if out_pages is None:
         out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
     if out_counts is None:
@@ -180,13 +201,19 @@ def sa_select_pages_no_alloc(q, summaries, page_table, seq_lens, page_size: int,
                              out_counts, dev_error=None, P_pool: int = None, stream=None):
     """sa_select_pages without a workspace: the score bounds go to the library's
     static device array (shared by all calls; calls must not overlap on the GPU).
-    The outputs must be preallocated; nothing is allocated here."""
+    The outputs must be preallocated and every tensor laid out as the C call
+    assumes (contiguous summaries and outputs): nothing is copied or allocated
+    here, so a strided view is refused rather than made contiguous."""
     lib = load()
     _need_cuda(q, summaries, page_table, seq_lens, out_pages, out_counts)
-    _bf16(q), _bf16(summaries), _i32(page_table), _i32(seq_lens)
+    _bf16(q), _i32(page_table), _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
     B, T, Hq, Dk = q.shape
     P_pool_, Hkv, _ = summaries.shape
     P_pool = P_pool_ if P_pool is None else P_pool
+    _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts,
+                   budget_tokens // page_size)
     st = lib.sa_select_pages_no_alloc(_ptr(q), _strides4(q), _ptr(summaries), _ptr(page_table),
                                       _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size,
                                       page_table.shape[1], P_pool, sink_tokens, local_tokens,

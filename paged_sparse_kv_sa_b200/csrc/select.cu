@@ -592,7 +592,9 @@ size_t select_workspace_bytes(int B, int Hkv, int max_pages) {
 }
 
 cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
-  if (a.k_top > 0) {
+  // (an empty page table holds no candidate: the choose pass alone writes the
+  // empty selections, without reading any score bound)
+  if (a.k_top > 0 && a.max_pages > 0) {
     // kv-head block: the largest divisor of Hkv with hb <= 8 and an hb-head
     // run of at most 2 KB
     int hb = 1;
@@ -642,23 +644,64 @@ static __device__ __align__(256) float2 g_static_score_bounds[kStaticScoreEntrie
 namespace {
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
-float2* g_static_ptr[kMaxDevices] = {};
+// Per device: the array's address in the context it was looked up in.  A
+// module's device globals live as long as the context that loaded it, so the
+// address is keyed by the context's unique id: after the primary context is
+// torn down and created again (cudaDeviceReset, say) the array may sit
+// elsewhere, and the next call looks it up afresh.
+struct StaticSlot {
+  unsigned long long ctx_id;
+  float2* ptr;
+};
+StaticSlot g_static_slot[kMaxDevices] = {};
 
-// Device address of the static array on the current device; looked up once per
-// device (the host-side symbol is only a stand-in and must not reach a kernel).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the static array in the current device's context, looked
+// up (cudaGetSymbolAddress) on the first call in that context: the host-side
+// symbol is only a stand-in and must never reach a kernel.
 cudaError_t static_scores_ptr(float2** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // the lookup below also makes the runtime create the context if needed, so
+  // read the id after it when there is none yet
+  unsigned long long id = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_static_mu);
-  if (!g_static_ptr[dev]) {
+  StaticSlot& s = g_static_slot[dev];
+  if (!s.ptr || id == 0 || s.ctx_id != id) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_static_score_bounds);
     if (e != cudaSuccess) return e;
-    g_static_ptr[dev] = static_cast<float2*>(p);
+    s.ptr = static_cast<float2*>(p);
+    s.ctx_id = id ? id : current_ctx_id();
   }
-  *out = g_static_ptr[dev];
+  *out = s.ptr;
   return cudaSuccess;
 }
 }  // namespace
