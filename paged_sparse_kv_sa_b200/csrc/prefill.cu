@@ -8,19 +8,26 @@
 //   warp 8      gathers K and V tiles from the paged pool with TMA (four
 //               16-key x 64-column boxes per 64-column chunk; an absent or
 //               invalid 16-key group is loaded from an out-of-range page
-//               coordinate, which TMA fills with zeros) into a 3-stage ring;
+//               coordinate, which TMA fills with zeros) into a 4-stage ring;
 //   warp 9      issues tcgen05.mma, alternating between the tiles: S_A = Q_A K^T
 //               and S_B = Q_B K^T (M=128, N=64, K=D) into double-buffered TMEM
 //               S buffers, then O_A += P_A V and O_B += P_B V (M=128, N=D) into
-//               TMEM, with tcgen05.commit arrivals on mbarriers;
+//               TMEM with P read from TMEM as the A operand, with
+//               tcgen05.commit arrivals on mbarriers;
 //   warps 0-3 / 4-7   (one warpgroup per tile) own one query row per thread:
 //               Q into shared memory, S rows from TMEM, masking (page validity,
 //               sequence end, causal position; skipped for tiles every row sees
 //               whole), a base-2 online softmax whose running max only moves when
 //               a row's max exceeds it by more than 2^8 (the O rescale through
-//               TMEM is then rare), P (bf16) to shared memory, and the epilogue.
-// While one warpgroup runs its softmax the tensor core works on the other's
-// tile, and QK^T of tile j+1 overlaps the softmax of tile j.
+//               TMEM is then rare), P back into the S buffer it came from, and
+//               the epilogue.
+// P enters PV as a bf16 pair hi + lo (hi = RNE_bf16(p), lo = RNE_bf16(p - hi)),
+// so its rounding is ~2^-17 relative rather than the 2^-9 of a single bf16: two
+// MMAs per 16 keys, both reading the pair from the TMEM columns where that
+// tile's scores were (64 keys = 32 columns of hi pairs + 32 of lo pairs).
+// A softmax warpgroup computes P of tile j while the tensor core still runs
+// PV of tile j-1 and QK^T of tile j+1; it waits for PV of tile j-1 only
+// before handing P of tile j over (and before the rare rescale of O).
 //
 // Sources: CompactAttention (abstract on the page titled "Causal Attention on
 // CPU: A Cache-Aware and Load-Balanced Scheduling Kernel for Prefill"):
@@ -35,7 +42,7 @@ namespace sa {
 namespace {
 
 constexpr int kPThreads = 320;    // 2 softmax warpgroups, producer warp, MMA warp
-constexpr int kPStages = 3;
+constexpr int kPStages = 4;
 constexpr int kKeys = 64;         // keys per tile
 constexpr int kM = 128;           // query rows per warpgroup tile
 constexpr int kRows = 2 * kM;     // query rows per CTA
@@ -48,9 +55,9 @@ struct PCfg {
   static constexpr int kQBytes = kM * D * 2;
   static constexpr int kTileBytes = kKeys * D * 2;     // one K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kPBytes = kM * kKeys * 2;
-  static constexpr int kDyn = 2 * kQBytes + 2 * kPBytes + kPStages * kStageBytes + 1024;
-  // per tile w: S buffers at 128w + {0, 64}, O at 256 + 128w
+  static constexpr int kDyn = 2 * kQBytes + kPStages * kStageBytes + 1024;
+  // per tile w: S buffers at 128w + {0, 64} (P hi + lo after the softmax:
+  // columns +0..31 and +32..63), O at 256 + 128w
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdQK = tc::idesc_bf16_f32(kM, kKeys, false, false);
   static constexpr uint32_t kIdPV = tc::idesc_bf16_f32(kM, D, false, true);
@@ -107,8 +114,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
   uint8_t* q_s = smem;                                       // 2 tiles
-  uint8_t* p_s = smem + 2 * C::kQBytes;                      // 2 tiles
-  uint8_t* kv_s = p_s + 2 * C::kPBytes;                      // kPStages x (K | V)
+  uint8_t* kv_s = smem + 2 * C::kQBytes;                     // kPStages x (K | V)
   __shared__ uint64_t kv_full[kPStages], kv_empty[kPStages];
   __shared__ uint64_t s_full[2][2], p_full[2], o_done[2], q_full;
   __shared__ uint32_t tmem_base_s;
@@ -244,18 +250,23 @@ __global__ void __launch_bounds__(kPThreads, 1)
   } else if (warp == 9) {
     // ================= MMA issuer (one thread), alternating tiles A and B
     if (lane == 0 && n_act > 0) {
-      const uint32_t q_addr = smem_u32(q_s), p_addr = smem_u32(p_s), kv_addr = smem_u32(kv_s);
+      const uint32_t q_addr = smem_u32(q_s), kv_addr = smem_u32(kv_s);
+      // O_w += P_w V for tile jp: P (hi, then lo) from the TMEM columns of the
+      // S buffer the tile's scores were in.  QK^T of tile jp + 2, issued after
+      // this, reuses those columns: MMAs of one thread execute in issue order.
       auto pv = [&](int jp) -> bool {
         const int st = jp % kPStages;
         const uint32_t vbase = kv_addr + st * C::kStageBytes + C::kTileBytes;
         for (int w = 0; w < 2; ++w) {
           if (!wait_or_abort(&p_full[w], jp & 1, abort_flag)) return false;
           tc::fence_after_sync();
+          const uint32_t pcol = tmem + 128 * w + (jp & 1) * kKeys;
 #pragma unroll
           for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(p_addr + w * C::kPBytes + kk * 32, 16, 1024);
             const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
-            tc::mma_bf16(tmem + 256 + 128 * w, ad, bd, C::kIdPV, (jp > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + 256 + 128 * w, pcol + 8 * kk, bd, C::kIdPV,
+                            (jp > 0 || kk > 0) ? 1u : 0u);
+            tc::mma_bf16_ts(tmem + 256 + 128 * w, pcol + 32 + 8 * kk, bd, C::kIdPV, 1u);
           }
           tc::commit(&o_done[w]);
         }
@@ -308,7 +319,6 @@ __global__ void __launch_bounds__(kPThreads, 1)
     mbar_arrive(&q_full);
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t s_col = 128 * wg, o_col = 256 + 128 * wg;
-    uint8_t* prow = p_s + wg * C::kPBytes + r * 128;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int jj = 0; jj < n_act; ++jj) {
@@ -341,16 +351,44 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       const float mr = sl >= 0.f ? reduce_n<false>(x) : reduce_n<true>(x);
       const float mx = mr != mr ? -INFINITY : mr * sl;
-      // PV(jj-1) must be done before O is rescaled or P is rewritten
+      const bool move = mx > m_ref + kLazyP;
+      const float m_new = move ? mx : m_ref;
+      const float nb = m_new == -INFINITY ? 0.f : -m_new;
+      // P = 2^(x sl - m_new) as bf16 hi + lo pairs, written over this tile's
+      // scores in TMEM (the S buffer is free: QK^T of the tile is complete and
+      // PV of tile jj - 2, the buffer's previous reader, completed before it)
+      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // (independent chains)
+      uint32_t ph[32], pl[32];
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        float p[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float v = x[ch * 8 + i];
+          p[i] = ex2_approx(fmaf(v, sl, nb));
+          if (masked) p[i] = v == v ? p[i] : 0.f;
+          ls[i] += p[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t h = pack_bf16(p[2 * i], p[2 * i + 1]);
+          ph[ch * 4 + i] = h;
+          pl[ch * 4 + i] = pack_bf16(p[2 * i] - bf16_bits_to_float(h & 0xffffu),
+                                     p[2 * i + 1] - bf16_bits_to_float(h >> 16));
+        }
+      }
+      tc::st32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(ph));
+      tc::st32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(pl));
+      tc::wait_st();
+      // PV(jj-1) must be done before O is rescaled and before P(jj) is handed
+      // over (its completion also keeps this barrier's phases in step)
       if (jj >= 1 && !wait_or_abort(&o_done[wg], (jj - 1) & 1, abort_flag)) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      const bool move = mx > m_ref + kLazyP;
       if (__any_sync(0xffffffffu, move)) {
         const float alpha = move ? exp2f(m_ref - mx) : 1.f;
-        if (move) m_ref = mx;
         l *= alpha;
         if (jj >= 1) {
 #pragma unroll
@@ -365,27 +403,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
           tc::wait_st();
         }
       }
-      const float nb = m_ref == -INFINITY ? 0.f : -m_ref;
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // (independent chains)
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float v = x[ch * 8 + i];
-          p[i] = ex2_approx(fmaf(v, sl, nb));
-          if (masked) p[i] = v == v ? p[i] : 0.f;
-          ls[i] += p[i];
-        }
-        uint4 w;
-        w.x = pack_bf16(p[0], p[1]);
-        w.y = pack_bf16(p[2], p[3]);
-        w.z = pack_bf16(p[4], p[5]);
-        w.w = pack_bf16(p[6], p[7]);
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = w;
-      }
+      m_ref = m_new;
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      tc::fence_proxy_async();
       tc::fence_before_sync();
       mbar_arrive(&p_full[wg]);
     }

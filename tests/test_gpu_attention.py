@@ -239,11 +239,11 @@ def test_attention_negative_scale(path):
     assert_attn_close(*_scaled_case(path, -1.0, 48))
 
 
-@pytest.mark.parametrize("path", ["gqa", "mla"])
-def test_attention_sharp_softmax(path):
-    # three times the usual 1/sqrt(D): a few keys dominate each row, so the
-    # probabilities' rounding before the PV product shows directly in O.  The
-    # warp-MMA and MLA kernels multiply by P as bf16 hi + lo (~2^-17 relative)
-    # and hold the bar; the tcgen05 many-row kernel rounds P once to bf16 and is
-    # held to it at the usual scale only (its other tests)
-    assert_attn_close(*_scaled_case(path, 3.0, 49))
+@pytest.mark.parametrize("mult", [3.0, 8.0])
+@pytest.mark.parametrize("path", ["gqa", "tensor_core", "mla"])
+def test_attention_sharp_softmax(path, mult):
+    # three and eight times the usual 1/sqrt(D): a few keys dominate each row, so
+    # the probabilities' rounding before the PV product shows directly in O.
+    # Every kernel multiplies by P as a bf16 pair hi + lo (~2^-17 relative; a
+    # single bf16 P, 2^-9, missed the bar at three times the scale)
+    assert_attn_close(*_scaled_case(path, mult, 49))

@@ -548,8 +548,28 @@ def test_prefill_tcgen05_vs_oracle(T, q_off, P, n_splits, ragged):
     assert_attn_close(o, lse, ro, rl)
 
 
+@pytest.mark.parametrize("mult", [3.0, 8.0, -3.0])
+@pytest.mark.parametrize("T,q_off,P,n_splits,ragged", [(96, 448, 64, 2, 0), (40, 1000, 32, 3, 17)])
+def test_prefill_tcgen05_sharp_scales(T, q_off, P, n_splits, ragged, mult):
+    # a few keys dominate every row: P's rounding before the PV product shows in O
+    # directly (P enters as a bf16 pair hi + lo); a negative scale flips the row max
+    q, k, v, pt, sl, lists, cnt = prefill_case(2, T, q_off, P, ragged=ragged)
+    Hq, Hkv, D = q.shape[2], k.shape[1], q.shape[3]
+    h2l = [h // (Hq // Hkv) for h in range(Hq)]
+    scale = mult / math.sqrt(D)
+    o_p, l_p = sa.sa_sparse_decode(q.to(DEV), k.to(DEV), v.to(DEV), pt.to(DEV), sl.to(DEV),
+                                   torch.from_numpy(lists).to(DEV), torch.from_numpy(cnt).to(DEV),
+                                   h2l, scale, n_splits)
+    o, _, lse = sa.sa_combine(o_p, l_p)
+    torch.cuda.synchronize()
+    ro, rl = O.sparse_attention(bits(q), bits(k), bits(v), np_i32(pt), np_i32(sl), lists, cnt,
+                                np.array(h2l), scale, P)
+    assert_attn_close(o, lse, ro, rl)
+
+
 @pytest.mark.slow
-def test_prefill_full_size_sampled_rows():
+@pytest.mark.parametrize("mult", [1.0, 3.0])
+def test_prefill_full_size_sampled_rows(mult):
     cfg = W.UNION_PREFILL
     s = W.block_union_scores(cfg, seed=0, device=DEV)
     inp = W.prefill_inputs(cfg, seed=0, device=DEV)
@@ -559,7 +579,7 @@ def test_prefill_full_size_sampled_rows():
     o_p, l_p = sa.sa_sparse_decode(inp["q"], inp["k"], inp["v"], inp["page_table"],
                                    inp["seq_lens"], tables.view(1, cfg.Hkv, -1).contiguous(),
                                    counts.view(1, cfg.Hkv).contiguous(), h2l,
-                                   1.0 / math.sqrt(cfg.D), 2)
+                                   mult / math.sqrt(cfg.D), 2)
     o, _, lse = sa.sa_combine(o_p, l_p)
     torch.cuda.synchronize()
     rng = np.random.default_rng(5)
@@ -569,7 +589,7 @@ def test_prefill_full_size_sampled_rows():
     cb = np_i32(counts).reshape(1, cfg.Hkv)
     ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
                                 np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), tb, cb,
-                                np.array(h2l), 1.0 / math.sqrt(cfg.D), cfg.block, rows=rows)
+                                np.array(h2l), mult / math.sqrt(cfg.D), cfg.block, rows=rows)
     og = o.cpu().double().numpy()
     lg = lse.cpu().double().numpy()
     for (b, t, h) in rows:
