@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "internal.h"
@@ -101,6 +102,114 @@ int check_cache_u8(const uint8_t* p, const int64_t s[4]) {
 
 
 }  // namespace
+
+unsigned long long current_context_id() {
+  using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+  using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+namespace {
+// Values computed once per (context, what, kernel, argument).
+struct CacheKey {
+  unsigned long long ctx;
+  int what;
+  const void* fn;
+  long long arg;
+  bool operator<(const CacheKey& o) const {
+    if (ctx != o.ctx) return ctx < o.ctx;
+    if (what != o.what) return what < o.what;
+    if (fn != o.fn) return fn < o.fn;
+    return arg < o.arg;
+  }
+};
+std::mutex g_cache_mu;
+std::map<CacheKey, int> g_cache;
+
+template <typename F>
+cudaError_t cached(int what, const void* fn, long long arg, int* out, F&& compute) {
+  // make sure a context exists before its id is read
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long ctx = current_context_id();
+  const CacheKey key{ctx, what, fn, arg};
+  if (ctx) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    auto it = g_cache.find(key);
+    if (it != g_cache.end()) {
+      *out = it->second;
+      return cudaSuccess;
+    }
+  }
+  int v = 0;
+  e = compute(dev, &v);
+  if (e != cudaSuccess) return e;
+  if (ctx) {
+    std::lock_guard<std::mutex> lock(g_cache_mu);
+    g_cache[key] = v;
+  }
+  *out = v;
+  return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t allow_max_dyn_smem(const void* kern) {
+  int unused = 0;
+  return cached(0, kern, 0, &unused, [&](int dev, int* v) {
+    cudaFuncAttributes fa;
+    int optin = 0;
+    cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+    if (e == cudaSuccess)
+      e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               optin - (int)fa.sharedSizeBytes);
+    *v = 1;
+    return e;
+  });
+}
+
+cudaError_t prefer_max_carveout(const void* kern) {
+  int unused = 0;
+  return cached(1, kern, 0, &unused, [&](int, int* v) {
+    *v = 1;
+    return cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+}
+
+cudaError_t sm_count(int* out) {
+  return cached(2, nullptr, 0, out, [](int dev, int* v) {
+    return cudaDeviceGetAttribute(v, cudaDevAttrMultiProcessorCount, dev);
+  });
+}
+
+cudaError_t max_blocks_per_sm(const void* kern, int threads, size_t dyn_smem, int* out) {
+  const long long arg = ((long long)threads << 32) | (long long)dyn_smem;
+  return cached(3, kern, arg, out, [&](int, int* v) {
+    cudaError_t e = allow_max_dyn_smem(kern);
+    if (e != cudaSuccess) return e;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(v, kern, threads, dyn_smem);
+  });
+}
 
 bool encode_kv_map(CUtensorMap* map, const void* base, int D, int P, int Hkv, int P_pool,
                    const int64_t strides[4], int box_rows) {

@@ -466,16 +466,13 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   DecodeParams prm;
   prm.a = a;
   prm.pairs = pairs;
-  cudaError_t e = cudaFuncSetAttribute(decode_gqa_kernel<D, F8>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDynBytes);
-  if (e != cudaSuccess) return e;
-  // one wave of resident CTAs (or fewer when there is less work)
-  int dev = 0, sms = 0, per_sm = 0;
-  e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e == cudaSuccess)
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, decode_gqa_kernel<D, F8>, kNW * 32,
-                                                      C::kDynBytes);
+  // one wave of resident CTAs (or fewer when there is less work); the set-up
+  // queries are answered once per context
+  const void* kern = reinterpret_cast<const void*>(decode_gqa_kernel<D, F8>);
+  int sms = 0, per_sm = 0;
+  cudaError_t e = allow_max_dyn_smem(kern);
+  if (e == cudaSuccess) e = sm_count(&sms);
+  if (e == cudaSuccess) e = max_blocks_per_sm(kern, kNW * 32, C::kDynBytes, &per_sm);
   if (e != cudaSuccess) return e;
   const long long items = (long long)a.n_splits * pairs.n_pairs * a.B;
   const long long want = (items + kNW - 1) / kNW;

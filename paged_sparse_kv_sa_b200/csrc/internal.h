@@ -35,6 +35,22 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// ---- host-side set-up done once per CUDA context, not once per call
+// (a context created anew, after cudaDeviceReset say, is set up again).
+// Unique id of the calling thread's current context; 0 if it cannot be read
+// (then nothing is cached and every call does the set-up).
+unsigned long long current_context_id();
+// Let `kern` request up to the device's opt-in maximum of dynamic shared
+// memory (a cap only: what a launch uses is what it asks for).
+cudaError_t allow_max_dyn_smem(const void* kern);
+// Ask for the largest shared-memory carveout for `kern` (more resident CTAs
+// when they are limited by shared memory).
+cudaError_t prefer_max_carveout(const void* kern);
+// Streaming multiprocessors of the current device.
+cudaError_t sm_count(int* out);
+// Resident CTAs of `kern` per SM at this block size and dynamic shared memory.
+cudaError_t max_blocks_per_sm(const void* kern, int threads, size_t dyn_smem, int* out);
+
 constexpr int kMaxPairs = 64;        // (list, kv head) pairs one decode call may touch
 constexpr int kMaxHeadsPerPair = 128;
 constexpr int kMaxHeads = 256;       // query heads of a decode call

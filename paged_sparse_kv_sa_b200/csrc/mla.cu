@@ -542,8 +542,7 @@ cudaError_t launch_mla(const DecodeArgs& a, const PairTable& pairs, const CUtens
       prm.item_qt[prm.n_items] = static_cast<int16_t>(qt);
       ++prm.n_items;
     }
-  cudaError_t e =
-      cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMDyn);
+  cudaError_t e = allow_max_dyn_smem(reinterpret_cast<const void*>(mla_kernel));
   if (e != cudaSuccess) return e;
   if (prm.n_items == 0) return cudaSuccess;
   dim3 grid(prm.n_items * a.n_splits, 1, a.B);

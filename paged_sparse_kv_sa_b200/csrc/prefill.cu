@@ -452,8 +452,7 @@ cudaError_t launch_p(const DecodeArgs& a, const PairTable& pairs, const CUtensor
   int max_rows = 0;
   for (int i = 0; i < pairs.n_pairs; ++i) max_rows = max(max_rows, a.T * pairs.n_heads[i]);
   const int qtiles = (max_rows + kRows - 1) / kRows;
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDyn);
+  cudaError_t e = allow_max_dyn_smem(reinterpret_cast<const void*>(prefill_kernel<D>));
   if (e != cudaSuccess) return e;
   dim3 grid(qtiles * a.n_splits, pairs.n_pairs, a.B);
   return launch_pdl(prefill_kernel<D>, grid, dim3(kPThreads), C::kDyn, stream, prm, kmap, vmap);

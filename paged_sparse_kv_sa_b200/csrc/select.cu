@@ -606,7 +606,7 @@ cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
       constexpr int DK = decltype(dk)::value;
       auto launch = [&](auto kern, int nt) {
         const int dyn = hb * 8 * nt * (DK * 2 + 16) + kScoreStages * 16 * (hb * DK * 2 + 16);
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+        cudaError_t e = allow_max_dyn_smem(reinterpret_cast<const void*>(kern));
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, g1, dim3((hb + 1) * 32), dyn, stream, a, hb);
       };
@@ -618,11 +618,9 @@ cudaError_t launch_select_gqa(const SelectArgs& a, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
   }
   const size_t dyn = (size_t)a.max_pages * (4 + 4 + 2 + 1) + 16;
-  cudaError_t e = cudaFuncSetAttribute(choose_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)dyn);
+  cudaError_t e = allow_max_dyn_smem(reinterpret_cast<const void*>(choose_kernel));
   // the largest shared-memory carveout: two CTAs per SM up to 8192 pages
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(choose_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e == cudaSuccess) e = prefer_max_carveout(reinterpret_cast<const void*>(choose_kernel));
   if (e != cudaSuccess) return e;
   return launch_pdl(choose_kernel, dim3(a.Hkv, a.B), dim3(kThreads), dyn, stream, a);
 }
@@ -655,32 +653,6 @@ struct StaticSlot {
 };
 StaticSlot g_static_slot[kMaxDevices] = {};
 
-using CtxGetCurrentFn = CUresult (*)(CUcontext*);
-using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
-
-// Unique id of the calling thread's current context (0 if it cannot be read).
-unsigned long long current_ctx_id() {
-  static CtxGetCurrentFn get_current = nullptr;
-  static CtxGetIdFn get_id = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
-    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess && q == cudaDriverEntryPointSuccess)
-      get_id = reinterpret_cast<CtxGetIdFn>(p);
-  });
-  CUcontext ctx = nullptr;
-  unsigned long long id = 0;
-  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx ||
-      get_id(ctx, &id) != CUDA_SUCCESS)
-    return 0;
-  return id;
-}
-
 // Device address of the static array in the current device's context, looked
 // up (cudaGetSymbolAddress) on the first call in that context: the host-side
 // symbol is only a stand-in and must never reach a kernel.
@@ -691,7 +663,7 @@ cudaError_t static_scores_ptr(float2** out) {
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   // the lookup below also makes the runtime create the context if needed, so
   // read the id after it when there is none yet
-  unsigned long long id = current_ctx_id();
+  unsigned long long id = current_context_id();
   std::lock_guard<std::mutex> lock(g_static_mu);
   StaticSlot& s = g_static_slot[dev];
   if (!s.ptr || id == 0 || s.ctx_id != id) {
@@ -699,7 +671,7 @@ cudaError_t static_scores_ptr(float2** out) {
     e = cudaGetSymbolAddress(&p, g_static_score_bounds);
     if (e != cudaSuccess) return e;
     s.ptr = static_cast<float2*>(p);
-    s.ctx_id = id ? id : current_ctx_id();
+    s.ctx_id = id ? id : current_context_id();
   }
   *out = s.ptr;
   return cudaSuccess;

@@ -638,20 +638,17 @@ cudaError_t launch_select_tiered(TieredArgs a, cudaStream_t stream) {
   a.exkey = a.rmask + nl;
   a.counter = reinterpret_cast<unsigned int*>(a.exkey + (size_t)a.B * a.max_pages);
   const int dyn1 = kSStages * kSStageBytes + 1024;   // + alignment slack
-  cudaError_t e = cudaFuncSetAttribute(tiered_score_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, dyn1);
+  cudaError_t e = allow_max_dyn_smem(reinterpret_cast<const void*>(tiered_score_kernel));
   if (e != cudaSuccess) return e;
   dim3 g1((a.max_pages + kSP - 1) / kSP, (a.T * a.Hq + kSR - 1) / kSR, a.B);
   e = launch_pdl(tiered_score_kernel, g1, dim3(kSThreads), dyn1, stream, a);
   if (e != cudaSuccess) return e;
   const size_t dyn2 = (size_t)a.max_pages * kChooseBytesPerPage + 16;
-  e = cudaFuncSetAttribute(tiered_choose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)dyn2);
+  e = allow_max_dyn_smem(reinterpret_cast<const void*>(tiered_choose_kernel));
   if (e != cudaSuccess) return e;
   // enough CTAs per sequence to spread the exact rescoring over the SMs
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int sms = 0;
+  e = sm_count(&sms);
   if (e != cudaSuccess) return e;
   const int n_cta = std::max(1, std::min(kChooseCtas, sms / std::max(1, a.B)));
   return launch_pdl(tiered_choose_kernel, dim3(a.B, n_cta), dim3(kChooseThreads), dyn2, stream, a);

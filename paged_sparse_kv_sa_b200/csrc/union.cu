@@ -119,8 +119,7 @@ cudaError_t launch_block_union(const float* scores, int Hq, int Hkv, int NQB, in
       launch_pdl(union_clear_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, stream, tables, n);
   if (e != cudaSuccess) return e;
   const size_t kbytes = sizeof(unsigned long long) * (size_t)NKB;
-  e = cudaFuncSetAttribute(union_mark_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kbytes);
+  e = allow_max_dyn_smem(reinterpret_cast<const void*>(union_mark_kernel));
   if (e != cudaSuccess) return e;
   if (NQB > 0) {
     e = launch_pdl(union_mark_kernel, dim3(NQB, Hq), dim3(kUThreads), kbytes, stream, scores, Hq,
