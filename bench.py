@@ -1,29 +1,51 @@
-"""Benchmark: sparse-attention decode steps on the Llama-3-8B-shaped workload.
+"""Benchmark: paged sparse-KV attention on one B200 per rank.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload all|llama8b|llama70b|mla|prefill|llama8b_fp8]
 
 A step is one pass of the whole hot path over one batch: page selection
-(sa_select_pages), the gather split-KV decode (sa_sparse_decode) and the
-split merge (sa_combine).  Workload: B=16 sequences of 32768 tokens, Hq=32,
-Hkv=8, D=128, 16-token pages in a shuffled 2 GiB pool, budget 1024 tokens
-(2 sink + 32 local + 30 top-k pages per kv head), 5% of pages per kv head
-lifted 3 sigma along the group query; bf16 N(0,1) data, seed 0; summaries
-built once by sa_build_page_summaries (not part of a step).
+(scoring against the per-page key summaries, forced sink and local pages,
+top-k), the gather split-KV decode over the selected lists and the split merge.
+The headline workload is the Llama-3-8B-shaped decode: B=16 sequences of 32768
+tokens, Hq=32, Hkv=8, D=128, 16-token pages in a shuffled 2 GiB pool per layer,
+budget 1024 tokens (2 sink + 32 local + 30 top-k pages per kv head), 5% of the
+pages per kv head lifted 3 sigma along the group query; bf16 N(0,1) data.  A
+step is the library's one-call entry (sa_sparse_step: four launches).
 
-The metric is selected-KV GB/s: K+V bytes of the selected pages' valid
-tokens per step divided by the step time (inputs resident in HBM, L2 flushed
-before every timed step by writing a 256 MiB buffer and reading another
-outside the timed events).  The line also carries calls/s, the decode
-kernel's roofline fraction against the measured HBM copy bandwidth (with two
-references beside it: a library copy of the same bytes in one launch, and
-the event-timed cost of launching a one-element kernel), an end-to-end number
-through the same API with the per-step inputs (q, page table, seq_lens)
-copied from pinned host memory and the outputs (O, LSE) copied back inside
-the timed region (each side packed into one buffer: one copy each way), and
-the float64 oracle timed on a bounded sample on the host cores.
+Timing.  Steps run back to back, each on its own layer's cache: four layers
+with distinct caches, cycled, so a step's inputs (64 MiB of summaries + 64 MiB
+of selected K/V) are not in L2 from the step before (the L2 holds 126 MB; a
+cache comes back every fourth step).  Every step is one CUDA-graph replay;
+CUDA events bracket exactly K steps on the launching stream, with a barrier and
+a synchronize on both sides.  The decode kernel's roofline takes its average
+launch duration from K back-to-back launches over the same rotating caches, and
+counts the method's bytes only: the selected pages' valid K+V, q, the final O
+and LSE, the lists and the page-table entries they resolve (not the split
+partials, which are the kernel's choice).  Beside it: the same kernel launched
+alone after an L2 flush, and the event-timed cost of a one-element launch.
 
-With --gpus N (torchrun), every rank runs its own batch of the same shape
-(replicas: the path has no exchange step); time is the max over ranks.
+The default run (--workload all, one GPU) adds the other four workloads in a
+`workloads` object of the same line: the Llama-70B-shaped long decode (32
+sequences of 64K-128K tokens; 256 MiB selected per step, one 12 GiB cache),
+the FP8-page variant of the headline, the MLA + MTP tiered decode timed as a
+CUDA graph of 61 back-to-back layer calls over 61 distinct latent caches (as a
+61-layer model runs them), and the block-union chunked prefill.  Each has its
+own value, step time, calls/s, roofline (HBM bytes or tensor FLOPs against the
+measured peaks) and end-to-end figure.
+
+End to end (`e2e`): the same steps through the public API with the step's
+inputs (q, page table, sequence lengths) copied from pinned host memory and its
+outputs (O, LSE) copied back inside the timed region, each side packed into one
+buffer (one copy each way), the step itself one C call.
+
+`cpu_baseline` (rank 0, one GPU): the float64 oracle, as it stands, on a
+bounded sample of (sequence, kv head) units of the headline workload, timed on
+the host cores (all of them, and one BLAS thread).  `--impl reference` times
+the same oracle as this build's reference arm (there is no reference code to
+run: the method comes from web pages) on the same workload and config.
+
+With --gpus N (torchrun), every rank runs its own replica of the headline
+workload (the path has no exchange step); time is the max over ranks.
 """
 from __future__ import annotations
 
@@ -33,29 +55,33 @@ import math
 import os
 import subprocess
 import sys
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "selected-KV GB/s (fraction of HBM peak) and sparse-attn calls/sec at 1 B200"
-FALLBACK_HBM_GBS = 6650.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GQA_LAYERS = 4          # distinct caches cycled by the Llama-8B-shaped steps
+MLA_LAYERS = 61         # one latent cache per layer of a 61-layer model
+L2_NOTE = ("inputs larger than L2: steps back to back, each on its own layer's cache "
+           "({n} distinct caches cycled; one step touches {mb:.0f} MB, L2 is 126 MB)")
 
 
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = heuristic)")
+    ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
-    ap.add_argument("--workload", choices=["llama8b", "llama70b", "mla", "prefill", "llama8b_fp8"],
-                    default="llama8b",
-                    help="llama8b (default, the headline workload); the others print the same "
-                         "line for the Llama-70B long decode, MLA+MTP tiered decode and "
-                         "block-union prefill workloads")
+    ap.add_argument("--workload", default="all",
+                    choices=["all", "llama8b", "llama70b", "mla", "prefill", "llama8b_fp8"],
+                    help="all (default): the Llama-8B headline line with every other workload "
+                         "in its `workloads` object; otherwise one workload's line alone")
     return ap.parse_args()
 
 
@@ -64,156 +90,99 @@ def peaks():
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return FALLBACK_HBM_GBS, "fallback"
+        return {k: float(d[k]) for k in FALLBACK}, "measured"
+    return dict(FALLBACK), "fallback"
 
 
+# ---------------------------------------------------------------------------
+# clocks: nvidia-smi sampled in the background for the whole run
+# ---------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi clock / throttle samples while the timed region runs."""
+    """nvidia-smi clock / throttle samples every 50 ms from before the first
+    warm-up to after the last timed region; `windows` marks the GPU-busy spans
+    (warm-up, graph capture, timed regions) whose samples the summary keeps."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
+        self.samples = []          # (host time, line)
+        self.windows = []
         self.proc = None
 
-    def __enter__(self):
+    def start(self, wait_s: float = 5.0):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
         except Exception:
             self.proc = None
+            return self
+        threading.Thread(target=self._read, daemon=True).start()
+        t0 = time.time()
+        while not self.samples and time.time() - t0 < wait_s:   # first sample in
+            time.sleep(0.01)
         return self
 
-    def __exit__(self, *exc):
-        self.lines = []
+    def _read(self):
+        for line in self.proc.stdout:
+            if line.strip():
+                self.samples.append((time.time(), line))
+
+    def busy(self):
+        """Context manager marking a GPU-busy span."""
+        sampler = self
+
+        class _W:
+            def __enter__(self):
+                self.t0 = time.time()
+
+            def __exit__(self, *exc):
+                sampler.windows.append((self.t0, time.time()))
+        return _W()
+
+    def stop(self):
         if self.proc is not None:
+            time.sleep(0.06)
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except Exception:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [l for l in out.splitlines() if l.strip()]
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for l in getattr(self, "lines", []):
+        sm, mx, reasons, n_all = [], None, set(), 0
+        for t, l in self.samples:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 7:
+                continue
+            n_all += 1
+            if not any(a - 0.06 <= t <= b + 0.06 for a, b in self.windows):
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                sm.append(float(f[0]))
+                mx = float(f[1])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, f[3:7]):
                 if v.lower().startswith("active"):
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
-        sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
-                "samples": len(sm)}
+        out = {"sm_mhz": None, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+               "samples_whole_run": n_all,
+               "window": "warm-up, graph capture and timed regions of every workload"}
+        if sm:
+            sm.sort()
+            out["sm_mhz"] = sm[len(sm) // 2]
+        return out
 
 
-def selected_kv_bytes(counts, pages, seq_lens, P, D, elem_bytes=2):
-    """K+V bytes of the valid tokens of every selected page (per step); FP8 pages
-    (elem_bytes 1) add their two float32 scales per selected (page, kv head)."""
-    import torch
-    B, Hkv, cap = pages.shape
-    L = seq_lens.to(torch.int64).view(B, 1, 1)
-    idx = torch.arange(cap, device=pages.device).view(1, 1, cap)
-    valid = idx < counts.view(B, Hkv, 1)
-    p = pages.to(torch.int64).clamp_min(0)
-    toks = (L - p * P).clamp(0, P)
-    toks = torch.where(valid, toks, torch.zeros_like(toks))
-    scales = int(valid.sum().item()) * 8 if elem_bytes == 1 else 0
-    return int(toks.sum().item()) * D * elem_bytes * 2 + scales
-
-
-def cpu_baseline(cfg, inp, sig_bits, n_units: int, budget_s: float = 20.0, f8=None,
-                 min_s: float = 0.0):
-    """Oracle (float64, host cores) on a bounded sample: n_units (b, kv head)
-    pairs, select + attention (over FP8 pages when f8 holds their codes and
-    scales), in repeated passes until min_s seconds have elapsed (and never
-    past budget_s).  Returns GB/s of selected KV, units done, seconds."""
-    import numpy as np
-
-    import oracle as O
-    from paged_sparse_kv_sa_b200 import workloads as W
-
-    pt = inp["page_table"].cpu().numpy()
-    sl = inp["seq_lens"].cpu().numpy()
-    qb = W.bf16_bits(inp["q"])
-    units = [(b, h) for b in range(cfg.B) for h in range(cfg.Hkv)][:n_units]
-    G = cfg.G
-    t0 = time.perf_counter()
-    done, kv_bytes = 0, 0
-    import itertools
-    for (b, h) in itertools.cycle(units):   # (ends by the checks at the bottom)
-        pages_np, counts_np = O.select_pages(qb, sig_bits, pt, sl, cfg.page_size, cfg.sink_tokens,
-                                             cfg.local_tokens, cfg.budget_tokens, units=[(b, h)])
-        lst = pages_np[b, h, :counts_np[b, h]]
-        phys = pt[b, lst]
-        # gather only this unit's pages from the device pool
-        import torch
-        loc_pt = np.full_like(pt, -1)
-        loc_pt[b, lst] = np.arange(len(lst))
-        lists = np.full((cfg.B, cfg.Hkv, pages_np.shape[2]), -1, dtype=np.int32)
-        counts = np.zeros((cfg.B, cfg.Hkv), dtype=np.int32)
-        lists[b, h, :len(lst)] = lst
-        counts[b, h] = len(lst)
-        rows = [(b, 0, hh) for hh in range(h * G, (h + 1) * G)]
-        # gather only this unit's pages from the device pool
-        ix = torch.as_tensor(phys, device=inp["q"].device)
-        if f8 is None:
-            O.sparse_attention(qb, W.bf16_bits(inp["k"][ix]), W.bf16_bits(inp["v"][ix]), loc_pt,
-                               sl, lists, counts, np.arange(cfg.Hq) // G, 1.0 / math.sqrt(cfg.D),
-                               cfg.page_size, rows=rows)
-        else:
-            O.sparse_attention_fp8(qb, f8["kc"][ix].cpu().numpy(), f8["ks"][ix].cpu().numpy(),
-                                   f8["vc"][ix].cpu().numpy(), f8["vs"][ix].cpu().numpy(), loc_pt,
-                                   sl, lists, counts, np.arange(cfg.Hq) // G,
-                                   1.0 / math.sqrt(cfg.D), cfg.page_size, rows=rows)
-        L = int(sl[b])
-        eb = 2 if f8 is None else 1
-        kv_bytes += sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst) * cfg.D * 2 * eb
-        done += 1
-        el = time.perf_counter() - t0
-        if el > budget_s or (done % len(units) == 0 and el >= min_s):
-            break
-    dt = time.perf_counter() - t0
-    return kv_bytes / dt / 1e9, done, dt
-
-
-def _timed_graphs(g_step, g_kernel, K, flush_l2, stream, local):
-    """Replay a whole-step graph and a single-kernel graph K times each, L2 flushed
-    before every replay outside the events; device seconds for each, and clocks."""
-    import torch
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(K):
-            flush_l2(i)
-            ev[i][0].record(stream)
-            g_step.replay()
-            ev[i][1].record(stream)
-            flush_l2(i + 1)
-            ev[i][2].record(stream)
-            g_kernel.replay()
-            ev[i][3].record(stream)
-        torch.cuda.synchronize()
-    t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_kern = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3
-    return t_step, t_kern, clk.summary()
-
-
+# ---------------------------------------------------------------------------
+# shared helpers
+# ---------------------------------------------------------------------------
 def max_over_ranks(x: float, world: int, dev) -> float:
     """The largest of every rank's x: a multi-GPU job takes as long as its slowest
     rank (replicas: each rank runs its own batch; no data-path collective)."""
@@ -243,146 +212,516 @@ def _packed(like, device):
     return buf, views
 
 
-def _launch_floor(flush_l2, stream, n):
-    """Event-timed seconds of one graph-replayed launch of a one-element kernel, L2
-    flushed first: the fixed cost inside every kernel time measured here (launch,
-    first wave, drain, timestamp granularity)."""
+class Flusher:
+    """Evicts L2 before an isolated launch: writes a 256 MiB buffer, then reads
+    another 256 MiB so the dirty lines are written back before the launch."""
+
+    def __init__(self, dev):
+        import torch
+        self.w = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device=dev)
+        self.sink = torch.empty((), dtype=torch.int64, device=dev)
+
+    def __call__(self, i):
+        import torch
+        self.w.fill_(i & 0xFF)
+        torch.sum(self.r, dim=0, dtype=torch.int64, out=self.sink)
+
+
+def capture(fn):
     import torch
-    x = torch.zeros(1, device=torch.device("cuda", torch.cuda.current_device()))
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
-        x.add_(1.0)
-    for _ in range(3):
-        g.replay()
+        fn()
+    return g
+
+
+def time_back_to_back(graphs, K, stream, world, dev):
+    """Device seconds of K back-to-back graph replays cycling `graphs` (events at
+    both ends, barrier + synchronize on both sides), max over ranks."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for i in range(K):
+        graphs[i % len(graphs)].replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    return max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+
+
+def time_isolated(graph, n, flush, stream):
+    """Mean device seconds of one replay of `graph` with L2 flushed before each."""
+    import torch
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
     for i in range(n):
-        flush_l2(i)
+        flush(i)
         ev[i][0].record(stream)
-        g.replay()
+        graph.replay()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     return sum(a.elapsed_time(b) for a, b in ev) / 1e3 / n
 
 
-LAUNCH_FLOOR_WHAT = ("event-timed graph replay of a one-element kernel, L2 flushed: the fixed "
-                     "cost inside every single-launch kernel time")
+E2E_WHAT = ("every step: its inputs host->device from pinned memory (one packed copy), the "
+            "step, its outputs device->host into pinned memory (one packed copy); copies on "
+            "their own streams, so the upload of the next step and the download of the last "
+            "overlap this step (a buffer is rewritten only after its last reader is done); "
+            "device time from the first upload to the last download")
 
 
-def _peak_tflops():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
-    return 1590.0, "fallback"
+def time_e2e(items, K, stream, world, dev):
+    """Device seconds of K end-to-end steps cycling `items` (each with h_in / d_in
+    packed inputs, `call` launching the step on `stream`, d_out / h_out packed
+    outputs), pipelined over an upload and a download stream; max over ranks."""
+    import torch
+    up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    n = len(items)
+    ev_in = [torch.cuda.Event() for _ in range(n)]
+    ev_done = [torch.cuda.Event() for _ in range(n)]
+    ev_out = [torch.cuda.Event() for _ in range(n)]
+    used = [False] * n
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    up.wait_event(e0)
+    down.wait_event(e0)
+    for k in range(K):
+        i = k % n
+        it = items[i]
+        if used[i]:
+            up.wait_event(ev_done[i])          # the last step reading d_in is done
+            stream.wait_event(ev_out[i])       # d_out of its last use is downloaded
+        with torch.cuda.stream(up):
+            it["d_in"].copy_(it["h_in"], non_blocking=True)
+        ev_in[i].record(up)
+        stream.wait_event(ev_in[i])
+        it["call"]()
+        ev_done[i].record(stream)
+        down.wait_event(ev_done[i])
+        with torch.cuda.stream(down):
+            it["h_out"].copy_(it["d_out"], non_blocking=True)
+        ev_out[i].record(down)
+        used[i] = True
+    for i in range(n):
+        if used[i]:
+            stream.wait_event(ev_out[i])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    t = max_over_ranks(e0.elapsed_time(e1) / 1e3, world, dev)
+    if world > 1:
+        dist.barrier()
+    return t
 
 
-def run_extra(args, dev, world, rank, local, cores):
-    """MLA+MTP tiered decode or block-union chunked prefill: same timing protocol."""
+def launch_floor(flush, stream, dev, n=50):
+    """Event-timed seconds of one flushed replay of a one-element kernel."""
+    import torch
+    x = torch.zeros(1, device=dev)
+    g = capture(lambda: x.add_(1.0))
+    for _ in range(3):
+        g.replay()
+    return time_isolated(g, n, flush, stream)
+
+
+def selected_kv_bytes(counts, pages, seq_lens, P, D, elem_bytes=2):
+    """K+V bytes of the valid tokens of every selected page; FP8 pages (elem_bytes
+    1) add their two float32 scales per selected (page, kv head)."""
+    import torch
+    B, Hkv, cap = pages.shape
+    L = seq_lens.to(torch.int64).view(B, 1, 1)
+    idx = torch.arange(cap, device=pages.device).view(1, 1, cap)
+    valid = idx < counts.view(B, Hkv, 1)
+    p = pages.to(torch.int64).clamp_min(0)
+    toks = (L - p * P).clamp(0, P)
+    toks = torch.where(valid, toks, torch.zeros_like(toks))
+    scales = int(valid.sum().item()) * 8 if elem_bytes == 1 else 0
+    return int(toks.sum().item()) * D * elem_bytes * 2 + scales
+
+
+def gqa_config(cfg, n_splits, world, fp8=False, n_layers=GQA_LAYERS):
+    """The `config` of a GQA decode line (both arms print the same one).  The
+    bytes a step touches are the nominal ones of the workload (mean sequence
+    length): the summaries it scores and the selected pages' K/V."""
+    mean_pages = -(-((cfg.seq_len_lo + cfg.seq_len_hi) // 2) // cfg.page_size)
+    budget_pages = cfg.budget_tokens // cfg.page_size
+    elem = 1 if fp8 else 2
+    step_mb = cfg.B * cfg.Hkv * (mean_pages * cfg.D * 2 +
+                                 budget_pages * cfg.page_size * cfg.D * elem * 2) / 1e6
+    c = {"workload": cfg.name + ("_fp8" if fp8 else ""), "B": cfg.B,
+         "seq_len": (cfg.seq_len_lo if cfg.seq_len_lo == cfg.seq_len_hi
+                     else f"U[{cfg.seq_len_lo},{cfg.seq_len_hi}]"),
+         "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
+         "kv_pages": "fp8 e4m3 + float32 scale per (page, kv head)" if fp8 else "bf16",
+         "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
+         "local_tokens": cfg.local_tokens, "n_splits": n_splits, "layer_caches": n_layers,
+         "parallelism": f"replicas x{world}",
+         "l2": L2_NOTE.format(n=n_layers, mb=step_mb)}
+    return c
+
+
+def gqa_splits(cfg, args):
+    from paged_sparse_kv_sa_b200.pipeline import default_splits
+    budget_pages = cfg.budget_tokens // cfg.page_size
+    return args.splits or default_splits(cfg.B * cfg.Hkv, budget_pages)
+
+
+# ---------------------------------------------------------------------------
+# GQA decode workloads (Llama-8B, its FP8 pages, Llama-70B)
+# ---------------------------------------------------------------------------
+def run_gqa(cfg, args, dev, world, rank, clk, K, fp8=False, n_layers=GQA_LAYERS):
+    import torch
+
+    import paged_sparse_kv_sa_b200 as sa
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    sa.load()
+    stream = torch.cuda.current_stream(dev)
+    n_splits = gqa_splits(cfg, args)
+    layers = []
+    for l in range(n_layers):
+        inp = W.gqa_decode_inputs(cfg, seed=args.seed + 1000 * rank + l, device=dev)
+        if fp8:
+            kc, ks = W.fp8_pages(inp.pop("k"))
+            vc, vs = W.fp8_pages(inp.pop("v"))
+            inp.update(kc=kc, ks=ks, vc=vc, vs=vs)
+            sig = sa.sa_build_page_summaries_fp8(kc, ks, inp["page_table"], inp["seq_lens"])
+        else:
+            sig = sa.sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
+        step = sa.SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size,
+                                   inp["page_table"].shape[1], cfg.sink_tokens, cfg.local_tokens,
+                                   cfg.budget_tokens, n_splits=n_splits, device=dev)
+        torch.cuda.synchronize()
+        layers.append(dict(inp=inp, sig=sig, step=step))
+
+    def step_fn(L):
+        i, s = L["inp"], L["step"]
+        if fp8:
+            s.select(i["q"], L["sig"], i["page_table"], i["seq_lens"])
+            s.attend_fp8(i["q"], i["kc"], i["vc"], i["ks"], i["vs"], i["page_table"],
+                         i["seq_lens"])
+        else:
+            s.run(i["q"], i["k"], i["v"], L["sig"], i["page_table"], i["seq_lens"])
+
+    def decode_fn(L):
+        i, s = L["inp"], L["step"]
+        if fp8:
+            s.decode_fp8(i["q"], i["kc"], i["vc"], i["ks"], i["vs"], i["page_table"],
+                         i["seq_lens"])
+        else:
+            s.decode(i["q"], i["k"], i["v"], i["page_table"], i["seq_lens"])
+
+    with clk.busy():
+        for L in layers:
+            L["step"].dev_error.zero_()
+            for _ in range(max(args.warmup, 3)):
+                step_fn(L)
+        torch.cuda.synchronize()
+        # algorithmic bytes of each layer's step (from the selection it made)
+        for L in layers:
+            s, i = L["step"], L["inp"]
+            L["kv"] = selected_kv_bytes(s.counts, s.pages, i["seq_lens"], cfg.page_size, cfg.D,
+                                        elem_bytes=1 if fp8 else 2)
+            L["alg"] = (L["kv"] + i["q"].numel() * 2 + s.o.numel() * 4 + s.lse.numel() * 4 +
+                        s.pages.numel() * 4 + s.counts.numel() * 4 +
+                        int(s.counts.sum().item()) * 4)
+            L["g_step"] = capture(lambda L=L: step_fn(L))
+            L["g_dec"] = capture(lambda L=L: decode_fn(L))
+        for L in layers:
+            for _ in range(3):
+                L["g_step"].replay()
+                L["g_dec"].replay()
+        torch.cuda.synchronize()
+        t_step = time_back_to_back([L["g_step"] for L in layers], K, stream, world, dev)
+        t_dec = time_back_to_back([L["g_dec"] for L in layers], K, stream, world, dev)
+    kv_total = sum(layers[i % n_layers]["kv"] for i in range(K))
+    alg_total = sum(layers[i % n_layers]["alg"] for i in range(K))
+    for L in layers:
+        assert int(L["step"].dev_error.item()) == 0, "device error flag set"
+        assert torch.isfinite(L["step"].o).all().item(), "non-finite output"
+
+    # the decode kernel alone after an L2 flush, and the cost of a launch itself
+    flush = Flusher(dev)
+    with clk.busy():
+        n_iso = min(K, 50)
+        t_iso = time_isolated(layers[0]["g_dec"], n_iso, flush, stream)
+        t_floor = launch_floor(flush, stream, dev)
+    del flush
+
+    # end to end through the public API: the step's inputs from pinned host memory
+    # (packed: one copy), the step's C calls (marshalled once: sa.bind), its
+    # outputs back (packed: one copy); at least two buffer sets alternate
+    items = []
+    for idx in range(max(2, n_layers)):
+        L = layers[idx % n_layers]
+        i = L["inp"]
+        s = L["step"] if idx < n_layers else sa.SparseDecodeStep(
+            cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, i["page_table"].shape[1],
+            cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens, n_splits=n_splits, device=dev)
+        srcs = (i["q"], i["page_table"], i["seq_lens"])
+        h_in, hv = _packed(srcs, "cpu")
+        for h_, x in zip(hv, srcs):
+            h_.copy_(x.cpu())
+        d_in, (q_d, pt_d, sl_d) = _packed(srcs, dev)
+        d_out, (s.o, s.lse) = _packed((s.o, s.lse), dev)   # the step writes these views
+        h_out, _ = _packed((s.o, s.lse), "cpu")
+        if fp8:
+            call = sa.bind(lambda s=s, L=L, q_d=q_d, pt_d=pt_d, sl_d=sl_d: (
+                s.select(q_d, L["sig"], pt_d, sl_d),
+                s.attend_fp8(q_d, L["inp"]["kc"], L["inp"]["vc"], L["inp"]["ks"],
+                             L["inp"]["vs"], pt_d, sl_d)))
+        else:
+            call = s.bind(q_d, i["k"], i["v"], L["sig"], pt_d, sl_d)
+        items.append(dict(h_in=h_in, d_in=d_in, d_out=d_out, h_out=h_out, call=call))
+
+    with clk.busy():
+        time_e2e(items, max(args.warmup, 3) * len(items), stream, 1, dev)
+        t_e2e = time_e2e(items, K, stream, world, dev)
+    h2d = items[0]["h_in"].numel()
+    d2h = items[0]["h_out"].numel()
+    del items
+
+    pk, peak_kind = peaks()
+    hbm = pk["hbm_gbs"]
+    dec_us = t_dec / K * 1e6
+    achieved = alg_total / t_dec / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tp) and not fp8:
+        with open(tp) as f:
+            td = json.load(f)
+        src = os.path.join(ROOT, "paged_sparse_kv_sa_b200", "csrc", "decode.cu")
+        import hashlib
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if (td.get("workload") == cfg.name and td.get("splits") == n_splits
+                and td.get("decode_cu_sha16") == sha):
+            traffic = td.get("bytes_per_launch")
+    kern = "decode_gqa_kernel" + ("<fp8>" if fp8 else "")
+    return {
+        "metric": METRIC, "value": round(world * kv_total / t_step / 1e9, 3), "unit": "GB/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * t_step / K, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": gqa_config(cfg, n_splits, world, fp8, n_layers),
+        "calls_per_sec": round(world * K / t_step, 2),
+        "selected_kv_bytes_per_step": kv_total // K,
+        "roofline": {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 2),
+                     "peak": hbm, "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                     "peak_kind": f"{peak_kind} (copy bandwidth)", "traffic": traffic,
+                     "alg_bytes_per_launch": alg_total // K,
+                     "alg_bytes_what": "selected valid K+V + q + final O and LSE (float32) + "
+                                       "list entries + page-table entries",
+                     "kernel_us": round(dec_us, 2),
+                     "kernel_us_what": f"average launch duration over {K} back-to-back "
+                                       f"launches cycling {n_layers} layer caches",
+                     "isolated_us": round(1e6 * t_iso, 2),
+                     "isolated_frac": round(alg_total / K / t_iso / 1e9 / hbm, 4),
+                     "isolated_what": "one launch after an L2 flush, event-timed",
+                     "launch_floor_us": round(1e6 * t_floor, 2),
+                     "launch_floor_what": "one flushed, event-timed launch of a one-element "
+                                          "kernel"},
+        "e2e": {"value": round(world * kv_total / t_e2e / 1e9, 3), "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(1e3 * t_e2e / K, 4),
+                "what": E2E_WHAT + ("; the step: select and attend, two C calls" if fp8
+                                    else "; the step: one C call (sa_sparse_step)")},
+        "gpu_launches": 4 * K,
+        "_layers": layers,
+    }
+
+
+# ---------------------------------------------------------------------------
+# MLA + MTP tiered decode: a graph of 61 layer calls over distinct caches
+# ---------------------------------------------------------------------------
+def run_mla(args, dev, world, rank, clk, reps):
     import numpy as np
     import torch
 
     import paged_sparse_kv_sa_b200 as sa
     from paged_sparse_kv_sa_b200 import workloads as W
 
-    if args.impl == "reference":
-        print(json.dumps({"impl": "reference", "unavailable":
-                          "the oracle arm is timed on the default (Llama-8B decode) workload"}))
-        return
-    sa.load()
+    lib = sa.load()
+    cfg = W.MLA_MTP
     stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
-
-    def flush_l2(i):
-        flush.fill_(i & 0xFF)
-        torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
-
-    K = args.steps
-    if args.workload == "mla":
-        cfg = W.MLA_MTP
-        inp = W.mla_decode_inputs(cfg, seed=args.seed + rank, device=dev)
-        q, kv, pt, sl = inp["q"], inp["kv"], inp["page_table"], inp["seq_lens"]
-        sig = sa.sa_build_page_summaries(kv, pt, sl)
+    n_splits = args.splits or 8
+    cap = cfg.alpha + cfg.beta
+    scale = 1.0 / math.sqrt(cfg.Dk)
+    o = torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
+    lse = torch.empty((cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
+    o_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
+    l_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
+    aws = sa.attention_workspace(cfg.B, cfg.T, cfg.Hq, cfg.Dv, n_splits, dev)
+    layers = []
+    for l in range(MLA_LAYERS):
+        inp = W.mla_decode_inputs(cfg, seed=args.seed + 1000 * rank + l, device=dev)
+        sig = sa.sa_build_page_summaries(inp["kv"], inp["page_table"], inp["seq_lens"])
         amb = set(int(h) for h in inp["ambient_heads"].tolist())
-        h2l = [1 if h in amb else 0 for h in range(cfg.Hq)]
-        cap = cfg.alpha + cfg.beta
-        lists = torch.empty((cfg.B, 2, cap), dtype=torch.int32, device=dev)
-        counts = torch.empty((cfg.B, 2), dtype=torch.int32, device=dev)
-        ws = torch.empty(max(int(sa.load().sa_select_tiered_workspace_size(
-            cfg.B, cfg.T, cfg.Hq, pt.shape[1])), 16), dtype=torch.uint8, device=dev)
-        n_splits = args.splits or 8
-        o_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
-        l_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
-        o = torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
-        lse = torch.empty((cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
-        scale = 1.0 / math.sqrt(cfg.Dk)
-
-        def select(qq, ptt, sll):
-            sa.sa_select_pages_tiered(qq, sig, ptt, sll, cfg.page_size, cfg.alpha, cfg.beta,
-                                      lists=lists, list_counts=counts, workspace=ws)
-
-        def decode(qq, ptt, sll):
-            sa.sa_sparse_decode(qq, kv, kv[..., :cfg.Dv], ptt, sll, lists, counts, h2l, scale,
-                                n_splits, o_partial=o_p, lse_partial=l_p)
-
-        step_inputs = (q, pt, sl)
-        kern = "mla_kernel"
-    else:
-        cfg = W.UNION_PREFILL
-        inp = W.prefill_inputs(cfg, seed=args.seed + rank, device=dev)
-        q, kk, vv, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
-        scores = W.block_union_scores(cfg, seed=args.seed + rank, device=dev)
-        off = cfg.q_offset // cfg.block
-        tables = torch.empty((cfg.Hkv, cfg.n_kv_blocks), dtype=torch.int32, device=dev)
-        tcounts = torch.empty((cfg.Hkv,), dtype=torch.int32, device=dev)
-        h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)]
-        n_splits = args.splits or 2
-        o_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
-        l_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
-        o = torch.empty((1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
-        lse = torch.empty((1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
-        scale = 1.0 / math.sqrt(cfg.D)
-
-        def select(sc, ptt, sll):
-            sa.sa_block_union(sc, cfg.Hkv, off, cfg.top_k, cfg.n_sink_blocks, tables=tables,
-                              counts=tcounts)
-
-        def decode(qq, ptt, sll):
-            sa.sa_sparse_decode(qq, kk, vv, ptt, sll, tables.view(1, cfg.Hkv, -1),
-                                tcounts.view(1, cfg.Hkv), h2l, scale, n_splits,
-                                o_partial=o_p, lse_partial=l_p)
-
-        step_inputs = (scores, pt, sl)
-        kern = "prefill_kernel"
-
-    def run_step(a0, ptt, sll, qq):
-        select(a0, ptt, sll)
-        decode(qq, ptt, sll)
-        sa.sa_combine(o_p, l_p, o_out=o, lse_out=lse)
-
-    first = step_inputs[0]
-    for _ in range(max(args.warmup, 3)):
-        run_step(first, pt, sl, q)
+        ws = torch.empty(max(int(lib.sa_select_tiered_workspace_size(
+            cfg.B, cfg.T, cfg.Hq, inp["page_table"].shape[1])), 16), dtype=torch.uint8, device=dev)
+        layers.append(dict(inp=inp, sig=sig, ws=ws, h2l=[1 if h in amb else 0 for h in range(cfg.Hq)],
+                           lists=torch.empty((cfg.B, 2, cap), dtype=torch.int32, device=dev),
+                           counts=torch.empty((cfg.B, 2), dtype=torch.int32, device=dev)))
     torch.cuda.synchronize()
 
-    # algorithmic work of one step (from the lists the step produced)
-    if args.workload == "mla":
-        L = sl.cpu().numpy()
-        ls, cs = lists.cpu().numpy(), counts.cpu().numpy()
+    def select(L, q, pt, sl):
+        sa.sa_select_pages_tiered(q, L["sig"], pt, sl, cfg.page_size, cfg.alpha, cfg.beta,
+                                  lists=L["lists"], list_counts=L["counts"], workspace=L["ws"])
+
+    def attend(L, q, pt, sl, oo, ll):
+        kv = L["inp"]["kv"]
+        sa.sa_sparse_attention(q, kv, kv[..., :cfg.Dv], pt, sl, L["lists"], L["counts"], L["h2l"],
+                               scale, n_splits, o_out=oo, lse_out=ll, workspace=aws)
+
+    def step(L):
+        i = L["inp"]
+        select(L, i["q"], i["page_table"], i["seq_lens"])
+        attend(L, i["q"], i["page_table"], i["seq_lens"], o, lse)
+
+    def decode(L):
+        i = L["inp"]
+        kv = i["kv"]
+        sa.sa_sparse_decode(i["q"], kv, kv[..., :cfg.Dv], i["page_table"], i["seq_lens"],
+                            L["lists"], L["counts"], L["h2l"], scale, n_splits, o_partial=o_p,
+                            lse_partial=l_p)
+
+    with clk.busy():
+        for _ in range(max(args.warmup, 3)):
+            for L in layers:
+                step(L)
+        torch.cuda.synchronize()
         flops, kv_bytes = 0, 0
-        for b in range(cfg.B):
-            for t in range(cfg.T):
-                qpos = int(L[b]) - cfg.T + t
-                for li, nh in ((0, cfg.Hq - len(amb)), (1, len(amb))):
-                    pg = ls[b, li, :cs[b, li]].astype(np.int64)
-                    keys = np.clip(np.minimum(qpos + 1, int(L[b])) - pg * cfg.page_size, 0,
-                                   cfg.page_size).sum()
-                    flops += 2 * nh * int(keys) * (cfg.Dk + cfg.Dv)
-            pg = ls[b, 1, :cs[b, 1]].astype(np.int64)
-            kv_bytes += int(np.clip(int(L[b]) - pg * cfg.page_size, 0, cfg.page_size).sum()) \
-                * cfg.Dk * 2
-    else:
+        for L in layers:
+            Ls = L["inp"]["seq_lens"].cpu().numpy()
+            ls, cs = L["lists"].cpu().numpy(), L["counts"].cpu().numpy()
+            amb_n = sum(L["h2l"])
+            for b in range(cfg.B):
+                for t in range(cfg.T):
+                    qpos = int(Ls[b]) - cfg.T + t
+                    for li, nh in ((0, cfg.Hq - amb_n), (1, amb_n)):
+                        pg = ls[b, li, :cs[b, li]].astype(np.int64)
+                        keys = np.clip(np.minimum(qpos + 1, int(Ls[b])) - pg * cfg.page_size, 0,
+                                       cfg.page_size).sum()
+                        flops += 2 * nh * int(keys) * (cfg.Dk + cfg.Dv)
+                pg = ls[b, 1, :cs[b, 1]].astype(np.int64)
+                kv_bytes += int(np.clip(int(Ls[b]) - pg * cfg.page_size, 0,
+                                        cfg.page_size).sum()) * cfg.Dk * 2
+        g_step = capture(lambda: [step(L) for L in layers])
+        g_dec = capture(lambda: [decode(L) for L in layers])
+        for _ in range(2):
+            g_step.replay()
+            g_dec.replay()
+        torch.cuda.synchronize()
+        t_step = time_back_to_back([g_step], reps, stream, world, dev)
+        t_dec = time_back_to_back([g_dec], reps, stream, world, dev)
+    n = reps * MLA_LAYERS
+    assert torch.isfinite(o).all().item(), "non-finite output"
+
+    # end to end through the public API over the first eight layers' caches (cycled):
+    # a step's inputs from the host, select + attend, its outputs back
+    items = []
+    for L in layers[:8]:
+        i0 = L["inp"]
+        srcs = (i0["q"], i0["page_table"], i0["seq_lens"])
+        h_in, hv = _packed(srcs, "cpu")
+        for h_, x in zip(hv, srcs):
+            h_.copy_(x.cpu())
+        d_in, (q_d, pt_d, sl_d) = _packed(srcs, dev)
+        d_out, (o_d, lse_d) = _packed((o, lse), dev)
+        h_out, _ = _packed((o, lse), "cpu")
+
+        call = sa.bind(lambda L=L, q_d=q_d, pt_d=pt_d, sl_d=sl_d, o_d=o_d, lse_d=lse_d: (
+            select(L, q_d, pt_d, sl_d), attend(L, q_d, pt_d, sl_d, o_d, lse_d)))
+        items.append(dict(h_in=h_in, d_in=d_in, d_out=d_out, h_out=h_out, call=call))
+    K = max(args.steps, 20)
+    with clk.busy():
+        time_e2e(items, 3 * len(items), stream, 1, dev)
+        t_e2e = time_e2e(items, K, stream, world, dev)
+    h_in, h_out = items[0]["h_in"], items[0]["h_out"]
+    pk, kind = peaks()
+    per_call_flops = flops / MLA_LAYERS
+    per_call_bytes = kv_bytes / MLA_LAYERS
+    achieved = per_call_flops / (t_dec / n) / 1e12
+    return {
+        "value": round(world * kv_bytes * reps / t_step / 1e9, 3), "unit": "GB/s",
+        "steps": n, "ms_per_step": round(1e3 * t_step / n, 4),
+        "calls_per_sec": round(world * n / t_step, 2),
+        "config": {"workload": cfg.name, "n_splits": n_splits, "layer_caches": MLA_LAYERS,
+                   "timing": f"CUDA graph of {MLA_LAYERS} back-to-back layer calls over "
+                             f"{MLA_LAYERS} distinct latent caches, replayed {reps} times",
+                   "l2": "inputs larger than L2 (61 x 604 MB of caches cycled)"},
+        "selected_kv_bytes_per_step": int(per_call_bytes), "flops_per_step": int(per_call_flops),
+        "step_tflops": round(world * flops * reps / t_step / 1e12, 2),
+        "roofline": {"kernel": "mla_kernel", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops_sustained"], 4),
+                     "peak_kind": f"{kind} bf16 GEMM, sustained (a long loop of launches)",
+                     "traffic": None,
+                     "kernel_us": round(1e6 * t_dec / n, 2),
+                     "kernel_us_what": f"average launch in a graph of {MLA_LAYERS} "
+                                       "back-to-back decode launches",
+                     "hbm_achieved_gbs": round(per_call_bytes / (t_dec / n) / 1e9, 1),
+                     "hbm_frac": round(per_call_bytes / (t_dec / n) / 1e9 / pk["hbm_gbs"], 4)},
+        "e2e": {"value": round(world * (kv_bytes / MLA_LAYERS) * K / t_e2e / 1e9, 3),
+                "unit": "GB/s", "h2d_bytes_per_step": h_in.numel(),
+                "d2h_bytes_per_step": h_out.numel(), "ms_per_step": round(1e3 * t_e2e / K, 4),
+                "what": E2E_WHAT + "; the step: select and attend (two C calls), eight layer "
+                                   "caches cycled"},
+        "gpu_launches": 4 * n,
+    }
+
+
+# ---------------------------------------------------------------------------
+# block-union chunked prefill
+# ---------------------------------------------------------------------------
+def run_prefill(args, dev, world, rank, clk, K):
+    import numpy as np
+    import torch
+
+    import paged_sparse_kv_sa_b200 as sa
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    sa.load()
+    cfg = W.UNION_PREFILL
+    stream = torch.cuda.current_stream(dev)
+    inp = W.prefill_inputs(cfg, seed=args.seed + rank, device=dev)
+    q, kk, vv, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
+    scores = W.block_union_scores(cfg, seed=args.seed + rank, device=dev)
+    off = cfg.q_offset // cfg.block
+    tables = torch.empty((cfg.Hkv, cfg.n_kv_blocks), dtype=torch.int32, device=dev)
+    tcounts = torch.empty((cfg.Hkv,), dtype=torch.int32, device=dev)
+    h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)]
+    n_splits = args.splits or 4
+    o = torch.empty((1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
+    o_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq, cfg.D), dtype=torch.float32, device=dev)
+    l_p = torch.empty((n_splits, 1, cfg.chunk, cfg.Hq), dtype=torch.float32, device=dev)
+    aws = sa.attention_workspace(1, cfg.chunk, cfg.Hq, cfg.D, n_splits, dev)
+    scale = 1.0 / math.sqrt(cfg.D)
+
+    def step(sc, qq, ptt, sll, oo, ll):
+        sa.sa_block_union(sc, cfg.Hkv, off, cfg.top_k, cfg.n_sink_blocks, tables=tables,
+                          counts=tcounts)
+        sa.sa_sparse_attention(qq, kk, vv, ptt, sll, tables.view(1, cfg.Hkv, -1),
+                               tcounts.view(1, cfg.Hkv), h2l, scale, n_splits, o_out=oo,
+                               lse_out=ll, workspace=aws)
+
+    def decode():
+        sa.sa_sparse_decode(q, kk, vv, pt, sl, tables.view(1, cfg.Hkv, -1),
+                            tcounts.view(1, cfg.Hkv), h2l, scale, n_splits, o_partial=o_p,
+                            lse_partial=l_p)
+
+    with clk.busy():
+        for _ in range(max(args.warmup, 3)):
+            step(scores, q, pt, sl, o, lse)
+        torch.cuda.synchronize()
         tb, tc_ = tables.cpu().numpy(), tcounts.cpu().numpy()
         G = cfg.Hq // cfg.Hkv
         qpos = cfg.q_offset + np.arange(cfg.chunk)
@@ -394,376 +733,275 @@ def run_extra(args, dev, world, rank, local, cores):
             flops += 2 * G * int(vis) * (2 * cfg.D)
             kv_bytes += int(np.clip(cfg.kv_len - blk * cfg.block, 0, cfg.block).sum()) \
                 * cfg.D * 2 * 2
-
-    g_step, g_kern = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        run_step(first, pt, sl, q)
-    with torch.cuda.graph(g_kern):
-        decode(q, pt, sl)
-    for _ in range(3):
-        g_step.replay()
-        g_kern.replay()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    t_step, t_kern, clocks = _timed_graphs(g_step, g_kern, K, flush_l2, stream, local)
-    if world > 1:
-        dist.barrier()
-
-    # end to end through the same API: the step's inputs from pinned host memory
-    # (packed: one host-to-device copy) and its outputs back (packed: one copy)
-    srcs = (first, pt, sl) if first is q else (first, pt, sl, q)
-    h_in, hosts = _packed(srcs, "cpu")
-    for h_, x in zip(hosts, srcs):
-        h_.copy_(x.cpu())
-    d_in, devs = _packed(srcs, dev)
-    d_out, (o, lse) = _packed((o, lse), dev)      # the step now writes these views
-    h_out, (o_h, lse_h) = _packed((o, lse), "cpu")
-
-    def e2e():
-        d_in.copy_(h_in, non_blocking=True)
-        run_step(devs[0], devs[1], devs[2], devs[-1] if len(devs) == 4 else devs[0])
-        h_out.copy_(d_out, non_blocking=True)
-
-    for _ in range(3):
-        e2e()
-    torch.cuda.synchronize()
-    e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    for i in range(K):
-        flush_l2(i)
-        e_ev[i][0].record(stream)
-        e2e()
-        e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    t_e2e = sum(a.elapsed_time(b) for a, b in e_ev) / 1e3
-    h2d = h_in.numel()
-    d2h = h_out.numel()
+        g_step = capture(lambda: step(scores, q, pt, sl, o, lse))
+        g_dec = capture(decode)
+        for _ in range(2):
+            g_step.replay()
+            g_dec.replay()
+        torch.cuda.synchronize()
+        t_step = time_back_to_back([g_step], K, stream, world, dev)
+        t_dec = time_back_to_back([g_dec], K, stream, world, dev)
     assert torch.isfinite(o).all().item(), "non-finite output"
 
-    t_step = max_over_ranks(t_step, world, dev)
-    t_e2e = max_over_ranks(t_e2e, world, dev)
-    peak, kind = _peak_tflops()
-    achieved = flops / (t_kern / K) / 1e12
-    t_floor = _launch_floor(flush_l2, stream, min(K, 50))
-    line = {
-        "metric": METRIC, "value": round(world * kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s",
-        "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": round(1e3 * t_step / K, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+    # end to end: two input / output buffer sets alternate (double buffering)
+    srcs = (scores, pt, sl, q)
+    items = []
+    for _ in range(2):
+        h_in, hv = _packed(srcs, "cpu")
+        for h_, x in zip(hv, srcs):
+            h_.copy_(x.cpu())
+        d_in, (sc_d, pt_d, sl_d, q_d) = _packed(srcs, dev)
+        d_out, (o_d, lse_d) = _packed((o, lse), dev)
+        h_out, _ = _packed((o, lse), "cpu")
+        items.append(dict(h_in=h_in, d_in=d_in, d_out=d_out, h_out=h_out,
+                          call=sa.bind(lambda a=(sc_d, q_d, pt_d, sl_d, o_d, lse_d): step(*a))))
+    with clk.busy():
+        time_e2e(items, 2, stream, 1, dev)
+        t_e2e = time_e2e(items, K, stream, world, dev)
+    h_in, h_out = items[0]["h_in"], items[0]["h_out"]
+    pk, kind = peaks()
+    achieved = flops / (t_dec / K) / 1e12
+    return {
+        "value": round(world * kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s", "steps": K,
+        "ms_per_step": round(1e3 * t_step / K, 4), "calls_per_sec": round(world * K / t_step, 2),
         "config": {"workload": cfg.name, "n_splits": n_splits,
-                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)"},
-        "calls_per_sec": round(world * K / t_step, 2),
-        "step_tflops": round(world * flops * K / t_step / 1e12, 2),
+                   "l2": "inputs larger than L2 (529 MB K/V pool, 217 MB selected per step), "
+                         "steps back to back"},
         "selected_kv_bytes_per_step": kv_bytes, "flops_per_step": flops,
-        "roofline": {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 2),
-                     "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_kind": kind, "traffic": None,
-                     "kernel_ms": round(1e3 * t_kern / K, 4),
-                     "launch_floor_us": round(1e6 * t_floor, 2),
-                     "launch_floor_what": LAUNCH_FLOOR_WHAT},
+        "step_tflops": round(world * flops * K / t_step / 1e12, 2),
+        "roofline": {"kernel": "prefill_kernel", "bound": "tensor", "achieved": round(achieved, 2),
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(achieved / pk["bf16_tflops"], 4),
+                     "peak_kind": f"{kind} bf16 GEMM, burst", "traffic": None,
+                     "kernel_ms": round(1e3 * t_dec / K, 4),
+                     "kernel_ms_what": f"average over {K} back-to-back launches"},
         "e2e": {"value": round(world * kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(1e3 * t_e2e / K, 4)},
-        "gpu_launches": (5 if args.workload == "prefill" else 4) * K,
-        "clocks": clocks,
+                "h2d_bytes_per_step": h_in.numel(), "d2h_bytes_per_step": h_out.numel(),
+                "ms_per_step": round(1e3 * t_e2e / K, 4),
+                "what": E2E_WHAT + "; inputs: block scores, page table, lengths and queries; "
+                                   "the step: union + attend (two C calls)"},
+        "gpu_launches": 5 * K,
     }
-    if rank == 0:
-        print(json.dumps(line))
-    if world > 1:
-        del g_step, g_kern
-        dist.barrier()
-        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the float64 oracle on the host cores (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_units(cfg, inp, units, fp8):
+    """Each sampled (b, kv head) unit as a local problem the oracle can run alone
+    (its query rows, its pages, an identity page table), with its summaries
+    computed by the oracle (not part of a step) and its selected KV bytes."""
+    import numpy as np
+    import torch
+
+    import oracle as O
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    G = cfg.Hq // cfg.Hkv
+    out = []
+    for b, kvh in units:
+        L = int(inp["seq_lens"][b].item())
+        N = -(-L // cfg.page_size)
+        phys = inp["page_table"][b, :N].to(torch.int64)
+        pt = np.arange(N, dtype=np.int32).reshape(1, N)
+        sl = np.array([L], dtype=np.int32)
+        u = dict(q=W.bf16_bits(inp["q"][b:b + 1, :, kvh * G:(kvh + 1) * G]), pt=pt, sl=sl, G=G)
+        if fp8:
+            u["kc"] = inp["kc"][phys, kvh].unsqueeze(1).cpu().numpy()
+            u["vc"] = inp["vc"][phys, kvh].unsqueeze(1).cpu().numpy()
+            u["ks"] = inp["ks"][phys, kvh].unsqueeze(1).cpu().numpy()
+            u["vs"] = inp["vs"][phys, kvh].unsqueeze(1).cpu().numpy()
+            u["sig"] = O.page_summaries_fp8(u["kc"], u["ks"], pt, sl, cfg.page_size)
+        else:
+            u["k"] = W.bf16_bits(inp["k"][phys, kvh].unsqueeze(1))
+            u["v"] = W.bf16_bits(inp["v"][phys, kvh].unsqueeze(1))
+            u["sig"] = O.page_summaries(u["k"], pt, sl, cfg.page_size)
+        out.append(u)
+    return out
+
+
+def oracle_step(cfg, u, fp8):
+    """One unit of the step on the oracle: selection, then attention over it.
+    Returns the selected valid K+V bytes."""
+    import numpy as np
+
+    import oracle as O
+
+    pages, counts = O.select_pages(u["q"], u["sig"], u["pt"], u["sl"], cfg.page_size,
+                                   cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    h2l = np.zeros(u["G"], np.int64)
+    scale = 1.0 / math.sqrt(cfg.D)
+    if fp8:
+        O.sparse_attention_fp8(u["q"], u["kc"], u["ks"], u["vc"], u["vs"], u["pt"], u["sl"],
+                               pages, counts, h2l, scale, cfg.page_size)
+    else:
+        O.sparse_attention(u["q"], u["k"], u["v"], u["pt"], u["sl"], pages, counts, h2l, scale,
+                           cfg.page_size)
+    L = int(u["sl"][0])
+    lst = pages[0, 0, :counts[0, 0]]
+    toks = sum(min(cfg.page_size, L - int(p) * cfg.page_size) for p in lst)
+    return toks * cfg.D * 2 * (1 if fp8 else 2) + (len(lst) * 8 if fp8 else 0)
+
+
+def time_oracle(cfg, prepared, fp8, min_s, max_s=60.0, n_steps=None):
+    """GB/s of the oracle over the prepared units (cycled): either until min_s
+    seconds have passed and every unit ran once, or exactly n_steps units."""
+    t0 = time.perf_counter()
+    done, nbytes = 0, 0
+    while True:
+        nbytes += oracle_step(cfg, prepared[done % len(prepared)], fp8)
+        done += 1
+        el = time.perf_counter() - t0
+        if n_steps is not None:
+            if done >= n_steps:
+                break
+        elif (el >= min_s and done >= len(prepared)) or el > max_s:
+            break
+    dt = time.perf_counter() - t0
+    return nbytes / dt / 1e9, done, dt
+
+
+def blas_threads(n):
+    from threadpoolctl import threadpool_limits
+    return threadpool_limits(limits=n)
+
+
+def oracle_sample_units(cfg, n, seed=7):
+    import numpy as np
+    rng = np.random.default_rng(seed)
+    units = set()
+    while len(units) < min(n, cfg.B * cfg.Hkv):
+        units.add((int(rng.integers(cfg.B)), int(rng.integers(cfg.Hkv))))
+    return sorted(units)
+
+
+def cpu_baseline(cfg, inp, fp8, cores):
+    prepared = oracle_units(cfg, inp, oracle_sample_units(cfg, 16), fp8)
+    gbs, n, dt = time_oracle(cfg, prepared, fp8, min_s=10.0)
+    with blas_threads(1):
+        gbs1, n1, dt1 = time_oracle(cfg, prepared, fp8, min_s=4.0)
+    return {"value": round(gbs, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} (sequence, kv head) units of select + attention (a fixed sample of "
+                      f"16 units of layer 0, cycled) in {dt:.1f} s; summaries computed beforehand",
+            "value_1_thread": round(gbs1, 6),
+            "sample_1_thread": f"{n1} units in {dt1:.1f} s, BLAS limited to one thread"}
+
+
+def run_reference(args, dev, cores):
+    """The oracle arm: the float64 oracle times K steps (one (sequence, kv head)
+    unit of select + attention each) of the headline workload on the host cores."""
+    import torch
+
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    fp8 = args.workload == "llama8b_fp8"
+    cfg = {"llama70b": W.LLAMA70B_LONG}.get(args.workload, W.LLAMA8B_DECODE)
+    inp = W.gqa_decode_inputs(cfg, seed=args.seed, device=dev)   # layer 0 of rank 0
+    if fp8:
+        kc, ks = W.fp8_pages(inp.pop("k"))
+        vc, vs = W.fp8_pages(inp.pop("v"))
+        inp.update(kc=kc, ks=ks, vc=vc, vs=vs)
+    prepared = oracle_units(cfg, inp, oracle_sample_units(cfg, 16), fp8)
+    del inp
+    torch.cuda.empty_cache()
+    for i in range(args.warmup):
+        oracle_step(cfg, prepared[i % len(prepared)], fp8)
+    gbs, n, dt = time_oracle(cfg, prepared, fp8, 0.0, n_steps=args.steps)
+    with blas_threads(1):
+        gbs1, n1, dt1 = time_oracle(cfg, prepared, fp8, 0.0, n_steps=min(args.steps, 16))
+    n_layers = GQA_LAYERS if cfg is W.LLAMA8B_DECODE else 1
+    line = {"metric": METRIC, "value": round(gbs, 6), "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1000 * dt / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": gqa_config(cfg, gqa_splits(cfg, args), args.gpus, fp8, n_layers),
+            "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"{n} steps, each one (sequence, kv head) unit of select "
+                                       f"+ attention from a fixed sample of 16 units, {dt:.1f} s",
+                             "value_1_thread": round(gbs1, 6),
+                             "sample_1_thread": f"{n1} units in {dt1:.1f} s, one BLAS thread"},
+            "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
 
 
 def main():
     args = parse()
-    import numpy as np
     import torch
-    import torch.distributed as dist
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.impl == "reference" and rank != 0:
-        return                      # the oracle arm runs on rank 0 only
-    if world > 1 and args.impl == "ours":
+    cores = len(os.sched_getaffinity(0))
+    if args.impl == "reference":
+        if rank != 0:
+            return                  # the oracle arm runs on rank 0 only
+        dev = torch.device("cuda", local)
+        torch.cuda.set_device(dev)
+        if args.workload in ("mla", "prefill"):
+            print(json.dumps({"impl": "reference", "unavailable":
+                              "the oracle arm is timed on the GQA decode workloads"}))
+            return
+        return run_reference(args, dev, cores)
+    if world > 1:
         torch.cuda.set_device(local)
         import datetime
+
+        import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
 
     from paged_sparse_kv_sa_b200 import workloads as W
 
-    cores = len(os.sched_getaffinity(0))
-    if args.workload in ("mla", "prefill"):
-        return run_extra(args, dev, world, rank, local, cores)
-    cfg = {"llama8b": W.LLAMA8B_DECODE, "llama70b": W.LLAMA70B_LONG,
-           "llama8b_fp8": W.LLAMA8B_DECODE}[args.workload]
-    fp8 = args.workload == "llama8b_fp8"
-
-    if args.impl == "reference":
-        # the reference arm is the float64 oracle on the host cores
-        import paged_sparse_kv_sa_b200 as sa
-        sa.load()
-        inp = W.gqa_decode_inputs(cfg, seed=args.seed, device=dev)
-        f8 = None
-        if fp8:
-            kc, ks = W.fp8_pages(inp["k"])
-            vc, vs = W.fp8_pages(inp["v"])
-            f8 = dict(kc=kc, ks=ks, vc=vc, vs=vs)
-            sig = sa.sa_build_page_summaries_fp8(kc, ks, inp["page_table"], inp["seq_lens"])
-        else:
-            sig = sa.sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
-        torch.cuda.synchronize()
-        sig_bits = W.bf16_bits(sig)
-        for _ in range(args.warmup):
-            cpu_baseline(cfg, inp, sig_bits, 1, budget_s=5, f8=f8)
-        tot_b, tot_t, units = 0.0, 0.0, 0
-        for _ in range(args.steps):
-            gbs, n, dt = cpu_baseline(cfg, inp, sig_bits, 2, budget_s=10, f8=f8)
-            tot_b += gbs * dt
-            tot_t += dt
-            units += n
-        val = tot_b / tot_t
-        line = {"metric": METRIC, "value": round(val, 6), "unit": "GB/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(1000 * tot_t / args.steps, 3), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "impl": "reference",
-                "config": {"workload": cfg.name + ("_fp8" if fp8 else ""), "B": cfg.B,
-                           "seq_len": cfg.seq_len_lo,
-                           "Hq": cfg.Hq, "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
-                           "budget_tokens": cfg.budget_tokens},
-                "cpu_baseline": {"value": round(val, 6), "unit": "GB/s", "cores": cores,
-                                 "kind": "oracle",
-                                 "sample": f"{units} (sequence, kv head) units of select + "
-                                           f"attention per {args.steps} steps"},
-                "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
-        return
-
-    import paged_sparse_kv_sa_b200 as sa
-    sa.load()
-    inp = W.gqa_decode_inputs(cfg, seed=args.seed + rank, device=dev)
-    q, k, v, pt, sl = inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"]
-    f8 = None
-    if fp8:
-        # FP8 E4M3 pages with per-(page, kv head) scales, quantized from the bf16 pools
-        kc, ks = W.fp8_pages(k)
-        vc, vs = W.fp8_pages(v)
-        f8 = dict(kc=kc, ks=ks, vc=vc, vs=vs)
-        sig = sa.sa_build_page_summaries_fp8(kc, ks, pt, sl)
-    else:
-        sig = sa.sa_build_page_summaries(k, pt, sl)
-    step = sa.SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size, pt.shape[1],
-                               cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens,
-                               n_splits=args.splits or None, device=dev)
-    stream = torch.cuda.current_stream(dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
-    flush_rd = torch.ones(64 * 1024 * 1024, dtype=torch.int32, device=dev)
-    flush_sink = torch.empty((), dtype=torch.int64, device=dev)
-
-    def flush_l2(i):
-        # write 256 MiB (evicts everything), then read 256 MiB of another buffer
-        # so the dirty lines are written back now, not inside the timed step
-        flush.fill_(i & 0xFF)
-        torch.sum(flush_rd, dim=0, dtype=torch.int64, out=flush_sink)
-
-    def decode_call(qq, ptt, sll):
-        if fp8:
-            step.decode_fp8(qq, kc, vc, ks, vs, ptt, sll)
-        else:
-            step.decode(qq, k, v, ptt, sll)
-
-    def run_step():
-        step.select(q, sig, pt, sl)
-        decode_call(q, pt, sl)
-        step.combine()
-
-    for _ in range(max(args.warmup, 3)):
-        run_step()
-    torch.cuda.synchronize()
-    kv_bytes = selected_kv_bytes(step.counts, step.pages, sl, cfg.page_size, cfg.D,
-                                 elem_bytes=1 if fp8 else 2)
-    q_bytes = q.numel() * 2
-    part_bytes = step.o_part.numel() * 4 + step.lse_part.numel() * 4
-    list_bytes = step.pages.numel() * 4 + step.counts.numel() * 4
-    decode_alg_bytes = kv_bytes + q_bytes + part_bytes + list_bytes + \
-        int(step.counts.sum().item()) * 4
-
-    # Whole steps and the decode kernel alone are replayed from CUDA graphs, so
-    # that the events bracket device work only (no host enqueue gaps).
-    g_step = torch.cuda.CUDAGraph()
-    g_dec = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_step):
-        run_step()
-    with torch.cuda.graph(g_dec):
-        decode_call(q, pt, sl)
-    for _ in range(3):
-        g_step.replay()
-        g_dec.replay()
-    torch.cuda.synchronize()
+    clk = ClockSampler(local).start()
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        for i in range(K):
-            flush_l2(i)
-            ev[i][0].record(stream)
-            g_step.replay()
-            ev[i][1].record(stream)
-            flush_l2(i + 1)
-            ev[i][2].record(stream)
-            g_dec.replay()
-            ev[i][3].record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    t_step = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3           # seconds, K steps
-    t_dec = sum(e[2].elapsed_time(e[3]) for e in ev) / 1e3            # decode kernel alone
-    # per-stage split of one eager step (informational)
-    st_ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
-    flush_l2(0)
-    st_ev[0].record(stream)
-    step.select(q, sig, pt, sl)
-    st_ev[1].record(stream)
-    decode_call(q, pt, sl)
-    st_ev[2].record(stream)
-    step.combine()
-    st_ev[3].record(stream)
-    torch.cuda.synchronize()
-    t_sel = st_ev[0].elapsed_time(st_ev[1]) / 1e3 * K
-    t_cmb = st_ev[2].elapsed_time(st_ev[3]) / 1e3 * K
-    t_step_max = max_over_ranks(t_step, world, dev)
-    value = world * kv_bytes * K / t_step_max / 1e9
-    calls_per_sec = world * K / t_step_max
-
-    # ---- end to end through the same API: host inputs in, host outputs out
-    # inputs packed in one pinned buffer (one host-to-device copy), outputs in one
-    # device buffer the step writes (one device-to-host copy)
-    h_in, (q_h, pt_h, sl_h) = _packed((q, pt, sl), "cpu")
-    q_h.copy_(q.cpu())
-    pt_h.copy_(pt.cpu())
-    sl_h.copy_(sl.cpu())
-    d_in, (q_d, pt_d, sl_d) = _packed((q, pt, sl), dev)
-    d_out, (step.o, step.lse) = _packed((step.o, step.lse), dev)
-    h_out, (o_h, lse_h) = _packed((step.o, step.lse), "cpu")
-
-    def e2e_step():
-        d_in.copy_(h_in, non_blocking=True)
-        step.select(q_d, sig, pt_d, sl_d)
-        decode_call(q_d, pt_d, sl_d)
-        step.combine()
-        h_out.copy_(d_out, non_blocking=True)
-
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
-    if world > 1:
-        dist.barrier()
-    for i in range(K):
-        flush_l2(i)
-        e2e_ev[i][0].record(stream)
-        e2e_step()
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    t_e2e = sum(a.elapsed_time(b) for a, b in e2e_ev) / 1e3
-    t_e2e = max_over_ranks(t_e2e, world, dev)
-    e2e_value = world * kv_bytes * K / t_e2e / 1e9
-    h2d = h_in.numel()
-    d2h = h_out.numel()
-
-    # correctness guard on what was timed: the outputs are finite and selections full
-    assert torch.isfinite(step.o).all().item(), "non-finite output"
-    assert int(step.dev_error.item()) == 0, "device error flag set"
-
-    hbm_peak, peak_kind = peaks()
-    dec_avg = t_dec / K
-    achieved = decode_alg_bytes / dec_avg / 1e9
-    # context for the roofline: one library device copy moving the same number
-    # of bytes (half read, half written) in one launch, from its own graph with
-    # L2 flushed first -- the kind of copy the peak is measured with, at this
-    # size (a single launch pays a fixed cost that a multi-GiB copy hides)
-    half = max(decode_alg_bytes // 2 // 16, 1)
-    rd_buf = torch.ones((half, 4), dtype=torch.int32, device=dev)
-    rd_out = torch.empty_like(rd_buf)
-    g_rd = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_rd):
-        rd_out.copy_(rd_buf)
-    for _ in range(3):
-        g_rd.replay()
-    rd_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(min(K, 50))]
-    for i in range(len(rd_ev)):
-        flush_l2(i)
-        rd_ev[i][0].record(stream)
-        g_rd.replay()
-        rd_ev[i][1].record(stream)
-    torch.cuda.synchronize()
-    t_rd = sum(a.elapsed_time(b) for a, b in rd_ev) / 1e3 / len(rd_ev)
-    read_gbs = 2 * rd_buf.numel() * 4 / t_rd / 1e9
-    del rd_buf, rd_out
-    t_floor = _launch_floor(flush_l2, stream, min(K, 50))
-    traffic = None
-    tp = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tp):
-        with open(tp) as f:
-            td = json.load(f)
-        if td.get("workload") == cfg.name and td.get("splits") == step.n_splits and not fp8:
-            traffic = td.get("bytes_per_launch")
-
-    line = {
-        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
-        "steps": K, "warmup": args.warmup, "ms_per_step": round(1e3 * t_step_max / K, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": cfg.name + ("_fp8" if fp8 else ""), "B": cfg.B,
-                   "seq_len": cfg.seq_len_lo, "Hq": cfg.Hq,
-                   "Hkv": cfg.Hkv, "D": cfg.D, "page_size": cfg.page_size,
-                   "kv_pages": ("fp8 e4m3 + float32 scale per (page, kv head)" if fp8
-                                else "bf16"),
-                   "budget_tokens": cfg.budget_tokens, "sink_tokens": cfg.sink_tokens,
-                   "local_tokens": cfg.local_tokens, "n_splits": step.n_splits,
-                   "l2": "flushed before every timed step (256 MiB write, then 256 MiB read)",
-                   "parallelism": f"replicas x{world}"},
-        "calls_per_sec": round(calls_per_sec, 2),
-        "stage_ms": {"select_eager": round(1e3 * t_sel / K, 4),
-                     "decode_graph": round(1e3 * t_dec / K, 4),
-                     "combine_eager": round(1e3 * t_cmb / K, 4)},
-        "selected_kv_bytes_per_step": kv_bytes,
-        "roofline": {"kernel": "decode_gqa_kernel" + ("<fp8>" if fp8 else ""), "bound": "hbm", "achieved": round(achieved, 2),
-                     "peak": hbm_peak, "unit": "GB/s", "frac": round(achieved / hbm_peak, 4),
-                     "peak_kind": peak_kind, "traffic": traffic,
-                     "alg_bytes_per_launch": decode_alg_bytes,
-                     "same_bytes_copy": {"gbs": round(read_gbs, 1),
-                                         "what": "one device copy (torch copy_) moving the same "
-                                                 "bytes, read + write, L2 flushed"},
-                     "frac_of_same_bytes_copy": round(achieved / read_gbs, 4),
-                     "kernel_us": round(1e6 * dec_avg, 2),
-                     "launch_floor_us": round(1e6 * t_floor, 2),
-                     "launch_floor_what": LAUNCH_FLOOR_WHAT},
-        "e2e": {"value": round(e2e_value, 3), "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(1e3 * t_e2e / K, 4)},
-        "gpu_launches": 4 * K,
-        "clocks": clk.summary(),
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        n_all = cfg.B * cfg.Hkv
-        gbs, n, dt = cpu_baseline(cfg, inp, W.bf16_bits(sig), n_units=n_all, budget_s=20.0, f8=f8,
-                                  min_s=10.0)
-        line["cpu_baseline"] = {"value": round(gbs, 6), "unit": "GB/s", "cores": cores,
-                                "kind": "oracle",
-                                "sample": f"{n} (sequence, kv head) units = {n / n_all:.2f} passes "
-                                          f"over all {n_all} of the workload: select + "
-                                          f"attention, {dt:.1f} s"}
+    wl = args.workload
+    try:
+        if wl in ("mla", "prefill"):
+            sub = (run_mla(args, dev, world, rank, clk, reps=max(1, -(-K // MLA_LAYERS)))
+                   if wl == "mla" else run_prefill(args, dev, world, rank, clk, K))
+            line = {"metric": METRIC, "n_gpus": world, "warmup": args.warmup,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                    "dtype": "bf16", "data": "synthetic", **sub}
+        else:
+            cfg = {"llama70b": W.LLAMA70B_LONG}.get(wl, W.LLAMA8B_DECODE)
+            fp8 = wl == "llama8b_fp8"
+            line = run_gqa(cfg, args, dev, world, rank, clk, K, fp8=fp8,
+                           n_layers=GQA_LAYERS if cfg is W.LLAMA8B_DECODE else 1)
+            layers = line.pop("_layers")
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(cfg, layers[0]["inp"], fp8, cores)
+            del layers
+            torch.cuda.empty_cache()
+            if wl == "all" and world == 1:
+                subs = {}
+                k_long = min(K, 100)
+                r = run_gqa(W.LLAMA70B_LONG, args, dev, world, rank, clk, k_long, n_layers=1)
+                r.pop("_layers")
+                subs["llama70b"] = r
+                torch.cuda.empty_cache()
+                r = run_gqa(W.LLAMA8B_DECODE, args, dev, world, rank, clk, K, fp8=True)
+                r.pop("_layers")
+                subs["llama8b_fp8"] = r
+                torch.cuda.empty_cache()
+                subs["mla"] = run_mla(args, dev, world, rank, clk, reps=max(2, -(-K // 61)))
+                torch.cuda.empty_cache()
+                subs["prefill"] = run_prefill(args, dev, world, rank, clk, min(K, 20))
+                for s in subs.values():
+                    for k_ in ("metric", "n_gpus", "warmup", "higher_is_better", "scaling",
+                               "vs_baseline", "dtype", "data"):
+                        s.pop(k_, None)
+                line["workloads"] = subs
+    finally:
+        clk.stop()
+    line["clocks"] = clk.summary()
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
+        import torch.distributed as dist
         dist.barrier()
         dist.destroy_process_group()
 

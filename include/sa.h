@@ -314,6 +314,42 @@ SA_API int sa_sparse_attention(const uint16_t* q, const int64_t q_strides[4],
                                void* stream);
 
 /*
+ * sa_sparse_step — the whole GQA sparse-attention call in one entry point:
+ * sa_select_pages (scoring against the page summaries, forced sink and local
+ * pages, top-k) and then sa_sparse_attention over the selected lists, every
+ * head h reading the list of its kv head h / (Hq/Hkv).  Sources: as
+ * sa_select_pages ("Universal Attention Engine — Declarative Sparse Attention
+ * for Production", "Content-Dependent Dynamic Routing": selected blocks get
+ * full attention) and sa_sparse_attention.
+ *
+ *  q, summaries, page_table, seq_lens, budget arguments   as sa_select_pages
+ *  k_cache, v_cache (dev) [P_pool,Hkv,P,D] bf16, strides as sa_sparse_decode
+ *  scale      s in s_j = scale * q.k_j (finite)
+ *  n_splits   decode splits per list; <= 0 picks the default for the current
+ *             device (the splits that fill one wave of resident decode warps)
+ *  out_pages  (dev) [B,Hkv,budget_pages] int32, out_counts (dev) [B,Hkv]: the
+ *             selection, as sa_select_pages writes it
+ *  o_out, o_out_bf16, lse_out   as sa_sparse_attention (at least one)
+ *  workspace  (dev) sa_sparse_step_workspace_size(...) bytes, 16-byte aligned,
+ *             caller-owned, no initial contents; calls sharing one must not
+ *             overlap
+ * Supported: D in {64,128,256}, T*Hq/Hkv <= 16, max_pages <= 16384, page_size
+ * a multiple of 16 up to 128, Hq <= 256.  Every argument is checked before the
+ * first launch; then four launches (score, choose, decode, merge).
+ */
+SA_API size_t sa_sparse_step_workspace_size(int B, int T, int Hq, int Hkv, int D, int page_size,
+                                            int max_pages, int budget_tokens, int n_splits);
+SA_API int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                          const uint16_t* k_cache, const int64_t k_strides[4],
+                          const uint16_t* v_cache, const int64_t v_strides[4],
+                          const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                          int B, int T, int Hq, int Hkv, int D, int page_size, int P_pool,
+                          int sink_tokens, int local_tokens, int budget_tokens, float scale,
+                          int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
+                          uint16_t* o_out_bf16, float* lse_out, void* workspace,
+                          size_t workspace_bytes, int32_t* dev_error, void* stream);
+
+/*
  * sa_sparse_attention_fp8 — sa_sparse_decode_fp8 followed by the merge, in one
  * call.  Arguments as sa_sparse_decode_fp8 for the inputs and as
  * sa_sparse_attention for the outputs and the workspace (sized with Dv = D).

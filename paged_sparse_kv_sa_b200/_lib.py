@@ -11,6 +11,7 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 
 import torch
 
@@ -47,7 +48,11 @@ _SIGNATURES = {
     "sa_sparse_attention_fp8": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _P, _P, _I,
                                      _P, _P, _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                                      _P, _P, _P, _P, ctypes.c_size_t, _P, _P]),
-    "sa_build_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_sparse_step_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I, _I, _I, _I, _I, _I]),
+    "sa_sparse_step": (_I, [_P, _c_i64_4, _P, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _I, _I, _I,
+                            _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _P,
+                            ctypes.c_size_t, _P, _P]),
+    "sa_build_page_summaries": (_I,[_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sa_update_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                       _P]),
     "sa_build_page_summaries_fp8": (_I, [_P, _c_i64_4, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P,
@@ -87,8 +92,51 @@ def _check(status: int, what: str):
         raise SAError(f"{what} failed: {msg} ({status})")
 
 
+# While bind() records, the wrappers' C calls are stored instead of issued, and
+# every tensor whose pointer is passed is kept alive with the recording.
+_REC = threading.local()
+
+
 def _ptr(t):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    if t is None:
+        return None
+    keep = getattr(_REC, "keep", None)
+    if keep is not None:
+        keep.append(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _call(fn, args, what):
+    prog = getattr(_REC, "prog", None)
+    if prog is not None:
+        prog.append((fn, args, what))
+        return
+    _check(fn(*args), what)
+
+
+def bind(fn):
+    """Run ``fn()`` once with the library's C calls recorded instead of issued
+    (arguments checked and marshalled as usual) and return a zero-argument
+    callable that issues the recorded calls, in order, with the same pointers,
+    sizes and streams -- for loops that run the same calls over the same
+    buffers many times (a serving step over preallocated tensors).  The tensors
+    the calls point to are kept alive by the callable; their contents may
+    change between calls, their storage must not move."""
+    _REC.prog, _REC.keep = [], []
+    try:
+        fn()
+        prog, keep = _REC.prog, _REC.keep
+    finally:
+        _REC.prog = _REC.keep = None
+
+    def run():
+        for f, a, what in prog:
+            st = f(*a)
+            if st != 0:
+                _check(st, what)
+    run.keep = keep
+    run.n_calls = len(prog)
+    return run
 
 
 def _strides4(t) -> "ctypes.Array":
@@ -187,12 +235,11 @@ def sa_select_pages(q, summaries, page_table, seq_lens, page_size: int, sink_tok
     if workspace is None:
         workspace = torch.empty(max(sa_select_workspace_size(B, Hkv, max_pages), 16),
                                 dtype=torch.uint8, device=q.device)
-    st = lib.sa_select_pages(_ptr(q), _strides4(q), _ptr(summaries.contiguous()), _ptr(page_table),
+    _call(lib.sa_select_pages, (_ptr(q), _strides4(q), _ptr(summaries.contiguous()), _ptr(page_table),
                              _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size, max_pages,
                              P_pool, sink_tokens, local_tokens, budget_tokens, _ptr(out_pages),
                              _ptr(out_counts), _ptr(workspace), workspace.numel(),
-                             _ptr(dev_error), _stream(stream))
-    _check(st, "sa_select_pages")
+                             _ptr(dev_error), _stream(stream)), "sa_select_pages")
     return out_pages, out_counts
 
 
@@ -214,12 +261,11 @@ def sa_select_pages_no_alloc(q, summaries, page_table, seq_lens, page_size: int,
     P_pool = P_pool_ if P_pool is None else P_pool
     _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts,
                    budget_tokens // page_size)
-    st = lib.sa_select_pages_no_alloc(_ptr(q), _strides4(q), _ptr(summaries), _ptr(page_table),
+    _call(lib.sa_select_pages_no_alloc, (_ptr(q), _strides4(q), _ptr(summaries), _ptr(page_table),
                                       _ptr(seq_lens), B, T, Hq, Hkv, Dk, page_size,
                                       page_table.shape[1], P_pool, sink_tokens, local_tokens,
                                       budget_tokens, _ptr(out_pages), _ptr(out_counts),
-                                      _ptr(dev_error), _stream(stream))
-    _check(st, "sa_select_pages_no_alloc")
+                                      _ptr(dev_error), _stream(stream)), "sa_select_pages_no_alloc")
     return out_pages, out_counts
 
 
@@ -241,12 +287,11 @@ def sa_select_pages_tiered(q, summaries, page_table, seq_lens, page_size: int, a
     if workspace is None:
         n = int(lib.sa_select_tiered_workspace_size(B, T, Hq, max_pages))
         workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
-    st = lib.sa_select_pages_tiered(_ptr(q), _strides4(q), _ptr(summaries.contiguous()),
+    _call(lib.sa_select_pages_tiered, (_ptr(q), _strides4(q), _ptr(summaries.contiguous()),
                                     _ptr(page_table), _ptr(seq_lens), B, T, Hq, Dk, page_size,
                                     max_pages, P_pool, alpha, beta, _ptr(lists),
                                     _ptr(list_counts), _ptr(workspace), workspace.numel(),
-                                    _ptr(dev_error), _stream(stream))
-    _check(st, "sa_select_pages_tiered")
+                                    _ptr(dev_error), _stream(stream)), "sa_select_pages_tiered")
     return lists, list_counts
 
 
@@ -269,13 +314,12 @@ def sa_sparse_decode(q, k_cache, v_cache, page_table, seq_lens, lists, list_coun
         o_partial = torch.empty((n_splits, B, T, Hq, Dv), dtype=torch.float32, device=q.device)
     if lse_partial is None:
         lse_partial = torch.empty((n_splits, B, T, Hq), dtype=torch.float32, device=q.device)
-    st = lib.sa_sparse_decode(_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
+    _call(lib.sa_sparse_decode, (_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
                               _ptr(v_cache), _strides4(v_cache), _ptr(page_table),
                               page_table.shape[1], _ptr(seq_lens), _ptr(lists), _ptr(list_counts),
                               n_lists, max_list, ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv,
                               Dk, Dv, P, P_pool, float(scale), n_splits, _ptr(o_partial),
-                              _ptr(lse_partial), _ptr(dev_error), _stream(stream))
-    _check(st, "sa_sparse_decode")
+                              _ptr(lse_partial), _ptr(dev_error), _stream(stream)), "sa_sparse_decode")
     return o_partial, lse_partial
 
 
@@ -296,14 +340,13 @@ def sa_sparse_decode_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_
         o_partial = torch.empty((n_splits, B, T, Hq, D), dtype=torch.float32, device=q.device)
     if lse_partial is None:
         lse_partial = torch.empty((n_splits, B, T, Hq), dtype=torch.float32, device=q.device)
-    st = lib.sa_sparse_decode_fp8(_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
+    _call(lib.sa_sparse_decode_fp8, (_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
                                   _ptr(v_codes), _strides4(v_codes), _ptr(k_scale), _ptr(v_scale),
                                   _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
                                   _ptr(lists), _ptr(list_counts), n_lists, max_list,
                                   ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, D, P, P_pool,
                                   float(scale), n_splits, _ptr(o_partial), _ptr(lse_partial),
-                                  _ptr(dev_error), _stream(stream))
-    _check(st, "sa_sparse_decode_fp8")
+                                  _ptr(dev_error), _stream(stream)), "sa_sparse_decode_fp8")
     return o_partial, lse_partial
 
 
@@ -343,16 +386,61 @@ def sa_sparse_attention(q, k_cache, v_cache, page_table, seq_lens, lists, list_c
                                                lse_out, want_f32, want_bf16)
     if workspace is None:
         workspace = attention_workspace(B, T, Hq, Dv, n_splits, q.device)
-    st = lib.sa_sparse_attention(_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
+    _call(lib.sa_sparse_attention, (_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache),
                                  _ptr(v_cache), _strides4(v_cache), _ptr(page_table),
                                  page_table.shape[1], _ptr(seq_lens), _ptr(lists),
                                  _ptr(list_counts), n_lists, max_list,
                                  ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, Dk, Dv, P,
                                  P_pool, float(scale), n_splits, _ptr(o_out), _ptr(o_out_bf16),
                                  _ptr(lse_out), _ptr(workspace), workspace.numel(),
-                                 _ptr(dev_error), _stream(stream))
-    _check(st, "sa_sparse_attention")
+                                 _ptr(dev_error), _stream(stream)), "sa_sparse_attention")
     return o_out, o_out_bf16, lse_out
+
+
+def sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens,
+                                  n_splits=0) -> int:
+    return int(load().sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, page_size, max_pages,
+                                                    budget_tokens, n_splits))
+
+
+def sa_sparse_step(q, summaries, k_cache, v_cache, page_table, seq_lens, page_size: int,
+                   sink_tokens: int, local_tokens: int, budget_tokens: int, scale: float,
+                   n_splits: int = 0, out_pages=None, out_counts=None, o_out=None,
+                   o_out_bf16=None, lse_out=None, want_f32: bool = True, want_bf16: bool = False,
+                   workspace=None, dev_error=None, stream=None):
+    """Selection + attention + merge in one C call (sa_sparse_step).  q [B,T,Hq,D];
+    summaries [P_pool,Hkv,D]; k_cache, v_cache [P_pool,Hkv,P,D]; n_splits 0 = the
+    library's default.  Returns (pages, counts, O f32 or None, O bf16 or None, lse)."""
+    lib = load()
+    _need_cuda(q, summaries, k_cache, v_cache, page_table, seq_lens)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(page_table), _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    B, T, Hq, D = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    if P != page_size:
+        raise ValueError("page_size differs from the cache's page dimension")
+    bp = budget_tokens // page_size
+    _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts, bp)
+    if out_pages is None:
+        out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
+    if out_counts is None:
+        out_counts = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, D, q.device, o_out, o_out_bf16,
+                                               lse_out, want_f32, want_bf16)
+    max_pages = page_table.shape[1]
+    if workspace is None:
+        n = sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens,
+                                          n_splits)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _call(lib.sa_sparse_step,
+          (_ptr(q), _strides4(q), _ptr(summaries), _ptr(k_cache), _strides4(k_cache),
+           _ptr(v_cache), _strides4(v_cache), _ptr(page_table), max_pages, _ptr(seq_lens), B, T,
+           Hq, Hkv, D, page_size, P_pool, sink_tokens, local_tokens, budget_tokens,
+           float(scale), int(n_splits), _ptr(out_pages), _ptr(out_counts), _ptr(o_out),
+           _ptr(o_out_bf16), _ptr(lse_out), _ptr(workspace), workspace.numel(),
+           _ptr(dev_error), _stream(stream)), "sa_sparse_step")
+    return out_pages, out_counts, o_out, o_out_bf16, lse_out
 
 
 def sa_sparse_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens, lists,
@@ -373,15 +461,14 @@ def sa_sparse_attention_fp8(q, k_codes, v_codes, k_scale, v_scale, page_table, s
                                                want_f32, want_bf16)
     if workspace is None:
         workspace = attention_workspace(B, T, Hq, D, n_splits, q.device)
-    st = lib.sa_sparse_attention_fp8(_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
+    _call(lib.sa_sparse_attention_fp8, (_ptr(q), _strides4(q), _ptr(k_codes), _strides4(k_codes),
                                      _ptr(v_codes), _strides4(v_codes), _ptr(k_scale),
                                      _ptr(v_scale), _ptr(page_table), page_table.shape[1],
                                      _ptr(seq_lens), _ptr(lists), _ptr(list_counts), n_lists,
                                      max_list, ctypes.cast(h2l, ctypes.c_void_p), B, T, Hq, Hkv, D,
                                      P, P_pool, float(scale), n_splits, _ptr(o_out),
                                      _ptr(o_out_bf16), _ptr(lse_out), _ptr(workspace),
-                                     workspace.numel(), _ptr(dev_error), _stream(stream))
-    _check(st, "sa_sparse_attention_fp8")
+                                     workspace.numel(), _ptr(dev_error), _stream(stream)), "sa_sparse_attention_fp8")
     return o_out, o_out_bf16, lse_out
 
 
@@ -395,11 +482,10 @@ def sa_build_page_summaries_fp8(k_codes, k_scale, page_table, seq_lens, summarie
     P_pool, Hkv, P, Dk = k_codes.shape
     if summaries is None:
         summaries = torch.zeros((P_pool, Hkv, Dk), dtype=torch.bfloat16, device=k_codes.device)
-    st = lib.sa_build_page_summaries_fp8(_ptr(k_codes), _strides4(k_codes), _ptr(k_scale),
+    _call(lib.sa_build_page_summaries_fp8, (_ptr(k_codes), _strides4(k_codes), _ptr(k_scale),
                                          _ptr(page_table), page_table.shape[1], _ptr(seq_lens),
                                          seq_lens.shape[0], Hkv, Dk, P, P_pool, _ptr(summaries),
-                                         _ptr(dev_error), _stream(stream))
-    _check(st, "sa_build_page_summaries_fp8")
+                                         _ptr(dev_error), _stream(stream)), "sa_build_page_summaries_fp8")
     return summaries
 
 
@@ -417,9 +503,8 @@ def sa_combine(o_partial, lse_partial, o_out=None, o_out_bf16=None, lse_out=None
         o_out = torch.empty(lead + (Dv,), dtype=torch.float32, device=o_partial.device)
     if lse_out is None:
         lse_out = torch.empty(lead, dtype=torch.float32, device=o_partial.device)
-    st = lib.sa_combine(_ptr(o_partial), _ptr(lse_partial), S, rows, Dv, _ptr(o_out),
-                        _ptr(o_out_bf16), _ptr(lse_out), _stream(stream))
-    _check(st, "sa_combine")
+    _call(lib.sa_combine, (_ptr(o_partial), _ptr(lse_partial), S, rows, Dv, _ptr(o_out),
+                        _ptr(o_out_bf16), _ptr(lse_out), _stream(stream)), "sa_combine")
     return o_out, o_out_bf16, lse_out
 
 
@@ -433,11 +518,10 @@ def sa_build_page_summaries(k_cache, page_table, seq_lens, summaries=None, dev_e
     P_pool, Hkv, P, Dk = k_cache.shape
     if summaries is None:
         summaries = torch.zeros((P_pool, Hkv, Dk), dtype=torch.bfloat16, device=k_cache.device)
-    st = lib.sa_build_page_summaries(_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
+    _call(lib.sa_build_page_summaries, (_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
                                      page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0], Hkv,
                                      Dk, P, P_pool, _ptr(summaries), _ptr(dev_error),
-                                     _stream(stream))
-    _check(st, "sa_build_page_summaries")
+                                     _stream(stream)), "sa_build_page_summaries")
     return summaries
 
 
@@ -449,11 +533,10 @@ def sa_update_page_summaries(k_cache, page_table, seq_lens, summaries, n_new: in
     _need_cuda(k_cache, page_table, seq_lens, summaries)
     _bf16(k_cache), _i32(page_table), _i32(seq_lens), _bf16(summaries)
     P_pool, Hkv, P, Dk = k_cache.shape
-    st = lib.sa_update_page_summaries(_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
+    _call(lib.sa_update_page_summaries, (_ptr(k_cache), _strides4(k_cache), _ptr(page_table),
                                       page_table.shape[1], _ptr(seq_lens), seq_lens.shape[0],
                                       Hkv, Dk, P, P_pool, int(n_new), _ptr(summaries),
-                                      _ptr(dev_error), _stream(stream))
-    _check(st, "sa_update_page_summaries")
+                                      _ptr(dev_error), _stream(stream)), "sa_update_page_summaries")
     return summaries
 
 
@@ -469,7 +552,6 @@ def sa_block_union(scores, Hkv: int, q_block_offset: int, top_k: int, n_sink_blo
         tables = torch.empty((Hkv, NKB), dtype=torch.int32, device=scores.device)
     if counts is None:
         counts = torch.empty((Hkv,), dtype=torch.int32, device=scores.device)
-    st = lib.sa_block_union(_ptr(scores), Hq, Hkv, NQB, NKB, q_block_offset, top_k,
-                            n_sink_blocks, _ptr(tables), _ptr(counts), _stream(stream))
-    _check(st, "sa_block_union")
+    _call(lib.sa_block_union, (_ptr(scores), Hq, Hkv, NQB, NKB, q_block_offset, top_k,
+                            n_sink_blocks, _ptr(tables), _ptr(counts), _stream(stream)), "sa_block_union")
     return tables, counts

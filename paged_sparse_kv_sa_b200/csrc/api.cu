@@ -646,6 +646,91 @@ int sa_sparse_attention(const uint16_t* q, const int64_t q_strides[4], const uin
                             reinterpret_cast<float*>(ws + w.o_bytes), dev_error, stream, &m);
 }
 
+}  // extern "C"
+
+namespace {
+// The split count a step uses (n_splits <= 0: the default policy for this
+// device) and its workspace: the selection's score bounds, then the split
+// partials.
+int step_plan(int B, int T, int Hq, int Hkv, int D, int page_size, int max_pages,
+              int budget_tokens, int n_splits, int* splits_out, size_t* sel_bytes,
+              size_t* total_bytes) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0 ||
+      max_pages < 0 || budget_tokens < 0)
+    return SA_ERR_INVALID_ARG;
+  const int budget_pages = budget_tokens / page_size;
+  if (budget_pages <= 0) return SA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128 && D != 256) return SA_ERR_UNSUPPORTED;
+  int s = n_splits;
+  if (s <= 0 && cuda_status(decode_default_splits(D, B * Hkv, budget_pages, &s)) != SA_OK)
+    return SA_ERR_CUDA;
+  *splits_out = s;
+  *sel_bytes = (select_workspace_bytes(B, Hkv, max_pages > 0 ? max_pages : 1) + 15) / 16 * 16;
+  const AttnWs w = attn_ws(B, T, Hq, D, s);
+  *total_bytes = *sel_bytes + w.o_bytes + w.lse_bytes;
+  return SA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t sa_sparse_step_workspace_size(int B, int T, int Hq, int Hkv, int D, int page_size,
+                                     int max_pages, int budget_tokens, int n_splits) {
+  int s = 0;
+  size_t sel = 0, total = 0;
+  if (step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &s, &sel,
+                &total) != SA_OK)
+    return 0;
+  return total;
+}
+
+int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                   const uint16_t* k_cache, const int64_t k_strides[4], const uint16_t* v_cache,
+                   const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                   const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D, int page_size,
+                   int P_pool, int sink_tokens, int local_tokens, int budget_tokens, float scale,
+                   int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
+                   uint16_t* o_out_bf16, float* lse_out, void* workspace,
+                   size_t workspace_bytes, int32_t* dev_error, void* stream) {
+  int splits = 0;
+  size_t sel_bytes = 0, total = 0;
+  if (int r = step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &splits,
+                        &sel_bytes, &total))
+    return r;
+  SelectArgs sa_args;
+  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, D,
+                          page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
+                          out_pages, out_counts, dev_error, &sa_args))
+    return r;
+  if (B == 0) return SA_OK;
+  MergeSpec m{o_out, o_out_bf16, lse_out};
+  if (int r = merge_outputs_ok(m)) return r;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < total) return SA_ERR_WORKSPACE;
+  // every argument of both halves is checked before the first launch
+  if (int r = check_cache(k_cache, k_strides)) return r;
+  if (int r = check_cache(v_cache, v_strides)) return r;
+  if (P_pool <= 0 || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
+  if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
+  const int budget_pages = sa_args.budget_pages;
+  if ((budget_pages + splits - 1) / splits > decode_max_split_entries() || splits > 64 ||
+      (int64_t)B * T * Hq * (D / 4) >= (int64_t(1) << 32))
+    return SA_ERR_UNSUPPORTED;
+  int32_t h2l[kMaxHeads];
+  if (Hq > kMaxHeads) return SA_ERR_UNSUPPORTED;
+  for (int h = 0; h < Hq; ++h) h2l[h] = h / (Hq / Hkv);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  sa_args.lohi = reinterpret_cast<float2*>(ws);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (int r = cuda_status(launch_select_gqa(sa_args, st))) return r;
+  const AttnWs w = attn_ws(B, T, Hq, D, splits);
+  uint8_t* parts = ws + sel_bytes;
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+                            max_pages, seq_lens, out_pages, out_counts, Hkv, budget_pages, h2l, B,
+                            T, Hq, Hkv, D, D, page_size, P_pool, scale, splits,
+                            reinterpret_cast<float*>(parts),
+                            reinterpret_cast<float*>(parts + w.o_bytes), dev_error, stream, &m);
+}
+
 int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],
                             const uint8_t* k_codes, const int64_t k_strides[4],
                             const uint8_t* v_codes, const int64_t v_strides[4],

@@ -486,6 +486,28 @@ cudaError_t launch_d(const DecodeArgs& a, const PairTable& pairs, const CUtensor
 int decode_max_split_entries() { return kWarpEntries; }
 int decode_warps_per_cta() { return kNW; }
 
+cudaError_t decode_default_splits(int D, int n_units, int max_list, int* out) {
+  *out = 1;
+  if (n_units <= 0 || max_list <= 0) return cudaSuccess;
+  const void* kern = D == 64    ? reinterpret_cast<const void*>(decode_gqa_kernel<64, false>)
+                     : D == 128 ? reinterpret_cast<const void*>(decode_gqa_kernel<128, false>)
+                                : reinterpret_cast<const void*>(decode_gqa_kernel<256, false>);
+  const int dyn = D == 64    ? DecodeCfg<64>::kDynBytes
+                  : D == 128 ? DecodeCfg<128>::kDynBytes
+                             : DecodeCfg<256>::kDynBytes;
+  int sms = 0, per_sm = 0;
+  cudaError_t e = sm_count(&sms);
+  if (e == cudaSuccess) e = max_blocks_per_sm(kern, kNW * 32, dyn, &per_sm);
+  if (e != cudaSuccess) return e;
+  // as many splits as fill one wave of resident warps, at least enough that no
+  // split holds more than a warp's list capacity, at most 64
+  int n = std::max(1, std::max(1, per_sm) * kNW * sms / n_units);
+  n = std::min(n, max_list);
+  while ((max_list + n - 1) / n > kWarpEntries) ++n;
+  *out = std::max(1, std::min(n, 64));
+  return cudaSuccess;
+}
+
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream) {
   switch (a.Dk) {

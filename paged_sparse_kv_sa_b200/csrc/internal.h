@@ -105,6 +105,10 @@ cudaError_t launch_mla(const DecodeArgs& a, const PairTable& pairs, const CUtens
 cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                            const CUtensorMap& vmap, cudaStream_t stream);
 int decode_warps_per_cta();
+// Split count for n_units (sequence, list) pairs of up to max_list pages with
+// head dim D: the splits that fill one wave of resident decode warps, at least
+// enough that no split exceeds a warp's list capacity, at most 64.
+cudaError_t decode_default_splits(int D, int n_units, int max_list, int* out);
 cudaError_t launch_decode_gqa(const DecodeArgs& a, const PairTable& pairs, const CUtensorMap& kmap,
                               const CUtensorMap& vmap, cudaStream_t stream);
 cudaError_t launch_decode_gqa_fp8(const DecodeArgs& a, const PairTable& pairs,

@@ -68,6 +68,10 @@ class SparseDecodeStep:
                                   dtype=torch.uint8, device=dev)
         # the split partials of sa_sparse_attention
         self.attn_ws = _lib.attention_workspace(B, T, Hq, D, self.n_splits, dev)
+        # score bounds + split partials of the one-call step (sa_sparse_step)
+        self.step_ws = torch.empty(max(_lib.sa_sparse_step_workspace_size(
+            B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, self.n_splits), 16),
+            dtype=torch.uint8, device=dev)
 
     def select(self, q, summaries, page_table, seq_lens, stream=None):
         _lib.sa_select_pages(q, summaries, page_table, seq_lens, self.P, self.sink, self.local,
@@ -108,7 +112,22 @@ class SparseDecodeStep:
         _lib.sa_combine(self.o_part, self.lse_part, o_out=self.o, o_out_bf16=self.o_bf16,
                         lse_out=self.lse, stream=stream)
 
+    def run(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
+        """select + decode + merge as one C call (sa_sparse_step) into self.pages,
+        self.counts, self.o / self.o_bf16 and self.lse."""
+        _lib.sa_sparse_step(q, summaries, k_cache, v_cache, page_table, seq_lens, self.P,
+                            self.sink, self.local, self.budget, self.scale, self.n_splits,
+                            out_pages=self.pages, out_counts=self.counts, o_out=self.o,
+                            o_out_bf16=self.o_bf16, lse_out=self.lse, workspace=self.step_ws,
+                            dev_error=self.dev_error, stream=stream)
+
+    def bind(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
+        """A zero-argument callable that runs `run` on these tensors: the arguments
+        are checked and marshalled once (_lib.bind; the tensors must stay where
+        they are)."""
+        return _lib.bind(lambda: self.run(q, k_cache, v_cache, summaries, page_table, seq_lens,
+                                          stream))
+
     def __call__(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
-        self.select(q, summaries, page_table, seq_lens, stream)
-        self.attend(q, k_cache, v_cache, page_table, seq_lens, stream)
+        self.run(q, k_cache, v_cache, summaries, page_table, seq_lens, stream)
         return self.o, self.lse

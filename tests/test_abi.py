@@ -130,6 +130,34 @@ def test_attention_workspace_size_and_host_checks():
                                        None, None) == 3
 
 
+def test_step_workspace_size_and_host_checks():
+    lib = sa.load()
+    r16 = lambda x: (x + 15) // 16 * 16
+    # score bounds [B, Hkv, max_pages] x 8 bytes, then the split partials
+    B, T, Hq, Hkv, D, P, mp, budget, ns = 16, 1, 32, 8, 128, 16, 2048, 1024, 13
+    rows = B * T * Hq
+    assert lib.sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, P, mp, budget, ns) == \
+        r16(B * Hkv * mp * 8) + r16(rows * D * ns * 4) + r16(rows * ns * 4)
+    assert lib.sa_sparse_step_workspace_size(B, T, 30, Hkv, D, P, mp, budget, ns) == 0   # Hq % Hkv
+    assert lib.sa_sparse_step_workspace_size(B, T, Hq, Hkv, 96, P, mp, budget, ns) == 0  # head dim
+    fake = ctypes.c_void_p(0x1000)      # never dereferenced: validation fails first
+    s = _i64x4(4096, 4096, 128, 1)
+    ks = _i64x4(4096, 2048, 128, 1)
+    need = lib.sa_sparse_step_workspace_size(2, 1, 8, 2, 128, 16, 64, 256, 2)
+
+    def call(ws, ws_bytes, o_out=fake, k=fake, scale=0.1, sink=32):
+        return lib.sa_sparse_step(fake, s, fake, k, ks, fake, ks, fake, 64, fake, 2, 1, 8, 2, 128,
+                                  16, 128, sink, 64, 256, scale, 2, fake, fake, o_out, None, None,
+                                  ws, ws_bytes, None, None)
+    assert call(None, need) == 3                              # no workspace
+    assert call(fake, need - 16) == 3                         # too small
+    assert call(ctypes.c_void_p(0x1008), need) == 3           # not 16-byte aligned
+    assert call(fake, need, o_out=None) == 1                  # no output at all
+    assert call(fake, need, k=ctypes.c_void_p(0x1004)) == 1   # cache base misaligned
+    assert call(fake, need, scale=float("inf")) == 1          # scale not finite
+    assert call(fake, need, sink=512) == 1                    # sink + local above the budget
+
+
 def test_default_split_policy():
     from paged_sparse_kv_sa_b200.pipeline import default_splits
     # one wave of decode warps (12 per SM on 148 SMs) over the (sequence, kv head) units

@@ -15,7 +15,7 @@ import paged_sparse_kv_sa_b200 as sa
 from oracle import sa_oracle as O
 from paged_sparse_kv_sa_b200 import workloads as W
 from test_gpu_parity import (DEV, assert_attn_close, bits, fp8_case, gqa_case, mla_lists_from_oracle,
-                             np_i32, oracle_fp8, oracle_lists, oracle_summaries)
+                             np_i32, oracle_fp8, oracle_lists, oracle_summaries, to_bf16_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -247,3 +247,59 @@ def test_attention_sharp_softmax(path, mult):
     # Every kernel multiplies by P as a bf16 pair hi + lo (~2^-17 relative; a
     # single bf16 P, 2^-9, missed the bar at three times the scale)
     assert_attn_close(*_scaled_case(path, mult, 49))
+
+
+@pytest.mark.parametrize("D,P,T,n_splits", [(128, 16, 1, 0), (64, 32, 2, 3), (256, 16, 1, 0),
+                                            (128, 64, 1, 5)])
+def test_step_vs_oracle(D, P, T, n_splits):
+    # sa_sparse_step: selection + attention + merge in one C call (n_splits 0 = the
+    # library's default), against the oracle's selection and attention
+    cfg = W.GQADecode("case", B=3, Hq=8, Hkv=2, D=D, page_size=P, seq_len_lo=0, seq_len_hi=0,
+                      sink_tokens=P, local_tokens=2 * P, budget_tokens=12 * P, T=T)
+    lens = [50 * P + 7, 9 * P, 3 * P + 1]
+    inp, g = gqa_case(cfg, seed=60, seq_lens=lens)
+    sig = oracle_summaries(inp, cfg)
+    scale = 1.0 / math.sqrt(D)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pages, counts, o, _, lse = sa.sa_sparse_step(g["q"], to_bf16_dev(sig), g["k"], g["v"],
+                                                 g["page_table"], g["seq_lens"], P,
+                                                 cfg.sink_tokens, cfg.local_tokens,
+                                                 cfg.budget_tokens, scale, n_splits,
+                                                 dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]),
+                            np_i32(inp["seq_lens"]), P, cfg.sink_tokens, cfg.local_tokens,
+                            cfg.budget_tokens)
+    assert np.array_equal(np_i32(counts), rc) and np.array_equal(np_i32(pages), rp)
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), rp, rc,
+                                np.arange(cfg.Hq) // cfg.G, scale, P)
+    assert_attn_close(o, lse, ro, rl)
+
+
+def test_bound_calls_replay_on_new_contents():
+    # sa.bind records the C calls of a step once; replaying them after the input
+    # tensors' contents change (same storage) must give what fresh calls give
+    cfg = W.GQADecode("case", B=2, Hq=8, Hkv=2, D=128, page_size=16, seq_len_lo=0, seq_len_hi=0,
+                      sink_tokens=16, local_tokens=64, budget_tokens=256)
+    inp, g = gqa_case(cfg, seed=61, seq_lens=[3000, 1111])
+    sig = to_bf16_dev(oracle_summaries(inp, cfg))
+    step = sa.SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size,
+                               g["page_table"].shape[1], cfg.sink_tokens, cfg.local_tokens,
+                               cfg.budget_tokens, device=DEV)
+    q = g["q"].clone()
+    run = step.bind(q, g["k"], g["v"], sig, g["page_table"], g["seq_lens"])
+    assert run.n_calls == 1
+    for seed in (62, 63):
+        q.copy_(torch.randn(q.shape, generator=torch.Generator().manual_seed(seed))
+                .to(torch.bfloat16).to(DEV))
+        run()
+        torch.cuda.synchronize()
+        got = (step.pages.clone(), step.o.clone(), step.lse.clone())
+        ref = sa.sa_sparse_step(q, sig, g["k"], g["v"], g["page_table"], g["seq_lens"],
+                                cfg.page_size, cfg.sink_tokens, cfg.local_tokens,
+                                cfg.budget_tokens, step.scale, step.n_splits)
+        torch.cuda.synchronize()
+        assert torch.equal(got[0], ref[0]) and torch.equal(got[1], ref[2])
+        assert torch.equal(got[2], ref[4])

@@ -120,6 +120,15 @@ def test_llama8b_workload_end_to_end_sampled():
                                          step.head_to_list, step.scale, step.n_splits)
     torch.cuda.synchronize()
     assert torch.equal(o2, step.o) and torch.equal(lse2, step.lse)
+    # and so does the one-call step (selection + attention + merge, sa_sparse_step)
+    pages, counts, o_ref, lse_ref = (step.pages.clone(), step.counts.clone(), step.o.clone(),
+                                     step.lse.clone())
+    step.pages.fill_(-7)
+    step.o.zero_()
+    step.run(inp["q"], inp["k"], inp["v"], sig, inp["page_table"], inp["seq_lens"])
+    torch.cuda.synchronize()
+    assert torch.equal(step.pages, pages) and torch.equal(step.counts, counts)
+    assert torch.equal(step.o, o_ref) and torch.equal(step.lse, lse_ref)
 
 
 @pytest.fixture(scope="module")
