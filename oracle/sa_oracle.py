@@ -55,7 +55,7 @@ __all__ = [
     "bf16_to_f64", "f64_to_bf16_rne", "e4m3_to_f64", "page_budget", "exact_dots",
     "page_summaries", "page_summaries_fp8", "page_scores", "rank_select", "select_pages",
     "select_pages_mla", "sparse_attention", "sparse_attention_fp8", "masked_dense_attention",
-    "combine", "block_union", "NEG_INF",
+    "combine", "block_union", "append_kv", "NEG_INF",
 ]
 
 NEG_INF = float("-inf")
@@ -519,3 +519,41 @@ def block_union(scores, Hkv: int, q_block_offset: int, top_k: int, n_sink_blocks
         tables[g, :len(ids)] = ids
         counts[g] = len(ids)
     return tables, counts
+
+
+# --------------------------------------------------------------------------
+# appending tokens to the paged cache ([UAE] "Content-Dependent Dynamic
+# Routing": the router reads mean(k_blocks), so a block's summary changes when
+# tokens land in it; "Architecture": a PagedAttention-compatible cache)
+# --------------------------------------------------------------------------
+def append_kv(k_bits, v_bits, sig_bits, page_table, seq_lens, k_new_bits, v_new_bits, n_new,
+              page_size: int):
+    """New pools, summaries and lengths after sequence b appends its n_new[b]
+    tokens (k_new[b, i], v_new[b, i] for i < n_new[b]; [B, max_new, Hkv, D] bf16
+    bits) at positions seq_lens[b] + i, i.e. page page_table[b, pos // P], row
+    pos % P.  The summaries of the pages those positions fall in are recomputed
+    from their definition (page_summaries over the new lengths); every other row
+    of the pools and of the summaries is left as it was."""
+    k = np.array(k_bits, dtype=np.uint16, copy=True)
+    v = np.array(v_bits, dtype=np.uint16, copy=True)
+    sig = np.array(sig_bits, dtype=np.uint16, copy=True)
+    pt = np.asarray(page_table, dtype=np.int64)
+    sl = np.asarray(seq_lens, dtype=np.int64)
+    nn = np.asarray(n_new, dtype=np.int64)
+    kn = np.asarray(k_new_bits, dtype=np.uint16)
+    vn = np.asarray(v_new_bits, dtype=np.uint16)
+    P = page_size
+    touched = set()
+    for b in range(len(sl)):
+        for i in range(int(nn[b])):
+            pos = int(sl[b]) + i
+            ph = int(pt[b, pos // P])
+            k[ph, :, pos % P, :] = kn[b, i]
+            v[ph, :, pos % P, :] = vn[b, i]
+            touched.add((b, pos // P))
+    new_lens = sl + nn
+    fresh = page_summaries(k, pt, new_lens, P, units=sorted(touched))
+    for b, p in touched:
+        ph = int(pt[b, p])
+        sig[ph] = fresh[ph]
+    return k, v, sig, new_lens.astype(np.int32)

@@ -576,3 +576,82 @@ def test_fp8_attention_closed_forms():
     np.testing.assert_array_equal(o[0, 0, 0], np.array([float(x) for x in v0]))
     qk = sum(bf16_fraction(a) * e4m3_fraction(c) for a, c in zip(q[0, 0, 0], kc[3, 0, 0]))
     assert abs(lse[0, 0, 0] - 0.5 * float(qk * Fraction(float(ks[3, 0])))) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# appending tokens to the paged cache
+# ----------------------------------------------------------------------------
+def _append_case(seed, P=4, Hkv=2, D=3, lens=(5, 8, 0), max_new=6):
+    rng = np.random.default_rng(seed)
+    B = len(lens)
+    npg = [-(-(L + max_new) // P) for L in lens]
+    pool = sum(npg) + 2                                  # two pages no sequence uses
+    perm = rng.permutation(pool)
+    pt = np.full((B, max(npg)), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npg):
+        pt[b, :n] = perm[off:off + n]
+        off += n
+    k = rand_bf16(rng, (pool, Hkv, P, D))
+    v = rand_bf16(rng, (pool, Hkv, P, D))
+    sig = rand_bf16(rng, (pool, Hkv, D))                 # stale rows: must stay unless touched
+    kn = rand_bf16(rng, (B, max_new, Hkv, D))
+    vn = rand_bf16(rng, (B, max_new, Hkv, D))
+    return k, v, sig, pt, np.array(lens, dtype=np.int32), kn, vn
+
+
+def test_append_kv_against_positions_and_exact_means():
+    P = 4
+    k, v, sig, pt, sl, kn, vn = _append_case(90, P=P)
+    nn = np.array([3, 6, 2], dtype=np.int32)             # crosses page boundaries
+    k2, v2, sig2, sl2 = O.append_kv(k, v, sig, pt, sl, kn, vn, nn, P)
+    assert list(sl2) == list(sl + nn)
+    written = set()
+    for b in range(len(sl)):
+        for i in range(int(nn[b])):
+            pos = int(sl[b]) + i
+            page, row = divmod(pos, P)                   # position -> (logical page, row)
+            ph = int(pt[b, page])
+            assert np.array_equal(k2[ph, :, row], kn[b, i])
+            assert np.array_equal(v2[ph, :, row], vn[b, i])
+            written.add((ph, row))
+    for ph in range(k.shape[0]):                         # nothing else moved
+        for row in range(P):
+            if (ph, row) not in written:
+                assert np.array_equal(k2[ph, :, row], k[ph, :, row])
+                assert np.array_equal(v2[ph, :, row], v[ph, :, row])
+    touched = {int(pt[b, (int(sl[b]) + i) // P]) for b in range(len(sl)) for i in range(int(nn[b]))}
+    for ph in range(k.shape[0]):
+        if ph not in touched:
+            assert np.array_equal(sig2[ph], sig[ph])
+            continue
+        b, p = [(b, p) for b in range(len(sl)) for p in range(pt.shape[1]) if pt[b, p] == ph][0]
+        nval = min(P, int(sl2[b]) - p * P)
+        for h in range(k.shape[1]):
+            for d in range(k.shape[3]):
+                s = sum(bf16_fraction(k2[ph, h, j, d]) for j in range(nval))
+                want = O.f64_to_bf16_rne(np.array([float(s) / nval]))[0]
+                assert sig2[ph, h, d] == want
+
+
+def test_append_kv_in_two_parts_equals_one_and_zero_is_identity():
+    P = 4
+    k, v, sig, pt, sl, kn, vn = _append_case(91, P=P)
+    n1 = np.array([2, 1, 4], dtype=np.int32)
+    n2 = np.array([3, 5, 1], dtype=np.int32)
+    ka, va, sa_, la = O.append_kv(k, v, sig, pt, sl, kn, vn, n1 + n2, P)
+    kb, vb, sb, lb = O.append_kv(k, v, sig, pt, sl, kn, vn, n1, P)
+    kn2 = np.zeros_like(kn)
+    vn2 = np.zeros_like(vn)
+    for b in range(len(sl)):                             # the second part's tokens, shifted
+        kn2[b, :n2[b]] = kn[b, n1[b]:n1[b] + n2[b]]
+        vn2[b, :n2[b]] = vn[b, n1[b]:n1[b] + n2[b]]
+    kc, vc, sc, lc = O.append_kv(kb, vb, sb, pt, lb, kn2, vn2, n2, P)
+    assert np.array_equal(ka, kc) and np.array_equal(va, vc)
+    assert np.array_equal(la, lc)
+    # both touch the same pages (the union of the parts'), and a page only the
+    # first part touches is full before the second part starts
+    assert np.array_equal(sa_, sc)
+    k0, v0, s0, l0 = O.append_kv(k, v, sig, pt, sl, kn, vn, np.zeros(3, np.int32), P)
+    assert np.array_equal(k0, k) and np.array_equal(v0, v) and np.array_equal(s0, sig)
+    assert np.array_equal(l0, sl)
