@@ -55,7 +55,8 @@ __all__ = [
     "bf16_to_f64", "f64_to_bf16_rne", "e4m3_to_f64", "page_budget", "exact_dots",
     "page_summaries", "page_summaries_fp8", "page_scores", "rank_select", "select_pages",
     "select_pages_mla", "sparse_attention", "sparse_attention_fp8", "masked_dense_attention",
-    "combine", "block_union", "append_kv", "NEG_INF",
+    "combine", "block_union", "append_kv", "ambient_head_scores", "select_ambient_heads",
+    "NEG_INF",
 ]
 
 NEG_INF = float("-inf")
@@ -557,3 +558,58 @@ def append_kv(k_bits, v_bits, sig_bits, page_table, seq_lens, k_new_bits, v_new_
         ph = int(pt[b, p])
         sig[ph] = fresh[ph]
     return k, v, sig, new_lens.astype(np.int32)
+
+
+# --------------------------------------------------------------------------
+# R16: the ambient head set ([TS] "Motivation": the Ambient Tier is computed
+# with h heads; "Configuration": an AutoTuner picks them per layer by
+# estimated attention-mass coverage)
+# --------------------------------------------------------------------------
+def ambient_head_scores(q_bits, sig_bits, page_table, seq_lens, crit_lists, crit_counts,
+                        amb_lists, amb_counts, scale: float, page_size: int):
+    """Estimated attention-mass coverage of the ambient pages per head (R16).
+
+    For sequence b, query token t and head h, page p of the sequence (all
+    N_b pages, one latent kv head) carries the estimated mass
+    m_p = n_p * exp(scale * (q[b,t,h] . sigma_p)), n_p its valid tokens: every
+    key of the page replaced by the page's mean key.  The coverage of (b, t, h)
+    is sum over ambient pages of m_p / sum over all pages of m_p; a head's score
+    is the sum of its coverages over b and t.  Dots are the exact ones rounded to
+    float64 (exact_dots), the rest float64.  Returns scores [Hq] float64."""
+    q = bf16_to_f64(q_bits)
+    sig = np.asarray(sig_bits, dtype=np.uint16)
+    pt = np.asarray(page_table, dtype=np.int64)
+    sl = np.asarray(seq_lens, dtype=np.int64)
+    B, T, Hq, Dk = q.shape
+    P = page_size
+    scores = np.zeros(Hq, dtype=np.float64)
+    for b in range(B):
+        L = int(sl[b])
+        nb = -(-L // P)
+        if nb == 0:
+            continue
+        pages = np.arange(nb)
+        n_p = np.minimum(P, L - pages * P).astype(np.float64)
+        amb = np.zeros(nb, dtype=bool)
+        amb[np.asarray(amb_lists[b][:int(amb_counts[b])], dtype=np.int64)] = True
+        crit = np.asarray(crit_lists[b][:int(crit_counts[b])], dtype=np.int64)
+        amb[crit] = False                                   # ambient = the tier past critical
+        s = bf16_to_f64(sig[pt[b, pages], 0, :])            # [nb, Dk]
+        dots = exact_dots(q[b].reshape(T * Hq, Dk), s)      # [T*Hq, nb]
+        z = scale * dots
+        m = z.max(axis=1, keepdims=True)
+        w = n_p[None, :] * np.exp(z - m)
+        cov = w[:, amb].sum(axis=1) / w.sum(axis=1)
+        scores += cov.reshape(T, Hq).sum(axis=0)
+    return scores
+
+
+def select_ambient_heads(q_bits, sig_bits, page_table, seq_lens, crit_lists, crit_counts,
+                         amb_lists, amb_counts, scale: float, page_size: int, h: int):
+    """The h heads of largest ambient coverage (R16), ties to the lower head,
+    ascending; and the scores."""
+    sc = ambient_head_scores(q_bits, sig_bits, page_table, seq_lens, crit_lists, crit_counts,
+                             amb_lists, amb_counts, scale, page_size)
+    heads = np.arange(len(sc))
+    win = rank_select(sc, heads, h)
+    return heads[win].astype(np.int32), sc

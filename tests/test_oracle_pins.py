@@ -655,3 +655,88 @@ def test_append_kv_in_two_parts_equals_one_and_zero_is_identity():
     k0, v0, s0, l0 = O.append_kv(k, v, sig, pt, sl, kn, vn, np.zeros(3, np.int32), P)
     assert np.array_equal(k0, k) and np.array_equal(v0, v) and np.array_equal(s0, sig)
     assert np.array_equal(l0, sl)
+
+
+# ----------------------------------------------------------------------------
+# the ambient head set (reading R16: estimated attention-mass coverage)
+# ----------------------------------------------------------------------------
+def _bf16_of(x):
+    return torch.from_numpy(np.asarray(x, dtype=np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _head_case(seed, B=2, T=2, Hq=6, Dk=8, P=4, lens=(22, 13)):
+    rng = np.random.default_rng(seed)
+    npg = [-(-L // P) for L in lens]
+    pool = sum(npg)
+    perm = rng.permutation(pool)
+    pt = np.full((B, max(npg)), -1, dtype=np.int32)
+    off = 0
+    for b, n in enumerate(npg):
+        pt[b, :n] = perm[off:off + n]
+        off += n
+    sig = _bf16_of(rng.integers(-3, 4, size=(pool, 1, Dk)))   # small integers: exact shifts
+    q = _bf16_of(rng.integers(-2, 3, size=(B, T, Hq, Dk)))
+    crit = [np.array([0, 2]), np.array([1])]
+    amb = [np.array([0, 2, 3, 5]), np.array([1, 3])]            # crit + ambient, as tiered lists
+    return q, sig, pt, np.array(lens, np.int32), crit, amb, npg
+
+
+def _counts(lists):
+    return np.array([len(x) for x in lists], dtype=np.int32)
+
+
+def test_ambient_heads_equal_scores_give_the_token_share():
+    # q = 0: every page's estimated mass is its token count, so each (b, t, h)
+    # covers (ambient tokens) / (all tokens), the partial last page counted by its
+    # valid tokens; all heads tie and the h lowest win
+    q, sig, pt, sl, crit, amb, npg = _head_case(100)
+    q[:] = 0
+    P = 4
+    sc = O.ambient_head_scores(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb), 0.7, P)
+    want = 0.0
+    for b, L in enumerate(sl):
+        n = [min(P, int(L) - p * P) for p in range(npg[b])]
+        amb_only = set(amb[b].tolist()) - set(crit[b].tolist())
+        want += 2 * sum(n[p] for p in amb_only) / sum(n)          # T = 2 tokens
+    assert np.allclose(sc, want, rtol=0, atol=1e-15)
+    heads, _ = O.select_ambient_heads(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb),
+                                      0.7, P, 3)
+    assert list(heads) == [0, 1, 2]
+
+
+def test_ambient_heads_follow_where_each_head_looks():
+    # head 4 looks hard at an ambient page of each sequence, head 1 at a critical
+    # one, the others see nothing (q = 0): head 4 covers ~1, head 1 ~0
+    q, sig, pt, sl, crit, amb, npg = _head_case(101)
+    q[:] = 0
+    for b, (a_page, c_page) in enumerate(((3, 0), (3, 1))):
+        q[b, :, 4, :] = sig[pt[b, a_page], 0, :]
+        q[b, :, 1, :] = sig[pt[b, c_page], 0, :]
+    sc = O.ambient_head_scores(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb), 40.0, 4)
+    assert sc[4] > 4 - 1e-6 and sc[1] < 1e-6              # 2 sequences x 2 tokens
+    heads, _ = O.select_ambient_heads(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb),
+                                      40.0, 4, 2)
+    assert 4 in heads and 1 not in heads
+    # all heads and no head
+    assert len(O.select_ambient_heads(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb),
+                                      40.0, 4, 6)[0]) == 6
+    assert len(O.select_ambient_heads(q, sig, pt, sl, crit, _counts(crit), amb, _counts(amb),
+                                      40.0, 4, 0)[0]) == 0
+
+
+def test_ambient_heads_invariant_to_page_ids_and_a_common_key_shift():
+    q, sig, pt, sl, crit, amb, npg = _head_case(102)
+    args = (crit, _counts(crit), amb, _counts(amb), 0.9, 4)
+    base = O.ambient_head_scores(q, sig, pt, sl, *args)
+    # relabel the physical pages
+    perm = np.random.default_rng(5).permutation(sig.shape[0])
+    inv = np.argsort(perm)
+    sig2 = sig[perm]
+    pt2 = np.where(pt >= 0, inv[np.clip(pt, 0, None)], -1).astype(np.int32)
+    assert np.allclose(O.ambient_head_scores(q, sig2, pt2, sl, *args), base, rtol=1e-13, atol=0)
+    # every summary moved by the same vector c: each row's scores move by q . c
+    # on every page alike, which the softmax shares cancel (small integers: exact)
+    c = np.array([1, -2, 0, 3, 1, 0, -1, 2], dtype=np.float32)
+    sig3 = _bf16_of(O.bf16_to_f64(sig) + c[None, None, :])
+    assert np.allclose(O.ambient_head_scores(q, sig3, pt, sl, *args), base, rtol=1e-12, atol=0)
