@@ -353,12 +353,13 @@ def _softmax_attend(s: np.ndarray, V: np.ndarray):
 
 
 def sparse_attention(q_bits, k_bits, v_bits, page_table, seq_lens, lists, counts, head_to_list,
-                     scale: float, page_size: int, rows=None):
+                     scale: float, page_size: int, rows=None, q_pos=None):
     """O [B,T,Hq,Dv] and lse [B,T,Hq] (float64) of softmax attention over the
     keys of each head's page list (reading R6 for the causal positions, R5 for
     the kv head).  Keys are the list's tokens at positions < L_b and <= the
-    query's position L_b - T + t.  s_j = scale * q . k_j; an empty key set gives
-    O = 0, lse = -inf.
+    query's position L_b - T + t (or q_pos[b] + t when the positions are given:
+    a prompt chunk computed while the cache already holds tokens past it).
+    s_j = scale * q . k_j; an empty key set gives O = 0, lse = -inf.
 
     q_bits [B,T,Hq,Dk]; k_bits [P_pool,Hkv,P,Dk]; v_bits [P_pool,Hkv,P,Dv];
     lists [B,n_lists,max_list] logical page ids; counts [B,n_lists];
@@ -370,7 +371,7 @@ def sparse_attention(q_bits, k_bits, v_bits, page_table, seq_lens, lists, counts
     return _sparse_attention(q_bits, lambda phys, kvh: bf16_to_f64(k_bits[phys, kvh]),
                              lambda phys, kvh: bf16_to_f64(v_bits[phys, kvh]), k_bits.shape[1],
                              v_bits.shape[-1], page_table, seq_lens, lists, counts,
-                             head_to_list, scale, page_size, rows)
+                             head_to_list, scale, page_size, rows, q_pos)
 
 
 def sparse_attention_fp8(q_bits, k_codes, k_scale, v_codes, v_scale, page_table, seq_lens, lists,
@@ -387,7 +388,7 @@ def sparse_attention_fp8(q_bits, k_codes, k_scale, v_codes, v_scale, page_table,
 
 
 def _sparse_attention(q_bits, k_of, v_of, Hkv, Dv, page_table, seq_lens, lists, counts,
-                      head_to_list, scale, page_size, rows):
+                      head_to_list, scale, page_size, rows, q_pos=None):
     q = bf16_to_f64(q_bits)
     pt = np.asarray(page_table, dtype=np.int64)
     sl = np.asarray(seq_lens, dtype=np.int64)
@@ -418,7 +419,7 @@ def _sparse_attention(q_bits, k_of, v_of, Hkv, Dv, page_table, seq_lens, lists, 
                 hs = [h for h in heads if want is None or (b, t, h) in want]
                 if not hs:
                     continue
-                qpos = Lb - T + t
+                qpos = (Lb - T if q_pos is None else int(q_pos[b])) + t
                 s = scale * (q[b, t, hs, :] @ K.T) if len(pos) else np.zeros((len(hs), 0))
                 s = np.where((pos <= qpos)[None, :], s, NEG_INF) if len(pos) else s
                 o, lse = _softmax_attend(s, V)

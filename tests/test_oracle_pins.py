@@ -305,6 +305,41 @@ def test_dense_budget_equals_sdpa(T, scale_mult):
         np.testing.assert_allclose(lse[b].T, scipy.special.logsumexp(s, axis=-1), rtol=0, atol=1e-12)
 
 
+def test_explicit_query_positions_equal_sdpa_with_their_mask():
+    # query token t of sequence b at q_pos[b] + t (a prompt chunk inside the
+    # cache, one past its end, one partly before its start): full budget against
+    # the library's attention with the mask those positions define
+    T = 3
+    rng = np.random.default_rng(37)
+    q, k, v, pt, sl, npages = _attn_case(rng, B=3, T=T, lens=(23, 14, 9))
+    B, _, Hq, D = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    P = 4
+    lists = np.full((B, Hkv, max(npages)), -1, dtype=np.int32)
+    counts = np.zeros((B, Hkv), dtype=np.int32)
+    for b in range(B):
+        lists[b, :, :npages[b]] = np.arange(npages[b])
+        counts[b] = npages[b]
+    q_pos = np.array([int(sl[0]) // 2, int(sl[1]) + 5, -1][:B], dtype=np.int32)
+    scale = 1.0 / math.sqrt(D)
+    o, lse = O.sparse_attention(q, k, v, pt, sl, lists, counts, np.arange(Hq) // G, scale, P,
+                                q_pos=q_pos)
+    for b in range(B):
+        L = int(sl[b])
+        phys = pt[b, :npages[b]]
+        K = torch.from_numpy(O.bf16_to_f64(k[phys]).transpose(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :L])
+        V = torch.from_numpy(O.bf16_to_f64(v[phys]).transpose(1, 0, 2, 3).reshape(Hkv, -1, D)[:, :L])
+        Q = torch.from_numpy(O.bf16_to_f64(q[b]).transpose(1, 0, 2))
+        mask = torch.arange(L)[None, :] <= (int(q_pos[b]) + torch.arange(T))[:, None]
+        seen = mask.any(dim=1).numpy()
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            Q, K.repeat_interleave(G, 0), V.repeat_interleave(G, 0), attn_mask=mask, scale=scale)
+        got = o[b].transpose(1, 0, 2)
+        np.testing.assert_allclose(got[:, seen], ref.numpy()[:, seen], rtol=0, atol=1e-12)
+        assert np.all(got[:, ~seen] == 0) and np.all(np.isneginf(lse[b][~seen]))
+
+
 @pytest.mark.parametrize("T", [1, 2])
 def test_sparse_equals_masked_dense(T):
     rng = np.random.default_rng(40 + T)
