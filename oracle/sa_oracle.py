@@ -20,6 +20,9 @@ Sources (page title, then section):
           CPU: A Cache-Aware and Load-Balanced Scheduling Kernel for Prefill"):
           Block-Union KV Selection, Q-block union + intra-group union into
           GQA-aware per-group KV block tables, blocks used in place.
+  [SPIN]  SPIN abstract (on the page titled "Vortex: Efficient and
+          Programmable Sparse Attention Serving for AI Agents"): a two-level
+          hierarchical page-metadata layout sized to the active working set.
 
 Readings where the pages are silent (each also listed in the design notes):
   R1 page budget: n_sink = ceil(sink/P), n_local = ceil(local/P),
@@ -44,6 +47,14 @@ Readings where the pages are silent (each also listed in the design notes):
      K and V pages stored as FP8 E4M3 codes with one float32 scale per
      (physical page, kv head); a key is e4m3(code) * scale, likewise a value.
      Attention and summaries are those of the dequantized pages.
+  R19 two-level page map ([SPIN] abstract on the page titled "Vortex:
+     Efficient and Programmable Sparse Attention Serving for AI Agents": page
+     metadata in two levels sized to the working set): a directory
+     [B, n_dir] of block ids and blocks [n_blocks, 2^e] of physical page
+     ids; logical page p of sequence b is blocks[dir[b, p >> e], p mod 2^e],
+     and a directory entry that names no block gives no page (-1).  Every
+     computation over such a map is the flat computation over the table it
+     defines.
 """
 from __future__ import annotations
 
@@ -56,7 +67,7 @@ __all__ = [
     "page_summaries", "page_summaries_fp8", "page_scores", "rank_select", "select_pages",
     "select_pages_mla", "sparse_attention", "sparse_attention_fp8", "masked_dense_attention",
     "combine", "block_union", "append_kv", "ambient_head_scores", "select_ambient_heads",
-    "NEG_INF",
+    "page_table_from_dir", "NEG_INF",
 ]
 
 NEG_INF = float("-inf")
@@ -521,6 +532,26 @@ def block_union(scores, Hkv: int, q_block_offset: int, top_k: int, n_sink_blocks
         tables[g, :len(ids)] = ids
         counts[g] = len(ids)
     return tables, counts
+
+
+# --------------------------------------------------------------------------
+# R19: the two-level page map ([SPIN]: metadata sized to the working set)
+# --------------------------------------------------------------------------
+def page_table_from_dir(page_dir, page_blocks, block_shift: int) -> np.ndarray:
+    """The flat page table [B, n_dir * 2^e] a two-level map defines (e =
+    block_shift): entry (b, p) is page_blocks[page_dir[b, p >> e], p mod 2^e]
+    when that directory entry is a block id in [0, n_blocks), else -1."""
+    d = np.asarray(page_dir, dtype=np.int64)
+    blk = np.asarray(page_blocks, dtype=np.int64).reshape(-1, 1 << block_shift)
+    n_blocks = blk.shape[0]
+    B, n_dir = d.shape
+    width = 1 << block_shift
+    out = np.full((B, n_dir * width), -1, dtype=np.int32)
+    for b in range(B):
+        for j in range(n_dir):
+            if 0 <= d[b, j] < n_blocks:
+                out[b, j * width:(j + 1) * width] = blk[d[b, j]]
+    return out
 
 
 # --------------------------------------------------------------------------

@@ -84,9 +84,10 @@ def test_bf16_rne_against_bruteforce():
 
 
 # ----------------------------------------------------------------------------
-# page budget (the workload statements, tests/golden/page_budget.txt)
+# page budget (tests/golden/page_budget.txt: the tiny workload's stated counts,
+# and reading R1's counts for the other two budgets worked out by hand)
 # ----------------------------------------------------------------------------
-def test_page_budget_matches_workload_statements():
+def test_page_budget_matches_golden_counts():
     rows = []
     for line in open(f"{GOLDEN}/page_budget.txt"):
         line = line.split("#")[0].strip()
@@ -95,6 +96,81 @@ def test_page_budget_matches_workload_statements():
     assert len(rows) == 3
     for sink, local, budget, P, n_sink, n_local, pages, k_top in rows:
         assert O.page_budget(sink, local, budget, P) == (n_sink, n_local, pages, k_top)
+
+
+# ----------------------------------------------------------------------------
+# two-level page map (reading R19)
+# ----------------------------------------------------------------------------
+def _read_page_dir_golden():
+    sections, cur, shift = {}, None, None
+    for line in open(f"{GOLDEN}/page_dir.txt"):
+        line = line.split("#")[0].strip()
+        if not line:
+            continue
+        if line.startswith("shift"):
+            shift = int(line.split()[1])
+        elif line in ("dir", "blocks", "table"):
+            cur = sections.setdefault(line, [])
+        else:
+            cur.append([int(x) for x in line.split()])
+    return shift, {k: np.array(v, dtype=np.int32) for k, v in sections.items()}
+
+
+def test_page_dir_golden_worked_example():
+    shift, g = _read_page_dir_golden()
+    got = O.page_table_from_dir(g["dir"], g["blocks"], shift)
+    assert got.dtype == np.int32 and got.shape == g["table"].shape
+    assert np.array_equal(got, g["table"])
+
+
+def _pack_dir(table, shift, rng):
+    """A two-level map holding a flat table: one block per run of 2^shift
+    columns that has any page, blocks numbered in a shuffled order."""
+    B, W = table.shape
+    width = 1 << shift
+    n_dir = -(-W // width)
+    padded = np.full((B, n_dir * width), -1, dtype=np.int32)
+    padded[:, :W] = table
+    used = [(b, j) for b in range(B) for j in range(n_dir)
+            if (padded[b, j * width:(j + 1) * width] >= 0).any()]
+    order = rng.permutation(len(used))
+    page_dir = np.full((B, n_dir), -1, dtype=np.int32)
+    blocks = np.full((max(len(used), 1), width), -1, dtype=np.int32)
+    for (b, j), bid in zip(used, order):
+        page_dir[b, j] = bid
+        blocks[bid] = padded[b, j * width:(j + 1) * width]
+    return page_dir, blocks, padded
+
+
+@pytest.mark.parametrize("shift", [0, 1, 3, 5])
+def test_page_dir_holds_any_flat_table(shift):
+    # a flat table packed into blocks by the inverse construction comes back
+    # unchanged; the metadata is the directory plus the used blocks only
+    rng = np.random.default_rng(40 + shift)
+    lens = [0, 1, 37, 200, 64]
+    W = max(lens)
+    table = np.full((len(lens), W), -1, dtype=np.int32)
+    ids = rng.permutation(sum(lens)).astype(np.int32)
+    off = 0
+    for b, n in enumerate(lens):
+        table[b, :n] = ids[off:off + n]
+        off += n
+    page_dir, blocks, padded = _pack_dir(table, shift, rng)
+    assert np.array_equal(O.page_table_from_dir(page_dir, blocks, shift), padded)
+    width = 1 << shift
+    assert blocks.shape[0] == sum(-(-n // width) for n in lens)
+
+
+def test_page_dir_block_numbering_is_irrelevant():
+    # renumbering the blocks (and the directory with them) changes nothing
+    shift, g = _read_page_dir_golden()
+    perm = np.array([2, 0, 1])                 # new id of old block i
+    blocks = np.empty_like(g["blocks"])
+    blocks[perm] = g["blocks"]
+    d = g["dir"].copy()
+    ok = (d >= 0) & (d < len(perm))
+    d[ok] = perm[d[ok]]
+    assert np.array_equal(O.page_table_from_dir(d, blocks, shift), g["table"])
 
 
 # ----------------------------------------------------------------------------
