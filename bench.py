@@ -78,11 +78,19 @@ def parse():
     ap.add_argument("--splits", type=int, default=0, help="decode split count (0 = default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="distinct layer caches the Llama-8B-shaped steps cycle (0 = %d); "
+                         "1 keeps a profiler capture to one 2 GiB cache" % GQA_LAYERS)
     ap.add_argument("--workload", default="all",
-                    choices=["all", "llama8b", "llama70b", "mla", "prefill", "llama8b_fp8"],
+                    choices=["all", "llama8b", "llama70b", "mla", "prefill", "llama8b_fp8",
+                             "dir_1m"],
                     help="all (default): the Llama-8B headline line with every other workload "
                          "in its `workloads` object; otherwise one workload's line alone")
     return ap.parse_args()
+
+
+def gqa_layers(args):
+    return args.layers if args.layers > 0 else GQA_LAYERS
 
 
 def peaks():
@@ -539,6 +547,114 @@ def run_gqa(cfg, args, dev, world, rank, clk, K, fp8=False, n_layers=GQA_LAYERS)
 
 
 # ---------------------------------------------------------------------------
+# million-token page tables: the step over a two-level page map, and the same
+# step over the flat table it stands for
+# ---------------------------------------------------------------------------
+def run_dir(args, dev, world, rank, clk, K):
+    import torch
+
+    import paged_sparse_kv_sa_b200 as sa
+    from paged_sparse_kv_sa_b200 import workloads as W
+
+    sa.load()
+    cfg, shift = W.LLAMA8B_DIR_1M, W.DIR_BLOCK_SHIFT
+    stream = torch.cuda.current_stream(dev)
+    n_splits = gqa_splits(cfg, args)
+    inp = W.gqa_decode_inputs(cfg, seed=args.seed + 1000 * rank, device=dev)
+    page_dir, blocks = W.page_directory(inp["page_table"], inp["seq_lens"], cfg.page_size, shift,
+                                        seed=args.seed + 1000 * rank)
+    pt = inp["page_table"]
+    q, k, v, sl = inp["q"], inp["k"], inp["v"], inp["seq_lens"]
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    sig = sa.sa_build_page_summaries_dir(k, page_dir, blocks, shift, sl, dev_error=err)
+    scale = 1.0 / math.sqrt(cfg.D)
+    bp = cfg.budget_tokens // cfg.page_size
+    outs = {}
+    for name in ("dir", "flat"):
+        cap = sa.dir_capacity(page_dir, shift) if name == "dir" else pt.shape[1]
+        n_ws = sa.sa_sparse_step_workspace_size(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D,
+                                                cfg.page_size, cap, cfg.budget_tokens, n_splits)
+        outs[name] = dict(
+            pages=torch.empty((cfg.B, cfg.Hkv, bp), dtype=torch.int32, device=dev),
+            counts=torch.empty((cfg.B, cfg.Hkv), dtype=torch.int32, device=dev),
+            o=torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.D), dtype=torch.float32, device=dev),
+            lse=torch.empty((cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev),
+            ws=torch.empty(n_ws, dtype=torch.uint8, device=dev))
+
+    def step(name):
+        r = outs[name]
+        common = dict(n_splits=n_splits, out_pages=r["pages"], out_counts=r["counts"],
+                      o_out=r["o"], lse_out=r["lse"], workspace=r["ws"], dev_error=err)
+        if name == "dir":
+            sa.sa_sparse_step_dir(q, sig, k, v, page_dir, blocks, shift, sl, cfg.page_size,
+                                  cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens, scale,
+                                  **common)
+        else:
+            sa.sa_sparse_step(q, sig, k, v, pt, sl, cfg.page_size, cfg.sink_tokens,
+                              cfg.local_tokens, cfg.budget_tokens, scale, **common)
+
+    flush = Flusher(dev)
+    with clk.busy():
+        for _ in range(max(args.warmup, 3)):
+            step("dir")
+            step("flat")
+        torch.cuda.synchronize()
+        graphs = {n: capture(sa.bind(lambda n=n: step(n))) for n in ("dir", "flat")}
+        for g in graphs.values():
+            for _ in range(3):
+                g.replay()
+        t = {n: time_isolated(graphs[n], K, flush, stream) for n in ("dir", "flat")}
+    del flush
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0, "device error flag set"
+    same = all(torch.equal(outs["dir"][x], outs["flat"][x]) for x in ("pages", "counts", "o",
+                                                                       "lse"))
+    r = outs["dir"]
+    kv = selected_kv_bytes(r["counts"], r["pages"], sl, cfg.page_size, cfg.D)
+    n_pages = ((sl.to(torch.int64) + cfg.page_size - 1) // cfg.page_size)
+    tot_pages = int(n_pages.sum().item())
+    sig_bytes = tot_pages * cfg.Hkv * cfg.D * 2
+    map_bytes_dir = page_dir.numel() * 4 + blocks.numel() * 4
+    map_bytes_flat = pt.numel() * 4
+    alg = (sig_bytes + kv + q.numel() * 2 + r["o"].numel() * 4 + r["lse"].numel() * 4 +
+           map_bytes_dir + r["pages"].numel() * 4 + r["counts"].numel() * 4)
+    t_dir = max_over_ranks(t["dir"], world, dev)
+    t_flat = max_over_ranks(t["flat"], world, dev)
+    pk, peak_kind = peaks()
+    hbm = pk["hbm_gbs"]
+    achieved = alg / t_dir / 1e9
+    return {
+        "metric": "sparse-attn calls/sec over million-token page tables (two-level page map)",
+        "value": round(world / t_dir, 2), "unit": "calls/s", "steps": K,
+        "ms_per_step": round(1e3 * t_dir, 4),
+        "config": {"workload": cfg.name, "B": cfg.B,
+                   "seq_len": f"U[{cfg.seq_len_lo},{cfg.seq_len_hi}]",
+                   "seq_lens": [int(x) for x in sl.tolist()], "Hq": cfg.Hq, "Hkv": cfg.Hkv,
+                   "D": cfg.D, "page_size": cfg.page_size, "budget_tokens": cfg.budget_tokens,
+                   "sink_tokens": cfg.sink_tokens, "local_tokens": cfg.local_tokens,
+                   "n_splits": n_splits, "block_pages": 1 << shift,
+                   "page_map_bytes": {"two_level": map_bytes_dir, "flat": map_bytes_flat},
+                   "l2": "L2 flushed before every timed step (each step alone, event-timed)",
+                   "parallelism": f"replicas x{world}"},
+        "flat_table_ms_per_step": round(1e3 * t_flat, 4),
+        "two_level_vs_flat": round(t_dir / t_flat, 4),
+        "same_bits_as_flat": bool(same),
+        "summary_bytes_scored_per_step": sig_bytes,
+        "selected_kv_bytes_per_step": kv,
+        "roofline": {"kernel": "whole step (score, choose, decode, combine)", "bound": "hbm",
+                     "achieved": round(achieved, 2), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4),
+                     "peak_kind": f"{peak_kind} (copy bandwidth)", "traffic": None,
+                     "alg_bytes_per_launch": alg,
+                     "alg_bytes_what": "summaries of every page of every sequence + selected "
+                                       "valid K+V + q + final O and LSE (float32) + directory "
+                                       "and blocks + selection outputs",
+                     "step_us": round(1e6 * t_dir, 2)},
+        "gpu_launches": 4 * K * 2,
+    }
+
+
+# ---------------------------------------------------------------------------
 # MLA + MTP tiered decode: a graph of 61 layer calls over distinct caches
 # ---------------------------------------------------------------------------
 def run_mla(args, dev, world, rank, clk, reps):
@@ -909,7 +1025,7 @@ def run_reference(args, dev, cores):
     gbs, n, dt = time_oracle(cfg, prepared, fp8, 0.0, n_steps=args.steps)
     with blas_threads(1):
         gbs1, n1, dt1 = time_oracle(cfg, prepared, fp8, 0.0, n_steps=min(args.steps, 16))
-    n_layers = GQA_LAYERS if cfg is W.LLAMA8B_DECODE else 1
+    n_layers = gqa_layers(args) if cfg is W.LLAMA8B_DECODE else 1
     line = {"metric": METRIC, "value": round(gbs, 6), "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(1000 * dt / args.steps, 3), "higher_is_better": True,
@@ -940,7 +1056,7 @@ def main():
             return                  # the oracle arm runs on rank 0 only
         dev = torch.device("cuda", local)
         torch.cuda.set_device(dev)
-        if args.workload in ("mla", "prefill"):
+        if args.workload in ("mla", "prefill", "dir_1m"):
             print(json.dumps({"impl": "reference", "unavailable":
                               "the oracle arm is timed on the GQA decode workloads"}))
             return
@@ -960,9 +1076,10 @@ def main():
     K = args.steps
     wl = args.workload
     try:
-        if wl in ("mla", "prefill"):
+        if wl in ("mla", "prefill", "dir_1m"):
             sub = (run_mla(args, dev, world, rank, clk, reps=max(1, -(-K // MLA_LAYERS)))
-                   if wl == "mla" else run_prefill(args, dev, world, rank, clk, K))
+                   if wl == "mla" else run_prefill(args, dev, world, rank, clk, K)
+                   if wl == "prefill" else run_dir(args, dev, world, rank, clk, K))
             line = {"metric": METRIC, "n_gpus": world, "warmup": args.warmup,
                     "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                     "dtype": "bf16", "data": "synthetic", **sub}
@@ -970,7 +1087,7 @@ def main():
             cfg = {"llama70b": W.LLAMA70B_LONG}.get(wl, W.LLAMA8B_DECODE)
             fp8 = wl == "llama8b_fp8"
             line = run_gqa(cfg, args, dev, world, rank, clk, K, fp8=fp8,
-                           n_layers=GQA_LAYERS if cfg is W.LLAMA8B_DECODE else 1)
+                           n_layers=gqa_layers(args) if cfg is W.LLAMA8B_DECODE else 1)
             layers = line.pop("_layers")
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 line["cpu_baseline"] = cpu_baseline(cfg, layers[0]["inp"], fp8, cores)
@@ -990,6 +1107,8 @@ def main():
                 subs["mla"] = run_mla(args, dev, world, rank, clk, reps=max(2, -(-K // 61)))
                 torch.cuda.empty_cache()
                 subs["prefill"] = run_prefill(args, dev, world, rank, clk, min(K, 20))
+                torch.cuda.empty_cache()
+                subs["dir_1m"] = run_dir(args, dev, world, rank, clk, min(K, 20))
                 for s in subs.values():
                     for k_ in ("metric", "n_gpus", "warmup", "higher_is_better", "scaling",
                                "vs_baseline", "dtype", "data"):

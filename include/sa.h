@@ -23,6 +23,16 @@
  *    means the router scores (all referenced pages / the pages an append
  *    changed)
  *    (UAE "Content-Dependent Dynamic Routing", mean(k_blocks)).
+ *  - sa_sparse_attention / sa_sparse_step: decode + merge, and selection +
+ *    decode + merge, in one call each.
+ *  - sa_append_kv: new tokens written into their pages and those pages'
+ *    summaries recomputed, in one launch.
+ *  - sa_select_ambient_heads: the ambient head set by estimated attention-mass
+ *    coverage (TileSparse's AutoTuner objective).
+ *  - sa_sparse_decode_at / sa_sparse_attention_at: query tokens at explicit
+ *    positions (a prompt chunk computed against a longer cache).
+ *  - *_dir: the same calls over a two-level page map sized to the pages in
+ *    use (SPIN's two-level metadata).
  *
  * Conventions for every call:
  *  - Pointers marked (dev) are caller-owned device memory on the current
@@ -186,6 +196,41 @@ SA_API int sa_select_pages_tiered(const uint16_t* q, const int64_t q_strides[4],
 SA_API size_t sa_select_tiered_workspace_size(int B, int T, int Hq, int max_pages);
 
 /*
+ * sa_select_ambient_heads — the h query heads that attend the ambient tier
+ * ("TileSparse: Arithmetic-Intensity-Aware Sparse Attention for Compute-Bound
+ * LLM Decoding", "Motivation": the Ambient Tier is computed with h heads;
+ * "Configuration": an AutoTuner picks them per layer by estimated
+ * attention-mass coverage).  This library's reading of that coverage: for
+ * sequence b, query token t and head h, page p carries the estimated mass
+ * n_p * exp(scale * (q[b,t,h] . sigma_p)) (n_p its valid tokens, sigma_p its
+ * summary: each key replaced by the page's mean); the coverage is the share of
+ * the sequence's estimated mass on its ambient pages (in lists[b,1] and not in
+ * lists[b,0]); a head's score sums its coverages over every b and t.  The h
+ * heads of largest score win, ties to the lower head.  A calibration call (once
+ * per layer and traffic sample): pass the chosen heads to sa_sparse_decode as
+ * head_to_list[h] = 1 for them, 0 for the others.
+ *
+ *  q, summaries, page_table, seq_lens   as sa_select_pages_tiered
+ *  lists      (dev) [B,2,list_cap] int32, list_counts (dev) [B,2]: the output of
+ *             sa_select_pages_tiered (critical pages; critical + ambient pages)
+ *  scale      the attention scale (finite)
+ *  out_heads  (dev) [h] int32: the chosen heads, ascending
+ *  out_scores (dev, optional) [Hq] float64: every head's score
+ *  workspace  (dev) sa_select_ambient_heads_workspace_size(B,T,Hq,max_pages)
+ *             bytes, 8-byte aligned
+ * Dot products in float64 from exact bf16 products, masses and scores in
+ * float64.  Supported: Dk <= 768, Hq <= 1024.
+ */
+SA_API size_t sa_select_ambient_heads_workspace_size(int B, int T, int Hq, int max_pages);
+SA_API int sa_select_ambient_heads(const uint16_t* q, const int64_t q_strides[4],
+                                   const uint16_t* summaries, const int32_t* page_table,
+                                   int max_pages, const int32_t* seq_lens, const int32_t* lists,
+                                   const int32_t* list_counts, int list_cap, int B, int T, int Hq,
+                                   int Dk, int page_size, int P_pool, float scale, int h,
+                                   int32_t* out_heads, double* out_scores, void* workspace,
+                                   size_t workspace_bytes, int32_t* dev_error, void* stream);
+
+/*
  * sa_sparse_decode — split-KV attention over per-head page lists.
  *
  * Query row (b, t, h) attends the keys of list l = head_to_list[h] of
@@ -264,6 +309,44 @@ SA_API int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4],
                                 int32_t* dev_error, void* stream);
 
 /*
+ * sa_sparse_decode_at / sa_sparse_attention_at — sa_sparse_decode and
+ * sa_sparse_attention with the query positions given explicitly: query token t
+ * of sequence b sits at position q_pos[b] + t and sees the listed keys at
+ * positions below seq_lens[b] and at most its own.  (The other calls put the
+ * queries at the end of the sequence, q_pos[b] = seq_lens[b] - T.)  For a chunk
+ * of a prompt computed while the cache already holds tokens past it -- chunked
+ * prefill over block tables used in place (CompactAttention abstract, on the
+ * page titled "Causal Attention on CPU: A Cache-Aware and Load-Balanced
+ * Scheduling Kernel for Prefill").  A token whose position is at or past
+ * seq_lens[b] sees every listed key; one before every listed key sees none
+ * (O = 0, LSE = -inf).
+ *
+ *  q_pos (dev) [B] int32 (required).  Every other argument as sa_sparse_decode
+ *  (resp. sa_sparse_attention).
+ */
+SA_API int sa_sparse_decode_at(const uint16_t* q, const int64_t q_strides[4],
+                               const uint16_t* k_cache, const int64_t k_strides[4],
+                               const uint16_t* v_cache, const int64_t v_strides[4],
+                               const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                               const int32_t* q_pos, const int32_t* lists,
+                               const int32_t* list_counts, int n_lists, int max_list,
+                               const int32_t* head_to_list, int B, int T, int Hq, int Hkv, int Dk,
+                               int Dv, int page_size, int P_pool, float scale, int n_splits,
+                               float* o_partial, float* lse_partial, int32_t* dev_error,
+                               void* stream);
+SA_API int sa_sparse_attention_at(const uint16_t* q, const int64_t q_strides[4],
+                                  const uint16_t* k_cache, const int64_t k_strides[4],
+                                  const uint16_t* v_cache, const int64_t v_strides[4],
+                                  const int32_t* page_table, int max_pages,
+                                  const int32_t* seq_lens, const int32_t* q_pos,
+                                  const int32_t* lists, const int32_t* list_counts, int n_lists,
+                                  int max_list, const int32_t* head_to_list, int B, int T, int Hq,
+                                  int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
+                                  int n_splits, float* o_out, uint16_t* o_out_bf16, float* lse_out,
+                                  void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                  void* stream);
+
+/*
  * sa_combine — merge split partials: lse = log sum_s exp(lse_s),
  * O = sum_s exp(lse_s - lse) O_s; splits with lse_s = -inf weigh nothing
  * (their O rows are not used, whatever they hold);
@@ -294,8 +377,8 @@ SA_API int sa_combine(const float* o_partial, const float* lse_partial, int n_sp
  *  o_out_bf16 (dev, optional) [B,T,Hq,Dv] bf16, 8-byte aligned
  *  lse_out    (dev, optional) [B,T,Hq] float32
  *  workspace  (dev) sa_sparse_attention_workspace_size(B,T,Hq,Dv,n_splits)
- *             bytes, 16-byte aligned, owned by the caller (the split partials;
- *             no initial contents needed).  Calls sharing a workspace must not
+ *             bytes, 16-byte aligned, owned by the caller (the partials; no
+ *             initial contents needed).  Calls sharing a workspace must not
  *             overlap.
  * At least one output must be given.  Errors: as sa_sparse_decode and
  * sa_combine (n_splits <= 64); SA_ERR_WORKSPACE for a missing, misaligned or
@@ -411,6 +494,96 @@ SA_API int sa_build_page_summaries_fp8(const uint8_t* k_codes, const int64_t k_s
                                        int max_pages, const int32_t* seq_lens, int B, int Hkv,
                                        int Dk, int page_size, int P_pool, uint16_t* summaries,
                                        int32_t* dev_error, void* stream);
+
+/*
+ * sa_append_kv — append tokens to the paged cache and refresh the summaries of
+ * the pages they land in, in one launch ("Universal Attention Engine —
+ * Declarative Sparse Attention for Production", "Content-Dependent Dynamic
+ * Routing": the router scores mean(k_blocks), so a block's mean changes when
+ * tokens land in it; "Architecture": a PagedAttention-compatible cache).
+ *
+ * Sequence b appends n_new[b] tokens: token i (i < n_new[b]) of k_new and v_new
+ * goes to position seq_lens[b] + i, i.e. row (pos % P) of physical page
+ * page_table[b, pos / P], every kv head.  Then, for every page those positions
+ * fall in, summaries[page, g, :] becomes the mean of the page's keys at
+ * positions below seq_lens[b] + n_new[b], computed as sa_build_page_summaries
+ * does (RNE_bf16(RN64(RN64(exact sum)/n))).  No other cache row or summary row
+ * changes.  The pages must already be in the page table (the caller allocates
+ * them); positions past its row are dropped and flagged (SA_DEVERR_PAGE_RANGE).
+ *
+ *  k_new, v_new (dev) [B,max_new,Hkv,D] bf16, strides kn_strides/vn_strides
+ *                     (unit feature stride, others multiples of 8, 16-byte base)
+ *  n_new        (dev) [B] int32 in [0, max_new] (outside: clamped, SA_DEVERR_COUNT)
+ *  k_cache, v_cache (dev) [P_pool,Hkv,P,D] bf16, written in place
+ *  seq_lens     (dev) [B] int32: the lengths BEFORE the append
+ *  out_seq_lens (dev, optional) [B] int32: receives seq_lens[b] + n_new[b]; must
+ *                     not be seq_lens itself (every block reads it)
+ *  summaries    (dev) [P_pool,Hkv,D] bf16, contiguous (the touched rows rewritten)
+ * D % 8 == 0.  Appends that touch the same page from two sequences race.
+ */
+SA_API int sa_append_kv(const uint16_t* k_new, const int64_t kn_strides[4], const uint16_t* v_new,
+                        const int64_t vn_strides[4], const int32_t* n_new, int max_new,
+                        uint16_t* k_cache, const int64_t k_strides[4], uint16_t* v_cache,
+                        const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                        const int32_t* seq_lens, int32_t* out_seq_lens, int B, int Hkv, int D,
+                        int page_size, int P_pool, uint16_t* summaries, int32_t* dev_error,
+                        void* stream);
+
+/*
+ * Two-level page metadata (the *_dir entry points).  SPIN ("Vortex: Efficient
+ * and Programmable Sparse Attention Serving for AI Agents", the SPIN abstract:
+ * a two-level hierarchical metadata layout sized to the active working set
+ * rather than the worst-case address space) keeps a batch's page map in two
+ * levels instead of one [B, max_pages] table:
+ *
+ *  page_dir    (dev) [B,n_dir] int32: entry j of row b is the block holding
+ *              logical pages [j << block_shift, (j + 1) << block_shift) of
+ *              sequence b, or -1 where the sequence has no pages
+ *  page_blocks (dev) [n_blocks, 1 << block_shift] int32: physical page ids
+ *
+ * Logical page p of sequence b is physical page
+ *   page_blocks[page_dir[b, p >> block_shift], p & ((1 << block_shift) - 1)],
+ * and the map holds n_dir << block_shift logical pages per sequence (the
+ * capacity that stands for max_pages).  Blocks are allocated only for the
+ * page ranges sequences use, so the metadata grows with the pages in use, not
+ * with B x the longest sequence.  A directory entry outside [0, n_blocks) for
+ * a page below ceil(seq_lens[b] / P) is reported as a physical id outside the
+ * pool (SA_DEVERR_POOL_RANGE) and that page is skipped, as a bad id of a flat
+ * table is.  0 <= block_shift <= 16, (n_dir << block_shift) <= 2^30.
+ *
+ * Every *_dir entry point computes exactly what its flat counterpart computes
+ * on the table this map defines (same kernels, same bits): arguments and
+ * errors as that counterpart, with (page_dir, n_dir, page_blocks, n_blocks,
+ * block_shift) in place of (page_table, max_pages).  sa_sparse_step_dir takes
+ * the workspace sa_sparse_step_workspace_size gives for max_pages = n_dir <<
+ * block_shift.
+ */
+SA_API int sa_build_page_summaries_dir(const uint16_t* k_cache, const int64_t k_strides[4],
+                                       const int32_t* page_dir, int n_dir,
+                                       const int32_t* page_blocks, int n_blocks, int block_shift,
+                                       const int32_t* seq_lens, int B, int Hkv, int Dk,
+                                       int page_size, int P_pool, uint16_t* summaries,
+                                       int32_t* dev_error, void* stream);
+SA_API int sa_sparse_step_dir(const uint16_t* q, const int64_t q_strides[4],
+                              const uint16_t* summaries, const uint16_t* k_cache,
+                              const int64_t k_strides[4], const uint16_t* v_cache,
+                              const int64_t v_strides[4], const int32_t* page_dir, int n_dir,
+                              const int32_t* page_blocks, int n_blocks, int block_shift,
+                              const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D,
+                              int page_size, int P_pool, int sink_tokens, int local_tokens,
+                              int budget_tokens, float scale, int n_splits, int32_t* out_pages,
+                              int32_t* out_counts, float* o_out, uint16_t* o_out_bf16,
+                              float* lse_out, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_error, void* stream);
+SA_API int sa_append_kv_dir(const uint16_t* k_new, const int64_t kn_strides[4],
+                            const uint16_t* v_new, const int64_t vn_strides[4],
+                            const int32_t* n_new, int max_new, uint16_t* k_cache,
+                            const int64_t k_strides[4], uint16_t* v_cache,
+                            const int64_t v_strides[4], const int32_t* page_dir, int n_dir,
+                            const int32_t* page_blocks, int n_blocks, int block_shift,
+                            const int32_t* seq_lens, int32_t* out_seq_lens, int B, int Hkv,
+                            int D, int page_size, int P_pool, uint16_t* summaries,
+                            int32_t* dev_error, void* stream);
 
 /*
  * sa_block_union — per-group KV block tables for chunked prefill.

@@ -10,5 +10,8 @@ from ._lib import (EXPORTED, LIB_PATH, SAError, bind, load, page_budget, sa_bloc
                    sa_select_workspace_size, sa_update_page_summaries,
                    sa_sparse_decode, sa_sparse_decode_fp8, sa_build_page_summaries_fp8,
                    sa_sparse_attention, sa_sparse_attention_fp8, attention_workspace,
-                   sa_sparse_step, sa_sparse_step_workspace_size)
+                   sa_sparse_step, sa_sparse_step_workspace_size, sa_append_kv,
+                   sa_select_ambient_heads, sa_sparse_decode_at, sa_sparse_attention_at,
+                   sa_build_page_summaries_dir, sa_sparse_step_dir, sa_append_kv_dir,
+                   dir_capacity)
 from .pipeline import SparseDecodeStep, default_splits  # noqa: F401

@@ -58,6 +58,24 @@ _SIGNATURES = {
     "sa_build_page_summaries_fp8": (_I, [_P, _c_i64_4, _P, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P,
                                          _P]),
     "sa_block_union": (_I, [_P, _I, _I, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_select_ambient_heads_workspace_size": (ctypes.c_size_t, [_I, _I, _I, _I]),
+    "sa_select_ambient_heads": (_I, [_P, _c_i64_4, _P, _P, _I, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                     _I, _F, _I, _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "sa_sparse_decode_at": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P, _P,
+                                 _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P,
+                                 _P]),
+    "sa_sparse_attention_at": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _P, _P,
+                                    _P, _I, _I, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P,
+                                    _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "sa_append_kv": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _c_i64_4, _P, _c_i64_4, _P, _I,
+                          _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sa_build_page_summaries_dir": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _P, _I, _I, _I, _I,
+                                         _I, _P, _P, _P]),
+    "sa_sparse_step_dir": (_I, [_P, _c_i64_4, _P, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _I, _I,
+                                _P, _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P,
+                                _P, _P, _P, ctypes.c_size_t, _P, _P]),
+    "sa_append_kv_dir": (_I, [_P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _c_i64_4, _P, _c_i64_4, _P,
+                              _I, _P, _I, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
 }
 
 EXPORTED = tuple(_SIGNATURES)
@@ -555,3 +573,210 @@ def sa_block_union(scores, Hkv: int, q_block_offset: int, top_k: int, n_sink_blo
     _call(lib.sa_block_union, (_ptr(scores), Hq, Hkv, NQB, NKB, q_block_offset, top_k,
                             n_sink_blocks, _ptr(tables), _ptr(counts), _stream(stream)), "sa_block_union")
     return tables, counts
+
+
+def sa_append_kv(k_new, v_new, n_new, k_cache, v_cache, page_table, seq_lens, summaries,
+                 out_seq_lens=None, dev_error=None, stream=None):
+    """Write sequence b's n_new[b] new tokens (k_new, v_new [B,max_new,Hkv,D] bf16) at
+    positions seq_lens[b] + i of the paged caches [P_pool,Hkv,P,D] and rewrite the
+    summaries of the pages they land in (in place).  seq_lens: lengths before the
+    append; out_seq_lens (optional, not seq_lens) receives the new lengths."""
+    lib = load()
+    _need_cuda(k_new, v_new, n_new, k_cache, v_cache, page_table, seq_lens, summaries)
+    _bf16(k_new), _bf16(v_new), _bf16(k_cache), _bf16(v_cache), _i32(n_new), _i32(page_table)
+    _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    if out_seq_lens is not None:
+        _i32(out_seq_lens)
+    B, max_new, Hkv, D = k_new.shape
+    P_pool, _, P, _ = k_cache.shape
+    _call(lib.sa_append_kv, (_ptr(k_new), _strides4(k_new), _ptr(v_new), _strides4(v_new),
+                             _ptr(n_new), max_new, _ptr(k_cache), _strides4(k_cache),
+                             _ptr(v_cache), _strides4(v_cache), _ptr(page_table),
+                             page_table.shape[1], _ptr(seq_lens), _ptr(out_seq_lens), B, Hkv, D,
+                             P, P_pool, _ptr(summaries), _ptr(dev_error), _stream(stream)),
+          "sa_append_kv")
+    return out_seq_lens
+
+
+def sa_select_ambient_heads(q, summaries, page_table, seq_lens, lists, list_counts, page_size: int,
+                            scale: float, h: int, out_heads=None, out_scores=None, workspace=None,
+                            dev_error=None, stream=None):
+    """The h heads of largest estimated ambient attention-mass coverage (ascending,
+    [h] int32) and every head's score ([Hq] float64).  lists [B,2,cap] / list_counts
+    [B,2]: sa_select_pages_tiered's output."""
+    lib = load()
+    _need_cuda(q, summaries, page_table, seq_lens, lists, list_counts)
+    _bf16(q), _i32(page_table), _i32(seq_lens), _i32(lists), _i32(list_counts)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    B, T, Hq, Dk = q.shape
+    P_pool = summaries.shape[0]
+    max_pages = page_table.shape[1]
+    if out_heads is None:
+        out_heads = torch.empty((max(h, 1),), dtype=torch.int32, device=q.device)
+    if out_scores is None:
+        out_scores = torch.empty((Hq,), dtype=torch.float64, device=q.device)
+    if workspace is None:
+        n = int(lib.sa_select_ambient_heads_workspace_size(B, T, Hq, max_pages))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _call(lib.sa_select_ambient_heads,
+          (_ptr(q), _strides4(q), _ptr(summaries), _ptr(page_table), max_pages, _ptr(seq_lens),
+           _ptr(lists), _ptr(list_counts), lists.shape[2], B, T, Hq, Dk, page_size, P_pool,
+           float(scale), int(h), _ptr(out_heads), _ptr(out_scores), _ptr(workspace),
+           workspace.numel(), _ptr(dev_error), _stream(stream)), "sa_select_ambient_heads")
+    return out_heads[:h], out_scores
+
+
+def sa_sparse_decode_at(q, k_cache, v_cache, page_table, seq_lens, q_pos, lists, list_counts,
+                        head_to_list, scale: float, n_splits: int = 1, o_partial=None,
+                        lse_partial=None, dev_error=None, stream=None):
+    """sa_sparse_decode with explicit query positions: token t of sequence b at
+    q_pos[b] + t (q_pos [B] int32 on the GPU).  Returns (o_partial, lse_partial)."""
+    lib = load()
+    _need_cuda(q, k_cache, v_cache, page_table, seq_lens, q_pos, lists, list_counts)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(page_table), _i32(seq_lens), _i32(q_pos)
+    _i32(lists), _i32(list_counts)
+    B, T, Hq, Dk = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    Dv = v_cache.shape[-1]
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    if o_partial is None:
+        o_partial = torch.empty((n_splits, B, T, Hq, Dv), dtype=torch.float32, device=q.device)
+    if lse_partial is None:
+        lse_partial = torch.empty((n_splits, B, T, Hq), dtype=torch.float32, device=q.device)
+    _call(lib.sa_sparse_decode_at,
+          (_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache), _ptr(v_cache),
+           _strides4(v_cache), _ptr(page_table), page_table.shape[1], _ptr(seq_lens), _ptr(q_pos),
+           _ptr(lists), _ptr(list_counts), n_lists, max_list, ctypes.cast(h2l, ctypes.c_void_p), B,
+           T, Hq, Hkv, Dk, Dv, P, P_pool, float(scale), n_splits, _ptr(o_partial),
+           _ptr(lse_partial), _ptr(dev_error), _stream(stream)), "sa_sparse_decode_at")
+    return o_partial, lse_partial
+
+
+def sa_sparse_attention_at(q, k_cache, v_cache, page_table, seq_lens, q_pos, lists, list_counts,
+                           head_to_list, scale: float, n_splits: int = 1, o_out=None,
+                           o_out_bf16=None, lse_out=None, want_f32: bool = True,
+                           want_bf16: bool = False, workspace=None, dev_error=None, stream=None):
+    """sa_sparse_attention with explicit query positions (q_pos [B] int32 on the GPU)."""
+    lib = load()
+    _need_cuda(q, k_cache, v_cache, page_table, seq_lens, q_pos, lists, list_counts)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(page_table), _i32(seq_lens), _i32(q_pos)
+    _i32(lists), _i32(list_counts)
+    B, T, Hq, Dk = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    Dv = v_cache.shape[-1]
+    _, n_lists, max_list = lists.shape
+    h2l = (ctypes.c_int32 * Hq)(*[int(x) for x in head_to_list])
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, Dv, q.device, o_out, o_out_bf16,
+                                               lse_out, want_f32, want_bf16)
+    if workspace is None:
+        workspace = attention_workspace(B, T, Hq, Dv, n_splits, q.device)
+    _call(lib.sa_sparse_attention_at,
+          (_ptr(q), _strides4(q), _ptr(k_cache), _strides4(k_cache), _ptr(v_cache),
+           _strides4(v_cache), _ptr(page_table), page_table.shape[1], _ptr(seq_lens), _ptr(q_pos),
+           _ptr(lists), _ptr(list_counts), n_lists, max_list, ctypes.cast(h2l, ctypes.c_void_p), B,
+           T, Hq, Hkv, Dk, Dv, P, P_pool, float(scale), n_splits, _ptr(o_out), _ptr(o_out_bf16),
+           _ptr(lse_out), _ptr(workspace), workspace.numel(), _ptr(dev_error), _stream(stream)),
+          "sa_sparse_attention_at")
+    return o_out, o_out_bf16, lse_out
+
+
+# ---------------------------------------------------------------------------
+# two-level page map: a directory [B, n_dir] of block ids over blocks
+# [n_blocks, 2^block_shift] of physical page ids, in place of a flat table
+# ---------------------------------------------------------------------------
+def _dir_args(page_dir, page_blocks, block_shift: int):
+    _i32(page_dir), _i32(page_blocks)
+    if page_dir.dim() != 2 or page_blocks.dim() != 2:
+        raise ValueError("page_dir must be [B, n_dir] and page_blocks [n_blocks, 2^block_shift]")
+    if page_blocks.shape[1] != (1 << block_shift):
+        raise ValueError("page_blocks rows must hold 2^block_shift entries")
+    return (_ptr(page_dir), page_dir.shape[1], _ptr(page_blocks), page_blocks.shape[0],
+            int(block_shift))
+
+
+def dir_capacity(page_dir, block_shift: int) -> int:
+    """Logical pages per sequence a two-level map holds (its flat max_pages)."""
+    return page_dir.shape[1] << block_shift
+
+
+def sa_build_page_summaries_dir(k_cache, page_dir, page_blocks, block_shift: int, seq_lens,
+                                summaries=None, dev_error=None, stream=None):
+    """sa_build_page_summaries over a two-level page map."""
+    lib = load()
+    _need_cuda(k_cache, page_dir, page_blocks, seq_lens)
+    _bf16(k_cache), _i32(seq_lens)
+    P_pool, Hkv, P, Dk = k_cache.shape
+    if summaries is None:
+        summaries = torch.zeros((P_pool, Hkv, Dk), dtype=torch.bfloat16, device=k_cache.device)
+    _call(lib.sa_build_page_summaries_dir,
+          (_ptr(k_cache), _strides4(k_cache), *_dir_args(page_dir, page_blocks, block_shift),
+           _ptr(seq_lens), seq_lens.shape[0], Hkv, Dk, P, P_pool, _ptr(summaries),
+           _ptr(dev_error), _stream(stream)), "sa_build_page_summaries_dir")
+    return summaries
+
+
+def sa_sparse_step_dir(q, summaries, k_cache, v_cache, page_dir, page_blocks, block_shift: int,
+                       seq_lens, page_size: int, sink_tokens: int, local_tokens: int,
+                       budget_tokens: int, scale: float, n_splits: int = 0, out_pages=None,
+                       out_counts=None, o_out=None, o_out_bf16=None, lse_out=None,
+                       want_f32: bool = True, want_bf16: bool = False, workspace=None,
+                       dev_error=None, stream=None):
+    """sa_sparse_step over a two-level page map; returns (pages, counts, O f32 or
+    None, O bf16 or None, lse)."""
+    lib = load()
+    _need_cuda(q, summaries, k_cache, v_cache, page_dir, page_blocks, seq_lens)
+    _bf16(q), _bf16(k_cache), _bf16(v_cache), _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    B, T, Hq, D = q.shape
+    P_pool, Hkv, P, _ = k_cache.shape
+    if P != page_size:
+        raise ValueError("page_size differs from the cache's page dimension")
+    dargs = _dir_args(page_dir, page_blocks, block_shift)
+    bp = budget_tokens // page_size
+    if out_pages is None:
+        out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
+    if out_counts is None:
+        out_counts = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    _select_shapes(q, summaries, page_dir, seq_lens, out_pages, out_counts, bp)
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, D, q.device, o_out, o_out_bf16,
+                                               lse_out, want_f32, want_bf16)
+    if workspace is None:
+        n = sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, page_size,
+                                          dir_capacity(page_dir, block_shift), budget_tokens,
+                                          n_splits)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _call(lib.sa_sparse_step_dir,
+          (_ptr(q), _strides4(q), _ptr(summaries), _ptr(k_cache), _strides4(k_cache),
+           _ptr(v_cache), _strides4(v_cache), *dargs, _ptr(seq_lens), B, T, Hq, Hkv, D,
+           page_size, P_pool, sink_tokens, local_tokens, budget_tokens, float(scale),
+           int(n_splits), _ptr(out_pages), _ptr(out_counts), _ptr(o_out), _ptr(o_out_bf16),
+           _ptr(lse_out), _ptr(workspace), workspace.numel(), _ptr(dev_error),
+           _stream(stream)), "sa_sparse_step_dir")
+    return out_pages, out_counts, o_out, o_out_bf16, lse_out
+
+
+def sa_append_kv_dir(k_new, v_new, n_new, k_cache, v_cache, page_dir, page_blocks,
+                     block_shift: int, seq_lens, summaries, out_seq_lens=None, dev_error=None,
+                     stream=None):
+    """sa_append_kv over a two-level page map."""
+    lib = load()
+    _need_cuda(k_new, v_new, n_new, k_cache, v_cache, page_dir, page_blocks, seq_lens, summaries)
+    _bf16(k_new), _bf16(v_new), _bf16(k_cache), _bf16(v_cache), _i32(n_new), _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    if out_seq_lens is not None:
+        _i32(out_seq_lens)
+    B, max_new, Hkv, D = k_new.shape
+    P_pool, _, P, _ = k_cache.shape
+    _call(lib.sa_append_kv_dir,
+          (_ptr(k_new), _strides4(k_new), _ptr(v_new), _strides4(v_new), _ptr(n_new), max_new,
+           _ptr(k_cache), _strides4(k_cache), _ptr(v_cache), _strides4(v_cache),
+           *_dir_args(page_dir, page_blocks, block_shift), _ptr(seq_lens), _ptr(out_seq_lens),
+           B, Hkv, D, P, P_pool, _ptr(summaries), _ptr(dev_error), _stream(stream)),
+          "sa_append_kv_dir")
+    return out_seq_lens

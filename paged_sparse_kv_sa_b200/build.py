@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsa.so")
-SOURCES = ["api.cu", "decode.cu", "prefill.cu", "mla.cu", "select.cu", "select_mla.cu", "combine.cu", "summaries.cu",
+SOURCES = ["api.cu", "decode.cu", "prefill.cu", "mla.cu", "select.cu", "select_mla.cu", "combine.cu", "summaries.cu", "append.cu", "heads.cu",
            "union.cu"]
 HEADERS = ["common.cuh", "exact.cuh", "tc05.cuh", "topk.cuh", "internal.h", os.path.join("..", "..", "include", "sa.h")]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -269,7 +269,7 @@ size_t sa_select_workspace_size(int B, int Hkv, int max_pages) {
 namespace {
 // Argument checks and argument block shared by the selection entry points.
 int select_args(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
-                const int32_t* page_table, const int32_t* seq_lens, int B, int T, int Hq, int Hkv,
+                const PageMap& pm, const int32_t* seq_lens, int B, int T, int Hq, int Hkv,
                 int Dk, int page_size, int max_pages, int P_pool, int sink_tokens,
                 int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
                 int32_t* dev_error, SelectArgs* a) {
@@ -283,7 +283,7 @@ int select_args(const uint16_t* q, const int64_t q_strides[4], const uint16_t* s
   if (k_top < 0 || budget_pages <= 0) return SA_ERR_INVALID_ARG;
   if (B == 0) return SA_OK;
   if (int r = check_q(q, q_strides)) return r;
-  if (!summaries || !page_table || !seq_lens || !out_pages || !out_counts)
+  if (!summaries || !pm.table || !seq_lens || !out_pages || !out_counts)
     return SA_ERR_INVALID_ARG;
   if (!aligned16(summaries)) return SA_ERR_INVALID_ARG;
   if (Dk != 64 && Dk != 128 && Dk != 256) return SA_ERR_UNSUPPORTED;
@@ -293,7 +293,7 @@ int select_args(const uint16_t* q, const int64_t q_strides[4], const uint16_t* s
   a->qs1 = q_strides[1];
   a->qs2 = q_strides[2];
   a->sig = summaries;
-  a->page_table = page_table;
+  a->pt = pm;
   a->seq_lens = seq_lens;
   a->B = B;
   a->T = T;
@@ -323,7 +323,8 @@ int sa_select_pages(const uint16_t* q, const int64_t q_strides[4], const uint16_
                     int local_tokens, int budget_tokens, int32_t* out_pages, int32_t* out_counts,
                     void* workspace, size_t workspace_bytes, int32_t* dev_error, void* stream) {
   SelectArgs a;
-  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
+  if (int r = select_args(q, q_strides, summaries, flat_map(page_table, max_pages), seq_lens, B,
+                          T, Hq, Hkv, Dk,
                           page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
                           out_pages, out_counts, dev_error, &a))
     return r;
@@ -342,7 +343,8 @@ int sa_select_pages_no_alloc(const uint16_t* q, const int64_t q_strides[4],
                              int local_tokens, int budget_tokens, int32_t* out_pages,
                              int32_t* out_counts, int32_t* dev_error, void* stream) {
   SelectArgs a;
-  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, Dk,
+  if (int r = select_args(q, q_strides, summaries, flat_map(page_table, max_pages), seq_lens, B,
+                          T, Hq, Hkv, Dk,
                           page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
                           out_pages, out_counts, dev_error, &a))
     return r;
@@ -417,6 +419,28 @@ int merge_outputs_ok(const MergeSpec& m) {
   return SA_OK;
 }
 
+// Workspace of a merged call: the split partials.
+struct AttnWs {
+  size_t o_bytes, lse_bytes;
+};
+AttnWs attn_ws(int B, int T, int Hq, int Dv, int n_splits) {
+  auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
+  AttnWs w;
+  const size_t rows = (size_t)B * T * Hq;
+  w.o_bytes = r16(rows * Dv * n_splits * sizeof(float));
+  w.lse_bytes = r16(rows * n_splits * sizeof(float));
+  return w;
+}
+
+// Where a decode call's partials go: the caller's o_partial / lse_partial
+// (ws null), or laid out in a merged call's workspace (n_splits slots).
+struct DecodeTarget {
+  uint8_t* ws = nullptr;
+  size_t ws_bytes = 0;
+  const int32_t* q_pos = nullptr;   // [B] query token 0's position (null: causal tail)
+  PageMap dir;                      // two-level map (dir.blocks set): page_table is its directory
+};
+
 int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
                        const int64_t k_strides[4], const uint16_t* v_cache,
                        const int64_t v_strides[4], const int32_t* page_table, int max_pages,
@@ -424,7 +448,7 @@ int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint
                        int n_lists, int max_list, const int32_t* head_to_list, int B, int T,
                        int Hq, int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
                        int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
-                       void* stream, const MergeSpec* merge) {
+                       void* stream, const MergeSpec* merge, DecodeTarget* tgt) {
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Dk <= 0 || Dv <= 0 ||
       page_size <= 0 || max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 ||
       n_splits <= 0 || !std::isfinite(scale) || !head_to_list)
@@ -433,9 +457,9 @@ int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint
   if (int r = check_q(q, q_strides)) return r;
   if (int r = check_cache(k_cache, k_strides)) return r;
   if (int r = check_cache(v_cache, v_strides)) return r;
-  if (!page_table || !seq_lens || !lists || !list_counts || !o_partial || !lse_partial)
+  if (!page_table || !seq_lens || !lists || !list_counts) return SA_ERR_INVALID_ARG;
+  if (!tgt->ws && (!o_partial || !lse_partial || !aligned16(o_partial)))
     return SA_ERR_INVALID_ARG;
-  if (!aligned16(o_partial)) return SA_ERR_INVALID_ARG;
   for (int h = 0; h < Hq; ++h)
     if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
   // MLA: keys of 576 columns whose first 512 are the values (V aliases K)
@@ -453,6 +477,12 @@ int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint
   const int cap = mla ? mla_max_split_entries(page_size)
                       : (wide ? prefill_max_split_entries() : decode_max_split_entries());
   if (!mla && wide && Dk > 128) return SA_ERR_UNSUPPORTED;
+  if (tgt->ws) {
+    const AttnWs w = attn_ws(B, T, Hq, Dv, n_splits);
+    if (tgt->ws_bytes < w.o_bytes + w.lse_bytes) return SA_ERR_WORKSPACE;
+    o_partial = reinterpret_cast<float*>(tgt->ws);
+    lse_partial = reinterpret_cast<float*>(tgt->ws + w.o_bytes);
+  }
   if ((max_list + n_splits - 1) / n_splits > cap) return SA_ERR_UNSUPPORTED;
   CUtensorMap kmap, vmap;
   // MLA tiles of 64 keys: one 64-row box per column chunk when a tile lies in one page
@@ -465,7 +495,7 @@ int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint
   a.qs0 = q_strides[0];
   a.qs1 = q_strides[1];
   a.qs2 = q_strides[2];
-  a.page_table = page_table;
+  a.pt = tgt->dir.blocks ? tgt->dir : flat_map(page_table, max_pages);
   a.max_pages = max_pages;
   a.seq_lens = seq_lens;
   a.lists = lists;
@@ -486,6 +516,7 @@ int sparse_decode_impl(const uint16_t* q, const int64_t q_strides[4], const uint
   a.lse_part = lse_partial;
   a.err = dev_error;
   a.k_scale = a.v_scale = nullptr;
+  a.q_pos = tgt->q_pos;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (merge && (n_splits > 64 || (int64_t)B * T * Hq * (Dv / 4) >= (int64_t(1) << 32)))
     return SA_ERR_UNSUPPORTED;   // the combine kernel's limits
@@ -507,7 +538,7 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
                            const int32_t* head_to_list, int B, int T, int Hq, int Hkv, int D,
                            int page_size, int P_pool, float scale, int n_splits, float* o_partial,
                            float* lse_partial, int32_t* dev_error, void* stream,
-                           const MergeSpec* merge) {
+                           const MergeSpec* merge, DecodeTarget* tgt) {
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || D <= 0 || page_size <= 0 ||
       max_pages < 0 || P_pool <= 0 || n_lists <= 0 || max_list < 0 || n_splits <= 0 ||
       !std::isfinite(scale) || !head_to_list)
@@ -516,10 +547,10 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
   if (int r = check_q(q, q_strides)) return r;
   if (int r = check_cache_u8(k_codes, k_strides)) return r;
   if (int r = check_cache_u8(v_codes, v_strides)) return r;
-  if (!k_scale || !v_scale || !page_table || !seq_lens || !lists || !list_counts || !o_partial ||
-      !lse_partial)
+  if (!k_scale || !v_scale || !page_table || !seq_lens || !lists || !list_counts)
     return SA_ERR_INVALID_ARG;
-  if (!aligned16(o_partial)) return SA_ERR_INVALID_ARG;
+  if (!tgt->ws && (!o_partial || !lse_partial || !aligned16(o_partial)))
+    return SA_ERR_INVALID_ARG;
   for (int h = 0; h < Hq; ++h)
     if (head_to_list[h] < 0 || head_to_list[h] >= n_lists) return SA_ERR_INVALID_ARG;
   if (D != 128 || page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
@@ -527,7 +558,14 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
   int max_rows = 0;
   if (int r = build_pairs(head_to_list, Hq, Hkv, T, &pairs, &max_rows)) return r;
   if (max_rows > kMaxRowsPerPair) return SA_ERR_UNSUPPORTED;
-  if ((max_list + n_splits - 1) / n_splits > decode_max_split_entries()) return SA_ERR_UNSUPPORTED;
+  if (tgt->ws) {
+    const AttnWs w = attn_ws(B, T, Hq, D, n_splits);
+    if (tgt->ws_bytes < w.o_bytes + w.lse_bytes) return SA_ERR_WORKSPACE;
+    o_partial = reinterpret_cast<float*>(tgt->ws);
+    lse_partial = reinterpret_cast<float*>(tgt->ws + w.o_bytes);
+  }
+  if ((max_list + n_splits - 1) / n_splits > decode_max_split_entries())
+    return SA_ERR_UNSUPPORTED;
   CUtensorMap kmap, vmap;
   if (!encode_kv_map_u8(&kmap, k_codes, D, page_size, Hkv, P_pool, k_strides) ||
       !encode_kv_map_u8(&vmap, v_codes, D, page_size, Hkv, P_pool, v_strides))
@@ -537,7 +575,7 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
   a.qs0 = q_strides[0];
   a.qs1 = q_strides[1];
   a.qs2 = q_strides[2];
-  a.page_table = page_table;
+  a.pt = tgt->dir.blocks ? tgt->dir : flat_map(page_table, max_pages);
   a.max_pages = max_pages;
   a.seq_lens = seq_lens;
   a.lists = lists;
@@ -559,6 +597,7 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
   a.err = dev_error;
   a.k_scale = k_scale;
   a.v_scale = v_scale;
+  a.q_pos = tgt->q_pos;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (merge && (n_splits > 64 || (int64_t)B * T * Hq * (D / 4) >= (int64_t(1) << 32)))
     return SA_ERR_UNSUPPORTED;   // the combine kernel's limits
@@ -567,19 +606,6 @@ int sparse_decode_fp8_impl(const uint16_t* q, const int64_t q_strides[4],
     e = launch_combine(o_partial, lse_partial, n_splits, (int64_t)B * T * Hq, D, merge->o_out,
                        merge->o_bf16, merge->lse_out, st);
   return cuda_status(e);
-}
-
-// Workspace of a merged call: the split partials.
-struct AttnWs {
-  size_t o_bytes, lse_bytes;
-};
-AttnWs attn_ws(int B, int T, int Hq, int Dv, int n_splits) {
-  auto r16 = [](size_t x) { return (x + 15) / 16 * 16; };
-  AttnWs w;
-  const size_t rows = (size_t)B * T * Hq;
-  w.o_bytes = r16(rows * Dv * n_splits * sizeof(float));
-  w.lse_bytes = r16(rows * n_splits * sizeof(float));
-  return w;
 }
 }  // namespace
 }  // namespace sa
@@ -594,10 +620,11 @@ int sa_sparse_decode(const uint16_t* q, const int64_t q_strides[4], const uint16
                      int Hkv, int Dk, int Dv, int page_size, int P_pool, float scale,
                      int n_splits, float* o_partial, float* lse_partial, int32_t* dev_error,
                      void* stream) {
+  DecodeTarget t;
   return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
                             max_pages, seq_lens, lists, list_counts, n_lists, max_list,
                             head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
-                            n_splits, o_partial, lse_partial, dev_error, stream, nullptr);
+                            n_splits, o_partial, lse_partial, dev_error, stream, nullptr, &t);
 }
 
 int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const uint8_t* k_codes,
@@ -608,11 +635,12 @@ int sa_sparse_decode_fp8(const uint16_t* q, const int64_t q_strides[4], const ui
                          int max_list, const int32_t* head_to_list, int B, int T, int Hq, int Hkv,
                          int D, int page_size, int P_pool, float scale, int n_splits,
                          float* o_partial, float* lse_partial, int32_t* dev_error, void* stream) {
+  DecodeTarget t;
   return sparse_decode_fp8_impl(q, q_strides, k_codes, k_strides, v_codes, v_strides, k_scale,
                                 v_scale, page_table, max_pages, seq_lens, lists, list_counts,
                                 n_lists, max_list, head_to_list, B, T, Hq, Hkv, D, page_size,
                                 P_pool, scale, n_splits, o_partial, lse_partial, dev_error, stream,
-                                nullptr);
+                                nullptr, &t);
 }
 
 size_t sa_sparse_attention_workspace_size(int B, int T, int Hq, int Dv, int n_splits) {
@@ -633,17 +661,54 @@ int sa_sparse_attention(const uint16_t* q, const int64_t q_strides[4], const uin
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || n_lists <= 0 || Dv <= 0 || n_splits <= 0)
     return SA_ERR_INVALID_ARG;
   if (B == 0) return SA_OK;
-  const AttnWs w = attn_ws(B, T, Hq, Dv, n_splits);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < w.o_bytes + w.lse_bytes)
-    return SA_ERR_WORKSPACE;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
   MergeSpec m{o_out, o_out_bf16, lse_out};
   if (int r = merge_outputs_ok(m)) return r;
+  DecodeTarget t{static_cast<uint8_t*>(workspace), workspace_bytes};
   return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
                             max_pages, seq_lens, lists, list_counts, n_lists, max_list,
                             head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
-                            n_splits, reinterpret_cast<float*>(ws),
-                            reinterpret_cast<float*>(ws + w.o_bytes), dev_error, stream, &m);
+                            n_splits, nullptr, nullptr, dev_error, stream, &m, &t);
+}
+
+int sa_sparse_decode_at(const uint16_t* q, const int64_t q_strides[4], const uint16_t* k_cache,
+                        const int64_t k_strides[4], const uint16_t* v_cache,
+                        const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                        const int32_t* seq_lens, const int32_t* q_pos, const int32_t* lists,
+                        const int32_t* list_counts, int n_lists, int max_list,
+                        const int32_t* head_to_list, int B, int T, int Hq, int Hkv, int Dk, int Dv,
+                        int page_size, int P_pool, float scale, int n_splits, float* o_partial,
+                        float* lse_partial, int32_t* dev_error, void* stream) {
+  if (!q_pos && B > 0) return SA_ERR_INVALID_ARG;
+  DecodeTarget t{nullptr, 0, q_pos};
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+                            max_pages, seq_lens, lists, list_counts, n_lists, max_list,
+                            head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
+                            n_splits, o_partial, lse_partial, dev_error, stream, nullptr, &t);
+}
+
+int sa_sparse_attention_at(const uint16_t* q, const int64_t q_strides[4],
+                           const uint16_t* k_cache, const int64_t k_strides[4],
+                           const uint16_t* v_cache, const int64_t v_strides[4],
+                           const int32_t* page_table, int max_pages, const int32_t* seq_lens,
+                           const int32_t* q_pos, const int32_t* lists, const int32_t* list_counts,
+                           int n_lists, int max_list, const int32_t* head_to_list, int B, int T,
+                           int Hq, int Hkv, int Dk, int Dv, int page_size, int P_pool,
+                           float scale, int n_splits, float* o_out, uint16_t* o_out_bf16,
+                           float* lse_out, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_error, void* stream) {
+  if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || n_lists <= 0 || Dv <= 0 || n_splits <= 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  if (!q_pos) return SA_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
+  MergeSpec m{o_out, o_out_bf16, lse_out};
+  if (int r = merge_outputs_ok(m)) return r;
+  DecodeTarget t{static_cast<uint8_t*>(workspace), workspace_bytes, q_pos};
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+                            max_pages, seq_lens, lists, list_counts, n_lists, max_list,
+                            head_to_list, B, T, Hq, Hkv, Dk, Dv, page_size, P_pool, scale,
+                            n_splits, nullptr, nullptr, dev_error, stream, &m, &t);
 }
 
 }  // extern "C"
@@ -670,35 +735,23 @@ int step_plan(int B, int T, int Hq, int Hkv, int D, int page_size, int max_pages
   *total_bytes = *sel_bytes + w.o_bytes + w.lse_bytes;
   return SA_OK;
 }
-}  // namespace
 
-extern "C" {
-
-size_t sa_sparse_step_workspace_size(int B, int T, int Hq, int Hkv, int D, int page_size,
-                                     int max_pages, int budget_tokens, int n_splits) {
-  int s = 0;
-  size_t sel = 0, total = 0;
-  if (step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &s, &sel,
-                &total) != SA_OK)
-    return 0;
-  return total;
-}
-
-int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
-                   const uint16_t* k_cache, const int64_t k_strides[4], const uint16_t* v_cache,
-                   const int64_t v_strides[4], const int32_t* page_table, int max_pages,
-                   const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D, int page_size,
-                   int P_pool, int sink_tokens, int local_tokens, int budget_tokens, float scale,
-                   int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
-                   uint16_t* o_out_bf16, float* lse_out, void* workspace,
-                   size_t workspace_bytes, int32_t* dev_error, void* stream) {
+// sa_sparse_step over either page map (max_pages: the map's capacity).
+int step_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+              const uint16_t* k_cache, const int64_t k_strides[4], const uint16_t* v_cache,
+              const int64_t v_strides[4], const PageMap& pm, int max_pages,
+              const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D, int page_size,
+              int P_pool, int sink_tokens, int local_tokens, int budget_tokens, float scale,
+              int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
+              uint16_t* o_out_bf16, float* lse_out, void* workspace, size_t workspace_bytes,
+              int32_t* dev_error, void* stream) {
   int splits = 0;
   size_t sel_bytes = 0, total = 0;
   if (int r = step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &splits,
                         &sel_bytes, &total))
     return r;
   SelectArgs sa_args;
-  if (int r = select_args(q, q_strides, summaries, page_table, seq_lens, B, T, Hq, Hkv, D,
+  if (int r = select_args(q, q_strides, summaries, pm, seq_lens, B, T, Hq, Hkv, D,
                           page_size, max_pages, P_pool, sink_tokens, local_tokens, budget_tokens,
                           out_pages, out_counts, dev_error, &sa_args))
     return r;
@@ -722,13 +775,41 @@ int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t
   sa_args.lohi = reinterpret_cast<float2*>(ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (int r = cuda_status(launch_select_gqa(sa_args, st))) return r;
-  const AttnWs w = attn_ws(B, T, Hq, D, splits);
-  uint8_t* parts = ws + sel_bytes;
-  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, page_table,
+  DecodeTarget t{ws + sel_bytes, total - sel_bytes};
+  if (pm.blocks) t.dir = pm;
+  return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, pm.table,
                             max_pages, seq_lens, out_pages, out_counts, Hkv, budget_pages, h2l, B,
-                            T, Hq, Hkv, D, D, page_size, P_pool, scale, splits,
-                            reinterpret_cast<float*>(parts),
-                            reinterpret_cast<float*>(parts + w.o_bytes), dev_error, stream, &m);
+                            T, Hq, Hkv, D, D, page_size, P_pool, scale, splits, nullptr, nullptr,
+                            dev_error, stream, &m, &t);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sa_sparse_step_workspace_size(int B, int T, int Hq, int Hkv, int D, int page_size,
+                                     int max_pages, int budget_tokens, int n_splits) {
+  int s = 0;
+  size_t sel = 0, total = 0;
+  if (step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &s, &sel,
+                &total) != SA_OK)
+    return 0;
+  return total;
+}
+
+int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                   const uint16_t* k_cache, const int64_t k_strides[4], const uint16_t* v_cache,
+                   const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                   const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D, int page_size,
+                   int P_pool, int sink_tokens, int local_tokens, int budget_tokens, float scale,
+                   int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
+                   uint16_t* o_out_bf16, float* lse_out, void* workspace,
+                   size_t workspace_bytes, int32_t* dev_error, void* stream) {
+  return step_impl(q, q_strides, summaries, k_cache, k_strides, v_cache, v_strides,
+                   flat_map(page_table, max_pages), max_pages, seq_lens, B, T, Hq, Hkv, D,
+                   page_size, P_pool, sink_tokens, local_tokens, budget_tokens, scale, n_splits,
+                   out_pages, out_counts, o_out, o_out_bf16, lse_out, workspace, workspace_bytes,
+                   dev_error, stream);
 }
 
 int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],
@@ -744,17 +825,15 @@ int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],
   if (B < 0 || T <= 0 || Hq <= 0 || Hkv <= 0 || n_lists <= 0 || D <= 0 || n_splits <= 0)
     return SA_ERR_INVALID_ARG;
   if (B == 0) return SA_OK;
-  const AttnWs w = attn_ws(B, T, Hq, D, n_splits);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < w.o_bytes + w.lse_bytes)
-    return SA_ERR_WORKSPACE;
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (!workspace || !aligned16(workspace)) return SA_ERR_WORKSPACE;
   MergeSpec m{o_out, o_out_bf16, lse_out};
   if (int r = merge_outputs_ok(m)) return r;
+  DecodeTarget t{static_cast<uint8_t*>(workspace), workspace_bytes};
   return sparse_decode_fp8_impl(q, q_strides, k_codes, k_strides, v_codes, v_strides, k_scale,
                                 v_scale, page_table, max_pages, seq_lens, lists, list_counts,
                                 n_lists, max_list, head_to_list, B, T, Hq, Hkv, D, page_size,
-                                P_pool, scale, n_splits, reinterpret_cast<float*>(ws),
-                                reinterpret_cast<float*>(ws + w.o_bytes), dev_error, stream, &m);
+                                P_pool, scale, n_splits, nullptr, nullptr, dev_error, stream, &m,
+                                &t);
 }
 
 int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, int64_t rows,
@@ -772,18 +851,18 @@ int sa_combine(const float* o_partial, const float* lse_partial, int n_splits, i
 
 namespace {
 int summaries_call(const uint16_t* k_cache, const int64_t k_strides[4],
-                   const int32_t* page_table, int max_pages, const int32_t* seq_lens, int B,
+                   const PageMap& pm, int max_pages, const int32_t* seq_lens, int B,
                    int Hkv, int Dk, int page_size, int P_pool, int n_new, uint16_t* summaries,
                    int32_t* dev_error, void* stream) {
   if (B < 0 || Hkv <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 || P_pool < 0 || n_new < 0)
     return SA_ERR_INVALID_ARG;
   if (B == 0 || max_pages == 0) return SA_OK;
-  if (!k_cache || !k_strides || k_strides[3] != 1 || !page_table || !seq_lens || !summaries)
+  if (!k_cache || !k_strides || k_strides[3] != 1 || !pm.table || !seq_lens || !summaries)
     return SA_ERR_INVALID_ARG;
   for (int i = 0; i < 3; ++i)
     if (k_strides[i] <= 0) return SA_ERR_INVALID_ARG;
   if (max_pages > 65535 || B > 65535) return SA_ERR_UNSUPPORTED;
-  return cuda_status(launch_summaries(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv,
+  return cuda_status(launch_summaries(k_cache, k_strides, pm, max_pages, seq_lens, B, Hkv,
                                       Dk, page_size, P_pool, n_new, summaries, dev_error,
                                       static_cast<cudaStream_t>(stream)));
 }
@@ -793,7 +872,8 @@ int sa_build_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4],
                             const int32_t* page_table, int max_pages, const int32_t* seq_lens,
                             int B, int Hkv, int Dk, int page_size, int P_pool,
                             uint16_t* summaries, int32_t* dev_error, void* stream) {
-  return summaries_call(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv, Dk,
+  return summaries_call(k_cache, k_strides, flat_map(page_table, max_pages), max_pages, seq_lens,
+                        B, Hkv, Dk,
                         page_size, P_pool, 0, summaries, dev_error, stream);
 }
 
@@ -802,7 +882,8 @@ int sa_update_page_summaries(const uint16_t* k_cache, const int64_t k_strides[4]
                              int B, int Hkv, int Dk, int page_size, int P_pool, int n_new,
                              uint16_t* summaries, int32_t* dev_error, void* stream) {
   if (n_new <= 0) return SA_ERR_INVALID_ARG;
-  return summaries_call(k_cache, k_strides, page_table, max_pages, seq_lens, B, Hkv, Dk,
+  return summaries_call(k_cache, k_strides, flat_map(page_table, max_pages), max_pages, seq_lens,
+                        B, Hkv, Dk,
                         page_size, P_pool, n_new, summaries, dev_error, stream);
 }
 
@@ -820,7 +901,8 @@ int sa_build_page_summaries_fp8(const uint8_t* k_codes, const int64_t k_strides[
   for (int i = 0; i < 3; ++i)
     if (k_strides[i] <= 0) return SA_ERR_INVALID_ARG;
   if (max_pages > 65535 || B > 65535 || page_size > 128) return SA_ERR_UNSUPPORTED;
-  return cuda_status(launch_summaries_fp8(k_codes, k_strides, k_scale, page_table, max_pages,
+  return cuda_status(launch_summaries_fp8(k_codes, k_strides, k_scale,
+                                          flat_map(page_table, max_pages), max_pages,
                                           seq_lens, B, Hkv, Dk, page_size, P_pool, summaries,
                                           dev_error, static_cast<cudaStream_t>(stream)));
 }
@@ -836,6 +918,191 @@ int sa_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q
   return cuda_status(launch_block_union(scores, Hq, Hkv, NQB, NKB, q_block_offset, top_k,
                                         n_sink_blocks, tables, counts,
                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t sa_select_ambient_heads_workspace_size(int B, int T, int Hq, int max_pages) {
+  if (B <= 0 || T <= 0 || Hq <= 0 || max_pages < 0) return 0;
+  return head_workspace_bytes(B, T, Hq, max_pages);
+}
+
+int sa_select_ambient_heads(const uint16_t* q, const int64_t q_strides[4],
+                            const uint16_t* summaries, const int32_t* page_table, int max_pages,
+                            const int32_t* seq_lens, const int32_t* lists,
+                            const int32_t* list_counts, int list_cap, int B, int T, int Hq,
+                            int Dk, int page_size, int P_pool, float scale, int h,
+                            int32_t* out_heads, double* out_scores, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_error, void* stream) {
+  if (B <= 0 || T <= 0 || Hq <= 0 || Dk <= 0 || page_size <= 0 || max_pages < 0 ||
+      P_pool <= 0 || list_cap <= 0 || h < 0 || h > Hq || !std::isfinite(scale))
+    return SA_ERR_INVALID_ARG;
+  if (int r = check_q(q, q_strides)) return r;
+  if (!summaries || !page_table || !seq_lens || !lists || !list_counts || (h > 0 && !out_heads))
+    return SA_ERR_INVALID_ARG;
+  if (Dk > head_max_dk() || Hq > 1024 || B > 65535 || T * Hq > 65535 * 32)
+    return SA_ERR_UNSUPPORTED;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 7u) ||
+      workspace_bytes < head_workspace_bytes(B, T, Hq, max_pages))
+    return SA_ERR_WORKSPACE;
+  HeadArgs a;
+  a.q = q;
+  a.qs0 = q_strides[0];
+  a.qs1 = q_strides[1];
+  a.qs2 = q_strides[2];
+  a.sig = summaries;
+  a.page_table = page_table;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.lists = lists;
+  a.counts = list_counts;
+  a.cap = list_cap;
+  a.B = B;
+  a.T = T;
+  a.Hq = Hq;
+  a.Dk = Dk;
+  a.P = page_size;
+  a.P_pool = P_pool;
+  a.scale = scale;
+  a.h_keep = h;
+  a.n_chunks = 0;
+  a.part = static_cast<double*>(workspace);
+  a.heads_out = out_heads;
+  a.scores_out = out_scores;
+  a.err = dev_error;
+  return cuda_status(launch_select_heads(a, static_cast<cudaStream_t>(stream)));
+}
+
+namespace {
+// sa_append_kv over either page map (max_pages: the map's capacity).
+int append_impl(const uint16_t* k_new, const int64_t kn_strides[4], const uint16_t* v_new,
+                const int64_t vn_strides[4], const int32_t* n_new, int max_new,
+                uint16_t* k_cache, const int64_t k_strides[4], uint16_t* v_cache,
+                const int64_t v_strides[4], const PageMap& pm, int max_pages,
+                const int32_t* seq_lens, int32_t* out_seq_lens, int B, int Hkv, int D,
+                int page_size, int P_pool, uint16_t* summaries, int32_t* dev_error,
+                void* stream) {
+  if (B < 0 || Hkv <= 0 || D <= 0 || page_size <= 0 || max_pages < 0 || P_pool <= 0 ||
+      max_new < 0 || D % 8 != 0)
+    return SA_ERR_INVALID_ARG;
+  if (B == 0) return SA_OK;
+  if (int r = check_q(k_new, kn_strides)) return r;   // same rules as q: [B, T, H, D]
+  if (int r = check_q(v_new, vn_strides)) return r;
+  if (int r = check_cache(k_cache, k_strides)) return r;
+  if (int r = check_cache(v_cache, v_strides)) return r;
+  if (!n_new || !pm.table || !seq_lens || !summaries) return SA_ERR_INVALID_ARG;
+  if (out_seq_lens == seq_lens) return SA_ERR_INVALID_ARG;   // read by every block
+  if (B > 65535 || Hkv > 65535) return SA_ERR_UNSUPPORTED;
+  AppendArgs a;
+  a.k_new = k_new;
+  a.kn0 = kn_strides[0];
+  a.kn1 = kn_strides[1];
+  a.kn2 = kn_strides[2];
+  a.v_new = v_new;
+  a.vn0 = vn_strides[0];
+  a.vn1 = vn_strides[1];
+  a.vn2 = vn_strides[2];
+  a.n_new = n_new;
+  a.max_new = max_new;
+  a.k_cache = k_cache;
+  a.ks0 = k_strides[0];
+  a.ks1 = k_strides[1];
+  a.ks2 = k_strides[2];
+  a.v_cache = v_cache;
+  a.vs0 = v_strides[0];
+  a.vs1 = v_strides[1];
+  a.vs2 = v_strides[2];
+  a.pt = pm;
+  a.max_pages = max_pages;
+  a.seq_lens = seq_lens;
+  a.out_seq_lens = out_seq_lens;
+  a.B = B;
+  a.Hkv = Hkv;
+  a.D = D;
+  a.P = page_size;
+  a.P_pool = P_pool;
+  a.sig = summaries;
+  a.err = dev_error;
+  return cuda_status(launch_append(a, static_cast<cudaStream_t>(stream)));
+}
+
+// The two-level map of a *_dir call, checked on the host; its capacity in
+// logical pages goes to *max_pages.
+int dir_map(const int32_t* page_dir, int n_dir, const int32_t* page_blocks, int n_blocks,
+            int block_shift, PageMap* m, int* max_pages) {
+  if (!page_dir || !page_blocks || n_dir < 0 || n_blocks < 0 || block_shift < 0 ||
+      block_shift > 16)
+    return SA_ERR_INVALID_ARG;
+  const int64_t cap = (int64_t)n_dir << block_shift;
+  if (cap > (int64_t(1) << 30)) return SA_ERR_UNSUPPORTED;
+  m->table = page_dir;
+  m->blocks = page_blocks;
+  m->stride = n_dir;
+  m->shift = block_shift;
+  m->n_blocks = n_blocks;
+  *max_pages = (int)cap;
+  return SA_OK;
+}
+}  // namespace
+
+int sa_append_kv(const uint16_t* k_new, const int64_t kn_strides[4], const uint16_t* v_new,
+                 const int64_t vn_strides[4], const int32_t* n_new, int max_new,
+                 uint16_t* k_cache, const int64_t k_strides[4], uint16_t* v_cache,
+                 const int64_t v_strides[4], const int32_t* page_table, int max_pages,
+                 const int32_t* seq_lens, int32_t* out_seq_lens, int B, int Hkv, int D,
+                 int page_size, int P_pool, uint16_t* summaries, int32_t* dev_error,
+                 void* stream) {
+  return append_impl(k_new, kn_strides, v_new, vn_strides, n_new, max_new, k_cache, k_strides,
+                     v_cache, v_strides, flat_map(page_table, max_pages), max_pages, seq_lens,
+                     out_seq_lens, B, Hkv, D, page_size, P_pool, summaries, dev_error, stream);
+}
+
+int sa_append_kv_dir(const uint16_t* k_new, const int64_t kn_strides[4], const uint16_t* v_new,
+                     const int64_t vn_strides[4], const int32_t* n_new, int max_new,
+                     uint16_t* k_cache, const int64_t k_strides[4], uint16_t* v_cache,
+                     const int64_t v_strides[4], const int32_t* page_dir, int n_dir,
+                     const int32_t* page_blocks, int n_blocks, int block_shift,
+                     const int32_t* seq_lens, int32_t* out_seq_lens, int B, int Hkv, int D,
+                     int page_size, int P_pool, uint16_t* summaries, int32_t* dev_error,
+                     void* stream) {
+  PageMap m;
+  int max_pages = 0;
+  if (int r = dir_map(page_dir, n_dir, page_blocks, n_blocks, block_shift, &m, &max_pages))
+    return r;
+  return append_impl(k_new, kn_strides, v_new, vn_strides, n_new, max_new, k_cache, k_strides,
+                     v_cache, v_strides, m, max_pages, seq_lens, out_seq_lens, B, Hkv, D,
+                     page_size, P_pool, summaries, dev_error, stream);
+}
+
+int sa_build_page_summaries_dir(const uint16_t* k_cache, const int64_t k_strides[4],
+                                const int32_t* page_dir, int n_dir, const int32_t* page_blocks,
+                                int n_blocks, int block_shift, const int32_t* seq_lens, int B,
+                                int Hkv, int Dk, int page_size, int P_pool, uint16_t* summaries,
+                                int32_t* dev_error, void* stream) {
+  PageMap m;
+  int max_pages = 0;
+  if (int r = dir_map(page_dir, n_dir, page_blocks, n_blocks, block_shift, &m, &max_pages))
+    return r;
+  return summaries_call(k_cache, k_strides, m, max_pages, seq_lens, B, Hkv, Dk, page_size, P_pool,
+                        0, summaries, dev_error, stream);
+}
+
+int sa_sparse_step_dir(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                       const uint16_t* k_cache, const int64_t k_strides[4],
+                       const uint16_t* v_cache, const int64_t v_strides[4],
+                       const int32_t* page_dir, int n_dir, const int32_t* page_blocks,
+                       int n_blocks, int block_shift, const int32_t* seq_lens, int B, int T,
+                       int Hq, int Hkv, int D, int page_size, int P_pool, int sink_tokens,
+                       int local_tokens, int budget_tokens, float scale, int n_splits,
+                       int32_t* out_pages, int32_t* out_counts, float* o_out,
+                       uint16_t* o_out_bf16, float* lse_out, void* workspace,
+                       size_t workspace_bytes, int32_t* dev_error, void* stream) {
+  PageMap m;
+  int max_pages = 0;
+  if (int r = dir_map(page_dir, n_dir, page_blocks, n_blocks, block_shift, &m, &max_pages))
+    return r;
+  return step_impl(q, q_strides, summaries, k_cache, k_strides, v_cache, v_strides, m, max_pages,
+                   seq_lens, B, T, Hq, Hkv, D, page_size, P_pool, sink_tokens, local_tokens,
+                   budget_tokens, scale, n_splits, out_pages, out_counts, o_out, o_out_bf16,
+                   lse_out, workspace, workspace_bytes, dev_error, stream);
 }
 
 }  // extern "C"

@@ -68,11 +68,40 @@ struct PairTable {
   int16_t heads[kMaxHeads];
 };
 
+// A batch's logical -> physical page map.  Flat (blocks null): table is
+// [B, stride] physical page ids.  Two-level (the working-set-sized layout):
+// table is a directory [B, stride] of block ids, block j of a row covering
+// logical pages [j << shift, (j + 1) << shift), and blocks [n_blocks,
+// 1 << shift] holds the physical ids; a directory entry outside [0, n_blocks)
+// (-1: no block) resolves to -1.  Capacity in logical pages: stride (flat) or
+// stride << shift.
+struct PageMap {
+  const int32_t* table = nullptr;
+  const int32_t* blocks = nullptr;
+  int stride = 0;
+  int shift = 0;
+  int n_blocks = 0;
+};
+inline PageMap flat_map(const int32_t* table, int max_pages) {
+  PageMap m;
+  m.table = table;
+  m.stride = max_pages;
+  return m;
+}
+#ifdef __CUDACC__
+__device__ __forceinline__ int page_at(const PageMap& m, int b, int p) {
+  if (!m.blocks) return m.table[(int64_t)b * m.stride + p];
+  const int blk = m.table[(int64_t)b * m.stride + (p >> m.shift)];
+  if (blk < 0 || blk >= m.n_blocks) return -1;
+  return m.blocks[((int64_t)blk << m.shift) + (p & ((1 << m.shift) - 1))];
+}
+#endif
+
 struct DecodeArgs {
   const uint16_t* q;
   int64_t qs0, qs1, qs2;
-  const int32_t* page_table;
-  int max_pages;
+  PageMap pt;
+  int max_pages;          // logical pages a sequence may hold (the map's capacity)
   const int32_t* seq_lens;
   const int32_t* lists;
   const int32_t* counts;
@@ -85,7 +114,15 @@ struct DecodeArgs {
   int32_t* err;
   const float* k_scale;   // FP8 pages: [P_pool, Hkv] float32 scales (null for bf16 pages)
   const float* v_scale;
+  const int32_t* q_pos;   // [B] position of query token 0 (null: the causal tail L - T)
 };
+
+// Position of query token 0 of sequence b of length L (token t sits at this
+// + t and sees the keys at positions up to its own): the caller's q_pos[b],
+// else the causal tail L - T.
+__host__ __device__ inline int query_base(const DecodeArgs& a, int b, int L) {
+  return a.q_pos ? a.q_pos[b] : L - a.T;
+}
 
 // Encode a 4-D bf16 tensor map over a [P_pool, Hkv, P, D] cache with
 // 64-column x box_rows-row boxes (box_rows 16 or 64, at most P) and 128-byte
@@ -119,7 +156,7 @@ struct SelectArgs {
   const uint16_t* q;
   int64_t qs0, qs1, qs2;
   const uint16_t* sig;
-  const int32_t* page_table;
+  PageMap pt;
   const int32_t* seq_lens;
   int B, T, Hq, Hkv, Dk, P, max_pages, P_pool;
   int n_sink, n_local, budget_pages, k_top;
@@ -156,14 +193,59 @@ cudaError_t launch_combine(const float* o_part, const float* lse_part, int n_spl
                            int Dv, float* o_out, uint16_t* o_bf16, float* lse_out,
                            cudaStream_t stream);
 
+// max_pages: the map's capacity in logical pages
 cudaError_t launch_summaries_fp8(const uint8_t* k, const int64_t ks[4], const float* k_scale,
-                                 const int32_t* pt, int max_pages, const int32_t* seq_lens, int B,
+                                 const PageMap& pt, int max_pages, const int32_t* seq_lens, int B,
                                  int Hkv, int Dk, int P, int P_pool, uint16_t* sig, int32_t* err,
                                  cudaStream_t stream);
-cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
+cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const PageMap& pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
                              int P, int P_pool, int n_new, uint16_t* sig, int32_t* err,
                              cudaStream_t stream);
+
+struct HeadArgs {
+  const uint16_t* q;       // [B, T, Hq, Dk]
+  int64_t qs0, qs1, qs2;
+  const uint16_t* sig;     // [P_pool, 1, Dk]
+  const int32_t* page_table;
+  int max_pages;
+  const int32_t* seq_lens;
+  const int32_t* lists;    // [B, 2, cap]: critical, critical + ambient
+  const int32_t* counts;   // [B, 2]
+  int cap;
+  int B, T, Hq, Dk, P, P_pool;
+  float scale;
+  int h_keep;
+  int n_chunks;            // set by the launcher
+  double* part;            // workspace [B, n_chunks, T*Hq, 3]
+  int32_t* heads_out;      // [h_keep]
+  double* scores_out;      // [Hq] (optional)
+  int32_t* err;
+};
+size_t head_workspace_bytes(int B, int T, int Hq, int max_pages);
+int head_max_dk();
+cudaError_t launch_select_heads(HeadArgs a, cudaStream_t stream);
+
+struct AppendArgs {
+  const uint16_t* k_new;   // [B, max_new, Hkv, D]
+  int64_t kn0, kn1, kn2;
+  const uint16_t* v_new;
+  int64_t vn0, vn1, vn2;
+  const int32_t* n_new;    // [B]
+  int max_new;
+  uint16_t* k_cache;       // [P_pool, Hkv, P, D]
+  int64_t ks0, ks1, ks2;
+  uint16_t* v_cache;
+  int64_t vs0, vs1, vs2;
+  PageMap pt;
+  int max_pages;           // the map's capacity in logical pages
+  const int32_t* seq_lens;
+  int32_t* out_seq_lens;
+  int B, Hkv, D, P, P_pool;
+  uint16_t* sig;           // [P_pool, Hkv, D]
+  int32_t* err;
+};
+cudaError_t launch_append(const AppendArgs& a, cudaStream_t stream);
 
 cudaError_t launch_block_union(const float* scores, int Hq, int Hkv, int NQB, int NKB, int q_off,
                                int top_k, int n_sink, int32_t* tables, int32_t* counts,

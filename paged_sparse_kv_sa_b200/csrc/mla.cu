@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
     return;
   }
   const int t_last = (min(rows_total, r0 + kMRows) - 1) / nh;
-  const int max_q = L - a.T + t_last;
+  const int max_q = query_base(a, b, L) + t_last;
 
   const int n_tiles = min((n_ent * a.P + kMKeys - 1) / kMKeys, kMMaxTiles);
   // query tile: 64 rows x 9 chunks of 128 bytes, 128-byte swizzle.  Each row
@@ -179,14 +179,13 @@ __global__ void __launch_bounds__(kMThreads, 1)
   int n_act = 0;
   if (warp == 4) {
     const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
-    const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
     for (int i = lane; i < n_ent; i += 32) {
       const int p = lrow[i];
       int ph = -1;
       if (p < 0 || p >= n_log) {
         set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
       } else {
-        ph = ptrow[p];
+        ph = page_at(a.pt, b, p);
         if (ph < 0 || ph >= a.P_pool) {
           set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
           ph = -1;
@@ -387,7 +386,7 @@ __global__ void __launch_bounds__(kMThreads, 1)
     const bool row_ok = rg < rows_total;
     const int t = row_ok ? rg / nh : 0;
     const int head = prm.pairs.heads[prm.pairs.head_off[pair] + (row_ok ? rg % nh : 0)];
-    const int qpos = row_ok ? L - a.T + t : -1;
+    const int qpos = row_ok ? query_base(a, b, L) + t : -1;
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const float sl2 = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;

@@ -151,18 +151,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
   }
   const int t_first = r0 / nh;
   const int t_last = (min(rows_total, r0 + kRows) - 1) / nh;
-  const int min_q = L - a.T + t_first, max_q = L - a.T + t_last;
+  const int qb = query_base(a, b, L);
+  const int min_q = qb + t_first, max_q = qb + t_last;
 
   // ---- resolve pages, set up barriers and TMEM
   const int32_t* lrow = a.lists + ((int64_t)b * a.n_lists + list) * a.max_list + e0;
-  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
   for (int i = tid; i < n_ent; i += kPThreads) {
     const int p = lrow[i];
     int ph = -1;
     if (p < 0 || p >= n_log) {
       set_dev_error(a.err, SA_DEVERR_PAGE_RANGE);
     } else {
-      ph = ptrow[p];
+      ph = page_at(a.pt, b, p);
       if (ph < 0 || ph >= a.P_pool) {
         set_dev_error(a.err, SA_DEVERR_POOL_RANGE);
         ph = -1;
@@ -303,7 +303,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     const bool row_ok = rg < rows_total;
     const int t = row_ok ? rg / nh : 0;
     const int head = prm.pairs.heads[prm.pairs.head_off[pair] + (row_ok ? rg % nh : 0)];
-    const int qpos = row_ok ? L - a.T + t : -1;
+    const int qpos = row_ok ? qb + t : -1;
     uint8_t* qt_s = q_s + wg * C::kQBytes;
     {
       const uint4* src = reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + head * a.qs2);

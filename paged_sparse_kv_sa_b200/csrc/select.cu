@@ -174,12 +174,11 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
 
   if (warp == hb) {
     // ================= producer: page-table lookups and bulk gathers
-    const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
     int ph_r[kScoreChunk / 32];
 #pragma unroll
     for (int i = 0; i < kScoreChunk / 32; ++i) {
       const int p = p0 + 32 * i + lane;
-      ph_r[i] = (p < N && p >= n_sink && p < local0) ? ptrow[p] : -1;
+      ph_r[i] = (p < N && p >= n_sink && p < local0) ? page_at(a.pt, b, p) : -1;
     }
     for (int g = 0; g < n_groups; ++g) {
       const int st = g % kScoreStages;
@@ -491,7 +490,6 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
     }
   }
   __syncthreads();
-  const int32_t* ptrow = a.page_table + (int64_t)b * a.max_pages;
 
   const int nu_ = n_unc;
   const int slots = k - n_certain;
@@ -506,7 +504,7 @@ __global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
       const int np = min(per, nu_ - u0);
       for (int pr = warp; pr < np * R; pr += nw) {
         const int r = pr % R;
-        const int ph = ptrow[S.u_list[u0 + pr / R]];
+        const int ph = page_at(a.pt, b, S.u_list[u0 + pr / R]);
         double e = -INFINITY;
         if (ph >= 0 && ph < a.P_pool) {
           const int t = r / G, h = kvh * G + r % G;

@@ -19,7 +19,7 @@ namespace {
 
 __global__ void __launch_bounds__(256)
     summaries_kernel(const uint16_t* __restrict__ k, int64_t ks0, int64_t ks1, int64_t ks2,
-                     const int32_t* __restrict__ pt, int max_pages,
+                     const PageMap pt, int max_pages,
                      const int32_t* __restrict__ seq_lens, int Hkv, int Dk, int P, int P_pool,
                      int n_new, uint16_t* __restrict__ sig, int32_t* err) {
   pdl_wait_and_release();
@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(256)
   const int p = (n_new > 0 ? max(L - n_new, 0) / P : 0) + blockIdx.x;
   const int n = min(P, L - p * P);
   if (n <= 0) return;
-  const int ph = pt[(int64_t)b * max_pages + p];
+  const int ph = page_at(pt, b, p);
   if (ph < 0 || ph >= P_pool) {
     if (threadIdx.x == 0) set_dev_error(err, SA_DEVERR_POOL_RANGE);
     return;
@@ -71,7 +71,7 @@ __global__ void __launch_bounds__(256)
 // RN64(exact sum of the dequantized keys / n), as for bf16 pages.
 __global__ void __launch_bounds__(256)
     summaries_fp8_kernel(const uint8_t* __restrict__ k, int64_t ks0, int64_t ks1, int64_t ks2,
-                         const float* __restrict__ k_scale, const int32_t* __restrict__ pt,
+                         const float* __restrict__ k_scale, const PageMap pt,
                          int max_pages, const int32_t* __restrict__ seq_lens, int Hkv, int Dk,
                          int P, int P_pool, uint16_t* __restrict__ sig, int32_t* err) {
   pdl_wait_and_release();
@@ -79,7 +79,7 @@ __global__ void __launch_bounds__(256)
   const int L = min(seq_lens[b], max_pages * P);
   const int n = min(P, L - p * P);
   if (n <= 0) return;
-  const int ph = pt[(int64_t)b * max_pages + p];
+  const int ph = page_at(pt, b, p);
   if (ph < 0 || ph >= P_pool) {
     if (threadIdx.x == 0) set_dev_error(err, SA_DEVERR_POOL_RANGE);
     return;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256)
 }  // namespace
 
 cudaError_t launch_summaries_fp8(const uint8_t* k, const int64_t ks[4], const float* k_scale,
-                                 const int32_t* pt, int max_pages, const int32_t* seq_lens, int B,
+                                 const PageMap& pt, int max_pages, const int32_t* seq_lens, int B,
                                  int Hkv, int Dk, int P, int P_pool, uint16_t* sig, int32_t* err,
                                  cudaStream_t stream) {
   if (B == 0 || max_pages == 0) return cudaSuccess;
@@ -106,7 +106,7 @@ cudaError_t launch_summaries_fp8(const uint8_t* k, const int64_t ks[4], const fl
                     k_scale, pt, max_pages, seq_lens, Hkv, Dk, P, P_pool, sig, err);
 }
 
-cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const int32_t* pt,
+cudaError_t launch_summaries(const uint16_t* k, const int64_t ks[4], const PageMap& pt,
                              int max_pages, const int32_t* seq_lens, int B, int Hkv, int Dk,
                              int P, int P_pool, int n_new, uint16_t* sig, int32_t* err,
                              cudaStream_t stream) {

@@ -109,6 +109,15 @@ LLAMA70B_LONG = GQADecode("llama70b_long_b32_hq64_hkv8_d128_p16_l64k-128k", B=32
                           local_tokens=512, budget_tokens=2048, table="shuffled")
 MLA_MTP = MLADecode("mla_mtp_b8_t2_hq128_dk576_dv512_p64_l65536", B=8, T=2, Hq=128, Dk=576, Dv=512,
                     page_size=64, seq_len=65536, alpha=8, beta=24, h_ambient=32)
+# Million-token page tables (SPIN's two-level metadata, on the page titled
+# "Vortex: Efficient and Programmable Sparse Attention Serving for AI Agents"):
+# 8 sequences of 64K to 1M tokens in 64-token pages, their page maps as
+# directories over blocks of 64 pages (block_shift 6); the UAE sink / local
+# pattern with a 2048-token budget.
+LLAMA8B_DIR_1M = GQADecode("llama8b_dir_b8_hq32_hkv8_d128_p64_l64k-1m", B=8, Hq=32, Hkv=8, D=128,
+                           page_size=64, seq_len_lo=65536, seq_len_hi=1048576, sink_tokens=64,
+                           local_tokens=512, budget_tokens=2048, table="shuffled")
+DIR_BLOCK_SHIFT = 6
 UNION_PREFILL = BlockUnionPrefill("union_prefill_c2048_off126976_hq32_hkv8_d128_b64", Hq=32, Hkv=8,
                                   D=128, block=64, chunk=2048, q_offset=126976, top_k=8)
 
@@ -194,6 +203,37 @@ def gqa_decode_inputs(cfg: GQADecode, seed: int = 0, device="cpu", seq_lens: Opt
                 shifted = k[phys, kvh].float() + cfg.lift_sigma * u
                 k[phys, kvh] = shifted.to(torch.bfloat16)
     return dict(q=q, k=k, v=v, page_table=pt, seq_lens=sl, pool=pool)
+
+
+def page_directory(page_table: torch.Tensor, seq_lens: torch.Tensor, page_size: int,
+                   block_shift: int, seed: int = 0):
+    """A two-level page map holding ``page_table``: a directory [B, n_dir] of block
+    ids (-1 where a run of 2^block_shift logical pages holds none of the
+    sequence's pages) and blocks [n_blocks, 2^block_shift] of physical page ids
+    (-1 past the sequence's last page).  Only the runs a sequence uses get a
+    block; blocks are numbered in a seeded random order.  Pure layout: the
+    table's entries are moved, not computed."""
+    device = page_table.device
+    B, W = page_table.shape
+    width = 1 << block_shift
+    n_dir = max(1, -(-W // width))
+    n_pages = ((seq_lens.to(torch.int64) + page_size - 1) // page_size).tolist()
+    runs = [(b, j) for b in range(B) for j in range(-(-int(n_pages[b]) // width))]
+    g = _gen("cpu", seed)
+    order = torch.randperm(max(len(runs), 1), generator=g)[:len(runs)].tolist()
+    padded = torch.full((B, n_dir * width), -1, dtype=torch.int32, device=device)
+    padded[:, :W] = page_table
+    for b in range(B):   # entries past a sequence's pages stay -1
+        padded[b, int(n_pages[b]):] = -1
+    page_dir = torch.full((B, n_dir), -1, dtype=torch.int32)
+    src = torch.empty(max(len(runs), 1), dtype=torch.int64)
+    for (b, j), bid in zip(runs, order):
+        page_dir[b, j] = bid
+        src[bid] = b * n_dir + j
+    blocks = torch.full((max(len(runs), 1), width), -1, dtype=torch.int32, device=device)
+    if runs:
+        blocks[:len(runs)] = padded.view(B * n_dir, width)[src[:len(runs)].to(device)]
+    return page_dir.to(device), blocks
 
 
 def fp8_pages(x):

@@ -158,6 +158,84 @@ def test_step_workspace_size_and_host_checks():
     assert call(fake, need, sink=512) == 1                    # sink + local above the budget
 
 
+def test_append_host_checks():
+    lib = sa.load()
+    fake = ctypes.c_void_p(0x1000)      # never dereferenced: validation fails first
+    kn = _i64x4(40 * 8 * 128, 8 * 128, 128, 1)
+    ks = _i64x4(8 * 16 * 128, 16 * 128, 128, 1)
+
+    def call(D=128, kn_=kn, out=None, seq=fake, max_new=40):
+        return lib.sa_append_kv(fake, kn_, fake, kn, fake, max_new, fake, ks, fake, ks, fake, 64,
+                                seq, out, 4, 8, D, 16, 1000, fake, None, None)
+    assert call(D=100) == 1                                   # D not a multiple of 8
+    assert call(kn_=_i64x4(40 * 8 * 128, 8 * 128, 128, 2)) == 1   # feature stride not 1
+    assert call(kn_=_i64x4(40 * 8 * 128, 8 * 128, 124, 1)) == 1   # head stride not 16 bytes
+    assert call(out=fake) == 1                                # new lengths over the old ones
+    assert call(seq=None) == 1                                # no lengths
+    assert call(max_new=-1) == 1
+
+
+def test_two_level_map_host_checks():
+    lib = sa.load()
+    fake = ctypes.c_void_p(0x1000)      # never dereferenced: validation fails first
+    ks = _i64x4(8 * 64 * 128, 64 * 128, 128, 1)
+
+    def summ(page_dir=fake, n_dir=4, blocks=fake, n_blocks=3, shift=6, B=2):
+        return lib.sa_build_page_summaries_dir(fake, ks, page_dir, n_dir, blocks, n_blocks, shift,
+                                               fake, B, 8, 128, 64, 100, fake, None, None)
+    assert summ(page_dir=None) == 1
+    assert summ(blocks=None) == 1
+    assert summ(n_dir=-1) == 1
+    assert summ(n_blocks=-1) == 1
+    assert summ(shift=-1) == 1
+    assert summ(shift=17) == 1
+    assert summ(n_dir=1 << 15, shift=16) == 2                 # capacity above 2^30 pages
+    assert summ(B=-1) == 1
+    assert summ(B=0) == 0                                     # nothing to do, nothing launched
+
+    qs = _i64x4(32 * 128, 32 * 128, 128, 1)
+    kvs = _i64x4(8 * 64 * 128, 64 * 128, 128, 1)
+
+    def step(n_dir=4, shift=6, ws_bytes=1 << 30):
+        return lib.sa_sparse_step_dir(fake, qs, fake, fake, kvs, fake, kvs, fake, n_dir, fake, 3,
+                                      shift, fake, 2, 1, 32, 8, 128, 64, 100, 64, 512, 2048, 0.08,
+                                      4, fake, fake, fake, None, None, fake, ws_bytes, None, None)
+    assert step(shift=20) == 1
+    assert step(n_dir=300) == 2                               # 19200 pages: above the selection's 16384
+    assert step(ws_bytes=16) == 3                             # workspace below the size call's
+    need = lib.sa_sparse_step_workspace_size(2, 1, 32, 8, 128, 64, 4 << 6, 2048, 4)
+    assert need > 0 and step(ws_bytes=need - 16) == 3
+
+    kn = _i64x4(40 * 8 * 128, 8 * 128, 128, 1)
+
+    def app(shift=3, blocks=fake):
+        return lib.sa_append_kv_dir(fake, kn, fake, kn, fake, 40, fake, kvs, fake, kvs, fake, 4,
+                                    blocks, 3, shift, fake, None, 4, 8, 128, 64, 1000, fake, None,
+                                    None)
+    assert app(shift=-2) == 1
+    assert app(blocks=None) == 1
+
+
+def test_ambient_heads_host_checks():
+    lib = sa.load()
+    fake = ctypes.c_void_p(0x1000)      # never dereferenced: validation fails first
+    s = _i64x4(2 * 128 * 576, 128 * 576, 576, 1)
+    # partials [B, chunks of 32 pages, T * Hq rows, 3] float64
+    assert lib.sa_select_ambient_heads_workspace_size(8, 2, 128, 1024) == 8 * 32 * 256 * 3 * 8
+    need = lib.sa_select_ambient_heads_workspace_size(8, 2, 128, 1024)
+
+    def call(h=32, Dk=576, ws=fake, ws_bytes=need, scale=0.04):
+        return lib.sa_select_ambient_heads(fake, s, fake, fake, 1024, fake, fake, fake, 32, 8, 2,
+                                           128, Dk, 64, 8192, scale, h, fake, None, ws, ws_bytes,
+                                           None, None)
+    assert call(h=129) == 1                                   # more heads than there are
+    assert call(h=-1) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(Dk=1024) == 2                                 # head dim above what it runs
+    assert call(ws=None) == 3
+    assert call(ws_bytes=need - 8) == 3
+
+
 def test_default_split_policy():
     from paged_sparse_kv_sa_b200.pipeline import default_splits
     # one wave of decode warps (12 per SM on 148 SMs) over the (sequence, kv head) units
