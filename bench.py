@@ -599,7 +599,7 @@ def run_dir(args, dev, world, rank, clk, K):
             step("dir")
             step("flat")
         torch.cuda.synchronize()
-        graphs = {n: capture(sa.bind(lambda n=n: step(n))) for n in ("dir", "flat")}
+        graphs = {n: capture(lambda n=n: step(n)) for n in ("dir", "flat")}
         for g in graphs.values():
             for _ in range(3):
                 g.replay()

@@ -20,8 +20,36 @@
 #include "common.cuh"
 #include "internal.h"
 
+// Diagnostic build (-DSA_DECODE_TIMELINE=1, off in the library): each warp's
+// first work item records %globaltimer stamps -- entry, list entries read,
+// pages resolved, each of its first 8 units' data arriving, partial stored --
+// plus its SM, item and unit count, read back with sa_decode_timeline().
+#ifndef SA_DECODE_TIMELINE
+#define SA_DECODE_TIMELINE 0
+#endif
+
 namespace sa {
+#if SA_DECODE_TIMELINE
+constexpr int kTlWarps = 8192, kTlSlots = 16;
+__device__ unsigned long long g_decode_tl[kTlWarps * kTlSlots];
+#endif
 namespace {
+
+#if SA_DECODE_TIMELINE
+SA_DEV unsigned long long tl_now() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+#define SA_TL(slot, value)                                              \
+  do {                                                                  \
+    if (tl_row >= 0 && lane == 0) g_decode_tl[tl_row + (slot)] = (value); \
+  } while (0)
+#else
+#define SA_TL(slot, value) \
+  do {                     \
+  } while (0)
+#endif
 
 // Build-time shape of a CTA: warps (= splits) per CTA and ring stages per warp.
 #ifndef SA_DECODE_WARPS
@@ -324,17 +352,6 @@ SA_DEV void store_partial(RowState<D>& st, const DecodeArgs& a, const PairTable&
   }
 }
 
-// LSE = -inf for every row of the pair in partial slot `slot` (the merge gives
-// such a slot no weight and reads none of its O rows).
-SA_DEV void store_empty(const DecodeArgs& a, const PairTable& pr, int pair, int b, int slot,
-                        int lane) {
-  const int nh = pr.n_heads[pair], R = a.T * nh;
-  for (int r = lane; r < R; r += 32) {
-    const int t = r / nh, head = pr.heads[pr.head_off[pair] + (r % nh)];
-    a.lse_part[(((int64_t)slot * a.B + b) * a.T + t) * a.Hq + head] = -INFINITY;
-  }
-}
-
 // ---------------------------------------------------------------------------
 // Split kernel: one warp per split of one (list, kv head) pair of one sequence
 // ---------------------------------------------------------------------------
@@ -347,6 +364,12 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
   using C = DecodeCfg<D, F8>;
   const DecodeArgs& a = prm.a;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#if SA_DECODE_TIMELINE
+  const unsigned long long tl_t0 = tl_now();
+  const int tl_gw = blockIdx.x * kNW + warp;
+  int tl_row = tl_gw < kTlWarps ? tl_gw * kTlSlots : -1;
+  SA_TL(0, tl_t0);
+#endif
 
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
@@ -404,6 +427,9 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     }
     const int e0 = min(s0, count);
     const int n_ent = min(chunk, count - e0);
+#if SA_DECODE_TIMELINE
+    SA_TL(1, tl_now());
+#endif
 
     // Resolve logical -> physical pages of this split.
 #pragma unroll
@@ -431,6 +457,15 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
 
     const int subs = a.P / kSub;
     const int n_units = n_ent * subs;
+#if SA_DECODE_TIMELINE
+    SA_TL(2, tl_now());
+    {
+      unsigned smid;
+      asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+      SA_TL(15, (unsigned long long)smid | ((unsigned long long)n_units << 16) |
+                    ((unsigned long long)item << 32));
+    }
+#endif
 
     auto unit_live = [&](int u, int& ph, int& tok0) {
       const int2 e = ent_s[warp][u / subs];
@@ -490,6 +525,9 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
         u_fail = u;
         break;
       }
+#if SA_DECODE_TIMELINE
+      if (u < 8) SA_TL(4 + u, tl_now());
+#endif
       int ph, tok0;
       if (unit_live(u, ph, tok0)) {
         float ksc = 1.f, vsc = 1.f;   // FP8: key scale, value scale / v_ref
@@ -514,6 +552,10 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     }
     store_partial<D>(st, a, prm.pairs, pair, b, split, v_ref, lane);
     base += n_units;
+#if SA_DECODE_TIMELINE
+    SA_TL(12, tl_now());
+    tl_row = -1;   // only the first item of a warp is recorded
+#endif
   }  // items
 }
 
@@ -584,3 +626,20 @@ cudaError_t launch_decode_gqa_fp8(const DecodeArgs& a, const PairTable& pairs,
 }
 
 }  // namespace sa
+
+#if SA_DECODE_TIMELINE
+// Diagnostic build only: copies the recorded stamps ([8192 warps][16] u64) to
+// host memory `out` (n entries at most) and clears them.  Not in the library's
+// header: the library proper is built without it.
+extern "C" SA_API int sa_decode_timeline(unsigned long long* out, int n) {
+  const int total = sa::kTlWarps * sa::kTlSlots;
+  if (!out || n <= 0) return SA_ERR_INVALID_ARG;
+  const size_t bytes = sizeof(unsigned long long) * (size_t)(n < total ? n : total);
+  if (cudaMemcpyFromSymbol(out, sa::g_decode_tl, bytes) != cudaSuccess) return SA_ERR_CUDA;
+  void* dev = nullptr;
+  if (cudaGetSymbolAddress(&dev, sa::g_decode_tl) != cudaSuccess ||
+      cudaMemset(dev, 0, sizeof(unsigned long long) * total) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_OK;
+}
+#endif
