@@ -22,7 +22,8 @@
 
 // Diagnostic build (-DSA_DECODE_TIMELINE=1, off in the library): each warp's
 // first work item records %globaltimer stamps -- entry, list entries read,
-// pages resolved, each of its first 8 units' data arriving, partial stored --
+// pages resolved, its first unit computed, each of its first 8 units' data
+// arriving, partial stored --
 // plus its SM, item and unit count, read back with sa_decode_timeline().
 #ifndef SA_DECODE_TIMELINE
 #define SA_DECODE_TIMELINE 0
@@ -538,6 +539,9 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
         }
         attend_unit<D, F8>(st, qa, ring + slot * C::kStageBytes, wide, tok0, L, lim,
                            a.scale_log2, ksc, vsc, lane);
+#if SA_DECODE_TIMELINE
+        if (u == 0) SA_TL(3, tl_now());
+#endif
       }
       __syncwarp();   // (FP8: the staging tiles are free again)
       if (lane == 0 && u + C::kStages < n_units) issue(u + C::kStages);

@@ -1,16 +1,19 @@
 """Per-warp timeline of the decode kernel at the Llama-8B-shaped decode workload.
 
-    python -m paged_sparse_kv_sa_b200.timeline [--splits N] [--reps R] [--seed S]
+    python -m paged_sparse_kv_sa_b200.timeline [--splits N] [--reps R] [--seed S] [--fp8]
 
 Builds a diagnostic copy of the library (``_build/timeline/libsa_timeline.so``,
 compiled with ``-DSA_DECODE_TIMELINE=1``: each decode warp records
 ``%globaltimer`` stamps for its first work item), selects the pages of the
-workload once, then times R decode launches, each after an L2 flush (a 256 MiB
-write, then a 256 MiB read), and prints where a launch's time goes:
+workload once (``--fp8``: the same pages stored as FP8 E4M3 codes with
+per-(page, kv head) scales), then times R decode launches, each after an L2
+flush (a 256 MiB write, then a 256 MiB read), and prints where a launch's time
+goes:
 
 * the phases of the warps (when they start, have read their list entries,
   have resolved their pages, see their first and last unit's data, and have
-  stored their partial), as percentiles over the warps;
+  stored their partial; and how long the arithmetic on the first unit takes),
+  as percentiles over the warps;
 * the bytes that arrive in each microsecond (K + V of every unit whose data
   has landed), i.e. the aggregate rate at which the launch moves its bytes;
 * how many warps are still running in each microsecond.
@@ -52,6 +55,8 @@ def analyse(stamps: np.ndarray, unit_bytes: int):
     meta = rows[:, 15]
     n_units = ((meta >> 16) & 0xFFFF).astype(np.int64)
     start, ents, pages, end = us(rows[:, 0]), us(rows[:, 1]), us(rows[:, 2]), us(rows[:, 12])
+    c0 = rows[:, 3] != 0
+    comp0 = us(rows[c0, 3]) - us(rows[c0, 4])    # first unit: data in -> arithmetic done
     arr = []
     first, last = [], []
     for i in range(len(rows)):
@@ -63,7 +68,7 @@ def analyse(stamps: np.ndarray, unit_bytes: int):
             last.append(a[-1])
     phases = [("warp start", start), ("list entries read", ents), ("pages resolved", pages),
               ("first unit's data in", np.array(first)), ("last unit's data in", np.array(last)),
-              ("partial stored", end)]
+              ("partial stored", end), ("first unit's arithmetic (duration)", comp0)]
     span = float(end.max())
     n_b = int(np.ceil(span)) + 1
     got = np.zeros(n_b)
@@ -80,6 +85,7 @@ def main():
     ap.add_argument("--splits", type=int, default=0)
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--fp8", action="store_true")
     args = ap.parse_args()
     path = _build_timeline_lib()
     lib = _lib.load(path)               # every wrapper below now calls this copy
@@ -90,12 +96,17 @@ def main():
 
     from . import workloads as W
     from .pipeline import SparseDecodeStep, default_splits
-    from ._lib import sa_build_page_summaries
+    from ._lib import sa_build_page_summaries, sa_build_page_summaries_fp8
 
     dev = torch.device("cuda", 0)
     cfg = W.LLAMA8B_DECODE
     inp = W.gqa_decode_inputs(cfg, seed=args.seed, device=dev)
-    sig = sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
+    if args.fp8:
+        kc, ks = W.fp8_pages(inp.pop("k"))
+        vc, vs = W.fp8_pages(inp.pop("v"))
+        sig = sa_build_page_summaries_fp8(kc, ks, inp["page_table"], inp["seq_lens"])
+    else:
+        sig = sa_build_page_summaries(inp["k"], inp["page_table"], inp["seq_lens"])
     bp = cfg.budget_tokens // cfg.page_size
     n_splits = args.splits or default_splits(cfg.B * cfg.Hkv, bp)
     step = SparseDecodeStep(cfg.B, cfg.T, cfg.Hq, cfg.Hkv, cfg.D, cfg.page_size,
@@ -106,7 +117,7 @@ def main():
     buf = np.zeros(TL_WARPS * TL_SLOTS, dtype=np.uint64)
     flush_w = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(64 << 20, dtype=torch.int32, device=dev)
-    unit_bytes = 16 * cfg.D * 2 * 2
+    unit_bytes = 16 * cfg.D * 2 * (1 if args.fp8 else 2)
     runs = []
     for r in range(args.reps + 3):
         flush_w.fill_(r & 0xFF)
@@ -114,7 +125,10 @@ def main():
         lib.sa_decode_timeline(buf.ctypes.data, buf.size)   # clears the stamps
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        step.decode(inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"])
+        if args.fp8:
+            step.decode_fp8(inp["q"], kc, vc, ks, vs, inp["page_table"], inp["seq_lens"])
+        else:
+            step.decode(inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"])
         e1.record()
         torch.cuda.synchronize()
         st = lib.sa_decode_timeline(buf.ctypes.data, buf.size)
@@ -127,7 +141,8 @@ def main():
     assert int(step.dev_error.item()) == 0
     runs.sort(key=lambda x: x["span"])
     med = runs[len(runs) // 2]
-    print(f"workload {cfg.name}, {n_splits} splits, {med['n_warps']} warps with an item, "
+    kind = " (FP8 pages)" if args.fp8 else ""
+    print(f"workload {cfg.name}{kind}, {n_splits} splits, {med['n_warps']} warps with an item, "
           f"{med['n_units']} units of {unit_bytes} B ({med['units_recorded']} stamped)")
     print("launches (span first start -> last partial stored / CUDA-event time), us: " +
           ", ".join(f"{x['span']:.1f}/{x['event_us']:.1f}" for x in runs))
