@@ -432,10 +432,14 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     SA_TL(1, tl_now());
 #endif
 
-    // Resolve logical -> physical pages of this split.
+    // Resolve logical -> physical pages of this split.  (FP8: the pages'
+    // scales are read after the first copies are issued, so that their round
+    // trip overlaps the copies instead of delaying them.)
+    int phs[kWarpEntries / 32];
 #pragma unroll
     for (int j = 0; j < kWarpEntries / 32; ++j) {
       const int i = lane + 32 * j;
+      phs[j] = -1;
       if (i >= n_ent) continue;
       const int p = pre[j];
       int ph = -1;
@@ -448,11 +452,8 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
           ph = -1;
         }
       }
+      phs[j] = ph;
       ent_s[warp][i] = make_int2(ph, p * a.P);
-      if constexpr (F8)
-        scl_s[warp][i] = ph >= 0 ? make_float2(a.k_scale[(int64_t)ph * a.Hkv + kvh],
-                                               a.v_scale[(int64_t)ph * a.Hkv + kvh])
-                                 : make_float2(0.f, 0.f);
     }
     __syncwarp();
 
@@ -500,9 +501,23 @@ __global__ void __launch_bounds__(kNW * 32, D <= 128 ? 3 : 1)
     if (lane == 0)
       for (int u = 0; u < n_units && u < C::kStages; ++u) issue(u);
 
+    float2 scl[F8 ? kWarpEntries / 32 : 1];
+    if constexpr (F8) {
+#pragma unroll
+      for (int j = 0; j < kWarpEntries / 32; ++j)
+        scl[j] = phs[j] >= 0 ? make_float2(a.k_scale[(int64_t)phs[j] * a.Hkv + kvh],
+                                           a.v_scale[(int64_t)phs[j] * a.Hkv + kvh])
+                             : make_float2(0.f, 0.f);
+    }
     uint32_t qa[D / 16][4];
     int qt[2];
     load_q_frags<D, F8>(qa, qt, a, prm.pairs, pair, b, lane);
+    if constexpr (F8) {
+#pragma unroll
+      for (int j = 0; j < kWarpEntries / 32; ++j)
+        if (lane + 32 * j < n_ent) scl_s[warp][lane + 32 * j] = scl[j];
+      __syncwarp();
+    }
     // FP8: values enter PV scaled by (page scale / v_ref), v_ref = the largest
     // value scale of the split's pages (so P stays <= 256 in f16); the output is
     // multiplied back by v_ref.
