@@ -189,6 +189,34 @@ SA_DEV float reduce_n(const float (&x)[N]) {
     for (int i = 0; i < w; ++i) m[i] = kMin ? fminf(m[i], m[i + w]) : fmaxf(m[i], m[i + w]);
   return m[0];
 }
+// Packed float32 pairs (sm_100 f32x2 arithmetic: each lane of the pair is
+// rounded exactly as the scalar instruction would round it).  `lo` is the low
+// half of the 64-bit register.
+SA_DEV unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+SA_DEV float2 f2_unpack(unsigned long long v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+SA_DEV unsigned long long f2_fma(unsigned long long a, unsigned long long b, unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+SA_DEV unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+SA_DEV unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 // Two floats -> packed bf16x2 (round to nearest even); `lo` in the low half.
 SA_DEV uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);

@@ -357,25 +357,37 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // P = 2^(x sl - m_new) as bf16 hi + lo pairs, written over this tile's
       // scores in TMEM (the S buffer is free: QK^T of the tile is complete and
       // PV of tile jj - 2, the buffer's previous reader, completed before it)
-      float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // (independent chains)
+      // (key pairs in packed float32: the same roundings as the scalar ops,
+      // half the instructions; the row sum in eight independent chains)
+      unsigned long long ls2[4] = {0ull, 0ull, 0ull, 0ull};
+      const unsigned long long sl2 = f2_pack(sl, sl), nb2 = f2_pack(nb, nb);
       uint32_t ph[32], pl[32];
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
-        float p[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float v = x[ch * 8 + i];
-          p[i] = ex2_approx(fmaf(v, sl, nb));
-          if (masked) p[i] = v == v ? p[i] : 0.f;
-          ls[i] += p[i];
-        }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const uint32_t h = pack_bf16(p[2 * i], p[2 * i + 1]);
+          const float v0 = x[ch * 8 + 2 * i], v1 = x[ch * 8 + 2 * i + 1];
+          const float2 z = f2_unpack(f2_fma(f2_pack(v0, v1), sl2, nb2));
+          float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
+          if (masked) {
+            p0 = v0 == v0 ? p0 : 0.f;
+            p1 = v1 == v1 ? p1 : 0.f;
+          }
+          const unsigned long long pp = f2_pack(p0, p1);
+          ls2[i] = f2_add(ls2[i], pp);
+          const uint32_t h = pack_bf16(p0, p1);
+          const float2 d = f2_unpack(f2_sub(
+              pp, f2_pack(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u))));
           ph[ch * 4 + i] = h;
-          pl[ch * 4 + i] = pack_bf16(p[2 * i] - bf16_bits_to_float(h & 0xffffu),
-                                     p[2 * i + 1] - bf16_bits_to_float(h >> 16));
+          pl[ch * 4 + i] = pack_bf16(d.x, d.y);
         }
+      }
+      float ls[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 v = f2_unpack(ls2[i]);
+        ls[2 * i] = v.x;
+        ls[2 * i + 1] = v.y;
       }
       tc::st32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(ph));
       tc::st32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(pl));
