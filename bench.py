@@ -413,9 +413,8 @@ def run_gqa(cfg, args, dev, world, rank, clk, K, fp8=False, n_layers=GQA_LAYERS)
     def step_fn(L):
         i, s = L["inp"], L["step"]
         if fp8:
-            s.select(i["q"], L["sig"], i["page_table"], i["seq_lens"])
-            s.attend_fp8(i["q"], i["kc"], i["vc"], i["ks"], i["vs"], i["page_table"],
-                         i["seq_lens"])
+            s.run_fp8(i["q"], i["kc"], i["vc"], i["ks"], i["vs"], L["sig"], i["page_table"],
+                      i["seq_lens"])
         else:
             s.run(i["q"], i["k"], i["v"], L["sig"], i["page_table"], i["seq_lens"])
 
@@ -482,10 +481,9 @@ def run_gqa(cfg, args, dev, world, rank, clk, K, fp8=False, n_layers=GQA_LAYERS)
         d_out, (s.o, s.lse) = _packed((s.o, s.lse), dev)   # the step writes these views
         h_out, _ = _packed((s.o, s.lse), "cpu")
         if fp8:
-            call = sa.bind(lambda s=s, L=L, q_d=q_d, pt_d=pt_d, sl_d=sl_d: (
-                s.select(q_d, L["sig"], pt_d, sl_d),
-                s.attend_fp8(q_d, L["inp"]["kc"], L["inp"]["vc"], L["inp"]["ks"],
-                             L["inp"]["vs"], pt_d, sl_d)))
+            call = sa.bind(lambda s=s, L=L, q_d=q_d, pt_d=pt_d, sl_d=sl_d: s.run_fp8(
+                q_d, L["inp"]["kc"], L["inp"]["vc"], L["inp"]["ks"], L["inp"]["vs"], L["sig"],
+                pt_d, sl_d))
         else:
             call = s.bind(q_d, i["k"], i["v"], L["sig"], pt_d, sl_d)
         items.append(dict(h_in=h_in, d_in=d_in, d_out=d_out, h_out=h_out, call=call))
@@ -539,7 +537,7 @@ def run_gqa(cfg, args, dev, world, rank, clk, K, fp8=False, n_layers=GQA_LAYERS)
         "e2e": {"value": round(world * kv_total / t_e2e / 1e9, 3), "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(1e3 * t_e2e / K, 4),
-                "what": E2E_WHAT + ("; the step: select and attend, two C calls" if fp8
+                "what": E2E_WHAT + ("; the step: one C call (sa_sparse_step_fp8)" if fp8
                                     else "; the step: one C call (sa_sparse_step)")},
         "gpu_launches": 4 * K,
         "_layers": layers,

@@ -433,6 +433,26 @@ SA_API int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const u
                           size_t workspace_bytes, int32_t* dev_error, void* stream);
 
 /*
+ * sa_sparse_step_fp8 — sa_sparse_step over FP8 E4M3 pages: the selection
+ * (bf16 queries against the bf16 summaries sa_build_page_summaries_fp8 gives),
+ * then sa_sparse_attention_fp8 over the selected lists, in one call.  K and V
+ * as sa_sparse_decode_fp8 (codes [P_pool,Hkv,P,D] with strides, scales
+ * [P_pool,Hkv] float32), D == 128; every other argument, the workspace (sized
+ * by sa_sparse_step_workspace_size) and the errors as sa_sparse_step.
+ */
+SA_API int sa_sparse_step_fp8(const uint16_t* q, const int64_t q_strides[4],
+                              const uint16_t* summaries, const uint8_t* k_codes,
+                              const int64_t k_strides[4], const uint8_t* v_codes,
+                              const int64_t v_strides[4], const float* k_scale,
+                              const float* v_scale, const int32_t* page_table, int max_pages,
+                              const int32_t* seq_lens, int B, int T, int Hq, int Hkv, int D,
+                              int page_size, int P_pool, int sink_tokens, int local_tokens,
+                              int budget_tokens, float scale, int n_splits, int32_t* out_pages,
+                              int32_t* out_counts, float* o_out, uint16_t* o_out_bf16,
+                              float* lse_out, void* workspace, size_t workspace_bytes,
+                              int32_t* dev_error, void* stream);
+
+/*
  * sa_sparse_attention_fp8 — sa_sparse_decode_fp8 followed by the merge, in one
  * call.  Arguments as sa_sparse_decode_fp8 for the inputs and as
  * sa_sparse_attention for the outputs and the workspace (sized with Dv = D).

@@ -11,6 +11,7 @@ from ._lib import (EXPORTED, LIB_PATH, SAError, bind, load, page_budget, sa_bloc
                    sa_sparse_decode, sa_sparse_decode_fp8, sa_build_page_summaries_fp8,
                    sa_sparse_attention, sa_sparse_attention_fp8, attention_workspace,
                    sa_sparse_step, sa_sparse_step_workspace_size, sa_append_kv,
+                   sa_sparse_step_fp8,
                    sa_select_ambient_heads, sa_sparse_decode_at, sa_sparse_attention_at,
                    sa_build_page_summaries_dir, sa_sparse_step_dir, sa_append_kv_dir,
                    dir_capacity)

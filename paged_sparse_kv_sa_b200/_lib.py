@@ -52,6 +52,9 @@ _SIGNATURES = {
     "sa_sparse_step": (_I, [_P, _c_i64_4, _P, _P, _c_i64_4, _P, _c_i64_4, _P, _I, _P, _I, _I, _I,
                             _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P, _P, _P,
                             ctypes.c_size_t, _P, _P]),
+    "sa_sparse_step_fp8": (_I, [_P, _c_i64_4, _P, _P, _c_i64_4, _P, _c_i64_4, _P, _P, _P, _I, _P,
+                                _I, _I, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _P, _P,
+                                _P, _P, ctypes.c_size_t, _P, _P]),
     "sa_build_page_summaries": (_I,[_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sa_update_page_summaries": (_I, [_P, _c_i64_4, _P, _I, _P, _I, _I, _I, _I, _I, _I, _P, _P,
                                       _P]),
@@ -458,6 +461,47 @@ def sa_sparse_step(q, summaries, k_cache, v_cache, page_table, seq_lens, page_si
            float(scale), int(n_splits), _ptr(out_pages), _ptr(out_counts), _ptr(o_out),
            _ptr(o_out_bf16), _ptr(lse_out), _ptr(workspace), workspace.numel(),
            _ptr(dev_error), _stream(stream)), "sa_sparse_step")
+    return out_pages, out_counts, o_out, o_out_bf16, lse_out
+
+
+def sa_sparse_step_fp8(q, summaries, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens,
+                       page_size: int, sink_tokens: int, local_tokens: int, budget_tokens: int,
+                       scale: float, n_splits: int = 0, out_pages=None, out_counts=None,
+                       o_out=None, o_out_bf16=None, lse_out=None, want_f32: bool = True,
+                       want_bf16: bool = False, workspace=None, dev_error=None, stream=None):
+    """sa_sparse_step over FP8 E4M3 pages (codes [P_pool,Hkv,P,D] uint8, scales
+    [P_pool,Hkv] float32, D == 128).  Returns (pages, counts, O f32 or None, O bf16
+    or None, lse)."""
+    lib = load()
+    _need_cuda(q, summaries, k_codes, v_codes, k_scale, v_scale, page_table, seq_lens)
+    _bf16(q), _u8(k_codes), _u8(v_codes), _f32c(k_scale), _f32c(v_scale), _i32(page_table)
+    _i32(seq_lens)
+    if summaries.dtype != torch.bfloat16 or not summaries.is_contiguous():
+        raise TypeError("summaries must be a contiguous bfloat16 tensor")
+    B, T, Hq, D = q.shape
+    P_pool, Hkv, P, _ = k_codes.shape
+    if P != page_size:
+        raise ValueError("page_size differs from the cache's page dimension")
+    bp = budget_tokens // page_size
+    _select_shapes(q, summaries, page_table, seq_lens, out_pages, out_counts, bp)
+    if out_pages is None:
+        out_pages = torch.empty((B, Hkv, max(bp, 1)), dtype=torch.int32, device=q.device)
+    if out_counts is None:
+        out_counts = torch.empty((B, Hkv), dtype=torch.int32, device=q.device)
+    o_out, o_out_bf16, lse_out = _attn_outputs(B, T, Hq, D, q.device, o_out, o_out_bf16,
+                                               lse_out, want_f32, want_bf16)
+    max_pages = page_table.shape[1]
+    if workspace is None:
+        n = sa_sparse_step_workspace_size(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens,
+                                          n_splits)
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=q.device)
+    _call(lib.sa_sparse_step_fp8,
+          (_ptr(q), _strides4(q), _ptr(summaries), _ptr(k_codes), _strides4(k_codes),
+           _ptr(v_codes), _strides4(v_codes), _ptr(k_scale), _ptr(v_scale), _ptr(page_table),
+           max_pages, _ptr(seq_lens), B, T, Hq, Hkv, D, page_size, P_pool, sink_tokens,
+           local_tokens, budget_tokens, float(scale), int(n_splits), _ptr(out_pages),
+           _ptr(out_counts), _ptr(o_out), _ptr(o_out_bf16), _ptr(lse_out), _ptr(workspace),
+           workspace.numel(), _ptr(dev_error), _stream(stream)), "sa_sparse_step_fp8")
     return out_pages, out_counts, o_out, o_out_bf16, lse_out
 
 

@@ -736,7 +736,17 @@ int step_plan(int B, int T, int Hq, int Hkv, int D, int page_size, int max_pages
   return SA_OK;
 }
 
-// sa_sparse_step over either page map (max_pages: the map's capacity).
+// FP8 E4M3 pages of a step: codes in place of the bf16 caches, and their
+// per-(page, kv head) scales.
+struct Fp8Pages {
+  const uint8_t* k_codes;
+  const uint8_t* v_codes;
+  const float* k_scale;
+  const float* v_scale;
+};
+
+// sa_sparse_step over either page map (max_pages: the map's capacity); over
+// FP8 pages when f8 is given (k_cache / v_cache unused then).
 int step_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
               const uint16_t* k_cache, const int64_t k_strides[4], const uint16_t* v_cache,
               const int64_t v_strides[4], const PageMap& pm, int max_pages,
@@ -744,7 +754,7 @@ int step_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* sum
               int P_pool, int sink_tokens, int local_tokens, int budget_tokens, float scale,
               int n_splits, int32_t* out_pages, int32_t* out_counts, float* o_out,
               uint16_t* o_out_bf16, float* lse_out, void* workspace, size_t workspace_bytes,
-              int32_t* dev_error, void* stream) {
+              int32_t* dev_error, void* stream, const Fp8Pages* f8 = nullptr) {
   int splits = 0;
   size_t sel_bytes = 0, total = 0;
   if (int r = step_plan(B, T, Hq, Hkv, D, page_size, max_pages, budget_tokens, n_splits, &splits,
@@ -760,8 +770,15 @@ int step_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* sum
   if (int r = merge_outputs_ok(m)) return r;
   if (!workspace || !aligned16(workspace) || workspace_bytes < total) return SA_ERR_WORKSPACE;
   // every argument of both halves is checked before the first launch
-  if (int r = check_cache(k_cache, k_strides)) return r;
-  if (int r = check_cache(v_cache, v_strides)) return r;
+  if (f8) {
+    if (int r = check_cache_u8(f8->k_codes, k_strides)) return r;
+    if (int r = check_cache_u8(f8->v_codes, v_strides)) return r;
+    if (!f8->k_scale || !f8->v_scale) return SA_ERR_INVALID_ARG;
+    if (D != 128) return SA_ERR_UNSUPPORTED;
+  } else {
+    if (int r = check_cache(k_cache, k_strides)) return r;
+    if (int r = check_cache(v_cache, v_strides)) return r;
+  }
   if (P_pool <= 0 || !std::isfinite(scale)) return SA_ERR_INVALID_ARG;
   if (page_size % 16 != 0 || page_size > 128) return SA_ERR_UNSUPPORTED;
   const int budget_pages = sa_args.budget_pages;
@@ -777,6 +794,12 @@ int step_impl(const uint16_t* q, const int64_t q_strides[4], const uint16_t* sum
   if (int r = cuda_status(launch_select_gqa(sa_args, st))) return r;
   DecodeTarget t{ws + sel_bytes, total - sel_bytes};
   if (pm.blocks) t.dir = pm;
+  if (f8)
+    return sparse_decode_fp8_impl(q, q_strides, f8->k_codes, k_strides, f8->v_codes, v_strides,
+                                  f8->k_scale, f8->v_scale, pm.table, max_pages, seq_lens,
+                                  out_pages, out_counts, Hkv, budget_pages, h2l, B, T, Hq, Hkv, D,
+                                  page_size, P_pool, scale, splits, nullptr, nullptr, dev_error,
+                                  stream, &m, &t);
   return sparse_decode_impl(q, q_strides, k_cache, k_strides, v_cache, v_strides, pm.table,
                             max_pages, seq_lens, out_pages, out_counts, Hkv, budget_pages, h2l, B,
                             T, Hq, Hkv, D, D, page_size, P_pool, scale, splits, nullptr, nullptr,
@@ -810,6 +833,24 @@ int sa_sparse_step(const uint16_t* q, const int64_t q_strides[4], const uint16_t
                    page_size, P_pool, sink_tokens, local_tokens, budget_tokens, scale, n_splits,
                    out_pages, out_counts, o_out, o_out_bf16, lse_out, workspace, workspace_bytes,
                    dev_error, stream);
+}
+
+int sa_sparse_step_fp8(const uint16_t* q, const int64_t q_strides[4], const uint16_t* summaries,
+                       const uint8_t* k_codes, const int64_t k_strides[4],
+                       const uint8_t* v_codes, const int64_t v_strides[4],
+                       const float* k_scale, const float* v_scale, const int32_t* page_table,
+                       int max_pages, const int32_t* seq_lens, int B, int T, int Hq, int Hkv,
+                       int D, int page_size, int P_pool, int sink_tokens, int local_tokens,
+                       int budget_tokens, float scale, int n_splits, int32_t* out_pages,
+                       int32_t* out_counts, float* o_out, uint16_t* o_out_bf16, float* lse_out,
+                       void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                       void* stream) {
+  const Fp8Pages f8{k_codes, v_codes, k_scale, v_scale};
+  return step_impl(q, q_strides, summaries, nullptr, k_strides, nullptr, v_strides,
+                   flat_map(page_table, max_pages), max_pages, seq_lens, B, T, Hq, Hkv, D,
+                   page_size, P_pool, sink_tokens, local_tokens, budget_tokens, scale, n_splits,
+                   out_pages, out_counts, o_out, o_out_bf16, lse_out, workspace, workspace_bytes,
+                   dev_error, stream, &f8);
 }
 
 int sa_sparse_attention_fp8(const uint16_t* q, const int64_t q_strides[4],

@@ -121,6 +121,16 @@ class SparseDecodeStep:
                             o_out_bf16=self.o_bf16, lse_out=self.lse, workspace=self.step_ws,
                             dev_error=self.dev_error, stream=stream)
 
+    def run_fp8(self, q, k_codes, v_codes, k_scale, v_scale, summaries, page_table, seq_lens,
+                stream=None):
+        """run over FP8 E4M3 pages with per-(page, kv head) scales, as one C call
+        (sa_sparse_step_fp8)."""
+        _lib.sa_sparse_step_fp8(q, summaries, k_codes, v_codes, k_scale, v_scale, page_table,
+                                seq_lens, self.P, self.sink, self.local, self.budget, self.scale,
+                                self.n_splits, out_pages=self.pages, out_counts=self.counts,
+                                o_out=self.o, o_out_bf16=self.o_bf16, lse_out=self.lse,
+                                workspace=self.step_ws, dev_error=self.dev_error, stream=stream)
+
     def bind(self, q, k_cache, v_cache, summaries, page_table, seq_lens, stream=None):
         """A zero-argument callable that runs `run` on these tensors: the arguments
         are checked and marshalled once (_lib.bind; the tensors must stay where

@@ -278,6 +278,43 @@ def test_step_vs_oracle(D, P, T, n_splits):
     assert_attn_close(o, lse, ro, rl)
 
 
+@pytest.mark.parametrize("P,T,n_splits", [(16, 1, 0), (32, 2, 3)])
+def test_step_fp8_vs_oracle(P, T, n_splits):
+    # sa_sparse_step_fp8: selection on the FP8 pages' summaries, attention over the
+    # FP8 pages and the merge in one C call, against the oracle; and the same bits
+    # as the selection and the FP8 attention called one after the other
+    cfg = W.GQADecode("case", B=3, Hq=8, Hkv=2, D=128, page_size=P, seq_len_lo=0, seq_len_hi=0,
+                      sink_tokens=P, local_tokens=2 * P, budget_tokens=12 * P, T=T)
+    lens = [50 * P + 7, 9 * P, 3 * P + 1]
+    inp, g, f8, f8d = fp8_case(cfg, seed=64, seq_lens=lens)
+    sig = O.page_summaries_fp8(f8["kc"].numpy(), f8["ks"].numpy(), np_i32(inp["page_table"]),
+                               np_i32(inp["seq_lens"]), P)
+    sig_d = to_bf16_dev(sig)
+    scale = 1.0 / math.sqrt(cfg.D)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    pages, counts, o, _, lse = sa.sa_sparse_step_fp8(
+        g["q"], sig_d, f8d["kc"], f8d["vc"], f8d["ks"], f8d["vs"], g["page_table"],
+        g["seq_lens"], P, cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens, scale, n_splits,
+        dev_error=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    rp, rc = O.select_pages(bits(inp["q"]), sig, np_i32(inp["page_table"]),
+                            np_i32(inp["seq_lens"]), P, cfg.sink_tokens, cfg.local_tokens,
+                            cfg.budget_tokens)
+    assert np.array_equal(np_i32(counts), rc) and np.array_equal(np_i32(pages), rp)
+    ro, rl = oracle_fp8(inp, f8, rp, rc, cfg)
+    assert_attn_close(o, lse, ro, rl)
+    # the two-call path gives the same bits
+    p2, c2 = sa.sa_select_pages(g["q"], sig_d, g["page_table"], g["seq_lens"], P,
+                                cfg.sink_tokens, cfg.local_tokens, cfg.budget_tokens)
+    ns = n_splits or sa.default_splits(cfg.B * cfg.Hkv, cfg.budget_tokens // P)
+    o2, _, l2 = sa.sa_sparse_attention_fp8(g["q"], f8d["kc"], f8d["vc"], f8d["ks"], f8d["vs"],
+                                           g["page_table"], g["seq_lens"], p2, c2,
+                                           [h // cfg.G for h in range(cfg.Hq)], scale, ns)
+    torch.cuda.synchronize()
+    assert torch.equal(p2, pages) and torch.equal(o2, o) and torch.equal(l2, lse)
+
+
 def test_bound_calls_replay_on_new_contents():
     # sa.bind records the C calls of a step once; replaying them after the input
     # tensors' contents change (same storage) must give what fresh calls give
