@@ -458,22 +458,31 @@ __global__ void __launch_bounds__(kMThreads, 1)
       // and QK of this tile is complete)
       uint8_t* prow = p_s + r * 128;
       uint8_t* lrow = k_s + (jj % kMStages) * kTileBytes + (kKC - 1) * kChunkBytes + r * 128;
+      // (key pairs in packed float32: the same roundings as the scalar ops)
+      const unsigned long long sl2x = f2_pack(sl2, sl2), nb2x = f2_pack(nb, nb);
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
         float p[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = v[ch * 8 + i];
-          p[i] = ex2_approx(fmaf(x, sl2, nb));
-          if (masked) p[i] = x == x ? p[i] : 0.f;
+        for (int i = 0; i < 4; ++i) {
+          const float x0 = v[ch * 8 + 2 * i], x1 = v[ch * 8 + 2 * i + 1];
+          const float2 z = f2_unpack(f2_fma(f2_pack(x0, x1), sl2x, nb2x));
+          p[2 * i] = ex2_approx(z.x);
+          p[2 * i + 1] = ex2_approx(z.y);
+          if (masked) {
+            p[2 * i] = x0 == x0 ? p[2 * i] : 0.f;
+            p[2 * i + 1] = x1 == x1 ? p[2 * i + 1] : 0.f;
+          }
         }
         l += ((p[0] + p[1]) + (p[2] + p[3])) + ((p[4] + p[5]) + (p[6] + p[7]));
         uint32_t hw[4], lw[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           hw[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
-          lw[i] = pack_bf16(p[2 * i] - bf16_bits_to_float(hw[i] & 0xffffu),
-                            p[2 * i + 1] - bf16_bits_to_float(hw[i] >> 16));
+          const float2 d = f2_unpack(f2_sub(f2_pack(p[2 * i], p[2 * i + 1]),
+                                            f2_pack(__uint_as_float(hw[i] << 16),
+                                                    __uint_as_float(hw[i] & 0xffff0000u))));
+          lw[i] = pack_bf16(d.x, d.y);
         }
         const int off = (((low ? 0 : 4) + ch) ^ (r & 7)) << 4;
         *reinterpret_cast<uint4*>(prow + off) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
@@ -492,17 +501,21 @@ __global__ void __launch_bounds__(kMThreads, 1)
     // the normalised O rows are staged in shared memory (the key ring is free:
     // every tile's PV is done) and leave with one 2 KB bulk store per row
     uint8_t* stg = k_s + r * kStageRow;
-    for (int c = 0; c < 256 / 32; ++c) {
-      float o[32];
+    for (int c = 0; c < 256 / 32; c += 2) {   // two TMEM loads in flight per wait
+      float o[2][32];
       if (n_act > 0) {
-        tc::ld32(tmem + lane_base + c * 32, o);
+        tc::ld32(tmem + lane_base + c * 32, o[0]);
+        tc::ld32(tmem + lane_base + (c + 1) * 32, o[1]);
         tc::wait_ld();
       }
 #pragma unroll
-      for (int i = 0; i < 32; i += 4)
-        *reinterpret_cast<float4*>(stg + (low ? 0 : 1024) + (c * 32 + i) * 4) =
-            empty ? make_float4(0.f, 0.f, 0.f, 0.f)
-                  : make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int i = 0; i < 32; i += 4)
+          *reinterpret_cast<float4*>(stg + (low ? 0 : 1024) + ((c + h) * 32 + i) * 4) =
+              empty ? make_float4(0.f, 0.f, 0.f, 0.f)
+                    : make_float4(o[h][i] * inv, o[h][i + 1] * inv, o[h][i + 2] * inv,
+                                  o[h][i + 3] * inv);
     }
     tc::fence_proxy_async();
     __syncwarp();
