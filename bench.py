@@ -79,8 +79,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0,
-                    help="distinct layer caches the Llama-8B-shaped steps cycle (0 = %d); "
-                         "1 keeps a profiler capture to one 2 GiB cache" % GQA_LAYERS)
+                    help="distinct layer caches the Llama-8B-shaped steps (0 = %d) and the MLA "
+                         "graph (0 = %d) cycle; a small count keeps a profiler capture to a few "
+                         "GB" % (GQA_LAYERS, MLA_LAYERS))
     ap.add_argument("--workload", default="all",
                     choices=["all", "llama8b", "llama70b", "mla", "prefill", "llama8b_fp8",
                              "dir_1m"],
@@ -91,6 +92,10 @@ def parse():
 
 def gqa_layers(args):
     return args.layers if args.layers > 0 else GQA_LAYERS
+
+
+def mla_layers(args):
+    return args.layers if args.layers > 0 else MLA_LAYERS
 
 
 def peaks():
@@ -666,6 +671,7 @@ def run_mla(args, dev, world, rank, clk, reps):
     cfg = W.MLA_MTP
     stream = torch.cuda.current_stream(dev)
     n_splits = args.splits or 8
+    n_ml = mla_layers(args)
     cap = cfg.alpha + cfg.beta
     scale = 1.0 / math.sqrt(cfg.Dk)
     o = torch.empty((cfg.B, cfg.T, cfg.Hq, cfg.Dv), dtype=torch.float32, device=dev)
@@ -674,7 +680,7 @@ def run_mla(args, dev, world, rank, clk, reps):
     l_p = torch.empty((n_splits, cfg.B, cfg.T, cfg.Hq), dtype=torch.float32, device=dev)
     aws = sa.attention_workspace(cfg.B, cfg.T, cfg.Hq, cfg.Dv, n_splits, dev)
     layers = []
-    for l in range(MLA_LAYERS):
+    for l in range(n_ml):
         inp = W.mla_decode_inputs(cfg, seed=args.seed + 1000 * rank + l, device=dev)
         sig = sa.sa_build_page_summaries(inp["kv"], inp["page_table"], inp["seq_lens"])
         amb = set(int(h) for h in inp["ambient_heads"].tolist())
@@ -735,7 +741,7 @@ def run_mla(args, dev, world, rank, clk, reps):
         torch.cuda.synchronize()
         t_step = time_back_to_back([g_step], reps, stream, world, dev)
         t_dec = time_back_to_back([g_dec], reps, stream, world, dev)
-    n = reps * MLA_LAYERS
+    n = reps * n_ml
     assert torch.isfinite(o).all().item(), "non-finite output"
 
     # end to end through the public API over the first eight layers' caches (cycled):
@@ -760,17 +766,17 @@ def run_mla(args, dev, world, rank, clk, reps):
         t_e2e = time_e2e(items, K, stream, world, dev)
     h_in, h_out = items[0]["h_in"], items[0]["h_out"]
     pk, kind = peaks()
-    per_call_flops = flops / MLA_LAYERS
-    per_call_bytes = kv_bytes / MLA_LAYERS
+    per_call_flops = flops / n_ml
+    per_call_bytes = kv_bytes / n_ml
     achieved = per_call_flops / (t_dec / n) / 1e12
     return {
         "value": round(world * kv_bytes * reps / t_step / 1e9, 3), "unit": "GB/s",
         "steps": n, "ms_per_step": round(1e3 * t_step / n, 4),
         "calls_per_sec": round(world * n / t_step, 2),
-        "config": {"workload": cfg.name, "n_splits": n_splits, "layer_caches": MLA_LAYERS,
-                   "timing": f"CUDA graph of {MLA_LAYERS} back-to-back layer calls over "
-                             f"{MLA_LAYERS} distinct latent caches, replayed {reps} times",
-                   "l2": "inputs larger than L2 (61 x 604 MB of caches cycled)"},
+        "config": {"workload": cfg.name, "n_splits": n_splits, "layer_caches": n_ml,
+                   "timing": f"CUDA graph of {n_ml} back-to-back layer calls over "
+                             f"{n_ml} distinct latent caches, replayed {reps} times",
+                   "l2": f"inputs larger than L2 ({n_ml} x 604 MB of caches cycled)"},
         "selected_kv_bytes_per_step": int(per_call_bytes), "flops_per_step": int(per_call_flops),
         "step_tflops": round(world * flops * reps / t_step / 1e12, 2),
         "roofline": {"kernel": "mla_kernel", "bound": "tensor", "achieved": round(achieved, 2),
@@ -779,11 +785,11 @@ def run_mla(args, dev, world, rank, clk, reps):
                      "peak_kind": f"{kind} bf16 GEMM, sustained (a long loop of launches)",
                      "traffic": None,
                      "kernel_us": round(1e6 * t_dec / n, 2),
-                     "kernel_us_what": f"average launch in a graph of {MLA_LAYERS} "
+                     "kernel_us_what": f"average launch in a graph of {n_ml} "
                                        "back-to-back decode launches",
                      "hbm_achieved_gbs": round(per_call_bytes / (t_dec / n) / 1e9, 1),
                      "hbm_frac": round(per_call_bytes / (t_dec / n) / 1e9 / pk["hbm_gbs"], 4)},
-        "e2e": {"value": round(world * (kv_bytes / MLA_LAYERS) * K / t_e2e / 1e9, 3),
+        "e2e": {"value": round(world * (kv_bytes / n_ml) * K / t_e2e / 1e9, 3),
                 "unit": "GB/s", "h2d_bytes_per_step": h_in.numel(),
                 "d2h_bytes_per_step": h_out.numel(), "ms_per_step": round(1e3 * t_e2e / K, 4),
                 "what": E2E_WHAT + "; the step: select and attend (two C calls), eight layer "
@@ -1075,7 +1081,7 @@ def main():
     wl = args.workload
     try:
         if wl in ("mla", "prefill", "dir_1m"):
-            sub = (run_mla(args, dev, world, rank, clk, reps=max(1, -(-K // MLA_LAYERS)))
+            sub = (run_mla(args, dev, world, rank, clk, reps=max(1, -(-K // mla_layers(args))))
                    if wl == "mla" else run_prefill(args, dev, world, rank, clk, K)
                    if wl == "prefill" else run_dir(args, dev, world, rank, clk, K))
             line = {"metric": METRIC, "n_gpus": world, "warmup": args.warmup,
@@ -1102,7 +1108,8 @@ def main():
                 r.pop("_layers")
                 subs["llama8b_fp8"] = r
                 torch.cuda.empty_cache()
-                subs["mla"] = run_mla(args, dev, world, rank, clk, reps=max(2, -(-K // 61)))
+                subs["mla"] = run_mla(args, dev, world, rank, clk,
+                                      reps=max(2, -(-K // mla_layers(args))))
                 torch.cuda.empty_cache()
                 subs["prefill"] = run_prefill(args, dev, world, rank, clk, min(K, 20))
                 torch.cuda.empty_cache()
