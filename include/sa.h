@@ -37,8 +37,11 @@
  * Conventions for every call:
  *  - Pointers marked (dev) are caller-owned device memory on the current
  *    device; (host) pointers are read before the call returns.  The library
- *    allocates nothing and keeps no state between calls; scratch space
- *    (workspace) is caller-owned device memory of the size a *_size call gives.
+ *    allocates no memory in a call and carries no data from one call to the
+ *    next (it caches only per-context launch set-up: shared-memory caps, SM
+ *    count, occupancy; sa_select_pages_no_alloc's static array is described
+ *    there); scratch space (workspace) is caller-owned device memory of the
+ *    size a *_size call gives.
  *  - bf16 tensors are passed as uint16_t bit patterns.  Strides are in
  *    elements; the innermost (feature) stride must be 1, other strides of
  *    bf16 tensors multiples of 8 elements, base pointers 16-byte aligned.

@@ -326,7 +326,7 @@ __global__ void __launch_bounds__((kScoreMaxHB + 1) * 32) score_kernel(const Sel
 // hi_p >= the k-th largest lo) over every page.  The undecided pages are then
 // rescored exactly and ranked, and the output is the sink pages, the selected
 // pages and the local pages, ascending.
-__global__ void __launch_bounds__(kThreads) choose_kernel(const SelectArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) choose_kernel(const SelectArgs a) {
   pdl_wait_and_release();
   const int kvh = blockIdx.x, b = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
