@@ -36,7 +36,10 @@ constexpr int kSelGroups = 256;     // choose_kernel: group maxima behind the pr
 constexpr int kCandCap = 1024;      // choose_kernel: candidates classified by counting (more:
                                     // order statistics of the bounds over every page)
 static_assert(kSelGroups <= kThreads, "one thread clears each group maximum");
-constexpr int kScoreChunk = 128;    // score_kernel: logical pages per CTA
+#ifndef SA_SCORE_CHUNK
+#define SA_SCORE_CHUNK 128
+#endif
+constexpr int kScoreChunk = SA_SCORE_CHUNK;   // score_kernel: logical pages per CTA
 constexpr int kScoreStages = 2;     // ring slots of 16 pages
 constexpr int kScoreMaxHB = 8;      // kv heads per CTA (one consumer warp each)
 
