@@ -7,7 +7,11 @@ library's default), a flat or a two-level page map, and a scale between -2 and
 +3 times 1/sqrt(D).  The selection must equal the oracle's bit for bit, O and
 LSE hold the 2e-3 / 1e-3 bar.  A second set appends a random number of tokens
 to random sequences through the two-level map and checks pools and summaries
-bit for bit.
+bit for bit.  A third draws MLA + MTP shapes (1-3 query tokens, 8-128 heads,
+pages of 16-128 tokens, tier depths, ambient head counts, splits, scales)
+through the tiered selection and the MLA decode, and a fourth many-row shapes
+(17-159 query tokens, the tcgen05 kernel) over random page lists with the
+queries at explicit positions.
 """
 import math
 
@@ -137,3 +141,91 @@ def test_fuzz_append_dir_vs_oracle(seed):
     assert np.array_equal(bits(kd), rk) and np.array_equal(bits(vd), rv)
     assert np.array_equal(bits(sd), rs)
     assert np.array_equal(out_len.cpu().numpy(), rl)
+
+
+@pytest.mark.parametrize("seed", range(16))
+def test_fuzz_mla_tiers_and_decode_vs_oracle(seed):
+    # MLA + MTP: tiered selection bit-exact, then the decode over the oracle's
+    # tiers (critical heads: list 0; ambient heads: critical + ambient, list 1)
+    rng = np.random.default_rng(5000 + seed)
+    T = int(rng.choice([1, 2, 3]))
+    Hq = int(rng.choice([8, 16, 32, 64, 128]))
+    P = int(rng.choice([16, 32, 64, 128]))
+    B = int(rng.integers(1, 4))
+    L = int(rng.integers(1, 3000))
+    alpha, beta = int(rng.integers(0, 9)), int(rng.integers(1, 25))
+    h = int(rng.integers(1, Hq + 1))
+    n_splits = int(rng.integers(1, 5))
+    mult = float(rng.choice([-1.0, 1.0, 2.0]))
+    cfg = W.MLADecode("fuzz", B=B, T=T, Hq=Hq, Dk=576, Dv=512, page_size=P, seq_len=L,
+                      alpha=alpha, beta=beta, h_ambient=h)
+    inp = W.mla_decode_inputs(cfg, seed=6000 + seed, device="cpu")
+    pt, sl = np_i32(inp["page_table"]), np_i32(inp["seq_lens"])
+    sig = O.page_summaries(bits(inp["kv"]), pt, sl, P)
+    g = {k: (v.to(DEV) if torch.is_tensor(v) else v) for k, v in inp.items()}
+    lists, counts = sa.sa_select_pages_tiered(g["q"], to_bf16_dev(sig), g["page_table"],
+                                              g["seq_lens"], P, alpha, beta)
+    torch.cuda.synchronize()
+    lists, counts = np_i32(lists), np_i32(counts)
+    crit, cc, amb, ac = O.select_pages_mla(bits(inp["q"]), sig, pt, sl, P, alpha, beta)
+    cap = alpha + beta
+    want = np.full((B, 2, cap), -1, dtype=np.int32)
+    wc = np.zeros((B, 2), dtype=np.int32)
+    for b in range(B):
+        c0 = list(crit[b, :cc[b]])
+        c1 = sorted(c0 + list(amb[b, :ac[b]]))
+        want[b, 0, :len(c0)], want[b, 1, :len(c1)] = c0, c1
+        wc[b] = len(c0), len(c1)
+    assert np.array_equal(counts, wc) and np.array_equal(lists, want), (seed, L, alpha, beta)
+    ambs = set(int(x) for x in inp["ambient_heads"].tolist())
+    h2l = [1 if hh in ambs else 0 for hh in range(Hq)]
+    scale = mult / math.sqrt(576)
+    kv = g["kv"]
+    o, _, lse = sa.sa_sparse_attention(g["q"], kv, kv[..., :512], g["page_table"], g["seq_lens"],
+                                       torch.from_numpy(want).to(DEV), torch.from_numpy(wc).to(DEV),
+                                       h2l, scale, n_splits)
+    torch.cuda.synchronize()
+    kvb = bits(inp["kv"])
+    ro, rl = O.sparse_attention(bits(inp["q"]), kvb, kvb[..., :512], pt, sl, want, wc,
+                                np.array(h2l), scale, P)
+    assert_attn_close(o, lse, ro, rl)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_fuzz_many_rows_at_positions_vs_oracle(seed):
+    # more than 16 query rows per (list, kv head) pair -- the tcgen05 kernel --
+    # over random per-group page lists, with queries at explicit positions
+    rng = np.random.default_rng(7000 + seed)
+    D = int(rng.choice([64, 128]))
+    P = int(rng.choice([16, 32, 64]))
+    Hkv = int(rng.choice([1, 2]))
+    G = int(rng.choice([1, 2, 4]))
+    T = int(rng.integers(17, 160))
+    B = int(rng.integers(1, 3))
+    lens = [int(rng.integers(P, 2500)) for _ in range(B)]
+    cfg = W.GQADecode("fuzz", B=B, Hq=Hkv * G, Hkv=Hkv, D=D, page_size=P, seq_len_lo=0,
+                      seq_len_hi=0, sink_tokens=P, local_tokens=P, budget_tokens=4 * P, T=T)
+    inp, g = gqa_case(cfg, seed=8000 + seed, seq_lens=lens)
+    cap = int(rng.integers(1, 40))
+    lists = np.full((B, Hkv, cap), -1, dtype=np.int32)
+    counts = np.zeros((B, Hkv), dtype=np.int32)
+    for b, L in enumerate(lens):
+        n_pg = -(-L // P)
+        for kvh in range(Hkv):
+            k = int(rng.integers(0, min(cap, n_pg) + 1))
+            sel = np.sort(rng.choice(n_pg, size=k, replace=False)).astype(np.int32)
+            lists[b, kvh, :k] = sel
+            counts[b, kvh] = k
+    q_pos = np.array([int(rng.integers(-T // 2, L + 50)) for L in lens], dtype=np.int32)
+    scale = float(rng.choice([-1.0, 1.0, 3.0])) / math.sqrt(D)
+    n_splits = int(rng.integers(1, 4))
+    h2l = [hh // G for hh in range(cfg.Hq)]
+    o, _, lse = sa.sa_sparse_attention_at(g["q"], g["k"], g["v"], g["page_table"], g["seq_lens"],
+                                          torch.from_numpy(q_pos).to(DEV),
+                                          torch.from_numpy(lists).to(DEV),
+                                          torch.from_numpy(counts).to(DEV), h2l, scale, n_splits)
+    torch.cuda.synchronize()
+    ro, rl = O.sparse_attention(bits(inp["q"]), bits(inp["k"]), bits(inp["v"]),
+                                np_i32(inp["page_table"]), np_i32(inp["seq_lens"]), lists, counts,
+                                np.array(h2l), scale, P, q_pos=q_pos)
+    assert_attn_close(o, lse, ro, rl)
