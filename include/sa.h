@@ -259,7 +259,7 @@ SA_API int sa_select_ambient_heads(const uint16_t* q, const int64_t q_strides[4]
  *  head_to_list (host) [Hq] int32 in [0, n_lists)
  *  o_partial    (dev) [n_splits,B,T,Hq,Dv] float32
  *  lse_partial  (dev) [n_splits,B,T,Hq] float32
- * Kernels, chosen from the shapes (P in {16,32,64,128} throughout):
+ * Kernels, chosen from the shapes (P a multiple of 16 up to 128 throughout):
  *  - at most 16 query rows (T x heads) per (list, kv head) pair, Dk == Dv in
  *    {64,128,256}: one warp per split, warp-level tensor-core MMAs;
  *  - more rows per pair (chunked prefill, long MTP), Dk == Dv in {64,128}:

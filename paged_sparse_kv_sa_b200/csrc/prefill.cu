@@ -1,33 +1,35 @@
 // Sparse attention over per-head page lists for many query rows per (list,
-// kv head) pair — chunked prefill over block-union tables, long MTP — on the
+// kv head) pair -- chunked prefill over block-union tables, long MTP -- on the
 // 5th-generation tensor cores.
 //
 // One CTA computes 256 query rows of a pair (token-major) as two 128-row tiles
-// A and B against the keys of its split of the list, 64 keys per tile; each
+// A and B against the keys of its split of the list, 128 keys per tile; each
 // K/V tile is loaded once and used by both:
-//   warp 8      gathers K and V tiles from the paged pool with TMA (four
-//               16-key x 64-column boxes per 64-column chunk; an absent or
-//               invalid 16-key group is loaded from an out-of-range page
-//               coordinate, which TMA fills with zeros) into a 4-stage ring;
-//   warp 9      issues tcgen05.mma, alternating between the tiles: S_A = Q_A K^T
-//               and S_B = Q_B K^T (M=128, N=64, K=D) into double-buffered TMEM
-//               S buffers, then O_A += P_A V and O_B += P_B V (M=128, N=D) into
-//               TMEM with P read from TMEM as the A operand, with
-//               tcgen05.commit arrivals on mbarriers;
+//   warp 8      gathers K and V tiles from the paged pool with TMA (16-key x
+//               64-column boxes; an absent or invalid 16-key group is loaded
+//               from an out-of-range page coordinate, which TMA fills with
+//               zeros) into separate K and V rings of two (D = 128) or four
+//               (D = 64) stages;
+//   warp 9      issues tcgen05.mma: S_w = Q_w K^T (M=128, N=128, K=D) into one
+//               TMEM S buffer per tile w, and O_w += P_w V (M=128, N=D) with P
+//               read from the TMEM columns of S_w as the A operand, in the order
+//               PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1): the tensor core works
+//               on one tile while the other tile's softmax runs;
 //   warps 0-3 / 4-7   (one warpgroup per tile) own one query row per thread:
 //               Q into shared memory, S rows from TMEM, masking (page validity,
 //               sequence end, causal position; skipped for tiles every row sees
 //               whole), a base-2 online softmax whose running max only moves when
 //               a row's max exceeds it by more than 2^8 (the O rescale through
-//               TMEM is then rare), P back into the S buffer it came from, and
-//               the epilogue.
+//               TMEM is then rare), P back into the S columns it came from, in
+//               two halves of 64 keys (PV of the first half runs while the
+//               second is computed), and the epilogue.
 // P enters PV as a bf16 pair hi + lo (hi = RNE_bf16(p), lo = RNE_bf16(p - hi)),
 // so its rounding is ~2^-17 relative rather than the 2^-9 of a single bf16: two
-// MMAs per 16 keys, both reading the pair from the TMEM columns where that
-// tile's scores were (64 keys = 32 columns of hi pairs + 32 of lo pairs).
-// A softmax warpgroup computes P of tile j while the tensor core still runs
-// PV of tile j-1 and QK^T of tile j+1; it waits for PV of tile j-1 only
-// before handing P of tile j over (and before the rare rescale of O).
+// MMAs per 16 keys, reading the pair from the TMEM columns where those keys'
+// scores were (per 16 keys: 8 columns of hi pairs, then 8 of lo pairs).
+// Single-buffered S costs no wait: the commit that announces S_w(j) tracks
+// every MMA issued before it, PV_w(j-1) included, so when the softmax sees
+// S_w(j) the previous P is consumed and O_w may be rescaled.
 //
 // Sources: CompactAttention (abstract on the page titled "Causal Attention on
 // CPU: A Cache-Aware and Load-Balanced Scheduling Kernel for Prefill"):
@@ -38,12 +40,24 @@
 #include "internal.h"
 #include "tc05.cuh"
 
+// Diagnostic build (-DSA_PREFILL_TIMELINE=1, off in the library): the first
+// kPtCtas CTAs of a launch record SM clock stamps per key tile -- the MMA
+// thread's waits and issues and both softmax warpgroups' phases -- read back
+// with sa_prefill_timeline().
+#ifndef SA_PREFILL_TIMELINE
+#define SA_PREFILL_TIMELINE 0
+#endif
+
 namespace sa {
+#if SA_PREFILL_TIMELINE
+constexpr int kPtCtas = 4, kPtIters = 256, kPtSlots = 12;
+__device__ long long g_prefill_tl[kPtCtas * kPtIters * kPtSlots];
+#endif
 namespace {
 
 constexpr int kPThreads = 320;    // 2 softmax warpgroups, producer warp, MMA warp
-constexpr int kPStages = 4;
-constexpr int kKeys = 64;         // keys per tile
+constexpr int kKeys = 128;        // keys per tile
+constexpr int kGroups = kKeys / 16;
 constexpr int kM = 128;           // query rows per warpgroup tile
 constexpr int kRows = 2 * kM;     // query rows per CTA
 constexpr int kMaxEnt = 1024;     // list entries per split
@@ -54,10 +68,9 @@ struct PCfg {
   static constexpr int kChunks = D / 64;               // 64-column (128-byte) chunks
   static constexpr int kQBytes = kM * D * 2;
   static constexpr int kTileBytes = kKeys * D * 2;     // one K (or V) tile
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kDyn = 2 * kQBytes + kPStages * kStageBytes + 1024;
-  // per tile w: S buffers at 128w + {0, 64} (P hi + lo after the softmax:
-  // columns +0..31 and +32..63), O at 256 + 128w
+  static constexpr int kStages = D == 64 ? 4 : 2;      // per ring (K and V)
+  static constexpr int kDyn = 2 * kQBytes + 2 * kStages * kTileBytes + 1024;
+  // tile w: S (then P hi + lo) at columns 128w .. 128w + 127, O at 256 + D w
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kIdQK = tc::idesc_bf16_f32(kM, kKeys, false, false);
   static constexpr uint32_t kIdPV = tc::idesc_bf16_f32(kM, D, false, true);
@@ -78,21 +91,15 @@ SA_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_fl
   return false;
 }
 
-// (physical page or -1, first token) of 16-key group g of tile j.
+// (physical page or -1, first token) of 16-key group g of tile j: the tiles cut
+// the concatenation of the split's pages into runs of kKeys keys (a page size
+// is a multiple of 16, so a group never straddles two pages).
 SA_DEV int2 group_of(const int2* ent, int n_ent, int P, int j, int g) {
-  int e, row0;
-  if (P <= kKeys) {
-    const int per = kKeys / P;                 // entries per tile
-    e = j * per + (g * 16) / P;
-    row0 = (g * 16) % P;
-  } else {
-    const int per = P / kKeys;                 // tiles per entry
-    e = j / per;
-    row0 = (j % per) * kKeys + g * 16;
-  }
+  const int key0 = (j * kGroups + g) * 16;
+  const int e = key0 / P;
   if (e >= n_ent) return make_int2(-1, 0);
   const int2 en = ent[e];
-  return make_int2(en.x, en.y + row0);
+  return make_int2(en.x, en.y + key0 % P);
 }
 
 template <int D>
@@ -110,13 +117,28 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (qt * kRows >= rows_total) return;               // whole CTA: nothing to do
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int list = prm.pairs.list_of[pair], kvh = prm.pairs.kvh_of[pair];
+#if SA_PREFILL_TIMELINE
+  // slots per key tile: 0 K in (before QK_A), 1 QK_B issued, 2 / 3 second half of
+  // P of tiles A / B in (the MMA thread), 4 / 7 S in, 5 / 8 all of P written,
+  // 6 / 9 first half of P written (softmax A / B); tile 0 slot 10: start,
+  // slot 11: tiles
+  const int pt_cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  long long* pt_row = pt_cta < kPtCtas ? g_prefill_tl + (int64_t)pt_cta * kPtIters * kPtSlots
+                                       : nullptr;
+  auto pt_mark = [&](int it, int slot) {
+    if (pt_row && it >= 0 && it < kPtIters) pt_row[it * kPtSlots + slot] = clock64();
+  };
+  if (tid == 0) pt_mark(0, 10);
+#endif
 
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = dyn_smem + ((1024 - (smem_u32(dyn_smem) & 1023)) & 1023);
   uint8_t* q_s = smem;                                       // 2 tiles
-  uint8_t* kv_s = smem + 2 * C::kQBytes;                     // kPStages x (K | V)
-  __shared__ uint64_t kv_full[kPStages], kv_empty[kPStages];
-  __shared__ uint64_t s_full[2][2], p_full[2], o_done[2], q_full;
+  uint8_t* k_s = smem + 2 * C::kQBytes;                      // kStages K tiles
+  uint8_t* v_s = k_s + C::kStages * C::kTileBytes;           // kStages V tiles
+  __shared__ uint64_t k_full[C::kStages], k_empty[C::kStages];
+  __shared__ uint64_t v_full[C::kStages], v_empty[C::kStages];
+  __shared__ uint64_t s_full[2], p_full[2][2], o_done[2], q_full;
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, n_act_s;
   __shared__ int2 ent_s[kMaxEnt];
@@ -171,14 +193,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
     ent_s[i] = make_int2(ph, p * a.P);
   }
   if (tid == 0) {
-    for (int s = 0; s < kPStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int w = 0; w < 2; ++w) {
-      mbar_init(&s_full[w][0], 1);
-      mbar_init(&s_full[w][1], 1);
-      mbar_init(&p_full[w], 128);
+      mbar_init(&s_full[w], 1);
+      mbar_init(&p_full[w][0], 128);
+      mbar_init(&p_full[w][1], 128);
       mbar_init(&o_done[w], 1);
     }
     mbar_init(&q_full, 256);
@@ -194,14 +218,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
   // ---- tiles with at least one causally visible key, in list order; a tile
   // every row of the CTA sees whole (all groups valid and below min_q) skips
   // the per-element mask
-  const int n_tiles = a.P <= kKeys ? (n_ent * a.P + kKeys - 1) / kKeys : n_ent * (a.P / kKeys);
+  const int n_tiles = (n_ent * a.P + kKeys - 1) / kKeys;
   if (warp == 0) {
     int n_act = 0;
     for (int j0 = 0; j0 < n_tiles; j0 += 32) {
       const int j = j0 + lane;
       bool live = false, whole = true;
       if (j < n_tiles)
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < kGroups; ++g) {
           const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
           live |= gr.x >= 0 && gr.y < L && gr.y <= max_q;
           whole &= gr.x >= 0 && gr.y + 15 < L && gr.y + 15 <= min_q;
@@ -215,6 +239,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __syncthreads();
   const int n_act = n_act_s;
   volatile int* abort_flag = &abort_s;
+#if SA_PREFILL_TIMELINE
+  if (tid == 0 && pt_row) pt_row[11] = n_act;
+#endif
 
   if (warp == 8) {
     // ================= producer: TMA gathers of K and V tiles
@@ -222,78 +249,122 @@ __global__ void __launch_bounds__(kPThreads, 1)
       prefetch_tmap(&kmap);
       prefetch_tmap(&vmap);
       for (int jj = 0; jj < n_act; ++jj) {
-        const int st = jj % kPStages;
-        if (jj >= kPStages &&
-            !wait_or_abort(&kv_empty[st], ((jj / kPStages) - 1) & 1, abort_flag))
-          break;
-        const int j = act_s[jj] >> 1;
-        uint8_t* kt = kv_s + st * C::kStageBytes;
-        uint8_t* vt = kt + C::kTileBytes;
-        mbar_arrive_expect_tx(&kv_full[st], C::kStageBytes);
+        const int st = jj % C::kStages, j = act_s[jj] >> 1;
+        const uint32_t ph = ((jj / C::kStages) - 1) & 1;
+        int page[kGroups], row0[kGroups];
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
+        for (int g = 0; g < kGroups; ++g) {
           const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
           const bool ok = gr.x >= 0 && gr.y < L;
           // an out-of-range page coordinate makes TMA write zeros for the box
-          const int page = ok ? gr.x : a.P_pool;
-          const int row0 = ok ? gr.y % a.P : 0;
-#pragma unroll
-          for (int c = 0; c < C::kChunks; ++c) {
-            tma_load_4d(kt + c * (kKeys * 128) + g * 2048, &kmap, &kv_full[st], c * 64, row0, kvh,
-                        page);
-            tma_load_4d(vt + c * (kKeys * 128) + g * 2048, &vmap, &kv_full[st], c * 64, row0, kvh,
-                        page);
-          }
+          page[g] = ok ? gr.x : a.P_pool;
+          row0[g] = ok ? gr.y % a.P : 0;
         }
+        // K(jj) waits for QK^T of tile jj - kStages, V(jj) for its PV
+        if (jj >= C::kStages && !wait_or_abort(&k_empty[st], ph, abort_flag)) break;
+        uint8_t* kt = k_s + st * C::kTileBytes;
+        mbar_arrive_expect_tx(&k_full[st], C::kTileBytes);
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g)
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(kt + c * (kKeys * 128) + g * 2048, &kmap, &k_full[st], c * 64, row0[g],
+                        kvh, page[g]);
+        if (jj >= C::kStages && !wait_or_abort(&v_empty[st], ph, abort_flag)) break;
+        uint8_t* vt = v_s + st * C::kTileBytes;
+        mbar_arrive_expect_tx(&v_full[st], C::kTileBytes);
+#pragma unroll
+        for (int g = 0; g < kGroups; ++g)
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_4d(vt + c * (kKeys * 128) + g * 2048, &vmap, &v_full[st], c * 64, row0[g],
+                        kvh, page[g]);
       }
     }
   } else if (warp == 9) {
-    // ================= MMA issuer (one thread), alternating tiles A and B
+    // ================= MMA issuer (one thread)
     if (lane == 0 && n_act > 0) {
-      const uint32_t q_addr = smem_u32(q_s), kv_addr = smem_u32(kv_s);
-      // O_w += P_w V for tile jp: P (hi, then lo) from the TMEM columns of the
-      // S buffer the tile's scores were in.  QK^T of tile jp + 2, issued after
-      // this, reuses those columns: MMAs of one thread execute in issue order.
-      auto pv = [&](int jp) -> bool {
-        const int st = jp % kPStages;
-        const uint32_t vbase = kv_addr + st * C::kStageBytes + C::kTileBytes;
-        for (int w = 0; w < 2; ++w) {
-          if (!wait_or_abort(&p_full[w], jp & 1, abort_flag)) return false;
-          tc::fence_after_sync();
-          const uint32_t pcol = tmem + 128 * w + (jp & 1) * kKeys;
+      const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
+      // S_w = Q_w K^T for tile jj into columns [128w, 128w + 128)
+      auto qk = [&](int jj, int w) {
+        const uint32_t kbase = k_addr + (jj % C::kStages) * C::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk) {
-            const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
-            tc::mma_bf16_ts(tmem + 256 + 128 * w, pcol + 8 * kk, bd, C::kIdPV,
-                            (jp > 0 || kk > 0) ? 1u : 0u);
-            tc::mma_bf16_ts(tmem + 256 + 128 * w, pcol + 32 + 8 * kk, bd, C::kIdPV, 1u);
-          }
-          tc::commit(&o_done[w]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = tc::sdesc_sw128(
+              q_addr + w * C::kQBytes + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd =
+              tc::sdesc_sw128(kbase + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_bf16(tmem + 128 * w, ad, bd, C::kIdQK, kk > 0 ? 1u : 0u);
         }
-        tc::commit(&kv_empty[st]);
-        return true;
+        tc::commit(&s_full[w]);
       };
-      bool ok = wait_or_abort(&q_full, 0, abort_flag);
-      tc::fence_after_sync();
-      for (int jj = 0; ok && jj < n_act; ++jj) {
-        const int st = jj % kPStages, sb = jj & 1;
-        if (!wait_or_abort(&kv_full[st], (jj / kPStages) & 1, abort_flag)) break;
-        tc::fence_after_sync();
-        const uint32_t kbase = kv_addr + st * C::kStageBytes;
-        for (int w = 0; w < 2; ++w) {
+      // O_w += P_w V over keys [64h, 64h + 64) of tile jj: P hi, then lo, of 16
+      // keys kk from columns 128w + 16 kk (+ 8 for lo)
+      auto pv = [&](int jj, int w, int h) {
+        const uint32_t vbase = v_addr + (jj % C::kStages) * C::kTileBytes;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = tc::sdesc_sw128(
-                q_addr + w * C::kQBytes + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd =
-                tc::sdesc_sw128(kbase + (kk >> 2) * (kKeys * 128) + (kk & 3) * 32, 16, 1024);
-            tc::mma_bf16(tmem + 128 * w + sb * kKeys, ad, bd, C::kIdQK, kk > 0 ? 1u : 0u);
-          }
-          tc::commit(&s_full[w][sb]);
+        for (int kk = 4 * h; kk < 4 * h + 4; ++kk) {
+          const uint64_t bd = tc::sdesc_sw128(vbase + kk * 2048, kKeys * 128, 1024);
+          const uint32_t hi = tmem + 128 * w + 16 * kk;
+          tc::mma_bf16_ts(tmem + 256 + D * w, hi, bd, C::kIdPV, (jj > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_bf16_ts(tmem + 256 + D * w, hi + 8, bd, C::kIdPV, 1u);
         }
-        if (jj >= 1 && !pv(jj - 1)) ok = false;
+      };
+      bool ok = wait_or_abort(&q_full, 0, abort_flag) && wait_or_abort(&k_full[0], 0, abort_flag);
+#if SA_PREFILL_TIMELINE
+      pt_mark(0, 0);
+#endif
+      tc::fence_after_sync();
+      if (ok) {
+        qk(0, 0);
+        qk(0, 1);
+        tc::commit(&k_empty[0]);
+#if SA_PREFILL_TIMELINE
+        pt_mark(0, 1);
+#endif
       }
-      if (ok) pv(n_act - 1);
+      for (int jj = 0; ok && jj < n_act; ++jj) {
+        const int st = jj % C::kStages;
+        for (int w = 0; ok && w < 2; ++w) {
+          for (int h = 0; h < 2; ++h) {
+            if (!wait_or_abort(&p_full[w][h], jj & 1, abort_flag) ||
+                (w == 0 && h == 0 &&
+                 !wait_or_abort(&v_full[st], (jj / C::kStages) & 1, abort_flag))) {
+              ok = false;
+              break;
+            }
+#if SA_PREFILL_TIMELINE
+            if (h == 1) pt_mark(jj, 2 + w);
+#endif
+            tc::fence_after_sync();
+            pv(jj, w, h);
+          }
+          if (!ok) break;
+          if (w == 1) tc::commit(&v_empty[st]);
+          if (jj + 1 < n_act) {
+            const int st1 = (jj + 1) % C::kStages;
+            if (w == 0) {
+              if (!wait_or_abort(&k_full[st1], ((jj + 1) / C::kStages) & 1, abort_flag)) {
+                ok = false;
+                break;
+              }
+#if SA_PREFILL_TIMELINE
+              pt_mark(jj + 1, 0);
+#endif
+              tc::fence_after_sync();
+            }
+            qk(jj + 1, w);
+            if (w == 1) {
+              tc::commit(&k_empty[st1]);
+#if SA_PREFILL_TIMELINE
+              pt_mark(jj + 1, 1);
+#endif
+            }
+          } else {
+            tc::commit(&o_done[w]);
+          }
+        }
+      }
     }
   } else {
     // ================= softmax / epilogue: one query row per thread
@@ -318,87 +389,60 @@ __global__ void __launch_bounds__(kPThreads, 1)
     tc::fence_proxy_async();
     mbar_arrive(&q_full);
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_col = 128 * wg, o_col = 256 + 128 * wg;
+    const uint32_t s_col = 128 * wg, o_col = 256 + D * wg;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
     for (int jj = 0; jj < n_act; ++jj) {
-      const int sb = jj & 1, code = act_s[jj], j = code >> 1;
-      if (!wait_or_abort(&s_full[wg][sb], (jj >> 1) & 1, abort_flag)) {
+      const int code = act_s[jj], j = code >> 1;
+      const bool masked = code & 1;
+      // visibility of the tile's keys for this row, one bit per key (before the
+      // wait: it needs only the list).  A group's keys are consecutive
+      // positions: key c of group g is visible iff the group is valid and
+      // c < min(L, qpos + 1) - (its first position).
+      uint32_t vis[kKeys / 32];
+      if (masked) {
+        const int vis_end = min(L, qpos + 1);
+#pragma unroll
+        for (int w = 0; w < kKeys / 32; ++w) {
+          uint32_t bits = 0;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int2 gr = group_of(ent_s, n_ent, a.P, j, 2 * w + h);
+            const int lim = gr.x >= 0 ? min(max(vis_end - gr.y, 0), 16) : 0;
+            bits |= ((1u << lim) - 1u) << (16 * h);
+          }
+          vis[w] = bits;
+        }
+      }
+      if (!wait_or_abort(&s_full[wg], jj & 1, abort_flag)) {
         ok = false;
         break;
       }
+#if SA_PREFILL_TIMELINE
+      if (r == 0) pt_mark(jj, 4 + 3 * wg);
+#endif
       tc::fence_after_sync();
-      float x[64];
-      tc::ld32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(&x[0]));
-      tc::ld32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+      float x[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c)
+        tc::ld32(tmem + lane_base + s_col + 32 * c, *reinterpret_cast<float(*)[32]>(&x[32 * c]));
       tc::wait_ld();
       // the row max of the scaled scores from the raw ones: x -> x s is monotone
       // (rounding included), so it is s max(x) for s >= 0 and s min(x) for s < 0;
       // invisible keys are NaN here (ignored by the reduction, p = 0 below)
       const float sl = a.scale_log2;
-      const bool masked = code & 1;
       if (masked) {
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int2 gr = group_of(ent_s, n_ent, a.P, j, g);
-          const bool gok = gr.x >= 0;
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const int kp = gr.y + c;
-            if (!(gok && kp < L && kp <= qpos)) x[g * 16 + c] = NAN;
-          }
-        }
+        for (int k = 0; k < kKeys; ++k)
+          if (!((vis[k >> 5] >> (k & 31)) & 1u)) x[k] = NAN;
       }
       const float mr = sl >= 0.f ? reduce_n<false>(x) : reduce_n<true>(x);
       const float mx = mr != mr ? -INFINITY : mr * sl;
       const bool move = mx > m_ref + kLazyP;
       const float m_new = move ? mx : m_ref;
       const float nb = m_new == -INFINITY ? 0.f : -m_new;
-      // P = 2^(x sl - m_new) as bf16 hi + lo pairs, written over this tile's
-      // scores in TMEM (the S buffer is free: QK^T of the tile is complete and
-      // PV of tile jj - 2, the buffer's previous reader, completed before it)
-      // (key pairs in packed float32: the same roundings as the scalar ops,
-      // half the instructions; the row sum in eight independent chains)
-      unsigned long long ls2[4] = {0ull, 0ull, 0ull, 0ull};
-      const unsigned long long sl2 = f2_pack(sl, sl), nb2 = f2_pack(nb, nb);
-      uint32_t ph[32], pl[32];
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float v0 = x[ch * 8 + 2 * i], v1 = x[ch * 8 + 2 * i + 1];
-          const float2 z = f2_unpack(f2_fma(f2_pack(v0, v1), sl2, nb2));
-          float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
-          if (masked) {
-            p0 = v0 == v0 ? p0 : 0.f;
-            p1 = v1 == v1 ? p1 : 0.f;
-          }
-          const unsigned long long pp = f2_pack(p0, p1);
-          ls2[i] = f2_add(ls2[i], pp);
-          const uint32_t h = pack_bf16(p0, p1);
-          const float2 d = f2_unpack(f2_sub(
-              pp, f2_pack(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u))));
-          ph[ch * 4 + i] = h;
-          pl[ch * 4 + i] = pack_bf16(d.x, d.y);
-        }
-      }
-      float ls[8];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 v = f2_unpack(ls2[i]);
-        ls[2 * i] = v.x;
-        ls[2 * i + 1] = v.y;
-      }
-      tc::st32(tmem + lane_base + s_col + sb * kKeys, *reinterpret_cast<float(*)[32]>(ph));
-      tc::st32(tmem + lane_base + s_col + sb * kKeys + 32, *reinterpret_cast<float(*)[32]>(pl));
-      tc::wait_st();
-      // PV(jj-1) must be done before O is rescaled and before P(jj) is handed
-      // over (its completion also keeps this barrier's phases in step)
-      if (jj >= 1 && !wait_or_abort(&o_done[wg], (jj - 1) & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc::fence_after_sync();
+      // O is rescaled before any of this tile's P is handed over; PV of the
+      // previous tile, its last writer, completed before these scores arrived
       if (__any_sync(0xffffffffu, move)) {
         const float alpha = move ? exp2f(m_ref - mx) : 1.f;
         l *= alpha;
@@ -412,15 +456,69 @@ __global__ void __launch_bounds__(kPThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             tc::st32(tmem + lane_base + o_col + c * 32, o);
           }
-          tc::wait_st();
         }
       }
       m_ref = m_new;
+      // P = 2^(x sl - m_new) as bf16 hi + lo pairs over this tile's scores in
+      // TMEM, 16 keys at a time (8 columns of hi pairs, then 8 of lo pairs).
+      // The scores are read a second time, 32 columns at a time with the next
+      // read in flight, so that the row of 128 never has to stay in registers.
+      // Key pairs in packed float32 (the same roundings as the scalar ops, half
+      // the instructions); the row sum in eight independent chains; P handed
+      // over in two halves of 64 keys.
+      unsigned long long ls2[4] = {0ull, 0ull, 0ull, 0ull};
+      const unsigned long long sl2 = f2_pack(sl, sl), nb2 = f2_pack(nb, nb);
+      float y[2][32];
+      tc::ld32(tmem + lane_base + s_col, y[0]);
+      tc::wait_ld();
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) {
+        if (c + 1 < kKeys / 32) tc::ld32(tmem + lane_base + s_col + 32 * (c + 1), y[(c + 1) & 1]);
+        const float* yc = y[c & 1];
+        const uint32_t vb = masked ? vis[c] : 0xffffffffu;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          uint32_t ph[8], pl[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int k = 16 * q + 2 * i;        // key within the 32-column chunk
+            const float2 z = f2_unpack(f2_fma(f2_pack(yc[k], yc[k + 1]), sl2, nb2));
+            float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
+            if (masked) {
+              p0 = (vb >> k) & 1u ? p0 : 0.f;
+              p1 = (vb >> (k + 1)) & 1u ? p1 : 0.f;
+            }
+            const unsigned long long pp = f2_pack(p0, p1);
+            ls2[i & 3] = f2_add(ls2[i & 3], pp);
+            const uint32_t hw = pack_bf16(p0, p1);
+            const float2 d = f2_unpack(f2_sub(
+                pp, f2_pack(__uint_as_float(hw << 16), __uint_as_float(hw & 0xffff0000u))));
+            ph[i] = hw;
+            pl[i] = pack_bf16(d.x, d.y);
+          }
+          tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q, ph);
+          tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q + 8, pl);
+        }
+        if (c + 1 < kKeys / 32) tc::wait_ld();
+        if (c == kKeys / 64 - 1 || c == kKeys / 32 - 1) {
+          tc::wait_st();
+          tc::fence_before_sync();
+          mbar_arrive(&p_full[wg][c == kKeys / 32 - 1 ? 1 : 0]);
+#if SA_PREFILL_TIMELINE
+          if (r == 0) pt_mark(jj, c == kKeys / 32 - 1 ? 5 + 3 * wg : 6 + 3 * wg);
+#endif
+        }
+      }
+      float ls[8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 v = f2_unpack(ls2[i]);
+        ls[2 * i] = v.x;
+        ls[2 * i + 1] = v.y;
+      }
       l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-      tc::fence_before_sync();
-      mbar_arrive(&p_full[wg]);
     }
-    if (ok && n_act > 0) ok = wait_or_abort(&o_done[wg], (n_act - 1) & 1, abort_flag);
+    if (ok && n_act > 0) ok = wait_or_abort(&o_done[wg], 0, abort_flag);
     tc::fence_after_sync();
     // ---- epilogue: O / l and LSE for this row
     const bool empty = !ok || n_act == 0 || l == 0.f;
@@ -484,3 +582,19 @@ cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CU
 }
 
 }  // namespace sa
+
+#if SA_PREFILL_TIMELINE
+// Diagnostic build only: copies the recorded stamps ([kPtCtas][kPtIters][12]
+// int64, SM clocks) to host memory `out` (n entries at most) and clears them.
+extern "C" SA_API int sa_prefill_timeline(long long* out, int n) {
+  const int total = sa::kPtCtas * sa::kPtIters * sa::kPtSlots;
+  if (!out || n <= 0) return SA_ERR_INVALID_ARG;
+  const size_t bytes = sizeof(long long) * (size_t)(n < total ? n : total);
+  if (cudaMemcpyFromSymbol(out, sa::g_prefill_tl, bytes) != cudaSuccess) return SA_ERR_CUDA;
+  void* dev = nullptr;
+  if (cudaGetSymbolAddress(&dev, sa::g_prefill_tl) != cudaSuccess ||
+      cudaMemset(dev, 0, sizeof(long long) * total) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_OK;
+}
+#endif

@@ -1,6 +1,7 @@
 """Per-warp timeline of the decode kernel at the Llama-8B-shaped decode workload.
 
     python -m paged_sparse_kv_sa_b200.timeline [--splits N] [--reps R] [--seed S] [--fp8]
+    python -m paged_sparse_kv_sa_b200.timeline --prefill [--reps R]
 
 Builds a diagnostic copy of the library (``_build/timeline/libsa_timeline.so``,
 compiled with ``-DSA_DECODE_TIMELINE=1``: each decode warp records
@@ -20,8 +21,15 @@ goes:
 
 Times are microseconds from the first warp's start, for the launch whose
 span (first start to last partial stored) is the median of the R launches.
-The CUDA-event time of each launch is printed beside its span.  GPU only; the
-library proper (``libsa.so``) has no timeline code.
+The CUDA-event time of each launch is printed beside its span.
+
+``--prefill``: the block-union chunked prefill instead (the tcgen05 many-row
+kernel, built with ``-DSA_PREFILL_TIMELINE=1``): the first CTAs of a launch
+stamp the SM clock per key tile -- the MMA thread's waits (K tile in, P of
+each row tile in) and issues, and both softmax warpgroups' phases (scores in,
+first half and all of the probabilities written) -- and the tool prints the
+median cycles of each step of a key tile's round trip.  GPU only; the library proper
+(``libsa.so``) has no timeline code.
 """
 from __future__ import annotations
 
@@ -37,10 +45,86 @@ from .build import OBJ, build
 TL_WARPS, TL_SLOTS = 8192, 16
 
 
+PT_CTAS, PT_ITERS, PT_SLOTS = 4, 256, 12
+
+
 def _build_timeline_lib() -> str:
     obj_dir = os.path.join(OBJ, "timeline")
     out = os.path.join(obj_dir, "libsa_timeline.so")
-    return build(defines=("SA_DECODE_TIMELINE=1",), out=out, obj_dir=obj_dir)
+    return build(defines=("SA_DECODE_TIMELINE=1", "SA_PREFILL_TIMELINE=1"), out=out,
+                 obj_dir=obj_dir)
+
+
+def analyse_prefill(stamps: np.ndarray):
+    """Median cycles of each step of a key tile's round trip, per CTA, from the
+    [CTAs, iterations, 12] clock stamps of one launch (tiles 2.. n-2: steady state)."""
+    out = []
+    for c in range(stamps.shape[0]):
+        st = stamps[c].astype(np.int64)
+        n = int(st[0, 11])
+        n_rec = min(n, st.shape[0])          # tiles past the record's end are not stamped
+        if n_rec < 6 or st[0, 10] == 0:
+            continue
+        j = np.arange(2, n_rec - 3)
+        med = lambda v: float(np.median(v))   # noqa: E731
+        row = {
+            "tiles": n,
+            "per tile (K in to next K in, MMA thread)": med(st[j + 1, 0] - st[j, 0]),
+            "softmax A (S in -> all of P written)": med(st[j, 5] - st[j, 4]),
+            "softmax B (S in -> all of P written)": med(st[j, 8] - st[j, 7]),
+            "softmax A: S in -> first half of P written": med(st[j, 6] - st[j, 4]),
+            "P_A written -> MMA thread sees it": med(st[j, 2] - st[j, 5]),
+            "P_B written -> MMA thread sees it": med(st[j, 3] - st[j, 8]),
+            "MMA thread: P_A(j) in -> K(j+1) in": med(st[j + 1, 0] - st[j, 2]),
+            "MMA thread: K(j+1) in -> P_B(j) in": med(st[j, 3] - st[j + 1, 0]),
+            "MMA thread: P_B(j) in -> QK_B(j+1) issued": med(st[j + 1, 1] - st[j, 3]),
+            "MMA thread: QK_B(j+1) issued -> P_A(j+1) in": med(st[j + 1, 2] - st[j + 1, 1]),
+            "softmax A: P(j) written -> S(j+1) in (PV + QK round trip)":
+                med(st[j + 1, 4] - st[j, 5]),
+            "softmax A: S(j) in -> S(j+1) in": med(st[j + 1, 4] - st[j, 4]),
+            "launch to first tile (cycles)": float(st[0, 0] - st[0, 10]),
+        }
+        out.append(row)
+    return out
+
+
+def main_prefill(lib, reps):
+    import math
+
+    import torch
+
+    from . import workloads as W
+    from ._lib import sa_block_union, sa_sparse_decode
+
+    lib.sa_prefill_timeline.restype = ctypes.c_int
+    lib.sa_prefill_timeline.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    dev = torch.device("cuda", 0)
+    cfg = W.UNION_PREFILL
+    inp = W.prefill_inputs(cfg, seed=0, device=dev)
+    scores = W.block_union_scores(cfg, seed=0, device=dev)
+    tables, counts = sa_block_union(scores, cfg.Hkv, cfg.q_offset // cfg.block, cfg.top_k,
+                                    cfg.n_sink_blocks)
+    h2l = [h // (cfg.Hq // cfg.Hkv) for h in range(cfg.Hq)]
+    buf = np.zeros(PT_CTAS * PT_ITERS * PT_SLOTS, dtype=np.int64)
+    rows = []
+    for r in range(reps + 1):
+        lib.sa_prefill_timeline(buf.ctypes.data, buf.size)    # clears the stamps
+        sa_sparse_decode(inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"],
+                         tables.view(1, cfg.Hkv, -1), counts.view(1, cfg.Hkv), h2l,
+                         1.0 / math.sqrt(cfg.D), 4)
+        torch.cuda.synchronize()
+        if lib.sa_prefill_timeline(buf.ctypes.data, buf.size) != 0:
+            raise RuntimeError("sa_prefill_timeline failed")
+        if r >= 1:
+            rows += analyse_prefill(buf.reshape(PT_CTAS, PT_ITERS, PT_SLOTS).copy())
+    print(f"workload {cfg.name}, 4 splits: {len(rows)} CTA records over {reps} launches "
+          f"(the first {PT_CTAS} CTAs of each)")
+    keys = [k for k in rows[0] if k != "tiles"]
+    print(f"key tiles per CTA: {int(np.median([r_['tiles'] for r_ in rows]))} (median)\n")
+    print("| step of a key tile (SM clock cycles, median over tiles, then over CTAs) | cycles |")
+    print("|---|---:|")
+    for k in keys:
+        print(f"| {k} | {np.median([r_[k] for r_ in rows]):.0f} |")
 
 
 def _pct(x, q):
@@ -86,9 +170,12 @@ def main():
     ap.add_argument("--reps", type=int, default=20)
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--fp8", action="store_true")
+    ap.add_argument("--prefill", action="store_true")
     args = ap.parse_args()
     path = _build_timeline_lib()
     lib = _lib.load(path)               # every wrapper below now calls this copy
+    if args.prefill:
+        return main_prefill(lib, args.reps)
     lib.sa_decode_timeline.restype = ctypes.c_int
     lib.sa_decode_timeline.argtypes = [ctypes.c_void_p, ctypes.c_int]
 

@@ -197,7 +197,7 @@ def test_fuzz_many_rows_at_positions_vs_oracle(seed):
     # over random per-group page lists, with queries at explicit positions
     rng = np.random.default_rng(7000 + seed)
     D = int(rng.choice([64, 128]))
-    P = int(rng.choice([16, 32, 64]))
+    P = int(rng.choice([16, 32, 48, 64, 128]))   # 48: a tile of 128 keys cuts a page
     Hkv = int(rng.choice([1, 2]))
     G = int(rng.choice([1, 2, 4]))
     T = int(rng.integers(17, 160))
