@@ -242,8 +242,10 @@ SA_API int sa_select_ambient_heads(const uint16_t* q, const int64_t q_strides[4]
  * seq_lens[b] and at most seq_lens[b] - T + t (query token t sits at that
  * position: causal MTP / chunked prefill).  s_j = scale * q.k_j; natural-log
  * LSE.  Split s takes the entries [s*c, (s+1)*c) of the list with
- * c = ceil(max_list/n_splits) (so a short list leaves its last splits empty)
- * and writes its own normalised output and LSE.  A split without a visible
+ * c = ceil(max_list/n_splits) (so a short list leaves its last splits empty;
+ * the many-row kernel instead takes c = ceil(list_count/n_splits), an equal
+ * share of each list's actual length) and writes its own normalised output
+ * and LSE.  A split without a visible
  * key writes LSE = -inf; its O rows are 0 when n_splits == 1 and otherwise
  * unspecified (sa_combine gives such a split no weight).  With n_splits == 1
  * the partials are the final result; otherwise pass them to sa_combine.

@@ -23,8 +23,10 @@
 //               TMEM is then rare), P back into the S columns it came from, in
 //               two halves of 64 keys (PV of the first half runs while the
 //               second is computed), and the epilogue.
-// P enters PV as a bf16 pair hi + lo (hi = RNE_bf16(p), lo = RNE_bf16(p - hi)),
-// so its rounding is ~2^-17 relative rather than the 2^-9 of a single bf16: two
+// P enters PV as a bf16 pair hi + lo (hi = p truncated to bf16, lo = p - hi,
+// exact in float32, truncated to bf16), so hi + lo is within 2^-16 relative of
+// p rather than the 2^-9 of a single rounded bf16, at the cost of two
+// bitwise operations per key and no conversion instruction: two
 // MMAs per 16 keys, reading the pair from the TMEM columns where those keys'
 // scores were (per 16 keys: 8 columns of hi pairs, then 8 of lo pairs).
 // Single-buffered S costs no wait: the commit that announces S_w(j) tracks
@@ -50,8 +52,27 @@
 
 namespace sa {
 #if SA_PREFILL_TIMELINE
-constexpr int kPtCtas = 4, kPtIters = 256, kPtSlots = 12;
+constexpr int kPtCtas = 4, kPtIters = 256, kPtSlots = 16;
 __device__ long long g_prefill_tl[kPtCtas * kPtIters * kPtSlots];
+// every CTA (up to kPtAll): %globaltimer at entry and exit, active tiles, SM id
+constexpr int kPtAll = 8192;
+__device__ long long g_prefill_cta[kPtAll * 4];
+SA_DEV long long pt_now() {
+  long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+SA_DEV void pt_cta_put(int slot, long long v) {
+  const int c = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  if (c < kPtAll) g_prefill_cta[c * 4 + slot] = v;
+}
+SA_DEV void pt_cta_end(int n_act) {
+  uint32_t sm;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(sm));
+  pt_cta_put(1, pt_now());
+  pt_cta_put(2, n_act);
+  pt_cta_put(3, sm);
+}
 #endif
 namespace {
 
@@ -114,13 +135,22 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int qt = blockIdx.x / a.n_splits, split = blockIdx.x % a.n_splits;
   const int nh = prm.pairs.n_heads[pair];
   const int rows_total = a.T * nh;
-  if (qt * kRows >= rows_total) return;               // whole CTA: nothing to do
+  if (qt * kRows >= rows_total) {                     // whole CTA: nothing to do
+#if SA_PREFILL_TIMELINE
+    if (threadIdx.x == 0) {
+      pt_cta_put(0, pt_now());
+      pt_cta_end(0);
+    }
+#endif
+    return;
+  }
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int list = prm.pairs.list_of[pair], kvh = prm.pairs.kvh_of[pair];
 #if SA_PREFILL_TIMELINE
   // slots per key tile: 0 K in (before QK_A), 1 QK_B issued, 2 / 3 second half of
   // P of tiles A / B in (the MMA thread), 4 / 7 S in, 5 / 8 all of P written,
-  // 6 / 9 first half of P written (softmax A / B); tile 0 slot 10: start,
+  // 6 / 9 first half of P written, 12 / 14 scores in registers, 13 / 15 row
+  // max (and any O rescale) done (softmax A / B); tile 0 slot 10: start,
   // slot 11: tiles
   const int pt_cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
   long long* pt_row = pt_cta < kPtCtas ? g_prefill_tl + (int64_t)pt_cta * kPtIters * kPtSlots
@@ -128,7 +158,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
   auto pt_mark = [&](int it, int slot) {
     if (pt_row && it >= 0 && it < kPtIters) pt_row[it * kPtSlots + slot] = clock64();
   };
-  if (tid == 0) pt_mark(0, 10);
+  if (tid == 0) {
+    pt_mark(0, 10);
+    pt_cta_put(0, pt_now());
+  }
 #endif
 
   extern __shared__ uint8_t dyn_smem[];
@@ -155,8 +188,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (tid == 0) set_dev_error(a.err, SA_DEVERR_COUNT);
     count = count < 0 ? 0 : a.max_list;
   }
-  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(max_list / n_splits)
-  const int chunk = (a.max_list + a.n_splits - 1) / a.n_splits;
+  // split s holds entries [s c, (s + 1) c) of the list, c = ceil(count / n_splits):
+  // shares of the list's actual length, so that no split idles while another
+  // holds a capacity's worth (c <= ceil(max_list / n_splits), checked on the host)
+  const int chunk = (count + a.n_splits - 1) / a.n_splits;
   const int e0 = min(split * chunk, count);
   const int n_ent = min(chunk, count - e0);
   const int r0 = qt * kRows;
@@ -169,6 +204,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
       *reinterpret_cast<float4*>(a.o_part + orow * D + c) = make_float4(0.f, 0.f, 0.f, 0.f);
       if (c == 0) a.lse_part[orow] = -INFINITY;
     }
+#if SA_PREFILL_TIMELINE
+    __syncthreads();
+    if (tid == 0) pt_cta_end(0);
+#endif
     return;
   }
   const int t_first = r0 / nh;
@@ -427,6 +466,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
       for (int c = 0; c < kKeys / 32; ++c)
         tc::ld32(tmem + lane_base + s_col + 32 * c, *reinterpret_cast<float(*)[32]>(&x[32 * c]));
       tc::wait_ld();
+#if SA_PREFILL_TIMELINE
+      if (r == 0) pt_mark(jj, 12 + 2 * wg);
+#endif
       // the row max of the scaled scores from the raw ones: x -> x s is monotone
       // (rounding included), so it is s max(x) for s >= 0 and s min(x) for s < 0;
       // invisible keys are NaN here (ignored by the reduction, p = 0 below)
@@ -459,6 +501,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
       }
       m_ref = m_new;
+#if SA_PREFILL_TIMELINE
+      if (r == 0) pt_mark(jj, 13 + 2 * wg);
+#endif
       // P = 2^(x sl - m_new) as bf16 hi + lo pairs over this tile's scores in
       // TMEM, 16 keys at a time (8 columns of hi pairs, then 8 of lo pairs).
       // The scores are read a second time, 32 columns at a time with the next
@@ -490,11 +535,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
             }
             const unsigned long long pp = f2_pack(p0, p1);
             ls2[i & 3] = f2_add(ls2[i & 3], pp);
-            const uint32_t hw = pack_bf16(p0, p1);
-            const float2 d = f2_unpack(f2_sub(
-                pp, f2_pack(__uint_as_float(hw << 16), __uint_as_float(hw & 0xffff0000u))));
-            ph[i] = hw;
-            pl[i] = pack_bf16(d.x, d.y);
+            // hi = p truncated to bf16 (its low 16 bits cleared), lo = p - hi
+            // (exact in float32) truncated likewise: integer and byte-permute
+            // instructions only, no conversions
+            const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffff0000u);
+            const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffff0000u);
+            const float2 d = f2_unpack(f2_sub(pp, f2_pack(h0, h1)));
+            ph[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);
+            pl[i] = __byte_perm(__float_as_uint(d.x), __float_as_uint(d.y), 0x7632);
           }
           tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q, ph);
           tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q + 8, pl);
@@ -550,6 +598,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, C::kTmemCols);
   }
+#if SA_PREFILL_TIMELINE
+  if (tid == 0) pt_cta_end(n_act);
+#endif
 }
 
 template <int D>
@@ -584,7 +635,21 @@ cudaError_t launch_prefill(const DecodeArgs& a, const PairTable& pairs, const CU
 }  // namespace sa
 
 #if SA_PREFILL_TIMELINE
-// Diagnostic build only: copies the recorded stamps ([kPtCtas][kPtIters][12]
+// Diagnostic build only: copies the per-CTA records ([8192][4] int64: entry and
+// exit %globaltimer, active tiles, SM id; unlaunched CTAs stay 0) to host memory
+// `out` (n entries at most) and clears them.
+extern "C" SA_API int sa_prefill_cta_timeline(long long* out, int n) {
+  const int total = sa::kPtAll * 4;
+  if (!out || n <= 0) return SA_ERR_INVALID_ARG;
+  const size_t bytes = sizeof(long long) * (size_t)(n < total ? n : total);
+  if (cudaMemcpyFromSymbol(out, sa::g_prefill_cta, bytes) != cudaSuccess) return SA_ERR_CUDA;
+  void* dev = nullptr;
+  if (cudaGetSymbolAddress(&dev, sa::g_prefill_cta) != cudaSuccess ||
+      cudaMemset(dev, 0, sizeof(long long) * total) != cudaSuccess)
+    return SA_ERR_CUDA;
+  return SA_OK;
+}
+// Diagnostic build only: copies the recorded stamps ([kPtCtas][kPtIters][16]
 // int64, SM clocks) to host memory `out` (n entries at most) and clears them.
 extern "C" SA_API int sa_prefill_timeline(long long* out, int n) {
   const int total = sa::kPtCtas * sa::kPtIters * sa::kPtSlots;

@@ -45,7 +45,7 @@ from .build import OBJ, build
 TL_WARPS, TL_SLOTS = 8192, 16
 
 
-PT_CTAS, PT_ITERS, PT_SLOTS = 4, 256, 12
+PT_CTAS, PT_ITERS, PT_SLOTS = 4, 256, 16
 
 
 def _build_timeline_lib() -> str:
@@ -57,7 +57,7 @@ def _build_timeline_lib() -> str:
 
 def analyse_prefill(stamps: np.ndarray):
     """Median cycles of each step of a key tile's round trip, per CTA, from the
-    [CTAs, iterations, 12] clock stamps of one launch (tiles 2.. n-2: steady state)."""
+    [CTAs, iterations, 16] clock stamps of one launch (tiles 2.. n-2: steady state)."""
     out = []
     for c in range(stamps.shape[0]):
         st = stamps[c].astype(np.int64)
@@ -72,7 +72,13 @@ def analyse_prefill(stamps: np.ndarray):
             "per tile (K in to next K in, MMA thread)": med(st[j + 1, 0] - st[j, 0]),
             "softmax A (S in -> all of P written)": med(st[j, 5] - st[j, 4]),
             "softmax B (S in -> all of P written)": med(st[j, 8] - st[j, 7]),
-            "softmax A: S in -> first half of P written": med(st[j, 6] - st[j, 4]),
+            "softmax A: S in -> scores in registers": med(st[j, 12] - st[j, 4]),
+            "softmax A: scores in registers -> row max (and O rescale) done":
+                med(st[j, 13] - st[j, 12]),
+            "softmax A: row max done -> first half of P written": med(st[j, 6] - st[j, 13]),
+            "softmax A: first half -> all of P written": med(st[j, 5] - st[j, 6]),
+            "softmax B: S in -> row max done": med(st[j, 15] - st[j, 7]),
+            "softmax B: row max done -> all of P written": med(st[j, 8] - st[j, 15]),
             "P_A written -> MMA thread sees it": med(st[j, 2] - st[j, 5]),
             "P_B written -> MMA thread sees it": med(st[j, 3] - st[j, 8]),
             "MMA thread: P_A(j) in -> K(j+1) in": med(st[j + 1, 0] - st[j, 2]),
@@ -88,6 +94,44 @@ def analyse_prefill(stamps: np.ndarray):
     return out
 
 
+PT_ALL = 8192
+
+
+def analyse_prefill_grid(cta: np.ndarray, n_sm: int):
+    """Whole-launch figures from the per-CTA [n, 4] records (entry ns, exit ns,
+    active tiles, SM id; rows of CTAs that never ran are 0)."""
+    c = cta[cta[:, 0] > 0].astype(np.int64)
+    if len(c) == 0:
+        return None
+    t0 = c[:, 0].min()
+    start, end, tiles = c[:, 0] - t0, c[:, 1] - t0, c[:, 2]
+    dur = end - start
+    span = float(end.max())
+    work = tiles > 0
+    # per-CTA duration = fixed + per_tile * tiles (least squares over CTAs with tiles)
+    if work.sum() >= 2 and np.ptp(tiles[work]) > 0:
+        per_tile, fixed = np.polyfit(tiles[work], dur[work], 1)
+    else:
+        per_tile, fixed = float("nan"), float("nan")
+    # SMs busy over time, in 2% steps of the span
+    grid = np.linspace(0, span, 51)
+    busy = [int(((start <= g) & (end > g)).sum()) for g in grid[:-1]]
+    return {
+        "ctas": int(len(c)), "ctas with tiles": int(work.sum()),
+        "tiles": int(tiles.sum()), "span_us": span / 1e3,
+        "sm utilisation": float(dur.sum()) / (span * n_sm),
+        "per tile ns (fit)": float(per_tile), "per CTA fixed ns (fit)": float(fixed),
+        "CTA duration us p50 / p90 / max": (float(np.median(dur)) / 1e3,
+                                            float(np.percentile(dur, 90)) / 1e3,
+                                            float(dur.max()) / 1e3),
+        "tiles per CTA p50 / p90 / max": (float(np.median(tiles[work])) if work.any() else 0.0,
+                                          float(np.percentile(tiles[work], 90)) if work.any()
+                                          else 0.0, int(tiles.max())),
+        "last CTA start us": float(start.max()) / 1e3,
+        "busy SMs over the span (2% steps)": busy,
+    }
+
+
 def main_prefill(lib, reps):
     import math
 
@@ -98,6 +142,10 @@ def main_prefill(lib, reps):
 
     lib.sa_prefill_timeline.restype = ctypes.c_int
     lib.sa_prefill_timeline.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    lib.sa_prefill_cta_timeline.restype = ctypes.c_int
+    lib.sa_prefill_cta_timeline.argtypes = [ctypes.c_void_p, ctypes.c_int]
+    cbuf = np.zeros(PT_ALL * 4, dtype=np.int64)
+    grids = []
     dev = torch.device("cuda", 0)
     cfg = W.UNION_PREFILL
     inp = W.prefill_inputs(cfg, seed=0, device=dev)
@@ -109,14 +157,19 @@ def main_prefill(lib, reps):
     rows = []
     for r in range(reps + 1):
         lib.sa_prefill_timeline(buf.ctypes.data, buf.size)    # clears the stamps
+        lib.sa_prefill_cta_timeline(cbuf.ctypes.data, cbuf.size)
         sa_sparse_decode(inp["q"], inp["k"], inp["v"], inp["page_table"], inp["seq_lens"],
                          tables.view(1, cfg.Hkv, -1), counts.view(1, cfg.Hkv), h2l,
                          1.0 / math.sqrt(cfg.D), 4)
         torch.cuda.synchronize()
         if lib.sa_prefill_timeline(buf.ctypes.data, buf.size) != 0:
             raise RuntimeError("sa_prefill_timeline failed")
+        if lib.sa_prefill_cta_timeline(cbuf.ctypes.data, cbuf.size) != 0:
+            raise RuntimeError("sa_prefill_cta_timeline failed")
         if r >= 1:
             rows += analyse_prefill(buf.reshape(PT_CTAS, PT_ITERS, PT_SLOTS).copy())
+            n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+            grids.append(analyse_prefill_grid(cbuf.reshape(PT_ALL, 4).copy(), n_sm))
     print(f"workload {cfg.name}, 4 splits: {len(rows)} CTA records over {reps} launches "
           f"(the first {PT_CTAS} CTAs of each)")
     keys = [k for k in rows[0] if k != "tiles"]
@@ -125,6 +178,12 @@ def main_prefill(lib, reps):
     print("|---|---:|")
     for k in keys:
         print(f"| {k} | {np.median([r_[k] for r_ in rows]):.0f} |")
+    g = [x for x in grids if x is not None]
+    if g:
+        mid = sorted(g, key=lambda x: x["span_us"])[len(g) // 2]
+        print(f"\nwhole launch (the launch of median span of {len(g)}):")
+        for k, v in mid.items():
+            print(f"  {k}: {v}")
 
 
 def _pct(x, q):

@@ -1,4 +1,4 @@
-"""The decode timeline tool's analysis of recorded stamps (CPU only: the stamps
+"""The timeline tool's analysis of recorded stamps, decode and prefill (CPU only: the stamps
 here are written by hand, the GPU build that records them is not involved)."""
 import numpy as np
 
@@ -29,3 +29,22 @@ def test_phases_span_and_bytes():
     got = r["bytes_per_us"]
     assert got[3] == 2 * 8192 and got[4] == 8192 and got.sum() == 3 * 8192
     assert r["running"][0] == 2 and r["running"][5] == 1 and r["running"][6] == 0
+
+
+def test_prefill_grid_analysis_recovers_per_tile_cost():
+    # CTAs of 5 us fixed cost + 100 ns per tile, started 50 ns apart: the fit
+    # recovers both, and utilisation / busy counts follow from the intervals
+    from paged_sparse_kv_sa_b200.timeline import analyse_prefill_grid
+    rng = np.random.default_rng(0)
+    c = np.zeros((8192, 4), dtype=np.int64)
+    for i in range(300):
+        t = int(rng.integers(1, 100))
+        s = 1000 + 50 * i
+        c[i] = [s, s + 5000 + 100 * t, t, i % 148]
+    g = analyse_prefill_grid(c, 148)
+    assert g["ctas"] == 300 and g["tiles"] == int(c[:300, 2].sum())
+    assert abs(g["per tile ns (fit)"] - 100.0) < 1e-6
+    assert abs(g["per CTA fixed ns (fit)"] - 5000.0) < 1e-3
+    dur = (c[:300, 1] - c[:300, 0]).sum()
+    assert abs(g["sm utilisation"] - dur / (g["span_us"] * 1e3 * 148)) < 1e-12
+    assert max(g["busy SMs over the span (2% steps)"]) <= 300
