@@ -5,24 +5,26 @@
 // One CTA computes 256 query rows of a pair (token-major) as two 128-row tiles
 // A and B against the keys of its split of the list, 128 keys per tile; each
 // K/V tile is loaded once and used by both:
-//   warp 8      gathers K and V tiles from the paged pool with TMA (16-key x
+//   warp 16     gathers K and V tiles from the paged pool with TMA (16-key x
 //               64-column boxes; an absent or invalid 16-key group is loaded
 //               from an out-of-range page coordinate, which TMA fills with
 //               zeros) into separate K and V rings of two (D = 128) or four
 //               (D = 64) stages;
-//   warp 9      issues tcgen05.mma: S_w = Q_w K^T (M=128, N=128, K=D) into one
+//   warp 17     issues tcgen05.mma: S_w = Q_w K^T (M=128, N=128, K=D) into one
 //               TMEM S buffer per tile w, and O_w += P_w V (M=128, N=D) with P
 //               read from the TMEM columns of S_w as the A operand, in the order
 //               PV_A(j), QK_A(j+1), PV_B(j), QK_B(j+1): the tensor core works
 //               on one tile while the other tile's softmax runs;
-//   warps 0-3 / 4-7   (one warpgroup per tile) own one query row per thread:
-//               Q into shared memory, S rows from TMEM, masking (page validity,
+//   warps 0-7 / 8-15   (tile A / B) own each query row with two threads, one
+//               per 64-key half of every tile (four softmax warps per SM
+//               sub-partition, so that they hide one another's latency): Q
+//               into shared memory, S from TMEM, masking (page validity,
 //               sequence end, causal position; skipped for tiles every row sees
-//               whole), a base-2 online softmax whose running max only moves when
-//               a row's max exceeds it by more than 2^8 (the O rescale through
-//               TMEM is then rare), P back into the S columns it came from, in
-//               two halves of 64 keys (PV of the first half runs while the
-//               second is computed), and the epilogue.
+//               whole), the row max from both halves (swapped through shared
+//               memory), a base-2 online softmax whose running max only moves
+//               when a row's max exceeds it by more than 2^8 (the O rescale
+//               through TMEM is then rare), P back into the S columns it came
+//               from, and the epilogue (each half of a row writes half of O).
 // P enters PV as a bf16 pair hi + lo (hi = p truncated to bf16, lo = p - hi,
 // exact in float32, truncated to bf16), so hi + lo is within 2^-16 relative of
 // p rather than the 2^-9 of a single rounded bf16, at the cost of two
@@ -76,7 +78,9 @@ SA_DEV void pt_cta_end(int n_act) {
 #endif
 namespace {
 
-constexpr int kPThreads = 320;    // 2 softmax warpgroups, producer warp, MMA warp
+constexpr int kSoftWarps = 16;    // two per (row tile, TMEM lane quarter, key half)
+constexpr int kProdWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1;
+constexpr int kPThreads = 32 * (kSoftWarps + 2);
 constexpr int kKeys = 128;        // keys per tile
 constexpr int kGroups = kKeys / 16;
 constexpr int kM = 128;           // query rows per warpgroup tile
@@ -101,6 +105,11 @@ struct __align__(64) PrefillParams {
   DecodeArgs a;
   PairTable pairs;
 };
+
+// Named barrier `id` (1-8; 0 is __syncthreads) over `n` threads.
+SA_DEV void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 // Bounded wait that also gives up as soon as another role has aborted.
 SA_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -148,10 +157,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
   const int list = prm.pairs.list_of[pair], kvh = prm.pairs.kvh_of[pair];
 #if SA_PREFILL_TIMELINE
   // slots per key tile: 0 K in (before QK_A), 1 QK_B issued, 2 / 3 second half of
-  // P of tiles A / B in (the MMA thread), 4 / 7 S in, 5 / 8 all of P written,
-  // 6 / 9 first half of P written, 12 / 14 scores in registers, 13 / 15 row
-  // max (and any O rescale) done (softmax A / B); tile 0 slot 10: start,
-  // slot 11: tiles
+  // P of tiles A / B in (the MMA thread), 4 / 7 S in, 5 / 8 P of keys 0-63
+  // written, 6 / 9 P of keys 64-127 written, 12 / 14 partial maxima exchanged,
+  // 13 / 15 row max (and any O rescale) done (softmax A / B); tile 0 slot 10:
+  // start, slot 11: tiles
   const int pt_cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
   long long* pt_row = pt_cta < kPtCtas ? g_prefill_tl + (int64_t)pt_cta * kPtIters * kPtSlots
                                        : nullptr;
@@ -175,6 +184,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __shared__ uint32_t tmem_base_s;
   __shared__ int abort_s, n_act_s;
   __shared__ int2 ent_s[kMaxEnt];
+  // partial row maxima (by tile parity), row sums and status of the two key
+  // halves of every row
+  __shared__ float pmax_s[2][2][2][kM];
+  __shared__ float lsum_s[2][2][kM];
+  __shared__ int okay_s[2][2][kM];
   __shared__ int act_s[kMaxEnt];     // (tile << 1) | needs_mask
 
   int L = a.seq_lens[b];
@@ -244,11 +258,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&p_full[w][1], 128);
       mbar_init(&o_done[w], 1);
     }
-    mbar_init(&q_full, 256);
+    mbar_init(&q_full, 32 * kSoftWarps);
     abort_s = 0;
     fence_mbar_init();
   }
-  if (warp == 9) tc::tmem_alloc(&tmem_base_s, C::kTmemCols);
+  if (warp == kMmaWarp) tc::tmem_alloc(&tmem_base_s, C::kTmemCols);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -282,7 +296,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
   if (tid == 0 && pt_row) pt_row[11] = n_act;
 #endif
 
-  if (warp == 8) {
+  if (warp == kProdWarp) {
     // ================= producer: TMA gathers of K and V tiles
     if (lane == 0) {
       prefetch_tmap(&kmap);
@@ -320,7 +334,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         kvh, page[g]);
       }
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ================= MMA issuer (one thread)
     if (lane == 0 && n_act > 0) {
       const uint32_t q_addr = smem_u32(q_s), k_addr = smem_u32(k_s), v_addr = smem_u32(v_s);
@@ -406,174 +420,192 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
     }
   } else {
-    // ================= softmax / epilogue: one query row per thread
-    const int wg = warp >> 2;                       // tile A (0) or B (1)
-    const int r = (warp & 3) * 32 + lane;           // row within the tile = TMEM lane
+    // ================= softmax / epilogue: two threads per query row, one per
+    // 64-key half of every tile (warps 0-7 tile A, 8-15 tile B; in each, warps
+    // 0-3 take keys 0-63 and warps 4-7 keys 64-127 of the same rows, so that
+    // four softmax warps share each sub-partition and hide one another's
+    // latency).  The two halves of a row swap their partial maxima through
+    // shared memory under a named barrier of their two warps.
+    const int wg = warp >> 3;                       // tile A (0) or B (1)
+    const int kh = (warp >> 2) & 1;                 // key half
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;              // row within the tile = TMEM lane
     const int rg = r0 + wg * kM + r;
     const bool row_ok = rg < rows_total;
     const int t = row_ok ? rg / nh : 0;
     const int head = prm.pairs.heads[prm.pairs.head_off[pair] + (row_ok ? rg % nh : 0)];
     const int qpos = row_ok ? qb + t : -1;
     uint8_t* qt_s = q_s + wg * C::kQBytes;
-    {
+    {   // this thread's half of the row's 16-byte pieces
       const uint4* src = reinterpret_cast<const uint4*>(a.q + b * a.qs0 + t * a.qs1 + head * a.qs2);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c)
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const uint4 v = row_ok ? src[c * 8 + ch] : make_uint4(0, 0, 0, 0);
-          *reinterpret_cast<uint4*>(qt_s + c * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
-        }
+      for (int pc = kh * (D / 16); pc < (kh + 1) * (D / 16); ++pc) {
+        const int c = pc >> 3, ch = pc & 7;
+        const uint4 v = row_ok ? src[pc] : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(qt_s + c * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+      }
     }
     tc::fence_proxy_async();
     mbar_arrive(&q_full);
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t s_col = 128 * wg, o_col = 256 + D * wg;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t s_col = 128 * wg + 64 * kh;      // this half's 64 score columns
+    const uint32_t o_col = 256 + D * wg + (D / 2) * kh;   // and its half of O
+    const int pair_bar = 1 + wg * 4 + quarter;      // the two warps of these rows
+    const float sl = a.scale_log2;
     float m_ref = -INFINITY, l = 0.f;
     bool ok = true;
+    // (after an abort the loop still runs to its end, skipping the work, so
+    // that the partner warp's barrier sees every arrival it counts on)
     for (int jj = 0; jj < n_act; ++jj) {
       const int code = act_s[jj], j = code >> 1;
       const bool masked = code & 1;
-      // visibility of the tile's keys for this row, one bit per key (before the
-      // wait: it needs only the list).  A group's keys are consecutive
+      // visibility of this half's keys for this row, one bit per key (before
+      // the wait: it needs only the list).  A group's keys are consecutive
       // positions: key c of group g is visible iff the group is valid and
       // c < min(L, qpos + 1) - (its first position).
-      uint32_t vis[kKeys / 32];
+      uint32_t vis[2];
       if (masked) {
         const int vis_end = min(L, qpos + 1);
 #pragma unroll
-        for (int w = 0; w < kKeys / 32; ++w) {
+        for (int w = 0; w < 2; ++w) {
           uint32_t bits = 0;
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int2 gr = group_of(ent_s, n_ent, a.P, j, 2 * w + h);
+            const int2 gr = group_of(ent_s, n_ent, a.P, j, 4 * kh + 2 * w + h);
             const int lim = gr.x >= 0 ? min(max(vis_end - gr.y, 0), 16) : 0;
             bits |= ((1u << lim) - 1u) << (16 * h);
           }
           vis[w] = bits;
         }
       }
-      if (!wait_or_abort(&s_full[wg], jj & 1, abort_flag)) {
-        ok = false;
-        break;
-      }
+      ok = __all_sync(0xffffffffu, ok && wait_or_abort(&s_full[wg], jj & 1, abort_flag));
 #if SA_PREFILL_TIMELINE
-      if (r == 0) pt_mark(jj, 4 + 3 * wg);
-#endif
-      tc::fence_after_sync();
-      float x[kKeys];
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c)
-        tc::ld32(tmem + lane_base + s_col + 32 * c, *reinterpret_cast<float(*)[32]>(&x[32 * c]));
-      tc::wait_ld();
-#if SA_PREFILL_TIMELINE
-      if (r == 0) pt_mark(jj, 12 + 2 * wg);
+      if (r == 0 && kh == 0) pt_mark(jj, 4 + 3 * wg);
 #endif
       // the row max of the scaled scores from the raw ones: x -> x s is monotone
       // (rounding included), so it is s max(x) for s >= 0 and s min(x) for s < 0;
-      // invisible keys are NaN here (ignored by the reduction, p = 0 below)
-      const float sl = a.scale_log2;
-      if (masked) {
+      // invisible keys are NaN here (ignored by the reductions, p = 0 below)
+      float part = NAN;
+      if (ok) {
+        tc::fence_after_sync();
+        float x[64];
+        tc::ld32(tmem + lane_base + s_col, *reinterpret_cast<float(*)[32]>(&x[0]));
+        tc::ld32(tmem + lane_base + s_col + 32, *reinterpret_cast<float(*)[32]>(&x[32]));
+        tc::wait_ld();
+        if (masked) {
 #pragma unroll
-        for (int k = 0; k < kKeys; ++k)
-          if (!((vis[k >> 5] >> (k & 31)) & 1u)) x[k] = NAN;
-      }
-      const float mr = sl >= 0.f ? reduce_n<false>(x) : reduce_n<true>(x);
-      const float mx = mr != mr ? -INFINITY : mr * sl;
-      const bool move = mx > m_ref + kLazyP;
-      const float m_new = move ? mx : m_ref;
-      const float nb = m_new == -INFINITY ? 0.f : -m_new;
-      // O is rescaled before any of this tile's P is handed over; PV of the
-      // previous tile, its last writer, completed before these scores arrived
-      if (__any_sync(0xffffffffu, move)) {
-        const float alpha = move ? exp2f(m_ref - mx) : 1.f;
-        l *= alpha;
-        if (jj >= 1) {
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tc::ld32(tmem + lane_base + o_col + c * 32, o);
-            tc::wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tc::st32(tmem + lane_base + o_col + c * 32, o);
-          }
+          for (int k = 0; k < 64; ++k)
+            if (!((vis[k >> 5] >> (k & 31)) & 1u)) x[k] = NAN;
         }
+        part = sl >= 0.f ? reduce_n<false>(x) : reduce_n<true>(x);
       }
-      m_ref = m_new;
+      pmax_s[jj & 1][wg][kh][r] = part;
+      named_sync(pair_bar, 64);
+      const float other = pmax_s[jj & 1][wg][kh ^ 1][r];
 #if SA_PREFILL_TIMELINE
-      if (r == 0) pt_mark(jj, 13 + 2 * wg);
+      if (r == 0 && kh == 0) pt_mark(jj, 12 + 2 * wg);
 #endif
-      // P = 2^(x sl - m_new) as bf16 hi + lo pairs over this tile's scores in
-      // TMEM, 16 keys at a time (8 columns of hi pairs, then 8 of lo pairs).
-      // The scores are read a second time, 32 columns at a time with the next
-      // read in flight, so that the row of 128 never has to stay in registers.
-      // Key pairs in packed float32 (the same roundings as the scalar ops, half
-      // the instructions); the row sum in eight independent chains; P handed
-      // over in two halves of 64 keys.
-      unsigned long long ls2[4] = {0ull, 0ull, 0ull, 0ull};
-      const unsigned long long sl2 = f2_pack(sl, sl), nb2 = f2_pack(nb, nb);
-      float y[2][32];
-      tc::ld32(tmem + lane_base + s_col, y[0]);
-      tc::wait_ld();
+      if (ok) {
+        const float mr = sl >= 0.f ? fmaxf(part, other) : fminf(part, other);
+        const float mx = mr != mr ? -INFINITY : mr * sl;
+        const bool move = mx > m_ref + kLazyP;
+        const float m_new = move ? mx : m_ref;
+        const float nb = m_new == -INFINITY ? 0.f : -m_new;
+        // this half of O is rescaled before any of this tile's P is handed
+        // over; PV of the previous tile, its last writer, completed before
+        // these scores arrived
+        if (__any_sync(0xffffffffu, move)) {
+          const float alpha = move ? exp2f(m_ref - mx) : 1.f;
+          l *= alpha;
+          if (jj >= 1) {
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
-        if (c + 1 < kKeys / 32) tc::ld32(tmem + lane_base + s_col + 32 * (c + 1), y[(c + 1) & 1]);
-        const float* yc = y[c & 1];
-        const uint32_t vb = masked ? vis[c] : 0xffffffffu;
+            for (int c = 0; c < D / 64; ++c) {
+              float o[32];
+              tc::ld32(tmem + lane_base + o_col + c * 32, o);
+              tc::wait_ld();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          uint32_t ph[8], pl[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int k = 16 * q + 2 * i;        // key within the 32-column chunk
-            const float2 z = f2_unpack(f2_fma(f2_pack(yc[k], yc[k + 1]), sl2, nb2));
-            float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
-            if (masked) {
-              p0 = (vb >> k) & 1u ? p0 : 0.f;
-              p1 = (vb >> (k + 1)) & 1u ? p1 : 0.f;
+              for (int i = 0; i < 32; ++i) o[i] *= alpha;
+              tc::st32(tmem + lane_base + o_col + c * 32, o);
             }
-            const unsigned long long pp = f2_pack(p0, p1);
-            ls2[i & 3] = f2_add(ls2[i & 3], pp);
-            // hi = p truncated to bf16 (its low 16 bits cleared), lo = p - hi
-            // (exact in float32) truncated likewise: integer and byte-permute
-            // instructions only, no conversions
-            const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffff0000u);
-            const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffff0000u);
-            const float2 d = f2_unpack(f2_sub(pp, f2_pack(h0, h1)));
-            ph[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);
-            pl[i] = __byte_perm(__float_as_uint(d.x), __float_as_uint(d.y), 0x7632);
           }
-          tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q, ph);
-          tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q + 8, pl);
         }
-        if (c + 1 < kKeys / 32) tc::wait_ld();
-        if (c == kKeys / 64 - 1 || c == kKeys / 32 - 1) {
-          tc::wait_st();
-          tc::fence_before_sync();
-          mbar_arrive(&p_full[wg][c == kKeys / 32 - 1 ? 1 : 0]);
+        m_ref = m_new;
 #if SA_PREFILL_TIMELINE
-          if (r == 0) pt_mark(jj, c == kKeys / 32 - 1 ? 5 + 3 * wg : 6 + 3 * wg);
+        if (r == 0 && kh == 0) pt_mark(jj, 13 + 2 * wg);
 #endif
-        }
-      }
-      float ls[8];
+        // P = 2^(x sl - m_new) as bf16 hi + lo pairs over this half's scores
+        // in TMEM, 16 keys at a time (8 columns of hi pairs, then 8 of lo
+        // pairs); the scores are read a second time, 32 columns at a time (the
+        // other warps of the sub-partition cover the read's latency).  Key
+        // pairs in packed float32 (the same roundings as the scalar ops); the
+        // row sum in eight chains.
+        unsigned long long ls2[4] = {0ull, 0ull, 0ull, 0ull};
+        const unsigned long long sl2 = f2_pack(sl, sl), nb2 = f2_pack(nb, nb);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float2 v = f2_unpack(ls2[i]);
-        ls[2 * i] = v.x;
-        ls[2 * i + 1] = v.y;
+        for (int c = 0; c < 2; ++c) {
+          float yc[32];
+          tc::ld32(tmem + lane_base + s_col + 32 * c, yc);
+          tc::wait_ld();
+          const uint32_t vb = masked ? vis[c] : 0xffffffffu;
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t ph[8], pl[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const int k = 16 * q + 2 * i;        // key within the 32-column chunk
+              const float2 z = f2_unpack(f2_fma(f2_pack(yc[k], yc[k + 1]), sl2, nb2));
+              float p0 = ex2_approx(z.x), p1 = ex2_approx(z.y);
+              if (masked) {
+                p0 = (vb >> k) & 1u ? p0 : 0.f;
+                p1 = (vb >> (k + 1)) & 1u ? p1 : 0.f;
+              }
+              const unsigned long long pp = f2_pack(p0, p1);
+              ls2[i & 3] = f2_add(ls2[i & 3], pp);
+              // hi = p truncated to bf16 (its low 16 bits cleared), lo = p - hi
+              // (exact in float32) truncated likewise: integer and byte-permute
+              // instructions only, no conversions
+              const float h0 = __uint_as_float(__float_as_uint(p0) & 0xffff0000u);
+              const float h1 = __uint_as_float(__float_as_uint(p1) & 0xffff0000u);
+              const float2 d = f2_unpack(f2_sub(pp, f2_pack(h0, h1)));
+              ph[i] = __byte_perm(__float_as_uint(p0), __float_as_uint(p1), 0x7632);
+              pl[i] = __byte_perm(__float_as_uint(d.x), __float_as_uint(d.y), 0x7632);
+            }
+            tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q, ph);
+            tc::st8(tmem + lane_base + s_col + 32 * c + 16 * q + 8, pl);
+          }
+        }
+        tc::wait_st();
+        tc::fence_before_sync();
+        mbar_arrive(&p_full[wg][kh]);
+#if SA_PREFILL_TIMELINE
+        if (r == 0 && kh == 0) pt_mark(jj, 5 + 3 * wg);
+        if (r == 0 && kh == 1) pt_mark(jj, 6 + 3 * wg);
+#endif
+        float ls[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 v = f2_unpack(ls2[i]);
+          ls[2 * i] = v.x;
+          ls[2 * i + 1] = v.y;
+        }
+        l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       }
-      l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
     }
     if (ok && n_act > 0) ok = wait_or_abort(&o_done[wg], 0, abort_flag);
     tc::fence_after_sync();
-    // ---- epilogue: O / l and LSE for this row
-    const bool empty = !ok || n_act == 0 || l == 0.f;
-    const float inv = empty ? 0.f : 1.f / l;
-    float* dst = a.o_part + ((((int64_t)split * a.B + b) * a.T + t) * a.Hq + head) * D;
+    // ---- epilogue: the row sum and status from both halves, then this half's
+    // columns of O / l, and the LSE (from the first half's thread)
+    lsum_s[wg][kh][r] = l;
+    okay_s[wg][kh][r] = ok ? 1 : 0;
+    named_sync(pair_bar, 64);
+    const float lt = lsum_s[wg][0][r] + lsum_s[wg][1][r];
+    const bool both_ok = okay_s[wg][0][r] && okay_s[wg][1][r];
+    const bool empty = !both_ok || n_act == 0 || lt == 0.f;
+    const float inv = empty ? 0.f : 1.f / lt;
+    float* dst = a.o_part + ((((int64_t)split * a.B + b) * a.T + t) * a.Hq + head) * D +
+                 (D / 2) * kh;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < D / 64; ++c) {
       float o[32];
       if (n_act > 0) {
         tc::ld32(tmem + lane_base + o_col + c * 32, o);
@@ -587,14 +619,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     : make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
       }
     }
-    if (row_ok)
+    if (row_ok && kh == 0)
       a.lse_part[(((int64_t)split * a.B + b) * a.T + t) * a.Hq + head] =
-          empty ? -INFINITY : (m_ref + log2f(l)) * kLn2;
+          empty ? -INFINITY : (m_ref + log2f(lt)) * kLn2;
     if (!ok && lane == 0) set_dev_error(a.err, SA_DEVERR_TIMEOUT);
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, C::kTmemCols);
   }

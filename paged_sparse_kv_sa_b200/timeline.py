@@ -26,9 +26,9 @@ The CUDA-event time of each launch is printed beside its span.
 ``--prefill``: the block-union chunked prefill instead (the tcgen05 many-row
 kernel, built with ``-DSA_PREFILL_TIMELINE=1``): the first CTAs of a launch
 stamp the SM clock per key tile -- the MMA thread's waits (K tile in, P of
-each row tile in) and issues, and both softmax warpgroups' phases (scores in,
-first half and all of the probabilities written) -- and the tool prints the
-median cycles of each step of a key tile's round trip.  GPU only; the library proper
+each row tile in) and issues, and the softmax warps' phases (scores in, row
+maxima exchanged and done, each half of the probabilities written) -- and the
+tool prints the median cycles of each step of a key tile's round trip.  GPU only; the library proper
 (``libsa.so``) has no timeline code.
 """
 from __future__ import annotations
@@ -70,17 +70,13 @@ def analyse_prefill(stamps: np.ndarray):
         row = {
             "tiles": n,
             "per tile (K in to next K in, MMA thread)": med(st[j + 1, 0] - st[j, 0]),
-            "softmax A (S in -> all of P written)": med(st[j, 5] - st[j, 4]),
-            "softmax B (S in -> all of P written)": med(st[j, 8] - st[j, 7]),
-            "softmax A: S in -> scores in registers": med(st[j, 12] - st[j, 4]),
-            "softmax A: scores in registers -> row max (and O rescale) done":
-                med(st[j, 13] - st[j, 12]),
-            "softmax A: row max done -> first half of P written": med(st[j, 6] - st[j, 13]),
-            "softmax A: first half -> all of P written": med(st[j, 5] - st[j, 6]),
+            "softmax A: S in -> partial maxima exchanged": med(st[j, 12] - st[j, 4]),
+            "softmax A: -> row max (and O rescale) done": med(st[j, 13] - st[j, 12]),
+            "softmax A: -> P of keys 0-63 written": med(st[j, 5] - st[j, 13]),
+            "softmax A: S in -> P of keys 64-127 written": med(st[j, 6] - st[j, 4]),
             "softmax B: S in -> row max done": med(st[j, 15] - st[j, 7]),
-            "softmax B: row max done -> all of P written": med(st[j, 8] - st[j, 15]),
-            "P_A written -> MMA thread sees it": med(st[j, 2] - st[j, 5]),
-            "P_B written -> MMA thread sees it": med(st[j, 3] - st[j, 8]),
+            "softmax B: row max done -> P of keys 0-63 written": med(st[j, 8] - st[j, 15]),
+            "P_A (second half) in at the MMA thread after S_A in": med(st[j, 2] - st[j, 4]),
             "MMA thread: P_A(j) in -> K(j+1) in": med(st[j + 1, 0] - st[j, 2]),
             "MMA thread: K(j+1) in -> P_B(j) in": med(st[j, 3] - st[j + 1, 0]),
             "MMA thread: P_B(j) in -> QK_B(j+1) issued": med(st[j + 1, 1] - st[j, 3]),
