@@ -110,6 +110,14 @@ struct __align__(64) PrefillParams {
 SA_DEV void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
+// Turn-taking of the two tiles' softmax warps (512 threads): tile A arrives on
+// kTurnA when it has handed over P of a key tile, tile B on kTurnB; the other
+// tile's warps wait there.
+constexpr int kTurnA = 9, kTurnB = 10;
+template <int kId>
+SA_DEV void turn_wait() { asm volatile("bar.sync %0, 512;" ::"n"(kId) : "memory"); }
+template <int kId>
+SA_DEV void turn_pass() { asm volatile("bar.arrive %0, 512;" ::"n"(kId) : "memory"); }
 
 // Bounded wait that also gives up as soon as another role has aborted.
 SA_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
@@ -482,6 +490,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #if SA_PREFILL_TIMELINE
       if (r == 0 && kh == 0) pt_mark(jj, 4 + 3 * wg);
 #endif
+      // The tiles take turns -- A(j) after B(j-1), B(j) after A(j) -- so that
+      // one tile's softmax runs while the tensor core works on the other's
+      // PV and QK^T, instead of both sharing the sub-partitions at once.
+      if (wg == 0) {
+        if (jj > 0) turn_wait<kTurnB>();
+      } else {
+        turn_wait<kTurnA>();
+      }
       // the row max of the scaled scores from the raw ones: x -> x s is monotone
       // (rounding included), so it is s max(x) for s >= 0 and s min(x) for s < 0;
       // invisible keys are NaN here (ignored by the reductions, p = 0 below)
@@ -590,7 +606,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
         }
         l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       }
+      if (wg == 0)
+        turn_pass<kTurnA>();
+      else
+        turn_pass<kTurnB>();
     }
+    // tile B's last pass is taken here, so that no arrival is left pending
+    if (wg == 0 && n_act > 0) turn_wait<kTurnB>();
     if (ok && n_act > 0) ok = wait_or_abort(&o_done[wg], 0, abort_flag);
     tc::fence_after_sync();
     // ---- epilogue: the row sum and status from both halves, then this half's
