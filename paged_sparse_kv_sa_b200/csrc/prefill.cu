@@ -25,6 +25,9 @@
 //               when a row's max exceeds it by more than 2^8 (the O rescale
 //               through TMEM is then rare), P back into the S columns it came
 //               from, and the epilogue (each half of a row writes half of O).
+//               The two tiles' softmax warps take turns (A(j) after B(j-1),
+//               B(j) after A(j)), so that one tile's softmax runs while the
+//               tensor core works on the other tile's PV and QK^T.
 // P enters PV as a bf16 pair hi + lo (hi = p truncated to bf16, lo = p - hi,
 // exact in float32, truncated to bf16), so hi + lo is within 2^-16 relative of
 // p rather than the 2^-9 of a single rounded bf16, at the cost of two
@@ -106,7 +109,8 @@ struct __align__(64) PrefillParams {
   PairTable pairs;
 };
 
-// Named barrier `id` (1-8; 0 is __syncthreads) over `n` threads.
+// Named barrier `id` over `n` threads: ids 1-8 pair the two key-half warps of
+// each (row tile, TMEM lane quarter); 0 is __syncthreads, 9 and 10 the turns.
 SA_DEV void named_sync(int id, int n) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
