@@ -881,6 +881,17 @@ def run_prefill(args, dev, world, rank, clk, K):
     h_in, h_out = items[0]["h_in"], items[0]["h_out"]
     pk, kind = peaks()
     achieved = flops / (t_dec / K) / 1e12
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "prefill_traffic.json")
+    if os.path.exists(tp):
+        with open(tp) as f:
+            td = json.load(f)
+        src = os.path.join(ROOT, "paged_sparse_kv_sa_b200", "csrc", "prefill.cu")
+        import hashlib
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if (td.get("workload") == cfg.name and td.get("splits") == n_splits
+                and td.get("prefill_cu_sha16") == sha):
+            traffic = td.get("bytes_per_launch")
     return {
         "value": round(world * kv_bytes * K / t_step / 1e9, 3), "unit": "GB/s", "steps": K,
         "ms_per_step": round(1e3 * t_step / K, 4), "calls_per_sec": round(world * K / t_step, 2),
@@ -892,7 +903,9 @@ def run_prefill(args, dev, world, rank, clk, K):
         "roofline": {"kernel": "prefill_kernel", "bound": "tensor", "achieved": round(achieved, 2),
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(achieved / pk["bf16_tflops"], 4),
-                     "peak_kind": f"{kind} bf16 GEMM, burst", "traffic": None,
+                     "peak_kind": f"{kind} bf16 GEMM, burst", "traffic": traffic,
+                     "traffic_what": "DRAM bytes read + written per launch (ncu, one launch of "
+                                     "this kernel at this workload and split count), or null",
                      "kernel_ms": round(1e3 * t_dec / K, 4),
                      "kernel_ms_what": f"average over {K} back-to-back launches"},
         "e2e": {"value": round(world * kv_bytes * K / t_e2e / 1e9, 3), "unit": "GB/s",
