@@ -48,3 +48,28 @@ def test_prefill_grid_analysis_recovers_per_tile_cost():
     dur = (c[:300, 1] - c[:300, 0]).sum()
     assert abs(g["sm utilisation"] - dur / (g["span_us"] * 1e3 * 148)) < 1e-12
     assert max(g["busy SMs over the span (2% steps)"]) <= 300
+
+
+def test_prefill_tile_analysis_reads_the_slots():
+    # one CTA of 40 tiles with a period of 5000 cycles: K in at 5000 j, QK_B
+    # issued 600 later, S_A in at +1000, P of A's halves at +3000 / +3200, P_A at
+    # the MMA thread at +3300; the medians come back as those differences
+    from paged_sparse_kv_sa_b200.timeline import analyse_prefill
+    st = np.zeros((1, 256, 16), dtype=np.int64)
+    n = 40
+    for j in range(n):
+        b = 100000 + 5000 * j
+        st[0, j, 0], st[0, j, 1] = b, b + 600
+        st[0, j, 4], st[0, j, 12], st[0, j, 13] = b + 1000, b + 1400, b + 1500
+        st[0, j, 5], st[0, j, 6], st[0, j, 2] = b + 3000, b + 3200, b + 3300
+        st[0, j, 7], st[0, j, 15], st[0, j, 8], st[0, j, 3] = b + 3500, b + 3900, b + 5400, b + 5600
+    st[0, 0, 10], st[0, 0, 11] = 90000, n
+    (row,) = analyse_prefill(st)
+    assert row["tiles"] == n
+    assert row["per tile (K in to next K in, MMA thread)"] == 5000
+    assert row["softmax A: S in -> partial maxima exchanged"] == 400
+    assert row["softmax A: -> P of keys 0-63 written"] == 1500
+    assert row["softmax A: S in -> P of keys 64-127 written"] == 2200
+    assert row["softmax A: P(j) written -> S(j+1) in (PV + QK round trip)"] == 3000
+    assert row["MMA thread: P_A(j) in -> K(j+1) in"] == 1700
+    assert row["launch to first tile (cycles)"] == 10000
